@@ -1,0 +1,331 @@
+"""Pins of the fp64 oracle against closed forms, hand-derived cases, brute force
+and independent library routines (no GPU).  Each test names what it pins."""
+import json
+import math
+import os
+from itertools import product
+
+import numpy as np
+import pytest
+
+import oracle as orc
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+# ---------------------------------------------------------------- shapes table
+def test_candidate_table_has_16_shapes_that_tile_a_zone():
+    # "16 candidate shapes with total volume B in {64,128,256}" (Ideias centrais)
+    edges, vol = orc.candidate_shapes()
+    assert edges.shape == (16, 3)
+    assert sorted(np.bincount(vol)[[64, 128, 256]].tolist()) == [3, 6, 7]
+    assert (edges.prod(axis=1) == vol).all()
+    assert (8 % edges == 0).all()                       # tiles the 8x8x8 zone exactly
+    # brute force: every (bT,bH,bW) in {1,2,4,8}^3 of volume B with all edges >= 2
+    brute = sorted((int(np.prod(e)),) + e for e in product((1, 2, 4, 8), repeat=3)
+                   if np.prod(e) in (64, 128, 256) and min(e) >= 2)
+    assert brute == sorted((int(v),) + tuple(int(x) for x in e) for e, v in zip(edges, vol))
+    # ids are sorted by (volume, edges)
+    keys = [(int(v),) + tuple(e) for e, v in zip(edges, vol)]
+    assert keys == sorted(keys)
+
+
+# ---------------------------------------------------------------- indicator
+def _grid(T, H, W):
+    t, h, w = np.meshgrid(np.arange(T), np.arange(H), np.arange(W), indexing="ij")
+    return t.reshape(-1).astype(float), h.reshape(-1).astype(float), w.reshape(-1).astype(float)
+
+
+@pytest.mark.parametrize("axis", [0, 1, 2])
+def test_indicator_linear_ramp_closed_form(axis):
+    # V_c = coef_c * x_axis (local coordinate) -> the axis profile is coef*(i - 3.5):
+    # population variance coef^2 * (8^2 - 1)/12 = 5.25 coef^2 along the ramp, 0 elsewhere.
+    T, H, W = 8, 16, 8
+    coords = _grid(T, H, W)
+    coef = np.array([1.0, -2.0, 0.5])
+    V = (coords[axis] % 8)[:, None] * coef[None, :]
+    hhat = np.zeros((T * H * W, 4))
+    ind = orc.zone_indicator(V, hhat, T, H, W)
+    expect = np.zeros(3)
+    expect[axis] = 5.25 * (coef ** 2).mean()
+    np.testing.assert_allclose(ind["sigma2_v"], np.tile(expect, (2, 1)), rtol=0, atol=1e-12)
+    r = np.zeros(3)
+    r[axis] = 1.0
+    np.testing.assert_allclose(ind["r_v"], np.tile(r, (2, 1)), atol=1e-15)
+    # token variance of a ramp = 5.25 coef^2 too (only one axis varies)
+    np.testing.assert_allclose(ind["rho_raw"], 5.25 * (coef ** 2).mean(), rtol=1e-12)
+    # no audio: abar = 0 and g = r + eps exactly
+    assert (ind["abar"] == 0).all()
+    np.testing.assert_array_equal(ind["g"], ind["r_v"] + orc.EPS)
+
+
+def test_indicator_two_axis_mix_and_constant():
+    T, H, W = 8, 8, 16
+    t, h, w = _grid(T, H, W)
+    V = np.stack([t % 8, 2.0 * (h % 8)], axis=1)
+    V[(w >= 8), :] = 3.0                                       # second zone constant
+    ind = orc.zone_indicator(V, np.zeros((len(t), 2)), T, H, W)
+    # zone 0: channel 0 ramps along T, channel 1 along H with 2x slope:
+    # sigma2 = (5.25/2, 4*5.25/2, 0) -> r = (0.2, 0.8, 0)
+    np.testing.assert_allclose(ind["sigma2_v"][0], [2.625, 10.5, 0.0], atol=1e-12)
+    np.testing.assert_allclose(ind["r_v"][0], [0.2, 0.8, 0.0], atol=1e-15)
+    # zone 1: constant -> zero variance -> ratios 1/3 each (R6), rho_raw = 0
+    np.testing.assert_allclose(ind["r_v"][1], [1 / 3] * 3, atol=1e-15)
+    assert ind["rho_raw"][1] == 0.0 and ind["rho_v"][1] == 0.0 and ind["rho_v"][0] == 1.0
+
+
+def test_indicator_checkerboard_has_token_variance_but_flat_profiles():
+    T, H, W = 8, 8, 8
+    t, h, w = _grid(T, H, W)
+    V = ((-1.0) ** (t + h + w))[:, None] * np.array([[1.0, 3.0]])
+    ind = orc.zone_indicator(V, np.zeros((512, 1)), T, H, W)
+    np.testing.assert_allclose(ind["sigma2_v"][0], 0.0, atol=1e-15)
+    np.testing.assert_allclose(ind["rho_raw"][0], (1 + 9) / 2, rtol=1e-14)
+
+
+def test_indicator_audio_guidance():
+    # a = ||hhat||_2 (Método 1); hhat = (t+1, 0) inside zone 0 only; others silent.
+    T, H, W = 8, 8, 24
+    t, h, w = _grid(T, H, W)
+    hhat = np.zeros((len(t), 3))
+    inz0 = w < 8
+    hhat[inz0, 0] = t[inz0] + 1.0
+    hhat[inz0, 2] = 0.0
+    V = np.random.default_rng(0).normal(size=(len(t), 4))
+    V[inz0] = 0.25                                   # zone 0: flat video, loud audio
+    ind = orc.zone_indicator(V, hhat, T, H, W)
+    np.testing.assert_allclose(ind["A"], [4.5, 0.0, 0.0], atol=1e-14)
+    np.testing.assert_allclose(ind["abar"], [1.0, 0.0, 0.0])
+    np.testing.assert_allclose(ind["vhat_a"][0], [1.0, 0.0, 0.0], atol=1e-15)
+    np.testing.assert_allclose(ind["vhat_a"][1:], 1 / 3, atol=1e-15)
+    np.testing.assert_allclose(ind["sigma2_a"][0], [5.25, 0, 0], atol=1e-12)
+    np.testing.assert_allclose(ind["g"], ind["r_v"] + ind["abar"][:, None] * ind["vhat_a"] + orc.EPS,
+                               rtol=0, atol=0)
+    np.testing.assert_allclose(ind["g"][0], ind["r_v"][0] + [1.0, 0, 0] + orc.EPS, atol=1e-15)
+    # rho = max(rho_v, abar) (R2): zone 0 has rho_v = 0 and carries abar = 1
+    assert ind["rho_v"][0] == 0.0 and ind["rho"][0] == 1.0
+    np.testing.assert_array_equal(ind["rho"][1:], ind["rho_v"][1:])
+    assert ind["rho_v"].max() == 1.0
+    # norm, not a channel sum: scaling the channel sign does not change a
+    hhat2 = hhat.copy()
+    hhat2[:, 0] *= -1
+    ind2 = orc.zone_indicator(V, hhat2, T, H, W)
+    np.testing.assert_array_equal(ind2["A"], ind["A"])
+
+
+def test_indicator_brute_force_loops():
+    # scalar loops straight from the definitions on a 8x8x16 grid, 3 channels
+    T, H, W = 8, 8, 16
+    rng = np.random.default_rng(1)
+    V = rng.normal(size=(T * H * W, 3))
+    hh = rng.normal(size=(T * H * W, 2))
+    ind = orc.zone_indicator(V, hh, T, H, W)
+    idx = lambda t, h, w: (t * H + h) * W + w
+    for m, zw in enumerate(range(W // 8)):
+        sig = [0.0, 0.0, 0.0]
+        rr = 0.0
+        for c in range(3):
+            vals = {(t, h, w): V[idx(t, h, 8 * zw + w), c] for t in range(8) for h in range(8) for w in range(8)}
+            mu = sum(vals.values()) / 512
+            for d in range(3):
+                acc = 0.0
+                for i in range(8):
+                    s = sum(v for k, v in vals.items() if k[d] == i) / 64
+                    acc += (s - mu) ** 2
+                sig[d] += acc / 8
+            rr += sum((v - mu) ** 2 for v in vals.values()) / 512
+        sig = [s / 3 for s in sig]
+        np.testing.assert_allclose(ind["sigma2_v"][m], sig, rtol=1e-12)
+        np.testing.assert_allclose(ind["rho_raw"][m], rr / 3, rtol=1e-12)
+        np.testing.assert_allclose(ind["r_v"][m], np.array(sig) / sum(sig), rtol=1e-12)
+
+
+def test_indicator_ratios_sum_to_one_and_anisotropy_direction():
+    import torch
+    from dynamic_block_sparse_macro_b200 import inputs
+    from dynamic_block_sparse_macro_b200.configs import get_config
+    rng = np.random.default_rng(2)
+    V = rng.normal(size=(8 * 16 * 16, 5))
+    hh = rng.normal(size=(8 * 16 * 16, 3))
+    ind = orc.zone_indicator(V, hh, 8, 16, 16)
+    np.testing.assert_allclose(ind["r_v"].sum(-1), 1.0, atol=1e-14)
+    np.testing.assert_allclose(ind["vhat_a"].sum(-1), 1.0, atol=1e-14)
+    assert ((ind["abar"] >= 0) & (ind["abar"] <= 1)).all() and ind["abar"].max() == 1.0
+    # smoothing along axis d* correlates tokens along d*: the profile along d*
+    # averages correlated-free slices, the other two average correlated values,
+    # so r_{d*} is the smallest of the three (statistical, large margin).
+    cfg = get_config("tiny", alpha=20.0)
+    axes = inputs._zone_axes(cfg, "cpu").reshape(-1).numpy()
+    _, _, Vt = inputs.make_qkv(cfg, "cpu")
+    ind = orc.zone_indicator(inputs.to_f64(Vt), np.zeros((cfg.n_tokens, 1)), cfg.T, cfg.H, cfg.W)
+    assert (ind["r_v"].argmin(axis=1) == axes).all()
+
+
+# ---------------------------------------------------------------- shapes
+def test_volume_thresholds():
+    rho = np.array([1.0, 0.5, 0.4999999, 0.25, 0.2499999, 0.0])
+    np.testing.assert_array_equal(orc.block_volume(rho), [64, 64, 128, 128, 256, 256])
+
+
+def test_optimal_edges_sum_and_closed_form_optimum():
+    from scipy.optimize import minimize
+    rng = np.random.default_rng(3)
+    for _ in range(20):
+        g = rng.uniform(0.05, 2.0, size=3)
+        B = int(rng.choice([64, 128, 256]))
+        ell = orc.optimal_log_edges(g, B)
+        assert abs(ell.sum() - math.log2(B)) < 1e-12          # prod b*_d = B
+        # independent: minimise sum g_d (b_d^2 - 1) s.t. prod b_d = B numerically
+        f = lambda x: float((g * (np.array([2 ** x[0], 2 ** x[1], B / 2 ** (x[0] + x[1])]) ** 2 - 1)).sum())
+        res = minimize(f, x0=[2.0, 2.0], method="Nelder-Mead",
+                       options={"xatol": 1e-11, "fatol": 1e-14, "maxiter": 20000})
+        num = np.array([res.x[0], res.x[1], math.log2(B) - res.x[0] - res.x[1]])
+        np.testing.assert_allclose(ell, num, atol=2e-5)
+
+
+def test_shapes_worked_cases():
+    with open(os.path.join(GOLDEN, "shapes_worked.json")) as f:
+        cases = json.load(f)["cases"]
+    edges, vol = orc.candidate_shapes()
+    tau_rho = {64: 1.0, 128: 0.3, 256: 0.0}
+    for c in cases:
+        out = orc.assign_shapes(np.array([c["g"]], float), np.array([tau_rho[c["B"]]]))
+        assert out["B"][0] == c["B"]
+        np.testing.assert_allclose(out["ell"][0], c["ell"], atol=1e-12)
+        assert tuple(out["edges"][0]) == tuple(c["edges"]), c
+        np.testing.assert_allclose(out["dist2"][0, out["shape_id"][0]], c["dist2"], atol=1e-12)
+        if c["tie"]:
+            assert out["margin_shape"][0] < 1e-12
+            other = [i for i in range(16) if tuple(edges[i]) == tuple(c["tied_with"])][0]
+            assert abs(out["dist2"][0, other] - c["dist2"]) < 1e-12
+        else:
+            assert out["margin_shape"][0] > 0.1
+
+
+def test_shapes_brute_force_random():
+    rng = np.random.default_rng(4)
+    Z = 300
+    g = np.exp(rng.uniform(-4, 1, size=(Z, 3)))
+    rho = rng.uniform(0, 1, size=Z)
+    out = orc.assign_shapes(g, rho)
+    for m in range(Z):
+        B = 64 if rho[m] >= 0.5 else 128 if rho[m] >= 0.25 else 256
+        S = math.log2(B)
+        lg = [math.log2(x) for x in g[m]]
+        ell = [-0.5 * lg[d] + (S + 0.5 * sum(lg)) / 3 for d in range(3)]
+        best = None
+        for e in product((2, 4, 8), repeat=3):
+            if e[0] * e[1] * e[2] != B:
+                continue
+            dd = sum((math.log2(e[d]) - ell[d]) ** 2 for d in range(3))
+            if best is None or dd < best[0] - 1e-12:
+                best = (dd, e)
+        assert tuple(out["edges"][m]) == best[1]
+
+
+# ---------------------------------------------------------------- permutation
+def test_permutation_bijection_boxes_and_inverse():
+    T, H, W = 16, 8, 24
+    Z = (T // 8) * (H // 8) * (W // 8)
+    rng = np.random.default_rng(5)
+    sid = rng.integers(0, 16, size=Z)
+    perm, bs = orc.build_permutation(sid, T, H, W)
+    N = T * H * W
+    assert sorted(perm.tolist()) == list(range(N))
+    edges, vol = orc.candidate_shapes()
+    # zone m owns permuted positions [512 m, 512 m + 512); blocks are boxes
+    b = 0
+    for m in range(Z):
+        zt, zh, zw = m // ((H // 8) * (W // 8)), (m // (W // 8)) % (H // 8), m % (W // 8)
+        nbz = 512 // vol[sid[m]]
+        for k in range(nbz):
+            s, e = bs[b], bs[b + 1]
+            assert e - s == vol[sid[m]] and s == 512 * m + k * (e - s)
+            toks = perm[s:e]
+            t, h, w = toks // (H * W), (toks // W) % H, toks % W
+            assert (t // 8 == zt).all() and (h // 8 == zh).all() and (w // 8 == zw).all()
+            ext = (t.max() - t.min() + 1, h.max() - h.min() + 1, w.max() - w.min() + 1)
+            assert ext == tuple(edges[sid[m]])
+            assert (np.diff(toks) > 0).all()                      # raster order inside the block
+            b += 1
+    assert b == len(bs) - 1
+    X = rng.normal(size=(N, 3, 4))
+    np.testing.assert_array_equal(orc.unpermute(orc.permute(X, perm), perm), X)
+
+
+def test_permutation_first_block_explicit():
+    # one zone, shape (8, 8, 2): block 0 is the w in {0,1} slab, raster order
+    edges, _ = orc.candidate_shapes()
+    sid = [i for i in range(16) if tuple(edges[i]) == (8, 8, 2)][0]
+    perm, bs = orc.build_permutation(np.array([sid]), 8, 8, 8)
+    expect = [(t * 8 + h) * 8 + w for t in range(8) for h in range(8) for w in range(2)]
+    assert perm[:128].tolist() == expect
+    assert bs.tolist() == [0, 128, 256, 384, 512]
+
+
+# ---------------------------------------------------------------- pool / score
+def test_pool_score_closed_form():
+    # two blocks of 2 tokens with constant rows: means are the constants;
+    # P_00 = 1 / (1 + exp(s_01 - s_00)) (2-way softmax)
+    d = 4
+    q = np.array([[1, 0, 0, 0], [1, 0, 0, 0], [0, 2, 0, 0], [0, 0, 0, 0]], float)
+    k = np.array([[3, 0, 0, 0], [1, 0, 0, 0], [0, 1, 1, 0], [0, 1, -1, 0]], float)
+    Qbar, Kbar, P = orc.block_pool_score(q[None], k[None], np.array([0, 2, 4]))
+    np.testing.assert_allclose(Qbar[0], [[1, 0, 0, 0], [0, 1, 0, 0]])
+    np.testing.assert_allclose(Kbar[0], [[2, 0, 0, 0], [0, 1, 0, 0]])
+    s = np.array([[2.0, 0.0], [0.0, 1.0]]) / math.sqrt(d)
+    np.testing.assert_allclose(P[0, 0, 0], 1 / (1 + math.exp(s[0, 1] - s[0, 0])), rtol=1e-14)
+    np.testing.assert_allclose(P[0, 1, 1], 1 / (1 + math.exp(s[1, 0] - s[1, 1])), rtol=1e-14)
+    np.testing.assert_allclose(P.sum(-1), 1.0, rtol=1e-15)
+
+
+# ---------------------------------------------------------------- select
+def test_select_worked_cases():
+    with open(os.path.join(GOLDEN, "select_worked.json")) as f:
+        cases = json.load(f)["cases"]
+    for c in cases:
+        out = orc.block_select(np.array([c["P"]]), c["k"], c["p"])
+        assert np.nonzero(out["sel"][0])[0].tolist() == c["sel"], c
+
+
+def test_select_brute_force_small():
+    rng = np.random.default_rng(6)
+    for trial in range(200):
+        nb = int(rng.integers(1, 11))
+        x = rng.normal(size=nb) * rng.uniform(0.1, 4)
+        if trial % 5 == 0:
+            x = np.round(x)                           # force equal probabilities
+        P = np.exp(x - x.max())
+        P /= P.sum()
+        k = int(rng.integers(1, 12))
+        p = float(rng.uniform(0.05, 1.0))
+        out = orc.block_select(P[None], k, p)
+        # brute force: Top-p = smallest cardinality n such that SOME n-subset has mass >= p;
+        # the chosen n-subset is the best by (P desc, j asc); union with the top-k prefix.
+        key = sorted(range(nb), key=lambda j: (-P[j], j))
+        n_p = nb
+        for n in range(1, nb + 1):
+            from itertools import combinations
+            if any(sum(P[list(c)]) >= p for c in combinations(range(nb), n)):
+                n_p = n
+                break
+        top_p_set = set(key[:n_p])
+        top_k_set = set(key[:min(k, nb)])
+        assert set(np.nonzero(out["sel"][0])[0].tolist()) == top_p_set | top_k_set
+        assert out["count"][0] == len(top_p_set | top_k_set)
+
+
+def test_select_invariants_and_dense_limits():
+    rng = np.random.default_rng(7)
+    x = rng.normal(size=(3, 50, 50)) * 2
+    P = np.exp(x) / np.exp(x).sum(-1, keepdims=True)
+    out = orc.block_select(P, 8, 0.9)
+    cnt = out["sel"].sum(-1)
+    assert (cnt >= 8).all() and (cnt == out["count"]).all()
+    assert ((P * out["sel"]).sum(-1) >= 0.9 - 1e-12).all()
+    # selected = a prefix of the sorted order: min selected P >= max unselected P
+    mn = np.where(out["sel"], P, np.inf).min(-1)
+    mx = np.where(out["sel"], -np.inf, P).max(-1)
+    assert (mn >= mx).all()
+    assert orc.block_select(P, 8, 1.0)["sel"].all()
+    assert orc.block_select(P, 50, 0.1)["sel"].all()
