@@ -1,0 +1,418 @@
+#!/usr/bin/env python
+"""Benchmark of the Prism sparse video self-attention layer (fwd + bwd) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config 2k] [--dense]
+    python bench.py --impl reference      # the fp64 CPU oracle on a bounded sample
+
+One step = one pass of the whole hot path over the configured synthetic layer:
+zone indicator -> shapes/permutation -> permute Q,K,V -> pooled block
+probabilities -> hybrid selection -> sparse attention forward -> unpermute O ->
+permute dO -> sparse attention backward -> unpermute dQ, dK, dV.
+``value`` is TFLOP/s on the selected blocks (algorithmic FLOPs 3.5 * F_fwd,
+F_fwd = 4 d sum_h sum_i sum_{j in S_i} |B_i||B_j|) over the device time of the
+sparse attention forward + backward calls, summed over ranks (each rank runs
+its own layer: weak scaling, no data-path collective).  Prints one JSON line
+on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from dynamic_block_sparse_macro_b200 import inputs  # noqa: E402
+from dynamic_block_sparse_macro_b200.configs import get_config  # noqa: E402
+
+METRIC = "sparse attn fwd+bwd ms/layer & TFLOP/s on selected blocks, 2K grid (295k tok)"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        d["source"] = "measured"
+        return d
+    d = dict(PEAKS_FALLBACK)
+    d["source"] = "fallback"
+    return d
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+        self.t = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.t = threading.Thread(target=self._read, daemon=True)
+        self.t.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.t:
+            self.t.join(timeout=2)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- helpers
+def unpack_sel_dev(words: torch.Tensor, nb: int) -> torch.Tensor:
+    """[h, MB, SW] int32 bitmask -> bool [h, nb, nb] on the device."""
+    w = words[:, :nb, :].to(torch.int64) & 0xFFFFFFFF
+    sh = torch.arange(32, device=words.device, dtype=torch.int64)
+    b = ((w.unsqueeze(-1) >> sh) & 1).reshape(w.shape[0], nb, -1)
+    return b[..., :nb].bool()
+
+
+def selected_flops(mod) -> dict:
+    """F_fwd = 4 d sum_h sum_i |B_i| sum_{j in S_i} |B_j| and density figures."""
+    nb = mod.num_blocks()
+    bs = mod.blk_start[: nb + 1].to(torch.int64)
+    sz = (bs[1:] - bs[:-1]).to(torch.float64)
+    sel = unpack_sel_dev(mod.sel, nb).to(torch.float64)
+    keys_per_row = sel @ sz                                   # [h, nb] selected key tokens
+    f_fwd = 4.0 * mod.d * float((keys_per_row * sz).sum().item())
+    dense = 4.0 * mod.d * mod.heads * float(sz.sum().item()) ** 2
+    vol = {int(v): int((sz == v).sum().item()) for v in (64, 128, 256)}
+    return {"F_fwd": f_fwd, "F_dense_fwd": dense, "n_blk": nb, "density": f_fwd / dense,
+            "mean_sel_blocks": float(sel.sum(-1).mean().item()),
+            "mean_sel_tokens": float(keys_per_row.mean().item()), "block_volumes": vol}
+
+
+class StepTimer:
+    """CUDA events around the stages of one step (on the launching stream)."""
+    NAMES = ("plan_select", "attn_fwd", "unpermute_o", "permute_do", "attn_bwd", "unpermute_grads")
+
+    def __init__(self):
+        self.ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(self.NAMES) + 1)]
+
+    def times(self):
+        return {n: self.ev[i].elapsed_time(self.ev[i + 1]) for i, n in enumerate(self.NAMES)}
+
+
+def run_step(mod, x, out, grads, timer=None):
+    ev = timer.ev if timer else None
+    rec = (lambda i: ev[i].record()) if ev else (lambda i: None)
+    rec(0)
+    mod.plan(x["V"], x["hhat"])
+    mod.select(x["Q"], x["K"], x["V"])
+    rec(1)
+    mod.attend()
+    rec(2)
+    from dynamic_block_sparse_macro_b200 import _abi
+    _abi.prism_unpermute(mod.prob, mod.Op, mod.perm, out)
+    rec(3)
+    _abi.prism_permute(mod.prob, x["dO"], mod.perm, mod.dOp)
+    rec(4)
+    _abi.prism_sparse_attn_bwd(mod.prob, mod.Qp, mod.Kp, mod.Vp, mod.Op, mod.dOp, mod.lse, mod.blk_start,
+                               mod.gran_blk, mod.n_blk, mod.sel, mod.selT, mod.scale, mod.dQp, mod.dKp,
+                               mod.dVp, mod.dev_status, mod.ws_bwd)
+    rec(5)
+    for src, dst in zip((mod.dQp, mod.dKp, mod.dVp), grads):
+        _abi.prism_unpermute(mod.prob, src, mod.perm, dst)
+    rec(6)
+
+
+# ---------------------------------------------------------------- CPU oracle sample
+def oracle_sample(cfg, host, target_s=15.0, max_blocks=None, seed=0):
+    """Time the fp64 oracle's sparse attention fwd+bwd on a bounded sample of
+    query blocks of head 0, under the given selection.  Returns a dict."""
+    import oracle as orc
+    from threadpoolctl import threadpool_info
+    Qb, Kb, Vb, dOb, bs, sel = (host[k] for k in ("Qb", "Kb", "Vb", "dOb", "bs", "sel"))
+    nb = len(bs) - 1
+    rng = np.random.default_rng(seed)
+    order = rng.permutation(nb)
+    sizes = np.diff(bs)
+    done, flops, t_used = 0, 0.0, 0.0
+    step = 2
+    while t_used < target_s and done < nb and (max_blocks is None or done < max_blocks):
+        blocks = sorted(order[done:done + step].tolist())
+        t0 = time.perf_counter()
+        orc.sparse_attention_fwd(Qb, Kb, Vb, bs, sel, heads=[0], q_blocks=blocks)
+        orc.sparse_attention_bwd(Qb, Kb, Vb, dOb, bs, sel, heads=[0], q_blocks=blocks)
+        t_used += time.perf_counter() - t0
+        for i in blocks:
+            flops += 3.5 * 4.0 * Qb.shape[-1] * sizes[i] * float(sizes[sel[0, i]].sum())
+        done += len(blocks)
+        step = min(step * 2, 64)
+    threads = 1
+    for lib in threadpool_info():
+        threads = max(threads, int(lib.get("num_threads", 1)))
+    return {"tflops": flops / t_used / 1e12, "seconds": t_used, "blocks": done, "flops": flops,
+            "threads": threads}
+
+
+def make_host_sample(mod, x):
+    """fp64 host copies of head 0's blocked tensors and the GPU's selection (for the oracle)."""
+    nb = mod.num_blocks()
+    sel = unpack_sel_dev(mod.sel[:1], nb).cpu().numpy()
+    bs = mod.blk_start[: nb + 1].cpu().numpy().astype(np.int64)
+    f = lambda t: t[:1].float().cpu().double().numpy()
+    from dynamic_block_sparse_macro_b200 import _abi
+    _abi.prism_permute(mod.prob, x["dO"], mod.perm, mod.dOp)
+    torch.cuda.synchronize()
+    return {"Qb": f(mod.Qp), "Kb": f(mod.Kp), "Vb": f(mod.Vp), "dOb": f(mod.dOp), "bs": bs, "sel": sel}
+
+
+# ---------------------------------------------------------------- arms
+def bench_prism(args, cfg, rank, world, local_rank):
+    from dynamic_block_sparse_macro_b200 import _abi
+    from dynamic_block_sparse_macro_b200.layer import PrismSparseAttention
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    x = inputs.make_inputs(cfg, dev)
+    torch.cuda.synchronize()
+    mod = PrismSparseAttention(cfg.T, cfg.H, cfg.W, cfg.heads, cfg.head_dim, cfg.audio_dim, cfg.dtype,
+                               cfg.top_k, cfg.top_p if not args.dense else 1.0, device=dev)
+    out = torch.empty_like(x["Q"])
+    grads = [torch.empty_like(x["Q"]) for _ in range(3)]
+    for _ in range(max(args.warmup, 1)):
+        run_step(mod, x, out, grads)
+    torch.cuda.synchronize()
+    fl = selected_flops(mod)
+
+    timers = [StepTimer() for _ in range(args.steps)]
+    clocks = ClockSampler(local_rank)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    start = torch.cuda.Event(enable_timing=True)
+    stop = torch.cuda.Event(enable_timing=True)
+    n0 = _abi.launch_count()
+    start.record()
+    for t in timers:
+        run_step(mod, x, out, grads, t)
+    stop.record()
+    torch.cuda.synchronize()
+    launches = _abi.launch_count() - n0
+    clk = clocks.stop()
+    total_ms = start.elapsed_time(stop)
+    per = [t.times() for t in timers]
+    stage_ms = {n: float(np.mean([p[n] for p in per])) for n in StepTimer.NAMES}
+    attn_ms = stage_ms["attn_fwd"] + stage_ms["attn_bwd"]
+    status = mod.status()
+    if world > 1:
+        tt = torch.tensor([total_ms, attn_ms], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
+        total_ms, attn_ms = float(tt[0]), float(tt[1])
+    ms_step = total_ms / args.steps
+    attn_flops = 3.5 * fl["F_fwd"]
+    tflops = world * attn_flops / (attn_ms * 1e-3) / 1e12
+
+    # end to end through the public API from pinned host buffers
+    e2e = None
+    if not args.no_e2e:
+        e2e = bench_e2e(args, cfg, mod, x, dev, world, attn_flops)
+
+    peaks = load_peaks()
+    fwd_ach = 4 * fl["F_fwd"] / (stage_ms["attn_fwd"] * 1e-3) / 1e12
+    bwd_ach = 2.5 * fl["F_fwd"] / (stage_ms["attn_bwd"] * 1e-3) / 1e12
+    dom = "attn_bwd" if stage_ms["attn_bwd"] >= stage_ms["attn_fwd"] else "attn_fwd"
+    ach = bwd_ach if dom == "attn_bwd" else fwd_ach
+    peak = peaks["bf16_tflops_sustained"]
+    res = {
+        "metric": METRIC, "value": round(tflops, 3), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+        "attn_ms_per_layer": round(attn_ms, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic",
+        "config": {"workload": f"prism {cfg.name} layer fwd+bwd", "grid": [cfg.T, cfg.H, cfg.W],
+                   "tokens": cfg.n_tokens, "heads": cfg.heads, "head_dim": cfg.head_dim,
+                   "top_k": cfg.top_k, "top_p": 1.0 if args.dense else cfg.top_p,
+                   "all_blocks_dense": bool(args.dense), "global_batch": world,
+                   "parallelism": f"replicas{world}" if world > 1 else "single",
+                   "l2": "inputs larger than L2 (126 MB): no flush"},
+        "stage_ms": {k: round(v, 4) for k, v in stage_ms.items()},
+        "selection": {k: (round(v, 6) if isinstance(v, float) else v) for k, v in fl.items()},
+        "roofline": {"kernel": "prism_sparse_attn_bwd" if dom == "attn_bwd" else "prism_sparse_attn_fwd",
+                     "bound": "tensor", "achieved": round(ach, 3), "peak": peak, "unit": "TFLOP/s",
+                     "frac": round(ach / peak, 4), "traffic": None,
+                     "peak_source": f"{peaks['source']} bf16_tflops_sustained"},
+        "gpu_launches": int(launches),
+        "clocks": clk,
+        "dev_status": status,
+        "e2e": e2e,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu:
+        host = make_host_sample(mod, x)
+        cs = oracle_sample(cfg, host, target_s=args.cpu_seconds)
+        res["cpu_baseline"] = {"value": round(cs["tflops"], 6), "unit": "TFLOP/s", "cores": cs["threads"],
+                               "kind": "oracle",
+                               "sample": f"fp64 numpy oracle, head 0, {cs['blocks']} random query blocks "
+                                         f"(fwd+bwd under the GPU's selection), {cs['seconds']:.1f} s"}
+    return res
+
+
+def bench_e2e(args, cfg, mod, x, dev, world, attn_flops):
+    names = ("Q", "K", "V", "hhat", "dO")
+    hin = {k: torch.empty(x[k].shape, dtype=x[k].dtype, pin_memory=True) for k in names}
+    for k in names:
+        hin[k].copy_(x[k])
+    dx = {k: torch.empty_like(x[k]) for k in names}
+    hout = [torch.empty(x["Q"].shape, dtype=x["Q"].dtype, pin_memory=True) for _ in range(4)]
+    out = torch.empty_like(x["Q"])
+    grads = [torch.empty_like(x["Q"]) for _ in range(3)]
+    steps = max(1, min(args.steps, 3))
+
+    def one():
+        for k in names:
+            dx[k].copy_(hin[k], non_blocking=True)
+        run_step(mod, dx, out, grads)
+        for h, d in zip(hout, [out] + grads):
+            h.copy_(d, non_blocking=True)
+
+    one()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(steps):
+        one()
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / steps
+    if world > 1:
+        t = torch.tensor([ms], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t[0])
+    h2d = sum(hin[k].numel() * hin[k].element_size() for k in names)
+    d2h = sum(h.numel() * h.element_size() for h in hout)
+    return {"value": round(world * attn_flops / (ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+            "ms_per_step": round(ms, 3), "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+            "steps": steps, "note": "selected-block FLOPs over the whole layer step incl. host copies"}
+
+
+def bench_reference(args, cfg):
+    """The fp64 oracle as it stands, on host cores: each step is a bounded sample
+    (query blocks of head 0) of the same workload's attention fwd+bwd."""
+    import oracle as orc
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    x = inputs.make_inputs(cfg, dev)
+    V = inputs.to_f64(x["V"])
+    hh = inputs.to_f64(x["hhat"])
+    ind = orc.zone_indicator(V, hh, cfg.T, cfg.H, cfg.W)
+    del V
+    shp = orc.assign_shapes(ind["g"], ind["rho"])
+    perm, bs = orc.build_permutation(shp["shape_id"], cfg.T, cfg.H, cfg.W)
+    q0 = lambda t: inputs.to_f64(t[:, :1, :])
+    Qb, Kb, Vb, dOb = (orc.permute(q0(x[k]), perm) for k in ("Q", "K", "V", "dO"))
+    _, _, P = orc.block_pool_score(Qb, Kb, bs)
+    sel = orc.block_select(P, cfg.top_k, cfg.top_p)["sel"]
+    host = {"Qb": Qb, "Kb": Kb, "Vb": Vb, "dOb": dOb, "bs": bs, "sel": sel}
+    per_step = max(2.0, args.cpu_seconds / max(1, args.steps + args.warmup))
+    for w in range(args.warmup):
+        oracle_sample(cfg, host, target_s=per_step, seed=1000 + w)
+    res = [oracle_sample(cfg, host, target_s=per_step, seed=s) for s in range(args.steps)]
+    fl = sum(r["flops"] for r in res)
+    sec = sum(r["seconds"] for r in res)
+    v = fl / sec / 1e12
+    blocks = sum(r["blocks"] for r in res)
+    return {"metric": METRIC, "value": round(v, 6), "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(1e3 * sec / args.steps, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": f"prism {cfg.name} layer fwd+bwd (oracle sample)",
+                       "grid": [cfg.T, cfg.H, cfg.W], "tokens": cfg.n_tokens, "heads": cfg.heads,
+                       "head_dim": cfg.head_dim, "top_k": cfg.top_k, "top_p": cfg.top_p},
+            "cpu_baseline": {"value": round(v, 6), "unit": "TFLOP/s", "cores": res[0]["threads"],
+                             "kind": "oracle",
+                             "sample": f"fp64 numpy oracle sparse attention fwd+bwd, head 0, {blocks} query "
+                                       f"blocks over {args.steps} steps, selection by the oracle's own stages"},
+            "e2e": {"value": round(v, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="prism", choices=["prism", "reference"])
+    ap.add_argument("--config", default="2k")
+    ap.add_argument("--dense", action="store_true", help="select every block (all-blocks dense run)")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--out", default=None, help="also append the JSON line to this file")
+    args = ap.parse_args()
+    cfg = get_config(args.config)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        res = bench_reference(args, cfg)
+    else:
+        if world > 1:
+            import datetime
+            torch.cuda.set_device(local_rank)
+            torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                                 device_id=torch.device("cuda", local_rank))
+        res = bench_prism(args, cfg, rank, world, local_rank)
+        if world > 1:
+            torch.distributed.barrier()
+            torch.distributed.destroy_process_group()
+    if rank == 0:
+        line = json.dumps(res)
+        print(line, flush=True)
+        if args.out:
+            with open(args.out, "a") as f:
+                f.write(line + "\n")
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,191 @@
+"""ctypes binding of ``libprism.so`` (the C ABI declared in ``include/prism.h``).
+
+Argument marshalling only: every function takes torch tensors that already
+live on the GPU (or raw integer device pointers) and forwards their addresses,
+sizes and the current CUDA stream.  Every step of the path runs in the CUDA
+library; if it is missing this module raises instead of falling back.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libprism.so")
+
+PRISM_F32, PRISM_BF16 = 0, 1
+STATUS = {0: "PRISM_OK", 1: "PRISM_ERR_INVALID_ARG", 2: "PRISM_ERR_SHAPE",
+          3: "PRISM_ERR_UNSUPPORTED", 4: "PRISM_ERR_WORKSPACE", 5: "PRISM_ERR_CUDA"}
+DEV_TIMEOUT, DEV_BAD_INDEX = 0x1, 0x2
+
+# every symbol include/prism.h declares
+EXPORTS = ("prism_query_sizes", "prism_zone_indicator", "prism_assign_shapes", "prism_permute",
+           "prism_unpermute", "prism_block_pool_score", "prism_block_select",
+           "prism_sparse_attn_fwd", "prism_sparse_attn_bwd", "prism_read_status",
+           "prism_status_string", "prism_version", "prism_launch_count")
+
+
+class Problem(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int32), ("H", ctypes.c_int32), ("W", ctypes.c_int32),
+                ("heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+                ("audio_dim", ctypes.c_int32), ("dtype", ctypes.c_int32)]
+
+
+class Sizes(ctypes.Structure):
+    _fields_ = [("n_tokens", ctypes.c_int64), ("n_zones", ctypes.c_int64),
+                ("max_blocks", ctypes.c_int64), ("sel_words", ctypes.c_int64),
+                ("ws_indicator", ctypes.c_size_t), ("ws_attn_fwd", ctypes.c_size_t),
+                ("ws_attn_bwd", ctypes.c_size_t), ("bytes_P_max", ctypes.c_size_t)]
+
+
+class PrismError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        super().__init__(f"{fn} returned {STATUS.get(code, code)}")
+        self.code = code
+
+
+_lib = None
+_P = ctypes.c_void_p
+_I = ctypes.c_int32
+_F = ctypes.c_float
+_SZ = ctypes.c_size_t
+_PROB = ctypes.POINTER(Problem)
+
+_SIGS = {
+    "prism_query_sizes": [_PROB, ctypes.POINTER(Sizes)],
+    "prism_zone_indicator": [_PROB, _P, _P, _F, _P, _P, _P, _P, _P, _SZ, _P],
+    "prism_assign_shapes": [_PROB, _P, _P, _F, _F, _P, _P, _P, _P, _P, _P, _P, _P],
+    "prism_permute": [_PROB, _P, _P, _P, _P],
+    "prism_unpermute": [_PROB, _P, _P, _P, _P],
+    "prism_block_pool_score": [_PROB, _P, _P, _P, _P, _F, _P, _P, _P, _P],
+    "prism_block_select": [_PROB, _P, _P, _I, _F, _P, _P, _P, _P, _P, _P],
+    "prism_sparse_attn_fwd": [_PROB, _P, _P, _P, _P, _P, _P, _P, _F, _P, _P, _P, _P, _SZ, _P],
+    "prism_sparse_attn_bwd": [_PROB, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _F, _P, _P, _P,
+                              _P, _P, _SZ, _P],
+    "prism_read_status": [_P, ctypes.POINTER(ctypes.c_uint32), _P],
+}
+
+
+def lib(path: str | None = None):
+    """Load the CUDA library once; raise if it is not built."""
+    global _lib
+    if _lib is None:
+        p = path or os.environ.get("PRISM_LIB", LIB_PATH)
+        if not os.path.exists(p):
+            raise RuntimeError(f"libprism.so not found at {p}: run `python -m "
+                               f"dynamic_block_sparse_macro_b200.build` (no CPU fallback exists)")
+        L = ctypes.CDLL(p)
+        for name, args in _SIGS.items():
+            f = getattr(L, name)
+            f.argtypes = args
+            f.restype = ctypes.c_int
+        L.prism_status_string.argtypes = [ctypes.c_int]
+        L.prism_status_string.restype = ctypes.c_char_p
+        L.prism_version.argtypes = []
+        L.prism_version.restype = ctypes.c_char_p
+        L.prism_launch_count.argtypes = []
+        L.prism_launch_count.restype = ctypes.c_ulonglong
+        _lib = L
+    return _lib
+
+
+def _ptr(x):
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(fn, code):
+    if code != 0:
+        raise PrismError(fn, code)
+
+
+def problem(T, H, W, heads, head_dim, audio_dim, dtype) -> Problem:
+    dt = {"f32": PRISM_F32, "bf16": PRISM_BF16, PRISM_F32: PRISM_F32, PRISM_BF16: PRISM_BF16}[dtype]
+    return Problem(T, H, W, heads, head_dim, audio_dim, dt)
+
+
+def query_sizes(prob: Problem) -> Sizes:
+    s = Sizes()
+    _check("prism_query_sizes", lib().prism_query_sizes(ctypes.byref(prob), ctypes.byref(s)))
+    return s
+
+
+def prism_zone_indicator(prob, V, hhat, eps, g, rho, abar, zone_stats, ws, stream=None):
+    _check("prism_zone_indicator", lib().prism_zone_indicator(
+        ctypes.byref(prob), _ptr(V), _ptr(hhat), eps, _ptr(g), _ptr(rho), _ptr(abar),
+        _ptr(zone_stats), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def prism_assign_shapes(prob, g, rho, tau128, tau256, shape_id, perm, inv_perm, blk_start,
+                        gran_blk, n_blk, margin, stream=None):
+    _check("prism_assign_shapes", lib().prism_assign_shapes(
+        ctypes.byref(prob), _ptr(g), _ptr(rho), tau128, tau256, _ptr(shape_id), _ptr(perm),
+        _ptr(inv_perm), _ptr(blk_start), _ptr(gran_blk), _ptr(n_blk), _ptr(margin), _stream(stream)))
+
+
+def prism_permute(prob, src_raster, perm, dst_blocked, stream=None):
+    _check("prism_permute", lib().prism_permute(ctypes.byref(prob), _ptr(src_raster), _ptr(perm),
+                                                _ptr(dst_blocked), _stream(stream)))
+
+
+def prism_unpermute(prob, src_blocked, perm, dst_raster, stream=None):
+    _check("prism_unpermute", lib().prism_unpermute(ctypes.byref(prob), _ptr(src_blocked), _ptr(perm),
+                                                    _ptr(dst_raster), _stream(stream)))
+
+
+def prism_block_pool_score(prob, Qp, Kp, blk_start, n_blk, scale, Qbar, Kbar, P, stream=None):
+    _check("prism_block_pool_score", lib().prism_block_pool_score(
+        ctypes.byref(prob), _ptr(Qp), _ptr(Kp), _ptr(blk_start), _ptr(n_blk), scale, _ptr(Qbar),
+        _ptr(Kbar), _ptr(P), _stream(stream)))
+
+
+def prism_block_select(prob, P, n_blk, top_k, top_p, sel, sel_count, selT, margin, dev_status,
+                       stream=None):
+    _check("prism_block_select", lib().prism_block_select(
+        ctypes.byref(prob), _ptr(P), _ptr(n_blk), int(top_k), float(top_p), _ptr(sel),
+        _ptr(sel_count), _ptr(selT), _ptr(margin), _ptr(dev_status), _stream(stream)))
+
+
+def prism_sparse_attn_fwd(prob, Qp, Kp, Vp, blk_start, gran_blk, n_blk, sel, scale, Op, lse,
+                          dev_status, ws=None, stream=None):
+    nbytes = 0 if ws is None else ws.numel() * ws.element_size()
+    _check("prism_sparse_attn_fwd", lib().prism_sparse_attn_fwd(
+        ctypes.byref(prob), _ptr(Qp), _ptr(Kp), _ptr(Vp), _ptr(blk_start), _ptr(gran_blk),
+        _ptr(n_blk), _ptr(sel), scale, _ptr(Op), _ptr(lse), _ptr(dev_status), _ptr(ws), nbytes,
+        _stream(stream)))
+
+
+def prism_sparse_attn_bwd(prob, Qp, Kp, Vp, Op, dOp, lse, blk_start, gran_blk, n_blk, sel, selT,
+                          scale, dQp, dKp, dVp, dev_status, ws, stream=None):
+    _check("prism_sparse_attn_bwd", lib().prism_sparse_attn_bwd(
+        ctypes.byref(prob), _ptr(Qp), _ptr(Kp), _ptr(Vp), _ptr(Op), _ptr(dOp), _ptr(lse),
+        _ptr(blk_start), _ptr(gran_blk), _ptr(n_blk), _ptr(sel), _ptr(selT), scale, _ptr(dQp),
+        _ptr(dKp), _ptr(dVp), _ptr(dev_status), _ptr(ws), ws.numel() * ws.element_size(),
+        _stream(stream)))
+
+
+def prism_read_status(dev_status, stream=None) -> int:
+    out = ctypes.c_uint32(0)
+    _check("prism_read_status", lib().prism_read_status(_ptr(dev_status), ctypes.byref(out),
+                                                        _stream(stream)))
+    return out.value
+
+
+def version() -> str:
+    return lib().prism_version().decode()
+
+
+def launch_count() -> int:
+    return int(lib().prism_launch_count())

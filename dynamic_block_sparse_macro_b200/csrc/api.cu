@@ -1,0 +1,101 @@
+// Host side of the C ABI: buffer sizes, argument checks and the attention
+// entry points (stages 6-7), which pick the kernel family for the dtype.
+#include <atomic>
+
+#include "common.cuh"
+
+namespace prism {
+size_t zone_indicator_ws_bytes(const Dims& d);
+prism_status_t attn_fwd_simt(const Dims& d, const void* Qp, const void* Kp, const void* Vp,
+                             const int32_t* blk_start, const int32_t* gran_blk, const int32_t* n_blk,
+                             const uint32_t* sel, float scale, void* Op, float* lse, cudaStream_t s);
+prism_status_t attn_bwd_simt(const Dims& d, const void* Qp, const void* Kp, const void* Vp, const void* Op,
+                             const void* dOp, const float* lse, const int32_t* blk_start,
+                             const int32_t* gran_blk, const int32_t* n_blk, const uint32_t* sel,
+                             const uint32_t* selT, float scale, void* dQp, void* dKp, void* dVp,
+                             float* delta, cudaStream_t s);
+
+static std::atomic<unsigned long long> g_launches{0};
+void note_launches(int n) { g_launches.fetch_add((unsigned long long)n, std::memory_order_relaxed); }
+
+size_t attn_fwd_ws_bytes(const Dims&) { return 0; }
+size_t attn_bwd_ws_bytes(const Dims& d) { return (size_t)d.heads * d.N * sizeof(float); }
+}  // namespace prism
+
+using namespace prism;
+
+extern "C" prism_status_t prism_query_sizes(const prism_problem_t* prob, prism_sizes_t* sizes) {
+    Dims d;
+    prism_status_t st = make_dims(prob, &d);
+    if (st != PRISM_OK) return st;
+    if (!sizes) return PRISM_ERR_INVALID_ARG;
+    sizes->n_tokens = d.N;
+    sizes->n_zones = d.Z;
+    sizes->max_blocks = d.MB;
+    sizes->sel_words = d.SW;
+    sizes->ws_indicator = zone_indicator_ws_bytes(d);
+    sizes->ws_attn_fwd = attn_fwd_ws_bytes(d);
+    sizes->ws_attn_bwd = attn_bwd_ws_bytes(d);
+    sizes->bytes_P_max = (size_t)d.heads * d.MB * d.MB * sizeof(float);
+    return PRISM_OK;
+}
+
+extern "C" prism_status_t prism_sparse_attn_fwd(const prism_problem_t* prob, const void* Qp, const void* Kp,
+                                                const void* Vp, const int32_t* blk_start,
+                                                const int32_t* gran_blk, const int32_t* n_blk,
+                                                const uint32_t* sel, float scale, void* Op, float* lse,
+                                                uint32_t* dev_status, void* ws, size_t ws_bytes,
+                                                cudaStream_t stream) {
+    Dims d;
+    prism_status_t st = make_dims(prob, &d);
+    if (st != PRISM_OK) return st;
+    if (!ok_ptr(Qp) || !ok_ptr(Kp) || !ok_ptr(Vp) || !ok_ptr(blk_start) || !ok_ptr(gran_blk) ||
+        !ok_ptr(n_blk) || !ok_ptr(sel) || !ok_ptr(Op) || !ok_ptr(lse) || !ok_ptr(dev_status) || !ok_opt(ws))
+        return PRISM_ERR_INVALID_ARG;
+    if (!(scale > 0.f) || !isfinite(scale)) return PRISM_ERR_INVALID_ARG;
+    if (ws_bytes < attn_fwd_ws_bytes(d)) return PRISM_ERR_WORKSPACE;
+    return attn_fwd_simt(d, Qp, Kp, Vp, blk_start, gran_blk, n_blk, sel, scale, Op, lse, stream);
+}
+
+extern "C" prism_status_t prism_sparse_attn_bwd(const prism_problem_t* prob, const void* Qp, const void* Kp,
+                                                const void* Vp, const void* Op, const void* dOp,
+                                                const float* lse, const int32_t* blk_start,
+                                                const int32_t* gran_blk, const int32_t* n_blk,
+                                                const uint32_t* sel, const uint32_t* selT, float scale,
+                                                void* dQp, void* dKp, void* dVp, uint32_t* dev_status,
+                                                void* ws, size_t ws_bytes, cudaStream_t stream) {
+    Dims d;
+    prism_status_t st = make_dims(prob, &d);
+    if (st != PRISM_OK) return st;
+    if (!ok_ptr(Qp) || !ok_ptr(Kp) || !ok_ptr(Vp) || !ok_ptr(Op) || !ok_ptr(dOp) || !ok_ptr(lse) ||
+        !ok_ptr(blk_start) || !ok_ptr(gran_blk) || !ok_ptr(n_blk) || !ok_ptr(sel) || !ok_ptr(selT) ||
+        !ok_ptr(dQp) || !ok_ptr(dKp) || !ok_ptr(dVp) || !ok_ptr(dev_status) || !ok_ptr(ws))
+        return PRISM_ERR_INVALID_ARG;
+    if (!(scale > 0.f) || !isfinite(scale)) return PRISM_ERR_INVALID_ARG;
+    if (ws_bytes < attn_bwd_ws_bytes(d)) return PRISM_ERR_WORKSPACE;
+    return attn_bwd_simt(d, Qp, Kp, Vp, Op, dOp, lse, blk_start, gran_blk, n_blk, sel, selT, scale, dQp, dKp,
+                         dVp, (float*)ws, stream);
+}
+
+extern "C" prism_status_t prism_read_status(const uint32_t* dev_status, uint32_t* host_out, cudaStream_t stream) {
+    if (!dev_status || !host_out) return PRISM_ERR_INVALID_ARG;
+    if (cudaMemcpyAsync(host_out, dev_status, sizeof(uint32_t), cudaMemcpyDeviceToHost, stream) != cudaSuccess)
+        return PRISM_ERR_CUDA;
+    return cudaStreamSynchronize(stream) == cudaSuccess ? PRISM_OK : PRISM_ERR_CUDA;
+}
+
+extern "C" const char* prism_status_string(prism_status_t s) {
+    switch (s) {
+        case PRISM_OK: return "ok";
+        case PRISM_ERR_INVALID_ARG: return "invalid argument (null or misaligned pointer, bad scalar)";
+        case PRISM_ERR_SHAPE: return "grid axes must be positive multiples of 8";
+        case PRISM_ERR_UNSUPPORTED: return "unsupported dtype, head_dim, heads, audio_dim or size";
+        case PRISM_ERR_WORKSPACE: return "workspace too small";
+        case PRISM_ERR_CUDA: return "CUDA error";
+    }
+    return "unknown status";
+}
+
+extern "C" const char* prism_version(void) { return "prism-b200 0.1.0 sm_100a"; }
+
+extern "C" unsigned long long prism_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }

@@ -1,0 +1,277 @@
+// Stage 1: macro-zone statistics and the dual-guidance variation indicator.
+//
+// Prism, Portuguese reading guide, "Método" 1 (Formulação do Indicador de
+// Variação): for each 8x8x8 macro-zone m and axis d in {T,H,W},
+//   sigma^2_{v,d}(m) = (1/D) sum_c (1/8) sum_i (Vbar^{(d)}_{m,i,c} - mu_{m,c})^2,
+//   r_{v,d} = sigma^2_{v,d} / sum_d' sigma^2_{v,d'},
+//   a = ||hhat||_2 per token, abar(m) in [0,1], vhat_{a,d}(m),
+//   g_d = r_{v,d} + abar * vhat_{a,d} + eps.
+// Readings of the unstated parts: D spans every head's channels; abar =
+// A / max A with A the zone mean of a; vhat_{a,d} is the r construction on
+// the scalar field a; rho = max(rho_v, abar) with rho_v the zone's mean
+// token variance of V over its grid maximum; zero total variance gives 1/3.
+//
+// Kernels (all reductions in a fixed order, no float atomics, so the result
+// is deterministic):
+//   k_zone_video    grid (Z, D/CH): one CTA per zone x channel chunk; warp w
+//                   holds temporal slice t = w of the zone, each lane CPL
+//                   channels, 64 tokens kept in registers for the two-pass
+//                   (mean first, then squared deviations) variance.
+//   k_zone_audio    grid Z: one thread per token of the zone.
+//   k_zone_finalize one CTA: per-zone sums over chunks, grid maxima, outputs.
+#include "common.cuh"
+
+namespace prism {
+
+template <typename T> struct VidTraits;
+template <> struct VidTraits<__nv_bfloat16> { static constexpr int CPL = 2; };  // 4 B per lane
+template <> struct VidTraits<float> { static constexpr int CPL = 1; };          // 4 B per lane
+
+// ws layout: video partial sums [Z][nchunk][4] then audio stats [Z][4]
+template <typename T>
+__global__ void __launch_bounds__(256) k_zone_video(const T* __restrict__ V, int H, int W, int64_t D,
+                                                    int nchunk, float* __restrict__ part) {
+    constexpr int CPL = VidTraits<T>::CPL;
+    constexpr int CH = 32 * CPL;                    // channels per CTA
+    __shared__ float sH[8][8][CH];                  // [t][h][c] row sums over w
+    __shared__ float sW[8][8][CH];                  // [t][w][c] column sums over h
+    __shared__ float sT[8][CH];                     // [t][c] slice sums
+    __shared__ float red[8][4];
+
+    const int lane = threadIdx.x & 31, t = threadIdx.x >> 5;
+    const int m = blockIdx.x, chunk = blockIdx.y;
+    const int ZH = H / 8, ZW = W / 8;
+    const int zt = m / (ZH * ZW), zh = (m / ZW) % ZH, zw = m % ZW;
+    const int64_t c0 = (int64_t)chunk * CH + lane * CPL;
+    const int64_t row0 = ((int64_t)(zt * 8 + t) * H + zh * 8) * W + zw * 8;
+
+    // raw storage: one 32-bit word per token (a bf16 pair or one float) keeps
+    // the zone slice at 64 registers for the second (deviation) pass
+    uint32_t raw[8][8];
+#pragma unroll
+    for (int h = 0; h < 8; ++h)
+#pragma unroll
+        for (int w = 0; w < 8; ++w)
+            raw[h][w] = __ldg(reinterpret_cast<const unsigned int*>(V + (row0 + (int64_t)h * W + w) * D + c0));
+    auto val = [&](int h, int w, int k) -> float {
+        if constexpr (CPL == 2) return __uint_as_float(k == 0 ? (raw[h][w] << 16) : (raw[h][w] & 0xffff0000u));
+        else return __uint_as_float(raw[h][w]);
+    };
+
+#pragma unroll
+    for (int k = 0; k < CPL; ++k) {
+        float tot = 0.f;
+#pragma unroll
+        for (int h = 0; h < 8; ++h) {
+            float rs = 0.f;
+#pragma unroll
+            for (int w = 0; w < 8; ++w) rs += val(h, w, k);
+            sH[t][h][lane * CPL + k] = rs;
+            tot += rs;
+        }
+#pragma unroll
+        for (int w = 0; w < 8; ++w) {
+            float cs = 0.f;
+#pragma unroll
+            for (int h = 0; h < 8; ++h) cs += val(h, w, k);
+            sW[t][w][lane * CPL + k] = cs;
+        }
+        sT[t][lane * CPL + k] = tot;
+    }
+    __syncthreads();
+
+    // this thread handles profile index i = t along every axis
+    float aT = 0.f, aH = 0.f, aW = 0.f, aTok = 0.f;
+#pragma unroll
+    for (int k = 0; k < CPL; ++k) {
+        const int c = lane * CPL + k;
+        float zsum = 0.f, hsum = 0.f, wsum = 0.f;
+#pragma unroll
+        for (int tt = 0; tt < 8; ++tt) {
+            zsum += sT[tt][c];
+            hsum += sH[tt][t][c];
+            wsum += sW[tt][t][c];
+        }
+        const float mu = zsum * (1.f / 512.f);
+        const float pT = sT[t][c] * (1.f / 64.f) - mu;
+        const float pH = hsum * (1.f / 64.f) - mu;
+        const float pW = wsum * (1.f / 64.f) - mu;
+        aT += pT * pT;
+        aH += pH * pH;
+        aW += pW * pW;
+        float tv = 0.f;
+#pragma unroll
+        for (int h = 0; h < 8; ++h)
+#pragma unroll
+            for (int w = 0; w < 8; ++w) {
+                float dv = val(h, w, k) - mu;
+                tv += dv * dv;
+            }
+        aTok += tv;
+    }
+    aT = warp_sum(aT); aH = warp_sum(aH); aW = warp_sum(aW); aTok = warp_sum(aTok);
+    if (lane == 0) { red[t][0] = aT; red[t][1] = aH; red[t][2] = aW; red[t][3] = aTok; }
+    __syncthreads();
+    if (threadIdx.x < 4) {
+        float s = 0.f;
+        for (int k = 0; k < 8; ++k) s += red[k][threadIdx.x];
+        part[((int64_t)m * nchunk + chunk) * 4 + threadIdx.x] = s;
+    }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(512) k_zone_audio(const T* __restrict__ hh, int H, int W, int Da,
+                                                    float* __restrict__ astat) {
+    __shared__ float a[512];
+    __shared__ float prof[3][8];
+    const int m = blockIdx.x, tid = threadIdx.x;
+    const int ZH = H / 8, ZW = W / 8;
+    const int zt = m / (ZH * ZW), zh = (m / ZW) % ZH, zw = m % ZW;
+    const int t = tid >> 6, h = (tid >> 3) & 7, w = tid & 7;
+    const int64_t r = ((int64_t)(zt * 8 + t) * H + zh * 8 + h) * W + zw * 8 + w;
+    const T* p = hh + r * Da;
+    float s = 0.f;
+    for (int c = 0; c < Da; c += 2) {
+        float2 v = load2(p + c);
+        s += v.x * v.x + v.y * v.y;
+    }
+    a[tid] = sqrtf(s);
+    __syncthreads();
+    if (tid < 24) {
+        const int ax = tid >> 3, i = tid & 7;
+        float acc = 0.f;
+        for (int u = 0; u < 8; ++u)
+            for (int v = 0; v < 8; ++v) {
+                int tt, hy, wx;
+                if (ax == 0) { tt = i; hy = u; wx = v; }
+                else if (ax == 1) { tt = u; hy = i; wx = v; }
+                else { tt = u; hy = v; wx = i; }
+                acc += a[tt * 64 + hy * 8 + wx];
+            }
+        prof[ax][i] = acc;
+    }
+    __syncthreads();
+    if (tid == 0) {
+        float tot = 0.f;
+        for (int i = 0; i < 8; ++i) tot += prof[0][i];
+        const float A = tot * (1.f / 512.f);
+        astat[m * 4 + 0] = A;
+        for (int ax = 0; ax < 3; ++ax) {
+            float v = 0.f;
+            for (int i = 0; i < 8; ++i) {
+                float dv = prof[ax][i] * (1.f / 64.f) - A;
+                v += dv * dv;
+            }
+            astat[m * 4 + 1 + ax] = v * (1.f / 8.f);
+        }
+    }
+}
+
+__global__ void __launch_bounds__(1024) k_zone_finalize(const float* __restrict__ part,
+                                                        const float* __restrict__ astat, int Z,
+                                                        int nchunk, float invD, float eps,
+                                                        float* __restrict__ g, float* __restrict__ rho,
+                                                        float* __restrict__ abar,
+                                                        float* __restrict__ zstat,
+                                                        float* __restrict__ vsum) {
+    __shared__ float rmx[32], amx[32];
+    const int tid = threadIdx.x;
+    float rmax = 0.f, Amax = 0.f;
+    for (int m = tid; m < Z; m += blockDim.x) {
+        float s[4] = {0.f, 0.f, 0.f, 0.f};
+        const float* pp = part + (int64_t)m * nchunk * 4;
+        for (int k = 0; k < nchunk; ++k)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) s[q] += pp[k * 4 + q];
+        // sigma^2_{v,d} = S_d / (8 D), rho_raw = S_tok / (512 D)
+        vsum[m * 4 + 0] = s[0] * (1.f / 8.f) * invD;
+        vsum[m * 4 + 1] = s[1] * (1.f / 8.f) * invD;
+        vsum[m * 4 + 2] = s[2] * (1.f / 8.f) * invD;
+        const float rr = s[3] * (1.f / 512.f) * invD;
+        vsum[m * 4 + 3] = rr;
+        rmax = fmaxf(rmax, rr);
+        Amax = fmaxf(Amax, astat[m * 4]);
+    }
+    rmax = warp_max(rmax);
+    Amax = warp_max(Amax);
+    if ((tid & 31) == 0) { rmx[tid >> 5] = rmax; amx[tid >> 5] = Amax; }
+    __syncthreads();
+    if (tid < 32) {
+        float a = tid < (int)(blockDim.x >> 5) ? rmx[tid] : 0.f;
+        float b = tid < (int)(blockDim.x >> 5) ? amx[tid] : 0.f;
+        a = warp_max(a);
+        b = warp_max(b);
+        if (tid == 0) { rmx[0] = a; amx[0] = b; }
+    }
+    __syncthreads();
+    rmax = rmx[0];
+    Amax = amx[0];
+    for (int m = tid; m < Z; m += blockDim.x) {
+        const float sv0 = vsum[m * 4 + 0], sv1 = vsum[m * 4 + 1], sv2 = vsum[m * 4 + 2];
+        const float rr = vsum[m * 4 + 3];
+        const float A = astat[m * 4], sa0 = astat[m * 4 + 1], sa1 = astat[m * 4 + 2],
+                    sa2 = astat[m * 4 + 3];
+        const float tv = sv0 + sv1 + sv2, ta = sa0 + sa1 + sa2;
+        const float third = 1.f / 3.f;
+        const float r0 = tv > 0.f ? sv0 / tv : third, r1 = tv > 0.f ? sv1 / tv : third,
+                    r2 = tv > 0.f ? sv2 / tv : third;
+        const float v0 = ta > 0.f ? sa0 / ta : third, v1 = ta > 0.f ? sa1 / ta : third,
+                    v2 = ta > 0.f ? sa2 / ta : third;
+        const float ab = Amax > 0.f ? A / Amax : 0.f;
+        g[m * 3 + 0] = r0 + ab * v0 + eps;
+        g[m * 3 + 1] = r1 + ab * v1 + eps;
+        g[m * 3 + 2] = r2 + ab * v2 + eps;
+        const float rv = rmax > 0.f ? rr / rmax : 0.f;
+        rho[m] = fmaxf(rv, ab);
+        abar[m] = ab;
+        if (zstat) {
+            float* o = zstat + (int64_t)m * 8;
+            o[0] = sv0; o[1] = sv1; o[2] = sv2; o[3] = rr;
+            o[4] = A; o[5] = sa0; o[6] = sa1; o[7] = sa2;
+        }
+    }
+}
+
+size_t zone_indicator_ws_bytes(const Dims& d) {
+    const int CH = d.dtype == PRISM_BF16 ? 64 : 32;
+    const int64_t nchunk = d.D / CH;
+    return (size_t)d.Z * (nchunk * 4 + 4 + 4) * sizeof(float);
+}
+
+}  // namespace prism
+
+using namespace prism;
+
+extern "C" prism_status_t prism_zone_indicator(const prism_problem_t* prob, const void* V,
+                                               const void* hhat, float eps, float* g, float* rho,
+                                               float* abar, float* zone_stats, void* ws,
+                                               size_t ws_bytes, cudaStream_t stream) {
+    Dims d;
+    prism_status_t st = make_dims(prob, &d);
+    if (st != PRISM_OK) return st;
+    if (!ok_ptr(V) || !ok_ptr(hhat) || !ok_ptr(g) || !ok_ptr(rho) || !ok_ptr(abar) ||
+        !ok_opt(zone_stats) || !ok_ptr(ws))
+        return PRISM_ERR_INVALID_ARG;
+    if (!(eps > 0.f) || !isfinite(eps)) return PRISM_ERR_INVALID_ARG;
+    if (d.Da & 1) return PRISM_ERR_UNSUPPORTED;
+    if (ws_bytes < zone_indicator_ws_bytes(d)) return PRISM_ERR_WORKSPACE;
+    const int CH = d.dtype == PRISM_BF16 ? 64 : 32;
+    const int nchunk = (int)(d.D / CH);
+    float* part = (float*)ws;
+    float* astat = part + d.Z * nchunk * 4;
+    float* vsum = astat + d.Z * 4;
+    dim3 gv((unsigned)d.Z, (unsigned)nchunk);
+    if (d.dtype == PRISM_BF16) {
+        k_zone_video<__nv_bfloat16><<<gv, 256, 0, stream>>>((const __nv_bfloat16*)V, d.H, d.W, d.D,
+                                                             nchunk, part);
+        k_zone_audio<__nv_bfloat16><<<(unsigned)d.Z, 512, 0, stream>>>((const __nv_bfloat16*)hhat,
+                                                                       d.H, d.W, d.Da, astat);
+    } else {
+        k_zone_video<float><<<gv, 256, 0, stream>>>((const float*)V, d.H, d.W, d.D, nchunk, part);
+        k_zone_audio<float><<<(unsigned)d.Z, 512, 0, stream>>>((const float*)hhat, d.H, d.W, d.Da,
+                                                               astat);
+    }
+    k_zone_finalize<<<1, 1024, 0, stream>>>(part, astat, (int)d.Z, nchunk, 1.f / (float)d.D, eps, g,
+                                            rho, abar, zone_stats, vsum);
+    return launch_status(3);
+}

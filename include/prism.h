@@ -1,0 +1,215 @@
+/*
+ * prism.h — C ABI of the B200 (sm_100a) implementation of Prism's dynamic,
+ * content-adaptive block-sparse video self-attention.
+ *
+ * Source of the operations: "Prism: Dynamic Sparse Attention for Native 2K
+ * Joint Video-Audio Generation Model Training" (arXiv 2610.05416).  Section
+ * names below refer to its Portuguese reading guide ("Método" 1-3, "Ideias
+ * centrais"), its Chinese reading guide (FAQ) and the sd114.wiki news page
+ * ("工作原理", how it works).
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - Every pointer argument except `prob`, `sizes` and `host_out` is a DEVICE
+ *    pointer, 16-byte aligned.  The caller allocates and owns every buffer
+ *    (sizes from prism_query_sizes); the library allocates nothing and keeps
+ *    no state between calls.
+ *  - Every call is asynchronous on `stream` (0 = legacy default stream).
+ *    Data-dependent counts (the number of blocks n_blk, selection counts)
+ *    stay in device memory; no call synchronises except prism_read_status.
+ *  - Argument and shape errors are returned before any launch, and then no
+ *    output is touched.  A failed launch returns PRISM_ERR_CUDA.  Conditions
+ *    only the device can see set bits in `dev_status` (PRISM_DEV_*); kernels
+ *    then return early instead of trapping.  No C++ exception crosses the ABI.
+ *  - Supported: dtype PRISM_F32 or PRISM_BF16, head_dim 64 or 128,
+ *    1 <= heads <= 64, even audio_dim <= 1024, T, H, W positive multiples of
+ *    8 with N = T*H*W <= 2^24.  Anything else -> PRISM_ERR_UNSUPPORTED or
+ *    PRISM_ERR_SHAPE.
+ *
+ * Notation: N = T*H*W tokens, raster token index r = (t*H + h)*W + w;
+ * Z = N/512 macro-zones of 8x8x8 tokens in raster zone order; D = heads*head_dim.
+ * Layouts (batch 1):
+ *    raster  [N][heads][head_dim]   (Q, K, V, O, dO, dQ, dK, dV as a DiT holds them)
+ *    blocked [heads][N][head_dim]   (tokens in permutation order; block j is the
+ *                                    row range [blk_start[j], blk_start[j+1]))
+ *    hhat    [N][audio_dim]
+ * Storage dtype of every tensor above is prob->dtype; per-zone, per-block and
+ * probability arrays are float32.
+ */
+#ifndef PRISM_H
+#define PRISM_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    PRISM_OK = 0,
+    PRISM_ERR_INVALID_ARG = 1,   /* null / misaligned pointer, bad scalar        */
+    PRISM_ERR_SHAPE = 2,         /* grid axes not positive multiples of 8        */
+    PRISM_ERR_UNSUPPORTED = 3,   /* dtype, head_dim, heads, audio_dim, N too big */
+    PRISM_ERR_WORKSPACE = 4,     /* workspace smaller than prism_query_sizes says */
+    PRISM_ERR_CUDA = 5           /* a CUDA launch or runtime call failed          */
+} prism_status_t;
+
+typedef enum { PRISM_F32 = 0, PRISM_BF16 = 1 } prism_dtype_t;
+
+/* Device status bits (written with atomicOr into a caller-owned uint32). */
+#define PRISM_DEV_TIMEOUT   0x1u   /* a bounded wait in a kernel gave up          */
+#define PRISM_DEV_BAD_INDEX 0x2u   /* an index read from device memory was out of range */
+
+typedef struct {
+    int32_t T, H, W;       /* latent video grid                                  */
+    int32_t heads;         /* attention heads                                    */
+    int32_t head_dim;      /* d                                                  */
+    int32_t audio_dim;     /* channels of hhat                                   */
+    int32_t dtype;         /* prism_dtype_t: storage dtype of the token tensors  */
+} prism_problem_t;
+
+typedef struct {
+    int64_t n_tokens;       /* N                                                 */
+    int64_t n_zones;        /* Z = N / 512                                       */
+    int64_t max_blocks;     /* N / 64: upper bound of n_blk                      */
+    int64_t sel_words;      /* uint32 words per selection row = ceil(max_blocks/32) */
+    size_t  ws_indicator;   /* workspace bytes of prism_zone_indicator           */
+    size_t  ws_attn_fwd;    /* workspace bytes of prism_sparse_attn_fwd          */
+    size_t  ws_attn_bwd;    /* workspace bytes of prism_sparse_attn_bwd          */
+    size_t  bytes_P_max;    /* bytes of P at n_blk = max_blocks (worst case)     */
+} prism_sizes_t;
+
+/* Sizes of every buffer of the path (host only, no CUDA call). */
+prism_status_t prism_query_sizes(const prism_problem_t* prob, prism_sizes_t* sizes);
+
+/*
+ * Stage 1 — macro-zones and the dual-guidance variation indicator
+ * ("Ideias centrais": 8x8x8 macro-zones; "Método" 1: sigma^2_{v,d}, r_{v,d},
+ * a = ||hhat||_2, abar, vhat_{a,d}, g_d = r_{v,d} + abar*vhat_{a,d} + eps).
+ *   V          raster [N][heads*head_dim] (all heads' channels form D)
+ *   hhat       [N][audio_dim], cached audio-to-video cross-attention output
+ *   eps        the indicator's epsilon (> 0)
+ * Outputs (float32, zone-major, raster zone order):
+ *   g [Z][3] (T, H, W);  rho [Z] = max(rho_v, abar) where rho_v is the zone's
+ *   channel-averaged token variance of V over its grid maximum;  abar [Z] =
+ *   A(m)/max A, A = zone mean of a;  zone_stats [Z][8] (nullable) =
+ *   (sigma2_vT, sigma2_vH, sigma2_vW, rho_raw, A, sigma2_aT, sigma2_aH, sigma2_aW).
+ * ws: >= sizes.ws_indicator bytes of scratch.
+ */
+prism_status_t prism_zone_indicator(const prism_problem_t* prob, const void* V, const void* hhat,
+                                    float eps, float* g, float* rho, float* abar,
+                                    float* zone_stats, void* ws, size_t ws_bytes,
+                                    cudaStream_t stream);
+
+/*
+ * Stage 2 — block volume and shape quantisation ("Método" 2): B(m) = 64 if
+ * rho >= tau128, 128 if tau256 <= rho < tau128, else 256; l*_d =
+ * -1/2 log2 g_d + (log2 B + 1/2 sum log2 g)/3; the shape is the candidate of
+ * volume B nearest to l* in log2 space (edges in {2,4,8}: 16 candidates
+ * numbered by (volume, b_T, b_H, b_W) ascending; exact ties go to the smaller
+ * id).  Also builds the token permutation (zones in raster order, blocks in
+ * raster order inside a zone, tokens in raster order inside a block).
+ *   shape_id  [Z] uint8           perm [N] int32: perm[p] = raster index of row p
+ *   inv_perm  [N] int32 (nullable): inv_perm[perm[p]] = p
+ *   blk_start [max_blocks+1] int32: entries past n_blk hold N
+ *   gran_blk  [N/64] int32: block index of each 64-row granule
+ *   n_blk     [1] int32 (device)  margin [Z][2] float32 (nullable): (second-best
+ *             minus best squared distance, min |rho - tau|)
+ */
+prism_status_t prism_assign_shapes(const prism_problem_t* prob, const float* g, const float* rho,
+                                   float tau128, float tau256, uint8_t* shape_id, int32_t* perm,
+                                   int32_t* inv_perm, int32_t* blk_start, int32_t* gran_blk,
+                                   int32_t* n_blk, float* margin, cudaStream_t stream);
+
+/*
+ * Stage 3 — gather raster tokens into block order and head-major layout
+ * (news page, "工作原理" step 4, and its inverse that restores the layout).
+ *   prism_permute:   dst_blocked[h][p][:] = src_raster[perm[p]][h][:]
+ *   prism_unpermute: dst_raster[perm[p]][h][:] = src_blocked[h][p][:]
+ * Bit copies in prob->dtype.
+ */
+prism_status_t prism_permute(const prism_problem_t* prob, const void* src_raster,
+                             const int32_t* perm, void* dst_blocked, cudaStream_t stream);
+prism_status_t prism_unpermute(const prism_problem_t* prob, const void* src_blocked,
+                               const int32_t* perm, void* dst_raster, cudaStream_t stream);
+
+/*
+ * Stage 4 — pooled block representatives and block probabilities ("Método" 3):
+ * Qbar_i, Kbar_j = means over the block's rows (float32 [heads][max_blocks][d]);
+ * s_ij = scale * Qbar_i . Kbar_j;  P_i = softmax_j over all n_blk key blocks.
+ * P is packed with the device n_blk: P[(h*n_blk + i)*n_blk + j]; it needs
+ * heads*n_blk^2 floats (at most sizes.bytes_P_max bytes).
+ */
+prism_status_t prism_block_pool_score(const prism_problem_t* prob, const void* Qp, const void* Kp,
+                                      const int32_t* blk_start, const int32_t* n_blk, float scale,
+                                      float* Qbar, float* Kbar, float* P, cudaStream_t stream);
+
+/*
+ * Stage 5 — hybrid selection S_i = Top-k(P_i, k) U Top-p(P_i, p) ("Método" 3).
+ * Both are prefixes of the order (P desc, j asc): Top-p is the shortest prefix
+ * whose sum reaches p (all blocks if p >= 1 or it never does), so S_i is the
+ * first max(min(k, n_blk), n_p) blocks.
+ *   sel       [heads][max_blocks][sel_words] uint32 bitmask, bit j of row i
+ *   sel_count [heads][max_blocks] int32 (|S_i|; rows past n_blk are 0)
+ *   selT      [heads][max_blocks][sel_words] uint32 (nullable): transpose of sel,
+ *             bit i of row j set when j is in S_i (the backward's key-major view)
+ *   margin    [heads][max_blocks] float32 (nullable): smallest gap (order or
+ *             cumulative-sum) that, crossed by rounding, could change S_i
+ *   dev_status  PRISM_DEV_BAD_INDEX if n_blk exceeds the 16384 keys a row can
+ *             sort in shared memory (then every row is left empty).
+ * Rows i >= n_blk are written as empty rows with count 0.
+ */
+prism_status_t prism_block_select(const prism_problem_t* prob, const float* P, const int32_t* n_blk,
+                                  int32_t top_k, float top_p, uint32_t* sel, int32_t* sel_count,
+                                  uint32_t* selT, float* margin, uint32_t* dev_status,
+                                  cudaStream_t stream);
+
+/*
+ * Stage 6 — exact online-softmax attention of every query block over the tokens
+ * of its selected key blocks ("Método" 3; non-causal, scale usually 1/sqrt(d)).
+ *   Qp, Kp, Vp blocked [heads][N][d];  Op blocked;  lse [heads][N] float32
+ *   (natural log of the softmax denominator; -inf for an empty S_i, whose O is 0).
+ * bf16 runs on tcgen05 tensor cores (fp32 accumulation); f32 on CUDA cores.
+ */
+prism_status_t prism_sparse_attn_fwd(const prism_problem_t* prob, const void* Qp, const void* Kp,
+                                     const void* Vp, const int32_t* blk_start,
+                                     const int32_t* gran_blk, const int32_t* n_blk,
+                                     const uint32_t* sel, float scale, void* Op, float* lse,
+                                     uint32_t* dev_status, void* ws, size_t ws_bytes,
+                                     cudaStream_t stream);
+
+/*
+ * Stage 7 — gradients of stage 6 under the fixed selection (Chinese guide,
+ * FAQ on error propagation: rho, g and P_i are constants; gradients flow only
+ * through the attention over the selected blocks).  Delta = rowsum(dO*O),
+ * P = exp(s - lse), dV = P^T dO, dS = P*(dO V^T - Delta), dQ = scale*dS K,
+ * dK = scale*dS^T Q.  Keys no query selected get dK = dV = 0.
+ * All tensors blocked; ws >= sizes.ws_attn_bwd bytes.
+ */
+prism_status_t prism_sparse_attn_bwd(const prism_problem_t* prob, const void* Qp, const void* Kp,
+                                     const void* Vp, const void* Op, const void* dOp,
+                                     const float* lse, const int32_t* blk_start,
+                                     const int32_t* gran_blk, const int32_t* n_blk,
+                                     const uint32_t* sel, const uint32_t* selT, float scale,
+                                     void* dQp, void* dKp, void* dVp, uint32_t* dev_status,
+                                     void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/* Copy a device status word to the host (synchronises `stream`). */
+prism_status_t prism_read_status(const uint32_t* dev_status, uint32_t* host_out, cudaStream_t stream);
+
+/* Static description of a status code. */
+const char* prism_status_string(prism_status_t status);
+
+/* Library version, e.g. "prism-b200 0.1.0 sm_100a". */
+const char* prism_version(void);
+
+/* Number of kernels this library has launched since it was loaded (all
+ * threads, all devices); a diagnostics counter for profiling harnesses. */
+unsigned long long prism_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* PRISM_H */
