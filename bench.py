@@ -157,9 +157,9 @@ def run_step(mod, x, out, grads, timer=None):
     rec(3)
     _abi.prism_permute(mod.prob, x["dO"], mod.perm, mod.dOp)
     rec(4)
-    _abi.prism_sparse_attn_bwd(mod.prob, mod.Qp, mod.Kp, mod.Vp, mod.Op, mod.dOp, mod.lse, mod.blk_start,
-                               mod.gran_blk, mod.n_blk, mod.sel, mod.selT, mod.scale, mod.dQp, mod.dKp,
-                               mod.dVp, mod.dev_status, mod.ws_bwd)
+    _abi.prism_sparse_attn_bwd(mod.prob, mod.Qp, mod.Kp, mod.Vp, mod.Op, mod.Of32, mod.dOp, mod.lse,
+                               mod.blk_start, mod.gran_blk, mod.n_blk, mod.sel, mod.selT, mod.scale,
+                               mod.dQp, mod.dKp, mod.dVp, mod.dev_status, mod.ws_bwd)
     rec(5)
     for src, dst in zip((mod.dQp, mod.dKp, mod.dVp), grads):
         _abi.prism_unpermute(mod.prob, src, mod.perm, dst)

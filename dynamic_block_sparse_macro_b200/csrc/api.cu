@@ -8,9 +8,10 @@ namespace prism {
 size_t zone_indicator_ws_bytes(const Dims& d);
 prism_status_t attn_fwd_simt(const Dims& d, const void* Qp, const void* Kp, const void* Vp,
                              const int32_t* blk_start, const int32_t* gran_blk, const int32_t* n_blk,
-                             const uint32_t* sel, float scale, void* Op, float* lse, cudaStream_t s);
+                             const uint32_t* sel, float scale, void* Op, float* lse, float* o_f32,
+                             cudaStream_t s);
 prism_status_t attn_bwd_simt(const Dims& d, const void* Qp, const void* Kp, const void* Vp, const void* Op,
-                             const void* dOp, const float* lse, const int32_t* blk_start,
+                             const float* o_f32, const void* dOp, const float* lse, const int32_t* blk_start,
                              const int32_t* gran_blk, const int32_t* n_blk, const uint32_t* sel,
                              const uint32_t* selT, float scale, void* dQp, void* dKp, void* dVp,
                              float* delta, cudaStream_t s);
@@ -44,22 +45,23 @@ extern "C" prism_status_t prism_sparse_attn_fwd(const prism_problem_t* prob, con
                                                 const void* Vp, const int32_t* blk_start,
                                                 const int32_t* gran_blk, const int32_t* n_blk,
                                                 const uint32_t* sel, float scale, void* Op, float* lse,
-                                                uint32_t* dev_status, void* ws, size_t ws_bytes,
+                                                float* o_f32, uint32_t* dev_status, void* ws, size_t ws_bytes,
                                                 cudaStream_t stream) {
     Dims d;
     prism_status_t st = make_dims(prob, &d);
     if (st != PRISM_OK) return st;
     if (!ok_ptr(Qp) || !ok_ptr(Kp) || !ok_ptr(Vp) || !ok_ptr(blk_start) || !ok_ptr(gran_blk) ||
-        !ok_ptr(n_blk) || !ok_ptr(sel) || !ok_ptr(Op) || !ok_ptr(lse) || !ok_ptr(dev_status) || !ok_opt(ws))
+        !ok_ptr(n_blk) || !ok_ptr(sel) || !ok_ptr(Op) || !ok_ptr(lse) || !ok_opt(o_f32) ||
+        !ok_ptr(dev_status) || !ok_opt(ws))
         return PRISM_ERR_INVALID_ARG;
     if (!(scale > 0.f) || !isfinite(scale)) return PRISM_ERR_INVALID_ARG;
     if (ws_bytes < attn_fwd_ws_bytes(d)) return PRISM_ERR_WORKSPACE;
-    return attn_fwd_simt(d, Qp, Kp, Vp, blk_start, gran_blk, n_blk, sel, scale, Op, lse, stream);
+    return attn_fwd_simt(d, Qp, Kp, Vp, blk_start, gran_blk, n_blk, sel, scale, Op, lse, o_f32, stream);
 }
 
 extern "C" prism_status_t prism_sparse_attn_bwd(const prism_problem_t* prob, const void* Qp, const void* Kp,
-                                                const void* Vp, const void* Op, const void* dOp,
-                                                const float* lse, const int32_t* blk_start,
+                                                const void* Vp, const void* Op, const float* o_f32,
+                                                const void* dOp, const float* lse, const int32_t* blk_start,
                                                 const int32_t* gran_blk, const int32_t* n_blk,
                                                 const uint32_t* sel, const uint32_t* selT, float scale,
                                                 void* dQp, void* dKp, void* dVp, uint32_t* dev_status,
@@ -67,13 +69,13 @@ extern "C" prism_status_t prism_sparse_attn_bwd(const prism_problem_t* prob, con
     Dims d;
     prism_status_t st = make_dims(prob, &d);
     if (st != PRISM_OK) return st;
-    if (!ok_ptr(Qp) || !ok_ptr(Kp) || !ok_ptr(Vp) || !ok_ptr(Op) || !ok_ptr(dOp) || !ok_ptr(lse) ||
+    if (!ok_ptr(Qp) || !ok_ptr(Kp) || !ok_ptr(Vp) || !ok_ptr(Op) || !ok_opt(o_f32) || !ok_ptr(dOp) || !ok_ptr(lse) ||
         !ok_ptr(blk_start) || !ok_ptr(gran_blk) || !ok_ptr(n_blk) || !ok_ptr(sel) || !ok_ptr(selT) ||
         !ok_ptr(dQp) || !ok_ptr(dKp) || !ok_ptr(dVp) || !ok_ptr(dev_status) || !ok_ptr(ws))
         return PRISM_ERR_INVALID_ARG;
     if (!(scale > 0.f) || !isfinite(scale)) return PRISM_ERR_INVALID_ARG;
     if (ws_bytes < attn_bwd_ws_bytes(d)) return PRISM_ERR_WORKSPACE;
-    return attn_bwd_simt(d, Qp, Kp, Vp, Op, dOp, lse, blk_start, gran_blk, n_blk, sel, selT, scale, dQp, dKp,
+    return attn_bwd_simt(d, Qp, Kp, Vp, Op, o_f32, dOp, lse, blk_start, gran_blk, n_blk, sel, selT, scale, dQp, dKp,
                          dVp, (float*)ws, stream);
 }
 

@@ -41,7 +41,7 @@ __global__ void __launch_bounds__(256) k_fwd_simt(const T* __restrict__ Q, const
                                                   const int32_t* __restrict__ n_blk,
                                                   const uint32_t* __restrict__ sel, int64_t N,
                                                   int64_t MB, int SW, float scale, T* __restrict__ O,
-                                                  float* __restrict__ lse) {
+                                                  float* __restrict__ lse, float* __restrict__ o_f32) {
     constexpr int LD = D + 1, CW = D / 16;
     extern __shared__ float sm[];
     float* Qs = sm;
@@ -138,19 +138,27 @@ __global__ void __launch_bounds__(256) k_fwd_simt(const T* __restrict__ Q, const
         const int64_t r = q0 + ty + 16 * u;
         const float inv = l[u] > 0.f ? 1.f / l[u] : 0.f;
 #pragma unroll
-        for (int w = 0; w < CW; ++w) O[hoff + r * D + tx + 16 * w] = from_f32<T>(acc[u][w] * inv);
+        for (int w = 0; w < CW; ++w) {
+            const float o = acc[u][w] * inv;
+            O[hoff + r * D + tx + 16 * w] = from_f32<T>(o);
+            if (o_f32) o_f32[hoff + r * D + tx + 16 * w] = o;
+        }
         if (tx == 0) lse[(int64_t)hh * N + r] = l[u] > 0.f ? (m2[u] + log2f(l[u])) * kLn2 : -INFINITY;
     }
 }
 
+// Delta = rowsum(dO * O), from the unrounded fp32 O when the forward kept it
 template <typename T, int D>
-__global__ void k_bwd_delta(const T* __restrict__ O, const T* __restrict__ dO, int64_t rows,
-                            float* __restrict__ delta) {
+__global__ void k_bwd_delta(const T* __restrict__ O, const float* __restrict__ o_f32,
+                            const T* __restrict__ dO, int64_t rows, float* __restrict__ delta) {
     const int64_t r = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
     if (r >= rows) return;
     float s = 0.f;
-    for (int c = lane; c < D; c += 32) s += to_f32(O[r * D + c]) * to_f32(dO[r * D + c]);
+    if (o_f32)
+        for (int c = lane; c < D; c += 32) s += o_f32[r * D + c] * to_f32(dO[r * D + c]);
+    else
+        for (int c = lane; c < D; c += 32) s += to_f32(O[r * D + c]) * to_f32(dO[r * D + c]);
     s = warp_sum(s);
     if (lane == 0) delta[r] = s;
 }
@@ -364,25 +372,26 @@ template <int D> constexpr size_t dq_smem() { return (4 * 64 * (D + 1) + 64 * 65
 template <typename T, int D>
 prism_status_t simt_fwd(const Dims& d, const void* Qp, const void* Kp, const void* Vp,
                         const int32_t* blk_start, const int32_t* gran_blk, const int32_t* n_blk,
-                        const uint32_t* sel, float scale, void* Op, float* lse, cudaStream_t s) {
+                        const uint32_t* sel, float scale, void* Op, float* lse, float* o_f32,
+                        cudaStream_t s) {
     auto k = k_fwd_simt<T, D>;
     if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fwd_smem<D>()) != cudaSuccess)
         return PRISM_ERR_CUDA;
     k<<<dim3((unsigned)d.MB, (unsigned)d.heads), 256, fwd_smem<D>(), s>>>(
         (const T*)Qp, (const T*)Kp, (const T*)Vp, blk_start, gran_blk, n_blk, sel, d.N, d.MB, (int)d.SW,
-        scale, (T*)Op, lse);
+        scale, (T*)Op, lse, o_f32);
     return launch_status(1);
 }
 
 template <typename T, int D>
 prism_status_t simt_bwd(const Dims& d, const void* Qp, const void* Kp, const void* Vp, const void* Op,
-                        const void* dOp, const float* lse, const int32_t* blk_start,
+                        const float* o_f32, const void* dOp, const float* lse, const int32_t* blk_start,
                         const int32_t* gran_blk, const int32_t* n_blk, const uint32_t* sel,
                         const uint32_t* selT, float scale, void* dQp, void* dKp, void* dVp,
                         float* delta, cudaStream_t s) {
     const int64_t rows = (int64_t)d.heads * d.N;
-    k_bwd_delta<T, D><<<(unsigned)((rows * 32 + 255) / 256), 256, 0, s>>>((const T*)Op, (const T*)dOp, rows,
-                                                                           delta);
+    k_bwd_delta<T, D><<<(unsigned)((rows * 32 + 255) / 256), 256, 0, s>>>((const T*)Op, o_f32,
+                                                                           (const T*)dOp, rows, delta);
     auto kk = k_bwd_dkdv_simt<T, D>;
     auto kq = k_bwd_dq_simt<T, D>;
     if (cudaFuncSetAttribute(kk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dkdv_smem<D>()) != cudaSuccess ||
@@ -400,21 +409,21 @@ prism_status_t simt_bwd(const Dims& d, const void* Qp, const void* Kp, const voi
 
 prism_status_t attn_fwd_simt(const Dims& d, const void* Qp, const void* Kp, const void* Vp,
                              const int32_t* blk_start, const int32_t* gran_blk, const int32_t* n_blk,
-                             const uint32_t* sel, float scale, void* Op, float* lse, cudaStream_t s) {
+                             const uint32_t* sel, float scale, void* Op, float* lse, float* o_f32,
+                             cudaStream_t s) {
+#define PRISM_FWD_ARGS d, Qp, Kp, Vp, blk_start, gran_blk, n_blk, sel, scale, Op, lse, o_f32, s
     if (d.dtype == PRISM_F32)
-        return d.d == 64 ? simt_fwd<float, 64>(d, Qp, Kp, Vp, blk_start, gran_blk, n_blk, sel, scale, Op, lse, s)
-                         : simt_fwd<float, 128>(d, Qp, Kp, Vp, blk_start, gran_blk, n_blk, sel, scale, Op, lse, s);
-    return d.d == 64
-               ? simt_fwd<__nv_bfloat16, 64>(d, Qp, Kp, Vp, blk_start, gran_blk, n_blk, sel, scale, Op, lse, s)
-               : simt_fwd<__nv_bfloat16, 128>(d, Qp, Kp, Vp, blk_start, gran_blk, n_blk, sel, scale, Op, lse, s);
+        return d.d == 64 ? simt_fwd<float, 64>(PRISM_FWD_ARGS) : simt_fwd<float, 128>(PRISM_FWD_ARGS);
+    return d.d == 64 ? simt_fwd<__nv_bfloat16, 64>(PRISM_FWD_ARGS) : simt_fwd<__nv_bfloat16, 128>(PRISM_FWD_ARGS);
+#undef PRISM_FWD_ARGS
 }
 
 prism_status_t attn_bwd_simt(const Dims& d, const void* Qp, const void* Kp, const void* Vp, const void* Op,
-                             const void* dOp, const float* lse, const int32_t* blk_start,
+                             const float* o_f32, const void* dOp, const float* lse, const int32_t* blk_start,
                              const int32_t* gran_blk, const int32_t* n_blk, const uint32_t* sel,
                              const uint32_t* selT, float scale, void* dQp, void* dKp, void* dVp,
                              float* delta, cudaStream_t s) {
-#define PRISM_BWD_ARGS d, Qp, Kp, Vp, Op, dOp, lse, blk_start, gran_blk, n_blk, sel, selT, scale, dQp, dKp, dVp, delta, s
+#define PRISM_BWD_ARGS d, Qp, Kp, Vp, Op, o_f32, dOp, lse, blk_start, gran_blk, n_blk, sel, selT, scale, dQp, dKp, dVp, delta, s
     if (d.dtype == PRISM_F32)
         return d.d == 64 ? simt_bwd<float, 64>(PRISM_BWD_ARGS) : simt_bwd<float, 128>(PRISM_BWD_ARGS);
     return d.d == 64 ? simt_bwd<__nv_bfloat16, 64>(PRISM_BWD_ARGS) : simt_bwd<__nv_bfloat16, 128>(PRISM_BWD_ARGS);

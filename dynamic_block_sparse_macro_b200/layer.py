@@ -64,6 +64,8 @@ class PrismSparseAttention:
         self.dev_status = torch.zeros(1, dtype=i32, device=dev)
         # stage 6-7
         self.Op = e(heads, N, head_dim, dt=self.tdt)
+        # unrounded O for the backward's Delta (bf16 storage only)
+        self.Of32 = e(heads, N, head_dim) if (with_backward and dtype == "bf16") else None
         self.lse = e(heads, N)
         self.ws_fwd = e(max(16, s.ws_attn_fwd), dt=torch.uint8)
         if with_backward:
@@ -94,8 +96,8 @@ class PrismSparseAttention:
     def attend(self, stream=None):
         """Stage 6 on the blocked tensors."""
         _abi.prism_sparse_attn_fwd(self.prob, self.Qp, self.Kp, self.Vp, self.blk_start, self.gran_blk,
-                                   self.n_blk, self.sel, self.scale, self.Op, self.lse, self.dev_status,
-                                   self.ws_fwd, stream)
+                                   self.n_blk, self.sel, self.scale, self.Op, self.lse, self.Of32,
+                                   self.dev_status, self.ws_fwd, stream)
 
     def forward(self, Q, K, V, hhat, out=None, stream=None):
         """Whole forward; returns O in raster layout."""
@@ -111,7 +113,8 @@ class PrismSparseAttention:
         """Stage 7 for the last forward; returns raster (dQ, dK, dV)."""
         p = self.prob
         _abi.prism_permute(p, dO, self.perm, self.dOp, stream)
-        _abi.prism_sparse_attn_bwd(p, self.Qp, self.Kp, self.Vp, self.Op, self.dOp, self.lse, self.blk_start,
+        _abi.prism_sparse_attn_bwd(p, self.Qp, self.Kp, self.Vp, self.Op, self.Of32, self.dOp, self.lse,
+                                   self.blk_start,
                                    self.gran_blk, self.n_blk, self.sel, self.selT, self.scale, self.dQp,
                                    self.dKp, self.dVp, self.dev_status, self.ws_bwd, stream)
         outs = []

@@ -171,13 +171,17 @@ prism_status_t prism_block_select(const prism_problem_t* prob, const float* P, c
  * of its selected key blocks ("Método" 3; non-causal, scale usually 1/sqrt(d)).
  *   Qp, Kp, Vp blocked [heads][N][d];  Op blocked;  lse [heads][N] float32
  *   (natural log of the softmax denominator; -inf for an empty S_i, whose O is 0).
+ *   o_f32 (nullable) blocked [heads][N][d] float32: the unrounded O, for the
+ *   backward's Delta (with a bf16 O, rowsum(dO*O) carries O's rounding error,
+ *   which dominates dQ/dK when the attention is diffuse).
+ * ws: >= sizes.ws_attn_fwd bytes (may be NULL when that is 0).
  * bf16 runs on tcgen05 tensor cores (fp32 accumulation); f32 on CUDA cores.
  */
 prism_status_t prism_sparse_attn_fwd(const prism_problem_t* prob, const void* Qp, const void* Kp,
                                      const void* Vp, const int32_t* blk_start,
                                      const int32_t* gran_blk, const int32_t* n_blk,
                                      const uint32_t* sel, float scale, void* Op, float* lse,
-                                     uint32_t* dev_status, void* ws, size_t ws_bytes,
+                                     float* o_f32, uint32_t* dev_status, void* ws, size_t ws_bytes,
                                      cudaStream_t stream);
 
 /*
@@ -186,11 +190,12 @@ prism_status_t prism_sparse_attn_fwd(const prism_problem_t* prob, const void* Qp
  * through the attention over the selected blocks).  Delta = rowsum(dO*O),
  * P = exp(s - lse), dV = P^T dO, dS = P*(dO V^T - Delta), dQ = scale*dS K,
  * dK = scale*dS^T Q.  Keys no query selected get dK = dV = 0.
+ * Delta uses o_f32 when it is given (the forward's unrounded O), else Op.
  * All tensors blocked; ws >= sizes.ws_attn_bwd bytes.
  */
 prism_status_t prism_sparse_attn_bwd(const prism_problem_t* prob, const void* Qp, const void* Kp,
-                                     const void* Vp, const void* Op, const void* dOp,
-                                     const float* lse, const int32_t* blk_start,
+                                     const void* Vp, const void* Op, const float* o_f32,
+                                     const void* dOp, const float* lse, const int32_t* blk_start,
                                      const int32_t* gran_blk, const int32_t* n_blk,
                                      const uint32_t* sel, const uint32_t* selT, float scale,
                                      void* dQp, void* dKp, void* dVp, uint32_t* dev_status,
