@@ -68,7 +68,8 @@ def test_degenerate_constant_video_silent_audio():
     x = _inputs(cfg)
     x["V"] = torch.full_like(x["V"], 0.5)
     x["hhat"] = torch.zeros_like(x["hhat"])
-    rep = check_layer(cfg, x)
+    # exact gradients are 0 here (dP - Delta = 0): measure fp32 noise against ||dO||
+    rep = check_layer(cfg, x, grad_floor=1.0)
     assert rep["volume_mix"] == {64: 0, 128: 0, 256: 4}
 
 
