@@ -22,7 +22,9 @@ DEV_TIMEOUT, DEV_BAD_INDEX = 0x1, 0x2
 EXPORTS = ("prism_query_sizes", "prism_zone_indicator", "prism_assign_shapes", "prism_permute",
            "prism_unpermute", "prism_block_pool_score", "prism_block_select",
            "prism_sparse_attn_fwd", "prism_sparse_attn_bwd", "prism_read_status",
-           "prism_status_string", "prism_version", "prism_launch_count")
+           "prism_status_string", "prism_version", "prism_launch_count",
+           "prism_zone_indicator_noalloc")
+NOALLOC_SCRATCH_BYTES = 2 << 20
 
 
 class Problem(ctypes.Structure):
@@ -54,6 +56,7 @@ _PROB = ctypes.POINTER(Problem)
 _SIGS = {
     "prism_query_sizes": [_PROB, ctypes.POINTER(Sizes)],
     "prism_zone_indicator": [_PROB, _P, _P, _F, _P, _P, _P, _P, _P, _SZ, _P],
+    "prism_zone_indicator_noalloc": [_PROB, _P, _P, _F, _P, _P, _P, _P, _P],
     "prism_assign_shapes": [_PROB, _P, _P, _F, _F, _P, _P, _P, _P, _P, _P, _P, _P],
     "prism_permute": [_PROB, _P, _P, _P, _P],
     "prism_unpermute": [_PROB, _P, _P, _P, _P],
@@ -126,6 +129,14 @@ def prism_zone_indicator(prob, V, hhat, eps, g, rho, abar, zone_stats, ws, strea
     _check("prism_zone_indicator", lib().prism_zone_indicator(
         ctypes.byref(prob), _ptr(V), _ptr(hhat), eps, _ptr(g), _ptr(rho), _ptr(abar),
         _ptr(zone_stats), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def prism_zone_indicator_noalloc(prob, V, hhat, eps, g, rho, abar, zone_stats, stream=None):
+    """Same as prism_zone_indicator with the library's own fixed scratch array,
+    for callers that cannot allocate a workspace (see include/prism.h)."""
+    _check("prism_zone_indicator_noalloc", lib().prism_zone_indicator_noalloc(
+        ctypes.byref(prob), _ptr(V), _ptr(hhat), eps, _ptr(g), _ptr(rho), _ptr(abar),
+        _ptr(zone_stats), _stream(stream)))
 
 
 def prism_assign_shapes(prob, g, rho, tau128, tau256, shape_id, perm, inv_perm, blk_start,

@@ -19,6 +19,8 @@
 //                   (mean first, then squared deviations) variance.
 //   k_zone_audio    grid Z: one thread per token of the zone.
 //   k_zone_finalize one CTA: per-zone sums over chunks, grid maxima, outputs.
+#include <mutex>
+
 #include "common.cuh"
 
 namespace prism {
@@ -274,4 +276,59 @@ extern "C" prism_status_t prism_zone_indicator(const prism_problem_t* prob, cons
     k_zone_finalize<<<1, 1024, 0, stream>>>(part, astat, (int)d.Z, nchunk, 1.f / (float)d.D, eps, g,
                                             rho, abar, zone_stats, vsum);
     return launch_status(3);
+}
+
+// ---------------------------------------------------------------------------
+// Allocation-free variant of prism_zone_indicator.
+//
+// Some callers cannot hand us a workspace: a host that has no device
+// allocator wired in (a plain C program driving the library through this
+// ABI), or a service whose memory footprint is fixed at start-up and which
+// forbids device allocations afterwards.  For them the indicator's scratch
+// (per zone x channel-chunk partial sums, per-zone audio statistics and
+// per-zone totals) lives in a fixed array inside this library instead.
+//
+// The array is a file-scope __device__ symbol, so every GPU that loads the
+// library holds PRISM_NOALLOC_SCRATCH_BYTES of it until the process exits.
+// Host code cannot use the symbol's name as a device address; the address is
+// looked up with cudaGetSymbolAddress once per device, the first time the
+// entry point runs with that device current (so that first call should come
+// before any stream capture).  Every call shares the one array: two calls
+// whose kernels overlap on the GPU race on it.  Each call writes every
+// scratch word it later reads, so nothing has to be cleared between calls.
+// ---------------------------------------------------------------------------
+static __device__ __align__(256) unsigned char g_noalloc_scratch[PRISM_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mu;
+void* g_scratch_ptr[kMaxDevices] = {};
+
+prism_status_t noalloc_scratch(void** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return PRISM_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_scratch_mu);
+    if (!g_scratch_ptr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return PRISM_ERR_CUDA;
+        g_scratch_ptr[dev] = p;
+    }
+    *out = g_scratch_ptr[dev];
+    return PRISM_OK;
+}
+}  // namespace
+
+extern "C" prism_status_t prism_zone_indicator_noalloc(const prism_problem_t* prob, const void* V,
+                                                       const void* hhat, float eps, float* g, float* rho,
+                                                       float* abar, float* zone_stats,
+                                                       cudaStream_t stream) {
+    Dims d;
+    prism_status_t st = make_dims(prob, &d);
+    if (st != PRISM_OK) return st;
+    if (zone_indicator_ws_bytes(d) > (size_t)PRISM_NOALLOC_SCRATCH_BYTES) return PRISM_ERR_WORKSPACE;
+    void* scratch = nullptr;
+    st = noalloc_scratch(&scratch);
+    if (st != PRISM_OK) return st;
+    return prism_zone_indicator(prob, V, hhat, eps, g, rho, abar, zone_stats, scratch,
+                                (size_t)PRISM_NOALLOC_SCRATCH_BYTES, stream);
 }

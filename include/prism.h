@@ -103,6 +103,31 @@ prism_status_t prism_zone_indicator(const prism_problem_t* prob, const void* V, 
                                     float* zone_stats, void* ws, size_t ws_bytes,
                                     cudaStream_t stream);
 
+/* Size of the library-owned scratch array behind prism_zone_indicator_noalloc. */
+#define PRISM_NOALLOC_SCRATCH_BYTES (2u << 20)
+
+/*
+ * prism_zone_indicator without a workspace argument: same inputs, outputs
+ * and results, for callers that cannot allocate device memory themselves (a
+ * C host with no device allocator of its own, or a service whose device
+ * footprint is fixed at start-up).  The paper has no counterpart; this is a
+ * library convenience.
+ *  - Scratch is a fixed PRISM_NOALLOC_SCRATCH_BYTES (2 MiB) array inside the
+ *    library, held by every GPU that loads it until the process exits.  A
+ *    problem needing more (zones * (4*D/CH + 8) floats, CH = 64 channels for
+ *    bf16, 32 for f32; the 1,032,192-token bf16 grid needs 1.6 MB) returns
+ *    PRISM_ERR_WORKSPACE before any launch.
+ *  - Nothing is allocated: no cudaMalloc/cudaFree or allocating library call.
+ *  - The first call on each device looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call
+ *    before any stream capture.
+ *  - All calls share the array: calls whose kernels overlap on the GPU (two
+ *    streams, two host threads) race on it and must be serialised by the caller.
+ */
+prism_status_t prism_zone_indicator_noalloc(const prism_problem_t* prob, const void* V,
+                                            const void* hhat, float eps, float* g, float* rho,
+                                            float* abar, float* zone_stats, cudaStream_t stream);
+
 /*
  * Stage 2 — block volume and shape quantisation ("Método" 2): B(m) = 64 if
  * rho >= tau128, 128 if tau256 <= rho < tau128, else 256; l*_d =
