@@ -6,6 +6,10 @@
 
 namespace prism {
 size_t zone_indicator_ws_bytes(const Dims& d);
+prism_status_t attn_fwd_sm100(const Dims& d, const void* Qp, const void* Kp, const void* Vp,
+                              const int32_t* blk_start, const int32_t* gran_blk, const int32_t* n_blk,
+                              const uint32_t* sel, float scale, void* Op, float* lse, float* o_f32,
+                              uint32_t* dev_status, cudaStream_t s);
 prism_status_t attn_fwd_simt(const Dims& d, const void* Qp, const void* Kp, const void* Vp,
                              const int32_t* blk_start, const int32_t* gran_blk, const int32_t* n_blk,
                              const uint32_t* sel, float scale, void* Op, float* lse, float* o_f32,
@@ -56,6 +60,9 @@ extern "C" prism_status_t prism_sparse_attn_fwd(const prism_problem_t* prob, con
         return PRISM_ERR_INVALID_ARG;
     if (!(scale > 0.f) || !isfinite(scale)) return PRISM_ERR_INVALID_ARG;
     if (ws_bytes < attn_fwd_ws_bytes(d)) return PRISM_ERR_WORKSPACE;
+    if (d.dtype == PRISM_BF16)
+        return attn_fwd_sm100(d, Qp, Kp, Vp, blk_start, gran_blk, n_blk, sel, scale, Op, lse, o_f32, dev_status,
+                              stream);
     return attn_fwd_simt(d, Qp, Kp, Vp, blk_start, gran_blk, n_blk, sel, scale, Op, lse, o_f32, stream);
 }
 

@@ -21,6 +21,15 @@ def test_tiny_f32_all_stages():
 
 
 @pytest.mark.parametrize("d", [128, 64])
+def test_bf16_tiny_grid(d):
+    # 8x16x16 grid, 2 heads: 16 query tiles per head
+    from gpu_parity import check_layer
+    cfg = get_config("720p", T=8, H=16, W=16, heads=2, head_dim=d)
+    rep = check_layer(cfg, _inputs(cfg))
+    print("bf16 tiny", d, rep)
+
+
+@pytest.mark.parametrize("d", [128, 64])
 def test_bf16_aniso_several_tiles(d):
     # 16x32x32 grid (16,384 tokens, 32 zones), 3 heads: mixed block volumes,
     # many 64-row tiles, several selected blocks per row
