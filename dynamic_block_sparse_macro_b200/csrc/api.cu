@@ -10,6 +10,11 @@ prism_status_t attn_fwd_sm100(const Dims& d, const void* Qp, const void* Kp, con
                               const int32_t* blk_start, const int32_t* gran_blk, const int32_t* n_blk,
                               const uint32_t* sel, float scale, void* Op, float* lse, float* o_f32,
                               uint32_t* dev_status, cudaStream_t s);
+prism_status_t attn_bwd_sm100(const Dims& d, const void* Qp, const void* Kp, const void* Vp, const void* Op,
+                              const float* o_f32, const void* dOp, const float* lse, const int32_t* blk_start,
+                              const int32_t* gran_blk, const int32_t* n_blk, const uint32_t* sel,
+                              const uint32_t* selT, float scale, void* dQp, void* dKp, void* dVp,
+                              uint32_t* dev_status, float* delta, cudaStream_t s);
 prism_status_t attn_fwd_simt(const Dims& d, const void* Qp, const void* Kp, const void* Vp,
                              const int32_t* blk_start, const int32_t* gran_blk, const int32_t* n_blk,
                              const uint32_t* sel, float scale, void* Op, float* lse, float* o_f32,
@@ -82,6 +87,9 @@ extern "C" prism_status_t prism_sparse_attn_bwd(const prism_problem_t* prob, con
         return PRISM_ERR_INVALID_ARG;
     if (!(scale > 0.f) || !isfinite(scale)) return PRISM_ERR_INVALID_ARG;
     if (ws_bytes < attn_bwd_ws_bytes(d)) return PRISM_ERR_WORKSPACE;
+    if (d.dtype == PRISM_BF16)
+        return attn_bwd_sm100(d, Qp, Kp, Vp, Op, o_f32, dOp, lse, blk_start, gran_blk, n_blk, sel, selT, scale, dQp,
+                              dKp, dVp, dev_status, (float*)ws, stream);
     return attn_bwd_simt(d, Qp, Kp, Vp, Op, o_f32, dOp, lse, blk_start, gran_blk, n_blk, sel, selT, scale, dQp, dKp,
                          dVp, (float*)ws, stream);
 }

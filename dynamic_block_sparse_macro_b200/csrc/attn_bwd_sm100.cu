@@ -1,0 +1,519 @@
+// Stage 7 on sm_100a tensor cores: block-sparse attention backward for bf16.
+//
+// Chinese reading guide of the Prism paper, FAQ on error propagation: rho, g
+// and the block probabilities P_i are constants in the backward; gradients
+// flow only through the attention over the selected key-value blocks.  With
+// P = exp(s - lse) over the selected keys and Delta = rowsum(dO * O):
+//   dV = P^T dO,  dP = dO V^T,  dS = P * (dP - Delta),  dQ = scale dS K,
+//   dK = scale dS^T Q.
+//
+// Two kernels, no atomics (deterministic):
+//   k_bwd_dq_sm100    query-stationary: per (128-row query tile, head) walk the
+//                     key granules of S_b0 U S_b1; per 64-key granule
+//                     S = Q K^T and dP = dO V^T (M=128, N=64) into TMEM, dS as
+//                     bf16 back into TMEM, dQ += dS K (K MN-major in smem).
+//   k_bwd_dkdv_sm100  key-stationary: per (128-key tile, head) walk the query
+//                     granules of the query blocks that selected the tile's key
+//                     blocks (the key-major selection); per 64-query granule
+//                     S^T = K Q^T and dP^T = V dO^T, then P^T and dS^T as bf16
+//                     in TMEM, dV += P^T dO and dK += dS^T Q.
+// Both double-buffer the granule products in TMEM so that the tensor core
+// works on granule g+1 while four warps do the elementwise step of granule g,
+// and stream granules through a 3-stage TMA ring.  Roles: warp 0 TMA, warp 1
+// TMEM allocation + MMA issue (one thread), warps 2-5 one tile row per thread.
+// Every wait is bounded; a timeout sets PRISM_DEV_TIMEOUT.
+#include "common.cuh"
+#include "sm100.cuh"
+
+namespace prism {
+
+using namespace sm100;
+
+prism_status_t bwd_delta(const Dims& d, const void* Op, const float* o_f32, const void* dOp, float* delta,
+                         cudaStream_t s);
+
+namespace {
+
+constexpr int kTile = 128 * 128;           // bytes: 128 rows x 64 bf16 columns
+constexpr int kGran = 64 * 128;            // bytes: 64 rows x 64 bf16 columns
+constexpr int kStages = 3;
+constexpr uint32_t kTmemCols = 512;
+constexpr float kLog2e = 1.4426950408889634f;
+
+template <int D>
+struct BwdLayout {
+    static constexpr int NR = D / 64;
+    static constexpr int A0 = 0;                       // stationary operand 1 (Q or K)
+    static constexpr int A1 = NR * kTile;              // stationary operand 2 (dO or V)
+    static constexpr int RING = 2 * NR * kTile;        // streamed granules
+    static constexpr int STAGE = 2 * NR * kGran;       // two operands per stage
+    static constexpr int CTRL = RING + kStages * STAGE;
+    static constexpr int BYTES = CTRL + 256;
+    static constexpr int ALLOC = BYTES + 1024;
+};
+
+struct Bars {
+    uint64_t* stat;            // stationary tiles landed
+    uint64_t* full;            // [kStages] streamed granule landed
+    uint64_t* empty;           // [kStages] granule stage free
+    uint64_t* prod;            // [2] products of a granule in TMEM
+    uint64_t* elem;            // [2] elementwise results of a granule in TMEM (128 arrivals)
+    uint64_t* fin;             // all MMAs done
+    uint32_t* tmem_slot;
+    volatile int* abort_flag;
+    int* ng_slot;
+};
+
+__device__ __forceinline__ Bars carve(uint8_t* ctrl) {
+    uint64_t* b = reinterpret_cast<uint64_t*>(ctrl);
+    Bars r;
+    r.stat = b;
+    r.full = b + 1;
+    r.empty = b + 1 + kStages;
+    r.prod = b + 1 + 2 * kStages;
+    r.elem = b + 3 + 2 * kStages;
+    r.fin = b + 5 + 2 * kStages;
+    r.tmem_slot = reinterpret_cast<uint32_t*>(b + 6 + 2 * kStages);
+    r.abort_flag = reinterpret_cast<volatile int*>(r.tmem_slot + 1);
+    r.ng_slot = reinterpret_cast<int*>(r.tmem_slot + 2);
+    return r;
+}
+
+__device__ __forceinline__ void init_bars(const Bars& B) {
+    mbar_init(B.stat, 1);
+    for (int s = 0; s < kStages; ++s) {
+        mbar_init(B.full + s, 1);
+        mbar_init(B.empty + s, 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+        mbar_init(B.prod + b, 1);
+        mbar_init(B.elem + b, 128);
+    }
+    mbar_init(B.fin, 1);
+    *B.abort_flag = 0;
+    fence_mbar_init();
+}
+
+// descriptor offsets: K-major operand, k-th 16-element step of the contraction over d
+__device__ __forceinline__ uint32_t kmaj_off(int k, int region) { return (k >> 2) * region + (k & 3) * 32; }
+
+// TMA producer shared by both kernels: stationary tiles once, then the
+// granule stream of the walk (two operands per granule).
+template <int D>
+__device__ void produce(const CUtensorMap* m0, const CUtensorMap* m1, const CUtensorMap* g0,
+                        const CUtensorMap* g1, uint8_t* sm, const Bars& B, int64_t row0, int tile_row,
+                        GranuleWalk& walk, int ng, uint32_t* dev_status) {
+    using L = BwdLayout<D>;
+    tma_prefetch_desc(m0);
+    tma_prefetch_desc(m1);
+    tma_prefetch_desc(g0);
+    tma_prefetch_desc(g1);
+    mbar_expect_tx(B.stat, 2 * L::NR * kTile);
+    for (int r = 0; r < L::NR; ++r) {
+        tma_load_2d(sm + L::A0 + r * kTile, m0, B.stat, 64 * r, (int)(row0 + tile_row));
+        tma_load_2d(sm + L::A1 + r * kTile, m1, B.stat, 64 * r, (int)(row0 + tile_row));
+    }
+    int issued = 0;
+    for (int g = 0; g < ng && !*B.abort_flag; ++g) {
+        int row;
+        uint32_t m;
+        walk.next(row, m);
+        const int s = g % kStages;
+        if (g >= kStages && !mbar_wait(B.empty + s, ((g / kStages) - 1) & 1, B.abort_flag, dev_status)) break;
+        uint8_t* st = sm + L::RING + s * L::STAGE;
+        mbar_expect_tx(B.full + s, L::STAGE);
+        for (int r = 0; r < L::NR; ++r) {
+            tma_load_2d(st + r * kGran, g0, B.full + s, 64 * r, (int)(row0 + row));
+            tma_load_2d(st + (L::NR + r) * kGran, g1, B.full + s, 64 * r, (int)(row0 + row));
+        }
+        ++issued;
+    }
+    if (*B.abort_flag) {
+        volatile int no_abort = 0;
+        for (int g = (issued > kStages ? issued - kStages : 0); g < issued; ++g)
+            mbar_wait(B.full + g % kStages, (g / kStages) & 1, &no_abort, dev_status);
+    }
+}
+
+// ============================================================================ dQ
+template <int D>
+__global__ void __launch_bounds__(192, 1)
+k_bwd_dq_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmdO,
+               const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+               const int32_t* __restrict__ blk_start, const int32_t* __restrict__ gran_blk,
+               const int32_t* __restrict__ n_blk, const uint32_t* __restrict__ sel,
+               const float* __restrict__ lse, const float* __restrict__ delta, int64_t N, int64_t MB, int SW,
+               float scale, __nv_bfloat16* __restrict__ dQ, uint32_t* __restrict__ dev_status) {
+    using L = BwdLayout<D>;
+    constexpr uint32_t cdQ = 0, cS = 128, cP = 192;   // + 128 * buffer for S / dP
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    Bars B = carve(sm + L::CTRL);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int tile = blockIdx.x, hh = blockIdx.y;
+    const int nb = *n_blk;
+    const int b0 = gran_blk[2 * tile], b1 = gran_blk[2 * tile + 1];
+    if (b0 < 0 || b0 >= nb || b1 < 0 || b1 >= nb) {
+        if (threadIdx.x == 0) atomicOr(dev_status, PRISM_DEV_BAD_INDEX);
+        return;
+    }
+    const uint32_t* r0 = sel + ((int64_t)hh * MB + b0) * SW;
+    const uint32_t* r1 = sel + ((int64_t)hh * MB + b1) * SW;
+    const int wn = (nb + 31) >> 5;
+    const int64_t row0 = (int64_t)hh * N;
+
+    if (threadIdx.x == 0) init_bars(B);
+    if (warp == 0) {
+        const int cnt = count_granules(r0, r1, blk_start, wn, lane);
+        if (lane == 0) *B.ng_slot = cnt;
+    } else if (warp == 1) {
+        tmem_alloc(B.tmem_slot, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tb = *B.tmem_slot;
+    const int ng = *B.ng_slot;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            GranuleWalk walk;
+            walk.init(r0, r1, blk_start, wn);
+            produce<D>(&tmQ, &tmdO, &tmK, &tmV, sm, B, row0, 128 * tile, walk, ng, dev_status);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            const uint32_t idPS = idesc_bf16_f32(128, 64, false, false);
+            const uint32_t idQ = idesc_bf16_f32(128, D, false, true);
+            const uint32_t aQ = smem_u32(sm + L::A0), adO = smem_u32(sm + L::A1), aR = smem_u32(sm + L::RING);
+            bool ok = mbar_wait(B.stat, 0, B.abort_flag, dev_status);
+            tc_fence_after();
+            for (int g = 0; ok && g <= ng; ++g) {
+                if (g < ng) {
+                    const int s = g % kStages, b = g & 1;
+                    if (!mbar_wait(B.full + s, (g / kStages) & 1, B.abort_flag, dev_status)) break;
+                    tc_fence_after();
+                    const uint32_t aK = aR + s * L::STAGE, aV = aK + L::NR * kGran;
+#pragma unroll
+                    for (int k = 0; k < D / 16; ++k)
+                        mma_ss(tb + cS + 128 * b, sdesc_sw128(aQ + kmaj_off(k, kTile), 16, 1024),
+                               sdesc_sw128(aK + kmaj_off(k, kGran), 16, 1024), idPS, k > 0);
+#pragma unroll
+                    for (int k = 0; k < D / 16; ++k)
+                        mma_ss(tb + cP + 128 * b, sdesc_sw128(adO + kmaj_off(k, kTile), 16, 1024),
+                               sdesc_sw128(aV + kmaj_off(k, kGran), 16, 1024), idPS, k > 0);
+                    tc_commit(B.prod + b);
+                }
+                if (g > 0) {
+                    const int gp = g - 1, s = gp % kStages, b = gp & 1;
+                    if (!mbar_wait(B.elem + b, (gp >> 1) & 1, B.abort_flag, dev_status)) break;
+                    tc_fence_after();
+                    const uint32_t aK = aR + s * L::STAGE;
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        mma_ts(tb + cdQ, tb + cS + 128 * b + 8 * k, sdesc_sw128(aK + k * 2048, kGran, 1024), idQ,
+                               (gp > 0 || k > 0) ? 1u : 0u);
+                    tc_commit(B.empty + s);
+                }
+            }
+            tc_commit(B.fin);
+            if (*B.abort_flag) {
+                volatile int no_abort = 0;
+                mbar_wait(B.fin, 0, &no_abort, dev_status);
+            }
+        }
+    } else {
+        const int sub = warp & 3, row = sub * 32 + lane, half = row >> 6;
+        const uint32_t tl = tb + ((uint32_t)(sub * 32) << 16);
+        const int64_t grow = row0 + 128 * tile + row;
+        const float lse2 = lse[grow] * kLog2e, dl = delta[grow];
+        const float sl2 = scale * kLog2e;
+        GranuleWalk walk;
+        if (lane == 0) walk.init(r0, r1, blk_start, wn);
+        bool ok = true;
+        for (int g = 0; g < ng; ++g) {
+            const int b = g & 1;
+            uint32_t mk = 0;
+            if (lane == 0) {
+                int rr;
+                walk.next(rr, mk);
+            }
+            mk = __shfl_sync(0xffffffffu, mk, 0);
+            const bool valid = (mk >> half) & 1u;
+            const bool got = mbar_wait(B.prod + b, (g >> 1) & 1, B.abort_flag, dev_status);
+            if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+            tc_fence_after();
+#pragma unroll
+            for (int hq = 0; hq < 2; ++hq) {
+                uint32_t s[32], p[32], o[16];
+                tmem_ld32(tl + cS + 128 * b + 32 * hq, s);
+                tmem_ld32(tl + cP + 128 * b + 32 * hq, p);
+                tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    float d0 = 0.f, d1 = 0.f;
+                    if (valid) {
+                        const float p0 = exp2f(fmaf(__uint_as_float(s[2 * i]), sl2, -lse2));
+                        const float p1 = exp2f(fmaf(__uint_as_float(s[2 * i + 1]), sl2, -lse2));
+                        d0 = p0 * (__uint_as_float(p[2 * i]) - dl);
+                        d1 = p1 * (__uint_as_float(p[2 * i + 1]) - dl);
+                    }
+                    o[i] = pack_bf16x2(d0, d1);
+                }
+                tmem_st16(tl + cS + 128 * b + 16 * hq, o);     // dS (bf16) over the consumed S columns
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(B.elem + b);
+        }
+        const bool fin = ok && mbar_wait(B.fin, 0, B.abort_flag, dev_status);
+        if (__all_sync(0xffffffffu, fin)) {
+            tc_fence_after();
+            __nv_bfloat16* out = dQ + grow * D;
+#pragma unroll
+            for (int q = 0; q < D / 32; ++q) {
+                uint32_t r[32];
+                tmem_ld32(tl + cdQ + 32 * q, r);
+                tmem_wait_ld();
+                uint32_t pk[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    pk[i] = ng > 0 ? pack_bf16x2(__uint_as_float(r[2 * i]) * scale, __uint_as_float(r[2 * i + 1]) * scale)
+                                   : 0u;
+                uint4* dst = reinterpret_cast<uint4*>(out + 32 * q);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tb, kTmemCols);
+}
+
+// ============================================================================ dK, dV
+template <int D>
+__global__ void __launch_bounds__(192, 1)
+k_bwd_dkdv_sm100(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                 const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmdO,
+                 const int32_t* __restrict__ blk_start, const int32_t* __restrict__ gran_blk,
+                 const int32_t* __restrict__ n_blk, const uint32_t* __restrict__ selT,
+                 const float* __restrict__ lse, const float* __restrict__ delta, int64_t N, int64_t MB, int SW,
+                 float scale, __nv_bfloat16* __restrict__ dK, __nv_bfloat16* __restrict__ dV,
+                 uint32_t* __restrict__ dev_status) {
+    using L = BwdLayout<D>;
+    constexpr uint32_t cdK = 0, cdV = 128, cS = 256, cP = 320;   // + 128 * buffer for S^T / dP^T
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    Bars B = carve(sm + L::CTRL);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int tile = blockIdx.x, hh = blockIdx.y;
+    const int nb = *n_blk;
+    const int k0 = gran_blk[2 * tile], k1 = gran_blk[2 * tile + 1];
+    if (k0 < 0 || k0 >= nb || k1 < 0 || k1 >= nb) {
+        if (threadIdx.x == 0) atomicOr(dev_status, PRISM_DEV_BAD_INDEX);
+        return;
+    }
+    const uint32_t* r0 = selT + ((int64_t)hh * MB + k0) * SW;
+    const uint32_t* r1 = selT + ((int64_t)hh * MB + k1) * SW;
+    const int wn = (nb + 31) >> 5;
+    const int64_t row0 = (int64_t)hh * N;
+
+    if (threadIdx.x == 0) init_bars(B);
+    if (warp == 0) {
+        const int cnt = count_granules(r0, r1, blk_start, wn, lane);
+        if (lane == 0) *B.ng_slot = cnt;
+    } else if (warp == 1) {
+        tmem_alloc(B.tmem_slot, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tb = *B.tmem_slot;
+    const int ng = *B.ng_slot;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            GranuleWalk walk;
+            walk.init(r0, r1, blk_start, wn);
+            produce<D>(&tmK, &tmV, &tmQ, &tmdO, sm, B, row0, 128 * tile, walk, ng, dev_status);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            const uint32_t idPS = idesc_bf16_f32(128, 64, false, false);
+            const uint32_t idKV = idesc_bf16_f32(128, D, false, true);
+            const uint32_t aK = smem_u32(sm + L::A0), aV = smem_u32(sm + L::A1), aR = smem_u32(sm + L::RING);
+            bool ok = mbar_wait(B.stat, 0, B.abort_flag, dev_status);
+            tc_fence_after();
+            for (int g = 0; ok && g <= ng; ++g) {
+                if (g < ng) {
+                    const int s = g % kStages, b = g & 1;
+                    if (!mbar_wait(B.full + s, (g / kStages) & 1, B.abort_flag, dev_status)) break;
+                    tc_fence_after();
+                    const uint32_t aQ = aR + s * L::STAGE, adO = aQ + L::NR * kGran;
+#pragma unroll
+                    for (int k = 0; k < D / 16; ++k)
+                        mma_ss(tb + cS + 128 * b, sdesc_sw128(aK + kmaj_off(k, kTile), 16, 1024),
+                               sdesc_sw128(aQ + kmaj_off(k, kGran), 16, 1024), idPS, k > 0);
+#pragma unroll
+                    for (int k = 0; k < D / 16; ++k)
+                        mma_ss(tb + cP + 128 * b, sdesc_sw128(aV + kmaj_off(k, kTile), 16, 1024),
+                               sdesc_sw128(adO + kmaj_off(k, kGran), 16, 1024), idPS, k > 0);
+                    tc_commit(B.prod + b);
+                }
+                if (g > 0) {
+                    const int gp = g - 1, s = gp % kStages, b = gp & 1;
+                    if (!mbar_wait(B.elem + b, (gp >> 1) & 1, B.abort_flag, dev_status)) break;
+                    tc_fence_after();
+                    const uint32_t aQ = aR + s * L::STAGE, adO = aQ + L::NR * kGran;
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const uint32_t acc = (gp > 0 || k > 0) ? 1u : 0u;
+                        mma_ts(tb + cdV, tb + cS + 128 * b + 8 * k, sdesc_sw128(adO + k * 2048, kGran, 1024), idKV,
+                               acc);
+                        mma_ts(tb + cdK, tb + cP + 128 * b + 8 * k, sdesc_sw128(aQ + k * 2048, kGran, 1024), idKV,
+                               acc);
+                    }
+                    tc_commit(B.empty + s);
+                }
+            }
+            tc_commit(B.fin);
+            if (*B.abort_flag) {
+                volatile int no_abort = 0;
+                mbar_wait(B.fin, 0, &no_abort, dev_status);
+            }
+        }
+    } else {
+        const int sub = warp & 3, row = sub * 32 + lane, half = row >> 6;
+        const uint32_t tl = tb + ((uint32_t)(sub * 32) << 16);
+        const float sl2 = scale * kLog2e;
+        GranuleWalk walk;
+        if (lane == 0) walk.init(r0, r1, blk_start, wn);
+        bool ok = true;
+        for (int g = 0; g < ng; ++g) {
+            const int b = g & 1;
+            uint32_t mk = 0;
+            int qrow = 0;
+            if (lane == 0) walk.next(qrow, mk);
+            mk = __shfl_sync(0xffffffffu, mk, 0);
+            qrow = __shfl_sync(0xffffffffu, qrow, 0);
+            const bool valid = (mk >> half) & 1u;
+            const float4* lse4 = reinterpret_cast<const float4*>(lse + row0 + qrow);
+            const float4* del4 = reinterpret_cast<const float4*>(delta + row0 + qrow);
+            const bool got = mbar_wait(B.prod + b, (g >> 1) & 1, B.abort_flag, dev_status);
+            if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+            tc_fence_after();
+#pragma unroll
+            for (int hq = 0; hq < 2; ++hq) {
+                uint32_t s[32], p[32], op[16], od[16];
+                tmem_ld32(tl + cS + 128 * b + 32 * hq, s);
+                tmem_ld32(tl + cP + 128 * b + 32 * hq, p);
+                tmem_wait_ld();
+#pragma unroll
+                for (int i4 = 0; i4 < 8; ++i4) {
+                    const float4 l4 = __ldg(lse4 + 8 * hq + i4);
+                    const float4 d4 = __ldg(del4 + 8 * hq + i4);
+                    const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+                    const float dv[4] = {d4.x, d4.y, d4.z, d4.w};
+                    float pp[4], dd[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int i = 4 * i4 + u;
+                        pp[u] = 0.f;
+                        dd[u] = 0.f;
+                        if (valid) {
+                            pp[u] = exp2f(fmaf(__uint_as_float(s[i]), sl2, -lv[u] * kLog2e));
+                            dd[u] = pp[u] * (__uint_as_float(p[i]) - dv[u]);
+                        }
+                    }
+                    op[2 * i4] = pack_bf16x2(pp[0], pp[1]);
+                    op[2 * i4 + 1] = pack_bf16x2(pp[2], pp[3]);
+                    od[2 * i4] = pack_bf16x2(dd[0], dd[1]);
+                    od[2 * i4 + 1] = pack_bf16x2(dd[2], dd[3]);
+                }
+                tmem_st16(tl + cS + 128 * b + 16 * hq, op);     // P^T over the consumed S^T columns
+                tmem_st16(tl + cP + 128 * b + 16 * hq, od);     // dS^T over the consumed dP^T columns
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(B.elem + b);
+        }
+        const bool fin = ok && mbar_wait(B.fin, 0, B.abort_flag, dev_status);
+        if (__all_sync(0xffffffffu, fin)) {
+            tc_fence_after();
+            const int64_t grow = row0 + 128 * tile + row;
+#pragma unroll
+            for (int which = 0; which < 2; ++which) {
+                __nv_bfloat16* out = (which ? dV : dK) + grow * D;
+                const float mul = which ? 1.f : scale;
+                const uint32_t col = which ? cdV : cdK;
+#pragma unroll
+                for (int q = 0; q < D / 32; ++q) {
+                    uint32_t r[32];
+                    tmem_ld32(tl + col + 32 * q, r);
+                    tmem_wait_ld();
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        pk[i] = ng > 0 ? pack_bf16x2(__uint_as_float(r[2 * i]) * mul, __uint_as_float(r[2 * i + 1]) * mul)
+                                       : 0u;
+                    uint4* dst = reinterpret_cast<uint4*>(out + 32 * q);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tb, kTmemCols);
+}
+
+template <int D>
+prism_status_t launch_bwd(const Dims& d, const void* Qp, const void* Kp, const void* Vp, const void* dOp,
+                          const float* lse, const float* delta, const int32_t* blk_start, const int32_t* gran_blk,
+                          const int32_t* n_blk, const uint32_t* sel, const uint32_t* selT, float scale, void* dQp,
+                          void* dKp, void* dVp, uint32_t* dev_status, cudaStream_t s) {
+    const int64_t rows = (int64_t)d.heads * d.N;
+    CUtensorMap tQ, tdO, tK, tV, gQ, gdO, gK, gV;
+    if (!make_map_bf16(&tQ, Qp, rows, D, 128) || !make_map_bf16(&tdO, dOp, rows, D, 128) ||
+        !make_map_bf16(&tK, Kp, rows, D, 128) || !make_map_bf16(&tV, Vp, rows, D, 128) ||
+        !make_map_bf16(&gQ, Qp, rows, D, 64) || !make_map_bf16(&gdO, dOp, rows, D, 64) ||
+        !make_map_bf16(&gK, Kp, rows, D, 64) || !make_map_bf16(&gV, Vp, rows, D, 64))
+        return PRISM_ERR_CUDA;
+    const int smem = BwdLayout<D>::ALLOC;
+    auto kq = k_bwd_dq_sm100<D>;
+    auto kk = k_bwd_dkdv_sm100<D>;
+    if (cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess ||
+        cudaFuncSetAttribute(kk, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+        return PRISM_ERR_CUDA;
+    dim3 grid((unsigned)(d.N / 128), (unsigned)d.heads);
+    kq<<<grid, 192, smem, s>>>(tQ, tdO, gK, gV, blk_start, gran_blk, n_blk, sel, lse, delta, d.N, d.MB, (int)d.SW,
+                               scale, (__nv_bfloat16*)dQp, dev_status);
+    kk<<<grid, 192, smem, s>>>(tK, tV, gQ, gdO, blk_start, gran_blk, n_blk, selT, lse, delta, d.N, d.MB, (int)d.SW,
+                               scale, (__nv_bfloat16*)dKp, (__nv_bfloat16*)dVp, dev_status);
+    return launch_status(2);
+}
+
+}  // namespace
+
+prism_status_t attn_bwd_sm100(const Dims& d, const void* Qp, const void* Kp, const void* Vp, const void* Op,
+                              const float* o_f32, const void* dOp, const float* lse, const int32_t* blk_start,
+                              const int32_t* gran_blk, const int32_t* n_blk, const uint32_t* sel,
+                              const uint32_t* selT, float scale, void* dQp, void* dKp, void* dVp,
+                              uint32_t* dev_status, float* delta, cudaStream_t s) {
+    prism_status_t st = bwd_delta(d, Op, o_f32, dOp, delta, s);
+    if (st != PRISM_OK) return st;
+    if (d.d == 128)
+        return launch_bwd<128>(d, Qp, Kp, Vp, dOp, lse, delta, blk_start, gran_blk, n_blk, sel, selT, scale, dQp,
+                               dKp, dVp, dev_status, s);
+    return launch_bwd<64>(d, Qp, Kp, Vp, dOp, lse, delta, blk_start, gran_blk, n_blk, sel, selT, scale, dQp, dKp,
+                          dVp, dev_status, s);
+}
+
+}  // namespace prism

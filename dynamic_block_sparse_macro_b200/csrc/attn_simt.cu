@@ -418,6 +418,22 @@ prism_status_t attn_fwd_simt(const Dims& d, const void* Qp, const void* Kp, cons
 #undef PRISM_FWD_ARGS
 }
 
+// Delta = rowsum(dO * O) for every blocked row (shared by both backward families)
+prism_status_t bwd_delta(const Dims& d, const void* Op, const float* o_f32, const void* dOp, float* delta,
+                         cudaStream_t s) {
+    const int64_t rows = (int64_t)d.heads * d.N;
+    const unsigned grid = (unsigned)((rows * 32 + 255) / 256);
+    if (d.dtype == PRISM_F32) {
+        if (d.d == 64) k_bwd_delta<float, 64><<<grid, 256, 0, s>>>((const float*)Op, o_f32, (const float*)dOp, rows, delta);
+        else k_bwd_delta<float, 128><<<grid, 256, 0, s>>>((const float*)Op, o_f32, (const float*)dOp, rows, delta);
+    } else {
+        using B = __nv_bfloat16;
+        if (d.d == 64) k_bwd_delta<B, 64><<<grid, 256, 0, s>>>((const B*)Op, o_f32, (const B*)dOp, rows, delta);
+        else k_bwd_delta<B, 128><<<grid, 256, 0, s>>>((const B*)Op, o_f32, (const B*)dOp, rows, delta);
+    }
+    return launch_status(1);
+}
+
 prism_status_t attn_bwd_simt(const Dims& d, const void* Qp, const void* Kp, const void* Vp, const void* Op,
                              const float* o_f32, const void* dOp, const float* lse, const int32_t* blk_start,
                              const int32_t* gran_blk, const int32_t* n_blk, const uint32_t* sel,

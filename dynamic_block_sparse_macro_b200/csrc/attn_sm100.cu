@@ -54,40 +54,6 @@ struct FwdLayout {
     static constexpr int ALLOC = (BYTES + 1024) > 80 * 1024 ? (BYTES + 1024) : 80 * 1024;
 };
 
-// Walks the union of two selection rows as 64-row granules, in block order.
-struct GranuleWalk {
-    const uint32_t* r0;
-    const uint32_t* r1;
-    const int32_t* blk_start;
-    int wn, w, g, ng, base;
-    uint32_t bits, mask;
-
-    __device__ void init(const uint32_t* a, const uint32_t* b, const int32_t* bs, int words) {
-        r0 = a; r1 = b; blk_start = bs; wn = words; w = 0; g = 0; ng = 0; base = 0; mask = 0;
-        bits = wn > 0 ? (r0[0] | r1[0]) : 0u;
-    }
-    // next granule: its first key row and 2-bit mask (bit0: rows 0-63 use it, bit1: rows 64-127)
-    __device__ bool next(int& row, uint32_t& m) {
-        while (g >= ng) {
-            while (bits == 0) {
-                if (++w >= wn) return false;
-                bits = r0[w] | r1[w];
-            }
-            const int b = __ffs(bits) - 1;
-            bits &= bits - 1;
-            const int j = w * 32 + b;
-            base = blk_start[j];
-            ng = (blk_start[j + 1] - base) >> 6;
-            g = 0;
-            mask = ((r0[w] >> b) & 1u) | (((r1[w] >> b) & 1u) << 1);
-        }
-        row = base + 64 * g;
-        ++g;
-        m = mask;
-        return true;
-    }
-};
-
 template <int D>
 __global__ void __launch_bounds__(192, 2)
 k_attn_fwd_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -141,17 +107,7 @@ k_attn_fwd_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         fence_mbar_init();
     }
     if (warp == 0) {                                       // count granules of the union
-        int cnt = 0;
-        for (int w = lane; w < wn; w += 32) {
-            uint32_t b = r0[w] | r1[w];
-            while (b) {
-                const int j = w * 32 + __ffs(b) - 1;
-                b &= b - 1;
-                cnt += (blk_start[j + 1] - blk_start[j]) >> 6;
-            }
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+        const int cnt = count_granules(r0, r1, blk_start, wn, lane);
         if (lane == 0) *nch_slot = (cnt + 1) >> 1;
     } else if (warp == 1) {
         tmem_alloc(tmem_slot, kTmemCols);
@@ -363,42 +319,14 @@ k_attn_fwd_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
 }
 
 // ------------------------------------------------------------------ host side
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    if (!fn) {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(p);
-    }
-    return fn;
-}
-
-// 2-D map over a [rows][d] bf16 tensor, box = 64 columns x box_rows rows, 128-byte swizzle
-bool make_map(CUtensorMap* m, const void* base, int64_t rows, int d, int box_rows) {
-    EncodeTiledFn enc = encode_fn();
-    if (!enc) return false;
-    cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
-    cuuint64_t strides[1] = {(cuuint64_t)d * 2};
-    cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
-    cuuint32_t estr[2] = {1, 1};
-    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 template <int D>
 prism_status_t launch_fwd(const Dims& d, const void* Qp, const void* Kp, const void* Vp, const int32_t* blk_start,
                           const int32_t* gran_blk, const int32_t* n_blk, const uint32_t* sel, float scale, void* Op,
                           float* lse, float* o_f32, uint32_t* dev_status, cudaStream_t s) {
     CUtensorMap mQ, mK, mV;
     const int64_t rows = (int64_t)d.heads * d.N;
-    if (!make_map(&mQ, Qp, rows, D, 128) || !make_map(&mK, Kp, rows, D, 64) || !make_map(&mV, Vp, rows, D, 64))
+    if (!make_map_bf16(&mQ, Qp, rows, D, 128) || !make_map_bf16(&mK, Kp, rows, D, 64) ||
+        !make_map_bf16(&mV, Vp, rows, D, 64))
         return PRISM_ERR_CUDA;
     auto k = k_attn_fwd_sm100<D>;
     const int smem = FwdLayout<D>::ALLOC;

@@ -151,6 +151,15 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
           "r"(r[31])
         : "memory");
 }
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};"
+        ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]),
+          "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+          "r"(r[15])
+        : "memory");
+}
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
@@ -178,6 +187,88 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     uint32_t r;
     asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
     return r;
+}
+
+// Walks the union of two bitmask rows (selection rows of two query blocks, or
+// key-major rows of two key blocks) as 64-row granules, in block order.  The
+// 2-bit mask of a granule says which of the two rows contains its block.
+struct GranuleWalk {
+    const uint32_t* r0;
+    const uint32_t* r1;
+    const int32_t* blk_start;
+    int wn, w, g, ng, base;
+    uint32_t bits, mask;
+
+    __device__ void init(const uint32_t* a, const uint32_t* b, const int32_t* bs, int words) {
+        r0 = a; r1 = b; blk_start = bs; wn = words; w = 0; g = 0; ng = 0; base = 0; mask = 0;
+        bits = wn > 0 ? (r0[0] | r1[0]) : 0u;
+    }
+    __device__ bool next(int& row, uint32_t& m) {
+        while (g >= ng) {
+            while (bits == 0) {
+                if (++w >= wn) return false;
+                bits = r0[w] | r1[w];
+            }
+            const int b = __ffs(bits) - 1;
+            bits &= bits - 1;
+            const int j = w * 32 + b;
+            base = blk_start[j];
+            ng = (blk_start[j + 1] - base) >> 6;
+            g = 0;
+            mask = ((r0[w] >> b) & 1u) | (((r1[w] >> b) & 1u) << 1);
+        }
+        row = base + 64 * g;
+        ++g;
+        m = mask;
+        return true;
+    }
+};
+
+// number of 64-row granules in the union of two bitmask rows (one warp)
+__device__ __forceinline__ int count_granules(const uint32_t* r0, const uint32_t* r1, const int32_t* blk_start,
+                                              int wn, int lane) {
+    int cnt = 0;
+    for (int w = lane; w < wn; w += 32) {
+        uint32_t b = r0[w] | r1[w];
+        while (b) {
+            const int j = w * 32 + __ffs(b) - 1;
+            b &= b - 1;
+            cnt += (blk_start[j + 1] - blk_start[j]) >> 6;
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+    return cnt;
+}
+
+// ------------------------------------------------------------------ host: TMA maps
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+inline EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+// 2-D map over a [rows][d] bf16 tensor: box = 64 columns x box_rows rows, 128-byte swizzle
+inline bool make_map_bf16(CUtensorMap* m, const void* base, int64_t rows, int d, int box_rows) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)d * 2};
+    cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 }  // namespace sm100
