@@ -127,9 +127,20 @@ def selected_flops(mod) -> dict:
     f_fwd = 4.0 * mod.d * float((keys_per_row * sz).sum().item())
     dense = 4.0 * mod.d * mod.heads * float(sz.sum().item()) ** 2
     vol = {int(v): int((sz == v).sum().item()) for v in (64, 128, 256)}
+    # work per 128-row tile of the attention kernels: union of its granules' selections
+    g = mod.gsel.to(torch.int64) & 0xFFFFFFFF
+    pop = lambda w: sum(((w >> s) & 1) for s in range(32))
+    tile_gran = pop(g[:, 0::2, :] | g[:, 1::2, :]).sum(-1).double()            # [h, N/128]
+    gT = mod.gselT.to(torch.int64) & 0xFFFFFFFF
+    key_gran = pop(gT[:, 0::2, :] | gT[:, 1::2, :]).sum(-1).double()
+    q = torch.tensor([0.5, 0.99, 1.0], dtype=torch.float64, device=tile_gran.device)
+    tq = torch.quantile(tile_gran.flatten(), q).tolist()
+    kq = torch.quantile(key_gran.flatten(), q).tolist()
     return {"F_fwd": f_fwd, "F_dense_fwd": dense, "n_blk": nb, "density": f_fwd / dense,
             "mean_sel_blocks": float(sel.sum(-1).mean().item()),
-            "mean_sel_tokens": float(keys_per_row.mean().item()), "block_volumes": vol}
+            "max_sel_blocks": float(sel.sum(-1).max().item()),
+            "mean_sel_tokens": float(keys_per_row.mean().item()), "block_volumes": vol,
+            "tile_key_granules_p50_p99_max": tq, "tile_query_granules_p50_p99_max": kq}
 
 
 class StepTimer:
@@ -158,8 +169,8 @@ def run_step(mod, x, out, grads, timer=None):
     _abi.prism_permute(mod.prob, x["dO"], mod.perm, mod.dOp)
     rec(4)
     _abi.prism_sparse_attn_bwd(mod.prob, mod.Qp, mod.Kp, mod.Vp, mod.Op, mod.Of32, mod.dOp, mod.lse,
-                               mod.blk_start, mod.gran_blk, mod.n_blk, mod.sel, mod.selT, mod.scale,
-                               mod.dQp, mod.dKp, mod.dVp, mod.dev_status, mod.ws_bwd)
+                               mod.gsel, mod.gselT, mod.scale, mod.dQp, mod.dKp, mod.dVp, mod.dev_status,
+                               mod.ws_bwd)
     rec(5)
     for src, dst in zip((mod.dQp, mod.dKp, mod.dVp), grads):
         _abi.prism_unpermute(mod.prob, src, mod.perm, dst)
@@ -380,13 +391,15 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="prism", choices=["prism", "reference"])
     ap.add_argument("--config", default="2k")
+    ap.add_argument("--heads", type=int, default=None,
+                    help="override the config's head count (smaller profiling captures)")
     ap.add_argument("--dense", action="store_true", help="select every block (all-blocks dense run)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--out", default=None, help="also append the JSON line to this file")
     args = ap.parse_args()
-    cfg = get_config(args.config)
+    cfg = get_config(args.config, **({"heads": args.heads} if args.heads else {}))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))

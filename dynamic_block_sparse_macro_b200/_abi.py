@@ -61,10 +61,9 @@ _SIGS = {
     "prism_permute": [_PROB, _P, _P, _P, _P],
     "prism_unpermute": [_PROB, _P, _P, _P, _P],
     "prism_block_pool_score": [_PROB, _P, _P, _P, _P, _F, _P, _P, _P, _P],
-    "prism_block_select": [_PROB, _P, _P, _I, _F, _P, _P, _P, _P, _P, _P],
-    "prism_sparse_attn_fwd": [_PROB, _P, _P, _P, _P, _P, _P, _P, _F, _P, _P, _P, _P, _P, _SZ, _P],
-    "prism_sparse_attn_bwd": [_PROB, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _F, _P, _P,
-                              _P, _P, _P, _SZ, _P],
+    "prism_block_select": [_PROB, _P, _P, _P, _P, _I, _F, _P, _P, _P, _P, _P, _P, _P],
+    "prism_sparse_attn_fwd": [_PROB, _P, _P, _P, _P, _F, _P, _P, _P, _P, _P, _SZ, _P],
+    "prism_sparse_attn_bwd": [_PROB, _P, _P, _P, _P, _P, _P, _P, _P, _P, _F, _P, _P, _P, _P, _P, _SZ, _P],
     "prism_read_status": [_P, ctypes.POINTER(ctypes.c_uint32), _P],
 }
 
@@ -162,29 +161,27 @@ def prism_block_pool_score(prob, Qp, Kp, blk_start, n_blk, scale, Qbar, Kbar, P,
         _ptr(Kbar), _ptr(P), _stream(stream)))
 
 
-def prism_block_select(prob, P, n_blk, top_k, top_p, sel, sel_count, selT, margin, dev_status,
-                       stream=None):
+def prism_block_select(prob, P, blk_start, gran_blk, n_blk, top_k, top_p, sel, sel_count, gsel, gselT,
+                       margin, dev_status, stream=None):
     _check("prism_block_select", lib().prism_block_select(
-        ctypes.byref(prob), _ptr(P), _ptr(n_blk), int(top_k), float(top_p), _ptr(sel),
-        _ptr(sel_count), _ptr(selT), _ptr(margin), _ptr(dev_status), _stream(stream)))
+        ctypes.byref(prob), _ptr(P), _ptr(blk_start), _ptr(gran_blk), _ptr(n_blk), int(top_k), float(top_p),
+        _ptr(sel), _ptr(sel_count), _ptr(gsel), _ptr(gselT), _ptr(margin), _ptr(dev_status), _stream(stream)))
 
 
-def prism_sparse_attn_fwd(prob, Qp, Kp, Vp, blk_start, gran_blk, n_blk, sel, scale, Op, lse,
-                          o_f32, dev_status, ws=None, stream=None):
+def prism_sparse_attn_fwd(prob, Qp, Kp, Vp, gsel, scale, Op, lse, o_f32, dev_status, ws=None,
+                          stream=None):
     nbytes = 0 if ws is None else ws.numel() * ws.element_size()
     _check("prism_sparse_attn_fwd", lib().prism_sparse_attn_fwd(
-        ctypes.byref(prob), _ptr(Qp), _ptr(Kp), _ptr(Vp), _ptr(blk_start), _ptr(gran_blk),
-        _ptr(n_blk), _ptr(sel), scale, _ptr(Op), _ptr(lse), _ptr(o_f32), _ptr(dev_status), _ptr(ws),
-        nbytes, _stream(stream)))
+        ctypes.byref(prob), _ptr(Qp), _ptr(Kp), _ptr(Vp), _ptr(gsel), scale, _ptr(Op), _ptr(lse),
+        _ptr(o_f32), _ptr(dev_status), _ptr(ws), nbytes, _stream(stream)))
 
 
-def prism_sparse_attn_bwd(prob, Qp, Kp, Vp, Op, o_f32, dOp, lse, blk_start, gran_blk, n_blk, sel,
-                          selT, scale, dQp, dKp, dVp, dev_status, ws, stream=None):
+def prism_sparse_attn_bwd(prob, Qp, Kp, Vp, Op, o_f32, dOp, lse, gsel, gselT, scale, dQp, dKp, dVp,
+                          dev_status, ws, stream=None):
     _check("prism_sparse_attn_bwd", lib().prism_sparse_attn_bwd(
         ctypes.byref(prob), _ptr(Qp), _ptr(Kp), _ptr(Vp), _ptr(Op), _ptr(o_f32), _ptr(dOp), _ptr(lse),
-        _ptr(blk_start), _ptr(gran_blk), _ptr(n_blk), _ptr(sel), _ptr(selT), scale, _ptr(dQp),
-        _ptr(dKp), _ptr(dVp), _ptr(dev_status), _ptr(ws), ws.numel() * ws.element_size(),
-        _stream(stream)))
+        _ptr(gsel), _ptr(gselT), scale, _ptr(dQp), _ptr(dKp), _ptr(dVp), _ptr(dev_status), _ptr(ws),
+        ws.numel() * ws.element_size(), _stream(stream)))
 
 
 def prism_read_status(dev_status, stream=None) -> int:

@@ -6,30 +6,29 @@
 
 namespace prism {
 size_t zone_indicator_ws_bytes(const Dims& d);
-prism_status_t attn_fwd_sm100(const Dims& d, const void* Qp, const void* Kp, const void* Vp,
-                              const int32_t* blk_start, const int32_t* gran_blk, const int32_t* n_blk,
-                              const uint32_t* sel, float scale, void* Op, float* lse, float* o_f32,
-                              uint32_t* dev_status, cudaStream_t s);
+prism_status_t attn_fwd_sm100(const Dims& d, const void* Qp, const void* Kp, const void* Vp, const uint32_t* gsel,
+                              float scale, void* Op, float* lse, float* o_f32, uint32_t* dev_status, void* ws,
+                              cudaStream_t s);
+size_t attn_fwd_sm100_ws_bytes(const Dims& d);
 prism_status_t attn_bwd_sm100(const Dims& d, const void* Qp, const void* Kp, const void* Vp, const void* Op,
-                              const float* o_f32, const void* dOp, const float* lse, const int32_t* blk_start,
-                              const int32_t* gran_blk, const int32_t* n_blk, const uint32_t* sel,
-                              const uint32_t* selT, float scale, void* dQp, void* dKp, void* dVp,
-                              uint32_t* dev_status, float* delta, cudaStream_t s);
-prism_status_t attn_fwd_simt(const Dims& d, const void* Qp, const void* Kp, const void* Vp,
-                             const int32_t* blk_start, const int32_t* gran_blk, const int32_t* n_blk,
-                             const uint32_t* sel, float scale, void* Op, float* lse, float* o_f32,
-                             cudaStream_t s);
+                              const float* o_f32, const void* dOp, const float* lse, const uint32_t* gsel,
+                              const uint32_t* gselT, float scale, void* dQp, void* dKp, void* dVp,
+                              uint32_t* dev_status, void* ws, cudaStream_t s);
+size_t attn_bwd_sm100_ws_bytes(const Dims& d);
+prism_status_t attn_fwd_simt(const Dims& d, const void* Qp, const void* Kp, const void* Vp, const uint32_t* gsel,
+                             float scale, void* Op, float* lse, float* o_f32, cudaStream_t s);
 prism_status_t attn_bwd_simt(const Dims& d, const void* Qp, const void* Kp, const void* Vp, const void* Op,
-                             const float* o_f32, const void* dOp, const float* lse, const int32_t* blk_start,
-                             const int32_t* gran_blk, const int32_t* n_blk, const uint32_t* sel,
-                             const uint32_t* selT, float scale, void* dQp, void* dKp, void* dVp,
-                             float* delta, cudaStream_t s);
+                             const float* o_f32, const void* dOp, const float* lse, const uint32_t* gsel,
+                             const uint32_t* gselT, float scale, void* dQp, void* dKp, void* dVp, float* delta,
+                             cudaStream_t s);
 
 static std::atomic<unsigned long long> g_launches{0};
 void note_launches(int n) { g_launches.fetch_add((unsigned long long)n, std::memory_order_relaxed); }
 
-size_t attn_fwd_ws_bytes(const Dims&) { return 0; }
-size_t attn_bwd_ws_bytes(const Dims& d) { return (size_t)d.heads * d.N * sizeof(float); }
+size_t attn_fwd_ws_bytes(const Dims& d) { return d.dtype == PRISM_BF16 ? attn_fwd_sm100_ws_bytes(d) : 0; }
+size_t attn_bwd_ws_bytes(const Dims& d) {
+    return d.dtype == PRISM_BF16 ? attn_bwd_sm100_ws_bytes(d) : (size_t)d.heads * d.N * sizeof(float);
+}
 }  // namespace prism
 
 using namespace prism;
@@ -51,47 +50,41 @@ extern "C" prism_status_t prism_query_sizes(const prism_problem_t* prob, prism_s
 }
 
 extern "C" prism_status_t prism_sparse_attn_fwd(const prism_problem_t* prob, const void* Qp, const void* Kp,
-                                                const void* Vp, const int32_t* blk_start,
-                                                const int32_t* gran_blk, const int32_t* n_blk,
-                                                const uint32_t* sel, float scale, void* Op, float* lse,
-                                                float* o_f32, uint32_t* dev_status, void* ws, size_t ws_bytes,
-                                                cudaStream_t stream) {
+                                                const void* Vp, const uint32_t* gsel, float scale, void* Op,
+                                                float* lse, float* o_f32, uint32_t* dev_status, void* ws,
+                                                size_t ws_bytes, cudaStream_t stream) {
     Dims d;
     prism_status_t st = make_dims(prob, &d);
     if (st != PRISM_OK) return st;
-    if (!ok_ptr(Qp) || !ok_ptr(Kp) || !ok_ptr(Vp) || !ok_ptr(blk_start) || !ok_ptr(gran_blk) ||
-        !ok_ptr(n_blk) || !ok_ptr(sel) || !ok_ptr(Op) || !ok_ptr(lse) || !ok_opt(o_f32) ||
-        !ok_ptr(dev_status) || !ok_opt(ws))
+    if (!ok_ptr(Qp) || !ok_ptr(Kp) || !ok_ptr(Vp) || !ok_ptr(gsel) || !ok_ptr(Op) || !ok_ptr(lse) ||
+        !ok_opt(o_f32) || !ok_ptr(dev_status) || !ok_opt(ws))
         return PRISM_ERR_INVALID_ARG;
     if (!(scale > 0.f) || !isfinite(scale)) return PRISM_ERR_INVALID_ARG;
     if (ws_bytes < attn_fwd_ws_bytes(d)) return PRISM_ERR_WORKSPACE;
     if (d.dtype == PRISM_BF16)
-        return attn_fwd_sm100(d, Qp, Kp, Vp, blk_start, gran_blk, n_blk, sel, scale, Op, lse, o_f32, dev_status,
-                              stream);
-    return attn_fwd_simt(d, Qp, Kp, Vp, blk_start, gran_blk, n_blk, sel, scale, Op, lse, o_f32, stream);
+        return attn_fwd_sm100(d, Qp, Kp, Vp, gsel, scale, Op, lse, o_f32, dev_status, ws, stream);
+    return attn_fwd_simt(d, Qp, Kp, Vp, gsel, scale, Op, lse, o_f32, stream);
 }
 
 extern "C" prism_status_t prism_sparse_attn_bwd(const prism_problem_t* prob, const void* Qp, const void* Kp,
                                                 const void* Vp, const void* Op, const float* o_f32,
-                                                const void* dOp, const float* lse, const int32_t* blk_start,
-                                                const int32_t* gran_blk, const int32_t* n_blk,
-                                                const uint32_t* sel, const uint32_t* selT, float scale,
-                                                void* dQp, void* dKp, void* dVp, uint32_t* dev_status,
-                                                void* ws, size_t ws_bytes, cudaStream_t stream) {
+                                                const void* dOp, const float* lse, const uint32_t* gsel,
+                                                const uint32_t* gselT, float scale, void* dQp, void* dKp,
+                                                void* dVp, uint32_t* dev_status, void* ws, size_t ws_bytes,
+                                                cudaStream_t stream) {
     Dims d;
     prism_status_t st = make_dims(prob, &d);
     if (st != PRISM_OK) return st;
-    if (!ok_ptr(Qp) || !ok_ptr(Kp) || !ok_ptr(Vp) || !ok_ptr(Op) || !ok_opt(o_f32) || !ok_ptr(dOp) || !ok_ptr(lse) ||
-        !ok_ptr(blk_start) || !ok_ptr(gran_blk) || !ok_ptr(n_blk) || !ok_ptr(sel) || !ok_ptr(selT) ||
-        !ok_ptr(dQp) || !ok_ptr(dKp) || !ok_ptr(dVp) || !ok_ptr(dev_status) || !ok_ptr(ws))
+    if (!ok_ptr(Qp) || !ok_ptr(Kp) || !ok_ptr(Vp) || !ok_ptr(Op) || !ok_opt(o_f32) || !ok_ptr(dOp) ||
+        !ok_ptr(lse) || !ok_ptr(gsel) || !ok_ptr(gselT) || !ok_ptr(dQp) || !ok_ptr(dKp) || !ok_ptr(dVp) ||
+        !ok_ptr(dev_status) || !ok_ptr(ws))
         return PRISM_ERR_INVALID_ARG;
     if (!(scale > 0.f) || !isfinite(scale)) return PRISM_ERR_INVALID_ARG;
     if (ws_bytes < attn_bwd_ws_bytes(d)) return PRISM_ERR_WORKSPACE;
     if (d.dtype == PRISM_BF16)
-        return attn_bwd_sm100(d, Qp, Kp, Vp, Op, o_f32, dOp, lse, blk_start, gran_blk, n_blk, sel, selT, scale, dQp,
-                              dKp, dVp, dev_status, (float*)ws, stream);
-    return attn_bwd_simt(d, Qp, Kp, Vp, Op, o_f32, dOp, lse, blk_start, gran_blk, n_blk, sel, selT, scale, dQp, dKp,
-                         dVp, (float*)ws, stream);
+        return attn_bwd_sm100(d, Qp, Kp, Vp, Op, o_f32, dOp, lse, gsel, gselT, scale, dQp, dKp, dVp, dev_status, ws,
+                              stream);
+    return attn_bwd_simt(d, Qp, Kp, Vp, Op, o_f32, dOp, lse, gsel, gselT, scale, dQp, dKp, dVp, (float*)ws, stream);
 }
 
 extern "C" prism_status_t prism_read_status(const uint32_t* dev_status, uint32_t* host_out, cudaStream_t stream) {

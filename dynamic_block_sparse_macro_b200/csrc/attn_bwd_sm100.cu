@@ -9,12 +9,12 @@
 //
 // Two kernels, no atomics (deterministic):
 //   k_bwd_dq_sm100    query-stationary: per (128-row query tile, head) walk the
-//                     key granules of S_b0 U S_b1; per 64-key granule
+//                     key granules of the union of its two granule-level rows; per 64-key granule
 //                     S = Q K^T and dP = dO V^T (M=128, N=64) into TMEM, dS as
 //                     bf16 back into TMEM, dQ += dS K (K MN-major in smem).
 //   k_bwd_dkdv_sm100  key-stationary: per (128-key tile, head) walk the query
-//                     granules of the query blocks that selected the tile's key
-//                     blocks (the key-major selection); per 64-query granule
+//                     granules whose blocks selected the tile's key blocks (the
+//                     transposed granule-level selection); per 64-query granule
 //                     S^T = K Q^T and dP^T = V dO^T, then P^T and dS^T as bf16
 //                     in TMEM, dV += P^T dO and dK += dS^T Q.
 // Both double-buffer the granule products in TMEM so that the tensor core
@@ -22,6 +22,7 @@
 // and stream granules through a 3-stage TMA ring.  Roles: warp 0 TMA, warp 1
 // TMEM allocation + MMA issue (one thread), warps 2-5 one tile row per thread.
 // Every wait is bounded; a timeout sets PRISM_DEV_TIMEOUT.
+#include "attn_plan.cuh"
 #include "common.cuh"
 #include "sm100.cuh"
 
@@ -48,8 +49,8 @@ struct BwdLayout {
     static constexpr int RING = 2 * NR * kTile;        // streamed granules
     static constexpr int STAGE = 2 * NR * kGran;       // two operands per stage
     static constexpr int CTRL = RING + kStages * STAGE;
-    static constexpr int BYTES = CTRL + 256;
-    static constexpr int ALLOC = BYTES + 1024;
+    static constexpr int ROWS = CTRL + 256;            // two selection rows of SW words follow
+    static int alloc(int SW) { return ROWS + 8 * SW + 1024; }
 };
 
 struct Bars {
@@ -140,33 +141,29 @@ template <int D>
 __global__ void __launch_bounds__(192, 1)
 k_bwd_dq_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmdO,
                const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-               const int32_t* __restrict__ blk_start, const int32_t* __restrict__ gran_blk,
-               const int32_t* __restrict__ n_blk, const uint32_t* __restrict__ sel,
-               const float* __restrict__ lse, const float* __restrict__ delta, int64_t N, int64_t MB, int SW,
-               float scale, __nv_bfloat16* __restrict__ dQ, uint32_t* __restrict__ dev_status) {
+               const uint32_t* __restrict__ gsel, const PlanHeader* __restrict__ hdr,
+               const int4* __restrict__ items, float* __restrict__ part, const float* __restrict__ lse,
+               const float* __restrict__ delta, int64_t N, int64_t MB, int SW, float scale,
+               __nv_bfloat16* __restrict__ dQ, uint32_t* __restrict__ dev_status) {
     using L = BwdLayout<D>;
     constexpr uint32_t cdQ = 0, cS = 128, cP = 192;   // + 128 * buffer for S / dP
+    if ((int)blockIdx.x >= hdr->n_items) return;      // uniform: beyond the item list
+    const int4 item = items[blockIdx.x];
+    const int tiles_per_head = (int)(N / 128);
+    const int hh = item.x / tiles_per_head, tile = item.x % tiles_per_head;
+    const int g_begin = item.y, ng = item.z - item.y, slot = item.w;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     Bars B = carve(sm + L::CTRL);
+    uint32_t* u0 = reinterpret_cast<uint32_t*>(sm + L::ROWS);
+    uint32_t* u1 = u0 + SW;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int tile = blockIdx.x, hh = blockIdx.y;
-    const int nb = *n_blk;
-    const int b0 = gran_blk[2 * tile], b1 = gran_blk[2 * tile + 1];
-    if (b0 < 0 || b0 >= nb || b1 < 0 || b1 >= nb) {
-        if (threadIdx.x == 0) atomicOr(dev_status, PRISM_DEV_BAD_INDEX);
-        return;
-    }
-    const uint32_t* r0 = sel + ((int64_t)hh * MB + b0) * SW;
-    const uint32_t* r1 = sel + ((int64_t)hh * MB + b1) * SW;
-    const int wn = (nb + 31) >> 5;
+    const int wn = SW;
     const int64_t row0 = (int64_t)hh * N;
 
+    load_rows(u0, u1, gsel + ((int64_t)hh * MB + 2 * tile) * SW, gsel + ((int64_t)hh * MB + 2 * tile + 1) * SW, wn);
     if (threadIdx.x == 0) init_bars(B);
-    if (warp == 0) {
-        const int cnt = count_granules(r0, r1, blk_start, wn, lane);
-        if (lane == 0) *B.ng_slot = cnt;
-    } else if (warp == 1) {
+    if (warp == 1) {
         tmem_alloc(B.tmem_slot, kTmemCols);
         tmem_relinquish();
     }
@@ -174,12 +171,12 @@ k_bwd_dq_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     __syncthreads();
     tc_fence_after();
     const uint32_t tb = *B.tmem_slot;
-    const int ng = *B.ng_slot;
 
     if (warp == 0) {
         if (lane == 0) {
             GranuleWalk walk;
-            walk.init(r0, r1, blk_start, wn);
+            walk.init(u0, u1, wn);
+            walk.skip(g_begin);
             produce<D>(&tmQ, &tmdO, &tmK, &tmV, sm, B, row0, 128 * tile, walk, ng, dev_status);
         }
     } else if (warp == 1) {
@@ -229,8 +226,12 @@ k_bwd_dq_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         const int64_t grow = row0 + 128 * tile + row;
         const float lse2 = lse[grow] * kLog2e, dl = delta[grow];
         const float sl2 = scale * kLog2e;
+        const uint64_t sl2x2 = f2pack(sl2, sl2), nlse2 = f2pack(-lse2, -lse2), ndl2 = f2pack(-dl, -dl);
         GranuleWalk walk;
-        if (lane == 0) walk.init(r0, r1, blk_start, wn);
+        if (lane == 0) {
+            walk.init(u0, u1, wn);
+            walk.skip(g_begin);
+        }
         bool ok = true;
         for (int g = 0; g < ng; ++g) {
             const int b = g & 1;
@@ -240,26 +241,32 @@ k_bwd_dq_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                 walk.next(rr, mk);
             }
             mk = __shfl_sync(0xffffffffu, mk, 0);
-            const bool valid = (mk >> half) & 1u;
+            const bool valid = (mk >> half) & 1u;              // warp-uniform
             const bool got = mbar_wait(B.prod + b, (g >> 1) & 1, B.abort_flag, dev_status);
             if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
             tc_fence_after();
 #pragma unroll
             for (int hq = 0; hq < 2; ++hq) {
-                uint32_t s[32], p[32], o[16];
-                tmem_ld32(tl + cS + 128 * b + 32 * hq, s);
-                tmem_ld32(tl + cP + 128 * b + 32 * hq, p);
-                tmem_wait_ld();
+                uint32_t o[16];
+                if (valid) {
+                    uint32_t s[32], p[32];
+                    tmem_ld32(tl + cS + 128 * b + 32 * hq, s);
+                    tmem_ld32(tl + cP + 128 * b + 32 * hq, p);
+                    tmem_wait_ld();
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    float d0 = 0.f, d1 = 0.f;
-                    if (valid) {
-                        const float p0 = exp2f(fmaf(__uint_as_float(s[2 * i]), sl2, -lse2));
-                        const float p1 = exp2f(fmaf(__uint_as_float(s[2 * i + 1]), sl2, -lse2));
-                        d0 = p0 * (__uint_as_float(p[2 * i]) - dl);
-                        d1 = p1 * (__uint_as_float(p[2 * i + 1]) - dl);
+                    for (int i = 0; i < 16; ++i) {
+                        float x0, x1;
+                        f2unpack(ffma2(f2pack(__uint_as_float(s[2 * i]), __uint_as_float(s[2 * i + 1])), sl2x2, nlse2),
+                                 x0, x1);
+                        const uint64_t pp = f2pack(ex2(x0), ex2(x1));
+                        const uint64_t dp = fadd2(f2pack(__uint_as_float(p[2 * i]), __uint_as_float(p[2 * i + 1])), ndl2);
+                        float d0, d1;
+                        f2unpack(fmul2(pp, dp), d0, d1);
+                        o[i] = pack_bf16x2(d0, d1);
                     }
-                    o[i] = pack_bf16x2(d0, d1);
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) o[i] = 0u;
                 }
                 tmem_st16(tl + cS + 128 * b + 16 * hq, o);     // dS (bf16) over the consumed S columns
             }
@@ -270,20 +277,31 @@ k_bwd_dq_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         const bool fin = ok && mbar_wait(B.fin, 0, B.abort_flag, dev_status);
         if (__all_sync(0xffffffffu, fin)) {
             tc_fence_after();
-            __nv_bfloat16* out = dQ + grow * D;
 #pragma unroll
             for (int q = 0; q < D / 32; ++q) {
                 uint32_t r[32];
                 tmem_ld32(tl + cdQ + 32 * q, r);
                 tmem_wait_ld();
-                uint32_t pk[16];
+                if (ng == 0) {                              // nothing selected: TMEM never written
 #pragma unroll
-                for (int i = 0; i < 16; ++i)
-                    pk[i] = ng > 0 ? pack_bf16x2(__uint_as_float(r[2 * i]) * scale, __uint_as_float(r[2 * i + 1]) * scale)
-                                   : 0u;
-                uint4* dst = reinterpret_cast<uint4*>(out + 32 * q);
+                    for (int i = 0; i < 32; ++i) r[i] = 0u;
+                }
+                if (slot < 0) {
+                    uint32_t pk[16];
 #pragma unroll
-                for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+                    for (int i = 0; i < 16; ++i)
+                        pk[i] = pack_bf16x2(__uint_as_float(r[2 * i]) * scale, __uint_as_float(r[2 * i + 1]) * scale);
+                    uint4* dst = reinterpret_cast<uint4*>(dQ + grow * D + 32 * q);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+                } else {                                    // partial of a split tile (unscaled)
+                    float4* df = reinterpret_cast<float4*>(part + ((int64_t)slot * 128 + row) * D + 32 * q);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i)
+                        df[i] = make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
+                                            __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]));
+                }
             }
         }
     }
@@ -298,34 +316,30 @@ template <int D>
 __global__ void __launch_bounds__(192, 1)
 k_bwd_dkdv_sm100(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                  const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmdO,
-                 const int32_t* __restrict__ blk_start, const int32_t* __restrict__ gran_blk,
-                 const int32_t* __restrict__ n_blk, const uint32_t* __restrict__ selT,
-                 const float* __restrict__ lse, const float* __restrict__ delta, int64_t N, int64_t MB, int SW,
-                 float scale, __nv_bfloat16* __restrict__ dK, __nv_bfloat16* __restrict__ dV,
+                 const uint32_t* __restrict__ gselT, const PlanHeader* __restrict__ hdr,
+                 const int4* __restrict__ items, float* __restrict__ part, const float* __restrict__ lse,
+                 const float* __restrict__ delta, int64_t N, int64_t MB, int SW, float scale,
+                 __nv_bfloat16* __restrict__ dK, __nv_bfloat16* __restrict__ dV,
                  uint32_t* __restrict__ dev_status) {
     using L = BwdLayout<D>;
     constexpr uint32_t cdK = 0, cdV = 128, cS = 256, cP = 320;   // + 128 * buffer for S^T / dP^T
+    if ((int)blockIdx.x >= hdr->n_items) return;      // uniform: beyond the item list
+    const int4 item = items[blockIdx.x];
+    const int tiles_per_head = (int)(N / 128);
+    const int hh = item.x / tiles_per_head, tile = item.x % tiles_per_head;
+    const int g_begin = item.y, ng = item.z - item.y, slot = item.w;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     Bars B = carve(sm + L::CTRL);
+    uint32_t* u0 = reinterpret_cast<uint32_t*>(sm + L::ROWS);
+    uint32_t* u1 = u0 + SW;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int tile = blockIdx.x, hh = blockIdx.y;
-    const int nb = *n_blk;
-    const int k0 = gran_blk[2 * tile], k1 = gran_blk[2 * tile + 1];
-    if (k0 < 0 || k0 >= nb || k1 < 0 || k1 >= nb) {
-        if (threadIdx.x == 0) atomicOr(dev_status, PRISM_DEV_BAD_INDEX);
-        return;
-    }
-    const uint32_t* r0 = selT + ((int64_t)hh * MB + k0) * SW;
-    const uint32_t* r1 = selT + ((int64_t)hh * MB + k1) * SW;
-    const int wn = (nb + 31) >> 5;
+    const int wn = SW;
     const int64_t row0 = (int64_t)hh * N;
 
+    load_rows(u0, u1, gselT + ((int64_t)hh * MB + 2 * tile) * SW, gselT + ((int64_t)hh * MB + 2 * tile + 1) * SW, wn);
     if (threadIdx.x == 0) init_bars(B);
-    if (warp == 0) {
-        const int cnt = count_granules(r0, r1, blk_start, wn, lane);
-        if (lane == 0) *B.ng_slot = cnt;
-    } else if (warp == 1) {
+    if (warp == 1) {
         tmem_alloc(B.tmem_slot, kTmemCols);
         tmem_relinquish();
     }
@@ -333,12 +347,12 @@ k_bwd_dkdv_sm100(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
     __syncthreads();
     tc_fence_after();
     const uint32_t tb = *B.tmem_slot;
-    const int ng = *B.ng_slot;
 
     if (warp == 0) {
         if (lane == 0) {
             GranuleWalk walk;
-            walk.init(r0, r1, blk_start, wn);
+            walk.init(u0, u1, wn);
+            walk.skip(g_begin);
             produce<D>(&tmK, &tmV, &tmQ, &tmdO, sm, B, row0, 128 * tile, walk, ng, dev_status);
         }
     } else if (warp == 1) {
@@ -390,8 +404,12 @@ k_bwd_dkdv_sm100(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
         const int sub = warp & 3, row = sub * 32 + lane, half = row >> 6;
         const uint32_t tl = tb + ((uint32_t)(sub * 32) << 16);
         const float sl2 = scale * kLog2e;
+        const uint64_t sl2x2 = f2pack(sl2, sl2), nlog2e = f2pack(-kLog2e, -kLog2e), neg1 = f2pack(-1.f, -1.f);
         GranuleWalk walk;
-        if (lane == 0) walk.init(r0, r1, blk_start, wn);
+        if (lane == 0) {
+            walk.init(u0, u1, wn);
+            walk.skip(g_begin);
+        }
         bool ok = true;
         for (int g = 0; g < ng; ++g) {
             const int b = g & 1;
@@ -400,7 +418,7 @@ k_bwd_dkdv_sm100(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
             if (lane == 0) walk.next(qrow, mk);
             mk = __shfl_sync(0xffffffffu, mk, 0);
             qrow = __shfl_sync(0xffffffffu, qrow, 0);
-            const bool valid = (mk >> half) & 1u;
+            const bool valid = (mk >> half) & 1u;              // warp-uniform
             const float4* lse4 = reinterpret_cast<const float4*>(lse + row0 + qrow);
             const float4* del4 = reinterpret_cast<const float4*>(delta + row0 + qrow);
             const bool got = mbar_wait(B.prod + b, (g >> 1) & 1, B.abort_flag, dev_status);
@@ -408,31 +426,35 @@ k_bwd_dkdv_sm100(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
             tc_fence_after();
 #pragma unroll
             for (int hq = 0; hq < 2; ++hq) {
-                uint32_t s[32], p[32], op[16], od[16];
-                tmem_ld32(tl + cS + 128 * b + 32 * hq, s);
-                tmem_ld32(tl + cP + 128 * b + 32 * hq, p);
-                tmem_wait_ld();
+                uint32_t op[16], od[16];
+                if (valid) {
+                    uint32_t s[32], p[32];
+                    tmem_ld32(tl + cS + 128 * b + 32 * hq, s);
+                    tmem_ld32(tl + cP + 128 * b + 32 * hq, p);
+                    tmem_wait_ld();
 #pragma unroll
-                for (int i4 = 0; i4 < 8; ++i4) {
-                    const float4 l4 = __ldg(lse4 + 8 * hq + i4);
-                    const float4 d4 = __ldg(del4 + 8 * hq + i4);
-                    const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
-                    const float dv[4] = {d4.x, d4.y, d4.z, d4.w};
-                    float pp[4], dd[4];
+                    for (int i4 = 0; i4 < 8; ++i4) {
+                        const float4 l4 = __ldg(lse4 + 8 * hq + i4);
+                        const float4 d4 = __ldg(del4 + 8 * hq + i4);
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const int i = 4 * i4 + u;
-                        pp[u] = 0.f;
-                        dd[u] = 0.f;
-                        if (valid) {
-                            pp[u] = exp2f(fmaf(__uint_as_float(s[i]), sl2, -lv[u] * kLog2e));
-                            dd[u] = pp[u] * (__uint_as_float(p[i]) - dv[u]);
+                        for (int u = 0; u < 2; ++u) {
+                            const int i = 4 * i4 + 2 * u;
+                            const uint64_t nl = fmul2(u ? f2pack(l4.z, l4.w) : f2pack(l4.x, l4.y), nlog2e);
+                            const uint64_t nd = fmul2(u ? f2pack(d4.z, d4.w) : f2pack(d4.x, d4.y), neg1);
+                            float x0, x1;
+                            f2unpack(ffma2(f2pack(__uint_as_float(s[i]), __uint_as_float(s[i + 1])), sl2x2, nl), x0, x1);
+                            const float p0 = ex2(x0), p1 = ex2(x1);
+                            float d0, d1;
+                            f2unpack(fmul2(f2pack(p0, p1),
+                                           fadd2(f2pack(__uint_as_float(p[i]), __uint_as_float(p[i + 1])), nd)),
+                                     d0, d1);
+                            op[2 * i4 + u] = pack_bf16x2(p0, p1);
+                            od[2 * i4 + u] = pack_bf16x2(d0, d1);
                         }
                     }
-                    op[2 * i4] = pack_bf16x2(pp[0], pp[1]);
-                    op[2 * i4 + 1] = pack_bf16x2(pp[2], pp[3]);
-                    od[2 * i4] = pack_bf16x2(dd[0], dd[1]);
-                    od[2 * i4 + 1] = pack_bf16x2(dd[2], dd[3]);
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) { op[i] = 0u; od[i] = 0u; }
                 }
                 tmem_st16(tl + cS + 128 * b + 16 * hq, op);     // P^T over the consumed S^T columns
                 tmem_st16(tl + cP + 128 * b + 16 * hq, od);     // dS^T over the consumed dP^T columns
@@ -447,7 +469,6 @@ k_bwd_dkdv_sm100(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
             const int64_t grow = row0 + 128 * tile + row;
 #pragma unroll
             for (int which = 0; which < 2; ++which) {
-                __nv_bfloat16* out = (which ? dV : dK) + grow * D;
                 const float mul = which ? 1.f : scale;
                 const uint32_t col = which ? cdV : cdK;
 #pragma unroll
@@ -455,15 +476,27 @@ k_bwd_dkdv_sm100(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
                     uint32_t r[32];
                     tmem_ld32(tl + col + 32 * q, r);
                     tmem_wait_ld();
-                    uint32_t pk[16];
+                    if (ng == 0) {                          // no query selected these keys: zeros
 #pragma unroll
-                    for (int i = 0; i < 16; ++i)
-                        pk[i] = ng > 0 ? pack_bf16x2(__uint_as_float(r[2 * i]) * mul, __uint_as_float(r[2 * i + 1]) * mul)
-                                       : 0u;
-                    uint4* dst = reinterpret_cast<uint4*>(out + 32 * q);
+                        for (int i = 0; i < 32; ++i) r[i] = 0u;
+                    }
+                    if (slot < 0) {
+                        uint32_t pk[16];
 #pragma unroll
-                    for (int i = 0; i < 4; ++i)
-                        dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+                        for (int i = 0; i < 16; ++i)
+                            pk[i] = pack_bf16x2(__uint_as_float(r[2 * i]) * mul, __uint_as_float(r[2 * i + 1]) * mul);
+                        uint4* dst = reinterpret_cast<uint4*>((which ? dV : dK) + grow * D + 32 * q);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+                            dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+                    } else {                                // partial of a split tile (unscaled)
+                        float4* df = reinterpret_cast<float4*>(part + (((int64_t)slot * 2 + which) * 128 + row) * D +
+                                                               32 * q);
+#pragma unroll
+                        for (int i = 0; i < 8; ++i)
+                            df[i] = make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
+                                                __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]));
+                    }
                 }
             }
         }
@@ -474,11 +507,38 @@ k_bwd_dkdv_sm100(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
     if (warp == 1) tmem_dealloc(tb, kTmemCols);
 }
 
+// ------------------------------------------------------------------ host side
+struct BwdWs {
+    float* delta;
+    Plan pq, pkv;
+    float* part_q;      // [slots][128][D]
+    float* part_kv;     // [slots][2][128][D]
+};
+
+BwdWs carve_bwd(void* ws, const Dims& d, size_t* total) {
+    const int64_t tiles = (int64_t)d.heads * (d.N / 128);
+    const int target = plan_target(device_sms());
+    const int64_t slots = 2 * (int64_t)target;
+    uint8_t* p = static_cast<uint8_t*>(ws);
+    BwdWs w;
+    w.delta = reinterpret_cast<float*>(p);
+    p += align16((int64_t)d.heads * d.N * 4);
+    w.pq = carve_plan(p, tiles, target);
+    p += plan_bytes(tiles, target);
+    w.pkv = carve_plan(p, tiles, target);
+    p += plan_bytes(tiles, target);
+    w.part_q = reinterpret_cast<float*>(p);
+    p += align16(slots * 128 * d.d * 4);
+    w.part_kv = reinterpret_cast<float*>(p);
+    p += align16(slots * 2 * 128 * d.d * 4);
+    if (total) *total = (size_t)(p - static_cast<uint8_t*>(ws));
+    return w;
+}
+
 template <int D>
 prism_status_t launch_bwd(const Dims& d, const void* Qp, const void* Kp, const void* Vp, const void* dOp,
-                          const float* lse, const float* delta, const int32_t* blk_start, const int32_t* gran_blk,
-                          const int32_t* n_blk, const uint32_t* sel, const uint32_t* selT, float scale, void* dQp,
-                          void* dKp, void* dVp, uint32_t* dev_status, cudaStream_t s) {
+                          const float* lse, const uint32_t* gsel, const uint32_t* gselT, float scale, void* dQp,
+                          void* dKp, void* dVp, uint32_t* dev_status, const BwdWs& w, cudaStream_t s) {
     const int64_t rows = (int64_t)d.heads * d.N;
     CUtensorMap tQ, tdO, tK, tV, gQ, gdO, gK, gV;
     if (!make_map_bf16(&tQ, Qp, rows, D, 128) || !make_map_bf16(&tdO, dOp, rows, D, 128) ||
@@ -486,34 +546,46 @@ prism_status_t launch_bwd(const Dims& d, const void* Qp, const void* Kp, const v
         !make_map_bf16(&gQ, Qp, rows, D, 64) || !make_map_bf16(&gdO, dOp, rows, D, 64) ||
         !make_map_bf16(&gK, Kp, rows, D, 64) || !make_map_bf16(&gV, Vp, rows, D, 64))
         return PRISM_ERR_CUDA;
-    const int smem = BwdLayout<D>::ALLOC;
+    const int target = plan_target(device_sms());
+    prism_status_t st = plan_work(w.pq, gsel, d, 1, target, kSegMinGranules, s);
+    if (st == PRISM_OK) st = plan_work(w.pkv, gselT, d, 1, target, kSegMinGranules, s);
+    if (st != PRISM_OK) return st;
+    const int smem = BwdLayout<D>::alloc((int)d.SW);
     auto kq = k_bwd_dq_sm100<D>;
     auto kk = k_bwd_dkdv_sm100<D>;
     if (cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess ||
         cudaFuncSetAttribute(kk, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return PRISM_ERR_CUDA;
-    dim3 grid((unsigned)(d.N / 128), (unsigned)d.heads);
-    kq<<<grid, 192, smem, s>>>(tQ, tdO, gK, gV, blk_start, gran_blk, n_blk, sel, lse, delta, d.N, d.MB, (int)d.SW,
-                               scale, (__nv_bfloat16*)dQp, dev_status);
-    kk<<<grid, 192, smem, s>>>(tK, tV, gQ, gdO, blk_start, gran_blk, n_blk, selT, lse, delta, d.N, d.MB, (int)d.SW,
-                               scale, (__nv_bfloat16*)dKp, (__nv_bfloat16*)dVp, dev_status);
-    return launch_status(2);
+    kq<<<(unsigned)w.pq.items_max, 192, smem, s>>>(tQ, tdO, gK, gV, gsel, w.pq.hdr, w.pq.items, w.part_q, lse,
+                                                   w.delta, d.N, d.MB, (int)d.SW, scale, (__nv_bfloat16*)dQp,
+                                                   dev_status);
+    kk<<<(unsigned)w.pkv.items_max, 192, smem, s>>>(tK, tV, gQ, gdO, gselT, w.pkv.hdr, w.pkv.items, w.part_kv, lse,
+                                                    w.delta, d.N, d.MB, (int)d.SW, scale, (__nv_bfloat16*)dKp,
+                                                    (__nv_bfloat16*)dVp, dev_status);
+    st = launch_status(2);
+    if (st == PRISM_OK) st = bwd_combine(w.pq, d, 1, w.part_q, dQp, scale, nullptr, 0.f, s);
+    if (st == PRISM_OK) st = bwd_combine(w.pkv, d, 2, w.part_kv, dKp, scale, dVp, 1.f, s);
+    return st;
 }
 
 }  // namespace
 
+size_t attn_bwd_sm100_ws_bytes(const Dims& d) {
+    size_t total = 0;
+    carve_bwd(reinterpret_cast<void*>(uintptr_t(256)), d, &total);
+    return total;
+}
+
 prism_status_t attn_bwd_sm100(const Dims& d, const void* Qp, const void* Kp, const void* Vp, const void* Op,
-                              const float* o_f32, const void* dOp, const float* lse, const int32_t* blk_start,
-                              const int32_t* gran_blk, const int32_t* n_blk, const uint32_t* sel,
-                              const uint32_t* selT, float scale, void* dQp, void* dKp, void* dVp,
-                              uint32_t* dev_status, float* delta, cudaStream_t s) {
-    prism_status_t st = bwd_delta(d, Op, o_f32, dOp, delta, s);
+                              const float* o_f32, const void* dOp, const float* lse, const uint32_t* gsel,
+                              const uint32_t* gselT, float scale, void* dQp, void* dKp, void* dVp,
+                              uint32_t* dev_status, void* ws, cudaStream_t s) {
+    BwdWs w = carve_bwd(ws, d, nullptr);
+    prism_status_t st = bwd_delta(d, Op, o_f32, dOp, w.delta, s);
     if (st != PRISM_OK) return st;
     if (d.d == 128)
-        return launch_bwd<128>(d, Qp, Kp, Vp, dOp, lse, delta, blk_start, gran_blk, n_blk, sel, selT, scale, dQp,
-                               dKp, dVp, dev_status, s);
-    return launch_bwd<64>(d, Qp, Kp, Vp, dOp, lse, delta, blk_start, gran_blk, n_blk, sel, selT, scale, dQp, dKp,
-                          dVp, dev_status, s);
+        return launch_bwd<128>(d, Qp, Kp, Vp, dOp, lse, gsel, gselT, scale, dQp, dKp, dVp, dev_status, w, s);
+    return launch_bwd<64>(d, Qp, Kp, Vp, dOp, lse, gsel, gselT, scale, dQp, dKp, dVp, dev_status, w, s);
 }
 
 }  // namespace prism

@@ -7,11 +7,11 @@
 // gradients flow only through the attention over the selected blocks.
 //
 // Work unit: a 64-row tile of one head.  Blocks are whole 64-row granules,
-// so a query tile lies in one query block and every 64-key chunk of a
-// selected key block is unmasked.
+// so a query tile lies in one query block and every selected 64-key
+// granule (a bit of the granule-level selection row) is unmasked.
 //   k_fwd_simt     query tile x selected key chunks, online softmax (exp2 form)
 //   k_bwd_delta    Delta = rowsum(dO * O)
-//   k_bwd_dkdv     key tile x query chunks of the blocks that selected it (selT)
+//   k_bwd_dkdv     key tile x query granules of the blocks that selected it (gselT)
 //   k_bwd_dq       query tile x selected key chunks
 // Shared tiles are row-major with one float of padding (row stride = 1 mod 32
 // banks); thread (ty, tx) owns rows ty + 16u and columns tx + 16v.
@@ -36,10 +36,7 @@ __device__ __forceinline__ void load_tile(float* dst, const T* src, int tid) {
 template <typename T, int D>
 __global__ void __launch_bounds__(256) k_fwd_simt(const T* __restrict__ Q, const T* __restrict__ K,
                                                   const T* __restrict__ V,
-                                                  const int32_t* __restrict__ blk_start,
-                                                  const int32_t* __restrict__ gran_blk,
-                                                  const int32_t* __restrict__ n_blk,
-                                                  const uint32_t* __restrict__ sel, int64_t N,
+                                                  const uint32_t* __restrict__ gsel, int64_t N,
                                                   int64_t MB, int SW, float scale, T* __restrict__ O,
                                                   float* __restrict__ lse, float* __restrict__ o_f32) {
     constexpr int LD = D + 1, CW = D / 16;
@@ -50,10 +47,7 @@ __global__ void __launch_bounds__(256) k_fwd_simt(const T* __restrict__ Q, const
     float* Ps = Vs + 64 * LD;            // [64][65]
     const int g = blockIdx.x, hh = blockIdx.y, tid = threadIdx.x;
     const int tx = tid & 15, ty = tid >> 4;
-    const int nb = *n_blk;
     const int64_t q0 = (int64_t)g * 64;
-    const int ib = gran_blk[g];
-    if (ib < 0 || ib >= nb) return;
     const int64_t hoff = (int64_t)hh * N * D;
     load_tile<T, D>(Qs, Q + hoff + q0 * D, tid);
 
@@ -66,14 +60,13 @@ __global__ void __launch_bounds__(256) k_fwd_simt(const T* __restrict__ Q, const
 #pragma unroll
         for (int w = 0; w < CW; ++w) acc[u][w] = 0.f;
     }
-    const uint32_t* srow = sel + ((int64_t)hh * MB + ib) * SW;
-    const int wn = (nb + 31) >> 5;
-    for (int wi = 0; wi < wn; ++wi) {
+    const uint32_t* srow = gsel + ((int64_t)hh * MB + g) * SW;
+    for (int wi = 0; wi < SW; ++wi) {
         uint32_t bits = srow[wi];
         while (bits) {
             const int j = wi * 32 + __ffs(bits) - 1;
             bits &= bits - 1;
-            const int ks = blk_start[j], ke = blk_start[j + 1];
+            const int ks = 64 * j, ke = ks + 64;        // key granule j
             for (int k0 = ks; k0 < ke; k0 += 64) {
                 __syncthreads();
                 load_tile<T, D>(Ks, K + hoff + (int64_t)k0 * D, tid);
@@ -167,8 +160,7 @@ template <typename T, int D>
 __global__ void __launch_bounds__(256) k_bwd_dkdv_simt(
     const T* __restrict__ Q, const T* __restrict__ K, const T* __restrict__ V,
     const T* __restrict__ dO, const float* __restrict__ lse, const float* __restrict__ delta,
-    const int32_t* __restrict__ blk_start, const int32_t* __restrict__ gran_blk,
-    const int32_t* __restrict__ n_blk, const uint32_t* __restrict__ selT, int64_t N, int64_t MB,
+    const uint32_t* __restrict__ gselT, int64_t N, int64_t MB,
     int SW, float scale, T* __restrict__ dK, T* __restrict__ dV) {
     constexpr int LD = D + 1, CW = D / 16;
     extern __shared__ float sm[];
@@ -182,10 +174,7 @@ __global__ void __launch_bounds__(256) k_bwd_dkdv_simt(
     float* dl = lse2 + 64;               // [64]
     const int g = blockIdx.x, hh = blockIdx.y, tid = threadIdx.x;
     const int tx = tid & 15, ty = tid >> 4;
-    const int nb = *n_blk;
     const int64_t k0 = (int64_t)g * 64;
-    const int jb = gran_blk[g];
-    if (jb < 0 || jb >= nb) return;
     const int64_t hoff = (int64_t)hh * N * D;
     load_tile<T, D>(Ks, K + hoff + k0 * D, tid);
     load_tile<T, D>(Vs, V + hoff + k0 * D, tid);
@@ -196,14 +185,13 @@ __global__ void __launch_bounds__(256) k_bwd_dkdv_simt(
 #pragma unroll
         for (int w = 0; w < CW; ++w) aK[u][w] = aV[u][w] = 0.f;
 
-    const uint32_t* trow = selT + ((int64_t)hh * MB + jb) * SW;
-    const int wn = (nb + 31) >> 5;
-    for (int wi = 0; wi < wn; ++wi) {
+    const uint32_t* trow = gselT + ((int64_t)hh * MB + g) * SW;
+    for (int wi = 0; wi < SW; ++wi) {
         uint32_t bits = trow[wi];
         while (bits) {
             const int i = wi * 32 + __ffs(bits) - 1;
             bits &= bits - 1;
-            const int qs = blk_start[i], qe = blk_start[i + 1];
+            const int qs = 64 * i, qe = qs + 64;        // query granule i
             for (int qc = qs; qc < qe; qc += 64) {
                 __syncthreads();
                 load_tile<T, D>(Qs, Q + hoff + (int64_t)qc * D, tid);
@@ -275,8 +263,7 @@ template <typename T, int D>
 __global__ void __launch_bounds__(256) k_bwd_dq_simt(
     const T* __restrict__ Q, const T* __restrict__ K, const T* __restrict__ V,
     const T* __restrict__ dO, const float* __restrict__ lse, const float* __restrict__ delta,
-    const int32_t* __restrict__ blk_start, const int32_t* __restrict__ gran_blk,
-    const int32_t* __restrict__ n_blk, const uint32_t* __restrict__ sel, int64_t N, int64_t MB,
+    const uint32_t* __restrict__ gsel, int64_t N, int64_t MB,
     int SW, float scale, T* __restrict__ dQ) {
     constexpr int LD = D + 1, CW = D / 16;
     extern __shared__ float sm[];
@@ -287,10 +274,7 @@ __global__ void __launch_bounds__(256) k_bwd_dq_simt(
     float* dSs = Vs + 64 * LD;           // [64 queries][65]
     const int g = blockIdx.x, hh = blockIdx.y, tid = threadIdx.x;
     const int tx = tid & 15, ty = tid >> 4;
-    const int nb = *n_blk;
     const int64_t q0 = (int64_t)g * 64;
-    const int ib = gran_blk[g];
-    if (ib < 0 || ib >= nb) return;
     const int64_t hoff = (int64_t)hh * N * D;
     load_tile<T, D>(Qs, Q + hoff + q0 * D, tid);
     load_tile<T, D>(dOs, dO + hoff + q0 * D, tid);
@@ -303,14 +287,13 @@ __global__ void __launch_bounds__(256) k_bwd_dq_simt(
 #pragma unroll
         for (int w = 0; w < CW; ++w) acc[u][w] = 0.f;
     }
-    const uint32_t* srow = sel + ((int64_t)hh * MB + ib) * SW;
-    const int wn = (nb + 31) >> 5;
-    for (int wi = 0; wi < wn; ++wi) {
+    const uint32_t* srow = gsel + ((int64_t)hh * MB + g) * SW;
+    for (int wi = 0; wi < SW; ++wi) {
         uint32_t bits = srow[wi];
         while (bits) {
             const int j = wi * 32 + __ffs(bits) - 1;
             bits &= bits - 1;
-            const int ks = blk_start[j], ke = blk_start[j + 1];
+            const int ks = 64 * j, ke = ks + 64;        // key granule j
             for (int kc = ks; kc < ke; kc += 64) {
                 __syncthreads();
                 load_tile<T, D>(Ks, K + hoff + (int64_t)kc * D, tid);
@@ -370,25 +353,21 @@ template <int D> constexpr size_t dkdv_smem() { return (4 * 64 * (D + 1) + 2 * 6
 template <int D> constexpr size_t dq_smem() { return (4 * 64 * (D + 1) + 64 * 65) * sizeof(float); }
 
 template <typename T, int D>
-prism_status_t simt_fwd(const Dims& d, const void* Qp, const void* Kp, const void* Vp,
-                        const int32_t* blk_start, const int32_t* gran_blk, const int32_t* n_blk,
-                        const uint32_t* sel, float scale, void* Op, float* lse, float* o_f32,
-                        cudaStream_t s) {
+prism_status_t simt_fwd(const Dims& d, const void* Qp, const void* Kp, const void* Vp, const uint32_t* gsel,
+                        float scale, void* Op, float* lse, float* o_f32, cudaStream_t s) {
     auto k = k_fwd_simt<T, D>;
     if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fwd_smem<D>()) != cudaSuccess)
         return PRISM_ERR_CUDA;
     k<<<dim3((unsigned)d.MB, (unsigned)d.heads), 256, fwd_smem<D>(), s>>>(
-        (const T*)Qp, (const T*)Kp, (const T*)Vp, blk_start, gran_blk, n_blk, sel, d.N, d.MB, (int)d.SW,
-        scale, (T*)Op, lse, o_f32);
+        (const T*)Qp, (const T*)Kp, (const T*)Vp, gsel, d.N, d.MB, (int)d.SW, scale, (T*)Op, lse, o_f32);
     return launch_status(1);
 }
 
 template <typename T, int D>
 prism_status_t simt_bwd(const Dims& d, const void* Qp, const void* Kp, const void* Vp, const void* Op,
-                        const float* o_f32, const void* dOp, const float* lse, const int32_t* blk_start,
-                        const int32_t* gran_blk, const int32_t* n_blk, const uint32_t* sel,
-                        const uint32_t* selT, float scale, void* dQp, void* dKp, void* dVp,
-                        float* delta, cudaStream_t s) {
+                        const float* o_f32, const void* dOp, const float* lse, const uint32_t* gsel,
+                        const uint32_t* gselT, float scale, void* dQp, void* dKp, void* dVp, float* delta,
+                        cudaStream_t s) {
     const int64_t rows = (int64_t)d.heads * d.N;
     k_bwd_delta<T, D><<<(unsigned)((rows * 32 + 255) / 256), 256, 0, s>>>((const T*)Op, o_f32,
                                                                            (const T*)dOp, rows, delta);
@@ -399,19 +378,15 @@ prism_status_t simt_bwd(const Dims& d, const void* Qp, const void* Kp, const voi
         return PRISM_ERR_CUDA;
     dim3 grid((unsigned)d.MB, (unsigned)d.heads);
     kk<<<grid, 256, dkdv_smem<D>(), s>>>((const T*)Qp, (const T*)Kp, (const T*)Vp, (const T*)dOp, lse, delta,
-                                         blk_start, gran_blk, n_blk, selT, d.N, d.MB, (int)d.SW, scale,
-                                         (T*)dKp, (T*)dVp);
+                                         gselT, d.N, d.MB, (int)d.SW, scale, (T*)dKp, (T*)dVp);
     kq<<<grid, 256, dq_smem<D>(), s>>>((const T*)Qp, (const T*)Kp, (const T*)Vp, (const T*)dOp, lse, delta,
-                                       blk_start, gran_blk, n_blk, sel, d.N, d.MB, (int)d.SW, scale,
-                                       (T*)dQp);
+                                       gsel, d.N, d.MB, (int)d.SW, scale, (T*)dQp);
     return launch_status(3);
 }
 
-prism_status_t attn_fwd_simt(const Dims& d, const void* Qp, const void* Kp, const void* Vp,
-                             const int32_t* blk_start, const int32_t* gran_blk, const int32_t* n_blk,
-                             const uint32_t* sel, float scale, void* Op, float* lse, float* o_f32,
-                             cudaStream_t s) {
-#define PRISM_FWD_ARGS d, Qp, Kp, Vp, blk_start, gran_blk, n_blk, sel, scale, Op, lse, o_f32, s
+prism_status_t attn_fwd_simt(const Dims& d, const void* Qp, const void* Kp, const void* Vp, const uint32_t* gsel,
+                             float scale, void* Op, float* lse, float* o_f32, cudaStream_t s) {
+#define PRISM_FWD_ARGS d, Qp, Kp, Vp, gsel, scale, Op, lse, o_f32, s
     if (d.dtype == PRISM_F32)
         return d.d == 64 ? simt_fwd<float, 64>(PRISM_FWD_ARGS) : simt_fwd<float, 128>(PRISM_FWD_ARGS);
     return d.d == 64 ? simt_fwd<__nv_bfloat16, 64>(PRISM_FWD_ARGS) : simt_fwd<__nv_bfloat16, 128>(PRISM_FWD_ARGS);
@@ -435,11 +410,10 @@ prism_status_t bwd_delta(const Dims& d, const void* Op, const float* o_f32, cons
 }
 
 prism_status_t attn_bwd_simt(const Dims& d, const void* Qp, const void* Kp, const void* Vp, const void* Op,
-                             const float* o_f32, const void* dOp, const float* lse, const int32_t* blk_start,
-                             const int32_t* gran_blk, const int32_t* n_blk, const uint32_t* sel,
-                             const uint32_t* selT, float scale, void* dQp, void* dKp, void* dVp,
-                             float* delta, cudaStream_t s) {
-#define PRISM_BWD_ARGS d, Qp, Kp, Vp, Op, o_f32, dOp, lse, blk_start, gran_blk, n_blk, sel, selT, scale, dQp, dKp, dVp, delta, s
+                             const float* o_f32, const void* dOp, const float* lse, const uint32_t* gsel,
+                             const uint32_t* gselT, float scale, void* dQp, void* dKp, void* dVp, float* delta,
+                             cudaStream_t s) {
+#define PRISM_BWD_ARGS d, Qp, Kp, Vp, Op, o_f32, dOp, lse, gsel, gselT, scale, dQp, dKp, dVp, delta, s
     if (d.dtype == PRISM_F32)
         return d.d == 64 ? simt_bwd<float, 64>(PRISM_BWD_ARGS) : simt_bwd<float, 128>(PRISM_BWD_ARGS);
     return d.d == 64 ? simt_bwd<__nv_bfloat16, 64>(PRISM_BWD_ARGS) : simt_bwd<__nv_bfloat16, 128>(PRISM_BWD_ARGS);

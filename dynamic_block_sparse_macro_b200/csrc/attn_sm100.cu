@@ -3,12 +3,13 @@
 // Prism, Portuguese reading guide, "Método" 3: an online-softmax kernel runs
 // the attention only over the selected set S_i of each query block.
 //
-// Work unit: one CTA per (128-row query tile, head).  Blocks are whole 64-row
-// granules, so a tile holds either half of a 256-block, one 128-block, or two
-// 64-blocks b0, b1 (rows 0-63 and 64-127).  The key stream is the union of
-// S_b0 and S_b1 walked as 64-row granules in block order; two granules form
-// one 128-key chunk, and a per-granule 2-bit mask says which half of the tile
-// selected it (an odd tail repeats its last granule with mask 0).
+// Tiles: 128 query rows (two 64-row granules, which lie in one block or in two
+// 64-blocks).  A tile's keys are the union of the granule-level selection rows
+// of its two granules, walked in ascending order; two key granules form one
+// 128-key chunk, and a per-granule 2-bit mask says which half of the tile
+// selected it (an odd tail repeats its last granule with mask 0).  The work
+// plan (attn_plan.cu) cuts heavy tiles into segments of chunks; one CTA runs
+// one segment, and split tiles leave (O, m, l) partials for k_fwd_combine.
 //
 // Roles (6 warps):
 //   warp 0      TMA producer: Q once, then per chunk K and V (64x64 bf16 boxes,
@@ -18,11 +19,12 @@
 //               P read from TMEM (aliasing S) and V MN-major from shared memory.
 //   warps 2-5   one query row per thread: S row from TMEM, masked online
 //               softmax in the exp2 domain with lazy rescaling (the running
-//               max only moves when it grows by more than 2^8), P as bf16 back
-//               into TMEM, then the epilogue (O / l, LSE).
-// Two CTAs share an SM (96 KB shared memory and 256 TMEM columns each), so
-// one CTA's softmax overlaps the other's MMAs.  Every wait is bounded; a
-// timeout sets PRISM_DEV_TIMEOUT and the CTA winds down without trapping.
+//               max only moves when it grows by more than 2^8), packed fp32
+//               arithmetic, P as bf16 back into TMEM, then the epilogue.
+// Two CTAs share an SM (about 100 KB shared memory and 256 TMEM columns
+// each), so one CTA's softmax overlaps the other's MMAs.  Every wait is
+// bounded; a timeout sets PRISM_DEV_TIMEOUT and the CTA winds down.
+#include "attn_plan.cuh"
 #include "common.cuh"
 #include "sm100.cuh"
 
@@ -48,21 +50,35 @@ struct FwdLayout {
     static constexpr int K = NR * kRegion;
     static constexpr int V = 2 * NR * kRegion;
     static constexpr int CTRL = 3 * NR * kRegion;
-    static constexpr int BYTES = CTRL + 256;
-    // + slack for 1024-byte alignment; at least 80 KB so that no more than two
-    // CTAs (2 x 256 of the SM's 512 TMEM columns) are ever resident on an SM
-    static constexpr int ALLOC = (BYTES + 1024) > 80 * 1024 ? (BYTES + 1024) : 80 * 1024;
+    static constexpr int ROWS = CTRL + 256;        // two selection rows of SW words follow
+    // bytes to request: + slack for 1024-byte alignment; at least 80 KB so that
+    // no more than two CTAs (2 x 256 of the SM's 512 TMEM columns) share an SM
+    static int alloc(int SW) {
+        const int b = ROWS + 8 * SW + 1024;
+        return b > 80 * 1024 ? b : 80 * 1024;
+    }
+};
+
+struct FwdParts {
+    float* o;       // [slots][128][D] unnormalised O
+    float* m;       // [slots][128] running max, log2 domain
+    float* l;       // [slots][128] denominator
 };
 
 template <int D>
 __global__ void __launch_bounds__(192, 2)
 k_attn_fwd_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                 const __grid_constant__ CUtensorMap tmV, const int32_t* __restrict__ blk_start,
-                 const int32_t* __restrict__ gran_blk, const int32_t* __restrict__ n_blk,
-                 const uint32_t* __restrict__ sel, int64_t N, int64_t MB, int SW, float scale,
-                 __nv_bfloat16* __restrict__ O, float* __restrict__ lse, float* __restrict__ o_f32,
-                 uint32_t* __restrict__ dev_status) {
+                 const __grid_constant__ CUtensorMap tmV, const uint32_t* __restrict__ gsel,
+                 const PlanHeader* __restrict__ hdr, const int4* __restrict__ items, FwdParts parts,
+                 int64_t N, int64_t MB, int SW, float scale, __nv_bfloat16* __restrict__ O,
+                 float* __restrict__ lse, float* __restrict__ o_f32, uint32_t* __restrict__ dev_status) {
     using L = FwdLayout<D>;
+    if ((int)blockIdx.x >= hdr->n_items) return;              // uniform: beyond the item list
+    const int4 item = items[blockIdx.x];
+    const int tiles_per_head = (int)(N / 128);
+    const int hh = item.x / tiles_per_head, tile = item.x % tiles_per_head;
+    const int c_begin = item.y, nch = item.z - item.y, slot = item.w;
+
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sQ = sm + L::Q;
@@ -79,21 +95,15 @@ k_attn_fwd_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     uint64_t* bar_o = bars + 7;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 8);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-    int* nch_slot = reinterpret_cast<int*>(tmem_slot + 2);
+    uint32_t* u0 = reinterpret_cast<uint32_t*>(sm + L::ROWS);
+    uint32_t* u1 = u0 + SW;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int tile = blockIdx.x, hh = blockIdx.y;
-    const int nb = *n_blk;
-    const int b0 = gran_blk[2 * tile], b1 = gran_blk[2 * tile + 1];
-    if (b0 < 0 || b0 >= nb || b1 < 0 || b1 >= nb) {      // uniform across the CTA
-        if (threadIdx.x == 0) atomicOr(dev_status, PRISM_DEV_BAD_INDEX);
-        return;
-    }
-    const uint32_t* r0 = sel + ((int64_t)hh * MB + b0) * SW;
-    const uint32_t* r1 = sel + ((int64_t)hh * MB + b1) * SW;
-    const int wn = (nb + 31) >> 5;
+    const int wn = SW;
     const int64_t row0 = (int64_t)hh * N;                  // first row of this head in [heads*N, D]
 
+    // the selection rows of the tile's two query granules
+    load_rows(u0, u1, gsel + ((int64_t)hh * MB + 2 * tile) * SW, gsel + ((int64_t)hh * MB + 2 * tile + 1) * SW, wn);
     if (threadIdx.x == 0) {
         mbar_init(bar_q, 1);
         mbar_init(bar_kf, 1);
@@ -106,10 +116,7 @@ k_attn_fwd_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         *abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == 0) {                                       // count granules of the union
-        const int cnt = count_granules(r0, r1, blk_start, wn, lane);
-        if (lane == 0) *nch_slot = (cnt + 1) >> 1;
-    } else if (warp == 1) {
+    if (warp == 1) {
         tmem_alloc(tmem_slot, kTmemCols);
         tmem_relinquish();
     }
@@ -117,7 +124,6 @@ k_attn_fwd_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     __syncthreads();
     tc_fence_after();
     const uint32_t tbase = *tmem_slot;
-    const int nch = *nch_slot;
 
     if (warp == 0) {
         if (lane == 0) {
@@ -129,7 +135,8 @@ k_attn_fwd_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             for (int r = 0; r < L::NR; ++r)
                 tma_load_2d(sQ + r * kRegion, &tmQ, bar_q, 64 * r, (int)(row0 + 128 * tile));
             GranuleWalk walk;
-            walk.init(r0, r1, blk_start, wn);
+            walk.init(u0, u1, wn);
+            walk.skip(2 * c_begin);
             int issued_k = 0, issued_v = 0;
             for (int c = 0; c < nch && !*abort_flag; ++c) {
                 int ra = 0, rb = 0;
@@ -200,9 +207,13 @@ k_attn_fwd_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         const uint32_t tl = tbase + ((uint32_t)(sub * 32) << 16);
         const int half = row >> 6;
         const float sl2 = scale * kLog2e;
+        const uint64_t sl2x2 = f2pack(sl2, sl2);
         float m_run = -INFINITY, l = 0.f;
         GranuleWalk walk;
-        if (lane == 0) walk.init(r0, r1, blk_start, wn);
+        if (lane == 0) {
+            walk.init(u0, u1, wn);
+            walk.skip(2 * c_begin);
+        }
         bool ok = true;
         for (int c = 0; c < nch; ++c) {
             uint32_t mk = 0;
@@ -214,7 +225,7 @@ k_attn_fwd_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                 mk = ma | (mb << 2);
             }
             mk = __shfl_sync(0xffffffffu, mk, 0);
-            const bool v0 = (mk >> half) & 1u, v1 = (mk >> (2 + half)) & 1u;
+            const bool v0 = (mk >> half) & 1u, v1 = (mk >> (2 + half)) & 1u;   // warp-uniform
             const bool got = mbar_wait(bar_s, c & 1, abort_flag, dev_status);
             if (!__all_sync(0xffffffffu, got)) { ok = false; break; }   // warp-uniform exit
             tc_fence_after();
@@ -227,21 +238,27 @@ k_attn_fwd_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                 tmem_ld32(tl + kColS + 32 * q, r);
                 tmem_wait_ld();
 #pragma unroll
-                for (int i = 0; i < 32; ++i) mx = fmaxf(mx, __uint_as_float(r[i]));
+                for (int i = 0; i < 32; i += 2) mx = fmax3(mx, __uint_as_float(r[i]), __uint_as_float(r[i + 1]));
             }
             const float mx2 = mx * sl2;
             const bool need = mx2 > m_run + kRescaleThreshold || (m_run == -INFINITY && mx2 > -INFINITY);
-            const float alpha = need ? exp2f(m_run - mx2) : 1.f;   // 0 when m_run = -inf
+            const float alpha = need ? ex2(m_run - mx2) : 1.f;      // 0 when m_run = -inf
             // O holds chunks < c, all complete (S of chunk c was issued after them).
             // TMEM access is warp-collective: the whole warp rescales if any row must.
             if (c > 0 && __any_sync(0xffffffffu, need && m_run > -INFINITY)) {
+                const uint64_t a2 = f2pack(alpha, alpha);
 #pragma unroll
                 for (int q = 0; q < D / 32; ++q) {
                     uint32_t r[32];
                     tmem_ld32(tl + kColO + 32 * q, r);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+                    for (int i = 0; i < 32; i += 2) {
+                        float x, y;
+                        f2unpack(fmul2(f2pack(__uint_as_float(r[i]), __uint_as_float(r[i + 1])), a2), x, y);
+                        r[i] = __float_as_uint(x);
+                        r[i + 1] = __float_as_uint(y);
+                    }
                     tmem_st32(tl + kColO + 32 * q, r);
                 }
             }
@@ -249,31 +266,40 @@ k_attn_fwd_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                 l *= alpha;
                 m_run = mx2;
             }
-            // pass 2: P = exp2(s * scale * log2e - m) as bf16 into the first 64 columns of S
-            float rs = 0.f;
+            // pass 2: P = 2^(s * scale * log2e - m) as bf16 into the first 64 columns of S
+            const uint64_t negm = f2pack(-m_run, -m_run);
+            uint64_t rs2 = f2pack(0.f, 0.f);
 #pragma unroll
             for (int hq = 0; hq < 2; ++hq) {
-                const bool v = hq == 0 ? v0 : v1;
+                const bool v = (hq == 0 ? v0 : v1) && m_run > -INFINITY;
                 uint32_t pk[32];
+                if (__any_sync(0xffffffffu, v)) {
 #pragma unroll
-                for (int q2 = 0; q2 < 2; ++q2) {
-                    uint32_t r[32];
-                    tmem_ld32(tl + kColS + 64 * hq + 32 * q2, r);
-                    tmem_wait_ld();
+                    for (int q2 = 0; q2 < 2; ++q2) {
+                        uint32_t r[32];
+                        tmem_ld32(tl + kColS + 64 * hq + 32 * q2, r);
+                        tmem_wait_ld();
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        float p0 = 0.f, p1 = 0.f;
-                        if (v && m_run > -INFINITY) {
-                            p0 = exp2f(fmaf(__uint_as_float(r[2 * i]), sl2, -m_run));
-                            p1 = exp2f(fmaf(__uint_as_float(r[2 * i + 1]), sl2, -m_run));
+                        for (int i = 0; i < 16; ++i) {
+                            float x0, x1;
+                            f2unpack(ffma2(f2pack(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1])), sl2x2,
+                                           negm),
+                                     x0, x1);
+                            float p0 = ex2(x0), p1 = ex2(x1);
+                            if (!v) { p0 = 0.f; p1 = 0.f; }
+                            rs2 = fadd2(rs2, f2pack(p0, p1));
+                            pk[16 * q2 + i] = pack_bf16x2(p0, p1);
                         }
-                        rs += p0 + p1;
-                        pk[16 * q2 + i] = pack_bf16x2(p0, p1);
                     }
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) pk[i] = 0u;
                 }
                 tmem_st32(tl + kColS + 32 * hq, pk);
             }
-            l += rs;
+            float rsa, rsb;
+            f2unpack(rs2, rsa, rsb);
+            l += rsa + rsb;
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(bar_p);
@@ -281,34 +307,58 @@ k_attn_fwd_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         const bool fin = ok && mbar_wait(bar_o, 0, abort_flag, dev_status);
         if (__all_sync(0xffffffffu, fin)) {
             tc_fence_after();
-            const float inv = l > 0.f ? 1.f / l : 0.f;
             const int64_t grow = row0 + 128 * tile + row;
-            __nv_bfloat16* orow = O + grow * D;
+            if (slot < 0) {
+                const float inv = l > 0.f ? 1.f / l : 0.f;
+                __nv_bfloat16* orow = O + grow * D;
 #pragma unroll
-            for (int q = 0; q < D / 32; ++q) {
-                uint32_t r[32];
-                tmem_ld32(tl + kColO + 32 * q, r);
-                tmem_wait_ld();
-                if (!(l > 0.f)) {                          // empty selection: O = 0 (TMEM never written)
+                for (int q = 0; q < D / 32; ++q) {
+                    uint32_t r[32];
+                    tmem_ld32(tl + kColO + 32 * q, r);
+                    tmem_wait_ld();
+                    if (!(l > 0.f) || nch == 0) {           // nothing selected: O = 0 (TMEM never written)
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) r[i] = 0u;
+                        for (int i = 0; i < 32; ++i) r[i] = 0u;
+                    }
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        pk[i] = pack_bf16x2(__uint_as_float(r[2 * i]) * inv, __uint_as_float(r[2 * i + 1]) * inv);
+                    uint4* dst = reinterpret_cast<uint4*>(orow + 32 * q);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+                    if (o_f32) {
+                        float4* df = reinterpret_cast<float4*>(o_f32 + grow * D + 32 * q);
+#pragma unroll
+                        for (int i = 0; i < 8; ++i)
+                            df[i] = make_float4(__uint_as_float(r[4 * i]) * inv, __uint_as_float(r[4 * i + 1]) * inv,
+                                                __uint_as_float(r[4 * i + 2]) * inv,
+                                                __uint_as_float(r[4 * i + 3]) * inv);
+                    }
                 }
-                uint32_t pk[16];
+                lse[grow] = l > 0.f ? (m_run + log2f(l)) * kLn2 : -INFINITY;
+            } else {
+                // partial of a split tile: unnormalised O, running max and denominator
+                float* po = parts.o + ((int64_t)slot * 128 + row) * D;
 #pragma unroll
-                for (int i = 0; i < 16; ++i)
-                    pk[i] = pack_bf16x2(__uint_as_float(r[2 * i]) * inv, __uint_as_float(r[2 * i + 1]) * inv);
-                uint4* dst = reinterpret_cast<uint4*>(orow + 32 * q);
+                for (int q = 0; q < D / 32; ++q) {
+                    uint32_t r[32];
+                    tmem_ld32(tl + kColO + 32 * q, r);
+                    tmem_wait_ld();
+                    if (nch == 0) {
 #pragma unroll
-                for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
-                if (o_f32) {
-                    float4* df = reinterpret_cast<float4*>(o_f32 + grow * D + 32 * q);
+                        for (int i = 0; i < 32; ++i) r[i] = 0u;
+                    }
+                    float4* df = reinterpret_cast<float4*>(po + 32 * q);
 #pragma unroll
                     for (int i = 0; i < 8; ++i)
-                        df[i] = make_float4(__uint_as_float(r[4 * i]) * inv, __uint_as_float(r[4 * i + 1]) * inv,
-                                            __uint_as_float(r[4 * i + 2]) * inv, __uint_as_float(r[4 * i + 3]) * inv);
+                        df[i] = make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
+                                            __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]));
                 }
+                parts.m[(int64_t)slot * 128 + row] = m_run;
+                parts.l[(int64_t)slot * 128 + row] = l;
             }
-            lse[grow] = l > 0.f ? (m_run + log2f(l)) * kLn2 : -INFINITY;
         }
     }
 
@@ -319,34 +369,66 @@ k_attn_fwd_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
 }
 
 // ------------------------------------------------------------------ host side
+struct FwdWs {
+    Plan plan;
+    FwdParts parts;
+};
+
+size_t fwd_ws_bytes_d(const Dims& d) {
+    const int64_t tiles = (int64_t)d.heads * (d.N / 128);
+    const int target = plan_target(device_sms());
+    const int64_t slots = 2 * (int64_t)target;
+    return plan_bytes(tiles, target) + align16(slots * 128 * d.d * 4) + 2 * align16(slots * 128 * 4);
+}
+
+FwdWs carve_fwd(void* ws, const Dims& d) {
+    const int64_t tiles = (int64_t)d.heads * (d.N / 128);
+    const int target = plan_target(device_sms());
+    const int64_t slots = 2 * (int64_t)target;
+    FwdWs w;
+    w.plan = carve_plan(ws, tiles, target);
+    uint8_t* p = static_cast<uint8_t*>(ws) + plan_bytes(tiles, target);
+    w.parts.o = reinterpret_cast<float*>(p);
+    p += align16(slots * 128 * d.d * 4);
+    w.parts.m = reinterpret_cast<float*>(p);
+    p += align16(slots * 128 * 4);
+    w.parts.l = reinterpret_cast<float*>(p);
+    return w;
+}
+
 template <int D>
-prism_status_t launch_fwd(const Dims& d, const void* Qp, const void* Kp, const void* Vp, const int32_t* blk_start,
-                          const int32_t* gran_blk, const int32_t* n_blk, const uint32_t* sel, float scale, void* Op,
-                          float* lse, float* o_f32, uint32_t* dev_status, cudaStream_t s) {
+prism_status_t launch_fwd(const Dims& d, const void* Qp, const void* Kp, const void* Vp, const uint32_t* gsel,
+                          float scale, void* Op, float* lse, float* o_f32, uint32_t* dev_status, void* ws,
+                          cudaStream_t s) {
     CUtensorMap mQ, mK, mV;
     const int64_t rows = (int64_t)d.heads * d.N;
     if (!make_map_bf16(&mQ, Qp, rows, D, 128) || !make_map_bf16(&mK, Kp, rows, D, 64) ||
         !make_map_bf16(&mV, Vp, rows, D, 64))
         return PRISM_ERR_CUDA;
+    FwdWs w = carve_fwd(ws, d);
+    const int target = plan_target(device_sms());
+    prism_status_t st = plan_work(w.plan, gsel, d, 2, target, kSegMinChunks, s);
+    if (st != PRISM_OK) return st;
     auto k = k_attn_fwd_sm100<D>;
-    const int smem = FwdLayout<D>::ALLOC;
+    const int smem = FwdLayout<D>::alloc((int)d.SW);
     if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return PRISM_ERR_CUDA;
-    dim3 grid((unsigned)(d.N / 128), (unsigned)d.heads);
-    k<<<grid, 192, smem, s>>>(mQ, mK, mV, blk_start, gran_blk, n_blk, sel, d.N, d.MB, (int)d.SW, scale,
-                              (__nv_bfloat16*)Op, lse, o_f32, dev_status);
-    return launch_status(1);
+    k<<<(unsigned)w.plan.items_max, 192, smem, s>>>(mQ, mK, mV, gsel, w.plan.hdr, w.plan.items, w.parts, d.N, d.MB,
+                                                    (int)d.SW, scale, (__nv_bfloat16*)Op, lse, o_f32, dev_status);
+    st = launch_status(1);
+    if (st != PRISM_OK) return st;
+    return fwd_combine(w.plan, d, w.parts.o, w.parts.m, w.parts.l, Op, o_f32, lse, s);
 }
 
 }  // namespace
 
-prism_status_t attn_fwd_sm100(const Dims& d, const void* Qp, const void* Kp, const void* Vp,
-                              const int32_t* blk_start, const int32_t* gran_blk, const int32_t* n_blk,
-                              const uint32_t* sel, float scale, void* Op, float* lse, float* o_f32,
-                              uint32_t* dev_status, cudaStream_t s) {
-    if (d.d == 128)
-        return launch_fwd<128>(d, Qp, Kp, Vp, blk_start, gran_blk, n_blk, sel, scale, Op, lse, o_f32, dev_status, s);
-    return launch_fwd<64>(d, Qp, Kp, Vp, blk_start, gran_blk, n_blk, sel, scale, Op, lse, o_f32, dev_status, s);
+size_t attn_fwd_sm100_ws_bytes(const Dims& d) { return fwd_ws_bytes_d(d); }
+
+prism_status_t attn_fwd_sm100(const Dims& d, const void* Qp, const void* Kp, const void* Vp, const uint32_t* gsel,
+                              float scale, void* Op, float* lse, float* o_f32, uint32_t* dev_status, void* ws,
+                              cudaStream_t s) {
+    if (d.d == 128) return launch_fwd<128>(d, Qp, Kp, Vp, gsel, scale, Op, lse, o_f32, dev_status, ws, s);
+    return launch_fwd<64>(d, Qp, Kp, Vp, gsel, scale, Op, lse, o_f32, dev_status, ws, s);
 }
 
 }  // namespace prism

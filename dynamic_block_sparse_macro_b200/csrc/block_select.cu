@@ -137,22 +137,58 @@ __global__ void __launch_bounds__(512) k_block_select(const float* __restrict__ 
     }
 }
 
-__global__ void k_select_transpose(const uint32_t* __restrict__ sel, const int32_t* __restrict__ n_blk,
-                                   int64_t MB, int SW, uint32_t* __restrict__ selT) {
-    const int i = blockIdx.x, hh = blockIdx.y;
+// Granule-level view of the selection for the attention kernels: row qg (a
+// 64-row query granule) has bit kg set when the block of key granule kg is
+// in S of the block of qg.  Same size as the block-level mask (N/64 rows of
+// N/64 bits), but a kernel reads key rows straight from the bit position.
+__global__ void __launch_bounds__(128) k_sel_expand(const uint32_t* __restrict__ sel,
+                                                    const int32_t* __restrict__ blk_start,
+                                                    const int32_t* __restrict__ gran_blk,
+                                                    const int32_t* __restrict__ n_blk, int64_t MB, int SW,
+                                                    uint32_t* __restrict__ gsel) {
+    extern __shared__ uint32_t row[];
+    const int qg = blockIdx.x, hh = blockIdx.y;
     const int nb = *n_blk;
-    if (i >= nb) return;
-    const uint32_t* row = sel + ((int64_t)hh * MB + i) * SW;
-    const int wn = (nb + 31) >> 5;
-    for (int w = threadIdx.x; w < wn; w += blockDim.x) {
-        uint32_t b = row[w];
-        while (b) {
-            const int k = __ffs(b) - 1;
-            b &= b - 1;
-            const int j = w * 32 + k;
-            atomicOr(&selT[((int64_t)hh * MB + j) * SW + (i >> 5)], 1u << (i & 31));
+    for (int w = threadIdx.x; w < SW; w += blockDim.x) row[w] = 0u;
+    __syncthreads();
+    const int i = gran_blk[qg];
+    if (i >= 0 && i < nb) {
+        const uint32_t* srow = sel + ((int64_t)hh * MB + i) * SW;
+        const int wn = (nb + 31) >> 5;
+        for (int w = threadIdx.x; w < wn; w += blockDim.x) {
+            uint32_t b = srow[w];
+            while (b) {
+                const int j = w * 32 + __ffs(b) - 1;
+                b &= b - 1;
+                const int g0 = blk_start[j] >> 6, g1 = blk_start[j + 1] >> 6;   // granules [g0, g1)
+                for (int g = g0; g < g1; ++g) atomicOr(&row[g >> 5], 1u << (g & 31));
+            }
         }
     }
+    __syncthreads();
+    uint32_t* out = gsel + ((int64_t)hh * MB + qg) * SW;
+    for (int w = threadIdx.x; w < SW; w += blockDim.x) out[w] = row[w];
+}
+
+// Bit-matrix transpose, one warp per 32x32 tile: lane l holds row (32 rt + l)
+// word wc; ballot over bit b gives row (32 wc + b) of the transpose.
+__global__ void __launch_bounds__(256) k_bit_transpose(const uint32_t* __restrict__ in, int64_t MB, int SW,
+                                                       uint32_t* __restrict__ out) {
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    const int wc = blockIdx.x;                         // source word column
+    const int rt = blockIdx.y * 8 + wid;               // source row tile
+    const int hh = blockIdx.z;
+    if (rt >= SW) return;                              // warp-uniform
+    const int64_t r = (int64_t)rt * 32 + lane;
+    const uint32_t x = r < MB ? in[((int64_t)hh * MB + r) * SW + wc] : 0u;
+    uint32_t mine = 0u;
+#pragma unroll
+    for (int b = 0; b < 32; ++b) {
+        const uint32_t t = __ballot_sync(0xffffffffu, (x >> b) & 1u);
+        if (lane == b) mine = t;
+    }
+    const int64_t orow = (int64_t)wc * 32 + lane;
+    if (orow < MB) out[((int64_t)hh * MB + orow) * SW + rt] = mine;
 }
 
 int select_keycap(const Dims& d) {
@@ -170,15 +206,16 @@ size_t select_smem_bytes(const Dims& d) {
 using namespace prism;
 
 extern "C" prism_status_t prism_block_select(const prism_problem_t* prob, const float* P,
+                                             const int32_t* blk_start, const int32_t* gran_blk,
                                              const int32_t* n_blk, int32_t top_k, float top_p,
-                                             uint32_t* sel, int32_t* sel_count, uint32_t* selT,
-                                             float* margin, uint32_t* dev_status,
+                                             uint32_t* sel, int32_t* sel_count, uint32_t* gsel,
+                                             uint32_t* gselT, float* margin, uint32_t* dev_status,
                                              cudaStream_t stream) {
     Dims d;
     prism_status_t st = make_dims(prob, &d);
     if (st != PRISM_OK) return st;
-    if (!ok_ptr(P) || !ok_ptr(n_blk) || !ok_ptr(sel) || !ok_ptr(sel_count) || !ok_opt(selT) ||
-        !ok_opt(margin) || !ok_ptr(dev_status))
+    if (!ok_ptr(P) || !ok_ptr(blk_start) || !ok_ptr(gran_blk) || !ok_ptr(n_blk) || !ok_ptr(sel) ||
+        !ok_ptr(sel_count) || !ok_ptr(gsel) || !ok_opt(gselT) || !ok_opt(margin) || !ok_ptr(dev_status))
         return PRISM_ERR_INVALID_ARG;
     if (top_k < 1 || !(top_p > 0.f) || !isfinite(top_p)) return PRISM_ERR_INVALID_ARG;
     size_t smem = select_smem_bytes(d);
@@ -188,11 +225,10 @@ extern "C" prism_status_t prism_block_select(const prism_problem_t* prob, const 
         return PRISM_ERR_CUDA;
     k_block_select<<<dim3((unsigned)d.MB, (unsigned)d.heads), 512, smem, stream>>>(
         P, n_blk, d.MB, (int)d.SW, select_keycap(d), top_k, top_p, sel, sel_count, margin, dev_status);
-    if (selT) {
-        if (cudaMemsetAsync(selT, 0, (size_t)d.heads * d.MB * d.SW * 4, stream) != cudaSuccess)
-            return PRISM_ERR_CUDA;
-        k_select_transpose<<<dim3((unsigned)d.MB, (unsigned)d.heads), 128, 0, stream>>>(sel, n_blk, d.MB,
-                                                                                       (int)d.SW, selT);
-    }
-    return launch_status(selT ? 2 : 1);
+    k_sel_expand<<<dim3((unsigned)d.MB, (unsigned)d.heads), 128, (size_t)d.SW * 4, stream>>>(
+        sel, blk_start, gran_blk, n_blk, d.MB, (int)d.SW, gsel);
+    if (gselT)
+        k_bit_transpose<<<dim3((unsigned)d.SW, (unsigned)((d.SW + 7) / 8), (unsigned)d.heads), 256, 0, stream>>>(
+            gsel, d.MB, (int)d.SW, gselT);
+    return launch_status(gselT ? 3 : 2);
 }

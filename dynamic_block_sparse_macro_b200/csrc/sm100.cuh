@@ -183,62 +183,105 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn, b
            ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
+// ------------------------------------------------------------------ packed fp32 math
+__device__ __forceinline__ uint64_t f2pack(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void f2unpack(uint64_t v, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+// (a, b) * (m, m) + (c, c), two lanes of fp32 in one instruction
+__device__ __forceinline__ uint64_t ffma2(uint64_t ab, uint64_t mm, uint64_t cc) {
+    uint64_t r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(ab), "l"(mm), "l"(cc));
+    return r;
+}
+__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ uint64_t fmul2(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+// 2^x (hardware approximation, flushes denormals)
+__device__ __forceinline__ float ex2(float x) {
+    float r;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     uint32_t r;
     asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
     return r;
 }
 
-// Walks the union of two bitmask rows (selection rows of two query blocks, or
-// key-major rows of two key blocks) as 64-row granules, in block order.  The
-// 2-bit mask of a granule says which of the two rows contains its block.
+// Walks the union of two granule-level selection rows (held in shared
+// memory) in ascending granule order.  A set bit g stands for the 64 rows
+// starting at row 64 g; the 2-bit mask says which of the two rows has it.
 struct GranuleWalk {
-    const uint32_t* r0;
-    const uint32_t* r1;
-    const int32_t* blk_start;
-    int wn, w, g, ng, base;
-    uint32_t bits, mask;
+    const uint32_t* u0;
+    const uint32_t* u1;
+    int wn, w;
+    uint32_t bits;
 
-    __device__ void init(const uint32_t* a, const uint32_t* b, const int32_t* bs, int words) {
-        r0 = a; r1 = b; blk_start = bs; wn = words; w = 0; g = 0; ng = 0; base = 0; mask = 0;
-        bits = wn > 0 ? (r0[0] | r1[0]) : 0u;
+    __device__ void init(const uint32_t* a, const uint32_t* b, int words) {
+        u0 = a; u1 = b; wn = words; w = 0;
+        bits = wn > 0 ? (u0[0] | u1[0]) : 0u;
+    }
+    // advance past n granules
+    __device__ void skip(int n) {
+        while (n > 0) {
+            const int c = __popc(bits);
+            if (c <= n) {
+                n -= c;
+                bits = 0u;
+                if (++w >= wn) return;
+                bits = u0[w] | u1[w];
+            } else {
+                for (; n > 0; --n) bits &= bits - 1;
+            }
+        }
     }
     __device__ bool next(int& row, uint32_t& m) {
-        while (g >= ng) {
-            while (bits == 0) {
-                if (++w >= wn) return false;
-                bits = r0[w] | r1[w];
-            }
-            const int b = __ffs(bits) - 1;
-            bits &= bits - 1;
-            const int j = w * 32 + b;
-            base = blk_start[j];
-            ng = (blk_start[j + 1] - base) >> 6;
-            g = 0;
-            mask = ((r0[w] >> b) & 1u) | (((r1[w] >> b) & 1u) << 1);
+        while (bits == 0) {
+            if (++w >= wn) return false;
+            bits = u0[w] | u1[w];
         }
-        row = base + 64 * g;
-        ++g;
-        m = mask;
+        const int b = __ffs(bits) - 1;
+        bits &= bits - 1;
+        row = 64 * (w * 32 + b);
+        m = ((u0[w] >> b) & 1u) | (((u1[w] >> b) & 1u) << 1);
         return true;
     }
 };
 
-// number of 64-row granules in the union of two bitmask rows (one warp)
-__device__ __forceinline__ int count_granules(const uint32_t* r0, const uint32_t* r1, const int32_t* blk_start,
-                                              int wn, int lane) {
+// number of granules in the union of two rows (one warp)
+__device__ __forceinline__ int count_granules(const uint32_t* u0, const uint32_t* u1, int wn, int lane) {
     int cnt = 0;
-    for (int w = lane; w < wn; w += 32) {
-        uint32_t b = r0[w] | r1[w];
-        while (b) {
-            const int j = w * 32 + __ffs(b) - 1;
-            b &= b - 1;
-            cnt += (blk_start[j + 1] - blk_start[j]) >> 6;
-        }
-    }
+    for (int w = lane; w < wn; w += 32) cnt += __popc(u0[w] | u1[w]);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
     return cnt;
+}
+
+// copy two selection rows of `wn` words into shared memory (whole CTA)
+__device__ __forceinline__ void load_rows(uint32_t* dst0, uint32_t* dst1, const uint32_t* src0,
+                                          const uint32_t* src1, int wn) {
+    for (int w = threadIdx.x; w < wn; w += blockDim.x) {
+        dst0[w] = src0[w];
+        dst1[w] = src1[w];
+    }
 }
 
 // ------------------------------------------------------------------ host: TMA maps

@@ -58,7 +58,9 @@ class PrismSparseAttention:
         self.p_blocks = pb
         self.P = e(heads * pb * pb)
         self.sel = e(heads, MB, SW, dt=torch.int32)
-        self.selT = e(heads, MB, SW, dt=torch.int32)
+        # granule-level selection (the attention kernels' view) and its transpose
+        self.gsel = e(heads, MB, SW, dt=torch.int32)
+        self.gselT = e(heads, MB, SW, dt=torch.int32)
         self.sel_count = e(heads, MB, dt=i32)
         self.margin_sel = e(heads, MB)
         self.dev_status = torch.zeros(1, dtype=i32, device=dev)
@@ -90,14 +92,14 @@ class PrismSparseAttention:
         _abi.prism_permute(p, V, self.perm, self.Vp, stream)
         _abi.prism_block_pool_score(p, self.Qp, self.Kp, self.blk_start, self.n_blk, self.scale,
                                     self.Qbar, self.Kbar, self.P, stream)
-        _abi.prism_block_select(p, self.P, self.n_blk, self.top_k, self.top_p, self.sel, self.sel_count,
-                                self.selT, self.margin_sel, self.dev_status, stream)
+        _abi.prism_block_select(p, self.P, self.blk_start, self.gran_blk, self.n_blk, self.top_k, self.top_p,
+                                self.sel, self.sel_count, self.gsel, self.gselT, self.margin_sel,
+                                self.dev_status, stream)
 
     def attend(self, stream=None):
         """Stage 6 on the blocked tensors."""
-        _abi.prism_sparse_attn_fwd(self.prob, self.Qp, self.Kp, self.Vp, self.blk_start, self.gran_blk,
-                                   self.n_blk, self.sel, self.scale, self.Op, self.lse, self.Of32,
-                                   self.dev_status, self.ws_fwd, stream)
+        _abi.prism_sparse_attn_fwd(self.prob, self.Qp, self.Kp, self.Vp, self.gsel, self.scale, self.Op,
+                                   self.lse, self.Of32, self.dev_status, self.ws_fwd, stream)
 
     def forward(self, Q, K, V, hhat, out=None, stream=None):
         """Whole forward; returns O in raster layout."""
@@ -114,9 +116,8 @@ class PrismSparseAttention:
         p = self.prob
         _abi.prism_permute(p, dO, self.perm, self.dOp, stream)
         _abi.prism_sparse_attn_bwd(p, self.Qp, self.Kp, self.Vp, self.Op, self.Of32, self.dOp, self.lse,
-                                   self.blk_start,
-                                   self.gran_blk, self.n_blk, self.sel, self.selT, self.scale, self.dQp,
-                                   self.dKp, self.dVp, self.dev_status, self.ws_bwd, stream)
+                                   self.gsel, self.gselT, self.scale, self.dQp, self.dKp, self.dVp,
+                                   self.dev_status, self.ws_bwd, stream)
         outs = []
         for src, dst in ((self.dQp, dQ), (self.dKp, dK), (self.dVp, dV)):
             if dst is None:

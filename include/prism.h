@@ -178,24 +178,30 @@ prism_status_t prism_block_pool_score(const prism_problem_t* prob, const void* Q
  * first max(min(k, n_blk), n_p) blocks.
  *   sel       [heads][max_blocks][sel_words] uint32 bitmask, bit j of row i
  *   sel_count [heads][max_blocks] int32 (|S_i|; rows past n_blk are 0)
- *   selT      [heads][max_blocks][sel_words] uint32 (nullable): transpose of sel,
- *             bit i of row j set when j is in S_i (the backward's key-major view)
+ *   gsel      [heads][N/64][sel_words] uint32: the same selection at granule
+ *             level, the view the attention kernels read: row qg (64-row query
+ *             granule) has bit kg set when the block of key granule kg is in S
+ *             of the block of qg (blk_start, gran_blk from prism_assign_shapes)
+ *   gselT     [heads][N/64][sel_words] uint32 (nullable): transpose of gsel, the
+ *             key-major view of the backward
  *   margin    [heads][max_blocks] float32 (nullable): smallest gap (order or
  *             cumulative-sum) that, crossed by rounding, could change S_i
  *   dev_status  PRISM_DEV_BAD_INDEX if n_blk exceeds the 16384 keys a row can
  *             sort in shared memory (then every row is left empty).
  * Rows i >= n_blk are written as empty rows with count 0.
  */
-prism_status_t prism_block_select(const prism_problem_t* prob, const float* P, const int32_t* n_blk,
-                                  int32_t top_k, float top_p, uint32_t* sel, int32_t* sel_count,
-                                  uint32_t* selT, float* margin, uint32_t* dev_status,
+prism_status_t prism_block_select(const prism_problem_t* prob, const float* P, const int32_t* blk_start,
+                                  const int32_t* gran_blk, const int32_t* n_blk, int32_t top_k,
+                                  float top_p, uint32_t* sel, int32_t* sel_count, uint32_t* gsel,
+                                  uint32_t* gselT, float* margin, uint32_t* dev_status,
                                   cudaStream_t stream);
 
 /*
  * Stage 6 — exact online-softmax attention of every query block over the tokens
  * of its selected key blocks ("Método" 3; non-causal, scale usually 1/sqrt(d)).
- *   Qp, Kp, Vp blocked [heads][N][d];  Op blocked;  lse [heads][N] float32
- *   (natural log of the softmax denominator; -inf for an empty S_i, whose O is 0).
+ *   Qp, Kp, Vp blocked [heads][N][d];  gsel granule-level selection from
+ *   prism_block_select;  Op blocked;  lse [heads][N] float32 (natural log of
+ *   the softmax denominator; -inf for an empty S_i, whose O is 0).
  *   o_f32 (nullable) blocked [heads][N][d] float32: the unrounded O, for the
  *   backward's Delta (with a bf16 O, rowsum(dO*O) carries O's rounding error,
  *   which dominates dQ/dK when the attention is diffuse).
@@ -203,11 +209,9 @@ prism_status_t prism_block_select(const prism_problem_t* prob, const float* P, c
  * bf16 runs on tcgen05 tensor cores (fp32 accumulation); f32 on CUDA cores.
  */
 prism_status_t prism_sparse_attn_fwd(const prism_problem_t* prob, const void* Qp, const void* Kp,
-                                     const void* Vp, const int32_t* blk_start,
-                                     const int32_t* gran_blk, const int32_t* n_blk,
-                                     const uint32_t* sel, float scale, void* Op, float* lse,
-                                     float* o_f32, uint32_t* dev_status, void* ws, size_t ws_bytes,
-                                     cudaStream_t stream);
+                                     const void* Vp, const uint32_t* gsel, float scale, void* Op,
+                                     float* lse, float* o_f32, uint32_t* dev_status, void* ws,
+                                     size_t ws_bytes, cudaStream_t stream);
 
 /*
  * Stage 7 — gradients of stage 6 under the fixed selection (Chinese guide,
@@ -216,15 +220,15 @@ prism_status_t prism_sparse_attn_fwd(const prism_problem_t* prob, const void* Qp
  * P = exp(s - lse), dV = P^T dO, dS = P*(dO V^T - Delta), dQ = scale*dS K,
  * dK = scale*dS^T Q.  Keys no query selected get dK = dV = 0.
  * Delta uses o_f32 when it is given (the forward's unrounded O), else Op.
- * All tensors blocked; ws >= sizes.ws_attn_bwd bytes.
+ * gsel, gselT from prism_block_select.  All tensors blocked;
+ * ws >= sizes.ws_attn_bwd bytes.
  */
 prism_status_t prism_sparse_attn_bwd(const prism_problem_t* prob, const void* Qp, const void* Kp,
                                      const void* Vp, const void* Op, const float* o_f32,
-                                     const void* dOp, const float* lse, const int32_t* blk_start,
-                                     const int32_t* gran_blk, const int32_t* n_blk,
-                                     const uint32_t* sel, const uint32_t* selT, float scale,
-                                     void* dQp, void* dKp, void* dVp, uint32_t* dev_status,
-                                     void* ws, size_t ws_bytes, cudaStream_t stream);
+                                     const void* dOp, const float* lse, const uint32_t* gsel,
+                                     const uint32_t* gselT, float scale, void* dQp, void* dKp,
+                                     void* dVp, uint32_t* dev_status, void* ws, size_t ws_bytes,
+                                     cudaStream_t stream);
 
 /* Copy a device status word to the host (synchronises `stream`). */
 prism_status_t prism_read_status(const uint32_t* dev_status, uint32_t* host_out, cudaStream_t stream);

@@ -120,8 +120,11 @@ def check_layer(cfg, x, top_k=None, top_p=None, backward=True, heads=None, grad_
     assert (e2e["margin"][badr2] < NEAR_TIE).all()
     rep["select_near_ties"] = int(badr2.sum())
     rep["density"] = float(sel_g.mean())
-    selT = unpack_sel(mod.selT, nb)
-    assert np.array_equal(selT, sel_g.transpose(0, 2, 1))
+    # granule-level view: row qg, bit kg set iff block(kg) in S_block(qg); and its transpose
+    G = unpack_sel(mod.gsel, cfg.n_tokens // 64)
+    gb = np.repeat(np.arange(nb), np.diff(bs) // 64)
+    assert np.array_equal(G, sel_g[:, gb][:, :, gb])
+    assert np.array_equal(unpack_sel(mod.gselT, cfg.n_tokens // 64), G.transpose(0, 2, 1))
 
     # stage 6: attention under the GPU's own selection
     hs = list(range(cfg.heads)) if heads is None else heads

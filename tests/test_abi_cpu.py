@@ -75,8 +75,13 @@ def test_bad_pointers_rejected_before_launch(L):
     # in place is refused
     assert L.prism_permute(ctypes.byref(p), fake, fake, fake, None) == 1
     # bad scalars
-    assert L.prism_block_select(ctypes.byref(p), fake, fake, 0, 0.9, fake, fake, None, None, fake, None) == 1
-    assert L.prism_block_select(ctypes.byref(p), fake, fake, 4, float("nan"), fake, fake, None, None, fake, None) == 1
+    assert L.prism_block_select(ctypes.byref(p), fake, fake, fake, fake, 0, 0.9, fake, fake, fake, None, None,
+                                fake, None) == 1
+    assert L.prism_block_select(ctypes.byref(p), fake, fake, fake, fake, 4, float("nan"), fake, fake, fake, None,
+                                None, fake, None) == 1
+    # granule-level selection is required
+    assert L.prism_block_select(ctypes.byref(p), fake, fake, fake, fake, 4, 0.9, fake, fake, None, None, None,
+                                fake, None) == 1
     assert L.prism_zone_indicator(ctypes.byref(p), fake, fake, 0.0, fake, fake, fake, None, fake, 1 << 20, None) == 1
     # workspace too small
     assert L.prism_zone_indicator(ctypes.byref(p), fake, fake, 1e-6, fake, fake, fake, None, fake, 4, None) == 4
