@@ -140,20 +140,34 @@ __global__ void __launch_bounds__(256) k_fwd_simt(const T* __restrict__ Q, const
     }
 }
 
-// Delta = rowsum(dO * O), from the unrounded fp32 O when the forward kept it
+// Delta = rowsum(dO * O), from the unrounded fp32 O when the forward kept it.
+// Each lane reads 4 consecutive elements (16-byte fp32 / 8-byte bf16 vectors);
+// D/4 lanes cover a row, so a warp covers 128/D rows.
+template <typename T> __device__ __forceinline__ float4 load4(const T* p);
+template <> __device__ __forceinline__ float4 load4<float>(const float* p) { return __ldg(reinterpret_cast<const float4*>(p)); }
+template <> __device__ __forceinline__ float4 load4<__nv_bfloat16>(const __nv_bfloat16* p) {
+    const uint2 u = __ldg(reinterpret_cast<const uint2*>(p));
+    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
+    const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
+    return make_float4(a.x, a.y, b.x, b.y);
+}
+
 template <typename T, int D>
 __global__ void k_bwd_delta(const T* __restrict__ O, const float* __restrict__ o_f32,
                             const T* __restrict__ dO, int64_t rows, float* __restrict__ delta) {
-    const int64_t r = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    const int lane = threadIdx.x & 31;
-    if (r >= rows) return;
+    constexpr int LPR = D / 4;                                // lanes per row
+    const int64_t gl = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t r = gl / LPR;
+    const int c = (int)(gl % LPR) * 4;
     float s = 0.f;
-    if (o_f32)
-        for (int c = lane; c < D; c += 32) s += o_f32[r * D + c] * to_f32(dO[r * D + c]);
-    else
-        for (int c = lane; c < D; c += 32) s += to_f32(O[r * D + c]) * to_f32(dO[r * D + c]);
-    s = warp_sum(s);
-    if (lane == 0) delta[r] = s;
+    if (r < rows) {
+        const float4 g = load4<T>(dO + r * D + c);
+        const float4 o = o_f32 ? __ldg(reinterpret_cast<const float4*>(o_f32 + r * D + c)) : load4<T>(O + r * D + c);
+        s = o.x * g.x + o.y * g.y + o.z * g.z + o.w * g.w;
+    }
+#pragma unroll
+    for (int off = LPR / 2; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+    if (r < rows && (gl % LPR) == 0) delta[r] = s;
 }
 
 template <typename T, int D>
@@ -369,8 +383,8 @@ prism_status_t simt_bwd(const Dims& d, const void* Qp, const void* Kp, const voi
                         const uint32_t* gselT, float scale, void* dQp, void* dKp, void* dVp, float* delta,
                         cudaStream_t s) {
     const int64_t rows = (int64_t)d.heads * d.N;
-    k_bwd_delta<T, D><<<(unsigned)((rows * 32 + 255) / 256), 256, 0, s>>>((const T*)Op, o_f32,
-                                                                           (const T*)dOp, rows, delta);
+    k_bwd_delta<T, D><<<(unsigned)((rows * (D / 4) + 255) / 256), 256, 0, s>>>((const T*)Op, o_f32,
+                                                                                (const T*)dOp, rows, delta);
     auto kk = k_bwd_dkdv_simt<T, D>;
     auto kq = k_bwd_dq_simt<T, D>;
     if (cudaFuncSetAttribute(kk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dkdv_smem<D>()) != cudaSuccess ||
@@ -397,7 +411,7 @@ prism_status_t attn_fwd_simt(const Dims& d, const void* Qp, const void* Kp, cons
 prism_status_t bwd_delta(const Dims& d, const void* Op, const float* o_f32, const void* dOp, float* delta,
                          cudaStream_t s) {
     const int64_t rows = (int64_t)d.heads * d.N;
-    const unsigned grid = (unsigned)((rows * 32 + 255) / 256);
+    const unsigned grid = (unsigned)((rows * (d.d / 4) + 255) / 256);
     if (d.dtype == PRISM_F32) {
         if (d.d == 64) k_bwd_delta<float, 64><<<grid, 256, 0, s>>>((const float*)Op, o_f32, (const float*)dOp, rows, delta);
         else k_bwd_delta<float, 128><<<grid, 256, 0, s>>>((const float*)Op, o_f32, (const float*)dOp, rows, delta);

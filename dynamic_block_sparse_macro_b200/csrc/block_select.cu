@@ -8,132 +8,184 @@
 // p (everything if p >= 1 or it never does), so S_i is the longer prefix,
 // max(min(k, n_blk), n_p) blocks.
 //
-// k_block_select     one CTA per (row, head): the row's (P, j) pairs packed
-//                    into 64-bit keys (P's bits are order-preserving since
-//                    P >= 0; ~j breaks ties towards smaller j), bitonic sort
-//                    in shared memory, block scan of the sorted probabilities,
-//                    bitmask of the first n entries.
-// k_select_transpose key-major copy of the bitmask for the backward pass.
+// k_block_select   one CTA per (row, head), no sort.  For P >= 0 the float bit
+//                  pattern orders like the value, so thresholds are found by
+//                  binary search over bit patterns with block reductions over
+//                  the row held in shared memory:
+//                    v* = largest t with sum{P_j : P_j >= t} >= p   (Top-p
+//                         crossing value; n_p = #{P > v*} + the fewest ties
+//                         at v* that reach p),
+//                    v_n = largest t with #{P_j >= t} >= n  (n-th value),
+//                  then S_i = {P > v_n} plus the lowest-index ties at v_n.
+//                  All reductions run in a fixed order (deterministic).
+// k_sel_expand     granule-level view of the selection for the attention
+//                  kernels; k_bit_transpose its key-major transpose.
 #include "common.cuh"
 
 namespace prism {
 
-constexpr int kSelectMaxRow = 16384;    // keys per row held in shared memory
+constexpr int kSelectThreads = 256;
+constexpr int kSelectMaxRow = 16384;    // P values of a row held in shared memory
 
-__device__ __forceinline__ float key_p(unsigned long long k) { return __uint_as_float((unsigned)(k >> 32)); }
-__device__ __forceinline__ int key_j(unsigned long long k) { return (int)(0xffffffffu - (unsigned)(k & 0xffffffffu)); }
+struct SelRed {
+    float f[kSelectThreads / 32];
+    int i[kSelectThreads / 32];
+};
 
-__global__ void __launch_bounds__(512) k_block_select(const float* __restrict__ P,
-                                                      const int32_t* __restrict__ n_blk, int64_t MB,
-                                                      int SW, int keycap, int top_k, float top_p,
-                                                      uint32_t* __restrict__ sel,
-                                                      int32_t* __restrict__ sel_count,
-                                                      float* __restrict__ margin,
-                                                      uint32_t* __restrict__ dev_status) {
-    extern __shared__ unsigned long long keys[];
-    __shared__ int s_first;
-    __shared__ float s_cat, s_cbef, s_tot;
-    __shared__ float wsum[16];
-    uint32_t* bits = reinterpret_cast<uint32_t*>(keys + keycap);   // SW words
+// fixed-order block reductions (every thread gets the result)
+__device__ __forceinline__ float sel_sum(float v, SelRed& r) {
+    v = warp_sum(v);
+    __syncthreads();
+    if ((threadIdx.x & 31) == 0) r.f[threadIdx.x >> 5] = v;
+    __syncthreads();
+    float s = 0.f;
+#pragma unroll
+    for (int w = 0; w < kSelectThreads / 32; ++w) s += r.f[w];
+    return s;
+}
+__device__ __forceinline__ int sel_count_i(int v, SelRed& r) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    __syncthreads();
+    if ((threadIdx.x & 31) == 0) r.i[threadIdx.x >> 5] = v;
+    __syncthreads();
+    int s = 0;
+#pragma unroll
+    for (int w = 0; w < kSelectThreads / 32; ++w) s += r.i[w];
+    return s;
+}
+__device__ __forceinline__ float sel_max(float v, SelRed& r) {
+    v = warp_max(v);
+    __syncthreads();
+    if ((threadIdx.x & 31) == 0) r.f[threadIdx.x >> 5] = v;
+    __syncthreads();
+    float s = r.f[0];
+#pragma unroll
+    for (int w = 1; w < kSelectThreads / 32; ++w) s = fmaxf(s, r.f[w]);
+    return s;
+}
 
-    const int i = blockIdx.x, hh = blockIdx.y, tid = threadIdx.x, nt = blockDim.x;
+__global__ void __launch_bounds__(kSelectThreads) k_block_select(const float* __restrict__ P,
+                                                                 const int32_t* __restrict__ n_blk, int64_t MB,
+                                                                 int SW, int top_k, float top_p,
+                                                                 uint32_t* __restrict__ sel,
+                                                                 int32_t* __restrict__ sel_count,
+                                                                 float* __restrict__ margin,
+                                                                 uint32_t* __restrict__ dev_status) {
+    extern __shared__ float row[];
+    __shared__ SelRed red;
+    const int i = blockIdx.x, hh = blockIdx.y, tid = threadIdx.x;
     const int nb = *n_blk;
     uint32_t* srow = sel + ((int64_t)hh * MB + i) * SW;
-    if (i >= nb || nb > keycap) {
-        for (int w = tid; w < SW; w += nt) srow[w] = 0u;
+    if (i >= nb || nb > kSelectMaxRow) {
+        for (int w = tid; w < SW; w += blockDim.x) srow[w] = 0u;
         if (tid == 0) {
             sel_count[(int64_t)hh * MB + i] = 0;
             if (margin) margin[(int64_t)hh * MB + i] = INFINITY;
-            if (nb > keycap && i == 0 && hh == 0) atomicOr(dev_status, PRISM_DEV_BAD_INDEX);
+            if (nb > kSelectMaxRow && i == 0 && hh == 0) atomicOr(dev_status, PRISM_DEV_BAD_INDEX);
         }
         return;
     }
-    int n2 = 1;
-    while (n2 < nb) n2 <<= 1;
     const float* prow = P + ((int64_t)hh * nb + i) * nb;
-    for (int j = tid; j < n2; j += nt)
-        keys[j] = j < nb ? (((unsigned long long)__float_as_uint(prow[j]) << 32) | (0xffffffffu - (unsigned)j))
-                         : 0ull;
-    for (int w = tid; w < SW; w += nt) bits[w] = 0u;
-    if (tid == 0) s_first = nb;
+    for (int j = tid; j < nb; j += blockDim.x) row[j] = prow[j];
     __syncthreads();
 
-    // bitonic sort, descending
-    for (int k = 2; k <= n2; k <<= 1) {
-        for (int j = k >> 1; j > 0; j >>= 1) {
-            for (int q = tid; q < (n2 >> 1); q += nt) {
-                const int a = 2 * j * (q / j) + (q % j), b = a + j;
-                const unsigned long long ka = keys[a], kb = keys[b];
-                const bool desc = (a & k) == 0;
-                if (desc ? (ka < kb) : (ka > kb)) { keys[a] = kb; keys[b] = ka; }
-            }
-            __syncthreads();
+    // sum and count of {P >= t}, {P > t}, {P == t} over the row
+    auto sum_ge = [&](uint32_t tb) {
+        float s = 0.f;
+        for (int j = tid; j < nb; j += blockDim.x) {
+            const float x = row[j];
+            if (__float_as_uint(x) >= tb) s += x;
         }
-    }
-
-    // cumulative sum in sorted order: contiguous segment per thread
-    const int L = (nb + nt - 1) / nt;
-    const int s0 = tid * L, s1 = min(nb, s0 + L);
-    float local = 0.f;
-    for (int q = s0; q < s1; ++q) local += key_p(keys[q]);
-    // exclusive scan of `local` over threads
-    const int lane = tid & 31, wid = tid >> 5;
-    float incl = local;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        float v = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += v;
-    }
-    if (lane == 31) wsum[wid] = incl;
-    __syncthreads();
-    float woff = 0.f;
-    for (int w = 0; w < wid; ++w) woff += wsum[w];
-    float c = woff + incl - local;
-    if (tid == nt - 1) s_tot = c + local;
-    bool found = false;
-    float cat = 0.f, cbef = 0.f;
-    int first = nb;
-    for (int q = s0; q < s1 && !found; ++q) {
-        const float prev = c;
-        c += key_p(keys[q]);
-        if (c >= top_p) { found = true; first = q; cat = c; cbef = prev; }
-    }
-    if (found) atomicMin(&s_first, first);
-    __syncthreads();
-    if (found && first == s_first) { s_cat = cat; s_cbef = cbef; }
-    __syncthreads();
+        return sel_sum(s, red);
+    };
+    auto count_ge = [&](uint32_t tb) {
+        int c = 0;
+        for (int j = tid; j < nb; j += blockDim.x) c += __float_as_uint(row[j]) >= tb;
+        return sel_count_i(c, red);
+    };
 
     const int n_k = min(top_k, nb);
-    int n_p;
+    int n_p = nb;
     float gap_p = INFINITY;
-    if (top_p >= 1.f) {
-        n_p = nb;
-    } else {
+    const float total = sum_ge(0u);
+    if (top_p < 1.f) {
         float c_at, c_before;
-        if (s_first < nb) {
-            n_p = s_first + 1;
-            c_at = s_cat;
-            c_before = n_p >= 2 ? s_cbef : -INFINITY;
-        } else {
+        if (total >= top_p) {
+            // largest bit pattern t with sum{P >= t} >= p: lo keeps the property, hi does not
+            uint32_t lo = 0u, hi = 0x3F800001u;                 // (1.0f bits) + 1
+            while (hi - lo > 1u) {
+                const uint32_t mid = lo + ((hi - lo) >> 1);
+                if (sum_ge(mid) >= top_p) lo = mid;
+                else hi = mid;
+            }
+            const float vstar = __uint_as_float(lo);
+            const float s_gt = sum_ge(lo + 1u);
+            const int c_gt = count_ge(lo + 1u), c_eq = count_ge(lo) - c_gt;
+            int m = c_eq;                                       // fewest ties at v* reaching p
+            if (vstar > 0.f) {
+                const float need = ceilf((top_p - s_gt) / vstar);
+                m = need < 1.f ? 1 : (need > (float)c_eq ? c_eq : (int)need);
+            }
+            n_p = c_gt + m;
+            c_at = s_gt + (float)m * vstar;
+            c_before = n_p >= 2 ? c_at - vstar : -INFINITY;
+        } else {                                                // the sum never reaches p: everything
             n_p = nb;
-            c_at = s_tot;
-            c_before = nb >= 2 ? s_tot - key_p(keys[nb - 1]) : -INFINITY;
+            c_at = total;
+            c_before = -INFINITY;                               // refined below if it matters
         }
         if (n_p >= n_k) gap_p = fminf(fabsf(c_at - top_p), fabsf(top_p - c_before));
     }
     const int n = max(n_k, n_p);
-    for (int q = tid; q < n; q += nt) {
-        const int j = key_j(keys[q]);
-        atomicOr(&bits[j >> 5], 1u << (j & 31));
+
+    // threshold of the first n entries of the order (P desc, j asc)
+    uint32_t vb = 0u;
+    int c_gt = 0, need_eq = n;
+    if (n < nb) {
+        uint32_t lo = 0u, hi = 0x3F800001u;                     // count{P >= lo} >= n > count{P >= hi}
+        while (hi - lo > 1u) {
+            const uint32_t mid = lo + ((hi - lo) >> 1);
+            if (count_ge(mid) >= n) lo = mid;
+            else hi = mid;
+        }
+        vb = lo;
+        c_gt = count_ge(lo + 1u);
+        need_eq = n - c_gt;
     }
-    __syncthreads();
-    for (int w = tid; w < SW; w += nt) srow[w] = bits[w];
+    // bitmask in index order (warp 0; a running count ranks ties by index)
+    if (tid < 32) {
+        int eq_seen = 0;
+        const int wn = (nb + 31) >> 5;
+        for (int w = 0; w < SW; ++w) {
+            uint32_t word = 0u;
+            if (w < wn) {
+                const int j = w * 32 + tid;
+                const uint32_t xb = j < nb ? __float_as_uint(row[j]) : 0u;
+                const bool in = j < nb;
+                const bool gt = in && (n >= nb || xb > vb);
+                const bool eq = in && n < nb && xb == vb;
+                const uint32_t eqmask = __ballot_sync(0xffffffffu, eq);
+                const int rank = eq_seen + __popc(eqmask & ((1u << tid) - 1u));
+                word = __ballot_sync(0xffffffffu, gt || (eq && rank < need_eq));
+                eq_seen += __popc(eqmask);
+            }
+            if (tid == 0) srow[w] = word;
+        }
+    }
+    // margins: order gap at the boundary, and the cumulative-sum gap
+    float gap_o = INFINITY;
+    if (n < nb) {
+        const int c_ge = count_ge(vb);
+        float below = -INFINITY;
+        for (int j = tid; j < nb; j += blockDim.x)
+            if (__float_as_uint(row[j]) < vb) below = fmaxf(below, row[j]);
+        below = sel_max(below, red);
+        gap_o = c_ge > n ? 0.f : __uint_as_float(vb) - below;
+    }
     if (tid == 0) {
         sel_count[(int64_t)hh * MB + i] = n;
-        if (margin) {
-            const float gap_o = n < nb ? key_p(keys[n - 1]) - key_p(keys[n]) : INFINITY;
-            margin[(int64_t)hh * MB + i] = fminf(gap_o, gap_p);
-        }
+        if (margin) margin[(int64_t)hh * MB + i] = fminf(gap_o, gap_p);
     }
 }
 
@@ -146,10 +198,10 @@ __global__ void __launch_bounds__(128) k_sel_expand(const uint32_t* __restrict__
                                                     const int32_t* __restrict__ gran_blk,
                                                     const int32_t* __restrict__ n_blk, int64_t MB, int SW,
                                                     uint32_t* __restrict__ gsel) {
-    extern __shared__ uint32_t row[];
+    extern __shared__ uint32_t gwords[];
     const int qg = blockIdx.x, hh = blockIdx.y;
     const int nb = *n_blk;
-    for (int w = threadIdx.x; w < SW; w += blockDim.x) row[w] = 0u;
+    for (int w = threadIdx.x; w < SW; w += blockDim.x) gwords[w] = 0u;
     __syncthreads();
     const int i = gran_blk[qg];
     if (i >= 0 && i < nb) {
@@ -161,13 +213,13 @@ __global__ void __launch_bounds__(128) k_sel_expand(const uint32_t* __restrict__
                 const int j = w * 32 + __ffs(b) - 1;
                 b &= b - 1;
                 const int g0 = blk_start[j] >> 6, g1 = blk_start[j + 1] >> 6;   // granules [g0, g1)
-                for (int g = g0; g < g1; ++g) atomicOr(&row[g >> 5], 1u << (g & 31));
+                for (int g = g0; g < g1; ++g) atomicOr(&gwords[g >> 5], 1u << (g & 31));
             }
         }
     }
     __syncthreads();
     uint32_t* out = gsel + ((int64_t)hh * MB + qg) * SW;
-    for (int w = threadIdx.x; w < SW; w += blockDim.x) out[w] = row[w];
+    for (int w = threadIdx.x; w < SW; w += blockDim.x) out[w] = gwords[w];
 }
 
 // Bit-matrix transpose, one warp per 32x32 tile: lane l holds row (32 rt + l)
@@ -191,16 +243,6 @@ __global__ void __launch_bounds__(256) k_bit_transpose(const uint32_t* __restric
     if (orow < MB) out[((int64_t)hh * MB + orow) * SW + rt] = mine;
 }
 
-int select_keycap(const Dims& d) {
-    int cap = 1;
-    while (cap < d.MB && cap < kSelectMaxRow) cap <<= 1;
-    return cap;
-}
-
-size_t select_smem_bytes(const Dims& d) {
-    return (size_t)select_keycap(d) * 8 + (size_t)d.SW * 4;
-}
-
 }  // namespace prism
 
 using namespace prism;
@@ -218,13 +260,13 @@ extern "C" prism_status_t prism_block_select(const prism_problem_t* prob, const 
         !ok_ptr(sel_count) || !ok_ptr(gsel) || !ok_opt(gselT) || !ok_opt(margin) || !ok_ptr(dev_status))
         return PRISM_ERR_INVALID_ARG;
     if (top_k < 1 || !(top_p > 0.f) || !isfinite(top_p)) return PRISM_ERR_INVALID_ARG;
-    size_t smem = select_smem_bytes(d);
-    if (smem > 227 * 1024) return PRISM_ERR_UNSUPPORTED;
+    const int64_t rowcap = d.MB < kSelectMaxRow ? d.MB : kSelectMaxRow;
+    const size_t smem = (size_t)rowcap * sizeof(float);
     if (cudaFuncSetAttribute(k_block_select, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
         cudaSuccess)
         return PRISM_ERR_CUDA;
-    k_block_select<<<dim3((unsigned)d.MB, (unsigned)d.heads), 512, smem, stream>>>(
-        P, n_blk, d.MB, (int)d.SW, select_keycap(d), top_k, top_p, sel, sel_count, margin, dev_status);
+    k_block_select<<<dim3((unsigned)d.MB, (unsigned)d.heads), kSelectThreads, smem, stream>>>(
+        P, n_blk, d.MB, (int)d.SW, top_k, top_p, sel, sel_count, margin, dev_status);
     k_sel_expand<<<dim3((unsigned)d.MB, (unsigned)d.heads), 128, (size_t)d.SW * 4, stream>>>(
         sel, blk_start, gran_blk, n_blk, d.MB, (int)d.SW, gsel);
     if (gselT)
