@@ -19,8 +19,10 @@
 //                     in TMEM, dV += P^T dO and dK += dS^T Q.
 // Both double-buffer the granule products in TMEM so that the tensor core
 // works on granule g+1 while four warps do the elementwise step of granule g,
-// and stream granules through a 3-stage TMA ring.  Roles: warp 0 TMA, warp 1
-// TMEM allocation + MMA issue (one thread), warps 2-5 one tile row per thread.
+// and stream granules through a TMA ring as deep as shared memory allows.
+// Roles: warp 0 TMA (one lane per ring stage and stream, one whole-row copy
+// per granule), warp 1 TMEM allocation + MMA issue (the whole warp, one
+// elected lane issues), warps 2-5 one tile row per thread.
 // Every wait is bounded; a timeout sets PRISM_DEV_TIMEOUT.
 #include "attn_plan.cuh"
 #include "common.cuh"
@@ -31,16 +33,21 @@ namespace prism {
 using namespace sm100;
 
 prism_status_t bwd_delta(const Dims& d, const void* Op, const float* o_f32, const void* dOp, float* delta,
-                         cudaStream_t s);
+                         const float* lse, float* nld, cudaStream_t s);
 
 namespace {
 
 constexpr int kTile = 128 * 128;           // bytes: 128 rows x 64 bf16 columns
 constexpr int kGran = 64 * 128;            // bytes: 64 rows x 64 bf16 columns
-constexpr int kStages = 3;
+constexpr int kStages = 6;                 // barrier slots; the ring uses nst <= kStages of them
+constexpr int kXs = 512;                   // per stage (dK/dV only): -lse*log2(e) and -Delta of 64 query rows
 constexpr uint32_t kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr int kSmemMax = 227 * 1024;
 
+// Shared memory: stationary tiles, then a ring of nst granule stages (as many
+// as fit: the TMA latency under load is about 4000 cycles, a granule's MMAs
+// take about 800), then barriers and the two selection rows.
 template <int D>
 struct BwdLayout {
     static constexpr int NR = D / 64;
@@ -48,14 +55,23 @@ struct BwdLayout {
     static constexpr int A1 = NR * kTile;              // stationary operand 2 (dO or V)
     static constexpr int RING = 2 * NR * kTile;        // streamed granules
     static constexpr int STAGE = 2 * NR * kGran;       // two operands per stage
-    static constexpr int CTRL = RING + kStages * STAGE;
-    static constexpr int ROWS = CTRL + 256;            // two selection rows of SW words follow
-    static int alloc(int SW) { return ROWS + 8 * SW + 1024; }
+    // xs: bytes of per-granule row data staged beside each stage (0 or kXs)
+    __host__ __device__ static int xs(int nst) { return RING + nst * STAGE; }
+    __host__ __device__ static int ctrl(int nst, int xsb) { return xs(nst) + nst * xsb; }
+    __host__ __device__ static int rows(int nst, int xsb) { return ctrl(nst, xsb) + 256; }
+    static int alloc(int nst, int xsb, int SW) { return rows(nst, xsb) + 8 * SW + 1024; }
+    static int stages(int xsb, int SW) {               // deepest ring that fits, at least 2
+        int n = kStages;
+        while (n > 2 && alloc(n, xsb, SW) > kSmemMax) --n;
+        return n;
+    }
 };
 
 struct Bars {
-    uint64_t* stat;            // stationary tiles landed
-    uint64_t* full;            // [kStages] streamed granule landed
+    uint64_t* stat;            // stationary tiles landed (one arrival per producer)
+    uint64_t* full0;           // [kStages] streamed operand 0 of a granule landed
+    uint64_t* full1;           // [kStages] streamed operand 1 of a granule landed
+    uint64_t* fullx;           // [kStages] row data of a granule landed (dK/dV only)
     uint64_t* empty;           // [kStages] granule stage free
     uint64_t* prod;            // [2] products of a granule in TMEM
     uint64_t* elem;            // [2] elementwise results of a granule in TMEM (128 arrivals)
@@ -69,21 +85,26 @@ __device__ __forceinline__ Bars carve(uint8_t* ctrl) {
     uint64_t* b = reinterpret_cast<uint64_t*>(ctrl);
     Bars r;
     r.stat = b;
-    r.full = b + 1;
-    r.empty = b + 1 + kStages;
-    r.prod = b + 1 + 2 * kStages;
-    r.elem = b + 3 + 2 * kStages;
-    r.fin = b + 5 + 2 * kStages;
-    r.tmem_slot = reinterpret_cast<uint32_t*>(b + 6 + 2 * kStages);
+    r.full0 = b + 1;
+    r.full1 = b + 1 + kStages;
+    r.fullx = b + 1 + 2 * kStages;
+    r.empty = b + 1 + 3 * kStages;
+    r.prod = b + 1 + 4 * kStages;
+    r.elem = b + 3 + 4 * kStages;
+    r.fin = b + 5 + 4 * kStages;
+    r.tmem_slot = reinterpret_cast<uint32_t*>(b + 6 + 4 * kStages);
     r.abort_flag = reinterpret_cast<volatile int*>(r.tmem_slot + 1);
     r.ng_slot = reinterpret_cast<int*>(r.tmem_slot + 2);
     return r;
 }
+static_assert((6 + 4 * kStages) * 8 + 12 <= 256, "barriers overflow the control block");
 
-__device__ __forceinline__ void init_bars(const Bars& B) {
-    mbar_init(B.stat, 1);
-    for (int s = 0; s < kStages; ++s) {
-        mbar_init(B.full + s, 1);
+__device__ __forceinline__ void init_bars(const Bars& B, int nst) {
+    mbar_init(B.stat, 2);
+    for (int s = 0; s < nst; ++s) {
+        mbar_init(B.full0 + s, 1);
+        mbar_init(B.full1 + s, 1);
+        mbar_init(B.fullx + s, 1);
         mbar_init(B.empty + s, 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -98,41 +119,53 @@ __device__ __forceinline__ void init_bars(const Bars& B) {
 // descriptor offsets: K-major operand, k-th 16-element step of the contraction over d
 __device__ __forceinline__ uint32_t kmaj_off(int k, int region) { return (k >> 2) * region + (k & 3) * 32; }
 
-// TMA producer shared by both kernels: stationary tiles once, then the
-// granule stream of the walk (two operands per granule).
+// The TMA producer warp.  A copy engine completes the copies issued by one
+// thread one after another, so every (ring stage, stream) pair gets a lane of
+// its own: lane kind * nst + stage issues stream `kind` (0: operand 0, 1:
+// operand 1, 2: the 512 bytes of row data, dK/dV only) of the granules that
+// use that stage, one copy per granule, and never has more than one copy in
+// flight.  Lanes 0 and nst also copy the two stationary tiles.
 template <int D>
-__device__ void produce(const CUtensorMap* m0, const CUtensorMap* m1, const CUtensorMap* g0,
-                        const CUtensorMap* g1, uint8_t* sm, const Bars& B, int64_t row0, int tile_row,
-                        GranuleWalk& walk, int ng, uint32_t* dev_status) {
+__device__ void produce(const CUtensorMap* m0, const CUtensorMap* m1, const CUtensorMap* g0, const CUtensorMap* g1,
+                        const float* nld, uint8_t* xs, uint8_t* sm, const Bars& B, int64_t row0, int tile_row,
+                        const uint32_t* u0, const uint32_t* u1, int wn, int g_begin, int ng, int nst,
+                        uint32_t* dev_status) {
     using L = BwdLayout<D>;
-    tma_prefetch_desc(m0);
-    tma_prefetch_desc(m1);
-    tma_prefetch_desc(g0);
-    tma_prefetch_desc(g1);
-    mbar_expect_tx(B.stat, 2 * L::NR * kTile);
-    for (int r = 0; r < L::NR; ++r) {
-        tma_load_2d(sm + L::A0 + r * kTile, m0, B.stat, 64 * r, (int)(row0 + tile_row));
-        tma_load_2d(sm + L::A1 + r * kTile, m1, B.stat, 64 * r, (int)(row0 + tile_row));
+    const int lane = threadIdx.x & 31;
+    if (lane >= (nld ? 3 : 2) * nst) return;
+    const int kind = lane / nst, stage = lane % nst;
+    uint64_t* full = kind == 0 ? B.full0 : kind == 1 ? B.full1 : B.fullx;
+    const CUtensorMap* mg = kind == 0 ? g0 : g1;
+    if (kind < 2) tma_prefetch_desc(mg);
+    if (stage == 0 && kind < 2) {
+        const CUtensorMap* ms = kind == 0 ? m0 : m1;
+        mbar_expect_tx(B.stat, L::NR * kTile);
+        tma_load_3d(sm + (kind ? L::A1 : L::A0), ms, B.stat, 0, (int)(row0 + tile_row), 0);
     }
-    int issued = 0;
+    GranuleWalk walk;
+    walk.init(u0, u1, wn);
+    walk.skip(g_begin);
+    int last = -1;
     for (int g = 0; g < ng && !*B.abort_flag; ++g) {
         int row;
         uint32_t m;
         walk.next(row, m);
-        const int s = g % kStages;
-        if (g >= kStages && !mbar_wait(B.empty + s, ((g / kStages) - 1) & 1, B.abort_flag, dev_status)) break;
-        uint8_t* st = sm + L::RING + s * L::STAGE;
-        mbar_expect_tx(B.full + s, L::STAGE);
-        for (int r = 0; r < L::NR; ++r) {
-            tma_load_2d(st + r * kGran, g0, B.full + s, 64 * r, (int)(row0 + row));
-            tma_load_2d(st + (L::NR + r) * kGran, g1, B.full + s, 64 * r, (int)(row0 + row));
+        if (g % nst != stage) continue;
+        if (g >= nst && !mbar_wait(B.empty + stage, ((g / nst) - 1) & 1, B.abort_flag, dev_status)) break;
+        if (kind == 2) {
+            mbar_expect_tx(full + stage, kXs);
+            bulk_load(xs + stage * kXs, nld + ((row0 + row) >> 6) * 128, kXs, full + stage);
+        } else {
+            mbar_expect_tx(full + stage, L::NR * kGran);
+            tma_load_3d(sm + L::RING + stage * L::STAGE + kind * L::NR * kGran, mg, full + stage, 0,
+                        (int)(row0 + row), 0);
         }
-        ++issued;
+        last = g;
     }
-    if (*B.abort_flag) {
+    if (*B.abort_flag && last >= 0) {
+        // let this lane's copy land before the CTA goes away
         volatile int no_abort = 0;
-        for (int g = (issued > kStages ? issued - kStages : 0); g < issued; ++g)
-            mbar_wait(B.full + g % kStages, (g / kStages) & 1, &no_abort, dev_status);
+        mbar_wait(full + stage, (last / nst) & 1, &no_abort, dev_status);
     }
 }
 
@@ -143,7 +176,7 @@ k_bwd_dq_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                const uint32_t* __restrict__ gsel, const PlanHeader* __restrict__ hdr,
                const int4* __restrict__ items, float* __restrict__ part, const float* __restrict__ lse,
-               const float* __restrict__ delta, int64_t N, int64_t MB, int SW, float scale,
+               const float* __restrict__ delta, int64_t N, int64_t MB, int SW, int nst, float scale,
                __nv_bfloat16* __restrict__ dQ, uint32_t* __restrict__ dev_status) {
     using L = BwdLayout<D>;
     constexpr uint32_t cdQ = 0, cS = 128, cP = 192;   // + 128 * buffer for S / dP
@@ -154,15 +187,15 @@ k_bwd_dq_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     const int g_begin = item.y, ng = item.z - item.y, slot = item.w;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    Bars B = carve(sm + L::CTRL);
-    uint32_t* u0 = reinterpret_cast<uint32_t*>(sm + L::ROWS);
+    Bars B = carve(sm + L::ctrl(nst, 0));
+    uint32_t* u0 = reinterpret_cast<uint32_t*>(sm + L::rows(nst, 0));
     uint32_t* u1 = u0 + SW;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int wn = SW;
     const int64_t row0 = (int64_t)hh * N;
 
     load_rows(u0, u1, gsel + ((int64_t)hh * MB + 2 * tile) * SW, gsel + ((int64_t)hh * MB + 2 * tile + 1) * SW, wn);
-    if (threadIdx.x == 0) init_bars(B);
+    if (threadIdx.x == 0) init_bars(B, nst);
     if (warp == 1) {
         tmem_alloc(B.tmem_slot, kTmemCols);
         tmem_relinquish();
@@ -173,48 +206,46 @@ k_bwd_dq_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     const uint32_t tb = *B.tmem_slot;
 
     if (warp == 0) {
-        if (lane == 0) {
-            GranuleWalk walk;
-            walk.init(u0, u1, wn);
-            walk.skip(g_begin);
-            produce<D>(&tmQ, &tmdO, &tmK, &tmV, sm, B, row0, 128 * tile, walk, ng, dev_status);
-        }
+        produce<D>(&tmQ, &tmdO, &tmK, &tmV, nullptr, nullptr, sm, B, row0, 128 * tile, u0, u1, wn, g_begin, ng, nst,
+                   dev_status);
     } else if (warp == 1) {
-        if (lane == 0) {
+        {   // the whole warp, converged; one elected lane issues
             const uint32_t idPS = idesc_bf16_f32(128, 64, false, false);
             const uint32_t idQ = idesc_bf16_f32(128, D, false, true);
             const uint32_t aQ = smem_u32(sm + L::A0), adO = smem_u32(sm + L::A1), aR = smem_u32(sm + L::RING);
-            bool ok = mbar_wait(B.stat, 0, B.abort_flag, dev_status);
+            bool ok = mbar_wait_w(B.stat, 0, B.abort_flag, dev_status);
             tc_fence_after();
             for (int g = 0; ok && g <= ng; ++g) {
                 if (g < ng) {
-                    const int s = g % kStages, b = g & 1;
-                    if (!mbar_wait(B.full + s, (g / kStages) & 1, B.abort_flag, dev_status)) break;
+                    const int s = g % nst, b = g & 1;
+                    if (!mbar_wait_w(B.full0 + s, (g / nst) & 1, B.abort_flag, dev_status) ||
+                        !mbar_wait_w(B.full1 + s, (g / nst) & 1, B.abort_flag, dev_status))
+                        break;
                     tc_fence_after();
                     const uint32_t aK = aR + s * L::STAGE, aV = aK + L::NR * kGran;
 #pragma unroll
                     for (int k = 0; k < D / 16; ++k)
-                        mma_ss(tb + cS + 128 * b, sdesc_sw128(aQ + kmaj_off(k, kTile), 16, 1024),
-                               sdesc_sw128(aK + kmaj_off(k, kGran), 16, 1024), idPS, k > 0);
+                        mma_ss_w(tb + cS + 128 * b, sdesc_sw128(aQ + kmaj_off(k, kTile), 16, 1024),
+                                 sdesc_sw128(aK + kmaj_off(k, kGran), 16, 1024), idPS, k > 0);
 #pragma unroll
                     for (int k = 0; k < D / 16; ++k)
-                        mma_ss(tb + cP + 128 * b, sdesc_sw128(adO + kmaj_off(k, kTile), 16, 1024),
-                               sdesc_sw128(aV + kmaj_off(k, kGran), 16, 1024), idPS, k > 0);
-                    tc_commit(B.prod + b);
+                        mma_ss_w(tb + cP + 128 * b, sdesc_sw128(adO + kmaj_off(k, kTile), 16, 1024),
+                                 sdesc_sw128(aV + kmaj_off(k, kGran), 16, 1024), idPS, k > 0);
+                    tc_commit_w(B.prod + b);
                 }
                 if (g > 0) {
-                    const int gp = g - 1, s = gp % kStages, b = gp & 1;
-                    if (!mbar_wait(B.elem + b, (gp >> 1) & 1, B.abort_flag, dev_status)) break;
+                    const int gp = g - 1, s = gp % nst, b = gp & 1;
+                    if (!mbar_wait_w(B.elem + b, (gp >> 1) & 1, B.abort_flag, dev_status)) break;
                     tc_fence_after();
                     const uint32_t aK = aR + s * L::STAGE;
 #pragma unroll
                     for (int k = 0; k < 4; ++k)
-                        mma_ts(tb + cdQ, tb + cS + 128 * b + 8 * k, sdesc_sw128(aK + k * 2048, kGran, 1024), idQ,
-                               (gp > 0 || k > 0) ? 1u : 0u);
-                    tc_commit(B.empty + s);
+                        mma_ts_w(tb + cdQ, tb + cS + 128 * b + 8 * k, sdesc_sw128(aK + k * 2048, kGran, 1024), idQ,
+                                 (gp > 0 || k > 0) ? 1u : 0u);
+                    tc_commit_w(B.empty + s);
                 }
             }
-            tc_commit(B.fin);
+            tc_commit_w(B.fin);
             if (*B.abort_flag) {
                 volatile int no_abort = 0;
                 mbar_wait(B.fin, 0, &no_abort, dev_status);
@@ -245,14 +276,21 @@ k_bwd_dq_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             const bool got = mbar_wait(B.prod + b, (g >> 1) & 1, B.abort_flag, dev_status);
             if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
             tc_fence_after();
+            // S and dP of the granule: all TMEM loads in flight before one wait
+            uint32_t sv[2][32], pv[2][32];
+            if (valid) {
+                tmem_ld32(tl + cS + 128 * b, sv[0]);
+                tmem_ld32(tl + cP + 128 * b, pv[0]);
+                tmem_ld32(tl + cS + 128 * b + 32, sv[1]);
+                tmem_ld32(tl + cP + 128 * b + 32, pv[1]);
+                tmem_wait_ld();
+            }
 #pragma unroll
             for (int hq = 0; hq < 2; ++hq) {
                 uint32_t o[16];
                 if (valid) {
-                    uint32_t s[32], p[32];
-                    tmem_ld32(tl + cS + 128 * b + 32 * hq, s);
-                    tmem_ld32(tl + cP + 128 * b + 32 * hq, p);
-                    tmem_wait_ld();
+                    const uint32_t (&s)[32] = sv[hq];
+                    const uint32_t (&p)[32] = pv[hq];
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
                         float x0, x1;
@@ -317,9 +355,8 @@ __global__ void __launch_bounds__(192, 1)
 k_bwd_dkdv_sm100(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                  const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmdO,
                  const uint32_t* __restrict__ gselT, const PlanHeader* __restrict__ hdr,
-                 const int4* __restrict__ items, float* __restrict__ part, const float* __restrict__ lse,
-                 const float* __restrict__ delta, int64_t N, int64_t MB, int SW, float scale,
-                 __nv_bfloat16* __restrict__ dK, __nv_bfloat16* __restrict__ dV,
+                 const int4* __restrict__ items, float* __restrict__ part, const float* __restrict__ nld,
+                 int64_t N, int64_t MB, int SW, int nst, float scale, __nv_bfloat16* __restrict__ dK, __nv_bfloat16* __restrict__ dV,
                  uint32_t* __restrict__ dev_status) {
     using L = BwdLayout<D>;
     constexpr uint32_t cdK = 0, cdV = 128, cS = 256, cP = 320;   // + 128 * buffer for S^T / dP^T
@@ -330,15 +367,16 @@ k_bwd_dkdv_sm100(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
     const int g_begin = item.y, ng = item.z - item.y, slot = item.w;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    Bars B = carve(sm + L::CTRL);
-    uint32_t* u0 = reinterpret_cast<uint32_t*>(sm + L::ROWS);
+    Bars B = carve(sm + L::ctrl(nst, kXs));
+    uint8_t* xs = sm + L::xs(nst);
+    uint32_t* u0 = reinterpret_cast<uint32_t*>(sm + L::rows(nst, kXs));
     uint32_t* u1 = u0 + SW;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int wn = SW;
     const int64_t row0 = (int64_t)hh * N;
 
     load_rows(u0, u1, gselT + ((int64_t)hh * MB + 2 * tile) * SW, gselT + ((int64_t)hh * MB + 2 * tile + 1) * SW, wn);
-    if (threadIdx.x == 0) init_bars(B);
+    if (threadIdx.x == 0) init_bars(B, nst);
     if (warp == 1) {
         tmem_alloc(B.tmem_slot, kTmemCols);
         tmem_relinquish();
@@ -349,52 +387,50 @@ k_bwd_dkdv_sm100(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
     const uint32_t tb = *B.tmem_slot;
 
     if (warp == 0) {
-        if (lane == 0) {
-            GranuleWalk walk;
-            walk.init(u0, u1, wn);
-            walk.skip(g_begin);
-            produce<D>(&tmK, &tmV, &tmQ, &tmdO, sm, B, row0, 128 * tile, walk, ng, dev_status);
-        }
+        produce<D>(&tmK, &tmV, &tmQ, &tmdO, nld, xs, sm, B, row0, 128 * tile, u0, u1, wn, g_begin, ng, nst,
+                   dev_status);
     } else if (warp == 1) {
-        if (lane == 0) {
+        {   // the whole warp, converged; one elected lane issues
             const uint32_t idPS = idesc_bf16_f32(128, 64, false, false);
             const uint32_t idKV = idesc_bf16_f32(128, D, false, true);
             const uint32_t aK = smem_u32(sm + L::A0), aV = smem_u32(sm + L::A1), aR = smem_u32(sm + L::RING);
-            bool ok = mbar_wait(B.stat, 0, B.abort_flag, dev_status);
+            bool ok = mbar_wait_w(B.stat, 0, B.abort_flag, dev_status);
             tc_fence_after();
             for (int g = 0; ok && g <= ng; ++g) {
                 if (g < ng) {
-                    const int s = g % kStages, b = g & 1;
-                    if (!mbar_wait(B.full + s, (g / kStages) & 1, B.abort_flag, dev_status)) break;
+                    const int s = g % nst, b = g & 1;
+                    if (!mbar_wait_w(B.full0 + s, (g / nst) & 1, B.abort_flag, dev_status) ||
+                        !mbar_wait_w(B.full1 + s, (g / nst) & 1, B.abort_flag, dev_status))
+                        break;
                     tc_fence_after();
                     const uint32_t aQ = aR + s * L::STAGE, adO = aQ + L::NR * kGran;
 #pragma unroll
                     for (int k = 0; k < D / 16; ++k)
-                        mma_ss(tb + cS + 128 * b, sdesc_sw128(aK + kmaj_off(k, kTile), 16, 1024),
-                               sdesc_sw128(aQ + kmaj_off(k, kGran), 16, 1024), idPS, k > 0);
+                        mma_ss_w(tb + cS + 128 * b, sdesc_sw128(aK + kmaj_off(k, kTile), 16, 1024),
+                                 sdesc_sw128(aQ + kmaj_off(k, kGran), 16, 1024), idPS, k > 0);
 #pragma unroll
                     for (int k = 0; k < D / 16; ++k)
-                        mma_ss(tb + cP + 128 * b, sdesc_sw128(aV + kmaj_off(k, kTile), 16, 1024),
-                               sdesc_sw128(adO + kmaj_off(k, kGran), 16, 1024), idPS, k > 0);
-                    tc_commit(B.prod + b);
+                        mma_ss_w(tb + cP + 128 * b, sdesc_sw128(aV + kmaj_off(k, kTile), 16, 1024),
+                                 sdesc_sw128(adO + kmaj_off(k, kGran), 16, 1024), idPS, k > 0);
+                    tc_commit_w(B.prod + b);
                 }
                 if (g > 0) {
-                    const int gp = g - 1, s = gp % kStages, b = gp & 1;
-                    if (!mbar_wait(B.elem + b, (gp >> 1) & 1, B.abort_flag, dev_status)) break;
+                    const int gp = g - 1, s = gp % nst, b = gp & 1;
+                    if (!mbar_wait_w(B.elem + b, (gp >> 1) & 1, B.abort_flag, dev_status)) break;
                     tc_fence_after();
                     const uint32_t aQ = aR + s * L::STAGE, adO = aQ + L::NR * kGran;
 #pragma unroll
                     for (int k = 0; k < 4; ++k) {
                         const uint32_t acc = (gp > 0 || k > 0) ? 1u : 0u;
-                        mma_ts(tb + cdV, tb + cS + 128 * b + 8 * k, sdesc_sw128(adO + k * 2048, kGran, 1024), idKV,
-                               acc);
-                        mma_ts(tb + cdK, tb + cP + 128 * b + 8 * k, sdesc_sw128(aQ + k * 2048, kGran, 1024), idKV,
-                               acc);
+                        mma_ts_w(tb + cdV, tb + cS + 128 * b + 8 * k, sdesc_sw128(adO + k * 2048, kGran, 1024), idKV,
+                                 acc);
+                        mma_ts_w(tb + cdK, tb + cP + 128 * b + 8 * k, sdesc_sw128(aQ + k * 2048, kGran, 1024), idKV,
+                                 acc);
                     }
-                    tc_commit(B.empty + s);
+                    tc_commit_w(B.empty + s);
                 }
             }
-            tc_commit(B.fin);
+            tc_commit_w(B.fin);
             if (*B.abort_flag) {
                 volatile int no_abort = 0;
                 mbar_wait(B.fin, 0, &no_abort, dev_status);
@@ -404,7 +440,7 @@ k_bwd_dkdv_sm100(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
         const int sub = warp & 3, row = sub * 32 + lane, half = row >> 6;
         const uint32_t tl = tb + ((uint32_t)(sub * 32) << 16);
         const float sl2 = scale * kLog2e;
-        const uint64_t sl2x2 = f2pack(sl2, sl2), nlog2e = f2pack(-kLog2e, -kLog2e), neg1 = f2pack(-1.f, -1.f);
+        const uint64_t sl2x2 = f2pack(sl2, sl2);
         GranuleWalk walk;
         if (lane == 0) {
             walk.init(u0, u1, wn);
@@ -412,35 +448,42 @@ k_bwd_dkdv_sm100(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
         }
         bool ok = true;
         for (int g = 0; g < ng; ++g) {
-            const int b = g & 1;
+            const int b = g & 1, st = g % nst;
             uint32_t mk = 0;
             int qrow = 0;
             if (lane == 0) walk.next(qrow, mk);
             mk = __shfl_sync(0xffffffffu, mk, 0);
-            qrow = __shfl_sync(0xffffffffu, qrow, 0);
             const bool valid = (mk >> half) & 1u;              // warp-uniform
-            const float4* lse4 = reinterpret_cast<const float4*>(lse + row0 + qrow);
-            const float4* del4 = reinterpret_cast<const float4*>(delta + row0 + qrow);
-            const bool got = mbar_wait(B.prod + b, (g >> 1) & 1, B.abort_flag, dev_status);
+            const float4* nl4 = reinterpret_cast<const float4*>(xs + st * kXs);   // -lse*log2(e), 64 rows
+            const float4* nd4 = nl4 + 16;                                          // -Delta, 64 rows
+            const bool got = mbar_wait(B.prod + b, (g >> 1) & 1, B.abort_flag, dev_status) &&
+                             mbar_wait(B.fullx + st, (g / nst) & 1, B.abort_flag, dev_status);
             if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
             tc_fence_after();
+            // S^T and dP^T of the granule: all TMEM loads in flight before one wait
+            uint32_t sv[2][32], pv[2][32];
+            if (valid) {
+                tmem_ld32(tl + cS + 128 * b, sv[0]);
+                tmem_ld32(tl + cP + 128 * b, pv[0]);
+                tmem_ld32(tl + cS + 128 * b + 32, sv[1]);
+                tmem_ld32(tl + cP + 128 * b + 32, pv[1]);
+                tmem_wait_ld();
+            }
 #pragma unroll
             for (int hq = 0; hq < 2; ++hq) {
                 uint32_t op[16], od[16];
                 if (valid) {
-                    uint32_t s[32], p[32];
-                    tmem_ld32(tl + cS + 128 * b + 32 * hq, s);
-                    tmem_ld32(tl + cP + 128 * b + 32 * hq, p);
-                    tmem_wait_ld();
+                    const uint32_t (&s)[32] = sv[hq];
+                    const uint32_t (&p)[32] = pv[hq];
 #pragma unroll
                     for (int i4 = 0; i4 < 8; ++i4) {
-                        const float4 l4 = __ldg(lse4 + 8 * hq + i4);
-                        const float4 d4 = __ldg(del4 + 8 * hq + i4);
+                        const float4 l4 = nl4[8 * hq + i4];
+                        const float4 d4 = nd4[8 * hq + i4];
 #pragma unroll
                         for (int u = 0; u < 2; ++u) {
                             const int i = 4 * i4 + 2 * u;
-                            const uint64_t nl = fmul2(u ? f2pack(l4.z, l4.w) : f2pack(l4.x, l4.y), nlog2e);
-                            const uint64_t nd = fmul2(u ? f2pack(d4.z, d4.w) : f2pack(d4.x, d4.y), neg1);
+                            const uint64_t nl = u ? f2pack(l4.z, l4.w) : f2pack(l4.x, l4.y);
+                            const uint64_t nd = u ? f2pack(d4.z, d4.w) : f2pack(d4.x, d4.y);
                             float x0, x1;
                             f2unpack(ffma2(f2pack(__uint_as_float(s[i]), __uint_as_float(s[i + 1])), sl2x2, nl), x0, x1);
                             const float p0 = ex2(x0), p1 = ex2(x1);
@@ -510,6 +553,7 @@ k_bwd_dkdv_sm100(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
 // ------------------------------------------------------------------ host side
 struct BwdWs {
     float* delta;
+    float* nld;         // [heads*N/64][128]: per 64-row granule -lse*log2(e), then -Delta
     Plan pq, pkv;
     float* part_q;      // [slots][128][D]
     float* part_kv;     // [slots][2][128][D]
@@ -523,6 +567,8 @@ BwdWs carve_bwd(void* ws, const Dims& d, size_t* total) {
     BwdWs w;
     w.delta = reinterpret_cast<float*>(p);
     p += align16((int64_t)d.heads * d.N * 4);
+    w.nld = reinterpret_cast<float*>(p);
+    p += align16((int64_t)d.heads * d.N * 8);
     w.pq = carve_plan(p, tiles, target);
     p += plan_bytes(tiles, target);
     w.pkv = carve_plan(p, tiles, target);
@@ -541,27 +587,29 @@ prism_status_t launch_bwd(const Dims& d, const void* Qp, const void* Kp, const v
                           void* dKp, void* dVp, uint32_t* dev_status, const BwdWs& w, cudaStream_t s) {
     const int64_t rows = (int64_t)d.heads * d.N;
     CUtensorMap tQ, tdO, tK, tV, gQ, gdO, gK, gV;
-    if (!make_map_bf16(&tQ, Qp, rows, D, 128) || !make_map_bf16(&tdO, dOp, rows, D, 128) ||
-        !make_map_bf16(&tK, Kp, rows, D, 128) || !make_map_bf16(&tV, Vp, rows, D, 128) ||
-        !make_map_bf16(&gQ, Qp, rows, D, 64) || !make_map_bf16(&gdO, dOp, rows, D, 64) ||
-        !make_map_bf16(&gK, Kp, rows, D, 64) || !make_map_bf16(&gV, Vp, rows, D, 64))
+    if (!make_map_bf16_rows(&tQ, Qp, rows, D, 128) || !make_map_bf16_rows(&tdO, dOp, rows, D, 128) ||
+        !make_map_bf16_rows(&tK, Kp, rows, D, 128) || !make_map_bf16_rows(&tV, Vp, rows, D, 128) ||
+        !make_map_bf16_rows(&gQ, Qp, rows, D, 64) || !make_map_bf16_rows(&gdO, dOp, rows, D, 64) ||
+        !make_map_bf16_rows(&gK, Kp, rows, D, 64) || !make_map_bf16_rows(&gV, Vp, rows, D, 64))
         return PRISM_ERR_CUDA;
     const int target = plan_target(device_sms());
-    prism_status_t st = plan_work(w.pq, gsel, d, 1, target, kSegMinGranules, s);
-    if (st == PRISM_OK) st = plan_work(w.pkv, gselT, d, 1, target, kSegMinGranules, s);
+    prism_status_t st = plan_work(w.pq, gsel, d, 2, 1, target, kSegMinGranules, s);
+    if (st == PRISM_OK) st = plan_work(w.pkv, gselT, d, 2, 1, target, kSegMinGranules, s);
     if (st != PRISM_OK) return st;
-    const int smem = BwdLayout<D>::alloc((int)d.SW);
+    const int nq = BwdLayout<D>::stages(0, (int)d.SW), nk = BwdLayout<D>::stages(kXs, (int)d.SW);
+    const int smq = BwdLayout<D>::alloc(nq, 0, (int)d.SW), smk = BwdLayout<D>::alloc(nk, kXs, (int)d.SW);
+    if (smq > kSmemMax || smk > kSmemMax) return PRISM_ERR_UNSUPPORTED;   // selection rows too long
     auto kq = k_bwd_dq_sm100<D>;
     auto kk = k_bwd_dkdv_sm100<D>;
-    if (cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess ||
-        cudaFuncSetAttribute(kk, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    if (cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, smq) != cudaSuccess ||
+        cudaFuncSetAttribute(kk, cudaFuncAttributeMaxDynamicSharedMemorySize, smk) != cudaSuccess)
         return PRISM_ERR_CUDA;
-    kq<<<(unsigned)w.pq.items_max, 192, smem, s>>>(tQ, tdO, gK, gV, gsel, w.pq.hdr, w.pq.items, w.part_q, lse,
-                                                   w.delta, d.N, d.MB, (int)d.SW, scale, (__nv_bfloat16*)dQp,
-                                                   dev_status);
-    kk<<<(unsigned)w.pkv.items_max, 192, smem, s>>>(tK, tV, gQ, gdO, gselT, w.pkv.hdr, w.pkv.items, w.part_kv, lse,
-                                                    w.delta, d.N, d.MB, (int)d.SW, scale, (__nv_bfloat16*)dKp,
-                                                    (__nv_bfloat16*)dVp, dev_status);
+    kq<<<(unsigned)w.pq.items_max, 192, smq, s>>>(tQ, tdO, gK, gV, gsel, w.pq.hdr, w.pq.items, w.part_q, lse,
+                                                  w.delta, d.N, d.MB, (int)d.SW, nq, scale, (__nv_bfloat16*)dQp,
+                                                  dev_status);
+    kk<<<(unsigned)w.pkv.items_max, 192, smk, s>>>(tK, tV, gQ, gdO, gselT, w.pkv.hdr, w.pkv.items, w.part_kv, w.nld,
+                                                   d.N, d.MB, (int)d.SW, nk, scale, (__nv_bfloat16*)dKp,
+                                                   (__nv_bfloat16*)dVp, dev_status);
     st = launch_status(2);
     if (st == PRISM_OK) st = bwd_combine(w.pq, d, 1, w.part_q, dQp, scale, nullptr, 0.f, s);
     if (st == PRISM_OK) st = bwd_combine(w.pkv, d, 2, w.part_kv, dKp, scale, dVp, 1.f, s);
@@ -581,7 +629,7 @@ prism_status_t attn_bwd_sm100(const Dims& d, const void* Qp, const void* Kp, con
                               const uint32_t* gselT, float scale, void* dQp, void* dKp, void* dVp,
                               uint32_t* dev_status, void* ws, cudaStream_t s) {
     BwdWs w = carve_bwd(ws, d, nullptr);
-    prism_status_t st = bwd_delta(d, Op, o_f32, dOp, w.delta, s);
+    prism_status_t st = bwd_delta(d, Op, o_f32, dOp, w.delta, lse, w.nld, s);
     if (st != PRISM_OK) return st;
     if (d.d == 128)
         return launch_bwd<128>(d, Qp, Kp, Vp, dOp, lse, gsel, gselT, scale, dQp, dKp, dVp, dev_status, w, s);

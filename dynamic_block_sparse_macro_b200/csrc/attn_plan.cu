@@ -1,7 +1,8 @@
 // Work planning for the tensor-core attention kernels.
 //
-// A 128-row tile's work is the union of the granule-level selection rows of
-// its two 64-row granules.  That union is data dependent and very uneven (a
+// A tile's work is the union of the granule-level selection rows of its
+// 64-row granules (two for the 128-row tiles of the backward, four for the
+// 256-row tiles of the forward).  That union is data dependent and very uneven (a
 // query block with flat block probabilities makes Top-p select most keys), so
 // one CTA per tile would leave a few CTAs running long after the rest.  The
 // plan cuts every tile into segments of at most `seg` work units, choosing
@@ -20,16 +21,19 @@
 namespace prism {
 
 __global__ void __launch_bounds__(256) k_plan_count(const uint32_t* __restrict__ rows, int64_t MB, int SW,
-                                                    int tiles_per_head, int heads, int unit_granules,
+                                                    int tiles_per_head, int heads, int tile_gran, int unit_granules,
                                                     int32_t* __restrict__ tile_units, PlanHeader* hdr) {
     const int lane = threadIdx.x & 31;
     const int64_t t = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     if (t >= (int64_t)tiles_per_head * heads) return;
     const int hh = (int)(t / tiles_per_head), tile = (int)(t % tiles_per_head);
-    const uint32_t* r0 = rows + ((int64_t)hh * MB + 2 * tile) * SW;
-    const uint32_t* r1 = r0 + SW;
+    const uint32_t* r0 = rows + ((int64_t)hh * MB + (int64_t)tile_gran * tile) * SW;
     int cnt = 0;
-    for (int w = lane; w < SW; w += 32) cnt += __popc(r0[w] | r1[w]);
+    for (int w = lane; w < SW; w += 32) {
+        uint32_t u = 0u;
+        for (int i = 0; i < tile_gran; ++i) u |= r0[(int64_t)i * SW + w];
+        cnt += __popc(u);
+    }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
     if (lane == 0) {
@@ -98,7 +102,7 @@ __global__ void __launch_bounds__(1024) k_plan_items(const int32_t* __restrict__
 // ------------------------------------------------------------------ combine
 // O = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s, lse = (M + log2 L) ln 2
 __global__ void __launch_bounds__(128) k_fwd_combine(const int2* __restrict__ tile_split, int tiles_per_head,
-                                                     int64_t N, int D, const float* __restrict__ opart,
+                                                     int tile_rows, int64_t N, int D, const float* __restrict__ opart,
                                                      const float* __restrict__ mpart,
                                                      const float* __restrict__ lpart,
                                                      __nv_bfloat16* __restrict__ O, float* __restrict__ o_f32,
@@ -107,17 +111,17 @@ __global__ void __launch_bounds__(128) k_fwd_combine(const int2* __restrict__ ti
     const int2 sp = tile_split[t];
     if (sp.y <= 1) return;
     const int hh = t / tiles_per_head, tile = t % tiles_per_head;
-    const int64_t grow0 = (int64_t)hh * N + 128 * (int64_t)tile;
-    for (int r = 0; r < 128; ++r) {
+    const int64_t grow0 = (int64_t)hh * N + (int64_t)tile_rows * tile;
+    for (int r = 0; r < tile_rows; ++r) {
         float M = -INFINITY;
-        for (int s = 0; s < sp.y; ++s) M = fmaxf(M, mpart[(int64_t)(sp.x + s) * 128 + r]);
+        for (int s = 0; s < sp.y; ++s) M = fmaxf(M, mpart[(int64_t)(sp.x + s) * tile_rows + r]);
         float L = 0.f, acc = 0.f;
         for (int s = 0; s < sp.y; ++s) {
             const int64_t slot = sp.x + s;
-            const float m = mpart[slot * 128 + r];
+            const float m = mpart[slot * tile_rows + r];
             const float w = m > -INFINITY ? exp2f(m - M) : 0.f;
-            L += w * lpart[slot * 128 + r];
-            if (threadIdx.x < D) acc += w * opart[(slot * 128 + r) * D + threadIdx.x];
+            L += w * lpart[slot * tile_rows + r];
+            if (threadIdx.x < D) acc += w * opart[(slot * tile_rows + r) * D + threadIdx.x];
         }
         const float inv = L > 0.f ? 1.f / L : 0.f;
         if (threadIdx.x < D) {
@@ -170,21 +174,22 @@ Plan carve_plan(void* base, int64_t tiles, int target) {
     return pl;
 }
 
-prism_status_t plan_work(const Plan& pl, const uint32_t* rows, const Dims& d, int unit_granules, int target,
-                         int seg_min, cudaStream_t s) {
+prism_status_t plan_work(const Plan& pl, const uint32_t* rows, const Dims& d, int tile_gran, int unit_granules,
+                         int target, int seg_min, cudaStream_t s) {
     if (cudaMemsetAsync(pl.hdr, 0, sizeof(PlanHeader), s) != cudaSuccess) return PRISM_ERR_CUDA;
-    const int tph = (int)(d.N / 128);
+    const int tph = (int)(d.N / (64 * tile_gran));
     const unsigned grid = (unsigned)((pl.tiles * 32 + 255) / 256);
-    k_plan_count<<<grid, 256, 0, s>>>(rows, d.MB, (int)d.SW, tph, d.heads, unit_granules, pl.tile_units, pl.hdr);
+    k_plan_count<<<grid, 256, 0, s>>>(rows, d.MB, (int)d.SW, tph, d.heads, tile_gran, unit_granules, pl.tile_units,
+                                      pl.hdr);
     k_plan_items<<<1, 1024, 0, s>>>(pl.tile_units, (int)pl.tiles, target, seg_min, pl.tile_split, pl.items,
                                     pl.hdr);
     return launch_status(2);
 }
 
-prism_status_t fwd_combine(const Plan& pl, const Dims& d, const float* opart, const float* mpart,
+prism_status_t fwd_combine(const Plan& pl, const Dims& d, int tile_rows, const float* opart, const float* mpart,
                            const float* lpart, void* Op, float* o_f32, float* lse, cudaStream_t s) {
-    k_fwd_combine<<<(unsigned)pl.tiles, 128, 0, s>>>(pl.tile_split, (int)(d.N / 128), d.N, d.d, opart, mpart,
-                                                     lpart, (__nv_bfloat16*)Op, o_f32, lse);
+    k_fwd_combine<<<(unsigned)pl.tiles, 128, 0, s>>>(pl.tile_split, (int)(d.N / tile_rows), tile_rows, d.N, d.d,
+                                                     opart, mpart, lpart, (__nv_bfloat16*)Op, o_f32, lse);
     return launch_status(1);
 }
 

@@ -18,7 +18,7 @@ struct Plan {
     int32_t* tile_units;              // [tiles] units per tile
     int2* tile_split;                 // [tiles] (first slot or -1, segments)
     int4* items;                      // [tiles + target] (tile, unit begin, unit end, slot or -1)
-    int64_t tiles;                    // heads * N / 128
+    int64_t tiles;                    // heads * N / tile rows
     int64_t items_max;
 };
 
@@ -31,9 +31,10 @@ constexpr int kSegMinGranules = 16;   // backward: 64-row granules
 
 size_t plan_bytes(int64_t tiles, int target);
 Plan carve_plan(void* base, int64_t tiles, int target);
-prism_status_t plan_work(const Plan& pl, const uint32_t* rows, const Dims& d, int unit_granules, int target,
-                         int seg_min, cudaStream_t s);
-prism_status_t fwd_combine(const Plan& pl, const Dims& d, const float* opart, const float* mpart,
+// tile_gran: 64-row granules per tile (2 or 4); unit_granules: granules per work unit
+prism_status_t plan_work(const Plan& pl, const uint32_t* rows, const Dims& d, int tile_gran, int unit_granules,
+                         int target, int seg_min, cudaStream_t s);
+prism_status_t fwd_combine(const Plan& pl, const Dims& d, int tile_rows, const float* opart, const float* mpart,
                            const float* lpart, void* Op, float* o_f32, float* lse, cudaStream_t s);
 prism_status_t bwd_combine(const Plan& pl, const Dims& d, int nout, const float* part, void* out0, float mul0,
                            void* out1, float mul1, cudaStream_t s);

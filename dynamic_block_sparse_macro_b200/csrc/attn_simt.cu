@@ -154,7 +154,8 @@ template <> __device__ __forceinline__ float4 load4<__nv_bfloat16>(const __nv_bf
 
 template <typename T, int D>
 __global__ void k_bwd_delta(const T* __restrict__ O, const float* __restrict__ o_f32,
-                            const T* __restrict__ dO, int64_t rows, float* __restrict__ delta) {
+                            const T* __restrict__ dO, int64_t rows, float* __restrict__ delta,
+                            const float* __restrict__ lse, float* __restrict__ nld) {
     constexpr int LPR = D / 4;                                // lanes per row
     const int64_t gl = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     const int64_t r = gl / LPR;
@@ -167,7 +168,14 @@ __global__ void k_bwd_delta(const T* __restrict__ O, const float* __restrict__ o
     }
 #pragma unroll
     for (int off = LPR / 2; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-    if (r < rows && (gl % LPR) == 0) delta[r] = s;
+    if (r < rows && (gl % LPR) == 0) {
+        delta[r] = s;
+        if (nld) {                       // per 64-row granule: -lse*log2(e) [64], then -Delta [64]
+            float* blk = nld + (r >> 6) * 128;
+            blk[r & 63] = -lse[r] * kLog2e;
+            blk[64 + (r & 63)] = -s;
+        }
+    }
 }
 
 template <typename T, int D>
@@ -384,7 +392,7 @@ prism_status_t simt_bwd(const Dims& d, const void* Qp, const void* Kp, const voi
                         cudaStream_t s) {
     const int64_t rows = (int64_t)d.heads * d.N;
     k_bwd_delta<T, D><<<(unsigned)((rows * (D / 4) + 255) / 256), 256, 0, s>>>((const T*)Op, o_f32,
-                                                                                (const T*)dOp, rows, delta);
+                                                                                (const T*)dOp, rows, delta, lse, nullptr);
     auto kk = k_bwd_dkdv_simt<T, D>;
     auto kq = k_bwd_dq_simt<T, D>;
     if (cudaFuncSetAttribute(kk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dkdv_smem<D>()) != cudaSuccess ||
@@ -409,16 +417,16 @@ prism_status_t attn_fwd_simt(const Dims& d, const void* Qp, const void* Kp, cons
 
 // Delta = rowsum(dO * O) for every blocked row (shared by both backward families)
 prism_status_t bwd_delta(const Dims& d, const void* Op, const float* o_f32, const void* dOp, float* delta,
-                         cudaStream_t s) {
+                         const float* lse, float* nld, cudaStream_t s) {
     const int64_t rows = (int64_t)d.heads * d.N;
     const unsigned grid = (unsigned)((rows * (d.d / 4) + 255) / 256);
     if (d.dtype == PRISM_F32) {
-        if (d.d == 64) k_bwd_delta<float, 64><<<grid, 256, 0, s>>>((const float*)Op, o_f32, (const float*)dOp, rows, delta);
-        else k_bwd_delta<float, 128><<<grid, 256, 0, s>>>((const float*)Op, o_f32, (const float*)dOp, rows, delta);
+        if (d.d == 64) k_bwd_delta<float, 64><<<grid, 256, 0, s>>>((const float*)Op, o_f32, (const float*)dOp, rows, delta, lse, nld);
+        else k_bwd_delta<float, 128><<<grid, 256, 0, s>>>((const float*)Op, o_f32, (const float*)dOp, rows, delta, lse, nld);
     } else {
         using B = __nv_bfloat16;
-        if (d.d == 64) k_bwd_delta<B, 64><<<grid, 256, 0, s>>>((const B*)Op, o_f32, (const B*)dOp, rows, delta);
-        else k_bwd_delta<B, 128><<<grid, 256, 0, s>>>((const B*)Op, o_f32, (const B*)dOp, rows, delta);
+        if (d.d == 64) k_bwd_delta<B, 64><<<grid, 256, 0, s>>>((const B*)Op, o_f32, (const B*)dOp, rows, delta, lse, nld);
+        else k_bwd_delta<B, 128><<<grid, 256, 0, s>>>((const B*)Op, o_f32, (const B*)dOp, rows, delta, lse, nld);
     }
     return launch_status(1);
 }

@@ -14,7 +14,8 @@
 // Roles (6 warps):
 //   warp 0      TMA producer: Q once, then per chunk K and V (64x64 bf16 boxes,
 //               128-byte swizzle) into one K and one V buffer.
-//   warp 1      allocates 256 TMEM columns; lane 0 issues tcgen05.mma:
+//   warp 1      allocates 256 TMEM columns and issues tcgen05.mma (the whole
+//               warp, one elected lane):
 //               S = Q K^T (M=128, N=128, fp32 in TMEM), then O += P V with
 //               P read from TMEM (aliasing S) and V MN-major from shared memory.
 //   warps 2-5   one query row per thread: S row from TMEM, masked online
@@ -166,35 +167,35 @@ k_attn_fwd_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             }
         }
     } else if (warp == 1) {
-        if (lane == 0) {
+        {   // the whole warp, converged; one elected lane issues
             // ------------------------------------------------ MMA issuer
             const uint32_t idS = idesc_bf16_f32(128, 128, false, false);
             const uint32_t idO = idesc_bf16_f32(128, D, false, true);
             const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV);
-            bool ok = mbar_wait(bar_q, 0, abort_flag, dev_status);
+            bool ok = mbar_wait_w(bar_q, 0, abort_flag, dev_status);
             tc_fence_after();
             for (int c = 0; ok && c < nch; ++c) {
-                if (!mbar_wait(bar_kf, c & 1, abort_flag, dev_status)) break;
+                if (!mbar_wait_w(bar_kf, c & 1, abort_flag, dev_status)) break;
                 tc_fence_after();
 #pragma unroll
                 for (int k = 0; k < D / 16; ++k) {
                     const uint32_t off = (k >> 2) * kRegion + (k & 3) * 32;
-                    mma_ss(tbase + kColS, sdesc_sw128(aQ + off, 16, 1024), sdesc_sw128(aK + off, 16, 1024), idS,
-                           k > 0 ? 1u : 0u);
+                    mma_ss_w(tbase + kColS, sdesc_sw128(aQ + off, 16, 1024), sdesc_sw128(aK + off, 16, 1024), idS,
+                             k > 0 ? 1u : 0u);
                 }
-                tc_commit(bar_ke);
-                tc_commit(bar_s);
-                if (!mbar_wait(bar_p, c & 1, abort_flag, dev_status)) break;
+                tc_commit_w(bar_ke);
+                tc_commit_w(bar_s);
+                if (!mbar_wait_w(bar_p, c & 1, abort_flag, dev_status)) break;
                 tc_fence_after();
-                if (!mbar_wait(bar_vf, c & 1, abort_flag, dev_status)) break;
+                if (!mbar_wait_w(bar_vf, c & 1, abort_flag, dev_status)) break;
                 tc_fence_after();
 #pragma unroll
                 for (int k = 0; k < 8; ++k)
-                    mma_ts(tbase + kColO, tbase + kColS + 8 * k, sdesc_sw128(aV + k * 2048, kRegion, 1024), idO,
-                           (c > 0 || k > 0) ? 1u : 0u);
-                tc_commit(bar_ve);
+                    mma_ts_w(tbase + kColO, tbase + kColS + 8 * k, sdesc_sw128(aV + k * 2048, kRegion, 1024), idO,
+                             (c > 0 || k > 0) ? 1u : 0u);
+                tc_commit_w(bar_ve);
             }
-            tc_commit(bar_o);
+            tc_commit_w(bar_o);
             if (*abort_flag) {
                 volatile int no_abort = 0;
                 mbar_wait(bar_o, 0, &no_abort, dev_status);
@@ -407,7 +408,7 @@ prism_status_t launch_fwd(const Dims& d, const void* Qp, const void* Kp, const v
         return PRISM_ERR_CUDA;
     FwdWs w = carve_fwd(ws, d);
     const int target = plan_target(device_sms());
-    prism_status_t st = plan_work(w.plan, gsel, d, 2, target, kSegMinChunks, s);
+    prism_status_t st = plan_work(w.plan, gsel, d, 2, 2, target, kSegMinChunks, s);
     if (st != PRISM_OK) return st;
     auto k = k_attn_fwd_sm100<D>;
     const int smem = FwdLayout<D>::alloc((int)d.SW);
@@ -417,7 +418,7 @@ prism_status_t launch_fwd(const Dims& d, const void* Qp, const void* Kp, const v
                                                     (int)d.SW, scale, (__nv_bfloat16*)Op, lse, o_f32, dev_status);
     st = launch_status(1);
     if (st != PRISM_OK) return st;
-    return fwd_combine(w.plan, d, w.parts.o, w.parts.m, w.parts.l, Op, o_f32, lse, s);
+    return fwd_combine(w.plan, d, 128, w.parts.o, w.parts.m, w.parts.l, Op, o_f32, lse, s);
 }
 
 }  // namespace

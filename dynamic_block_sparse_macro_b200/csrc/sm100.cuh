@@ -77,6 +77,33 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
         ::"r"(smem_u32(dst)), "l"(map), "r"(smem_u32(bar)), "r"(x), "r"(y)
         : "memory");
 }
+// 1-D bulk copy of `bytes` contiguous bytes (16-byte aligned, a multiple of 16)
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar))
+                 : "memory");
+}
+// 3-D form used for whole-row tiles: coordinates (column within a 64-column
+// region, row, region index)
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y, int z) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];"
+        ::"r"(smem_u32(dst)), "l"(map), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
+        : "memory");
+}
+// TMA tile store from shared memory (a bulk group; coordinates must be >= 0)
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* src, int x, int y, int z) {
+    asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];"
+                 ::"l"(map), "r"(smem_u32(src)), "r"(x), "r"(y), "r"(z)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// wait until every bulk store this thread committed has finished reading shared memory
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// make this thread's generic shared-memory writes visible to the async (TMA) proxy
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
 }
@@ -126,6 +153,44 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
         : "memory");
 }
 
+// Warp-wide forms: the whole warp executes them converged and one lane, picked
+// by elect.sync, issues the instruction.  Issued this way tcgen05.mma streams
+// at the tensor pipe's rate; issued from a lone lane of a diverged warp each
+// instruction costs about 65 cycles of issue overhead.
+__device__ __forceinline__ void mma_ss_w(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                         uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p, e;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+__device__ __forceinline__ void mma_ts_w(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                         uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p, e;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+__device__ __forceinline__ void tc_commit_w(uint64_t* bar) {
+    asm volatile(
+        "{\n\t.reg .pred e;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}"
+        ::"r"(smem_u32(bar))
+        : "memory");
+}
+// bounded wait taken by a whole warp; the verdict is made warp-uniform
+__device__ __forceinline__ bool mbar_wait_w(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                            uint32_t* dev_status) {
+    return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, dev_status));
+}
+
 // 32 lanes x 32 consecutive 32-bit columns: thread t of the warp gets lane (base lane + t)
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
     asm volatile(
@@ -150,6 +215,15 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
           "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]),
           "r"(r[31])
         : "memory");
+}
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+          "=r"(r[15])
+        : "r"(taddr));
 }
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
     asm volatile(
@@ -181,6 +255,21 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_byt
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn, bool b_mn) {
     return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16) |
            ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// barrier among `threads` threads (a multiple of 32) of the block, by id (1..15)
+__device__ __forceinline__ void named_sync(int id, int threads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+// Register split between warpgroups (all four warps of a warpgroup execute it
+// together): the block launches with an even share per thread and then
+// producer-side warpgroups give registers back for the math warpgroups.
+template <uint32_t R> __device__ __forceinline__ void regs_dec() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(R));
+}
+template <uint32_t R> __device__ __forceinline__ void regs_inc() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(R));
 }
 
 // ------------------------------------------------------------------ packed fp32 math
@@ -225,6 +314,80 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
     return r;
 }
+
+// 2^x on the FMA pipe, two values at a time, for x <= 0 (the softmax
+// exponents after the running max is subtracted).  Cody and Waite's range
+// reduction: x = j + f with j = round(x) (by adding 1.5 * 2^23, whose ulp is 1)
+// and f in [-1/2, 1/2]; 2^f by a cubic fitted to 2^f on that interval
+// (weighted least squares towards minimal relative error; in fp32 its
+// relative error stays below 8e-5, far under the bf16 rounding of P); the
+// result's exponent field is then raised by j.  x is clamped at -126 so that
+// the exponent field stays >= 0 (2^-126 is nothing next to the row maximum's 1).
+constexpr float kExp2C0 = 0.99992806f, kExp2C1 = 0.69326097f, kExp2C2 = 0.24261113f, kExp2C3 = 0.05517166f;
+__device__ __forceinline__ void exp2_poly2(float x0, float x1, float& y0, float& y1) {
+    const float kRound = 12582912.0f;                       // 1.5 * 2^23
+    x0 = fmaxf(x0, -126.f);
+    x1 = fmaxf(x1, -126.f);
+    const uint64_t t = fadd2(f2pack(x0, x1), f2pack(kRound, kRound));
+    const uint64_t j = fadd2(t, f2pack(-kRound, -kRound));
+    const uint64_t f = ffma2(j, f2pack(-1.f, -1.f), f2pack(x0, x1));
+    uint64_t p = ffma2(f, f2pack(kExp2C3, kExp2C3), f2pack(kExp2C2, kExp2C2));
+    p = ffma2(p, f, f2pack(kExp2C1, kExp2C1));
+    p = ffma2(p, f, f2pack(kExp2C0, kExp2C0));
+    float p0, p1, t0, t1;
+    f2unpack(p, p0, p1);
+    f2unpack(t, t0, t1);
+    // the low bits of t hold j (two's complement); j << 23 lands on the exponent field
+    y0 = __int_as_float(__float_as_int(t0) * (1 << 23) + __float_as_int(p0));
+    y1 = __int_as_float(__float_as_int(t1) * (1 << 23) + __float_as_int(p1));
+}
+
+// Walks the union of R granule-level selection rows held consecutively in
+// shared memory (row i at rows + i * words) in ascending granule order; the
+// R-bit mask says which rows have the granule.
+template <int R>
+struct GranuleWalkN {
+    const uint32_t* rows;
+    int wn, w;
+    uint32_t bits;
+
+    __device__ uint32_t word(int i) const {
+        uint32_t u = 0u;
+#pragma unroll
+        for (int r = 0; r < R; ++r) u |= rows[r * wn + i];
+        return u;
+    }
+    __device__ void init(const uint32_t* r, int words) {
+        rows = r; wn = words; w = 0;
+        bits = wn > 0 ? word(0) : 0u;
+    }
+    __device__ void skip(int n) {
+        while (n > 0) {
+            const int c = __popc(bits);
+            if (c <= n) {
+                n -= c;
+                bits = 0u;
+                if (++w >= wn) return;
+                bits = word(w);
+            } else {
+                for (; n > 0; --n) bits &= bits - 1;
+            }
+        }
+    }
+    __device__ bool next(int& row, uint32_t& m) {
+        while (bits == 0) {
+            if (++w >= wn) return false;
+            bits = word(w);
+        }
+        const int b = __ffs(bits) - 1;
+        bits &= bits - 1;
+        row = 64 * (w * 32 + b);
+        m = 0u;
+#pragma unroll
+        for (int r = 0; r < R; ++r) m |= ((rows[r * wn + w] >> b) & 1u) << r;
+        return true;
+    }
+};
 
 // Walks the union of two granule-level selection rows (held in shared
 // memory) in ascending granule order.  A set bit g stands for the 64 rows
@@ -310,6 +473,39 @@ inline bool make_map_bf16(CUtensorMap* m, const void* base, int64_t rows, int d,
     cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
     cuuint32_t estr[2] = {1, 1};
     return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 3-D map over the same [rows][d] bf16 tensor viewed as (64 columns, rows,
+// d/64 regions), region stride 128 bytes: one copy of box {64, box_rows, d/64}
+// lands box_rows full rows as d/64 consecutive 128-byte-swizzled regions of
+// box_rows x 128 bytes, the K-major operand image tcgen05.mma reads.  A copy
+// engine completes the copies of one issuing thread one after another at a
+// roughly fixed cost per copy (about 600 cycles, whatever the size up to
+// 32 KB), so whole-row copies (16 KB per 64-row granule at d = 128) move four
+// times the bytes per copy of 64-column, 64-row boxes.
+// the same whole-row view of a [rows][d] fp32 tensor: d/32 regions of 32 columns
+inline bool make_map_f32_rows(CUtensorMap* m, const void* base, int64_t rows, int d, int box_rows) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {32, (cuuint64_t)rows, (cuuint64_t)(d / 32)};
+    cuuint64_t strides[2] = {(cuuint64_t)d * 4, 128};
+    cuuint32_t box[3] = {32, (cuuint32_t)box_rows, (cuuint32_t)(d / 32)};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+inline bool make_map_bf16_rows(CUtensorMap* m, const void* base, int64_t rows, int d, int box_rows) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {64, (cuuint64_t)rows, (cuuint64_t)(d / 64)};
+    cuuint64_t strides[2] = {(cuuint64_t)d * 2, 128};
+    cuuint32_t box[3] = {64, (cuuint32_t)box_rows, (cuuint32_t)(d / 64)};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
