@@ -9,9 +9,10 @@
 //
 // Two kernels, no atomics (deterministic):
 //   k_bwd_dq_sm100    query-stationary: per (128-row query tile, head) walk the
-//                     key granules of the union of its two granule-level rows; per 64-key granule
-//                     S = Q K^T and dP = dO V^T (M=128, N=64) into TMEM, dS as
-//                     bf16 back into TMEM, dQ += dS K (K MN-major in smem).
+//                     key granules of the union of its two granule-level rows;
+//                     Q and dO sit in TMEM as bf16; per 64-key granule S = Q K^T
+//                     and dP = dO V^T (M=128, N=64, A from TMEM) into TMEM, dS
+//                     as bf16 back into TMEM, dQ += dS K (K MN-major in smem).
 //   k_bwd_dkdv_sm100  key-stationary: per (128-key tile, head) walk the query
 //                     granules whose blocks selected the tile's key blocks (the
 //                     transposed granule-level selection); per 64-query granule
@@ -39,26 +40,32 @@ namespace {
 
 constexpr int kTile = 128 * 128;           // bytes: 128 rows x 64 bf16 columns
 constexpr int kGran = 64 * 128;            // bytes: 64 rows x 64 bf16 columns
-constexpr int kStages = 6;                 // barrier slots; the ring uses nst <= kStages of them
+constexpr int kStages = 8;                 // barrier slots; the ring uses nst <= kStages of them
+constexpr int kCtrl = 512;                 // bytes of barriers and flags
 constexpr int kXs = 512;                   // per stage (dK/dV only): -lse*log2(e) and -Delta of 64 query rows
 constexpr uint32_t kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kSmemMax = 227 * 1024;
+// dK/dV kernel register split: 384 threads launch with 168 each; warpgroup 0
+// (TMA, MMA) drops to 96 and the two elementwise warpgroups rise to 200
+// (128 * (96 + 2 * 200) <= 384 * 168)
+constexpr uint32_t kRegsLow = 96, kRegsHigh = 200;
 
-// Shared memory: stationary tiles, then a ring of nst granule stages (as many
-// as fit: the TMA latency under load is about 4000 cycles, a granule's MMAs
-// take about 800), then barriers and the two selection rows.
-template <int D>
+// Shared memory: stationary tiles (dK/dV only; the dQ kernel keeps Q and dO
+// in TMEM), then a ring of nst granule stages (as many as fit: the TMA latency
+// under load is about 4000 cycles, a granule's MMAs take about 800), then
+// barriers and the two selection rows.
+template <int D, bool STAT>
 struct BwdLayout {
     static constexpr int NR = D / 64;
-    static constexpr int A0 = 0;                       // stationary operand 1 (Q or K)
-    static constexpr int A1 = NR * kTile;              // stationary operand 2 (dO or V)
-    static constexpr int RING = 2 * NR * kTile;        // streamed granules
+    static constexpr int A0 = 0;                       // stationary operand 1 (K)
+    static constexpr int A1 = NR * kTile;              // stationary operand 2 (V)
+    static constexpr int RING = STAT ? 2 * NR * kTile : 0;   // streamed granules
     static constexpr int STAGE = 2 * NR * kGran;       // two operands per stage
     // xs: bytes of per-granule row data staged beside each stage (0 or kXs)
     __host__ __device__ static int xs(int nst) { return RING + nst * STAGE; }
     __host__ __device__ static int ctrl(int nst, int xsb) { return xs(nst) + nst * xsb; }
-    __host__ __device__ static int rows(int nst, int xsb) { return ctrl(nst, xsb) + 256; }
+    __host__ __device__ static int rows(int nst, int xsb) { return ctrl(nst, xsb) + kCtrl; }
     static int alloc(int nst, int xsb, int SW) { return rows(nst, xsb) + 8 * SW + 1024; }
     static int stages(int xsb, int SW) {               // deepest ring that fits, at least 2
         int n = kStages;
@@ -97,10 +104,10 @@ __device__ __forceinline__ Bars carve(uint8_t* ctrl) {
     r.ng_slot = reinterpret_cast<int*>(r.tmem_slot + 2);
     return r;
 }
-static_assert((6 + 4 * kStages) * 8 + 12 <= 256, "barriers overflow the control block");
+static_assert((6 + 4 * kStages) * 8 + 12 <= kCtrl, "barriers overflow the control block");
 
-__device__ __forceinline__ void init_bars(const Bars& B, int nst) {
-    mbar_init(B.stat, 2);
+__device__ __forceinline__ void init_bars(const Bars& B, int nst, int stat_arrivals) {
+    mbar_init(B.stat, stat_arrivals);
     for (int s = 0; s < nst; ++s) {
         mbar_init(B.full0 + s, 1);
         mbar_init(B.full1 + s, 1);
@@ -124,20 +131,21 @@ __device__ __forceinline__ uint32_t kmaj_off(int k, int region) { return (k >> 2
 // its own: lane kind * nst + stage issues stream `kind` (0: operand 0, 1:
 // operand 1, 2: the 512 bytes of row data, dK/dV only) of the granules that
 // use that stage, one copy per granule, and never has more than one copy in
-// flight.  Lanes 0 and nst also copy the two stationary tiles.
-template <int D>
+// flight.  With stationary tiles in shared memory (dK/dV), lanes 0 and nst
+// also copy those.
+template <int D, bool STAT>
 __device__ void produce(const CUtensorMap* m0, const CUtensorMap* m1, const CUtensorMap* g0, const CUtensorMap* g1,
                         const float* nld, uint8_t* xs, uint8_t* sm, const Bars& B, int64_t row0, int tile_row,
                         const uint32_t* u0, const uint32_t* u1, int wn, int g_begin, int ng, int nst,
                         uint32_t* dev_status) {
-    using L = BwdLayout<D>;
+    using L = BwdLayout<D, STAT>;
     const int lane = threadIdx.x & 31;
     if (lane >= (nld ? 3 : 2) * nst) return;
     const int kind = lane / nst, stage = lane % nst;
     uint64_t* full = kind == 0 ? B.full0 : kind == 1 ? B.full1 : B.fullx;
     const CUtensorMap* mg = kind == 0 ? g0 : g1;
     if (kind < 2) tma_prefetch_desc(mg);
-    if (stage == 0 && kind < 2) {
+    if (STAT && stage == 0 && kind < 2) {
         const CUtensorMap* ms = kind == 0 ? m0 : m1;
         mbar_expect_tx(B.stat, L::NR * kTile);
         tma_load_3d(sm + (kind ? L::A1 : L::A0), ms, B.stat, 0, (int)(row0 + tile_row), 0);
@@ -172,14 +180,17 @@ __device__ void produce(const CUtensorMap* m0, const CUtensorMap* m1, const CUte
 // ============================================================================ dQ
 template <int D>
 __global__ void __launch_bounds__(192, 1)
-k_bwd_dq_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmdO,
+k_bwd_dq_sm100(const __nv_bfloat16* __restrict__ Qg, const __nv_bfloat16* __restrict__ dOg,
                const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                const uint32_t* __restrict__ gsel, const PlanHeader* __restrict__ hdr,
                const int4* __restrict__ items, float* __restrict__ part, const float* __restrict__ lse,
                const float* __restrict__ delta, int64_t N, int64_t MB, int SW, int nst, float scale,
                __nv_bfloat16* __restrict__ dQ, uint32_t* __restrict__ dev_status) {
-    using L = BwdLayout<D>;
+    using L = BwdLayout<D, false>;
+    // TMEM: dQ, S / dP of two granules, and the tile's Q and dO as bf16 (the A
+    // operands of S = Q K^T and dP = dO V^T, read by the tensor core from TMEM)
     constexpr uint32_t cdQ = 0, cS = 128, cP = 192;   // + 128 * buffer for S / dP
+    constexpr uint32_t cQ = 384, cdO = 384 + D / 2;
     if ((int)blockIdx.x >= hdr->n_items) return;      // uniform: beyond the item list
     const int4 item = items[blockIdx.x];
     const int tiles_per_head = (int)(N / 128);
@@ -195,7 +206,7 @@ k_bwd_dq_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     const int64_t row0 = (int64_t)hh * N;
 
     load_rows(u0, u1, gsel + ((int64_t)hh * MB + 2 * tile) * SW, gsel + ((int64_t)hh * MB + 2 * tile + 1) * SW, wn);
-    if (threadIdx.x == 0) init_bars(B, nst);
+    if (threadIdx.x == 0) init_bars(B, nst, 128);     // Q, dO: one arrival per tile row
     if (warp == 1) {
         tmem_alloc(B.tmem_slot, kTmemCols);
         tmem_relinquish();
@@ -206,13 +217,13 @@ k_bwd_dq_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     const uint32_t tb = *B.tmem_slot;
 
     if (warp == 0) {
-        produce<D>(&tmQ, &tmdO, &tmK, &tmV, nullptr, nullptr, sm, B, row0, 128 * tile, u0, u1, wn, g_begin, ng, nst,
-                   dev_status);
+        produce<D, false>(nullptr, nullptr, &tmK, &tmV, nullptr, nullptr, sm, B, row0, 128 * tile, u0, u1, wn,
+                          g_begin, ng, nst, dev_status);
     } else if (warp == 1) {
         {   // the whole warp, converged; one elected lane issues
             const uint32_t idPS = idesc_bf16_f32(128, 64, false, false);
             const uint32_t idQ = idesc_bf16_f32(128, D, false, true);
-            const uint32_t aQ = smem_u32(sm + L::A0), adO = smem_u32(sm + L::A1), aR = smem_u32(sm + L::RING);
+            const uint32_t aR = smem_u32(sm + L::RING);
             bool ok = mbar_wait_w(B.stat, 0, B.abort_flag, dev_status);
             tc_fence_after();
             for (int g = 0; ok && g <= ng; ++g) {
@@ -225,12 +236,12 @@ k_bwd_dq_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                     const uint32_t aK = aR + s * L::STAGE, aV = aK + L::NR * kGran;
 #pragma unroll
                     for (int k = 0; k < D / 16; ++k)
-                        mma_ss_w(tb + cS + 128 * b, sdesc_sw128(aQ + kmaj_off(k, kTile), 16, 1024),
-                                 sdesc_sw128(aK + kmaj_off(k, kGran), 16, 1024), idPS, k > 0);
+                        mma_ts_w(tb + cS + 128 * b, tb + cQ + 8 * k, sdesc_sw128(aK + kmaj_off(k, kGran), 16, 1024),
+                                 idPS, k > 0);
 #pragma unroll
                     for (int k = 0; k < D / 16; ++k)
-                        mma_ss_w(tb + cP + 128 * b, sdesc_sw128(adO + kmaj_off(k, kTile), 16, 1024),
-                                 sdesc_sw128(aV + kmaj_off(k, kGran), 16, 1024), idPS, k > 0);
+                        mma_ts_w(tb + cP + 128 * b, tb + cdO + 8 * k, sdesc_sw128(aV + kmaj_off(k, kGran), 16, 1024),
+                                 idPS, k > 0);
                     tc_commit_w(B.prod + b);
                 }
                 if (g > 0) {
@@ -255,6 +266,29 @@ k_bwd_dq_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         const int sub = warp & 3, row = sub * 32 + lane, half = row >> 6;
         const uint32_t tl = tb + ((uint32_t)(sub * 32) << 16);
         const int64_t grow = row0 + 128 * tile + row;
+        {
+            // this row of Q and of dO into TMEM (two bf16 per column)
+#pragma unroll
+            for (int which = 0; which < 2; ++which) {
+                const uint4* src = reinterpret_cast<const uint4*>((which ? dOg : Qg) + grow * D);
+#pragma unroll
+                for (int q = 0; q < D / 64; ++q) {
+                    uint32_t r[32];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const uint4 v = __ldg(src + 8 * q + i);
+                        r[4 * i] = v.x;
+                        r[4 * i + 1] = v.y;
+                        r[4 * i + 2] = v.z;
+                        r[4 * i + 3] = v.w;
+                    }
+                    tmem_st32(tl + (which ? cdO : cQ) + 32 * q, r);
+                }
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(B.stat);
+        }
         const float lse2 = lse[grow] * kLog2e, dl = delta[grow];
         const float sl2 = scale * kLog2e;
         const uint64_t sl2x2 = f2pack(sl2, sl2), nlse2 = f2pack(-lse2, -lse2), ndl2 = f2pack(-dl, -dl);
@@ -351,14 +385,14 @@ k_bwd_dq_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 
 // ============================================================================ dK, dV
 template <int D>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(384, 1)
 k_bwd_dkdv_sm100(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                  const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmdO,
                  const uint32_t* __restrict__ gselT, const PlanHeader* __restrict__ hdr,
                  const int4* __restrict__ items, float* __restrict__ part, const float* __restrict__ nld,
                  int64_t N, int64_t MB, int SW, int nst, float scale, __nv_bfloat16* __restrict__ dK, __nv_bfloat16* __restrict__ dV,
                  uint32_t* __restrict__ dev_status) {
-    using L = BwdLayout<D>;
+    using L = BwdLayout<D, true>;
     constexpr uint32_t cdK = 0, cdV = 128, cS = 256, cP = 320;   // + 128 * buffer for S^T / dP^T
     if ((int)blockIdx.x >= hdr->n_items) return;      // uniform: beyond the item list
     const int4 item = items[blockIdx.x];
@@ -376,7 +410,7 @@ k_bwd_dkdv_sm100(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
     const int64_t row0 = (int64_t)hh * N;
 
     load_rows(u0, u1, gselT + ((int64_t)hh * MB + 2 * tile) * SW, gselT + ((int64_t)hh * MB + 2 * tile + 1) * SW, wn);
-    if (threadIdx.x == 0) init_bars(B, nst);
+    if (threadIdx.x == 0) init_bars(B, nst, 2);       // K, V: one arrival per stationary copy
     if (warp == 1) {
         tmem_alloc(B.tmem_slot, kTmemCols);
         tmem_relinquish();
@@ -386,10 +420,12 @@ k_bwd_dkdv_sm100(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
     tc_fence_after();
     const uint32_t tb = *B.tmem_slot;
 
-    if (warp == 0) {
-        produce<D>(&tmK, &tmV, &tmQ, &tmdO, nld, xs, sm, B, row0, 128 * tile, u0, u1, wn, g_begin, ng, nst,
-                   dev_status);
-    } else if (warp == 1) {
+    if (warp < 4) {
+      regs_dec<kRegsLow>();
+      if (warp == 0) {
+        produce<D, true>(&tmK, &tmV, &tmQ, &tmdO, nld, xs, sm, B, row0, 128 * tile, u0, u1, wn, g_begin, ng, nst,
+                         dev_status);
+      } else if (warp == 1) {
         {   // the whole warp, converged; one elected lane issues
             const uint32_t idPS = idesc_bf16_f32(128, 64, false, false);
             const uint32_t idKV = idesc_bf16_f32(128, D, false, true);
@@ -436,7 +472,12 @@ k_bwd_dkdv_sm100(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
                 mbar_wait(B.fin, 0, &no_abort, dev_status);
             }
         }
+      }
     } else {
+        regs_inc<kRegsHigh>();
+        // two elementwise warpgroups take alternate granules (warpgroup wg uses
+        // TMEM buffer wg), so one's latency hides behind the other's work
+        const int wg = (warp - 4) >> 2;
         const int sub = warp & 3, row = sub * 32 + lane, half = row >> 6;
         const uint32_t tl = tb + ((uint32_t)(sub * 32) << 16);
         const float sl2 = scale * kLog2e;
@@ -452,6 +493,7 @@ k_bwd_dkdv_sm100(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
             uint32_t mk = 0;
             int qrow = 0;
             if (lane == 0) walk.next(qrow, mk);
+            if (b != wg) continue;                             // the other warpgroup's granule
             mk = __shfl_sync(0xffffffffu, mk, 0);
             const bool valid = (mk >> half) & 1u;              // warp-uniform
             const float4* nl4 = reinterpret_cast<const float4*>(xs + st * kXs);   // -lse*log2(e), 64 rows
@@ -460,21 +502,15 @@ k_bwd_dkdv_sm100(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
                              mbar_wait(B.fullx + st, (g / nst) & 1, B.abort_flag, dev_status);
             if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
             tc_fence_after();
-            // S^T and dP^T of the granule: all TMEM loads in flight before one wait
-            uint32_t sv[2][32], pv[2][32];
-            if (valid) {
-                tmem_ld32(tl + cS + 128 * b, sv[0]);
-                tmem_ld32(tl + cP + 128 * b, pv[0]);
-                tmem_ld32(tl + cS + 128 * b + 32, sv[1]);
-                tmem_ld32(tl + cP + 128 * b + 32, pv[1]);
-                tmem_wait_ld();
-            }
 #pragma unroll
             for (int hq = 0; hq < 2; ++hq) {
                 uint32_t op[16], od[16];
                 if (valid) {
-                    const uint32_t (&s)[32] = sv[hq];
-                    const uint32_t (&p)[32] = pv[hq];
+                    // 32 columns of S^T and of dP^T: both TMEM loads in flight before one wait
+                    uint32_t s[32], p[32];
+                    tmem_ld32(tl + cS + 128 * b + 32 * hq, s);
+                    tmem_ld32(tl + cP + 128 * b + 32 * hq, p);
+                    tmem_wait_ld();
 #pragma unroll
                     for (int i4 = 0; i4 < 8; ++i4) {
                         const float4 l4 = nl4[8 * hq + i4];
@@ -510,8 +546,8 @@ k_bwd_dkdv_sm100(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
         if (__all_sync(0xffffffffu, fin)) {
             tc_fence_after();
             const int64_t grow = row0 + 128 * tile + row;
-#pragma unroll
-            for (int which = 0; which < 2; ++which) {
+            {
+                const int which = wg;                          // warpgroup 0 writes dK, warpgroup 1 dV
                 const float mul = which ? 1.f : scale;
                 const uint32_t col = which ? cdV : cdK;
 #pragma unroll
@@ -586,9 +622,8 @@ prism_status_t launch_bwd(const Dims& d, const void* Qp, const void* Kp, const v
                           const float* lse, const uint32_t* gsel, const uint32_t* gselT, float scale, void* dQp,
                           void* dKp, void* dVp, uint32_t* dev_status, const BwdWs& w, cudaStream_t s) {
     const int64_t rows = (int64_t)d.heads * d.N;
-    CUtensorMap tQ, tdO, tK, tV, gQ, gdO, gK, gV;
-    if (!make_map_bf16_rows(&tQ, Qp, rows, D, 128) || !make_map_bf16_rows(&tdO, dOp, rows, D, 128) ||
-        !make_map_bf16_rows(&tK, Kp, rows, D, 128) || !make_map_bf16_rows(&tV, Vp, rows, D, 128) ||
+    CUtensorMap tK, tV, gQ, gdO, gK, gV;
+    if (!make_map_bf16_rows(&tK, Kp, rows, D, 128) || !make_map_bf16_rows(&tV, Vp, rows, D, 128) ||
         !make_map_bf16_rows(&gQ, Qp, rows, D, 64) || !make_map_bf16_rows(&gdO, dOp, rows, D, 64) ||
         !make_map_bf16_rows(&gK, Kp, rows, D, 64) || !make_map_bf16_rows(&gV, Vp, rows, D, 64))
         return PRISM_ERR_CUDA;
@@ -596,18 +631,19 @@ prism_status_t launch_bwd(const Dims& d, const void* Qp, const void* Kp, const v
     prism_status_t st = plan_work(w.pq, gsel, d, 2, 1, target, kSegMinGranules, s);
     if (st == PRISM_OK) st = plan_work(w.pkv, gselT, d, 2, 1, target, kSegMinGranules, s);
     if (st != PRISM_OK) return st;
-    const int nq = BwdLayout<D>::stages(0, (int)d.SW), nk = BwdLayout<D>::stages(kXs, (int)d.SW);
-    const int smq = BwdLayout<D>::alloc(nq, 0, (int)d.SW), smk = BwdLayout<D>::alloc(nk, kXs, (int)d.SW);
+    const int nq = BwdLayout<D, false>::stages(0, (int)d.SW), nk = BwdLayout<D, true>::stages(kXs, (int)d.SW);
+    const int smq = BwdLayout<D, false>::alloc(nq, 0, (int)d.SW);
+    const int smk = BwdLayout<D, true>::alloc(nk, kXs, (int)d.SW);
     if (smq > kSmemMax || smk > kSmemMax) return PRISM_ERR_UNSUPPORTED;   // selection rows too long
     auto kq = k_bwd_dq_sm100<D>;
     auto kk = k_bwd_dkdv_sm100<D>;
     if (cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, smq) != cudaSuccess ||
         cudaFuncSetAttribute(kk, cudaFuncAttributeMaxDynamicSharedMemorySize, smk) != cudaSuccess)
         return PRISM_ERR_CUDA;
-    kq<<<(unsigned)w.pq.items_max, 192, smq, s>>>(tQ, tdO, gK, gV, gsel, w.pq.hdr, w.pq.items, w.part_q, lse,
+    kq<<<(unsigned)w.pq.items_max, 192, smq, s>>>((const __nv_bfloat16*)Qp, (const __nv_bfloat16*)dOp, gK, gV, gsel, w.pq.hdr, w.pq.items, w.part_q, lse,
                                                   w.delta, d.N, d.MB, (int)d.SW, nq, scale, (__nv_bfloat16*)dQp,
                                                   dev_status);
-    kk<<<(unsigned)w.pkv.items_max, 192, smk, s>>>(tK, tV, gQ, gdO, gselT, w.pkv.hdr, w.pkv.items, w.part_kv, w.nld,
+    kk<<<(unsigned)w.pkv.items_max, 384, smk, s>>>(tK, tV, gQ, gdO, gselT, w.pkv.hdr, w.pkv.items, w.part_kv, w.nld,
                                                    d.N, d.MB, (int)d.SW, nk, scale, (__nv_bfloat16*)dKp,
                                                    (__nv_bfloat16*)dVp, dev_status);
     st = launch_status(2);
