@@ -47,9 +47,9 @@ constexpr uint32_t kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kSmemMax = 227 * 1024;
 // dK/dV kernel register split: 384 threads launch with 168 each; warpgroup 0
-// (TMA, MMA) drops to 96 and the two elementwise warpgroups rise to 200
-// (128 * (96 + 2 * 200) <= 384 * 168)
-constexpr uint32_t kRegsLow = 96, kRegsHigh = 200;
+// (TMA, MMA) drops to 120 and the two elementwise warpgroups rise to 192
+// (128 * (120 + 2 * 192) = 384 * 168)
+constexpr uint32_t kRegsLow = 120, kRegsHigh = 192;
 
 // Shared memory: stationary tiles (dK/dV only; the dQ kernel keeps Q and dO
 // in TMEM), then a ring of nst granule stages (as many as fit: the TMA latency
@@ -106,7 +106,7 @@ __device__ __forceinline__ Bars carve(uint8_t* ctrl) {
 }
 static_assert((6 + 4 * kStages) * 8 + 12 <= kCtrl, "barriers overflow the control block");
 
-__device__ __forceinline__ void init_bars(const Bars& B, int nst, int stat_arrivals) {
+__device__ __forceinline__ void init_bars(const Bars& B, int nst, int stat_arrivals, int elem_arrivals) {
     mbar_init(B.stat, stat_arrivals);
     for (int s = 0; s < nst; ++s) {
         mbar_init(B.full0 + s, 1);
@@ -116,7 +116,7 @@ __device__ __forceinline__ void init_bars(const Bars& B, int nst, int stat_arriv
     }
     for (int b = 0; b < 2; ++b) {
         mbar_init(B.prod + b, 1);
-        mbar_init(B.elem + b, 128);
+        mbar_init(B.elem + b, elem_arrivals);
     }
     mbar_init(B.fin, 1);
     *B.abort_flag = 0;
@@ -206,7 +206,7 @@ k_bwd_dq_sm100(const __nv_bfloat16* __restrict__ Qg, const __nv_bfloat16* __rest
     const int64_t row0 = (int64_t)hh * N;
 
     load_rows(u0, u1, gsel + ((int64_t)hh * MB + 2 * tile) * SW, gsel + ((int64_t)hh * MB + 2 * tile + 1) * SW, wn);
-    if (threadIdx.x == 0) init_bars(B, nst, 128);     // Q, dO: one arrival per tile row
+    if (threadIdx.x == 0) init_bars(B, nst, 128, 128);   // Q, dO: one arrival per tile row
     if (warp == 1) {
         tmem_alloc(B.tmem_slot, kTmemCols);
         tmem_relinquish();
@@ -410,7 +410,7 @@ k_bwd_dkdv_sm100(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
     const int64_t row0 = (int64_t)hh * N;
 
     load_rows(u0, u1, gselT + ((int64_t)hh * MB + 2 * tile) * SW, gselT + ((int64_t)hh * MB + 2 * tile + 1) * SW, wn);
-    if (threadIdx.x == 0) init_bars(B, nst, 2);       // K, V: one arrival per stationary copy
+    if (threadIdx.x == 0) init_bars(B, nst, 2, 256);     // K, V: one arrival per stationary copy
     if (warp == 1) {
         tmem_alloc(B.tmem_slot, kTmemCols);
         tmem_relinquish();
@@ -475,8 +475,12 @@ k_bwd_dkdv_sm100(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
       }
     } else {
         regs_inc<kRegsHigh>();
-        // two elementwise warpgroups take alternate granules (warpgroup wg uses
-        // TMEM buffer wg), so one's latency hides behind the other's work
+        // Both elementwise warpgroups work on every granule, warpgroup wg on
+        // its 32 query columns (16 wg .. 16 wg + 15 of P^T / dS^T), which halves
+        // the latency from the granule's products to its dK/dV MMAs.  bf16 P^T
+        // and dS^T of warpgroup 1 overwrite fp32 columns that warpgroup 0
+        // reads, so the stores wait at a named barrier for both warpgroups'
+        // loads; every thread runs every barrier, also after a timeout.
         const int wg = (warp - 4) >> 2;
         const int sub = warp & 3, row = sub * 32 + lane, half = row >> 6;
         const uint32_t tl = tb + ((uint32_t)(sub * 32) << 16);
@@ -493,51 +497,53 @@ k_bwd_dkdv_sm100(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
             uint32_t mk = 0;
             int qrow = 0;
             if (lane == 0) walk.next(qrow, mk);
-            if (b != wg) continue;                             // the other warpgroup's granule
             mk = __shfl_sync(0xffffffffu, mk, 0);
             const bool valid = (mk >> half) & 1u;              // warp-uniform
-            const float4* nl4 = reinterpret_cast<const float4*>(xs + st * kXs);   // -lse*log2(e), 64 rows
-            const float4* nd4 = nl4 + 16;                                          // -Delta, 64 rows
-            const bool got = mbar_wait(B.prod + b, (g >> 1) & 1, B.abort_flag, dev_status) &&
-                             mbar_wait(B.fullx + st, (g / nst) & 1, B.abort_flag, dev_status);
-            if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
-            tc_fence_after();
-#pragma unroll
-            for (int hq = 0; hq < 2; ++hq) {
-                uint32_t op[16], od[16];
+            const float4* nl4 = reinterpret_cast<const float4*>(xs + st * kXs) + 8 * wg;   // -lse*log2(e)
+            const float4* nd4 = nl4 + 16;                                                   // -Delta
+            if (ok)
+                ok = __all_sync(0xffffffffu, mbar_wait(B.prod + b, (g >> 1) & 1, B.abort_flag, dev_status) &&
+                                                 mbar_wait(B.fullx + st, (g / nst) & 1, B.abort_flag, dev_status));
+            // 32 columns of S^T and of dP^T: both TMEM loads in flight before one wait
+            uint32_t sv[32], pv[32];
+            if (ok) {
+                tc_fence_after();
                 if (valid) {
-                    // 32 columns of S^T and of dP^T: both TMEM loads in flight before one wait
-                    uint32_t s[32], p[32];
-                    tmem_ld32(tl + cS + 128 * b + 32 * hq, s);
-                    tmem_ld32(tl + cP + 128 * b + 32 * hq, p);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int i4 = 0; i4 < 8; ++i4) {
-                        const float4 l4 = nl4[8 * hq + i4];
-                        const float4 d4 = nd4[8 * hq + i4];
-#pragma unroll
-                        for (int u = 0; u < 2; ++u) {
-                            const int i = 4 * i4 + 2 * u;
-                            const uint64_t nl = u ? f2pack(l4.z, l4.w) : f2pack(l4.x, l4.y);
-                            const uint64_t nd = u ? f2pack(d4.z, d4.w) : f2pack(d4.x, d4.y);
-                            float x0, x1;
-                            f2unpack(ffma2(f2pack(__uint_as_float(s[i]), __uint_as_float(s[i + 1])), sl2x2, nl), x0, x1);
-                            const float p0 = ex2(x0), p1 = ex2(x1);
-                            float d0, d1;
-                            f2unpack(fmul2(f2pack(p0, p1),
-                                           fadd2(f2pack(__uint_as_float(p[i]), __uint_as_float(p[i + 1])), nd)),
-                                     d0, d1);
-                            op[2 * i4 + u] = pack_bf16x2(p0, p1);
-                            od[2 * i4 + u] = pack_bf16x2(d0, d1);
-                        }
-                    }
-                } else {
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) { op[i] = 0u; od[i] = 0u; }
+                    tmem_ld32(tl + cS + 128 * b + 32 * wg, sv);
+                    tmem_ld32(tl + cP + 128 * b + 32 * wg, pv);
                 }
-                tmem_st16(tl + cS + 128 * b + 16 * hq, op);     // P^T over the consumed S^T columns
-                tmem_st16(tl + cP + 128 * b + 16 * hq, od);     // dS^T over the consumed dP^T columns
+                tmem_wait_ld();
             }
+            named_sync(1, 256);                                // both warpgroups hold their columns
+            if (!ok) continue;
+            uint32_t op[16], od[16];
+            if (valid) {
+#pragma unroll
+                for (int i4 = 0; i4 < 8; ++i4) {
+                    const float4 l4 = nl4[i4];
+                    const float4 d4 = nd4[i4];
+#pragma unroll
+                    for (int u = 0; u < 2; ++u) {
+                        const int i = 4 * i4 + 2 * u;
+                        const uint64_t nl = u ? f2pack(l4.z, l4.w) : f2pack(l4.x, l4.y);
+                        const uint64_t nd = u ? f2pack(d4.z, d4.w) : f2pack(d4.x, d4.y);
+                        float x0, x1;
+                        f2unpack(ffma2(f2pack(__uint_as_float(sv[i]), __uint_as_float(sv[i + 1])), sl2x2, nl), x0, x1);
+                        const float p0 = ex2(x0), p1 = ex2(x1);
+                        float d0, d1;
+                        f2unpack(fmul2(f2pack(p0, p1),
+                                       fadd2(f2pack(__uint_as_float(pv[i]), __uint_as_float(pv[i + 1])), nd)),
+                                 d0, d1);
+                        op[2 * i4 + u] = pack_bf16x2(p0, p1);
+                        od[2 * i4 + u] = pack_bf16x2(d0, d1);
+                    }
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) { op[i] = 0u; od[i] = 0u; }
+            }
+            tmem_st16(tl + cS + 128 * b + 16 * wg, op);        // P^T
+            tmem_st16(tl + cP + 128 * b + 16 * wg, od);        // dS^T
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(B.elem + b);
