@@ -23,7 +23,8 @@ EXPORTS = ("prism_query_sizes", "prism_zone_indicator", "prism_assign_shapes", "
            "prism_unpermute", "prism_block_pool_score", "prism_block_select",
            "prism_sparse_attn_fwd", "prism_sparse_attn_bwd", "prism_read_status",
            "prism_status_string", "prism_version", "prism_launch_count",
-           "prism_zone_indicator_noalloc")
+           "prism_zone_indicator_noalloc", "prism_zone_indicator_ex", "prism_assign_shapes_ex")
+GUIDANCE = {"joint": 0, "video": 1, "audio": 2}
 NOALLOC_SCRATCH_BYTES = 2 << 20
 
 
@@ -58,6 +59,8 @@ _SIGS = {
     "prism_zone_indicator": [_PROB, _P, _P, _F, _P, _P, _P, _P, _P, _SZ, _P],
     "prism_zone_indicator_noalloc": [_PROB, _P, _P, _F, _P, _P, _P, _P, _P],
     "prism_assign_shapes": [_PROB, _P, _P, _F, _F, _P, _P, _P, _P, _P, _P, _P, _P],
+    "prism_zone_indicator_ex": [_PROB, _P, _P, _F, _I, _P, _P, _P, _P, _P, _SZ, _P],
+    "prism_assign_shapes_ex": [_PROB, _P, _P, _F, _F, _I, _P, _P, _P, _P, _P, _P, _P, _P],
     "prism_permute": [_PROB, _P, _P, _P, _P],
     "prism_unpermute": [_PROB, _P, _P, _P, _P],
     "prism_block_pool_score": [_PROB, _P, _P, _P, _P, _F, _P, _P, _P, _P],
@@ -130,6 +133,15 @@ def prism_zone_indicator(prob, V, hhat, eps, g, rho, abar, zone_stats, ws, strea
         _ptr(zone_stats), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
 
 
+def prism_zone_indicator_ex(prob, V, hhat, eps, guidance, g, rho, abar, zone_stats, ws, stream=None):
+    """prism_zone_indicator with one guidance term removed: guidance is
+    "joint", "video" or "audio" (or its integer code)."""
+    code = GUIDANCE[guidance] if isinstance(guidance, str) else int(guidance)
+    _check("prism_zone_indicator_ex", lib().prism_zone_indicator_ex(
+        ctypes.byref(prob), _ptr(V), _ptr(hhat), eps, code, _ptr(g), _ptr(rho), _ptr(abar),
+        _ptr(zone_stats), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
+
+
 def prism_zone_indicator_noalloc(prob, V, hhat, eps, g, rho, abar, zone_stats, stream=None):
     """Same as prism_zone_indicator with the library's own fixed scratch array,
     for callers that cannot allocate a workspace (see include/prism.h)."""
@@ -143,6 +155,16 @@ def prism_assign_shapes(prob, g, rho, tau128, tau256, shape_id, perm, inv_perm, 
     _check("prism_assign_shapes", lib().prism_assign_shapes(
         ctypes.byref(prob), _ptr(g), _ptr(rho), tau128, tau256, _ptr(shape_id), _ptr(perm),
         _ptr(inv_perm), _ptr(blk_start), _ptr(gran_blk), _ptr(n_blk), _ptr(margin), _stream(stream)))
+
+
+def prism_assign_shapes_ex(prob, g, rho, tau128, tau256, fixed_shape, shape_id, perm, inv_perm,
+                           blk_start, gran_blk, n_blk, margin, stream=None):
+    """prism_assign_shapes with the fixed-shape baseline: fixed_shape = -1 is
+    adaptive, 0..15 gives every zone that candidate."""
+    _check("prism_assign_shapes_ex", lib().prism_assign_shapes_ex(
+        ctypes.byref(prob), _ptr(g), _ptr(rho), tau128, tau256, int(fixed_shape), _ptr(shape_id),
+        _ptr(perm), _ptr(inv_perm), _ptr(blk_start), _ptr(gran_blk), _ptr(n_blk), _ptr(margin),
+        _stream(stream)))
 
 
 def prism_permute(prob, src_raster, perm, dst_blocked, stream=None):

@@ -32,7 +32,7 @@ __global__ void __launch_bounds__(1024) k_assign_shapes(const float* __restrict_
                                                         int32_t* __restrict__ blk_start,
                                                         int32_t* __restrict__ gran_blk,
                                                         int32_t* __restrict__ n_blk,
-                                                        float* __restrict__ margin) {
+                                                        float* __restrict__ margin, int fixed) {
     __shared__ int sE[16][3];
     __shared__ int warp_tot[32];
     __shared__ int carry;
@@ -45,7 +45,8 @@ __global__ void __launch_bounds__(1024) k_assign_shapes(const float* __restrict_
     int nz = 0;
     for (int m = tid; m < Z; m += nt, ++nz) {
         const float r = rho[m];
-        const int S = r >= tau128 ? 6 : (r >= tau256 ? 7 : 8);
+        const int S = fixed >= 0 ? sE[fixed][0] + sE[fixed][1] + sE[fixed][2]   // fixed-shape baseline
+                                 : (r >= tau128 ? 6 : (r >= tau256 ? 7 : 8));
         const float l0 = log2f(g[m * 3 + 0]), l1 = log2f(g[m * 3 + 1]), l2 = log2f(g[m * 3 + 2]);
         const float common_term = ((float)S + 0.5f * (l0 + l1 + l2)) / 3.f;
         const float e0 = -0.5f * l0 + common_term, e1 = -0.5f * l1 + common_term,
@@ -60,11 +61,11 @@ __global__ void __launch_bounds__(1024) k_assign_shapes(const float* __restrict_
             if (dd < best) { second = best; best = dd; bid = id; }
             else if (dd < second) second = dd;
         }
-        shape_id[m] = (uint8_t)bid;
+        shape_id[m] = (uint8_t)(fixed >= 0 ? fixed : bid);
         myB[nz] = 1 << S;
-        if (margin) {
-            margin[m * 2 + 0] = second - best;
-            margin[m * 2 + 1] = fminf(fabsf(r - tau128), fabsf(r - tau256));
+        if (margin) {                                   // no decision is taken for a fixed shape
+            margin[m * 2 + 0] = fixed >= 0 ? INFINITY : second - best;
+            margin[m * 2 + 1] = fixed >= 0 ? INFINITY : fminf(fabsf(r - tau128), fabsf(r - tau256));
         }
     }
 
@@ -136,11 +137,12 @@ __global__ void k_build_perm(const uint8_t* __restrict__ shape_id, int H, int W,
 
 using namespace prism;
 
-extern "C" prism_status_t prism_assign_shapes(const prism_problem_t* prob, const float* g,
-                                              const float* rho, float tau128, float tau256,
-                                              uint8_t* shape_id, int32_t* perm, int32_t* inv_perm,
-                                              int32_t* blk_start, int32_t* gran_blk,
-                                              int32_t* n_blk, float* margin, cudaStream_t stream) {
+extern "C" prism_status_t prism_assign_shapes_ex(const prism_problem_t* prob, const float* g,
+                                                 const float* rho, float tau128, float tau256,
+                                                 int32_t fixed_shape, uint8_t* shape_id, int32_t* perm,
+                                                 int32_t* inv_perm, int32_t* blk_start, int32_t* gran_blk,
+                                                 int32_t* n_blk, float* margin, cudaStream_t stream) {
+    if (fixed_shape < -1 || fixed_shape > 15) return PRISM_ERR_INVALID_ARG;
     Dims d;
     prism_status_t st = make_dims(prob, &d);
     if (st != PRISM_OK) return st;
@@ -149,9 +151,18 @@ extern "C" prism_status_t prism_assign_shapes(const prism_problem_t* prob, const
         return PRISM_ERR_INVALID_ARG;
     if (!isfinite(tau128) || !isfinite(tau256) || !(tau256 <= tau128)) return PRISM_ERR_INVALID_ARG;
     k_assign_shapes<<<1, 1024, 0, stream>>>(g, rho, (int)d.Z, tau128, tau256, d.MB, (int)d.N,
-                                            shape_id, blk_start, gran_blk, n_blk, margin);
+                                            shape_id, blk_start, gran_blk, n_blk, margin, fixed_shape);
     const int thr = 256;
     k_build_perm<<<(unsigned)((d.N + thr - 1) / thr), thr, 0, stream>>>(shape_id, d.H, d.W,
                                                                          (int)d.N, perm, inv_perm);
     return launch_status(2);
+}
+
+extern "C" prism_status_t prism_assign_shapes(const prism_problem_t* prob, const float* g,
+                                              const float* rho, float tau128, float tau256,
+                                              uint8_t* shape_id, int32_t* perm, int32_t* inv_perm,
+                                              int32_t* blk_start, int32_t* gran_blk,
+                                              int32_t* n_blk, float* margin, cudaStream_t stream) {
+    return prism_assign_shapes_ex(prob, g, rho, tau128, tau256, -1, shape_id, perm, inv_perm, blk_start,
+                                  gran_blk, n_blk, margin, stream);
 }

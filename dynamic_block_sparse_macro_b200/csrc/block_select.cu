@@ -259,7 +259,7 @@ extern "C" prism_status_t prism_block_select(const prism_problem_t* prob, const 
     if (!ok_ptr(P) || !ok_ptr(blk_start) || !ok_ptr(gran_blk) || !ok_ptr(n_blk) || !ok_ptr(sel) ||
         !ok_ptr(sel_count) || !ok_ptr(gsel) || !ok_opt(gselT) || !ok_opt(margin) || !ok_ptr(dev_status))
         return PRISM_ERR_INVALID_ARG;
-    if (top_k < 1 || !(top_p > 0.f) || !isfinite(top_p)) return PRISM_ERR_INVALID_ARG;
+    if (top_k < 0 || !(top_p > 0.f) || !isfinite(top_p)) return PRISM_ERR_INVALID_ARG;
     const int64_t rowcap = d.MB < kSelectMaxRow ? d.MB : kSelectMaxRow;
     const size_t smem = (size_t)rowcap * sizeof(float);
     if (cudaFuncSetAttribute(k_block_select, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=

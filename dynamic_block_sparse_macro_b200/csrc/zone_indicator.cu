@@ -175,7 +175,9 @@ __global__ void __launch_bounds__(1024) k_zone_finalize(const float* __restrict_
                                                         float* __restrict__ g, float* __restrict__ rho,
                                                         float* __restrict__ abar,
                                                         float* __restrict__ zstat,
-                                                        float* __restrict__ vsum) {
+                                                        float* __restrict__ vsum, int guide) {
+    // guidance ablation: the video term, the audio term or both (g and rho)
+    const float wv = guide == PRISM_GUIDE_AUDIO ? 0.f : 1.f, wa = guide == PRISM_GUIDE_VIDEO ? 0.f : 1.f;
     __shared__ float rmx[32], amx[32];
     const int tid = threadIdx.x;
     float rmax = 0.f, Amax = 0.f;
@@ -220,11 +222,11 @@ __global__ void __launch_bounds__(1024) k_zone_finalize(const float* __restrict_
         const float v0 = ta > 0.f ? sa0 / ta : third, v1 = ta > 0.f ? sa1 / ta : third,
                     v2 = ta > 0.f ? sa2 / ta : third;
         const float ab = Amax > 0.f ? A / Amax : 0.f;
-        g[m * 3 + 0] = r0 + ab * v0 + eps;
-        g[m * 3 + 1] = r1 + ab * v1 + eps;
-        g[m * 3 + 2] = r2 + ab * v2 + eps;
+        g[m * 3 + 0] = wv * r0 + wa * ab * v0 + eps;
+        g[m * 3 + 1] = wv * r1 + wa * ab * v1 + eps;
+        g[m * 3 + 2] = wv * r2 + wa * ab * v2 + eps;
         const float rv = rmax > 0.f ? rr / rmax : 0.f;
-        rho[m] = fmaxf(rv, ab);
+        rho[m] = fmaxf(wv * rv, wa * ab);
         abar[m] = ab;
         if (zstat) {
             float* o = zstat + (int64_t)m * 8;
@@ -244,10 +246,12 @@ size_t zone_indicator_ws_bytes(const Dims& d) {
 
 using namespace prism;
 
-extern "C" prism_status_t prism_zone_indicator(const prism_problem_t* prob, const void* V,
-                                               const void* hhat, float eps, float* g, float* rho,
-                                               float* abar, float* zone_stats, void* ws,
-                                               size_t ws_bytes, cudaStream_t stream) {
+extern "C" prism_status_t prism_zone_indicator_ex(const prism_problem_t* prob, const void* V,
+                                                  const void* hhat, float eps, int32_t guidance, float* g,
+                                                  float* rho, float* abar, float* zone_stats, void* ws,
+                                                  size_t ws_bytes, cudaStream_t stream) {
+    if (guidance != PRISM_GUIDE_JOINT && guidance != PRISM_GUIDE_VIDEO && guidance != PRISM_GUIDE_AUDIO)
+        return PRISM_ERR_INVALID_ARG;
     Dims d;
     prism_status_t st = make_dims(prob, &d);
     if (st != PRISM_OK) return st;
@@ -274,8 +278,16 @@ extern "C" prism_status_t prism_zone_indicator(const prism_problem_t* prob, cons
                                                                astat);
     }
     k_zone_finalize<<<1, 1024, 0, stream>>>(part, astat, (int)d.Z, nchunk, 1.f / (float)d.D, eps, g,
-                                            rho, abar, zone_stats, vsum);
+                                            rho, abar, zone_stats, vsum, guidance);
     return launch_status(3);
+}
+
+extern "C" prism_status_t prism_zone_indicator(const prism_problem_t* prob, const void* V,
+                                               const void* hhat, float eps, float* g, float* rho,
+                                               float* abar, float* zone_stats, void* ws,
+                                               size_t ws_bytes, cudaStream_t stream) {
+    return prism_zone_indicator_ex(prob, V, hhat, eps, PRISM_GUIDE_JOINT, g, rho, abar, zone_stats, ws,
+                                   ws_bytes, stream);
 }
 
 // ---------------------------------------------------------------------------

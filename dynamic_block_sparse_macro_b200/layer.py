@@ -26,13 +26,15 @@ _TORCH_DT = {"f32": torch.float32, "bf16": torch.bfloat16}
 class PrismSparseAttention:
     def __init__(self, T, H, W, heads, head_dim, audio_dim=64, dtype="bf16", top_k=8, top_p=0.9,
                  eps=1e-6, tau128=0.5, tau256=0.25, scale=None, device="cuda", p_blocks=None,
-                 with_backward=True):
+                 with_backward=True, guidance="joint", fixed_shape=-1):
         self.prob = _abi.problem(T, H, W, heads, head_dim, audio_dim, dtype)
         self.sizes = _abi.query_sizes(self.prob)
         self.dtype = dtype
         self.tdt = _TORCH_DT[dtype]
         self.top_k, self.top_p = int(top_k), float(top_p)
         self.eps, self.tau128, self.tau256 = float(eps), float(tau128), float(tau256)
+        # ablations the pages compare against: one guidance term only, one fixed block shape
+        self.guidance, self.fixed_shape = guidance, int(fixed_shape)
         self.scale = float(scale) if scale is not None else 1.0 / math.sqrt(head_dim)
         self.heads, self.d = heads, head_dim
         dev = torch.device(device)
@@ -79,10 +81,11 @@ class PrismSparseAttention:
     def plan(self, V, hhat, stream=None):
         """Stages 1-2: zone indicator, shapes, permutation, block table."""
         p = self.prob
-        _abi.prism_zone_indicator(p, V, hhat, self.eps, self.g, self.rho, self.abar, self.zone_stats,
-                                  self.ws_ind, stream)
-        _abi.prism_assign_shapes(p, self.g, self.rho, self.tau128, self.tau256, self.shape_id, self.perm,
-                                 None, self.blk_start, self.gran_blk, self.n_blk, self.margin_shape, stream)
+        _abi.prism_zone_indicator_ex(p, V, hhat, self.eps, self.guidance, self.g, self.rho, self.abar,
+                                     self.zone_stats, self.ws_ind, stream)
+        _abi.prism_assign_shapes_ex(p, self.g, self.rho, self.tau128, self.tau256, self.fixed_shape,
+                                    self.shape_id, self.perm, None, self.blk_start, self.gran_blk, self.n_blk,
+                                    self.margin_shape, stream)
 
     def select(self, Q, K, V, stream=None):
         """Stages 3-5: permute Q, K, V; pooled probabilities; hybrid selection."""

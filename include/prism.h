@@ -103,6 +103,20 @@ prism_status_t prism_zone_indicator(const prism_problem_t* prob, const void* V, 
                                     float* zone_stats, void* ws, size_t ws_bytes,
                                     cudaStream_t stream);
 
+/*
+ * Stage 1 with one guidance term removed (the pages' ablations of the dual
+ * guidance; Portuguese reading guide, "Método" 1 and the ablations of its
+ * experiments).  guidance = PRISM_GUIDE_JOINT gives prism_zone_indicator;
+ * PRISM_GUIDE_VIDEO drops the audio term from both outputs that combine the
+ * two (g_d = r_{v,d} + eps, rho = rho_v); PRISM_GUIDE_AUDIO drops the video
+ * term (g_d = abar*vhat_{a,d} + eps, rho = abar).  abar and zone_stats are as
+ * in prism_zone_indicator.  Any other guidance value: PRISM_ERR_INVALID_ARG.
+ */
+typedef enum { PRISM_GUIDE_JOINT = 0, PRISM_GUIDE_VIDEO = 1, PRISM_GUIDE_AUDIO = 2 } prism_guidance_t;
+prism_status_t prism_zone_indicator_ex(const prism_problem_t* prob, const void* V, const void* hhat,
+                                       float eps, int32_t guidance, float* g, float* rho, float* abar,
+                                       float* zone_stats, void* ws, size_t ws_bytes, cudaStream_t stream);
+
 /* Size of the library-owned scratch array behind prism_zone_indicator_noalloc. */
 #define PRISM_NOALLOC_SCRATCH_BYTES (2u << 20)
 
@@ -149,6 +163,20 @@ prism_status_t prism_assign_shapes(const prism_problem_t* prob, const float* g, 
                                    int32_t* n_blk, float* margin, cudaStream_t stream);
 
 /*
+ * Stage 2 with the fixed-shape block-sparse baseline the pages compare
+ * against: fixed_shape = -1 is prism_assign_shapes; fixed_shape in [0, 15]
+ * gives every zone that candidate (ids as above: 0-6 volume 64, 7-12 volume
+ * 128, 13-15 volume 256), ignoring g, rho and the thresholds; margin (if
+ * given) is then +inf (no decision is taken).  Outside [-1, 15]:
+ * PRISM_ERR_INVALID_ARG.
+ */
+prism_status_t prism_assign_shapes_ex(const prism_problem_t* prob, const float* g, const float* rho,
+                                      float tau128, float tau256, int32_t fixed_shape, uint8_t* shape_id,
+                                      int32_t* perm, int32_t* inv_perm, int32_t* blk_start,
+                                      int32_t* gran_blk, int32_t* n_blk, float* margin,
+                                      cudaStream_t stream);
+
+/*
  * Stage 3 — gather raster tokens into block order and head-major layout
  * (news page, "工作原理" step 4, and its inverse that restores the layout).
  *   prism_permute:   dst_blocked[h][p][:] = src_raster[perm[p]][h][:]
@@ -175,7 +203,9 @@ prism_status_t prism_block_pool_score(const prism_problem_t* prob, const void* Q
  * Stage 5 — hybrid selection S_i = Top-k(P_i, k) U Top-p(P_i, p) ("Método" 3).
  * Both are prefixes of the order (P desc, j asc): Top-p is the shortest prefix
  * whose sum reaches p (all blocks if p >= 1 or it never does), so S_i is the
- * first max(min(k, n_blk), n_p) blocks.
+ * first max(min(k, n_blk), n_p) blocks.  k >= 0 and 0 < p: k = 0 is the
+ * Top-p-only ablation and a tiny p (n_p = 1) the Top-k-only one; k < 0 or
+ * p <= 0 (or not finite): PRISM_ERR_INVALID_ARG.
  *   sel       [heads][max_blocks][sel_words] uint32 bitmask, bit j of row i
  *   sel_count [heads][max_blocks] int32 (|S_i|; rows past n_blk are 0)
  *   gsel      [heads][N/64][sel_words] uint32: the same selection at granule

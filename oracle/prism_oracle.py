@@ -65,7 +65,7 @@ TIE_TOL = 1e-12               # R9
 __all__ = [
     "ZONE", "TAU_128", "TAU_256", "EPS", "VOLUMES",
     "candidate_shapes", "zone_indicator", "block_volume", "optimal_log_edges",
-    "assign_shapes", "build_permutation", "permute", "unpermute",
+    "assign_shapes", "assign_shapes_fixed", "build_permutation", "permute", "unpermute",
     "block_pool_score", "block_select", "sparse_attention_fwd",
     "sparse_attention_bwd", "run_layer",
 ]
@@ -120,8 +120,13 @@ def _directional_variance(Xz):
     return np.stack(sig, axis=-1), mu
 
 
-def zone_indicator(V, hhat, T, H, W, eps=EPS):
+def zone_indicator(V, hhat, T, H, W, eps=EPS, guidance="joint"):
     """Per-zone g_d(m), rho(m), abar(m) and the statistics they come from.
+
+    guidance: "joint" (the method), or the single-guidance ablations the
+    pages compare against (R19): "video" keeps only the video term of every
+    output that combines the two (g_d = r_{v,d} + eps, rho = rho_v), "audio"
+    only the audio term (g_d = abar * vhat_{a,d} + eps, rho = abar).
 
     V: raster [N, D] (or [N, heads, d], flattened to D = heads*d, R1), any float
     dtype (converted to fp64 one temporal slab of zones at a time).
@@ -156,10 +161,14 @@ def zone_indicator(V, hhat, T, H, W, eps=EPS):
     abar = A / Amax if Amax > 0 else np.zeros_like(A)
     vhat = _ratio(sig_a)
 
-    g = r_v + abar[..., None] * vhat + eps
+    if guidance not in ("joint", "video", "audio"):
+        raise ValueError(guidance)
+    use_v = 0.0 if guidance == "audio" else 1.0
+    use_a = 0.0 if guidance == "video" else 1.0
+    g = use_v * r_v + use_a * abar[..., None] * vhat + eps
     rmax = rho_raw.max()
     rho_v = rho_raw / rmax if rmax > 0 else np.zeros_like(rho_raw)
-    rho = np.maximum(rho_v, abar)
+    rho = np.maximum(use_v * rho_v, use_a * abar)
 
     Z = ZT * ZH * ZW
     return {
@@ -184,6 +193,14 @@ def optimal_log_edges(g, B):
     lg = np.log2(np.asarray(g, dtype=np.float64))
     S = np.log2(np.asarray(B, dtype=np.float64))
     return -0.5 * lg + ((S + 0.5 * lg.sum(axis=-1)) / 3.0)[..., None]
+
+
+def assign_shapes_fixed(Z, fixed_shape):
+    """The fixed-shape block-sparse baseline (R20): every zone takes candidate
+    `fixed_shape` (the id order of candidate_shapes), whatever g and rho."""
+    edges, vol = candidate_shapes()
+    sid = np.full(Z, int(fixed_shape), dtype=np.int64)
+    return {"shape_id": sid, "edges": edges[sid], "B": vol[sid].astype(np.int64)}
 
 
 def assign_shapes(g, rho, tau128=TAU_128, tau256=TAU_256):

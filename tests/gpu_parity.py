@@ -45,26 +45,28 @@ def bits(t: torch.Tensor) -> np.ndarray:
     return t.detach().cpu().contiguous().view(it).numpy()
 
 
-def run_gpu(cfg, x, top_k=None, top_p=None, backward=True):
+def run_gpu(cfg, x, top_k=None, top_p=None, backward=True, guidance="joint", fixed_shape=-1):
     mod = PrismSparseAttention(cfg.T, cfg.H, cfg.W, cfg.heads, cfg.head_dim, cfg.audio_dim,
-                               cfg.dtype, top_k or cfg.top_k, cfg.top_p if top_p is None else top_p)
+                               cfg.dtype, cfg.top_k if top_k is None else top_k, cfg.top_p if top_p is None else top_p,
+                               guidance=guidance, fixed_shape=fixed_shape)
     O = mod.forward(x["Q"], x["K"], x["V"], x["hhat"])
     grads = mod.backward(x["dO"]) if backward else None
     torch.cuda.synchronize()
     return mod, O, grads
 
 
-def check_layer(cfg, x, top_k=None, top_p=None, backward=True, heads=None, grad_floor=1e-4):
+def check_layer(cfg, x, top_k=None, top_p=None, backward=True, heads=None, grad_floor=1e-4,
+                guidance="joint", fixed_shape=-1):
     """Run the GPU layer and check every stage; returns a report dict."""
-    top_k = top_k or cfg.top_k
+    top_k = cfg.top_k if top_k is None else top_k
     top_p = cfg.top_p if top_p is None else top_p
-    mod, O, grads = run_gpu(cfg, x, top_k, top_p, backward)
+    mod, O, grads = run_gpu(cfg, x, top_k, top_p, backward, guidance, fixed_shape)
     rep = {}
     T, H, W = cfg.T, cfg.H, cfg.W
     Vh, hh = host(x["V"]), host(x["hhat"])
 
     # stage 1: indicator (fp32 on the GPU vs fp64 oracle)
-    ind = orc.zone_indicator(Vh, hh, T, H, W)
+    ind = orc.zone_indicator(Vh, hh, T, H, W, guidance=guidance)
     g, rho, abar = (mod.g.cpu().double().numpy(), mod.rho.cpu().double().numpy(),
                     mod.abar.cpu().double().numpy())
     zs = mod.zone_stats.cpu().double().numpy()
@@ -77,15 +79,20 @@ def check_layer(cfg, x, top_k=None, top_p=None, backward=True, heads=None, grad_
 
     # stage 2: shapes, teacher-forced on the GPU's g / rho, and end to end
     sid = mod.shape_id.cpu().numpy().astype(np.int64)
-    tf = orc.assign_shapes(g, rho)
-    margin = np.minimum(tf["margin_shape"], tf["margin_volume"])
-    bad = sid != tf["shape_id"]
-    assert (margin[bad] < NEAR_TIE).all(), (np.nonzero(bad), margin[bad])
-    e2e = orc.assign_shapes(ind["g"], ind["rho"])
-    m2 = np.minimum(e2e["margin_shape"], e2e["margin_volume"])
-    bad2 = sid != e2e["shape_id"]
-    assert (m2[bad2] < NEAR_TIE).all()
-    rep["shape_near_ties"] = int(bad2.sum())
+    if fixed_shape >= 0:                              # the fixed-shape baseline takes no decision
+        tf = orc.assign_shapes_fixed(len(sid), fixed_shape)
+        assert np.array_equal(sid, tf["shape_id"])
+        rep["shape_near_ties"] = 0
+    else:
+        tf = orc.assign_shapes(g, rho)
+        margin = np.minimum(tf["margin_shape"], tf["margin_volume"])
+        bad = sid != tf["shape_id"]
+        assert (margin[bad] < NEAR_TIE).all(), (np.nonzero(bad), margin[bad])
+        e2e = orc.assign_shapes(ind["g"], ind["rho"])
+        m2 = np.minimum(e2e["margin_shape"], e2e["margin_volume"])
+        bad2 = sid != e2e["shape_id"]
+        assert (m2[bad2] < NEAR_TIE).all()
+        rep["shape_near_ties"] = int(bad2.sum())
     rep["volume_mix"] = {int(b): int((tf["B"] == b).sum()) for b in (64, 128, 256)}
 
     # permutation and block table: bit-exact from the GPU's shapes

@@ -75,8 +75,17 @@ def test_bad_pointers_rejected_before_launch(L):
     # in place is refused
     assert L.prism_permute(ctypes.byref(p), fake, fake, fake, None) == 1
     # bad scalars
-    assert L.prism_block_select(ctypes.byref(p), fake, fake, fake, fake, 0, 0.9, fake, fake, fake, None, None,
+    assert L.prism_block_select(ctypes.byref(p), fake, fake, fake, fake, -1, 0.9, fake, fake, fake, None, None,
                                 fake, None) == 1
+    assert L.prism_block_select(ctypes.byref(p), fake, fake, fake, fake, 0, 0.0, fake, fake, fake, None, None,
+                                fake, None) == 1
+    # ablation options out of range
+    assert L.prism_zone_indicator_ex(ctypes.byref(p), fake, fake, 1e-6, 3, fake, fake, fake, None, fake, 1 << 30,
+                                     None) == 1
+    assert L.prism_assign_shapes_ex(ctypes.byref(p), fake, fake, 0.5, 0.25, 16, fake, fake, None, fake, fake,
+                                    fake, None, None) == 1
+    assert L.prism_assign_shapes_ex(ctypes.byref(p), fake, fake, 0.5, 0.25, -2, fake, fake, None, fake, fake,
+                                    fake, None, None) == 1
     assert L.prism_block_select(ctypes.byref(p), fake, fake, fake, fake, 4, float("nan"), fake, fake, fake, None,
                                 None, fake, None) == 1
     # granule-level selection is required

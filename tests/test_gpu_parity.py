@@ -70,6 +70,31 @@ def test_top_k_only():
     assert rep["density"] > 0
 
 
+@pytest.mark.parametrize("guidance", ["video", "audio"])
+def test_single_guidance_ablation(guidance):
+    # the pages' ablations of the dual guidance: g and rho from one term only
+    from gpu_parity import check_layer
+    cfg = get_config("tiny")
+    check_layer(cfg, _inputs(cfg), guidance=guidance)
+
+
+@pytest.mark.parametrize("fixed_shape", [3, 10, 14])
+def test_fixed_shape_baseline(fixed_shape):
+    # the fixed-shape block-sparse baseline: one candidate (64, 128 or 256 tokens) everywhere
+    from gpu_parity import check_layer
+    cfg = get_config("tiny")
+    rep = check_layer(cfg, _inputs(cfg), fixed_shape=fixed_shape)
+    vol = {3: 64, 10: 128, 14: 256}[fixed_shape]
+    assert rep["volume_mix"][vol] == cfg.n_tokens // 512
+
+
+def test_top_p_only():
+    from gpu_parity import check_layer
+    cfg = get_config("tiny", heads=1)
+    rep = check_layer(cfg, _inputs(cfg), top_k=0, top_p=0.5)
+    assert rep["density"] > 0
+
+
 def test_degenerate_constant_video_silent_audio():
     # constant V and hhat = 0: zero variances -> r = 1/3, abar = 0, rho = 0 -> B = 256 everywhere
     from gpu_parity import check_layer

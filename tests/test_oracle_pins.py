@@ -113,6 +113,54 @@ def test_indicator_audio_guidance():
     np.testing.assert_array_equal(ind2["A"], ind["A"])
 
 
+def test_indicator_single_guidance_ablations():
+    # zone 0: flat video (zero variances: r = 1/3 each, rho_v = 0, R6) with an audio ramp along T
+    # (vhat = (1, 0, 0), abar = 1); zones 1, 2: random video, silent audio (abar = 0, vhat = 1/3)
+    T, H, W = 8, 8, 24
+    t, h, w = _grid(T, H, W)
+    hhat = np.zeros((len(t), 2))
+    inz0 = w < 8
+    hhat[inz0, 0] = t[inz0] + 1.0
+    V = np.random.default_rng(3).normal(size=(len(t), 4))
+    V[inz0] = -0.5
+    joint = orc.zone_indicator(V, hhat, T, H, W)
+    vid = orc.zone_indicator(V, hhat, T, H, W, guidance="video")
+    aud = orc.zone_indicator(V, hhat, T, H, W, guidance="audio")
+    e = orc.EPS
+    # video only: the flat zone keeps the isotropic 1/3 and rho_v = 0 (its loud audio is ignored)
+    np.testing.assert_allclose(vid["g"][0], 1 / 3 + e, atol=1e-15)
+    assert vid["rho"][0] == 0.0 and joint["rho"][0] == 1.0
+    # audio only: the flat zone follows the audio ramp, silent zones get only eps
+    np.testing.assert_allclose(aud["g"][0], [1 + e, e, e], atol=1e-15)
+    np.testing.assert_allclose(aud["g"][1:], e, atol=1e-18)
+    np.testing.assert_array_equal(aud["rho"], [1.0, 0.0, 0.0])
+    # silent zones: the video-only indicator equals the joint one (abar = 0 there)
+    np.testing.assert_array_equal(vid["g"][1:], joint["g"][1:])
+    np.testing.assert_array_equal(vid["rho"][1:], joint["rho"][1:])
+    # abar and the statistics do not depend on the ablation
+    np.testing.assert_array_equal(vid["abar"], joint["abar"])
+    np.testing.assert_array_equal(aud["sigma2_v"], joint["sigma2_v"])
+    with pytest.raises(ValueError):
+        orc.zone_indicator(V, hhat, T, H, W, guidance="both")
+
+
+@pytest.mark.parametrize("fixed", [0, 6, 7, 12, 13, 15])
+def test_fixed_shape_baseline_tiles_every_zone(fixed):
+    # the fixed-shape baseline: every zone cut into 512/B boxes of the one candidate
+    T, H, W = 16, 8, 16
+    Z = (T // 8) * (H // 8) * (W // 8)
+    edges, vol = orc.candidate_shapes()
+    fx = orc.assign_shapes_fixed(Z, fixed)
+    assert (fx["shape_id"] == fixed).all() and (fx["B"] == vol[fixed]).all()
+    perm, bs = orc.build_permutation(fx["shape_id"], T, H, W)
+    assert len(bs) - 1 == Z * 512 // int(vol[fixed])
+    for b in range(len(bs) - 1):
+        toks = perm[bs[b]:bs[b + 1]]
+        t, h, w = toks // (H * W), (toks // W) % H, toks % W
+        ext = (t.max() - t.min() + 1, h.max() - h.min() + 1, w.max() - w.min() + 1)
+        assert ext == tuple(edges[fixed]) and len(toks) == int(np.prod(edges[fixed]))
+
+
 def test_indicator_brute_force_loops():
     # scalar loops straight from the definitions on a 8x8x16 grid, 3 channels
     T, H, W = 8, 8, 16
