@@ -67,7 +67,7 @@ __all__ = [
     "candidate_shapes", "zone_indicator", "block_volume", "optimal_log_edges",
     "assign_shapes", "assign_shapes_fixed", "build_permutation", "permute", "unpermute",
     "block_pool_score", "block_select", "sparse_attention_fwd",
-    "sparse_attention_bwd", "run_layer",
+    "sparse_attention_bwd", "sparse_attention_bwd_keys", "run_layer",
 ]
 
 
@@ -462,6 +462,45 @@ def sparse_attention_bwd(Qb, Kb, Vb, dOb, blk_start, sel, scale=None, heads=None
             dK[a, r0:r1] = gK[r0:r1]
             dV[a, r0:r1] = gV[r0:r1]
     return dQ, dK, dV
+
+
+def sparse_attention_bwd_keys(Qb, Kb, Vb, dOb, blk_start, sel, lse, O, scale=None, heads=None, k_blocks=()):
+    """dK, dV of the sampled key blocks from given per-row LSE and O (teacher
+    forcing: the forward's LSE and O are taken as known, so that no query row
+    has to be re-normalised over its whole key set).  Same gradients as
+    sparse_attention_bwd [ZH-FAQ4]:
+      P_ij = exp(s_ij - lse_i), Delta_i = dO_i . O_i,
+      dV_j = sum_i P_ij dO_i,  dK_j = scale sum_i P_ij (dO_i . V_j - Delta_i) Q_i
+    over the query rows i whose block selected the block of key j.
+    lse: [h_sel, N], O: [h_sel, N, d] (rows of the heads in ``heads``).
+    Returns (dK, dV) blocked [h_sel, N, d] in fp64, NaN outside the sample."""
+    Qb, Kb, Vb, dOb = (np.asarray(x) for x in (Qb, Kb, Vb, dOb))
+    hs = list(range(Qb.shape[0])) if heads is None else list(heads)
+    d = Qb.shape[-1]
+    N = Qb.shape[1]
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    dK = np.full((len(hs), N, d), np.nan)
+    dV = np.full((len(hs), N, d), np.nan)
+    for a, hh in enumerate(hs):
+        selh = np.asarray(sel[hh])
+        for j in k_blocks:
+            k0, k1 = blk_start[j], blk_start[j + 1]
+            Kj = Kb[hh, k0:k1].astype(np.float64)
+            Vj = Vb[hh, k0:k1].astype(np.float64)
+            gK = np.zeros((k1 - k0, d))
+            gV = np.zeros((k1 - k0, d))
+            for i in np.nonzero(selh[:, j])[0]:
+                r0, r1 = blk_start[i], blk_start[i + 1]
+                q = Qb[hh, r0:r1].astype(np.float64)
+                do = dOb[hh, r0:r1].astype(np.float64)
+                P = np.exp(q @ Kj.T * scale - np.asarray(lse[a, r0:r1], dtype=np.float64)[:, None])
+                delta = (do * np.asarray(O[a, r0:r1], dtype=np.float64)).sum(axis=-1, keepdims=True)
+                dS = P * (do @ Vj.T - delta)
+                gV += P.T @ do
+                gK += (dS.T @ q) * scale
+            dK[a, k0:k1] = gK
+            dV[a, k0:k1] = gV
+    return dK, dV
 
 
 # --------------------------------------------------------------------------

@@ -116,6 +116,19 @@ def test_sampled_equals_full():
     assert np.isnan(sk[0, bs[0]:bs[1]]).all()
 
 
+def test_key_block_gradients_from_known_lse_and_o():
+    # teacher-forced dK, dV of sampled key blocks equal the full backward (itself pinned
+    # against torch autograd and finite differences) when given the forward's LSE and O
+    Q, K, V, dO, bs, sel = _case(8)
+    O, lse = orc.sparse_attention_fwd(Q, K, V, bs, sel)
+    dQ, dK, dV = orc.sparse_attention_bwd(Q, K, V, dO, bs, sel)
+    sk, sv = orc.sparse_attention_bwd_keys(Q, K, V, dO, bs, sel, lse[[1]], O[[1]], heads=[1], k_blocks=[0, 2, 4])
+    for j in (0, 2, 4):
+        np.testing.assert_allclose(sk[0, bs[j]:bs[j + 1]], dK[1, bs[j]:bs[j + 1]], rtol=1e-12, atol=1e-14)
+        np.testing.assert_allclose(sv[0, bs[j]:bs[j + 1]], dV[1, bs[j]:bs[j + 1]], rtol=1e-12, atol=1e-14)
+    assert np.isnan(sk[0, bs[1]:bs[2]]).all()
+
+
 def test_unselected_keys_get_zero_gradient():
     Q, K, V, dO, bs, sel = _case(7)
     sel[:, :, 2] = False                                  # nobody attends key block 2
