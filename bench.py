@@ -36,6 +36,11 @@ from dynamic_block_sparse_macro_b200.configs import get_config  # noqa: E402
 
 METRIC = "sparse attn fwd+bwd ms/layer & TFLOP/s on selected blocks, 2K grid (295k tok)"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# DRAM bytes (read + write) of one backward call on the 2K layer with 24 heads, from an ncu
+# capture of the backward kernels on 4 heads scaled by 6 (their per-head working set is the
+# same) plus the Delta kernel's algorithmic bytes: profiles/bwd_kernels_2k_4heads.txt.
+# Only valid for the kernels as they were captured; None elsewhere.
+BWD_DRAM_BYTES = {("2k", 24): 31.3e9}
 
 
 def load_peaks():
@@ -275,6 +280,7 @@ def bench_prism(args, cfg, rank, world, local_rank):
     bwd_ach = 2.5 * fl["F_fwd"] / (stage_ms["attn_bwd"] * 1e-3) / 1e12
     dom = "attn_bwd" if stage_ms["attn_bwd"] >= stage_ms["attn_fwd"] else "attn_fwd"
     ach = bwd_ach if dom == "attn_bwd" else fwd_ach
+    traffic = BWD_DRAM_BYTES.get((cfg.name, cfg.heads)) if dom == "attn_bwd" and not args.dense else None
     peak = peaks["bf16_tflops_sustained"]
     res = {
         "metric": METRIC, "value": round(tflops, 3), "unit": "TFLOP/s", "n_gpus": world,
@@ -291,7 +297,7 @@ def bench_prism(args, cfg, rank, world, local_rank):
         "selection": {k: (round(v, 6) if isinstance(v, float) else v) for k, v in fl.items()},
         "roofline": {"kernel": "prism_sparse_attn_bwd" if dom == "attn_bwd" else "prism_sparse_attn_fwd",
                      "bound": "tensor", "achieved": round(ach, 3), "peak": peak, "unit": "TFLOP/s",
-                     "frac": round(ach / peak, 4), "traffic": None,
+                     "frac": round(ach / peak, 4), "traffic": traffic,
                      "peak_source": f"{peaks['source']} bf16_tflops_sustained"},
         "gpu_launches": int(launches),
         "clocks": clk,

@@ -8,7 +8,8 @@
 // p (everything if p >= 1 or it never does), so S_i is the longer prefix,
 // max(min(k, n_blk), n_p) blocks.
 //
-// k_block_select   one CTA per (row, head), no sort.  For P >= 0 the float bit
+// k_block_select   one warp per (row, head) for rows of up to 4096 blocks, one
+//                  256-thread CTA per row above that; no sort.  For P >= 0 the float bit
 //                  pattern orders like the value, so thresholds are found by
 //                  binary search over bit patterns with block reductions over
 //                  the row held in shared memory:
@@ -17,7 +18,10 @@
 //                         at v* that reach p),
 //                    v_n = largest t with #{P_j >= t} >= n  (n-th value),
 //                  then S_i = {P > v_n} plus the lowest-index ties at v_n.
-//                  All reductions run in a fixed order (deterministic).
+//                  All reductions run in a fixed order (deterministic).  Every
+//                  search step is a pass over the row and a reduction, so the
+//                  warp form (shuffles, no block barrier) does the same work
+//                  in a fraction of the time.
 // k_sel_expand     granule-level view of the selection for the attention
 //                  kernels; k_bit_transpose its key-major transpose.
 #include "common.cuh"
@@ -26,6 +30,8 @@ namespace prism {
 
 constexpr int kSelectThreads = 256;
 constexpr int kSelectMaxRow = 16384;    // P values of a row held in shared memory
+constexpr int kWarpRowMax = 4096;       // rows up to this many blocks: one warp each
+constexpr int kWarpRowsPerCta = 4;
 
 struct SelRed {
     float f[kSelectThreads / 32];
@@ -54,6 +60,13 @@ __device__ __forceinline__ int sel_count_i(int v, SelRed& r) {
     for (int w = 0; w < kSelectThreads / 32; ++w) s += r.i[w];
     return s;
 }
+// the same reductions over one warp (butterfly: every lane gets the result)
+__device__ __forceinline__ int warp_sum_i(int v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
 __device__ __forceinline__ float sel_max(float v, SelRed& r) {
     v = warp_max(v);
     __syncthreads();
@@ -65,20 +78,28 @@ __device__ __forceinline__ float sel_max(float v, SelRed& r) {
     return s;
 }
 
+// TPR threads per row: 32 (one warp per row, kWarpRowsPerCta rows per CTA)
+// or kSelectThreads (one CTA per row); each form leaves the other's rows alone.
+template <int TPR>
 __global__ void __launch_bounds__(kSelectThreads) k_block_select(const float* __restrict__ P,
                                                                  const int32_t* __restrict__ n_blk, int64_t MB,
-                                                                 int SW, int top_k, float top_p,
+                                                                 int SW, int rowcap, int top_k, float top_p,
                                                                  uint32_t* __restrict__ sel,
                                                                  int32_t* __restrict__ sel_count,
                                                                  float* __restrict__ margin,
                                                                  uint32_t* __restrict__ dev_status) {
-    extern __shared__ float row[];
+    constexpr bool kWarp = TPR == 32;
+    extern __shared__ float smem_rows[];
     __shared__ SelRed red;
-    const int i = blockIdx.x, hh = blockIdx.y, tid = threadIdx.x;
     const int nb = *n_blk;
+    if (kWarp ? nb > kWarpRowMax : nb <= kWarpRowMax) return;      // the other form's rows
+    const int tid = kWarp ? (threadIdx.x & 31) : threadIdx.x;
+    const int i = kWarp ? blockIdx.x * kWarpRowsPerCta + (threadIdx.x >> 5) : blockIdx.x, hh = blockIdx.y;
+    if (kWarp && i >= MB) return;                                   // warp-uniform
+    float* row = smem_rows + (kWarp ? (threadIdx.x >> 5) * rowcap : 0);
     uint32_t* srow = sel + ((int64_t)hh * MB + i) * SW;
     if (i >= nb || nb > kSelectMaxRow) {
-        for (int w = tid; w < SW; w += blockDim.x) srow[w] = 0u;
+        for (int w = tid; w < SW; w += TPR) srow[w] = 0u;
         if (tid == 0) {
             sel_count[(int64_t)hh * MB + i] = 0;
             if (margin) margin[(int64_t)hh * MB + i] = INFINITY;
@@ -87,22 +108,23 @@ __global__ void __launch_bounds__(kSelectThreads) k_block_select(const float* __
         return;
     }
     const float* prow = P + ((int64_t)hh * nb + i) * nb;
-    for (int j = tid; j < nb; j += blockDim.x) row[j] = prow[j];
-    __syncthreads();
+    for (int j = tid; j < nb; j += TPR) row[j] = prow[j];
+    if (kWarp) __syncwarp();
+    else __syncthreads();
 
     // sum and count of {P >= t}, {P > t}, {P == t} over the row
     auto sum_ge = [&](uint32_t tb) {
         float s = 0.f;
-        for (int j = tid; j < nb; j += blockDim.x) {
+        for (int j = tid; j < nb; j += TPR) {
             const float x = row[j];
             if (__float_as_uint(x) >= tb) s += x;
         }
-        return sel_sum(s, red);
+        return kWarp ? warp_sum(s) : sel_sum(s, red);
     };
     auto count_ge = [&](uint32_t tb) {
         int c = 0;
-        for (int j = tid; j < nb; j += blockDim.x) c += __float_as_uint(row[j]) >= tb;
-        return sel_count_i(c, red);
+        for (int j = tid; j < nb; j += TPR) c += __float_as_uint(row[j]) >= tb;
+        return kWarp ? warp_sum_i(c) : sel_count_i(c, red);
     };
 
     const int n_k = min(top_k, nb);
@@ -178,9 +200,9 @@ __global__ void __launch_bounds__(kSelectThreads) k_block_select(const float* __
     if (n < nb) {
         const int c_ge = count_ge(vb);
         float below = -INFINITY;
-        for (int j = tid; j < nb; j += blockDim.x)
+        for (int j = tid; j < nb; j += TPR)
             if (__float_as_uint(row[j]) < vb) below = fmaxf(below, row[j]);
-        below = sel_max(below, red);
+        below = kWarp ? warp_max(below) : sel_max(below, red);
         gap_o = c_ge > n ? 0.f : __uint_as_float(vb) - below;
     }
     if (tid == 0) {
@@ -260,17 +282,25 @@ extern "C" prism_status_t prism_block_select(const prism_problem_t* prob, const 
         !ok_ptr(sel_count) || !ok_ptr(gsel) || !ok_opt(gselT) || !ok_opt(margin) || !ok_ptr(dev_status))
         return PRISM_ERR_INVALID_ARG;
     if (top_k < 0 || !(top_p > 0.f) || !isfinite(top_p)) return PRISM_ERR_INVALID_ARG;
-    const int64_t rowcap = d.MB < kSelectMaxRow ? d.MB : kSelectMaxRow;
-    const size_t smem = (size_t)rowcap * sizeof(float);
-    if (cudaFuncSetAttribute(k_block_select, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-        cudaSuccess)
+    // n_blk is known on the device only: both forms are launched and each
+    // handles the rows of its own size class (the other exits at once)
+    const int rowcap = (int)(d.MB < kSelectMaxRow ? d.MB : kSelectMaxRow);
+    const int wrowcap = (int)(d.MB < kWarpRowMax ? d.MB : kWarpRowMax);
+    const size_t smem = (size_t)rowcap * sizeof(float), wsmem = (size_t)kWarpRowsPerCta * wrowcap * sizeof(float);
+    if (cudaFuncSetAttribute(k_block_select<kSelectThreads>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem) != cudaSuccess ||
+        cudaFuncSetAttribute(k_block_select<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)wsmem) !=
+            cudaSuccess)
         return PRISM_ERR_CUDA;
-    k_block_select<<<dim3((unsigned)d.MB, (unsigned)d.heads), kSelectThreads, smem, stream>>>(
-        P, n_blk, d.MB, (int)d.SW, top_k, top_p, sel, sel_count, margin, dev_status);
+    k_block_select<32><<<dim3((unsigned)((d.MB + kWarpRowsPerCta - 1) / kWarpRowsPerCta), (unsigned)d.heads),
+                         32 * kWarpRowsPerCta, wsmem, stream>>>(P, n_blk, d.MB, (int)d.SW, wrowcap, top_k, top_p,
+                                                                sel, sel_count, margin, dev_status);
+    k_block_select<kSelectThreads><<<dim3((unsigned)d.MB, (unsigned)d.heads), kSelectThreads, smem, stream>>>(
+        P, n_blk, d.MB, (int)d.SW, rowcap, top_k, top_p, sel, sel_count, margin, dev_status);
     k_sel_expand<<<dim3((unsigned)d.MB, (unsigned)d.heads), 128, (size_t)d.SW * 4, stream>>>(
         sel, blk_start, gran_blk, n_blk, d.MB, (int)d.SW, gsel);
     if (gselT)
         k_bit_transpose<<<dim3((unsigned)d.SW, (unsigned)((d.SW + 7) / 8), (unsigned)d.heads), 256, 0, stream>>>(
             gsel, d.MB, (int)d.SW, gselT);
-    return launch_status(gselT ? 3 : 2);
+    return launch_status(gselT ? 4 : 3);
 }

@@ -29,14 +29,17 @@ def _f64(t):
     return t.detach().float().cpu().numpy().astype(np.float64)
 
 
-@pytest.mark.parametrize("name", ["720p", "1080p", "2k"])
-def test_full_size_sampled(name):
+@pytest.mark.parametrize("name,fixed", [("720p", -1), ("1080p", -1), ("2k", -1), ("2k", 3)])
+def test_full_size_sampled(name, fixed):
+    # ("2k", 3): the fixed-shape baseline with 64-token blocks everywhere, 4608 blocks a row,
+    # which takes the one-CTA-per-row selection (rows of more than 4096 blocks)
     cfg = get_config(name)
     T, H, W = cfg.T, cfg.H, cfg.W
     N, Z = cfg.n_tokens, cfg.n_tokens // 512
     dev = torch.device("cuda")
     x = inputs.make_inputs(cfg, "cuda")
-    mod = PrismSparseAttention(T, H, W, cfg.heads, cfg.head_dim, cfg.audio_dim, cfg.dtype, cfg.top_k, cfg.top_p)
+    mod = PrismSparseAttention(T, H, W, cfg.heads, cfg.head_dim, cfg.audio_dim, cfg.dtype, cfg.top_k, cfg.top_p,
+                               fixed_shape=fixed)
     O = mod.forward(x["Q"], x["K"], x["V"], x["hhat"])
     grads = mod.backward(x["dO"])
     torch.cuda.synchronize()
@@ -67,10 +70,13 @@ def test_full_size_sampled(name):
 
     # stage 2: every zone's shape (teacher-forced), the permutation and the block table bit-exact
     sid = mod.shape_id.cpu().numpy().astype(np.int64)
-    tf = orc.assign_shapes(g, rho)
-    margin = np.minimum(tf["margin_shape"], tf["margin_volume"])
-    bad = sid != tf["shape_id"]
-    assert (margin[bad] < NEAR_TIE).all()
+    if fixed >= 0:
+        assert (sid == fixed).all()
+    else:
+        tf = orc.assign_shapes(g, rho)
+        margin = np.minimum(tf["margin_shape"], tf["margin_volume"])
+        bad = sid != tf["shape_id"]
+        assert (margin[bad] < NEAR_TIE).all()
     perm, bs = orc.build_permutation(sid, T, H, W)
     nb = mod.num_blocks()
     assert nb == len(bs) - 1
