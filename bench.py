@@ -114,6 +114,25 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------- helpers
+# ---------------------------------------------------------------- ranks
+def max_over_ranks(values, device):
+    """Element-wise max of per-rank timings over all ranks (identity with one rank).
+
+    Every rank must call it at the same point (it is a collective)."""
+    if not (torch.distributed.is_available() and torch.distributed.is_initialized()):
+        return [float(v) for v in values]
+    if torch.distributed.get_world_size() == 1:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], device=device, dtype=torch.float64)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def job_tflops(world, flops_per_rank, ms):
+    """Whole-job throughput: every rank runs one replica of the layer in `ms` (the max over ranks)."""
+    return world * flops_per_rank / (ms * 1e-3) / 1e12
+
+
 def unpack_sel_dev(words: torch.Tensor, nb: int) -> torch.Tensor:
     """[h, MB, SW] int32 bitmask -> bool [h, nb, nb] on the device."""
     w = words[:, :nb, :].to(torch.int64) & 0xFFFFFFFF
@@ -262,13 +281,10 @@ def bench_prism(args, cfg, rank, world, local_rank):
     stage_ms = {n: float(np.mean([p[n] for p in per])) for n in StepTimer.NAMES}
     attn_ms = stage_ms["attn_fwd"] + stage_ms["attn_bwd"]
     status = mod.status()
-    if world > 1:
-        tt = torch.tensor([total_ms, attn_ms], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
-        total_ms, attn_ms = float(tt[0]), float(tt[1])
+    total_ms, attn_ms = max_over_ranks([total_ms, attn_ms], dev)
     ms_step = total_ms / args.steps
     attn_flops = 3.5 * fl["F_fwd"]
-    tflops = world * attn_flops / (attn_ms * 1e-3) / 1e12
+    tflops = job_tflops(world, attn_flops, attn_ms)
 
     # end to end through the public API from pinned host buffers
     e2e = None
@@ -341,13 +357,10 @@ def bench_e2e(args, cfg, mod, x, dev, world, attn_flops):
     b.record()
     torch.cuda.synchronize()
     ms = a.elapsed_time(b) / steps
-    if world > 1:
-        t = torch.tensor([ms], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t[0])
+    ms = max_over_ranks([ms], dev)[0]
     h2d = sum(hin[k].numel() * hin[k].element_size() for k in names)
     d2h = sum(h.numel() * h.element_size() for h in hout)
-    return {"value": round(world * attn_flops / (ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+    return {"value": round(job_tflops(world, attn_flops, ms), 3), "unit": "TFLOP/s",
             "ms_per_step": round(ms, 3), "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
             "steps": steps, "note": "selected-block FLOPs over the whole layer step incl. host copies"}
 
