@@ -177,11 +177,67 @@ __device__ void produce(const CUtensorMap* m0, const CUtensorMap* m1, const CUte
     }
 }
 
+// Epilogue of a 128-row accumulator tile (D fp32 columns in TMEM; this thread
+// holds row `row`, TMEM address `tacc` = its lane quarter + first column):
+// scaled bf16 (a finished tile) or raw fp32 (the partial of a split tile),
+// written as 16-byte chunks in the 128-byte-swizzled image of the whole-row
+// TMA maps into `stage` (free shared memory, 1024-byte aligned), then stored by
+// the group's leader with one TMA copy.  Per-row 16-byte stores straight to
+// global memory would touch 32 lines per warp instruction.  Every thread of
+// the group (nthreads, named barrier bar_id) runs the barrier, also when `ok`
+// is false after a timeout.
+template <int D>
+__device__ void store_tile(uint32_t tacc, int row, bool ok, bool zero, bool part, float mul, uint8_t* stage,
+                           const CUtensorMap* map_bf16, const CUtensorMap* map_f32, int y_bf16, int y_f32,
+                           int bar_id, int nthreads, bool leader) {
+    if (ok) {
+        const uint32_t sw = (uint32_t)(row & 7);
+#pragma unroll 1
+        for (int q = 0; q < D / 32; ++q) {
+            uint32_t r[32];
+            tmem_ld32(tacc + 32 * q, r);
+            tmem_wait_ld();
+            if (zero) {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) r[i] = 0u;
+            }
+            if (!part) {
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {                          // 4 chunks of 8 bf16
+                    const int g = 4 * q + k;
+                    uint4 v;
+                    v.x = pack_bf16x2(__uint_as_float(r[8 * k + 0]) * mul, __uint_as_float(r[8 * k + 1]) * mul);
+                    v.y = pack_bf16x2(__uint_as_float(r[8 * k + 2]) * mul, __uint_as_float(r[8 * k + 3]) * mul);
+                    v.z = pack_bf16x2(__uint_as_float(r[8 * k + 4]) * mul, __uint_as_float(r[8 * k + 5]) * mul);
+                    v.w = pack_bf16x2(__uint_as_float(r[8 * k + 6]) * mul, __uint_as_float(r[8 * k + 7]) * mul);
+                    *reinterpret_cast<uint4*>(stage + (g >> 3) * kTile + row * 128 + (((g & 7) ^ sw) << 4)) = v;
+                }
+            } else {
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {                          // 8 chunks of 4 fp32
+                    const int g = 8 * q + k;
+                    const float4 v = make_float4(__uint_as_float(r[4 * k]), __uint_as_float(r[4 * k + 1]),
+                                                 __uint_as_float(r[4 * k + 2]), __uint_as_float(r[4 * k + 3]));
+                    *reinterpret_cast<float4*>(stage + (g >> 3) * kTile + row * 128 + (((g & 7) ^ sw) << 4)) = v;
+                }
+            }
+        }
+        fence_proxy_async_smem();
+    }
+    named_sync(bar_id, nthreads);
+    if (ok && leader) {
+        tma_store_3d(part ? map_f32 : map_bf16, stage, 0, part ? y_f32 : y_bf16, 0);
+        bulk_commit();
+        bulk_wait_read();                                              // shared memory stays valid until read
+    }
+}
+
 // ============================================================================ dQ
 template <int D>
 __global__ void __launch_bounds__(192, 1)
 k_bwd_dq_sm100(const __nv_bfloat16* __restrict__ Qg, const __nv_bfloat16* __restrict__ dOg,
                const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+               const __grid_constant__ CUtensorMap tmdQ, const __grid_constant__ CUtensorMap tmPq,
                const uint32_t* __restrict__ gsel, const PlanHeader* __restrict__ hdr,
                const int4* __restrict__ items, float* __restrict__ part, const float* __restrict__ lse,
                const float* __restrict__ delta, int64_t N, int64_t MB, int SW, int nst, float scale,
@@ -346,36 +402,11 @@ k_bwd_dq_sm100(const __nv_bfloat16* __restrict__ Qg, const __nv_bfloat16* __rest
             tc_fence_before();
             mbar_arrive(B.elem + b);
         }
-        const bool fin = ok && mbar_wait(B.fin, 0, B.abort_flag, dev_status);
-        if (__all_sync(0xffffffffu, fin)) {
-            tc_fence_after();
-#pragma unroll
-            for (int q = 0; q < D / 32; ++q) {
-                uint32_t r[32];
-                tmem_ld32(tl + cdQ + 32 * q, r);
-                tmem_wait_ld();
-                if (ng == 0) {                              // nothing selected: TMEM never written
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) r[i] = 0u;
-                }
-                if (slot < 0) {
-                    uint32_t pk[16];
-#pragma unroll
-                    for (int i = 0; i < 16; ++i)
-                        pk[i] = pack_bf16x2(__uint_as_float(r[2 * i]) * scale, __uint_as_float(r[2 * i + 1]) * scale);
-                    uint4* dst = reinterpret_cast<uint4*>(dQ + grow * D + 32 * q);
-#pragma unroll
-                    for (int i = 0; i < 4; ++i)
-                        dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
-                } else {                                    // partial of a split tile (unscaled)
-                    float4* df = reinterpret_cast<float4*>(part + ((int64_t)slot * 128 + row) * D + 32 * q);
-#pragma unroll
-                    for (int i = 0; i < 8; ++i)
-                        df[i] = make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
-                                            __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]));
-                }
-            }
-        }
+        const bool fin = __all_sync(0xffffffffu, ok && mbar_wait(B.fin, 0, B.abort_flag, dev_status));
+        if (fin) tc_fence_after();
+        // nothing selected (ng == 0): TMEM never written, the tile is zero.  The ring is free.
+        store_tile<D>(tl + cdQ, row, fin, ng == 0, slot >= 0, scale, sm + L::RING, &tmdQ, &tmPq,
+                      (int)(row0 + 128 * tile), slot * 128, 1, 128, warp == 2 && lane == 0);
     }
     tc_fence_before();
     __syncthreads();
@@ -388,6 +419,8 @@ template <int D>
 __global__ void __launch_bounds__(384, 1)
 k_bwd_dkdv_sm100(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                  const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmdO,
+                 const __grid_constant__ CUtensorMap tmdK, const __grid_constant__ CUtensorMap tmdV,
+                 const __grid_constant__ CUtensorMap tmPkv,
                  const uint32_t* __restrict__ gselT, const PlanHeader* __restrict__ hdr,
                  const int4* __restrict__ items, float* __restrict__ part, const float* __restrict__ nld,
                  int64_t N, int64_t MB, int SW, int nst, float scale, __nv_bfloat16* __restrict__ dK, __nv_bfloat16* __restrict__ dV,
@@ -548,43 +581,13 @@ k_bwd_dkdv_sm100(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
             tc_fence_before();
             mbar_arrive(B.elem + b);
         }
-        const bool fin = ok && mbar_wait(B.fin, 0, B.abort_flag, dev_status);
-        if (__all_sync(0xffffffffu, fin)) {
-            tc_fence_after();
-            const int64_t grow = row0 + 128 * tile + row;
-            {
-                const int which = wg;                          // warpgroup 0 writes dK, warpgroup 1 dV
-                const float mul = which ? 1.f : scale;
-                const uint32_t col = which ? cdV : cdK;
-#pragma unroll
-                for (int q = 0; q < D / 32; ++q) {
-                    uint32_t r[32];
-                    tmem_ld32(tl + col + 32 * q, r);
-                    tmem_wait_ld();
-                    if (ng == 0) {                          // no query selected these keys: zeros
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) r[i] = 0u;
-                    }
-                    if (slot < 0) {
-                        uint32_t pk[16];
-#pragma unroll
-                        for (int i = 0; i < 16; ++i)
-                            pk[i] = pack_bf16x2(__uint_as_float(r[2 * i]) * mul, __uint_as_float(r[2 * i + 1]) * mul);
-                        uint4* dst = reinterpret_cast<uint4*>((which ? dV : dK) + grow * D + 32 * q);
-#pragma unroll
-                        for (int i = 0; i < 4; ++i)
-                            dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
-                    } else {                                // partial of a split tile (unscaled)
-                        float4* df = reinterpret_cast<float4*>(part + (((int64_t)slot * 2 + which) * 128 + row) * D +
-                                                               32 * q);
-#pragma unroll
-                        for (int i = 0; i < 8; ++i)
-                            df[i] = make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
-                                                __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]));
-                    }
-                }
-            }
-        }
+        const bool fin = __all_sync(0xffffffffu, ok && mbar_wait(B.fin, 0, B.abort_flag, dev_status));
+        if (fin) tc_fence_after();
+        // warpgroup 0 writes dK, warpgroup 1 dV, each staged in its half of the (now free) ring;
+        // no query selected these keys (ng == 0): TMEM never written, zeros
+        store_tile<D>(tl + (wg ? cdV : cdK), row, fin, ng == 0, slot >= 0, wg ? 1.f : scale,
+                      sm + L::RING + wg * 2 * L::NR * kTile, wg ? &tmdV : &tmdK, &tmPkv, (int)(row0 + 128 * tile),
+                      (slot * 2 + wg) * 128, 2 + wg, 128, (warp & 3) == 0 && lane == 0);
     }
     tc_fence_before();
     __syncthreads();
@@ -634,6 +637,12 @@ prism_status_t launch_bwd(const Dims& d, const void* Qp, const void* Kp, const v
         !make_map_bf16_rows(&gK, Kp, rows, D, 64) || !make_map_bf16_rows(&gV, Vp, rows, D, 64))
         return PRISM_ERR_CUDA;
     const int target = plan_target(device_sms());
+    const int64_t slots = 2 * (int64_t)target;
+    CUtensorMap tdQ, tdK, tdV, tPq, tPkv;
+    if (!make_map_bf16_rows(&tdQ, dQp, rows, D, 128) || !make_map_bf16_rows(&tdK, dKp, rows, D, 128) ||
+        !make_map_bf16_rows(&tdV, dVp, rows, D, 128) || !make_map_f32_rows(&tPq, w.part_q, slots * 128, D, 128) ||
+        !make_map_f32_rows(&tPkv, w.part_kv, slots * 2 * 128, D, 128))
+        return PRISM_ERR_CUDA;
     prism_status_t st = plan_work(w.pq, gsel, d, 2, 1, target, kSegMinGranules, s);
     if (st == PRISM_OK) st = plan_work(w.pkv, gselT, d, 2, 1, target, kSegMinGranules, s);
     if (st != PRISM_OK) return st;
@@ -646,10 +655,12 @@ prism_status_t launch_bwd(const Dims& d, const void* Qp, const void* Kp, const v
     if (cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, smq) != cudaSuccess ||
         cudaFuncSetAttribute(kk, cudaFuncAttributeMaxDynamicSharedMemorySize, smk) != cudaSuccess)
         return PRISM_ERR_CUDA;
-    kq<<<(unsigned)w.pq.items_max, 192, smq, s>>>((const __nv_bfloat16*)Qp, (const __nv_bfloat16*)dOp, gK, gV, gsel, w.pq.hdr, w.pq.items, w.part_q, lse,
+    kq<<<(unsigned)w.pq.items_max, 192, smq, s>>>((const __nv_bfloat16*)Qp, (const __nv_bfloat16*)dOp, gK, gV, tdQ, tPq,
+                                                  gsel, w.pq.hdr, w.pq.items, w.part_q, lse,
                                                   w.delta, d.N, d.MB, (int)d.SW, nq, scale, (__nv_bfloat16*)dQp,
                                                   dev_status);
-    kk<<<(unsigned)w.pkv.items_max, 384, smk, s>>>(tK, tV, gQ, gdO, gselT, w.pkv.hdr, w.pkv.items, w.part_kv, w.nld,
+    kk<<<(unsigned)w.pkv.items_max, 384, smk, s>>>(tK, tV, gQ, gdO, tdK, tdV, tPkv, gselT, w.pkv.hdr, w.pkv.items,
+                                                   w.part_kv, w.nld,
                                                    d.N, d.MB, (int)d.SW, nk, scale, (__nv_bfloat16*)dKp,
                                                    (__nv_bfloat16*)dVp, dev_status);
     st = launch_status(2);
