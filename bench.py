@@ -3,6 +3,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config 2k] [--dense]
     python bench.py --impl reference      # the fp64 CPU oracle on a bounded sample
+    python bench.py --forward-only        # inference: the forward stages, no backward state
 
 One step = one pass of the whole hot path over the configured synthetic layer:
 zone indicator -> shapes/permutation -> permute Q,K,V -> pooled block
@@ -12,7 +13,8 @@ permute dO -> sparse attention backward -> unpermute dQ, dK, dV.
 F_fwd = 4 d sum_h sum_i sum_{j in S_i} |B_i||B_j|) over the device time of the
 sparse attention forward + backward calls, summed over ranks (each rank runs
 its own layer: weak scaling, no data-path collective).  Prints one JSON line
-on rank 0.
+on rank 0.  With --forward-only a step ends at the unpermuted O, the layer holds
+no backward buffers, and ``value`` is F_fwd over the forward call's time.
 """
 from __future__ import annotations
 
@@ -35,6 +37,7 @@ from dynamic_block_sparse_macro_b200 import inputs  # noqa: E402
 from dynamic_block_sparse_macro_b200.configs import get_config  # noqa: E402
 
 METRIC = "sparse attn fwd+bwd ms/layer & TFLOP/s on selected blocks, 2K grid (295k tok)"
+METRIC_FWD = "sparse attn fwd ms/layer & TFLOP/s on selected blocks, 2K grid (295k tok), inference"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # DRAM bytes (read + write) of one backward call on the 2K layer with 24 heads, from an ncu
 # capture of the backward kernels on 4 heads scaled by 6 (their per-head working set is the
@@ -155,11 +158,13 @@ def selected_flops(mod) -> dict:
     g = mod.gsel.to(torch.int64) & 0xFFFFFFFF
     pop = lambda w: sum(((w >> s) & 1) for s in range(32))
     tile_gran = pop(g[:, 0::2, :] | g[:, 1::2, :]).sum(-1).double()            # [h, N/128]
-    gT = mod.gselT.to(torch.int64) & 0xFFFFFFFF
-    key_gran = pop(gT[:, 0::2, :] | gT[:, 1::2, :]).sum(-1).double()
     q = torch.tensor([0.5, 0.99, 1.0], dtype=torch.float64, device=tile_gran.device)
     tq = torch.quantile(tile_gran.flatten(), q).tolist()
-    kq = torch.quantile(key_gran.flatten(), q).tolist()
+    kq = None
+    if mod.gselT is not None:
+        gT = mod.gselT.to(torch.int64) & 0xFFFFFFFF
+        key_gran = pop(gT[:, 0::2, :] | gT[:, 1::2, :]).sum(-1).double()
+        kq = torch.quantile(key_gran.flatten(), q).tolist()
     return {"F_fwd": f_fwd, "F_dense_fwd": dense, "n_blk": nb, "density": f_fwd / dense,
             "mean_sel_blocks": float(sel.sum(-1).mean().item()),
             "max_sel_blocks": float(sel.sum(-1).max().item()),
@@ -190,6 +195,10 @@ def run_step(mod, x, out, grads, timer=None):
     from dynamic_block_sparse_macro_b200 import _abi
     _abi.prism_unpermute(mod.prob, mod.Op, mod.perm, out)
     rec(3)
+    if not mod.with_backward:                 # inference: the step ends with O
+        for i in (4, 5, 6):
+            rec(i)
+        return
     _abi.prism_permute(mod.prob, x["dO"], mod.perm, mod.dOp)
     rec(4)
     _abi.prism_sparse_attn_bwd(mod.prob, mod.Qp, mod.Kp, mod.Vp, mod.Op, mod.Of32, mod.dOp, mod.lse,
@@ -202,9 +211,9 @@ def run_step(mod, x, out, grads, timer=None):
 
 
 # ---------------------------------------------------------------- CPU oracle sample
-def oracle_sample(cfg, host, target_s=15.0, max_blocks=None, seed=0):
-    """Time the fp64 oracle's sparse attention fwd+bwd on a bounded sample of
-    query blocks of head 0, under the given selection.  Returns a dict."""
+def oracle_sample(cfg, host, target_s=15.0, max_blocks=None, seed=0, forward_only=False):
+    """Time the fp64 oracle's sparse attention fwd+bwd (or fwd alone) on a bounded
+    sample of query blocks of head 0, under the given selection.  Returns a dict."""
     import oracle as orc
     from threadpoolctl import threadpool_info
     Qb, Kb, Vb, dOb, bs, sel = (host[k] for k in ("Qb", "Kb", "Vb", "dOb", "bs", "sel"))
@@ -218,10 +227,12 @@ def oracle_sample(cfg, host, target_s=15.0, max_blocks=None, seed=0):
         blocks = sorted(order[done:done + step].tolist())
         t0 = time.perf_counter()
         orc.sparse_attention_fwd(Qb, Kb, Vb, bs, sel, heads=[0], q_blocks=blocks)
-        orc.sparse_attention_bwd(Qb, Kb, Vb, dOb, bs, sel, heads=[0], q_blocks=blocks)
+        if not forward_only:
+            orc.sparse_attention_bwd(Qb, Kb, Vb, dOb, bs, sel, heads=[0], q_blocks=blocks)
         t_used += time.perf_counter() - t0
+        mult = 1.0 if forward_only else 3.5
         for i in blocks:
-            flops += 3.5 * 4.0 * Qb.shape[-1] * sizes[i] * float(sizes[sel[0, i]].sum())
+            flops += mult * 4.0 * Qb.shape[-1] * sizes[i] * float(sizes[sel[0, i]].sum())
         done += len(blocks)
         step = min(step * 2, 64)
     threads = 1
@@ -238,9 +249,12 @@ def make_host_sample(mod, x):
     bs = mod.blk_start[: nb + 1].cpu().numpy().astype(np.int64)
     f = lambda t: t[:1].float().cpu().double().numpy()
     from dynamic_block_sparse_macro_b200 import _abi
-    _abi.prism_permute(mod.prob, x["dO"], mod.perm, mod.dOp)
-    torch.cuda.synchronize()
-    return {"Qb": f(mod.Qp), "Kb": f(mod.Kp), "Vb": f(mod.Vp), "dOb": f(mod.dOp), "bs": bs, "sel": sel}
+    dOb = None
+    if mod.with_backward:
+        _abi.prism_permute(mod.prob, x["dO"], mod.perm, mod.dOp)
+        torch.cuda.synchronize()
+        dOb = f(mod.dOp)
+    return {"Qb": f(mod.Qp), "Kb": f(mod.Kp), "Vb": f(mod.Vp), "dOb": dOb, "bs": bs, "sel": sel}
 
 
 # ---------------------------------------------------------------- arms
@@ -251,10 +265,15 @@ def bench_prism(args, cfg, rank, world, local_rank):
     torch.cuda.set_device(dev)
     x = inputs.make_inputs(cfg, dev)
     torch.cuda.synchronize()
+    fwd_only = bool(args.forward_only)
+    if fwd_only:
+        del x["dO"]
+    torch.cuda.reset_peak_memory_stats(dev)
     mod = PrismSparseAttention(cfg.T, cfg.H, cfg.W, cfg.heads, cfg.head_dim, cfg.audio_dim, cfg.dtype,
-                               cfg.top_k, cfg.top_p if not args.dense else 1.0, device=dev)
+                               cfg.top_k, cfg.top_p if not args.dense else 1.0, device=dev,
+                               with_backward=not fwd_only)
     out = torch.empty_like(x["Q"])
-    grads = [torch.empty_like(x["Q"]) for _ in range(3)]
+    grads = [] if fwd_only else [torch.empty_like(x["Q"]) for _ in range(3)]
     for _ in range(max(args.warmup, 1)):
         run_step(mod, x, out, grads)
     torch.cuda.synchronize()
@@ -283,8 +302,12 @@ def bench_prism(args, cfg, rank, world, local_rank):
     status = mod.status()
     total_ms, attn_ms = max_over_ranks([total_ms, attn_ms], dev)
     ms_step = total_ms / args.steps
-    attn_flops = 3.5 * fl["F_fwd"]
+    # fwd: 2 contractions of 2 d |B_i||B_j| flops each; bwd adds 5 at half the weight each (2.5x)
+    attn_flops = (1.0 if fwd_only else 3.5) * fl["F_fwd"]
     tflops = job_tflops(world, attn_flops, attn_ms)
+    memory = mod.memory_report()
+    memory["inputs_outputs"] = int(sum(t.numel() * t.element_size() for t in list(x.values()) + [out] + grads))
+    memory["peak_allocated"] = int(torch.cuda.max_memory_allocated(dev))
 
     # end to end through the public API from pinned host buffers
     e2e = None
@@ -292,18 +315,21 @@ def bench_prism(args, cfg, rank, world, local_rank):
         e2e = bench_e2e(args, cfg, mod, x, dev, world, attn_flops)
 
     peaks = load_peaks()
-    fwd_ach = 4 * fl["F_fwd"] / (stage_ms["attn_fwd"] * 1e-3) / 1e12
+    # F_fwd already counts both forward contractions (4 d |B_i||B_j| per selected pair)
+    fwd_ach = fl["F_fwd"] / (stage_ms["attn_fwd"] * 1e-3) / 1e12
     bwd_ach = 2.5 * fl["F_fwd"] / (stage_ms["attn_bwd"] * 1e-3) / 1e12
     dom = "attn_bwd" if stage_ms["attn_bwd"] >= stage_ms["attn_fwd"] else "attn_fwd"
     ach = bwd_ach if dom == "attn_bwd" else fwd_ach
     traffic = BWD_DRAM_BYTES.get((cfg.name, cfg.heads)) if dom == "attn_bwd" and not args.dense else None
     peak = peaks["bf16_tflops_sustained"]
     res = {
-        "metric": METRIC, "value": round(tflops, 3), "unit": "TFLOP/s", "n_gpus": world,
+        "metric": METRIC_FWD if fwd_only else METRIC, "value": round(tflops, 3), "unit": "TFLOP/s",
+        "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
         "attn_ms_per_layer": round(attn_ms, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic",
-        "config": {"workload": f"prism {cfg.name} layer fwd+bwd", "grid": [cfg.T, cfg.H, cfg.W],
+        "config": {"workload": f"prism {cfg.name} layer " + ("fwd (inference)" if fwd_only else "fwd+bwd"),
+                   "grid": [cfg.T, cfg.H, cfg.W],
                    "tokens": cfg.n_tokens, "heads": cfg.heads, "head_dim": cfg.head_dim,
                    "top_k": cfg.top_k, "top_p": 1.0 if args.dense else cfg.top_p,
                    "all_blocks_dense": bool(args.dense), "global_batch": world,
@@ -316,29 +342,32 @@ def bench_prism(args, cfg, rank, world, local_rank):
                      "frac": round(ach / peak, 4), "traffic": traffic,
                      "peak_source": f"{peaks['source']} bf16_tflops_sustained"},
         "gpu_launches": int(launches),
+        "memory_bytes": memory,
         "clocks": clk,
         "dev_status": status,
         "e2e": e2e,
     }
     if rank == 0 and world == 1 and not args.no_cpu:
         host = make_host_sample(mod, x)
-        cs = oracle_sample(cfg, host, target_s=args.cpu_seconds)
+        cs = oracle_sample(cfg, host, target_s=args.cpu_seconds, forward_only=fwd_only)
         res["cpu_baseline"] = {"value": round(cs["tflops"], 6), "unit": "TFLOP/s", "cores": cs["threads"],
                                "kind": "oracle",
                                "sample": f"fp64 numpy oracle, head 0, {cs['blocks']} random query blocks "
-                                         f"(fwd+bwd under the GPU's selection), {cs['seconds']:.1f} s"}
+                                         f"({'fwd' if fwd_only else 'fwd+bwd'} under the GPU's selection), "
+                                         f"{cs['seconds']:.1f} s"}
     return res
 
 
 def bench_e2e(args, cfg, mod, x, dev, world, attn_flops):
-    names = ("Q", "K", "V", "hhat", "dO")
+    names = ("Q", "K", "V", "hhat", "dO") if mod.with_backward else ("Q", "K", "V", "hhat")
     hin = {k: torch.empty(x[k].shape, dtype=x[k].dtype, pin_memory=True) for k in names}
     for k in names:
         hin[k].copy_(x[k])
     dx = {k: torch.empty_like(x[k]) for k in names}
-    hout = [torch.empty(x["Q"].shape, dtype=x["Q"].dtype, pin_memory=True) for _ in range(4)]
+    n_out = 4 if mod.with_backward else 1
+    hout = [torch.empty(x["Q"].shape, dtype=x["Q"].dtype, pin_memory=True) for _ in range(n_out)]
     out = torch.empty_like(x["Q"])
-    grads = [torch.empty_like(x["Q"]) for _ in range(3)]
+    grads = [torch.empty_like(x["Q"]) for _ in range(n_out - 1)]
     steps = max(1, min(args.steps, 3))
 
     def one():
@@ -383,22 +412,26 @@ def bench_reference(args, cfg):
     sel = orc.block_select(P, cfg.top_k, cfg.top_p)["sel"]
     host = {"Qb": Qb, "Kb": Kb, "Vb": Vb, "dOb": dOb, "bs": bs, "sel": sel}
     per_step = max(2.0, args.cpu_seconds / max(1, args.steps + args.warmup))
+    fo = bool(args.forward_only)
     for w in range(args.warmup):
-        oracle_sample(cfg, host, target_s=per_step, seed=1000 + w)
-    res = [oracle_sample(cfg, host, target_s=per_step, seed=s) for s in range(args.steps)]
+        oracle_sample(cfg, host, target_s=per_step, seed=1000 + w, forward_only=fo)
+    res = [oracle_sample(cfg, host, target_s=per_step, seed=s, forward_only=fo) for s in range(args.steps)]
+    what = "fwd" if fo else "fwd+bwd"
     fl = sum(r["flops"] for r in res)
     sec = sum(r["seconds"] for r in res)
     v = fl / sec / 1e12
     blocks = sum(r["blocks"] for r in res)
-    return {"metric": METRIC, "value": round(v, 6), "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps,
+    return {"metric": METRIC_FWD if fo else METRIC, "value": round(v, 6), "unit": "TFLOP/s", "n_gpus": 1,
+            "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(1e3 * sec / args.steps, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
-            "config": {"workload": f"prism {cfg.name} layer fwd+bwd (oracle sample)",
+            "config": {"workload": f"prism {cfg.name} layer " + ("fwd (inference)" if fo else "fwd+bwd")
+                                   + " (oracle sample)",
                        "grid": [cfg.T, cfg.H, cfg.W], "tokens": cfg.n_tokens, "heads": cfg.heads,
                        "head_dim": cfg.head_dim, "top_k": cfg.top_k, "top_p": cfg.top_p},
             "cpu_baseline": {"value": round(v, 6), "unit": "TFLOP/s", "cores": res[0]["threads"],
                              "kind": "oracle",
-                             "sample": f"fp64 numpy oracle sparse attention fwd+bwd, head 0, {blocks} query "
+                             "sample": f"fp64 numpy oracle sparse attention {what}, head 0, {blocks} query "
                                        f"blocks over {args.steps} steps, selection by the oracle's own stages"},
             "e2e": {"value": round(v, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
@@ -413,6 +446,8 @@ def main():
     ap.add_argument("--heads", type=int, default=None,
                     help="override the config's head count (smaller profiling captures)")
     ap.add_argument("--dense", action="store_true", help="select every block (all-blocks dense run)")
+    ap.add_argument("--forward-only", action="store_true",
+                    help="inference: the forward stages alone, no backward buffers (value = forward TFLOP/s)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)

@@ -56,7 +56,7 @@ extern "C" prism_status_t prism_sparse_attn_fwd(const prism_problem_t* prob, con
     Dims d;
     prism_status_t st = make_dims(prob, &d);
     if (st != PRISM_OK) return st;
-    if (!ok_ptr(Qp) || !ok_ptr(Kp) || !ok_ptr(Vp) || !ok_ptr(gsel) || !ok_ptr(Op) || !ok_ptr(lse) ||
+    if (!ok_ptr(Qp) || !ok_ptr(Kp) || !ok_ptr(Vp) || !ok_ptr(gsel) || !ok_ptr(Op) || !ok_opt(lse) ||
         !ok_opt(o_f32) || !ok_ptr(dev_status) || !ok_opt(ws))
         return PRISM_ERR_INVALID_ARG;
     if (!(scale > 0.f) || !isfinite(scale)) return PRISM_ERR_INVALID_ARG;

@@ -129,7 +129,7 @@ __global__ void __launch_bounds__(128) k_fwd_combine(const int2* __restrict__ ti
             O[(grow0 + r) * D + threadIdx.x] = __float2bfloat16_rn(o);
             if (o_f32) o_f32[(grow0 + r) * D + threadIdx.x] = o;
         }
-        if (threadIdx.x == 0) lse[grow0 + r] = L > 0.f ? (M + log2f(L)) * 0.6931471805599453f : -INFINITY;
+        if (threadIdx.x == 0 && lse) lse[grow0 + r] = L > 0.f ? (M + log2f(L)) * 0.6931471805599453f : -INFINITY;
     }
 }
 

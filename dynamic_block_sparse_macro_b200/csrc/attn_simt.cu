@@ -136,7 +136,7 @@ __global__ void __launch_bounds__(256) k_fwd_simt(const T* __restrict__ Q, const
             O[hoff + r * D + tx + 16 * w] = from_f32<T>(o);
             if (o_f32) o_f32[hoff + r * D + tx + 16 * w] = o;
         }
-        if (tx == 0) lse[(int64_t)hh * N + r] = l[u] > 0.f ? (m2[u] + log2f(l[u])) * kLn2 : -INFINITY;
+        if (tx == 0 && lse) lse[(int64_t)hh * N + r] = l[u] > 0.f ? (m2[u] + log2f(l[u])) * kLn2 : -INFINITY;
     }
 }
 

@@ -338,7 +338,7 @@ k_attn_fwd_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                                                 __uint_as_float(r[4 * i + 3]) * inv);
                     }
                 }
-                lse[grow] = l > 0.f ? (m_run + log2f(l)) * kLn2 : -INFINITY;
+                if (lse) lse[grow] = l > 0.f ? (m_run + log2f(l)) * kLn2 : -INFINITY;
             } else {
                 // partial of a split tile: unnormalised O, running max and denominator
                 float* po = parts.o + ((int64_t)slot * 128 + row) * D;

@@ -37,6 +37,9 @@ class PrismSparseAttention:
         self.guidance, self.fixed_shape = guidance, int(fixed_shape)
         self.scale = float(scale) if scale is not None else 1.0 / math.sqrt(head_dim)
         self.heads, self.d = heads, head_dim
+        # with_backward=False is the inference path: no backward buffers, no key-major
+        # selection, no fp32 copy of O and no LSE
+        self.with_backward = bool(with_backward)
         dev = torch.device(device)
         self.device = dev
         s = self.sizes
@@ -62,7 +65,7 @@ class PrismSparseAttention:
         self.sel = e(heads, MB, SW, dt=torch.int32)
         # granule-level selection (the attention kernels' view) and its transpose
         self.gsel = e(heads, MB, SW, dt=torch.int32)
-        self.gselT = e(heads, MB, SW, dt=torch.int32)
+        self.gselT = e(heads, MB, SW, dt=torch.int32) if with_backward else None
         self.sel_count = e(heads, MB, dt=i32)
         self.margin_sel = e(heads, MB)
         self.dev_status = torch.zeros(1, dtype=i32, device=dev)
@@ -70,7 +73,7 @@ class PrismSparseAttention:
         self.Op = e(heads, N, head_dim, dt=self.tdt)
         # unrounded O for the backward's Delta (bf16 storage only)
         self.Of32 = e(heads, N, head_dim) if (with_backward and dtype == "bf16") else None
-        self.lse = e(heads, N)
+        self.lse = e(heads, N) if with_backward else None
         self.ws_fwd = e(max(16, s.ws_attn_fwd), dt=torch.uint8)
         if with_backward:
             self.dOp = e(heads, N, head_dim, dt=self.tdt)
@@ -116,6 +119,8 @@ class PrismSparseAttention:
 
     def backward(self, dO, dQ=None, dK=None, dV=None, stream=None):
         """Stage 7 for the last forward; returns raster (dQ, dK, dV)."""
+        if not self.with_backward:
+            raise RuntimeError("this layer was built for inference (with_backward=False)")
         p = self.prob
         _abi.prism_permute(p, dO, self.perm, self.dOp, stream)
         _abi.prism_sparse_attn_bwd(p, self.Qp, self.Kp, self.Vp, self.Op, self.Of32, self.dOp, self.lse,
@@ -128,6 +133,24 @@ class PrismSparseAttention:
             _abi.prism_unpermute(p, src, self.perm, dst, stream)
             outs.append(dst)
         return tuple(outs)
+
+    # ------------------------------------------------------------------ memory
+    def memory_report(self) -> dict:
+        """Device bytes this layer holds, by stage (the caller's raster inputs and
+        outputs are not included)."""
+        def nb(*ts):
+            return int(sum(t.numel() * t.element_size() for t in ts if t is not None))
+        rep = {
+            "plan": nb(self.g, self.rho, self.abar, self.zone_stats, self.ws_ind, self.shape_id, self.perm,
+                       self.blk_start, self.gran_blk, self.n_blk, self.margin_shape),
+            "blocked_qkv": nb(self.Qp, self.Kp, self.Vp),
+            "scores": nb(self.Qbar, self.Kbar, self.P),
+            "selection": nb(self.sel, self.gsel, self.gselT, self.sel_count, self.margin_sel, self.dev_status),
+            "forward": nb(self.Op, self.Of32, self.lse, self.ws_fwd),
+            "backward": nb(self.dOp, self.dQp, self.dKp, self.dVp, self.ws_bwd) if self.with_backward else 0,
+        }
+        rep["total"] = sum(rep.values())
+        return rep
 
     # ------------------------------------------------------------------ views
     def num_blocks(self) -> int:

@@ -230,8 +230,9 @@ prism_status_t prism_block_select(const prism_problem_t* prob, const float* P, c
  * Stage 6 — exact online-softmax attention of every query block over the tokens
  * of its selected key blocks ("Método" 3; non-causal, scale usually 1/sqrt(d)).
  *   Qp, Kp, Vp blocked [heads][N][d];  gsel granule-level selection from
- *   prism_block_select;  Op blocked;  lse [heads][N] float32 (natural log of
- *   the softmax denominator; -inf for an empty S_i, whose O is 0).
+ *   prism_block_select;  Op blocked;  lse [heads][N] float32 (nullable: the
+ *   backward's input only, so inference passes NULL) = natural log of the
+ *   softmax denominator; -inf for an empty S_i, whose O is 0.
  *   o_f32 (nullable) blocked [heads][N][d] float32: the unrounded O, for the
  *   backward's Delta (with a bf16 O, rowsum(dO*O) carries O's rounding error,
  *   which dominates dQ/dK when the attention is diffuse).

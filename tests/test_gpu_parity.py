@@ -123,3 +123,22 @@ def test_deterministic_repeat():
     assert torch.equal(O1, O2)
     for a, b in zip(g1, g2):
         assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_inference_layer_matches_training_forward(dtype):
+    # with_backward=False: no LSE, no fp32 O, no key-major selection; O and every decision
+    # are the bits of the training layer's forward (whose O the other tests check against
+    # the oracle)
+    from dynamic_block_sparse_macro_b200.layer import PrismSparseAttention
+    from gpu_parity import run_gpu
+    cfg = get_config("720p", T=16, H=32, W=32, heads=3, dtype=dtype)
+    x = _inputs(cfg)
+    mt, Ot, _ = run_gpu(cfg, x, backward=False)
+    mi = PrismSparseAttention(cfg.T, cfg.H, cfg.W, cfg.heads, cfg.head_dim, cfg.audio_dim, cfg.dtype,
+                              cfg.top_k, cfg.top_p, with_backward=False)
+    Oi = mi.forward(x["Q"], x["K"], x["V"], x["hhat"])
+    torch.cuda.synchronize()
+    assert mi.status() == 0 and mi.lse is None
+    assert torch.equal(mi.perm, mt.perm) and torch.equal(mi.gsel, mt.gsel)
+    assert torch.equal(Oi, Ot)
