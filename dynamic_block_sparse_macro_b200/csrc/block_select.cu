@@ -8,20 +8,21 @@
 // p (everything if p >= 1 or it never does), so S_i is the longer prefix,
 // max(min(k, n_blk), n_p) blocks.
 //
-// k_block_select   one warp per (row, head) for rows of up to 4096 blocks, one
-//                  256-thread CTA per row above that; no sort.  For P >= 0 the float bit
-//                  pattern orders like the value, so thresholds are found by
-//                  binary search over bit patterns with block reductions over
-//                  the row held in shared memory:
-//                    v* = largest t with sum{P_j : P_j >= t} >= p   (Top-p
-//                         crossing value; n_p = #{P > v*} + the fewest ties
-//                         at v* that reach p),
-//                    v_n = largest t with #{P_j >= t} >= n  (n-th value),
-//                  then S_i = {P > v_n} plus the lowest-index ties at v_n.
-//                  All reductions run in a fixed order (deterministic).  Every
-//                  search step is a pass over the row and a reduction, so the
-//                  warp form (shuffles, no block barrier) does the same work
-//                  in a fraction of the time.
+// For P >= 0 the float bit pattern orders like the value, so thresholds are
+// found by binary search over bit patterns, each step a pass over the row
+// and a fixed-order reduction (deterministic):
+//   v_k = largest t with #{P_j >= t} >= k       (k-th value of the order),
+//   v*  = largest t with sum{P_j : P_j >= t} >= p (Top-p crossing value).
+// One search per row suffices.  With S_k the sum of the first k entries, Top-k
+// sets the size when S_k >= p (then n_p <= k, and n_p = k exactly when
+// S_k - v_k < p); otherwise n_p > k and the Top-p search gives both n_p and the
+// threshold.  S_i = {P > v_n} plus the lowest-index ties at v_n.
+//
+// k_select_reg<C>  one warp per (row, head), the row in registers (C values a
+//                  lane, rows of 32*CLO < n_blk <= 32*C blocks); one kernel
+//                  per size class, each exits for the others' rows.
+// k_select_cta     one 256-thread CTA per row above 4096 blocks, the row in
+//                  shared memory.
 // k_sel_expand     granule-level view of the selection for the attention
 //                  kernels; k_bit_transpose its key-major transpose.
 #include "common.cuh"
@@ -29,9 +30,10 @@
 namespace prism {
 
 constexpr int kSelectThreads = 256;
-constexpr int kSelectMaxRow = 16384;    // P values of a row held in shared memory
-constexpr int kWarpRowMax = 4096;       // rows up to this many blocks: one warp each
+constexpr int kSelectMaxRow = 16384;    // P values of a row held in shared memory (CTA form)
+constexpr int kWarpRowMax = 4096;       // rows up to this many blocks: one warp each, in registers
 constexpr int kWarpRowsPerCta = 4;
+static_assert(kWarpRowMax == 32 * 128, "the largest register class holds 128 values a lane");
 
 struct SelRed {
     float f[kSelectThreads / 32];
@@ -60,13 +62,6 @@ __device__ __forceinline__ int sel_count_i(int v, SelRed& r) {
     for (int w = 0; w < kSelectThreads / 32; ++w) s += r.i[w];
     return s;
 }
-// the same reductions over one warp (butterfly: every lane gets the result)
-__device__ __forceinline__ int warp_sum_i(int v) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    return v;
-}
-
 __device__ __forceinline__ float sel_max(float v, SelRed& r) {
     v = warp_max(v);
     __syncthreads();
@@ -77,104 +72,213 @@ __device__ __forceinline__ float sel_max(float v, SelRed& r) {
     for (int w = 1; w < kSelectThreads / 32; ++w) s = fmaxf(s, r.f[w]);
     return s;
 }
+__device__ __forceinline__ int warp_sum_i(int v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
 
-// TPR threads per row: 32 (one warp per row, kWarpRowsPerCta rows per CTA)
-// or kSelectThreads (one CTA per row); each form leaves the other's rows alone.
-template <int TPR>
-__global__ void __launch_bounds__(kSelectThreads) k_block_select(const float* __restrict__ P,
-                                                                 const int32_t* __restrict__ n_blk, int64_t MB,
-                                                                 int SW, int rowcap, int top_k, float top_p,
-                                                                 uint32_t* __restrict__ sel,
-                                                                 int32_t* __restrict__ sel_count,
-                                                                 float* __restrict__ margin,
-                                                                 uint32_t* __restrict__ dev_status) {
-    constexpr bool kWarp = TPR == 32;
-    extern __shared__ float smem_rows[];
-    __shared__ SelRed red;
-    const int nb = *n_blk;
-    if (kWarp ? nb > kWarpRowMax : nb <= kWarpRowMax) return;      // the other form's rows
-    const int tid = kWarp ? (threadIdx.x & 31) : threadIdx.x;
-    const int i = kWarp ? blockIdx.x * kWarpRowsPerCta + (threadIdx.x >> 5) : blockIdx.x, hh = blockIdx.y;
-    if (kWarp && i >= MB) return;                                   // warp-uniform
-    float* row = smem_rows + (kWarp ? (threadIdx.x >> 5) * rowcap : 0);
-    uint32_t* srow = sel + ((int64_t)hh * MB + i) * SW;
-    if (i >= nb || nb > kSelectMaxRow) {
-        for (int w = tid; w < SW; w += TPR) srow[w] = 0u;
-        if (tid == 0) {
-            sel_count[(int64_t)hh * MB + i] = 0;
-            if (margin) margin[(int64_t)hh * MB + i] = INFINITY;
-            if (nb > kSelectMaxRow && i == 0 && hh == 0) atomicOr(dev_status, PRISM_DEV_BAD_INDEX);
+// size of S_i and its threshold: the first n entries of (P desc, j asc) are
+// {P > vb} plus the first need_eq ties at vb (all of the row when n >= nb)
+struct SelCut {
+    int n;
+    uint32_t vb;
+    int need_eq;
+    float gap_p;     // cumulative-sum margin of the Top-p decision (inf if Top-p cannot set n)
+};
+
+// count_ge(t) = #{P >= t}, sum_ge(t) = sum{P >= t} for bit patterns t (row-wide)
+template <class CountGe, class SumGe>
+__device__ __forceinline__ SelCut select_cut(int nb, int top_k, float top_p, CountGe count_ge, SumGe sum_ge) {
+    SelCut c{nb, 0u, nb, INFINITY};
+    const int n_k = min(top_k, nb);
+    const float total = sum_ge(0u);
+    if (!(top_p < 1.f) || total < top_p) {       // Top-p takes the whole row
+        if (top_p < 1.f) c.gap_p = fabsf(total - top_p);
+        return c;
+    }
+    constexpr uint32_t kHi = 0x3F800001u;        // (1.0f bits) + 1: no P reaches it
+    // Top-k threshold and S_k
+    uint32_t lo_k = 0u;
+    int gt_k = 0;
+    bool k_sets = false;
+    if (n_k > 0) {
+        uint32_t lo = 0u, hi = kHi;              // count{P >= lo} >= n_k > count{P >= hi}
+        while (hi - lo > 1u) {
+            const uint32_t mid = lo + ((hi - lo) >> 1);
+            if (count_ge(mid) >= n_k) lo = mid;
+            else hi = mid;
         }
+        lo_k = lo;
+        gt_k = count_ge(lo + 1u);
+        const float vk = __uint_as_float(lo);
+        const float S_k = sum_ge(lo + 1u) + (float)(n_k - gt_k) * vk;
+        if (S_k >= top_p) {                      // n_p <= n_k
+            k_sets = true;
+            const float S_prev = n_k >= 2 ? S_k - vk : -INFINITY;
+            if (S_prev < top_p) c.gap_p = fminf(fabsf(S_k - top_p), fabsf(top_p - S_prev));   // n_p == n_k
+        }
+    }
+    if (!k_sets) {
+        // largest bit pattern t with sum{P >= t} >= p: lo keeps the property, hi does not
+        uint32_t lo = 0u, hi = kHi;
+        while (hi - lo > 1u) {
+            const uint32_t mid = lo + ((hi - lo) >> 1);
+            if (sum_ge(mid) >= top_p) lo = mid;
+            else hi = mid;
+        }
+        const float vstar = __uint_as_float(lo);
+        const float s_gt = sum_ge(lo + 1u);
+        const int c_gt = count_ge(lo + 1u), c_eq = count_ge(lo) - c_gt;
+        int m = c_eq;                                           // fewest ties at v* reaching p
+        if (vstar > 0.f) {
+            const float need = ceilf((top_p - s_gt) / vstar);
+            m = need < 1.f ? 1 : (need > (float)c_eq ? c_eq : (int)need);
+        }
+        const int n_p = c_gt + m;
+        if (n_p >= n_k) {
+            const float c_at = s_gt + (float)m * vstar;
+            const float c_before = n_p >= 2 ? c_at - vstar : -INFINITY;
+            c.gap_p = fminf(fabsf(c_at - top_p), fabsf(top_p - c_before));
+            c.n = n_p;
+            c.vb = lo;
+            c.need_eq = m;
+            return c;
+        }
+        // rounding put n_p below n_k after S_k fell short of p: Top-k sets n
+    }
+    c.n = n_k;
+    c.vb = lo_k;
+    c.need_eq = n_k - gt_k;
+    return c;
+}
+
+__device__ __forceinline__ void clear_row(uint32_t* srow, int SW, int lane, int nthreads, int32_t* cnt, float* mg) {
+    for (int w = lane; w < SW; w += nthreads) srow[w] = 0u;
+    if (lane == 0) {
+        *cnt = 0;
+        if (mg) *mg = INFINITY;
+    }
+}
+
+// One warp per row, C values a lane in registers (value j = 32 c + lane; the
+// padding lanes hold -1, below every threshold since thresholds are >= 0).
+template <int C, int CLO>
+__global__ void __launch_bounds__(32 * kWarpRowsPerCta) k_select_reg(const float* __restrict__ P,
+                                                                     const int32_t* __restrict__ n_blk, int64_t MB,
+                                                                     int SW, int top_k, float top_p,
+                                                                     uint32_t* __restrict__ sel,
+                                                                     int32_t* __restrict__ sel_count,
+                                                                     float* __restrict__ margin) {
+    const int nb = *n_blk;
+    if ((CLO > 0 && nb <= 32 * CLO) || nb > 32 * C) return;          // another size class
+    const int lane = threadIdx.x & 31;
+    const int i = blockIdx.x * kWarpRowsPerCta + (threadIdx.x >> 5), hh = blockIdx.y;
+    if (i >= MB) return;                                             // warp-uniform
+    const int64_t ri = (int64_t)hh * MB + i;
+    uint32_t* srow = sel + ri * SW;
+    if (i >= nb) {
+        clear_row(srow, SW, lane, 32, sel_count + ri, margin ? margin + ri : nullptr);
         return;
     }
     const float* prow = P + ((int64_t)hh * nb + i) * nb;
-    for (int j = tid; j < nb; j += TPR) row[j] = prow[j];
-    if (kWarp) __syncwarp();
-    else __syncthreads();
+    float x[C];
+#pragma unroll
+    for (int c = 0; c < C; ++c) {
+        const int j = 32 * c + lane;
+        x[c] = j < nb ? __ldg(prow + j) : -1.f;
+    }
+    // four accumulators in a fixed pattern, then a butterfly: a fixed order
+    auto count_ge = [&](uint32_t t) {
+        const float tf = __uint_as_float(t);
+        int a[4] = {0, 0, 0, 0};
+#pragma unroll
+        for (int c = 0; c < C; ++c) a[c & 3] += x[c] >= tf ? 1 : 0;
+        return warp_sum_i((a[0] + a[1]) + (a[2] + a[3]));
+    };
+    auto sum_ge = [&](uint32_t t) {
+        const float tf = __uint_as_float(t);
+        float a[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int c = 0; c < C; ++c) a[c & 3] += x[c] >= tf ? x[c] : 0.f;
+        return warp_sum((a[0] + a[1]) + (a[2] + a[3]));
+    };
+    const SelCut cut = select_cut(nb, top_k, top_p, count_ge, sum_ge);
+    const bool all = cut.n >= nb;
+    const float vbf = __uint_as_float(cut.vb);
+    // bitmask in index order: word c is chunk c; a running count ranks ties by index
+    const uint32_t below_me = (1u << lane) - 1u;
+    int eq_seen = 0;
+#pragma unroll
+    for (int c = 0; c < C; ++c) {
+        if (32 * c < nb) {                                           // warp-uniform
+            const bool in = 32 * c + lane < nb;
+            const bool gt = in && (all || x[c] > vbf);
+            const bool eq = in && !all && x[c] == vbf;
+            const uint32_t eqmask = __ballot_sync(0xffffffffu, eq);
+            const int rank = eq_seen + __popc(eqmask & below_me);
+            const uint32_t word = __ballot_sync(0xffffffffu, gt || (eq && rank < cut.need_eq));
+            eq_seen += __popc(eqmask);
+            if (lane == 0) srow[c] = word;
+        }
+    }
+    for (int w = (nb + 31) / 32 + lane; w < SW; w += 32) srow[w] = 0u;
+    // margins: order gap at the boundary, and the cumulative-sum gap
+    float gap_o = INFINITY;
+    if (!all) {
+        const int c_ge = count_ge(cut.vb);
+        float below = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < C; ++c)
+            if (x[c] >= 0.f && x[c] < vbf) below = fmaxf(below, x[c]);
+        below = warp_max(below);
+        gap_o = c_ge > cut.n ? 0.f : vbf - below;
+    }
+    if (lane == 0) {
+        sel_count[ri] = cut.n;
+        if (margin) margin[ri] = fminf(gap_o, cut.gap_p);
+    }
+}
 
-    // sum and count of {P >= t}, {P > t}, {P == t} over the row
+// One CTA per row, the row in shared memory (rows above kWarpRowMax blocks).
+__global__ void __launch_bounds__(kSelectThreads) k_select_cta(const float* __restrict__ P,
+                                                              const int32_t* __restrict__ n_blk, int64_t MB,
+                                                              int SW, int top_k, float top_p,
+                                                              uint32_t* __restrict__ sel,
+                                                              int32_t* __restrict__ sel_count,
+                                                              float* __restrict__ margin,
+                                                              uint32_t* __restrict__ dev_status) {
+    extern __shared__ float row[];
+    __shared__ SelRed red;
+    const int nb = *n_blk;
+    if (nb <= kWarpRowMax) return;                                  // the warp form's rows
+    const int tid = threadIdx.x;
+    const int i = blockIdx.x, hh = blockIdx.y;
+    const int64_t ri = (int64_t)hh * MB + i;
+    uint32_t* srow = sel + ri * SW;
+    if (i >= nb || nb > kSelectMaxRow) {
+        clear_row(srow, SW, tid, kSelectThreads, sel_count + ri, margin ? margin + ri : nullptr);
+        if (tid == 0 && nb > kSelectMaxRow && i == 0 && hh == 0) atomicOr(dev_status, PRISM_DEV_BAD_INDEX);
+        return;
+    }
+    const float* prow = P + ((int64_t)hh * nb + i) * nb;
+    for (int j = tid; j < nb; j += kSelectThreads) row[j] = prow[j];
+    __syncthreads();
     auto sum_ge = [&](uint32_t tb) {
         float s = 0.f;
-        for (int j = tid; j < nb; j += TPR) {
+        for (int j = tid; j < nb; j += kSelectThreads) {
             const float x = row[j];
             if (__float_as_uint(x) >= tb) s += x;
         }
-        return kWarp ? warp_sum(s) : sel_sum(s, red);
+        return sel_sum(s, red);
     };
     auto count_ge = [&](uint32_t tb) {
         int c = 0;
-        for (int j = tid; j < nb; j += TPR) c += __float_as_uint(row[j]) >= tb;
-        return kWarp ? warp_sum_i(c) : sel_count_i(c, red);
+        for (int j = tid; j < nb; j += kSelectThreads) c += __float_as_uint(row[j]) >= tb;
+        return sel_count_i(c, red);
     };
-
-    const int n_k = min(top_k, nb);
-    int n_p = nb;
-    float gap_p = INFINITY;
-    const float total = sum_ge(0u);
-    if (top_p < 1.f) {
-        float c_at, c_before;
-        if (total >= top_p) {
-            // largest bit pattern t with sum{P >= t} >= p: lo keeps the property, hi does not
-            uint32_t lo = 0u, hi = 0x3F800001u;                 // (1.0f bits) + 1
-            while (hi - lo > 1u) {
-                const uint32_t mid = lo + ((hi - lo) >> 1);
-                if (sum_ge(mid) >= top_p) lo = mid;
-                else hi = mid;
-            }
-            const float vstar = __uint_as_float(lo);
-            const float s_gt = sum_ge(lo + 1u);
-            const int c_gt = count_ge(lo + 1u), c_eq = count_ge(lo) - c_gt;
-            int m = c_eq;                                       // fewest ties at v* reaching p
-            if (vstar > 0.f) {
-                const float need = ceilf((top_p - s_gt) / vstar);
-                m = need < 1.f ? 1 : (need > (float)c_eq ? c_eq : (int)need);
-            }
-            n_p = c_gt + m;
-            c_at = s_gt + (float)m * vstar;
-            c_before = n_p >= 2 ? c_at - vstar : -INFINITY;
-        } else {                                                // the sum never reaches p: everything
-            n_p = nb;
-            c_at = total;
-            c_before = -INFINITY;                               // refined below if it matters
-        }
-        if (n_p >= n_k) gap_p = fminf(fabsf(c_at - top_p), fabsf(top_p - c_before));
-    }
-    const int n = max(n_k, n_p);
-
-    // threshold of the first n entries of the order (P desc, j asc)
-    uint32_t vb = 0u;
-    int c_gt = 0, need_eq = n;
-    if (n < nb) {
-        uint32_t lo = 0u, hi = 0x3F800001u;                     // count{P >= lo} >= n > count{P >= hi}
-        while (hi - lo > 1u) {
-            const uint32_t mid = lo + ((hi - lo) >> 1);
-            if (count_ge(mid) >= n) lo = mid;
-            else hi = mid;
-        }
-        vb = lo;
-        c_gt = count_ge(lo + 1u);
-        need_eq = n - c_gt;
-    }
+    const SelCut cut = select_cut(nb, top_k, top_p, count_ge, sum_ge);
+    const bool all = cut.n >= nb;
     // bitmask in index order (warp 0; a running count ranks ties by index)
     if (tid < 32) {
         int eq_seen = 0;
@@ -183,31 +287,30 @@ __global__ void __launch_bounds__(kSelectThreads) k_block_select(const float* __
             uint32_t word = 0u;
             if (w < wn) {
                 const int j = w * 32 + tid;
-                const uint32_t xb = j < nb ? __float_as_uint(row[j]) : 0u;
                 const bool in = j < nb;
-                const bool gt = in && (n >= nb || xb > vb);
-                const bool eq = in && n < nb && xb == vb;
+                const uint32_t xb = in ? __float_as_uint(row[j]) : 0u;
+                const bool gt = in && (all || xb > cut.vb);
+                const bool eq = in && !all && xb == cut.vb;
                 const uint32_t eqmask = __ballot_sync(0xffffffffu, eq);
                 const int rank = eq_seen + __popc(eqmask & ((1u << tid) - 1u));
-                word = __ballot_sync(0xffffffffu, gt || (eq && rank < need_eq));
+                word = __ballot_sync(0xffffffffu, gt || (eq && rank < cut.need_eq));
                 eq_seen += __popc(eqmask);
             }
             if (tid == 0) srow[w] = word;
         }
     }
-    // margins: order gap at the boundary, and the cumulative-sum gap
     float gap_o = INFINITY;
-    if (n < nb) {
-        const int c_ge = count_ge(vb);
+    if (!all) {
+        const int c_ge = count_ge(cut.vb);
         float below = -INFINITY;
-        for (int j = tid; j < nb; j += TPR)
-            if (__float_as_uint(row[j]) < vb) below = fmaxf(below, row[j]);
-        below = kWarp ? warp_max(below) : sel_max(below, red);
-        gap_o = c_ge > n ? 0.f : __uint_as_float(vb) - below;
+        for (int j = tid; j < nb; j += kSelectThreads)
+            if (__float_as_uint(row[j]) < cut.vb) below = fmaxf(below, row[j]);
+        below = sel_max(below, red);
+        gap_o = c_ge > cut.n ? 0.f : __uint_as_float(cut.vb) - below;
     }
     if (tid == 0) {
-        sel_count[(int64_t)hh * MB + i] = n;
-        if (margin) margin[(int64_t)hh * MB + i] = fminf(gap_o, gap_p);
+        sel_count[ri] = cut.n;
+        if (margin) margin[ri] = fminf(gap_o, cut.gap_p);
     }
 }
 
@@ -282,25 +385,36 @@ extern "C" prism_status_t prism_block_select(const prism_problem_t* prob, const 
         !ok_ptr(sel_count) || !ok_ptr(gsel) || !ok_opt(gselT) || !ok_opt(margin) || !ok_ptr(dev_status))
         return PRISM_ERR_INVALID_ARG;
     if (top_k < 0 || !(top_p > 0.f) || !isfinite(top_p)) return PRISM_ERR_INVALID_ARG;
-    // n_blk is known on the device only: both forms are launched and each
-    // handles the rows of its own size class (the other exits at once)
-    const int rowcap = (int)(d.MB < kSelectMaxRow ? d.MB : kSelectMaxRow);
-    const int wrowcap = (int)(d.MB < kWarpRowMax ? d.MB : kWarpRowMax);
-    const size_t smem = (size_t)rowcap * sizeof(float), wsmem = (size_t)kWarpRowsPerCta * wrowcap * sizeof(float);
-    if (cudaFuncSetAttribute(k_block_select<kSelectThreads>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem) != cudaSuccess ||
-        cudaFuncSetAttribute(k_block_select<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)wsmem) !=
+    // n_blk is known on the device only: every size class that n_blk <= MB can
+    // reach is launched, and each kernel handles only the rows of its own class
+    const dim3 wgrid((unsigned)((d.MB + kWarpRowsPerCta - 1) / kWarpRowsPerCta), (unsigned)d.heads);
+    const int wthreads = 32 * kWarpRowsPerCta;
+    int launches = 0;
+#define PRISM_SELECT_CLASS(C, CLO)                                                                        \
+    if (d.MB > 32 * (CLO)) {                                                                             \
+        k_select_reg<C, CLO><<<wgrid, wthreads, 0, stream>>>(P, n_blk, d.MB, (int)d.SW, top_k, top_p, sel, \
+                                                              sel_count, margin);                        \
+        ++launches;                                                                                      \
+    }
+    PRISM_SELECT_CLASS(16, 0)
+    PRISM_SELECT_CLASS(32, 16)
+    PRISM_SELECT_CLASS(64, 32)
+    PRISM_SELECT_CLASS(128, 64)
+#undef PRISM_SELECT_CLASS
+    if (d.MB > kWarpRowMax) {
+        const int rowcap = (int)(d.MB < kSelectMaxRow ? d.MB : kSelectMaxRow);
+        const size_t smem = (size_t)rowcap * sizeof(float);
+        if (cudaFuncSetAttribute(k_select_cta, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
             cudaSuccess)
-        return PRISM_ERR_CUDA;
-    k_block_select<32><<<dim3((unsigned)((d.MB + kWarpRowsPerCta - 1) / kWarpRowsPerCta), (unsigned)d.heads),
-                         32 * kWarpRowsPerCta, wsmem, stream>>>(P, n_blk, d.MB, (int)d.SW, wrowcap, top_k, top_p,
-                                                                sel, sel_count, margin, dev_status);
-    k_block_select<kSelectThreads><<<dim3((unsigned)d.MB, (unsigned)d.heads), kSelectThreads, smem, stream>>>(
-        P, n_blk, d.MB, (int)d.SW, rowcap, top_k, top_p, sel, sel_count, margin, dev_status);
+            return PRISM_ERR_CUDA;
+        k_select_cta<<<dim3((unsigned)d.MB, (unsigned)d.heads), kSelectThreads, smem, stream>>>(
+            P, n_blk, d.MB, (int)d.SW, top_k, top_p, sel, sel_count, margin, dev_status);
+        ++launches;
+    }
     k_sel_expand<<<dim3((unsigned)d.MB, (unsigned)d.heads), 128, (size_t)d.SW * 4, stream>>>(
         sel, blk_start, gran_blk, n_blk, d.MB, (int)d.SW, gsel);
     if (gselT)
         k_bit_transpose<<<dim3((unsigned)d.SW, (unsigned)((d.SW + 7) / 8), (unsigned)d.heads), 256, 0, stream>>>(
             gsel, d.MB, (int)d.SW, gselT);
-    return launch_status(gselT ? 4 : 3);
+    return launch_status(launches + (gselT ? 2 : 1));
 }

@@ -31,7 +31,7 @@ template <> struct VidTraits<float> { static constexpr int CPL = 1; };          
 
 // ws layout: video partial sums [Z][nchunk][4] then audio stats [Z][4]
 template <typename T>
-__global__ void __launch_bounds__(256) k_zone_video(const T* __restrict__ V, int H, int W, int64_t D,
+__global__ void __launch_bounds__(256, 2) k_zone_video(const T* __restrict__ V, int H, int W, int64_t D,
                                                     int nchunk, float* __restrict__ part) {
     constexpr int CPL = VidTraits<T>::CPL;
     constexpr int CH = 32 * CPL;                    // channels per CTA
