@@ -51,3 +51,18 @@ def test_inference_layer_keeps_no_backward_state():
     assert a["plan"] == b["plan"] and a["blocked_qkv"] == b["blocked_qkv"] and a["scores"] == b["scores"]
     with pytest.raises(RuntimeError):
         m.backward(torch.empty(1))
+
+
+def test_long_clip_layer_fits_one_gpu():
+    # 112x72x128 grid (1,032,192 tokens), 24 heads of 128, bf16: the training layer's buffers
+    # (P at its worst case, n_blk = N/64) plus raster Q, K, V, dO, O, dQ, dK, dV and hhat stay
+    # inside the 180 GB of one GPU; inference needs about half
+    T, H, W, heads, d = 112, 72, 128, 24, 128
+    N = T * H * W
+    io_train = 8 * N * heads * d * 2 + N * 64 * 2
+    io_infer = 4 * N * heads * d * 2 + N * 64 * 2
+    for wb, io in ((True, io_train), (False, io_infer)):
+        m = PrismSparseAttention(T, H, W, heads, d, 64, "bf16", 8, 0.95, device="meta", with_backward=wb)
+        tot = m.memory_report()["total"] + io
+        assert tot < 180e9, (wb, tot)
+    assert m.memory_report()["scores"] == 2 * heads * (N // 64) * d * 4 + heads * (N // 64) ** 2 * 4
