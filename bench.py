@@ -69,6 +69,7 @@ class ClockSampler:
         self.proc = None
         self.lines = []
         self.t = None
+        self.t0 = None
 
     def start(self):
         try:
@@ -81,14 +82,29 @@ class ClockSampler:
             return
         self.t = threading.Thread(target=self._read, daemon=True)
         self.t.start()
+        # the first sample must precede the timed region: a short region would otherwise end
+        # before nvidia-smi prints anything
+        t_end = time.monotonic() + 5.0
+        while not self.lines and time.monotonic() < t_end and self.proc.poll() is None:
+            time.sleep(0.01)
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.lines.append((time.monotonic(), line.strip()))
+
+    def mark(self):
+        """Start of the timed region: samples before it only stand in when none falls inside."""
+        self.t0 = time.monotonic()
 
     def stop(self):
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        # a region shorter than the 200 ms period: take the first sample after it (the clocks
+        # right after the load) rather than the idle one before it
+        t_end = time.monotonic() + 1.0
+        while (self.t0 is not None and not any(t >= self.t0 for t, _ in self.lines)
+               and time.monotonic() < t_end):
+            time.sleep(0.01)
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
@@ -98,7 +114,9 @@ class ClockSampler:
             self.t.join(timeout=2)
         sm, smax, reasons = [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
+        inside = [ln for t, ln in self.lines if self.t0 is None or t >= self.t0]
+        n_inside = len(inside)
+        for ln in inside:
             parts = [x.strip() for x in ln.split(",")]
             if len(parts) < 9:
                 continue
@@ -113,7 +131,7 @@ class ClockSampler:
         if not sm:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
-                "samples": len(sm)}
+                "samples": len(sm), "samples_from_region_start": n_inside}
 
 
 # ---------------------------------------------------------------- helpers
@@ -288,6 +306,7 @@ def bench_prism(args, cfg, rank, world, local_rank):
     start = torch.cuda.Event(enable_timing=True)
     stop = torch.cuda.Event(enable_timing=True)
     n0 = _abi.launch_count()
+    clocks.mark()
     start.record()
     for t in timers:
         run_step(mod, x, out, grads, t)

@@ -13,7 +13,9 @@
 //
 // Kernels (all reductions in a fixed order, no float atomics, so the result
 // is deterministic):
-//   k_zone_video    grid (Z, D/CH): one CTA per zone x channel chunk; warp w
+//   k_zone_video    grid (D/CH, Z): one CTA per channel chunk x zone, chunks
+//                   fastest (the CTAs resident together read whole token rows
+//                   of one zone; zones fastest measured the same); warp w
 //                   holds temporal slice t = w of the zone, each lane CPL
 //                   channels, 64 tokens kept in registers for the two-pass
 //                   (mean first, then squared deviations) variance.
@@ -41,7 +43,7 @@ __global__ void __launch_bounds__(256, 2) k_zone_video(const T* __restrict__ V, 
     __shared__ float red[8][4];
 
     const int lane = threadIdx.x & 31, t = threadIdx.x >> 5;
-    const int m = blockIdx.x, chunk = blockIdx.y;
+    const int chunk = blockIdx.x, m = blockIdx.y;
     const int ZH = H / 8, ZW = W / 8;
     const int zt = m / (ZH * ZW), zh = (m / ZW) % ZH, zw = m % ZW;
     const int64_t c0 = (int64_t)chunk * CH + lane * CPL;
@@ -266,7 +268,7 @@ extern "C" prism_status_t prism_zone_indicator_ex(const prism_problem_t* prob, c
     float* part = (float*)ws;
     float* astat = part + d.Z * nchunk * 4;
     float* vsum = astat + d.Z * 4;
-    dim3 gv((unsigned)d.Z, (unsigned)nchunk);
+    dim3 gv((unsigned)nchunk, (unsigned)d.Z);                 // Z <= 2^24 / 512 = 32768 < 65536
     if (d.dtype == PRISM_BF16) {
         k_zone_video<__nv_bfloat16><<<gv, 256, 0, stream>>>((const __nv_bfloat16*)V, d.H, d.W, d.D,
                                                              nchunk, part);
