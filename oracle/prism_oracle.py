@@ -22,8 +22,7 @@ guides and a news page.  Citation keys used below:
   [NEWS-4]     sd114.wiki news page, "工作原理" step 4: sparse kernel over the
                selected blocks, then restore the original spatio-temporal layout
 
-Readings where the pages are silent, garbled or ambiguous (each also listed in
-the design notes, numbered as there):
+Readings where the pages are silent, garbled or ambiguous:
   R1  D = all heads x head_dim channels of V; one shape per zone, shared by heads.
   R2  rho(m) = max(rho_v(m), abar(m)), rho_v = zone's mean token variance of V
       over channels, divided by its maximum over the zones of the grid.
@@ -42,6 +41,16 @@ the design notes, numbered as there):
   R13 Top-p = the shortest prefix of the order (P desc, j asc) whose sum is
       >= p; p >= 1 or a sum that never reaches p -> all blocks.
   R14 no forced diagonal block.   R15 non-causal, scale 1/sqrt(d).   R16 batch 1.
+  R17 the GPU accumulates stages 1-5 in fp32 from the stored dtype; this oracle
+      reads the same stored values in fp64, and decisions are compared outside a
+      1e-5 near-tie margin.
+  R18 Delta = rowsum(dO * O) uses the unrounded O (an fp32 copy for bf16 storage).
+  R19 single-guidance ablations: video only -> g_d = r_{v,d} + eps, rho = rho_v;
+      audio only -> g_d = abar * vhat_{a,d} + eps, rho = abar.
+  R20 fixed-shape baseline: one candidate shape for every zone, ignoring g, rho
+      and tau; the permutation and everything after it are unchanged.
+  R21 Top-p only is k = 0; Top-k only is a p so small that the Top-p prefix is
+      one block.
 
 Shape ids: the 16 candidates numbered by (volume, b_T, b_H, b_W) ascending.
 
