@@ -239,9 +239,9 @@ k_bwd_dq_sm100(const __nv_bfloat16* __restrict__ Qg, const __nv_bfloat16* __rest
                const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                const __grid_constant__ CUtensorMap tmdQ, const __grid_constant__ CUtensorMap tmPq,
                const uint32_t* __restrict__ gsel, const PlanHeader* __restrict__ hdr,
-               const int4* __restrict__ items, float* __restrict__ part, const float* __restrict__ lse,
+               const int4* __restrict__ items, const float* __restrict__ lse,
                const float* __restrict__ delta, int64_t N, int64_t MB, int SW, int nst, float scale,
-               __nv_bfloat16* __restrict__ dQ, uint32_t* __restrict__ dev_status) {
+               uint32_t* __restrict__ dev_status) {
     using L = BwdLayout<D, false>;
     // TMEM: dQ, S / dP of two granules, and the tile's Q and dO as bf16 (the A
     // operands of S = Q K^T and dP = dO V^T, read by the tensor core from TMEM)
@@ -422,9 +422,8 @@ k_bwd_dkdv_sm100(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
                  const __grid_constant__ CUtensorMap tmdK, const __grid_constant__ CUtensorMap tmdV,
                  const __grid_constant__ CUtensorMap tmPkv,
                  const uint32_t* __restrict__ gselT, const PlanHeader* __restrict__ hdr,
-                 const int4* __restrict__ items, float* __restrict__ part, const float* __restrict__ nld,
-                 int64_t N, int64_t MB, int SW, int nst, float scale, __nv_bfloat16* __restrict__ dK, __nv_bfloat16* __restrict__ dV,
-                 uint32_t* __restrict__ dev_status) {
+                 const int4* __restrict__ items, const float* __restrict__ nld,
+                 int64_t N, int64_t MB, int SW, int nst, float scale, uint32_t* __restrict__ dev_status) {
     using L = BwdLayout<D, true>;
     constexpr uint32_t cdK = 0, cdV = 128, cS = 256, cP = 320;   // + 128 * buffer for S^T / dP^T
     if ((int)blockIdx.x >= hdr->n_items) return;      // uniform: beyond the item list
@@ -656,13 +655,10 @@ prism_status_t launch_bwd(const Dims& d, const void* Qp, const void* Kp, const v
         cudaFuncSetAttribute(kk, cudaFuncAttributeMaxDynamicSharedMemorySize, smk) != cudaSuccess)
         return PRISM_ERR_CUDA;
     kq<<<(unsigned)w.pq.items_max, 192, smq, s>>>((const __nv_bfloat16*)Qp, (const __nv_bfloat16*)dOp, gK, gV, tdQ, tPq,
-                                                  gsel, w.pq.hdr, w.pq.items, w.part_q, lse,
-                                                  w.delta, d.N, d.MB, (int)d.SW, nq, scale, (__nv_bfloat16*)dQp,
-                                                  dev_status);
+                                                  gsel, w.pq.hdr, w.pq.items, lse,
+                                                  w.delta, d.N, d.MB, (int)d.SW, nq, scale, dev_status);
     kk<<<(unsigned)w.pkv.items_max, 384, smk, s>>>(tK, tV, gQ, gdO, tdK, tdV, tPkv, gselT, w.pkv.hdr, w.pkv.items,
-                                                   w.part_kv, w.nld,
-                                                   d.N, d.MB, (int)d.SW, nk, scale, (__nv_bfloat16*)dKp,
-                                                   (__nv_bfloat16*)dVp, dev_status);
+                                                   w.nld, d.N, d.MB, (int)d.SW, nk, scale, dev_status);
     st = launch_status(2);
     if (st == PRISM_OK) st = bwd_combine(w.pq, d, 1, w.part_q, dQp, scale, nullptr, 0.f, s);
     if (st == PRISM_OK) st = bwd_combine(w.pkv, d, 2, w.part_kv, dKp, scale, dVp, 1.f, s);
