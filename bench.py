@@ -39,11 +39,11 @@ from dynamic_block_sparse_macro_b200.configs import get_config  # noqa: E402
 METRIC = "sparse attn fwd+bwd ms/layer & TFLOP/s on selected blocks, 2K grid (295k tok)"
 METRIC_FWD = "sparse attn fwd ms/layer & TFLOP/s on selected blocks, 2K grid (295k tok), inference"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-# DRAM bytes (read + write) of one backward call on the 2K layer with 24 heads, from an ncu
-# capture of the backward kernels on 4 heads scaled by 6 (their per-head working set is the
-# same) plus the Delta kernel's algorithmic bytes: profiles/bwd_kernels_2k_4heads.txt.
-# Only valid for the kernels as they were captured; None elsewhere.
-BWD_DRAM_BYTES = {("2k", 24): 31.3e9}
+# DRAM bytes (read + write) of one backward call, by (config, heads), from an ncu capture of
+# the backward kernels as they now stand.  The last capture (profiles/bwd_kernels_2k_4heads.txt:
+# 31.3 GB at 24 heads) predates the TMA-store epilogues, so no entry is valid and the
+# roofline's traffic is null until the kernels are captured again.
+BWD_DRAM_BYTES = {}
 
 
 def metric_name(cfg, fwd_only):
