@@ -213,11 +213,12 @@ prism_status_t prism_block_pool_score(const prism_problem_t* prob, const void* Q
  *             granule) has bit kg set when the block of key granule kg is in S
  *             of the block of qg (blk_start, gran_blk from prism_assign_shapes)
  *   gselT     [heads][N/64][sel_words] uint32 (nullable): transpose of gsel, the
- *             key-major view of the backward
+ *             key-major view of the backward (inference passes NULL)
  *   margin    [heads][max_blocks] float32 (nullable): smallest gap (order or
  *             cumulative-sum) that, crossed by rounding, could change S_i
- *   dev_status  PRISM_DEV_BAD_INDEX if n_blk exceeds the 16384 keys a row can
- *             sort in shared memory (then every row is left empty).
+ *   dev_status  PRISM_DEV_BAD_INDEX if n_blk exceeds 16384, the longest row the
+ *             selection holds on chip (rows of up to 4096 blocks sit in registers,
+ *             longer ones in shared memory); every row is then left empty.
  * Rows i >= n_blk are written as empty rows with count 0.
  */
 prism_status_t prism_block_select(const prism_problem_t* prob, const float* P, const int32_t* blk_start,
