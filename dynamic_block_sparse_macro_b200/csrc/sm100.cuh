@@ -315,33 +315,6 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return r;
 }
 
-// 2^x on the FMA pipe, two values at a time, for x <= 0 (the softmax
-// exponents after the running max is subtracted).  Cody and Waite's range
-// reduction: x = j + f with j = round(x) (by adding 1.5 * 2^23, whose ulp is 1)
-// and f in [-1/2, 1/2]; 2^f by a cubic fitted to 2^f on that interval
-// (weighted least squares towards minimal relative error; in fp32 its
-// relative error stays below 8e-5, far under the bf16 rounding of P); the
-// result's exponent field is then raised by j.  x is clamped at -126 so that
-// the exponent field stays >= 0 (2^-126 is nothing next to the row maximum's 1).
-constexpr float kExp2C0 = 0.99992806f, kExp2C1 = 0.69326097f, kExp2C2 = 0.24261113f, kExp2C3 = 0.05517166f;
-__device__ __forceinline__ void exp2_poly2(float x0, float x1, float& y0, float& y1) {
-    const float kRound = 12582912.0f;                       // 1.5 * 2^23
-    x0 = fmaxf(x0, -126.f);
-    x1 = fmaxf(x1, -126.f);
-    const uint64_t t = fadd2(f2pack(x0, x1), f2pack(kRound, kRound));
-    const uint64_t j = fadd2(t, f2pack(-kRound, -kRound));
-    const uint64_t f = ffma2(j, f2pack(-1.f, -1.f), f2pack(x0, x1));
-    uint64_t p = ffma2(f, f2pack(kExp2C3, kExp2C3), f2pack(kExp2C2, kExp2C2));
-    p = ffma2(p, f, f2pack(kExp2C1, kExp2C1));
-    p = ffma2(p, f, f2pack(kExp2C0, kExp2C0));
-    float p0, p1, t0, t1;
-    f2unpack(p, p0, p1);
-    f2unpack(t, t0, t1);
-    // the low bits of t hold j (two's complement); j << 23 lands on the exponent field
-    y0 = __int_as_float(__float_as_int(t0) * (1 << 23) + __float_as_int(p0));
-    y1 = __int_as_float(__float_as_int(t1) * (1 << 23) + __float_as_int(p1));
-}
-
 // Walks the union of R granule-level selection rows held consecutively in
 // shared memory (row i at rows + i * words) in ascending granule order; the
 // R-bit mask says which rows have the granule.
