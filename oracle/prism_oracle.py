@@ -217,7 +217,10 @@ def assign_shapes(g, rho, tau128=TAU_128, tau256=TAU_256):
 
     Returns dict: shape_id [Z], edges [Z,3], B [Z], ell [Z,3], dist2 [Z,16]
     (inf for candidates of another volume), margin_shape (second best minus
-    best squared distance), margin_volume (min |rho - tau|).
+    best squared distance: moving l* by delta shifts the gap between candidates
+    c and c' by 2 delta . (e_c - e_c'), so the choice holds while that stays
+    below the gap), margin_volume (min |rho - tau|: the distance rho may move
+    before B changes).
     """
     edges, vol = candidate_shapes()
     loge = np.log2(edges.astype(np.float64))
@@ -322,8 +325,9 @@ def block_select(P, top_k, top_p):
     """S_i = Top-k(P_i, k) U Top-p(P_i, p), both prefixes of the order (P desc, j asc).
 
     P: [..., n_blk, n_blk].  Returns dict: sel bool [..., nb, nb], count
-    [..., nb], n_k, n_p, and margin [..., nb]: the smallest gap that, if
-    crossed by rounding, could change the selected set (inf if none).
+    [..., nb], n_k, n_p, and margin [..., nb]: the L1 norm below which no
+    perturbation of the row (rounding of P included) can change the selected
+    set, and above which one can (inf if none can).
     """
     P = np.asarray(P, dtype=np.float64)
     nb = P.shape[-1]
@@ -342,23 +346,30 @@ def block_select(P, top_k, top_p):
     sel = np.zeros(P.shape, dtype=bool)
     np.put_along_axis(sel, order, sel_sorted, axis=-1)
 
-    # decision margins
+    # Decision margin: the L1 size of the smallest perturbation of the row (kept
+    # non-negative) that can change S_i.  S_i is the n = max(n_k, n_p) largest
+    # values, and the sum of the m largest values moves by at most the L1 norm
+    # of a perturbation, so S_i changes only through one of three events:
+    #   order: a value outside S_i overtakes one inside (gap between the n-th
+    #          and the (n+1)-th value of the order);
+    #   up:    the sum of the n largest drops below p, so that n_p exceeds n;
+    #   down:  Top-p sets n (n_p > n_k) and the sum of the n-1 largest reaches
+    #          p, so that n_p, and with it n, drops by one.
+    # When n_p <= n_k a lower n_p leaves n = n_k, so the sum before the Top-p
+    # crossing decides nothing there.
     inf = np.full(P.shape[:-1], np.inf)
-    nn = np.minimum(n, nb - 1)
-    gap_order = np.where(n < nb,
-                         np.take_along_axis(Ps, (n - 1)[..., None], -1)[..., 0]
-                         - np.take_along_axis(Ps, nn[..., None], -1)[..., 0], inf)
+
+    def at(a, i):
+        return np.take_along_axis(a, np.clip(i, 0, nb - 1)[..., None], -1)[..., 0]
+
+    gap_order = np.where(n < nb, at(Ps, n - 1) - at(Ps, n), inf)
     if top_p < 1.0:
-        c_at = np.take_along_axis(csum, (n_p - 1)[..., None], -1)[..., 0]
-        c_before = np.where(n_p >= 2,
-                            np.take_along_axis(csum, np.maximum(n_p - 2, 0)[..., None], -1)[..., 0],
-                            -np.inf)
-        gap_p = np.minimum(np.abs(c_at - top_p), np.abs(top_p - c_before))
-        gap_p = np.where(n_p >= n_k, gap_p, inf)    # top-p only matters when it can set n
+        gap_up = np.where(n < nb, at(csum, n - 1) - top_p, inf)
+        gap_down = np.where((n_p > n_k) & (n_p >= 2), top_p - at(csum, n - 2), inf)
     else:
-        gap_p = inf
+        gap_up = gap_down = inf
     return {"sel": sel, "count": n, "n_k": n_k, "n_p": n_p,
-            "margin": np.minimum(gap_order, gap_p)}
+            "margin": np.minimum(gap_order, np.minimum(gap_up, gap_down))}
 
 
 # --------------------------------------------------------------------------
