@@ -47,6 +47,16 @@ class PrismError(RuntimeError):
         self.code = code
 
 
+class PrismDeviceError(RuntimeError):
+    """A kernel set a bit of the device status word."""
+
+    def __init__(self, bits: int):
+        names = [n for b, n in ((DEV_TIMEOUT, "PRISM_DEV_TIMEOUT"), (DEV_BAD_INDEX, "PRISM_DEV_BAD_INDEX"))
+                 if bits & b]
+        super().__init__(f"device status 0x{bits:x} ({', '.join(names) or 'unknown bit'})")
+        self.bits = bits
+
+
 _lib = None
 _P = ctypes.c_void_p
 _I = ctypes.c_int32

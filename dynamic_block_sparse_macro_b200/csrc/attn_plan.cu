@@ -1,8 +1,7 @@
 // Work planning for the tensor-core attention kernels.
 //
 // A tile's work is the union of the granule-level selection rows of its
-// 64-row granules (two for the 128-row tiles of the backward, four for the
-// 256-row tiles of the forward).  That union is data dependent and very uneven (a
+// 64-row granules (two: forward and backward both use 128-row tiles).  That union is data dependent and very uneven (a
 // query block with flat block probabilities makes Top-p select most keys), so
 // one CTA per tile would leave a few CTAs running long after the rest.  The
 // plan cuts every tile into segments of at most `seg` work units, choosing

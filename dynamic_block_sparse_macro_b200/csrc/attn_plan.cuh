@@ -1,6 +1,8 @@
 // Work plan shared by the tensor-core attention kernels (see attn_plan.cu).
 #pragma once
 
+#include <atomic>
+
 #include "common.cuh"
 
 namespace prism {
@@ -31,7 +33,8 @@ constexpr int kSegMinGranules = 16;   // backward: 64-row granules
 
 size_t plan_bytes(int64_t tiles, int target);
 Plan carve_plan(void* base, int64_t tiles, int target);
-// tile_gran: 64-row granules per tile (2 or 4); unit_granules: granules per work unit
+// tile_gran: 64-row granules per tile (2: the 128-row tiles of the forward and
+// the backward); unit_granules: granules per work unit
 prism_status_t plan_work(const Plan& pl, const uint32_t* rows, const Dims& d, int tile_gran, int unit_granules,
                          int target, int seg_min, cudaStream_t s);
 prism_status_t fwd_combine(const Plan& pl, const Dims& d, int tile_rows, const float* opart, const float* mpart,
@@ -39,14 +42,18 @@ prism_status_t fwd_combine(const Plan& pl, const Dims& d, int tile_rows, const f
 prism_status_t bwd_combine(const Plan& pl, const Dims& d, int nout, const float* part, void* out0, float mul0,
                            void* out1, float mul1, cudaStream_t s);
 
-// number of SMs of the current device (cached)
+// number of SMs of the current device (cached per device ordinal; the plan
+// target and the workspace sizes depend on it)
 inline int device_sms() {
-    static int sms = 0;
-    if (!sms) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        if (sms <= 0) sms = 148;
+    constexpr int kMaxDev = 64;
+    static std::atomic<int> cache[kMaxDev];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) dev = 0;
+    int sms = dev < kMaxDev ? cache[dev].load(std::memory_order_relaxed) : 0;
+    if (sms <= 0) {
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+            sms = 148;
+        if (dev < kMaxDev) cache[dev].store(sms, std::memory_order_relaxed);
     }
     return sms;
 }

@@ -307,7 +307,8 @@ extern "C" prism_status_t prism_zone_indicator(const prism_problem_t* prob, cons
 // Host code cannot use the symbol's name as a device address; the address is
 // looked up with cudaGetSymbolAddress once per device, the first time the
 // entry point runs with that device current (so that first call should come
-// before any stream capture).  Every call shares the one array: two calls
+// before any stream capture), and kept for the life of the process: a
+// cudaDeviceReset (or any teardown of the primary context) invalidates it.  Every call shares the one array: two calls
 // whose kernels overlap on the GPU race on it.  Each call writes every
 // scratch word it later reads, so nothing has to be cleared between calls.
 // ---------------------------------------------------------------------------

@@ -107,18 +107,27 @@ class PrismSparseAttention:
         _abi.prism_sparse_attn_fwd(self.prob, self.Qp, self.Kp, self.Vp, self.gsel, self.scale, self.Op,
                                    self.lse, self.Of32, self.dev_status, self.ws_fwd, stream)
 
-    def forward(self, Q, K, V, hhat, out=None, stream=None):
-        """Whole forward; returns O in raster layout."""
+    def forward(self, Q, K, V, hhat, out=None, stream=None, check=True):
+        """Whole forward; returns O in raster layout.
+
+        check: read the device status word once the forward has run (this
+        synchronises the stream) and raise if a kernel flagged a condition:
+        rows beyond the selection's capacity leave every selection row empty
+        and O = 0, and a timed-out wait leaves outputs incomplete.  With
+        check=False nothing synchronises; call ``check_status()`` later."""
         self.plan(V, hhat, stream)
         self.select(Q, K, V, stream)
         self.attend(stream)
         if out is None:
             out = torch.empty_like(Q)
         _abi.prism_unpermute(self.prob, self.Op, self.perm, out, stream)
+        if check:
+            self.check_status(stream)
         return out
 
-    def backward(self, dO, dQ=None, dK=None, dV=None, stream=None):
-        """Stage 7 for the last forward; returns raster (dQ, dK, dV)."""
+    def backward(self, dO, dQ=None, dK=None, dV=None, stream=None, check=True):
+        """Stage 7 for the last forward; returns raster (dQ, dK, dV).  ``check``
+        as in ``forward``."""
         if not self.with_backward:
             raise RuntimeError("this layer was built for inference (with_backward=False)")
         p = self.prob
@@ -132,6 +141,8 @@ class PrismSparseAttention:
                 dst = torch.empty_like(dO)
             _abi.prism_unpermute(p, src, self.perm, dst, stream)
             outs.append(dst)
+        if check:
+            self.check_status(stream)
         return tuple(outs)
 
     # ------------------------------------------------------------------ memory
@@ -161,8 +172,15 @@ class PrismSparseAttention:
         nb = self.num_blocks()
         return self.P[: self.heads * nb * nb].view(self.heads, nb, nb)
 
-    def status(self) -> int:
-        return _abi.prism_read_status(self.dev_status)
+    def status(self, stream=None) -> int:
+        """The device status word (synchronises the stream)."""
+        return _abi.prism_read_status(self.dev_status, stream)
+
+    def check_status(self, stream=None) -> None:
+        """Raise ``PrismDeviceError`` if a kernel of this layer set a status bit."""
+        st = self.status(stream)
+        if st:
+            raise _abi.PrismDeviceError(st)
 
 
 class _PrismFn(torch.autograd.Function):

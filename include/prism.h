@@ -134,7 +134,10 @@ prism_status_t prism_zone_indicator_ex(const prism_problem_t* prob, const void* 
  *  - Nothing is allocated: no cudaMalloc/cudaFree or allocating library call.
  *  - The first call on each device looks up the array's device address
  *    (cudaGetSymbolAddress) with that device current; make that first call
- *    before any stream capture.
+ *    before any stream capture.  The address is kept for the life of the
+ *    process: it does not survive cudaDeviceReset or any other teardown of
+ *    the device's primary context, after which this entry point must not be
+ *    called again on that device in the same process.
  *  - All calls share the array: calls whose kernels overlap on the GPU (two
  *    streams, two host threads) race on it and must be serialised by the caller.
  */

@@ -128,10 +128,11 @@ def test_deterministic_repeat():
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
 def test_inference_layer_matches_training_forward(dtype):
     # with_backward=False: no LSE, no fp32 O, no key-major selection; O and every decision
-    # are the bits of the training layer's forward (whose O the other tests check against
-    # the oracle)
+    # are the bits of the training layer's forward, and O matches the oracle's attention
+    # under the inference layer's own selection
+    import oracle as orc
     from dynamic_block_sparse_macro_b200.layer import PrismSparseAttention
-    from gpu_parity import run_gpu
+    from gpu_parity import REL_L2, block_rel_l2, host, rel_l2, run_gpu, unpack_sel
     cfg = get_config("720p", T=16, H=32, W=32, heads=3, dtype=dtype)
     x = _inputs(cfg)
     mt, Ot, _ = run_gpu(cfg, x, backward=False)
@@ -142,3 +143,11 @@ def test_inference_layer_matches_training_forward(dtype):
     assert mi.status() == 0 and mi.lse is None
     assert torch.equal(mi.perm, mt.perm) and torch.equal(mi.gsel, mt.gsel)
     assert torch.equal(Oi, Ot)
+    nb = mi.num_blocks()
+    bs = mi.blk_start[: nb + 1].cpu().numpy().astype(np.int64)
+    O_ref, _ = orc.sparse_attention_fwd(host(mi.Qp), host(mi.Kp), host(mi.Vp), bs, unpack_sel(mi.sel, nb))
+    Ob = host(mi.Op)
+    tol = REL_L2[dtype]
+    assert rel_l2(Ob, O_ref) <= tol and block_rel_l2(Ob, O_ref, bs) <= 2 * tol
+    perm = mi.perm.cpu().numpy().astype(np.int64)
+    np.testing.assert_array_equal(host(Oi), orc.unpermute(Ob, perm))

@@ -2,11 +2,13 @@
 allocate device memory (a C host with no device allocator of its own, or a
 service whose device footprint is fixed at start-up).  Its scratch is a
 fixed array inside the library; these tests check, through the C ABI, that
-it gives the same results as prism_zone_indicator with a caller-owned
-workspace, on two calls in a row, and that oversize problems are refused.
+it gives the same bits as prism_zone_indicator with a caller-owned
+workspace (both run the same deterministic kernels), on calls in a row and on
+the largest problem the array holds, and that oversize problems are refused.
 
 This file is named so that pytest collects it last."""
 import ctypes
+import types
 
 import numpy as np
 import pytest
@@ -59,4 +61,25 @@ def test_noalloc_matches_workspace_entry_point_twice_in_a_row():
         got = _run(cfg, x, noalloc=True)
         for k in ref:
             assert np.isfinite(got[k]).all(), k
-            np.testing.assert_allclose(got[k], ref[k], rtol=2e-5, atol=1e-6, err_msg=k)
+            np.testing.assert_array_equal(got[k], ref[k], err_msg=k)
+
+
+@pytest.mark.gpu
+def test_noalloc_at_the_scratch_limit():
+    # 256^3 tokens (the most a problem may have: 32,768 zones), one bf16 head of 128
+    # channels: 32,768 zones x 16 floats = exactly the 2 MiB of the array
+    T = H = W = 256
+    prob = _abi.problem(T, H, W, 1, 128, 64, "bf16")
+    sz = _abi.query_sizes(prob)
+    assert sz.ws_indicator == _abi.NOALLOC_SCRATCH_BYTES
+    gen = torch.Generator(device="cuda").manual_seed(20261231)
+    N = T * H * W
+    x = {"V": torch.randn((N, 1, 128), generator=gen, device="cuda", dtype=torch.bfloat16),
+         "hhat": torch.randn((N, 64), generator=gen, device="cuda", dtype=torch.bfloat16)}
+    cfg = types.SimpleNamespace(T=T, H=H, W=W, heads=1, head_dim=128, audio_dim=64, dtype="bf16")
+    for _ in range(2):
+        ref = _run(cfg, x, noalloc=False)
+        got = _run(cfg, x, noalloc=True)
+        for k in ref:
+            assert np.isfinite(got[k]).all(), k
+            np.testing.assert_array_equal(got[k], ref[k], err_msg=k)
