@@ -7,23 +7,26 @@
 //   dV = P^T dO,  dP = dO V^T,  dS = P * (dP - Delta),  dQ = scale dS K,
 //   dK = scale dS^T Q.
 //
-// Two kernels, no atomics (deterministic):
-//   k_bwd_dq_sm100    query-stationary: per (128-row query tile, head) walk the
-//                     key granules of the union of its two granule-level rows;
-//                     Q and dO sit in TMEM as bf16; per 64-key granule S = Q K^T
-//                     and dP = dO V^T (M=128, N=64, A from TMEM) into TMEM, dS
-//                     as bf16 back into TMEM, dQ += dS K (K MN-major in smem).
-//   k_bwd_dkdv_sm100  key-stationary: per (128-key tile, head) walk the query
-//                     granules whose blocks selected the tile's key blocks (the
-//                     transposed granule-level selection); per 64-query granule
-//                     S^T = K Q^T and dP^T = V dO^T, then P^T and dS^T as bf16
-//                     in TMEM, dV += P^T dO and dK += dS^T Q.
+// Two persistent kernels (one CTA per SM looping over the work plan's items),
+// no atomics (deterministic):
+//   k_bwd_dq_persist    query-stationary: per (128-row query tile, head) walk the
+//                       key granules of the union of its two granule-level rows;
+//                       Q and dO sit in TMEM as bf16; per 64-key granule S = Q K^T
+//                       and dP = dO V^T (M=128, N=64, A from TMEM) into TMEM, dS
+//                       as bf16 back into TMEM, dQ += dS K (K MN-major in smem).
+//   k_bwd_dkdv_persist  key-stationary: per (128-key tile, head) walk the query
+//                       granules whose blocks selected the tile's key blocks (the
+//                       transposed granule-level selection); per 64-query granule
+//                       S^T = K Q^T and dP^T = V dO^T, then P^T and dS^T as bf16
+//                       in TMEM, dV += P^T dO and dK += dS^T Q.
 // Both double-buffer the granule products in TMEM so that the tensor core
-// works on granule g+1 while four warps do the elementwise step of granule g,
-// and stream granules through a TMA ring as deep as shared memory allows.
+// works on granule g+1 while the elementwise warps work on granule g, and
+// stream granules through a TMA ring as deep as shared memory allows; ring
+// stages, buffers and barrier phases carry across item edges, so the next
+// item's loads and first products overlap the current item's epilogue.
 // Roles: warp 0 TMA (one lane per ring stage and stream, one whole-row copy
 // per granule), warp 1 TMEM allocation + MMA issue (the whole warp, one
-// elected lane issues), warps 2-5 one tile row per thread.
+// elected lane issues), the other warps one tile row per thread.
 // Every wait is bounded; a timeout sets PRISM_DEV_TIMEOUT.
 #include "attn_plan.cuh"
 #include "common.cuh"
@@ -47,222 +50,212 @@ constexpr uint32_t kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kSmemMax = 227 * 1024;
 // dK/dV kernel register split: 384 threads launch with 168 each; warpgroup 0
-// (TMA, MMA) drops to 120 and the two elementwise warpgroups rise to 192
-// (128 * (120 + 2 * 192) = 384 * 168)
-constexpr uint32_t kRegsLow = 120, kRegsHigh = 192;
-
-// Shared memory: stationary tiles (dK/dV only; the dQ kernel keeps Q and dO
-// in TMEM), then a ring of nst granule stages (as many as fit: the TMA latency
-// under load is about 4000 cycles, a granule's MMAs take about 800), then
-// barriers and the two selection rows.
-template <int D, bool STAT>
-struct BwdLayout {
-    static constexpr int NR = D / 64;
-    static constexpr int A0 = 0;                       // stationary operand 1 (K)
-    static constexpr int A1 = NR * kTile;              // stationary operand 2 (V)
-    static constexpr int RING = STAT ? 2 * NR * kTile : 0;   // streamed granules
-    static constexpr int STAGE = 2 * NR * kGran;       // two operands per stage
-    // xs: bytes of per-granule row data staged beside each stage (0 or kXs)
-    __host__ __device__ static int xs(int nst) { return RING + nst * STAGE; }
-    __host__ __device__ static int ctrl(int nst, int xsb) { return xs(nst) + nst * xsb; }
-    __host__ __device__ static int rows(int nst, int xsb) { return ctrl(nst, xsb) + kCtrl; }
-    static int alloc(int nst, int xsb, int SW) { return rows(nst, xsb) + 8 * SW + 1024; }
-    static int stages(int xsb, int SW) {               // deepest ring that fits, at least 2
-        int n = kStages;
-        while (n > 2 && alloc(n, xsb, SW) > kSmemMax) --n;
-        return n;
-    }
-};
-
-struct Bars {
-    uint64_t* stat;            // stationary tiles landed (one arrival per producer)
-    uint64_t* full0;           // [kStages] streamed operand 0 of a granule landed
-    uint64_t* full1;           // [kStages] streamed operand 1 of a granule landed
-    uint64_t* fullx;           // [kStages] row data of a granule landed (dK/dV only)
-    uint64_t* empty;           // [kStages] granule stage free
-    uint64_t* prod;            // [2] products of a granule in TMEM
-    uint64_t* elem;            // [2] elementwise results of a granule in TMEM (128 arrivals)
-    uint64_t* fin;             // all MMAs done
-    uint32_t* tmem_slot;
-    volatile int* abort_flag;
-    int* ng_slot;
-};
-
-__device__ __forceinline__ Bars carve(uint8_t* ctrl) {
-    uint64_t* b = reinterpret_cast<uint64_t*>(ctrl);
-    Bars r;
-    r.stat = b;
-    r.full0 = b + 1;
-    r.full1 = b + 1 + kStages;
-    r.fullx = b + 1 + 2 * kStages;
-    r.empty = b + 1 + 3 * kStages;
-    r.prod = b + 1 + 4 * kStages;
-    r.elem = b + 3 + 4 * kStages;
-    r.fin = b + 5 + 4 * kStages;
-    r.tmem_slot = reinterpret_cast<uint32_t*>(b + 6 + 4 * kStages);
-    r.abort_flag = reinterpret_cast<volatile int*>(r.tmem_slot + 1);
-    r.ng_slot = reinterpret_cast<int*>(r.tmem_slot + 2);
-    return r;
-}
-static_assert((6 + 4 * kStages) * 8 + 12 <= kCtrl, "barriers overflow the control block");
-
-__device__ __forceinline__ void init_bars(const Bars& B, int nst, int stat_arrivals, int elem_arrivals) {
-    mbar_init(B.stat, stat_arrivals);
-    for (int s = 0; s < nst; ++s) {
-        mbar_init(B.full0 + s, 1);
-        mbar_init(B.full1 + s, 1);
-        mbar_init(B.fullx + s, 1);
-        mbar_init(B.empty + s, 1);
-    }
-    for (int b = 0; b < 2; ++b) {
-        mbar_init(B.prod + b, 1);
-        mbar_init(B.elem + b, elem_arrivals);
-    }
-    mbar_init(B.fin, 1);
-    *B.abort_flag = 0;
-    fence_mbar_init();
-}
+// (TMA, MMA) drops to 152 and the two elementwise warpgroups rise to 176
+// (128 * (152 + 2 * 176) = 384 * 168); the persistent item loop needs more
+// than 136 registers on the TMA/MMA side and fits 176 on the elementwise side
+constexpr uint32_t kRegsLow = 152, kRegsHigh = 176;
 
 // descriptor offsets: K-major operand, k-th 16-element step of the contraction over d
 __device__ __forceinline__ uint32_t kmaj_off(int k, int region) { return (k >> 2) * region + (k & 3) * 32; }
 
-// The TMA producer warp.  A copy engine completes the copies issued by one
-// thread one after another, so every (ring stage, stream) pair gets a lane of
-// its own: lane kind * nst + stage issues stream `kind` (0: operand 0, 1:
-// operand 1, 2: the 512 bytes of row data, dK/dV only) of the granules that
-// use that stage, one copy per granule, and never has more than one copy in
-// flight.  With stationary tiles in shared memory (dK/dV), lanes 0 and nst
-// also copy those.
-template <int D, bool STAT>
-__device__ void produce(const CUtensorMap* m0, const CUtensorMap* m1, const CUtensorMap* g0, const CUtensorMap* g1,
-                        const float* nld, uint8_t* xs, uint8_t* sm, const Bars& B, int64_t row0, int tile_row,
-                        const uint32_t* u0, const uint32_t* u1, int wn, int g_begin, int ng, int nst,
-                        uint32_t* dev_status) {
-    using L = BwdLayout<D, STAT>;
-    const int lane = threadIdx.x & 31;
-    if (lane >= (nld ? 3 : 2) * nst) return;
-    const int kind = lane / nst, stage = lane % nst;
-    uint64_t* full = kind == 0 ? B.full0 : kind == 1 ? B.full1 : B.fullx;
-    const CUtensorMap* mg = kind == 0 ? g0 : g1;
-    if (kind < 2) tma_prefetch_desc(mg);
-    if (STAT && stage == 0 && kind < 2) {
-        const CUtensorMap* ms = kind == 0 ? m0 : m1;
-        mbar_expect_tx(B.stat, L::NR * kTile);
-        tma_load_3d(sm + (kind ? L::A1 : L::A0), ms, B.stat, 0, (int)(row0 + tile_row), 0);
-    }
-    GranuleWalk walk;
-    walk.init(u0, u1, wn);
-    walk.skip(g_begin);
-    int last = -1;
-    for (int g = 0; g < ng && !*B.abort_flag; ++g) {
-        int row;
-        uint32_t m;
-        walk.next(row, m);
-        if (g % nst != stage) continue;
-        if (g >= nst && !mbar_wait(B.empty + stage, ((g / nst) - 1) & 1, B.abort_flag, dev_status)) break;
-        if (kind == 2) {
-            mbar_expect_tx(full + stage, kXs);
-            bulk_load(xs + stage * kXs, nld + ((row0 + row) >> 6) * 128, kXs, full + stage);
-        } else {
-            mbar_expect_tx(full + stage, L::NR * kGran);
-            tma_load_3d(sm + L::RING + stage * L::STAGE + kind * L::NR * kGran, mg, full + stage, 0,
-                        (int)(row0 + row), 0);
-        }
-        last = g;
-    }
-    if (*B.abort_flag && last >= 0) {
-        // let this lane's copy land before the CTA goes away
-        volatile int no_abort = 0;
-        mbar_wait(full + stage, (last / nst) & 1, &no_abort, dev_status);
-    }
-}
+// ============================================================================ dQ (persistent)
+// One CTA per SM takes items blockIdx.x, blockIdx.x + gridDim.x, ...  Granules
+// are numbered G = 0, 1, ... over all of the CTA's items, so the ring stages,
+// the double-buffered S/dP columns and every phase carry across item edges:
+// the producer runs ahead into the next item while the current one finishes,
+// the next item's Q and dO go into TMEM as soon as the current item's last
+// products are consumed, and its first S/dP MMAs overlap the current epilogue.
+// Per local item j:
+//   rows[j & 1]  the tile's two selection rows: the producer's 32 lanes write
+//                them (rows_full, 32 arrivals), the four elementwise warps
+//                release them after their walk (rows_empty, 4 arrivals)
+// Per non-empty item k (items with no granule, ng = 0, never reach the MMA
+// warp: their dQ is zero and written without TMEM, so that no barrier can
+// complete two phases before its waiter has seen the first):
+//   qdo_full     Q, dO of item k in TMEM (128 arrivals), phase k & 1
+//   fin          every MMA of item k complete, phase k & 1
+// The dQ columns are free for item j+1's first dQ MMA once the elementwise
+// warps have arrived on that granule's elem barrier: they do so only after the
+// epilogue of item j has read dQ.
+constexpr int kStagingP = 2 * kTile;       // 32 KB: two 128-byte regions of 128 rows
 
-// Epilogue of a 128-row accumulator tile (D fp32 columns in TMEM; this thread
-// holds row `row`, TMEM address `tacc` = its lane quarter + first column):
-// scaled bf16 (a finished tile) or raw fp32 (the partial of a split tile),
-// written as 16-byte chunks in the 128-byte-swizzled image of the whole-row
-// TMA maps into `stage` (free shared memory, 1024-byte aligned), then stored by
-// the group's leader with one TMA copy.  Per-row 16-byte stores straight to
-// global memory would touch 32 lines per warp instruction.  Every thread of
-// the group (nthreads, named barrier bar_id) runs the barrier, also when `ok`
-// is false after a timeout.
 template <int D>
-__device__ void store_tile(uint32_t tacc, int row, bool ok, bool zero, bool part, float mul, uint8_t* stage,
-                           const CUtensorMap* map_bf16, const CUtensorMap* map_f32, int y_bf16, int y_f32,
-                           int bar_id, int nthreads, bool leader) {
-    if (ok) {
-        const uint32_t sw = (uint32_t)(row & 7);
-#pragma unroll 1
-        for (int q = 0; q < D / 32; ++q) {
-            uint32_t r[32];
-            tmem_ld32(tacc + 32 * q, r);
-            tmem_wait_ld();
-            if (zero) {
-#pragma unroll
-                for (int i = 0; i < 32; ++i) r[i] = 0u;
-            }
-            if (!part) {
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {                          // 4 chunks of 8 bf16
-                    const int g = 4 * q + k;
-                    uint4 v;
-                    v.x = pack_bf16x2(__uint_as_float(r[8 * k + 0]) * mul, __uint_as_float(r[8 * k + 1]) * mul);
-                    v.y = pack_bf16x2(__uint_as_float(r[8 * k + 2]) * mul, __uint_as_float(r[8 * k + 3]) * mul);
-                    v.z = pack_bf16x2(__uint_as_float(r[8 * k + 4]) * mul, __uint_as_float(r[8 * k + 5]) * mul);
-                    v.w = pack_bf16x2(__uint_as_float(r[8 * k + 6]) * mul, __uint_as_float(r[8 * k + 7]) * mul);
-                    *reinterpret_cast<uint4*>(stage + (g >> 3) * kTile + row * 128 + (((g & 7) ^ sw) << 4)) = v;
-                }
-            } else {
-#pragma unroll
-                for (int k = 0; k < 8; ++k) {                          // 8 chunks of 4 fp32
-                    const int g = 8 * q + k;
-                    const float4 v = make_float4(__uint_as_float(r[4 * k]), __uint_as_float(r[4 * k + 1]),
-                                                 __uint_as_float(r[4 * k + 2]), __uint_as_float(r[4 * k + 3]));
-                    *reinterpret_cast<float4*>(stage + (g >> 3) * kTile + row * 128 + (((g & 7) ^ sw) << 4)) = v;
-                }
-            }
-        }
-        fence_proxy_async_smem();
+struct DqpLayout {
+    static constexpr int NR = D / 64;
+    static constexpr int STAGE = 2 * NR * kGran;       // K and V of one granule
+    __host__ __device__ static int staging(int nst) { return nst * STAGE; }
+    __host__ __device__ static int ctrl(int nst) { return staging(nst) + kStagingP; }
+    __host__ __device__ static int rows(int nst) { return ctrl(nst) + kCtrl; }
+    static int alloc(int nst, int SW) { return rows(nst) + 16 * SW + 1024; }   // 2 slots x 2 rows
+    static int stages(int SW) {
+        int n = kStages;
+        while (n > 2 && alloc(n, SW) > kSmemMax) --n;
+        return n;
     }
-    named_sync(bar_id, nthreads);
-    if (ok && leader) {
-        tma_store_3d(part ? map_f32 : map_bf16, stage, 0, part ? y_f32 : y_bf16, 0);
-        bulk_commit();
-        bulk_wait_read();                                              // shared memory stays valid until read
+};
+
+struct BarsP {
+    uint64_t* full0;           // [kStages]
+    uint64_t* full1;           // [kStages]
+    uint64_t* empty;           // [kStages]
+    uint64_t* prod;            // [2]
+    uint64_t* elem;            // [2]
+    uint64_t* qdo_full;
+    uint64_t* fin;
+    uint64_t* drain;           // teardown after an abort: every issued MMA complete
+    uint64_t* rows_full;       // [2]
+    uint64_t* rows_empty;      // [2]
+    uint32_t* tmem_slot;
+    volatile int* abort_flag;
+};
+
+__device__ __forceinline__ BarsP carve_p(uint8_t* ctrl) {
+    uint64_t* b = reinterpret_cast<uint64_t*>(ctrl);
+    BarsP r;
+    r.full0 = b;
+    r.full1 = b + kStages;
+    r.empty = b + 2 * kStages;
+    r.prod = b + 3 * kStages;
+    r.elem = b + 3 * kStages + 2;
+    r.qdo_full = b + 3 * kStages + 4;
+    r.fin = b + 3 * kStages + 5;
+    r.drain = b + 3 * kStages + 6;
+    r.rows_full = b + 3 * kStages + 7;
+    r.rows_empty = b + 3 * kStages + 9;
+    r.tmem_slot = reinterpret_cast<uint32_t*>(b + 3 * kStages + 11);
+    r.abort_flag = reinterpret_cast<volatile int*>(r.tmem_slot + 1);
+    return r;
+}
+static_assert((3 * kStages + 11) * 8 + 8 <= kCtrl, "barriers overflow the control block");
+
+// Epilogue with a 32 KB staging area of its own (the ring is busy with the
+// next item): the bf16 tile (D/64 regions) in one store, the fp32 partial
+// (D/32 regions) in passes of two regions.  The barrier at the top of every
+// pass makes the staging free: the leader passes it only after its previous
+// store has finished reading shared memory.  Every thread of the group runs
+// the same barriers whatever `ok` is (passes depend on `part` only).
+template <int D>
+__device__ void store_tile_p(uint32_t tacc, int row, bool ok, bool zero, bool part, float mul, uint8_t* stage,
+                             const CUtensorMap* map_bf16, const CUtensorMap* map_f32h, int y_bf16, int y_f32,
+                             int bar_id, int nthreads, bool leader) {
+    const int regions = part ? D / 32 : D / 64;            // 128-byte regions of a row
+    const int per_pass = regions < 2 ? regions : 2;
+    const int passes = regions / per_pass;
+    const uint32_t sw = (uint32_t)(row & 7);
+#pragma unroll 1
+    for (int p = 0; p < passes; ++p) {
+        named_sync(bar_id, nthreads);
+        if (ok) {
+            // 32 fp32 TMEM columns per load: a quarter of a bf16 region pair, one fp32 region
+            const int q0 = part ? p * per_pass : 0, q1 = part ? q0 + per_pass : D / 32;
+#pragma unroll 1
+            for (int q = q0; q < q1; ++q) {
+                uint32_t r[32];
+                if (zero) {                                           // an empty item: TMEM is not read
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) r[i] = 0u;
+                } else {
+                    tmem_ld32(tacc + 32 * q, r);
+                    tmem_wait_ld();
+                }
+                if (!part) {
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const int g = 4 * q + k;                      // 16-byte chunk of the bf16 row
+                        uint4 v;
+                        v.x = pack_bf16x2(__uint_as_float(r[8 * k + 0]) * mul, __uint_as_float(r[8 * k + 1]) * mul);
+                        v.y = pack_bf16x2(__uint_as_float(r[8 * k + 2]) * mul, __uint_as_float(r[8 * k + 3]) * mul);
+                        v.z = pack_bf16x2(__uint_as_float(r[8 * k + 4]) * mul, __uint_as_float(r[8 * k + 5]) * mul);
+                        v.w = pack_bf16x2(__uint_as_float(r[8 * k + 6]) * mul, __uint_as_float(r[8 * k + 7]) * mul);
+                        *reinterpret_cast<uint4*>(stage + (g >> 3) * kTile + row * 128 + (((g & 7) ^ sw) << 4)) = v;
+                    }
+                } else {
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        const int g = 8 * (q - q0) + k;               // 16-byte chunk within this pass
+                        const float4 v = make_float4(__uint_as_float(r[4 * k]), __uint_as_float(r[4 * k + 1]),
+                                                     __uint_as_float(r[4 * k + 2]), __uint_as_float(r[4 * k + 3]));
+                        *reinterpret_cast<float4*>(stage + (g >> 3) * kTile + row * 128 + (((g & 7) ^ sw) << 4)) = v;
+                    }
+                }
+            }
+            fence_proxy_async_smem();
+        }
+        named_sync(bar_id, nthreads);
+        if (ok && leader) {
+            if (part) tma_store_3d(map_f32h, stage, 0, y_f32, p * per_pass);
+            else tma_store_3d(map_bf16, stage, 0, y_bf16, 0);
+            bulk_commit();
+            bulk_wait_read();
+        }
     }
 }
 
-// ============================================================================ dQ
+// Q and dO rows of one tile into TMEM as bf16 (two per 32-bit column)
+template <int D>
+__device__ __forceinline__ void load_qdo(uint32_t tl, uint32_t cQ, uint32_t cdO, const __nv_bfloat16* Qg,
+                                         const __nv_bfloat16* dOg, int64_t grow) {
+#pragma unroll
+    for (int which = 0; which < 2; ++which) {
+        const uint4* src = reinterpret_cast<const uint4*>((which ? dOg : Qg) + grow * D);
+#pragma unroll
+        for (int q = 0; q < D / 64; ++q) {
+            uint32_t r[32];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const uint4 v = __ldg(src + 8 * q + i);
+                r[4 * i] = v.x;
+                r[4 * i + 1] = v.y;
+                r[4 * i + 2] = v.z;
+                r[4 * i + 3] = v.w;
+            }
+            tmem_st32(tl + (which ? cdO : cQ) + 32 * q, r);
+        }
+    }
+    tmem_wait_st();
+}
+
 template <int D>
 __global__ void __launch_bounds__(192, 1)
-k_bwd_dq_sm100(const __nv_bfloat16* __restrict__ Qg, const __nv_bfloat16* __restrict__ dOg,
-               const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-               const __grid_constant__ CUtensorMap tmdQ, const __grid_constant__ CUtensorMap tmPq,
-               const uint32_t* __restrict__ gsel, const PlanHeader* __restrict__ hdr,
-               const int4* __restrict__ items, const float* __restrict__ lse,
-               const float* __restrict__ delta, int64_t N, int64_t MB, int SW, int nst, float scale,
-               uint32_t* __restrict__ dev_status) {
-    using L = BwdLayout<D, false>;
-    // TMEM: dQ, S / dP of two granules, and the tile's Q and dO as bf16 (the A
-    // operands of S = Q K^T and dP = dO V^T, read by the tensor core from TMEM)
+k_bwd_dq_persist(const __nv_bfloat16* __restrict__ Qg, const __nv_bfloat16* __restrict__ dOg,
+                 const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                 const __grid_constant__ CUtensorMap tmdQ, const __grid_constant__ CUtensorMap tmPqh,
+                 const uint32_t* __restrict__ gsel, const PlanHeader* __restrict__ hdr,
+                 const int4* __restrict__ items, const float* __restrict__ lse,
+                 const float* __restrict__ delta, int64_t N, int64_t MB, int SW, int nst, float scale,
+                 uint32_t* __restrict__ dev_status) {
+    using L = DqpLayout<D>;
     constexpr uint32_t cdQ = 0, cS = 128, cP = 192;   // + 128 * buffer for S / dP
     constexpr uint32_t cQ = 384, cdO = 384 + D / 2;
-    if ((int)blockIdx.x >= hdr->n_items) return;      // uniform: beyond the item list
-    const int4 item = items[blockIdx.x];
+    const int n_items = hdr->n_items;
+    if ((int)blockIdx.x >= n_items) return;           // uniform: more CTAs than items
     const int tiles_per_head = (int)(N / 128);
-    const int hh = item.x / tiles_per_head, tile = item.x % tiles_per_head;
-    const int g_begin = item.y, ng = item.z - item.y, slot = item.w;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    Bars B = carve(sm + L::ctrl(nst, 0));
-    uint32_t* u0 = reinterpret_cast<uint32_t*>(sm + L::rows(nst, 0));
-    uint32_t* u1 = u0 + SW;
+    BarsP B = carve_p(sm + L::ctrl(nst));
+    uint32_t* rows_base = reinterpret_cast<uint32_t*>(sm + L::rows(nst));   // [2 slots][2 rows][SW]
+    uint8_t* staging = sm + L::staging(nst);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int wn = SW;
-    const int64_t row0 = (int64_t)hh * N;
 
-    load_rows(u0, u1, gsel + ((int64_t)hh * MB + 2 * tile) * SW, gsel + ((int64_t)hh * MB + 2 * tile + 1) * SW, wn);
-    if (threadIdx.x == 0) init_bars(B, nst, 128, 128);   // Q, dO: one arrival per tile row
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < nst; ++s) {
+            mbar_init(B.full0 + s, 1);
+            mbar_init(B.full1 + s, 1);
+            mbar_init(B.empty + s, 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(B.prod + b, 1);
+            mbar_init(B.elem + b, 128);
+            mbar_init(B.rows_full + b, 32);
+            mbar_init(B.rows_empty + b, 4);
+        }
+        mbar_init(B.qdo_full, 128);
+        mbar_init(B.fin, 1);
+        mbar_init(B.drain, 1);
+        *B.abort_flag = 0;
+        fence_mbar_init();
+    }
     if (warp == 1) {
         tmem_alloc(B.tmem_slot, kTmemCols);
         tmem_relinquish();
@@ -273,21 +266,94 @@ k_bwd_dq_sm100(const __nv_bfloat16* __restrict__ Qg, const __nv_bfloat16* __rest
     const uint32_t tb = *B.tmem_slot;
 
     if (warp == 0) {
-        produce<D, false>(nullptr, nullptr, &tmK, &tmV, nullptr, nullptr, sm, B, row0, 128 * tile, u0, u1, wn,
-                          g_begin, ng, nst, dev_status);
+        // ---------------------------------------------------------------- producer
+        // lane kind * nst + stage (kind 0: K, 1: V) issues its stream's copies for
+        // the granules of that stage; all 32 lanes copy the selection rows
+        const int kind = lane / nst, stage = lane % nst;
+        const bool copier = lane < 2 * nst;
+        uint64_t* full = kind == 0 ? B.full0 : B.full1;
+        const CUtensorMap* mg = kind == 0 ? &tmK : &tmV;
+        if (copier) tma_prefetch_desc(mg);
+        bool ok = true;
+        int last_cyc = -1;                                 // ring cycle of this lane's last copy
+        int st0 = 0, cyc0 = 0;                             // stage and ring cycle of the item's first granule
+        for (int it = blockIdx.x, j = 0; it < n_items; it += gridDim.x, ++j) {
+            const int4 item = items[it];
+            const int hh = item.x / tiles_per_head, tile = item.x % tiles_per_head;
+            const int g_begin = item.y, ng = item.z - item.y;
+            const int64_t row0 = (int64_t)hh * N;
+            uint32_t* u0 = rows_base + (j & 1) * 2 * SW;
+            uint32_t* u1 = u0 + SW;
+            if (ok && j >= 2) ok = mbar_wait(B.rows_empty + (j & 1), ((j >> 1) - 1) & 1, B.abort_flag, dev_status);
+            if (ok) {
+                const uint32_t* s0 = gsel + ((int64_t)hh * MB + 2 * tile) * SW;
+                for (int w = lane; w < wn; w += 32) {
+                    u0[w] = s0[w];
+                    u1[w] = s0[SW + w];
+                }
+            }
+            mbar_arrive(B.rows_full + (j & 1));
+            __syncwarp();                                  // every lane's rows visible to the walkers
+            int s_ = st0, c_ = cyc0;
+            if (copier && ok) {
+                GranuleWalk walk;
+                walk.init(u0, u1, wn);
+                walk.skip(g_begin);
+                for (int g = 0; g < ng; ++g) {
+                    int row;
+                    uint32_t m;
+                    walk.next(row, m);
+                    if (s_ == stage) {
+                        if (c_ >= 1 && !mbar_wait(B.empty + stage, (uint32_t)(c_ - 1) & 1, B.abort_flag, dev_status)) {
+                            ok = false;
+                            break;
+                        }
+                        mbar_expect_tx(full + stage, L::NR * kGran);
+                        tma_load_3d(sm + stage * L::STAGE + kind * L::NR * kGran, mg, full + stage, 0,
+                                    (int)(row0 + row), 0);
+                        last_cyc = c_;
+                    }
+                    if (++s_ == nst) { s_ = 0; ++c_; }
+                }
+            }
+            __syncwarp();                                  // no lane walks rows a later item overwrites
+            if (*B.abort_flag) ok = false;
+            // every lane advances the ring position by the item's granules
+            const int tot = st0 + ng;
+            cyc0 += tot / nst;
+            st0 = tot % nst;
+        }
+        if (!ok && copier && last_cyc >= 0) {
+            volatile int no_abort = 0;                     // let this lane's last copy land
+            mbar_wait(full + stage, (uint32_t)last_cyc & 1, &no_abort, dev_status);
+        }
     } else if (warp == 1) {
-        {   // the whole warp, converged; one elected lane issues
-            const uint32_t idPS = idesc_bf16_f32(128, 64, false, false);
-            const uint32_t idQ = idesc_bf16_f32(128, D, false, true);
-            const uint32_t aR = smem_u32(sm + L::RING);
-            bool ok = mbar_wait_w(B.stat, 0, B.abort_flag, dev_status);
+        // ---------------------------------------------------------------- MMA (whole warp, elected issue)
+        const uint32_t idPS = idesc_bf16_f32(128, 64, false, false);
+        const uint32_t idQ = idesc_bf16_f32(128, D, false, true);
+        const uint32_t aR = smem_u32(sm);
+        bool ok = true;
+        int G = 0;                                         // granules of this CTA so far
+        int s_ = 0, c_ = 0;                                // stage and ring cycle of granule G
+        int kq = 0;                                        // non-empty items so far
+        for (int it = blockIdx.x; ok && it < n_items; it += gridDim.x) {
+            const int4 item = items[it];
+            const int ng = item.z - item.y;
+            if (ng == 0) continue;
+            ok = mbar_wait_w(B.qdo_full, kq & 1, B.abort_flag, dev_status);
+            if (!ok) break;
             tc_fence_after();
+            int prev_s = 0;
             for (int g = 0; ok && g <= ng; ++g) {
                 if (g < ng) {
-                    const int s = g % nst, b = g & 1;
-                    if (!mbar_wait_w(B.full0 + s, (g / nst) & 1, B.abort_flag, dev_status) ||
-                        !mbar_wait_w(B.full1 + s, (g / nst) & 1, B.abort_flag, dev_status))
+                    const int GG = G + g;
+                    const int s = s_, b = GG & 1;
+                    const uint32_t ph = (uint32_t)c_ & 1;
+                    if (!mbar_wait_w(B.full0 + s, ph, B.abort_flag, dev_status) ||
+                        !mbar_wait_w(B.full1 + s, ph, B.abort_flag, dev_status)) {
+                        ok = false;
                         break;
+                    }
                     tc_fence_after();
                     const uint32_t aK = aR + s * L::STAGE, aV = aK + L::NR * kGran;
 #pragma unroll
@@ -301,8 +367,13 @@ k_bwd_dq_sm100(const __nv_bfloat16* __restrict__ Qg, const __nv_bfloat16* __rest
                     tc_commit_w(B.prod + b);
                 }
                 if (g > 0) {
-                    const int gp = g - 1, s = gp % nst, b = gp & 1;
-                    if (!mbar_wait_w(B.elem + b, (gp >> 1) & 1, B.abort_flag, dev_status)) break;
+                    const int gp = g - 1;
+                    const int GGp = G + gp;
+                    const int s = prev_s, b = GGp & 1;
+                    if (!mbar_wait_w(B.elem + b, (uint32_t)(GGp >> 1) & 1, B.abort_flag, dev_status)) {
+                        ok = false;
+                        break;
+                    }
                     tc_fence_after();
                     const uint32_t aK = aR + s * L::STAGE;
 #pragma unroll
@@ -311,102 +382,129 @@ k_bwd_dq_sm100(const __nv_bfloat16* __restrict__ Qg, const __nv_bfloat16* __rest
                                  (gp > 0 || k > 0) ? 1u : 0u);
                     tc_commit_w(B.empty + s);
                 }
+                if (g < ng) {
+                    prev_s = s_;
+                    if (++s_ == nst) { s_ = 0; ++c_; }
+                }
             }
+            if (!ok) break;
             tc_commit_w(B.fin);
-            if (*B.abort_flag) {
-                volatile int no_abort = 0;
-                mbar_wait(B.fin, 0, &no_abort, dev_status);
-            }
+            G += ng;
+            ++kq;
+        }
+        if (!ok) {
+            tc_commit_w(B.drain);                          // every MMA issued so far complete
+            volatile int no_abort = 0;
+            mbar_wait(B.drain, 0, &no_abort, dev_status);
         }
     } else {
+        // ---------------------------------------------------------------- elementwise + epilogue
         const int sub = warp & 3, row = sub * 32 + lane, half = row >> 6;
         const uint32_t tl = tb + ((uint32_t)(sub * 32) << 16);
-        const int64_t grow = row0 + 128 * tile + row;
-        {
-            // this row of Q and of dO into TMEM (two bf16 per column)
-#pragma unroll
-            for (int which = 0; which < 2; ++which) {
-                const uint4* src = reinterpret_cast<const uint4*>((which ? dOg : Qg) + grow * D);
-#pragma unroll
-                for (int q = 0; q < D / 64; ++q) {
-                    uint32_t r[32];
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        const uint4 v = __ldg(src + 8 * q + i);
-                        r[4 * i] = v.x;
-                        r[4 * i + 1] = v.y;
-                        r[4 * i + 2] = v.z;
-                        r[4 * i + 3] = v.w;
-                    }
-                    tmem_st32(tl + (which ? cdO : cQ) + 32 * q, r);
-                }
-            }
-            tmem_wait_st();
-            tc_fence_before();
-            mbar_arrive(B.stat);
-        }
-        const float lse2 = lse[grow] * kLog2e, dl = delta[grow];
         const float sl2 = scale * kLog2e;
-        const uint64_t sl2x2 = f2pack(sl2, sl2), nlse2 = f2pack(-lse2, -lse2), ndl2 = f2pack(-dl, -dl);
-        GranuleWalk walk;
-        if (lane == 0) {
-            walk.init(u0, u1, wn);
-            walk.skip(g_begin);
-        }
+        const uint64_t sl2x2 = f2pack(sl2, sl2);
         bool ok = true;
-        for (int g = 0; g < ng; ++g) {
-            const int b = g & 1;
-            uint32_t mk = 0;
+        int G = 0;
+        int kf = 0;                                        // non-empty items so far
+        // Q and dO of a non-empty item go into TMEM once the previous non-empty
+        // item's S/dP products are consumed; the first one before the loop
+        auto qdo_ahead = [&](int itn) {
+            if (itn >= n_items) return;
+            const int4 nx = items[itn];
+            if (nx.z == nx.y) return;                      // empty: never reaches the MMA warp
+            if (ok) {
+                const int64_t ngrow = (int64_t)(nx.x / tiles_per_head) * N + 128 * (nx.x % tiles_per_head) + row;
+                load_qdo<D>(tl, cQ, cdO, Qg, dOg, ngrow);
+                tc_fence_before();
+            }
+            mbar_arrive(B.qdo_full);
+        };
+        qdo_ahead(blockIdx.x);
+        for (int it = blockIdx.x, j = 0; it < n_items; it += gridDim.x, ++j) {
+            const int4 item = items[it];
+            const int hh = item.x / tiles_per_head, tile = item.x % tiles_per_head;
+            const int g_begin = item.y, ng = item.z - item.y, slot = item.w;
+            const int64_t row0 = (int64_t)hh * N;
+            const int64_t grow = row0 + 128 * tile + row;
+            const float lse2 = lse[grow] * kLog2e, dl = delta[grow];
+            const uint64_t nlse2 = f2pack(-lse2, -lse2), ndl2 = f2pack(-dl, -dl);
+            const uint32_t* u0 = rows_base + (j & 1) * 2 * SW;
+            GranuleWalk walk;
             if (lane == 0) {
-                int rr;
-                walk.next(rr, mk);
-            }
-            mk = __shfl_sync(0xffffffffu, mk, 0);
-            const bool valid = (mk >> half) & 1u;              // warp-uniform
-            const bool got = mbar_wait(B.prod + b, (g >> 1) & 1, B.abort_flag, dev_status);
-            if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
-            tc_fence_after();
-            // S and dP of the granule: all TMEM loads in flight before one wait
-            uint32_t sv[2][32], pv[2][32];
-            if (valid) {
-                tmem_ld32(tl + cS + 128 * b, sv[0]);
-                tmem_ld32(tl + cP + 128 * b, pv[0]);
-                tmem_ld32(tl + cS + 128 * b + 32, sv[1]);
-                tmem_ld32(tl + cP + 128 * b + 32, pv[1]);
-                tmem_wait_ld();
-            }
-#pragma unroll
-            for (int hq = 0; hq < 2; ++hq) {
-                uint32_t o[16];
-                if (valid) {
-                    const uint32_t (&s)[32] = sv[hq];
-                    const uint32_t (&p)[32] = pv[hq];
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        float x0, x1;
-                        f2unpack(ffma2(f2pack(__uint_as_float(s[2 * i]), __uint_as_float(s[2 * i + 1])), sl2x2, nlse2),
-                                 x0, x1);
-                        const uint64_t pp = f2pack(ex2(x0), ex2(x1));
-                        const uint64_t dp = fadd2(f2pack(__uint_as_float(p[2 * i]), __uint_as_float(p[2 * i + 1])), ndl2);
-                        float d0, d1;
-                        f2unpack(fmul2(pp, dp), d0, d1);
-                        o[i] = pack_bf16x2(d0, d1);
-                    }
+                const bool got = ok && mbar_wait(B.rows_full + (j & 1), (j >> 1) & 1, B.abort_flag, dev_status);
+                if (got) {
+                    walk.init(u0, u0 + SW, wn);
+                    walk.skip(g_begin);
                 } else {
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) o[i] = 0u;
+                    walk.init(u0, u0 + SW, 0);             // empty walk; ok drops below
                 }
-                tmem_st16(tl + cS + 128 * b + 16 * hq, o);     // dS (bf16) over the consumed S columns
+                ok = got;
             }
-            tmem_wait_st();
-            tc_fence_before();
-            mbar_arrive(B.elem + b);
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            for (int g = 0; ok && g < ng; ++g) {
+                const int GG = G + g;
+                const int b = GG & 1;
+                uint32_t mk = 0;
+                if (lane == 0) {
+                    int rr;
+                    walk.next(rr, mk);
+                }
+                mk = __shfl_sync(0xffffffffu, mk, 0);
+                const bool valid = (mk >> half) & 1u;          // warp-uniform
+                const bool got = mbar_wait(B.prod + b, (uint32_t)(GG >> 1) & 1, B.abort_flag, dev_status);
+                if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+                tc_fence_after();
+                // one 32-column half of S and dP at a time (both loads in flight before one wait)
+#pragma unroll
+                for (int hq = 0; hq < 2; ++hq) {
+                    uint32_t sv[32], pv[32];
+                    if (valid) {
+                        tmem_ld32(tl + cS + 128 * b + 32 * hq, sv);
+                        tmem_ld32(tl + cP + 128 * b + 32 * hq, pv);
+                        tmem_wait_ld();
+                    }
+                    uint32_t o[16];
+                    if (valid) {
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            float x0, x1;
+                            f2unpack(ffma2(f2pack(__uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1])), sl2x2,
+                                           nlse2),
+                                     x0, x1);
+                            const uint64_t pp = f2pack(ex2(x0), ex2(x1));
+                            const uint64_t dp =
+                                fadd2(f2pack(__uint_as_float(pv[2 * i]), __uint_as_float(pv[2 * i + 1])), ndl2);
+                            float d0, d1;
+                            f2unpack(fmul2(pp, dp), d0, d1);
+                            o[i] = pack_bf16x2(d0, d1);
+                        }
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) o[i] = 0u;
+                    }
+                    // dS (bf16) over S columns this half has consumed: half hq writes 16 hq .. 16 hq + 15,
+                    // inside the 32 columns the first half already read
+                    tmem_st16(tl + cS + 128 * b + 16 * hq, o);
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(B.elem + b);
+            }
+            if (lane == 0) mbar_arrive(B.rows_empty + (j & 1));
+            // the next non-empty item's Q and dO: this item's S/dP products are all consumed
+            qdo_ahead(it + (int)gridDim.x);
+            bool fin = ok;
+            if (ng > 0) {
+                fin = __all_sync(0xffffffffu, ok && mbar_wait(B.fin, kf & 1, B.abort_flag, dev_status));
+                if (fin) tc_fence_after();
+                ++kf;
+            }
+            ok = fin;
+            // the item's dQ (or zeros when nothing was selected: ng == 0)
+            store_tile_p<D>(tl + cdQ, row, fin, ng == 0, slot >= 0, scale, staging, &tmdQ, &tmPqh,
+                            (int)(row0 + 128 * tile), slot * 128, 1, 128, warp == 2 && lane == 0);
+            G += ng;
         }
-        const bool fin = __all_sync(0xffffffffu, ok && mbar_wait(B.fin, 0, B.abort_flag, dev_status));
-        if (fin) tc_fence_after();
-        // nothing selected (ng == 0): TMEM never written, the tile is zero.  The ring is free.
-        store_tile<D>(tl + cdQ, row, fin, ng == 0, slot >= 0, scale, sm + L::RING, &tmdQ, &tmPq,
-                      (int)(row0 + 128 * tile), slot * 128, 1, 128, warp == 2 && lane == 0);
     }
     tc_fence_before();
     __syncthreads();
@@ -414,35 +512,115 @@ k_bwd_dq_sm100(const __nv_bfloat16* __restrict__ Qg, const __nv_bfloat16* __rest
     if (warp == 1) tmem_dealloc(tb, kTmemCols);
 }
 
-// ============================================================================ dK, dV
+// ============================================================================ dK, dV (persistent)
+// One CTA per SM takes items blockIdx.x, blockIdx.x + gridDim.x, ...; granules
+// are numbered over all of the CTA's items, so the ring and the double-buffered
+// S^T/dP^T columns carry across item edges.  The next non-empty item's K and V
+// tiles are loaded as soon as the current item's last S^T/dP^T MMAs complete
+// (kv_free), which hides the load behind the current item's tail and epilogue.
+// Items with no granule (no query selected these keys) never reach the MMA
+// warp; their dK and dV are zero, written without TMEM.  The epilogue shares one
+// 16 KB staging region: one 128-row region of dK or dV per pass.
+template <int D>
+struct DkvpLayout {
+    static constexpr int NR = D / 64;
+    static constexpr int A0 = 0;                       // K tile
+    static constexpr int A1 = NR * kTile;              // V tile
+    static constexpr int STG = 2 * NR * kTile;         // one region of 128 rows x 128 bytes
+    static constexpr int RING = STG + kTile;
+    static constexpr int STAGE = 2 * NR * kGran;       // Q and dO of one granule
+    __host__ __device__ static int xs(int nst) { return RING + nst * STAGE; }
+    __host__ __device__ static int ctrl(int nst) { return xs(nst) + nst * kXs; }
+    __host__ __device__ static int rows(int nst) { return ctrl(nst) + kCtrl; }
+    static int alloc(int nst, int SW) { return rows(nst) + 16 * SW + 1024; }   // 2 slots x 2 rows
+    static int stages(int SW) {
+        int n = kStages;
+        while (n > 2 && alloc(n, SW) > kSmemMax) --n;
+        return n;
+    }
+};
+
+struct BarsKV {
+    uint64_t* full0;           // [kStages] Q granule landed
+    uint64_t* full1;           // [kStages] dO granule landed
+    uint64_t* fullx;           // [kStages] row data landed
+    uint64_t* empty;           // [kStages]
+    uint64_t* prod;            // [2]
+    uint64_t* elem;            // [2] (256 arrivals)
+    uint64_t* stat;            // K, V tiles of a non-empty item landed (2 copies)
+    uint64_t* kv_free;         // the item's last S^T/dP^T MMAs complete
+    uint64_t* fin;
+    uint64_t* drain;
+    uint64_t* rows_full;       // [2] (32 arrivals)
+    uint64_t* rows_empty;      // [2] (8 arrivals: one per elementwise warp)
+    uint32_t* tmem_slot;
+    volatile int* abort_flag;
+};
+
+__device__ __forceinline__ BarsKV carve_kv(uint8_t* ctrl) {
+    uint64_t* b = reinterpret_cast<uint64_t*>(ctrl);
+    BarsKV r;
+    r.full0 = b;
+    r.full1 = b + kStages;
+    r.fullx = b + 2 * kStages;
+    r.empty = b + 3 * kStages;
+    r.prod = b + 4 * kStages;
+    r.elem = b + 4 * kStages + 2;
+    r.stat = b + 4 * kStages + 4;
+    r.kv_free = b + 4 * kStages + 5;
+    r.fin = b + 4 * kStages + 6;
+    r.drain = b + 4 * kStages + 7;
+    r.rows_full = b + 4 * kStages + 8;
+    r.rows_empty = b + 4 * kStages + 10;
+    r.tmem_slot = reinterpret_cast<uint32_t*>(b + 4 * kStages + 12);
+    r.abort_flag = reinterpret_cast<volatile int*>(r.tmem_slot + 1);
+    return r;
+}
+static_assert((4 * kStages + 12) * 8 + 8 <= kCtrl, "barriers overflow the control block");
+
 template <int D>
 __global__ void __launch_bounds__(384, 1)
-k_bwd_dkdv_sm100(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-                 const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmdO,
-                 const __grid_constant__ CUtensorMap tmdK, const __grid_constant__ CUtensorMap tmdV,
-                 const __grid_constant__ CUtensorMap tmPkv,
-                 const uint32_t* __restrict__ gselT, const PlanHeader* __restrict__ hdr,
-                 const int4* __restrict__ items, const float* __restrict__ nld,
-                 int64_t N, int64_t MB, int SW, int nst, float scale, uint32_t* __restrict__ dev_status) {
-    using L = BwdLayout<D, true>;
+k_bwd_dkdv_persist(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                   const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmdO,
+                   const __grid_constant__ CUtensorMap tmdK1, const __grid_constant__ CUtensorMap tmdV1,
+                   const __grid_constant__ CUtensorMap tmPkv1,
+                   const uint32_t* __restrict__ gselT, const PlanHeader* __restrict__ hdr,
+                   const int4* __restrict__ items, const float* __restrict__ nld,
+                   int64_t N, int64_t MB, int SW, int nst, float scale, uint32_t* __restrict__ dev_status) {
+    using L = DkvpLayout<D>;
     constexpr uint32_t cdK = 0, cdV = 128, cS = 256, cP = 320;   // + 128 * buffer for S^T / dP^T
-    if ((int)blockIdx.x >= hdr->n_items) return;      // uniform: beyond the item list
-    const int4 item = items[blockIdx.x];
+    const int n_items = hdr->n_items;
+    if ((int)blockIdx.x >= n_items) return;
     const int tiles_per_head = (int)(N / 128);
-    const int hh = item.x / tiles_per_head, tile = item.x % tiles_per_head;
-    const int g_begin = item.y, ng = item.z - item.y, slot = item.w;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    Bars B = carve(sm + L::ctrl(nst, kXs));
+    BarsKV B = carve_kv(sm + L::ctrl(nst));
     uint8_t* xs = sm + L::xs(nst);
-    uint32_t* u0 = reinterpret_cast<uint32_t*>(sm + L::rows(nst, kXs));
-    uint32_t* u1 = u0 + SW;
+    uint32_t* rows_base = reinterpret_cast<uint32_t*>(sm + L::rows(nst));
+    uint8_t* staging = sm + L::STG;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int wn = SW;
-    const int64_t row0 = (int64_t)hh * N;
 
-    load_rows(u0, u1, gselT + ((int64_t)hh * MB + 2 * tile) * SW, gselT + ((int64_t)hh * MB + 2 * tile + 1) * SW, wn);
-    if (threadIdx.x == 0) init_bars(B, nst, 2, 256);     // K, V: one arrival per stationary copy
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < nst; ++s) {
+            mbar_init(B.full0 + s, 1);
+            mbar_init(B.full1 + s, 1);
+            mbar_init(B.fullx + s, 1);
+            mbar_init(B.empty + s, 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(B.prod + b, 1);
+            mbar_init(B.elem + b, 256);
+            mbar_init(B.rows_full + b, 32);
+            mbar_init(B.rows_empty + b, 8);
+        }
+        mbar_init(B.stat, 2);
+        mbar_init(B.kv_free, 1);
+        mbar_init(B.fin, 1);
+        mbar_init(B.drain, 1);
+        *B.abort_flag = 0;
+        fence_mbar_init();
+    }
     if (warp == 1) {
         tmem_alloc(B.tmem_slot, kTmemCols);
         tmem_relinquish();
@@ -455,21 +633,117 @@ k_bwd_dkdv_sm100(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
     if (warp < 4) {
       regs_dec<kRegsLow>();
       if (warp == 0) {
-        produce<D, true>(&tmK, &tmV, &tmQ, &tmdO, nld, xs, sm, B, row0, 128 * tile, u0, u1, wn, g_begin, ng, nst,
-                         dev_status);
+        // ---------------------------------------------------------------- producer
+        // lanes kind * nst + stage (kind 0: Q, 1: dO, 2: the granule's row data)
+        // stream the ring; lanes 30 (K) and 31 (V) load the stationary tiles of
+        // each non-empty item once the previous one's S^T/dP^T MMAs are done
+        const int kind = lane / nst, stage = lane % nst;
+        const bool copier = lane < 3 * nst;
+        const bool stat_lane = lane >= 30;
+        uint64_t* full = kind == 0 ? B.full0 : kind == 1 ? B.full1 : B.fullx;
+        const CUtensorMap* mg = kind == 0 ? &tmQ : &tmdO;
+        if (copier && kind < 2) tma_prefetch_desc(mg);
+        bool ok = true;
+        int last_cyc = -1;
+        int last_stat = -1;                                // index of the last stationary copy issued
+        int st0 = 0, cyc0 = 0;
+        int kq = 0;                                        // non-empty items so far
+        for (int it = blockIdx.x, j = 0; it < n_items; it += gridDim.x, ++j) {
+            const int4 item = items[it];
+            const int hh = item.x / tiles_per_head, tile = item.x % tiles_per_head;
+            const int g_begin = item.y, ng = item.z - item.y;
+            const int64_t row0 = (int64_t)hh * N;
+            uint32_t* u0 = rows_base + (j & 1) * 2 * SW;
+            uint32_t* u1 = u0 + SW;
+            if (ok && j >= 2) ok = mbar_wait(B.rows_empty + (j & 1), ((j >> 1) - 1) & 1, B.abort_flag, dev_status);
+            if (ok) {
+                const uint32_t* s0 = gselT + ((int64_t)hh * MB + 2 * tile) * SW;
+                for (int w = lane; w < wn; w += 32) {
+                    u0[w] = s0[w];
+                    u1[w] = s0[SW + w];
+                }
+            }
+            mbar_arrive(B.rows_full + (j & 1));
+            __syncwarp();
+            if (ng > 0) {
+                if (stat_lane && ok) {
+                    if (kq >= 1) ok = mbar_wait(B.kv_free, (uint32_t)(kq - 1) & 1, B.abort_flag, dev_status);
+                    if (ok) {
+                        mbar_expect_tx(B.stat, L::NR * kTile);
+                        tma_load_3d(sm + (lane == 30 ? L::A0 : L::A1), lane == 30 ? &tmK : &tmV, B.stat, 0,
+                                    (int)(row0 + 128 * tile), 0);
+                        last_stat = kq;
+                    }
+                }
+                ++kq;
+            }
+            int s_ = st0, c_ = cyc0;
+            if (copier && ok) {
+                GranuleWalk walk;
+                walk.init(u0, u1, wn);
+                walk.skip(g_begin);
+                for (int g = 0; g < ng; ++g) {
+                    int row;
+                    uint32_t m;
+                    walk.next(row, m);
+                    if (s_ == stage) {
+                        if (c_ >= 1 && !mbar_wait(B.empty + stage, (uint32_t)(c_ - 1) & 1, B.abort_flag, dev_status)) {
+                            ok = false;
+                            break;
+                        }
+                        if (kind == 2) {
+                            mbar_expect_tx(full + stage, kXs);
+                            bulk_load(xs + stage * kXs, nld + ((row0 + row) >> 6) * 128, kXs, full + stage);
+                        } else {
+                            mbar_expect_tx(full + stage, L::NR * kGran);
+                            tma_load_3d(sm + L::RING + stage * L::STAGE + kind * L::NR * kGran, mg, full + stage, 0,
+                                        (int)(row0 + row), 0);
+                        }
+                        last_cyc = c_;
+                    }
+                    if (++s_ == nst) { s_ = 0; ++c_; }
+                }
+            }
+            __syncwarp();
+            if (*B.abort_flag) ok = false;
+            const int tot = st0 + ng;
+            cyc0 += tot / nst;
+            st0 = tot % nst;
+        }
+        if (!ok && copier && last_cyc >= 0) {
+            volatile int no_abort = 0;
+            mbar_wait(full + stage, (uint32_t)last_cyc & 1, &no_abort, dev_status);
+        }
+        // a stationary copy in flight lands before the CTA goes away
+        if (!ok && stat_lane && last_stat >= 0) {
+            volatile int no_abort = 0;                     // bounded: the other lane's copy may be missing
+            mbar_wait(B.stat, (uint32_t)last_stat & 1, &no_abort, dev_status);
+        }
       } else if (warp == 1) {
-        {   // the whole warp, converged; one elected lane issues
-            const uint32_t idPS = idesc_bf16_f32(128, 64, false, false);
-            const uint32_t idKV = idesc_bf16_f32(128, D, false, true);
-            const uint32_t aK = smem_u32(sm + L::A0), aV = smem_u32(sm + L::A1), aR = smem_u32(sm + L::RING);
-            bool ok = mbar_wait_w(B.stat, 0, B.abort_flag, dev_status);
+        // ---------------------------------------------------------------- MMA (whole warp, elected issue)
+        const uint32_t idPS = idesc_bf16_f32(128, 64, false, false);
+        const uint32_t idKV = idesc_bf16_f32(128, D, false, true);
+        const uint32_t aK = smem_u32(sm + L::A0), aV = smem_u32(sm + L::A1), aR = smem_u32(sm + L::RING);
+        bool ok = true;
+        int G = 0, s_ = 0, c_ = 0, kq = 0;
+        for (int it = blockIdx.x; ok && it < n_items; it += gridDim.x) {
+            const int4 item = items[it];
+            const int ng = item.z - item.y;
+            if (ng == 0) continue;
+            ok = mbar_wait_w(B.stat, kq & 1, B.abort_flag, dev_status);
+            if (!ok) break;
             tc_fence_after();
+            int prev_s = 0;
             for (int g = 0; ok && g <= ng; ++g) {
                 if (g < ng) {
-                    const int s = g % nst, b = g & 1;
-                    if (!mbar_wait_w(B.full0 + s, (g / nst) & 1, B.abort_flag, dev_status) ||
-                        !mbar_wait_w(B.full1 + s, (g / nst) & 1, B.abort_flag, dev_status))
+                    const int GG = G + g;
+                    const int s = s_, b = GG & 1;
+                    const uint32_t ph = (uint32_t)c_ & 1;
+                    if (!mbar_wait_w(B.full0 + s, ph, B.abort_flag, dev_status) ||
+                        !mbar_wait_w(B.full1 + s, ph, B.abort_flag, dev_status)) {
+                        ok = false;
                         break;
+                    }
                     tc_fence_after();
                     const uint32_t aQ = aR + s * L::STAGE, adO = aQ + L::NR * kGran;
 #pragma unroll
@@ -481,10 +755,16 @@ k_bwd_dkdv_sm100(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
                         mma_ss_w(tb + cP + 128 * b, sdesc_sw128(aV + kmaj_off(k, kTile), 16, 1024),
                                  sdesc_sw128(adO + kmaj_off(k, kGran), 16, 1024), idPS, k > 0);
                     tc_commit_w(B.prod + b);
+                    if (g == ng - 1) tc_commit_w(B.kv_free);   // K and V no longer read by this item
                 }
                 if (g > 0) {
-                    const int gp = g - 1, s = gp % nst, b = gp & 1;
-                    if (!mbar_wait_w(B.elem + b, (gp >> 1) & 1, B.abort_flag, dev_status)) break;
+                    const int gp = g - 1;
+                    const int GGp = G + gp;
+                    const int s = prev_s, b = GGp & 1;
+                    if (!mbar_wait_w(B.elem + b, (uint32_t)(GGp >> 1) & 1, B.abort_flag, dev_status)) {
+                        ok = false;
+                        break;
+                    }
                     tc_fence_after();
                     const uint32_t aQ = aR + s * L::STAGE, adO = aQ + L::NR * kGran;
 #pragma unroll
@@ -497,96 +777,176 @@ k_bwd_dkdv_sm100(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
                     }
                     tc_commit_w(B.empty + s);
                 }
+                if (g < ng) {
+                    prev_s = s_;
+                    if (++s_ == nst) { s_ = 0; ++c_; }
+                }
             }
+            if (!ok) break;
             tc_commit_w(B.fin);
-            if (*B.abort_flag) {
-                volatile int no_abort = 0;
-                mbar_wait(B.fin, 0, &no_abort, dev_status);
-            }
+            G += ng;
+            ++kq;
+        }
+        if (!ok) {
+            tc_commit_w(B.drain);
+            volatile int no_abort = 0;
+            mbar_wait(B.drain, 0, &no_abort, dev_status);
         }
       }
     } else {
         regs_inc<kRegsHigh>();
-        // Both elementwise warpgroups work on every granule, warpgroup wg on
-        // its 32 query columns (16 wg .. 16 wg + 15 of P^T / dS^T), which halves
-        // the latency from the granule's products to its dK/dV MMAs.  bf16 P^T
-        // and dS^T of warpgroup 1 overwrite fp32 columns that warpgroup 0
-        // reads, so the stores wait at a named barrier for both warpgroups'
-        // loads; every thread runs every barrier, also after a timeout.
+        // both warpgroups on every granule, warpgroup wg on its 32 query columns
+        // (see the non-persistent kernel); every thread runs every named barrier
         const int wg = (warp - 4) >> 2;
         const int sub = warp & 3, row = sub * 32 + lane, half = row >> 6;
         const uint32_t tl = tb + ((uint32_t)(sub * 32) << 16);
         const float sl2 = scale * kLog2e;
         const uint64_t sl2x2 = f2pack(sl2, sl2);
-        GranuleWalk walk;
-        if (lane == 0) {
-            walk.init(u0, u1, wn);
-            walk.skip(g_begin);
-        }
         bool ok = true;
-        for (int g = 0; g < ng; ++g) {
-            const int b = g & 1, st = g % nst;
-            uint32_t mk = 0;
-            int qrow = 0;
-            if (lane == 0) walk.next(qrow, mk);
-            mk = __shfl_sync(0xffffffffu, mk, 0);
-            const bool valid = (mk >> half) & 1u;              // warp-uniform
-            const float4* nl4 = reinterpret_cast<const float4*>(xs + st * kXs) + 8 * wg;   // -lse*log2(e)
-            const float4* nd4 = nl4 + 16;                                                   // -Delta
-            if (ok)
-                ok = __all_sync(0xffffffffu, mbar_wait(B.prod + b, (g >> 1) & 1, B.abort_flag, dev_status) &&
-                                                 mbar_wait(B.fullx + st, (g / nst) & 1, B.abort_flag, dev_status));
-            // 32 columns of S^T and of dP^T: both TMEM loads in flight before one wait
-            uint32_t sv[32], pv[32];
-            if (ok) {
-                tc_fence_after();
-                if (valid) {
-                    tmem_ld32(tl + cS + 128 * b + 32 * wg, sv);
-                    tmem_ld32(tl + cP + 128 * b + 32 * wg, pv);
-                }
-                tmem_wait_ld();
+        int G = 0, kf = 0;
+        int st_ = 0, cy_ = 0;                              // ring stage and cycle of granule G
+        for (int it = blockIdx.x, j = 0; it < n_items; it += gridDim.x, ++j) {
+            const int4 item = items[it];
+            const int hh = item.x / tiles_per_head, tile = item.x % tiles_per_head;
+            const int g_begin = item.y, ng = item.z - item.y, slot = item.w;
+            const int64_t row0 = (int64_t)hh * N;
+            const uint32_t* u0 = rows_base + (j & 1) * 2 * SW;
+            GranuleWalk walk;
+            if (lane == 0) {
+                const bool got = ok && mbar_wait(B.rows_full + (j & 1), (j >> 1) & 1, B.abort_flag, dev_status);
+                walk.init(u0, u0 + SW, got ? wn : 0);
+                if (got) walk.skip(g_begin);
+                ok = got;
             }
-            named_sync(1, 256);                                // both warpgroups hold their columns
-            if (!ok) continue;
-            uint32_t op[16], od[16];
-            if (valid) {
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            for (int g = 0; g < ng; ++g) {
+                const int GG = G + g;
+                const int b = GG & 1;
+                const int st = st_;
+                const uint32_t cph = (uint32_t)cy_ & 1;
+                if (++st_ == nst) { st_ = 0; ++cy_; }
+                uint32_t mk = 0;
+                int qrow = 0;
+                if (lane == 0) walk.next(qrow, mk);
+                mk = __shfl_sync(0xffffffffu, mk, 0);
+                const bool valid = (mk >> half) & 1u;
+                const float4* nl4 = reinterpret_cast<const float4*>(xs + st * kXs) + 8 * wg;
+                const float4* nd4 = nl4 + 16;
+                if (ok)
+                    ok = __all_sync(0xffffffffu,
+                                    mbar_wait(B.prod + b, (uint32_t)(GG >> 1) & 1, B.abort_flag, dev_status) &&
+                                        mbar_wait(B.fullx + st, cph, B.abort_flag, dev_status));
+                uint32_t sv[32], pv[32];
+                if (ok) {
+                    tc_fence_after();
+                    if (valid) {
+                        tmem_ld32(tl + cS + 128 * b + 32 * wg, sv);
+                        tmem_ld32(tl + cP + 128 * b + 32 * wg, pv);
+                    }
+                    tmem_wait_ld();
+                }
+                named_sync(1, 256);
+                if (!ok) continue;
+                uint32_t op[16], od[16];
+                if (valid) {
 #pragma unroll
-                for (int i4 = 0; i4 < 8; ++i4) {
-                    const float4 l4 = nl4[i4];
-                    const float4 d4 = nd4[i4];
+                    for (int i4 = 0; i4 < 8; ++i4) {
+                        const float4 l4 = nl4[i4];
+                        const float4 d4 = nd4[i4];
 #pragma unroll
-                    for (int u = 0; u < 2; ++u) {
-                        const int i = 4 * i4 + 2 * u;
-                        const uint64_t nl = u ? f2pack(l4.z, l4.w) : f2pack(l4.x, l4.y);
-                        const uint64_t nd = u ? f2pack(d4.z, d4.w) : f2pack(d4.x, d4.y);
-                        float x0, x1;
-                        f2unpack(ffma2(f2pack(__uint_as_float(sv[i]), __uint_as_float(sv[i + 1])), sl2x2, nl), x0, x1);
-                        const float p0 = ex2(x0), p1 = ex2(x1);
-                        float d0, d1;
-                        f2unpack(fmul2(f2pack(p0, p1),
-                                       fadd2(f2pack(__uint_as_float(pv[i]), __uint_as_float(pv[i + 1])), nd)),
-                                 d0, d1);
-                        op[2 * i4 + u] = pack_bf16x2(p0, p1);
-                        od[2 * i4 + u] = pack_bf16x2(d0, d1);
+                        for (int u = 0; u < 2; ++u) {
+                            const int i = 4 * i4 + 2 * u;
+                            const uint64_t nl = u ? f2pack(l4.z, l4.w) : f2pack(l4.x, l4.y);
+                            const uint64_t nd = u ? f2pack(d4.z, d4.w) : f2pack(d4.x, d4.y);
+                            float x0, x1;
+                            f2unpack(ffma2(f2pack(__uint_as_float(sv[i]), __uint_as_float(sv[i + 1])), sl2x2, nl), x0,
+                                     x1);
+                            const float p0 = ex2(x0), p1 = ex2(x1);
+                            float d0, d1;
+                            f2unpack(fmul2(f2pack(p0, p1),
+                                           fadd2(f2pack(__uint_as_float(pv[i]), __uint_as_float(pv[i + 1])), nd)),
+                                     d0, d1);
+                            op[2 * i4 + u] = pack_bf16x2(p0, p1);
+                            od[2 * i4 + u] = pack_bf16x2(d0, d1);
+                        }
+                    }
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) { op[i] = 0u; od[i] = 0u; }
+                }
+                tmem_st16(tl + cS + 128 * b + 16 * wg, op);
+                tmem_st16(tl + cP + 128 * b + 16 * wg, od);
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(B.elem + b);
+            }
+            if (lane == 0) mbar_arrive(B.rows_empty + (j & 1));
+            bool fin = ok;
+            if (ng > 0) {
+                fin = __all_sync(0xffffffffu, ok && mbar_wait(B.fin, kf & 1, B.abort_flag, dev_status));
+                if (fin) tc_fence_after();
+                ++kf;
+            }
+            ok = fin;
+            // epilogue: dK (warpgroup 0) then dV (warpgroup 1), one 128-row region a pass
+            const bool part = slot >= 0, zero = ng == 0;
+            const int regions = part ? D / 32 : D / 64;
+            const uint32_t sw = (uint32_t)(row & 7);
+#pragma unroll 1
+            for (int out = 0; out < 2; ++out) {
+#pragma unroll 1
+                for (int r = 0; r < regions; ++r) {
+                    named_sync(2, 256);                    // the previous store has read the staging
+                    if (ok && wg == out) {
+                        const float mul = out ? 1.f : scale;
+                        const uint32_t tacc = tl + (out ? cdV : cdK);
+                        // bf16: region r = TMEM columns 64 r .. 64 r + 63; fp32: 32 r .. 32 r + 31
+                        const int nq = part ? 1 : 2;
+#pragma unroll 1
+                        for (int qq = 0; qq < nq; ++qq) {
+                            const int q = part ? r : 2 * r + qq;
+                            uint32_t v[32];
+                            if (zero) {
+#pragma unroll
+                                for (int i = 0; i < 32; ++i) v[i] = 0u;
+                            } else {
+                                tmem_ld32(tacc + 32 * q, v);
+                                tmem_wait_ld();
+                            }
+                            if (!part) {
+#pragma unroll
+                                for (int k = 0; k < 4; ++k) {
+                                    const int c = 4 * qq + k;              // 16-byte chunk within the region
+                                    uint4 w4;
+                                    w4.x = pack_bf16x2(__uint_as_float(v[8 * k + 0]) * mul, __uint_as_float(v[8 * k + 1]) * mul);
+                                    w4.y = pack_bf16x2(__uint_as_float(v[8 * k + 2]) * mul, __uint_as_float(v[8 * k + 3]) * mul);
+                                    w4.z = pack_bf16x2(__uint_as_float(v[8 * k + 4]) * mul, __uint_as_float(v[8 * k + 5]) * mul);
+                                    w4.w = pack_bf16x2(__uint_as_float(v[8 * k + 6]) * mul, __uint_as_float(v[8 * k + 7]) * mul);
+                                    *reinterpret_cast<uint4*>(staging + row * 128 + ((c ^ sw) << 4)) = w4;
+                                }
+                            } else {
+#pragma unroll
+                                for (int k = 0; k < 8; ++k) {
+                                    const float4 w4 = make_float4(__uint_as_float(v[4 * k]), __uint_as_float(v[4 * k + 1]),
+                                                                  __uint_as_float(v[4 * k + 2]),
+                                                                  __uint_as_float(v[4 * k + 3]));
+                                    *reinterpret_cast<float4*>(staging + row * 128 + ((k ^ sw) << 4)) = w4;
+                                }
+                            }
+                        }
+                        fence_proxy_async_smem();
+                    }
+                    named_sync(2, 256);
+                    if (ok && wg == out && (warp & 3) == 0 && lane == 0) {
+                        if (part) tma_store_3d(&tmPkv1, staging, 0, (slot * 2 + out) * 128, r);
+                        else tma_store_3d(out ? &tmdV1 : &tmdK1, staging, 0, (int)(row0 + 128 * tile), r);
+                        bulk_commit();
+                        bulk_wait_read();
                     }
                 }
-            } else {
-#pragma unroll
-                for (int i = 0; i < 16; ++i) { op[i] = 0u; od[i] = 0u; }
             }
-            tmem_st16(tl + cS + 128 * b + 16 * wg, op);        // P^T
-            tmem_st16(tl + cP + 128 * b + 16 * wg, od);        // dS^T
-            tmem_wait_st();
-            tc_fence_before();
-            mbar_arrive(B.elem + b);
+            G += ng;
         }
-        const bool fin = __all_sync(0xffffffffu, ok && mbar_wait(B.fin, 0, B.abort_flag, dev_status));
-        if (fin) tc_fence_after();
-        // warpgroup 0 writes dK, warpgroup 1 dV, each staged in its half of the (now free) ring;
-        // no query selected these keys (ng == 0): TMEM never written, zeros
-        store_tile<D>(tl + (wg ? cdV : cdK), row, fin, ng == 0, slot >= 0, wg ? 1.f : scale,
-                      sm + L::RING + wg * 2 * L::NR * kTile, wg ? &tmdV : &tmdK, &tmPkv, (int)(row0 + 128 * tile),
-                      (slot * 2 + wg) * 128, 2 + wg, 128, (warp & 3) == 0 && lane == 0);
     }
     tc_fence_before();
     __syncthreads();
@@ -595,6 +955,33 @@ k_bwd_dkdv_sm100(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
 }
 
 // ------------------------------------------------------------------ host side
+// whole-row view of a [rows][d] fp32 tensor (d/32 regions of 32 columns) whose
+// box covers `box_regions` regions: the persistent dQ epilogue stores an fp32
+// partial tile in passes of two regions
+bool make_map_bf16_rows_box(CUtensorMap* m, const void* base, int64_t rows, int d, int box_rows, int box_regions) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {64, (cuuint64_t)rows, (cuuint64_t)(d / 64)};
+    cuuint64_t strides[2] = {(cuuint64_t)d * 2, 128};
+    cuuint32_t box[3] = {64, (cuuint32_t)box_rows, (cuuint32_t)box_regions};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool make_map_f32_rows_box(CUtensorMap* m, const void* base, int64_t rows, int d, int box_rows, int box_regions) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {32, (cuuint64_t)rows, (cuuint64_t)(d / 32)};
+    cuuint64_t strides[2] = {(cuuint64_t)d * 4, 128};
+    cuuint32_t box[3] = {32, (cuuint32_t)box_rows, (cuuint32_t)box_regions};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 struct BwdWs {
     float* delta;
     float* nld;         // [heads*N/64][128]: per 64-row granule -lse*log2(e), then -Delta
@@ -637,28 +1024,33 @@ prism_status_t launch_bwd(const Dims& d, const void* Qp, const void* Kp, const v
         return PRISM_ERR_CUDA;
     const int target = plan_target(device_sms());
     const int64_t slots = 2 * (int64_t)target;
-    CUtensorMap tdQ, tdK, tdV, tPq, tPkv;
-    if (!make_map_bf16_rows(&tdQ, dQp, rows, D, 128) || !make_map_bf16_rows(&tdK, dKp, rows, D, 128) ||
-        !make_map_bf16_rows(&tdV, dVp, rows, D, 128) || !make_map_f32_rows(&tPq, w.part_q, slots * 128, D, 128) ||
-        !make_map_f32_rows(&tPkv, w.part_kv, slots * 2 * 128, D, 128))
+    // output maps: dQ whole rows; dK, dV and the dK/dV partials one 128-byte region a box
+    CUtensorMap tdQ, tdK1, tdV1, tPqh, tPkv1;
+    if (!make_map_bf16_rows(&tdQ, dQp, rows, D, 128) || !make_map_bf16_rows_box(&tdK1, dKp, rows, D, 128, 1) ||
+        !make_map_bf16_rows_box(&tdV1, dVp, rows, D, 128, 1) ||
+        !make_map_f32_rows_box(&tPqh, w.part_q, slots * 128, D, 128, D / 32 < 2 ? D / 32 : 2) ||
+        !make_map_f32_rows_box(&tPkv1, w.part_kv, slots * 2 * 128, D, 128, 1))
         return PRISM_ERR_CUDA;
     prism_status_t st = plan_work(w.pq, gsel, d, 2, 1, target, kSegMinGranules, s);
     if (st == PRISM_OK) st = plan_work(w.pkv, gselT, d, 2, 1, target, kSegMinGranules, s);
     if (st != PRISM_OK) return st;
-    const int nq = BwdLayout<D, false>::stages(0, (int)d.SW), nk = BwdLayout<D, true>::stages(kXs, (int)d.SW);
-    const int smq = BwdLayout<D, false>::alloc(nq, 0, (int)d.SW);
-    const int smk = BwdLayout<D, true>::alloc(nk, kXs, (int)d.SW);
+    const int nq = DqpLayout<D>::stages((int)d.SW), nk = DkvpLayout<D>::stages((int)d.SW);
+    const int smq = DqpLayout<D>::alloc(nq, (int)d.SW);
+    const int smk = DkvpLayout<D>::alloc(nk, (int)d.SW);
     if (smq > kSmemMax || smk > kSmemMax) return PRISM_ERR_UNSUPPORTED;   // selection rows too long
-    auto kq = k_bwd_dq_sm100<D>;
-    auto kk = k_bwd_dkdv_sm100<D>;
+    auto kq = k_bwd_dq_persist<D>;
+    auto kk = k_bwd_dkdv_persist<D>;
     if (cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, smq) != cudaSuccess ||
         cudaFuncSetAttribute(kk, cudaFuncAttributeMaxDynamicSharedMemorySize, smk) != cudaSuccess)
         return PRISM_ERR_CUDA;
-    kq<<<(unsigned)w.pq.items_max, 192, smq, s>>>((const __nv_bfloat16*)Qp, (const __nv_bfloat16*)dOp, gK, gV, tdQ, tPq,
-                                                  gsel, w.pq.hdr, w.pq.items, lse,
-                                                  w.delta, d.N, d.MB, (int)d.SW, nq, scale, dev_status);
-    kk<<<(unsigned)w.pkv.items_max, 384, smk, s>>>(tK, tV, gQ, gdO, tdK, tdV, tPkv, gselT, w.pkv.hdr, w.pkv.items,
-                                                   w.nld, d.N, d.MB, (int)d.SW, nk, scale, dev_status);
+    // persistent: one CTA per SM (all 512 TMEM columns each), items strided over the CTAs
+    const int64_t gq = w.pq.items_max < device_sms() ? w.pq.items_max : device_sms();
+    kq<<<(unsigned)gq, 192, smq, s>>>((const __nv_bfloat16*)Qp, (const __nv_bfloat16*)dOp, gK, gV, tdQ, tPqh,
+                                      gsel, w.pq.hdr, w.pq.items, lse, w.delta, d.N, d.MB, (int)d.SW, nq, scale,
+                                      dev_status);
+    const int64_t gk = w.pkv.items_max < device_sms() ? w.pkv.items_max : device_sms();
+    kk<<<(unsigned)gk, 384, smk, s>>>(tK, tV, gQ, gdO, tdK1, tdV1, tPkv1, gselT, w.pkv.hdr, w.pkv.items, w.nld, d.N,
+                                      d.MB, (int)d.SW, nk, scale, dev_status);
     st = launch_status(2);
     if (st == PRISM_OK) st = bwd_combine(w.pq, d, 1, w.part_q, dQp, scale, nullptr, 0.f, s);
     if (st == PRISM_OK) st = bwd_combine(w.pkv, d, 2, w.part_kv, dKp, scale, dVp, 1.f, s);

@@ -69,7 +69,9 @@ struct FwdParts {
 template <int D>
 __global__ void __launch_bounds__(192, 2)
 k_attn_fwd_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                 const __grid_constant__ CUtensorMap tmV, const uint32_t* __restrict__ gsel,
+                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                 const __grid_constant__ CUtensorMap tmOf, const __grid_constant__ CUtensorMap tmPo,
+                 const uint32_t* __restrict__ gsel,
                  const PlanHeader* __restrict__ hdr, const int4* __restrict__ items, FwdParts parts,
                  int64_t N, int64_t MB, int SW, float scale, __nv_bfloat16* __restrict__ O,
                  float* __restrict__ lse, float* __restrict__ o_f32, uint32_t* __restrict__ dev_status) {
@@ -106,10 +108,10 @@ k_attn_fwd_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     // the selection rows of the tile's two query granules
     load_rows(u0, u1, gsel + ((int64_t)hh * MB + 2 * tile) * SW, gsel + ((int64_t)hh * MB + 2 * tile + 1) * SW, wn);
     if (threadIdx.x == 0) {
-        mbar_init(bar_q, 1);
-        mbar_init(bar_kf, 1);
+        mbar_init(bar_q, L::NR);                           // one copy lane per region
+        mbar_init(bar_kf, L::NR);
         mbar_init(bar_ke, 1);
-        mbar_init(bar_vf, 1);
+        mbar_init(bar_vf, L::NR);
         mbar_init(bar_ve, 1);
         mbar_init(bar_s, 1);
         mbar_init(bar_p, 128);
@@ -127,43 +129,42 @@ k_attn_fwd_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     const uint32_t tbase = *tmem_slot;
 
     if (warp == 0) {
-        if (lane == 0) {
-            // ------------------------------------------------ TMA producer
-            tma_prefetch_desc(&tmQ);
-            tma_prefetch_desc(&tmK);
-            tma_prefetch_desc(&tmV);
-            mbar_expect_tx(bar_q, L::NR * kRegion);
-            for (int r = 0; r < L::NR; ++r)
+        // ---------------------------------------------------- TMA producer
+        // A copy engine completes the copies of one issuing thread one after
+        // another, so each (tensor, 64-column region) has a lane of its own:
+        // lane tensor * NR + r loads region r of Q (tensor 0 only, once), then of
+        // K (tensor 0) or V (tensor 1) for both key granules of every chunk.
+        if (lane < 2 * L::NR) {
+            const int tensor = lane / L::NR, r = lane % L::NR;
+            const CUtensorMap* mt = tensor ? &tmV : &tmK;
+            uint64_t* bfull = tensor ? bar_vf : bar_kf;
+            uint64_t* bempty = tensor ? bar_ve : bar_ke;
+            uint8_t* buf = tensor ? sV : sK;
+            tma_prefetch_desc(mt);
+            if (tensor == 0) {
+                tma_prefetch_desc(&tmQ);
+                mbar_expect_tx(bar_q, kRegion);
                 tma_load_2d(sQ + r * kRegion, &tmQ, bar_q, 64 * r, (int)(row0 + 128 * tile));
+            }
             GranuleWalk walk;
             walk.init(u0, u1, wn);
             walk.skip(2 * c_begin);
-            int issued_k = 0, issued_v = 0;
+            int issued = 0;
             for (int c = 0; c < nch && !*abort_flag; ++c) {
                 int ra = 0, rb = 0;
                 uint32_t ma, mb;
                 walk.next(ra, ma);
                 if (!walk.next(rb, mb)) rb = ra;
-                if (c > 0 && !mbar_wait(bar_ke, (c - 1) & 1, abort_flag, dev_status)) break;
-                mbar_expect_tx(bar_kf, 2 * L::NR * kGranBytes);
-                for (int r = 0; r < L::NR; ++r) {
-                    tma_load_2d(sK + r * kRegion, &tmK, bar_kf, 64 * r, (int)(row0 + ra));
-                    tma_load_2d(sK + r * kRegion + kGranBytes, &tmK, bar_kf, 64 * r, (int)(row0 + rb));
-                }
-                ++issued_k;
-                if (c > 0 && !mbar_wait(bar_ve, (c - 1) & 1, abort_flag, dev_status)) break;
-                mbar_expect_tx(bar_vf, 2 * L::NR * kGranBytes);
-                for (int r = 0; r < L::NR; ++r) {
-                    tma_load_2d(sV + r * kRegion, &tmV, bar_vf, 64 * r, (int)(row0 + ra));
-                    tma_load_2d(sV + r * kRegion + kGranBytes, &tmV, bar_vf, 64 * r, (int)(row0 + rb));
-                }
-                ++issued_v;
+                if (c > 0 && !mbar_wait(bempty, (c - 1) & 1, abort_flag, dev_status)) break;
+                mbar_expect_tx(bfull, 2 * kGranBytes);
+                tma_load_2d(buf + r * kRegion, mt, bfull, 64 * r, (int)(row0 + ra));
+                tma_load_2d(buf + r * kRegion + kGranBytes, mt, bfull, 64 * r, (int)(row0 + rb));
+                ++issued;
             }
-            if (*abort_flag) {
-                // let the copies already in flight land before the CTA goes away
+            if (*abort_flag && issued) {
+                // let this lane's copies land before the CTA goes away
                 volatile int no_abort = 0;
-                if (issued_k) mbar_wait(bar_kf, (issued_k - 1) & 1, &no_abort, dev_status);
-                if (issued_v) mbar_wait(bar_vf, (issued_v - 1) & 1, &no_abort, dev_status);
+                mbar_wait(bfull, (issued - 1) & 1, &no_abort, dev_status);
             }
         }
     } else if (warp == 1) {
@@ -305,61 +306,71 @@ k_attn_fwd_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             tc_fence_before();
             mbar_arrive(bar_p);
         }
-        const bool fin = ok && mbar_wait(bar_o, 0, abort_flag, dev_status);
-        if (__all_sync(0xffffffffu, fin)) {
-            tc_fence_after();
-            const int64_t grow = row0 + 128 * tile + row;
-            if (slot < 0) {
-                const float inv = l > 0.f ? 1.f / l : 0.f;
-                __nv_bfloat16* orow = O + grow * D;
+        const bool fin = __all_sync(0xffffffffu, ok && mbar_wait(bar_o, 0, abort_flag, dev_status));
+        if (fin) tc_fence_after();
+        // Epilogue.  Every MMA is complete, so Q, K and V are free: O (bf16) is
+        // staged in the Q buffer and the fp32 O or a split tile's partial in the
+        // K and V buffers, as 16-byte chunks in the 128-byte-swizzled image of the
+        // whole-row maps, and each goes out in one TMA store.  Every thread runs
+        // the barrier, also after a timeout.
+        const int64_t grow = row0 + 128 * tile + row;
+        const bool part = slot >= 0;
+        const bool zero = part ? nch == 0 : (!(l > 0.f) || nch == 0);   // nothing selected: O = 0
+        const float inv = l > 0.f ? 1.f / l : 0.f;
+        const uint32_t sw = (uint32_t)(row & 7);
+        if (fin) {
+#pragma unroll 1
+            for (int q = 0; q < D / 32; ++q) {
+                uint32_t r[32];
+                if (zero) {                                 // TMEM never written
 #pragma unroll
-                for (int q = 0; q < D / 32; ++q) {
-                    uint32_t r[32];
+                    for (int i = 0; i < 32; ++i) r[i] = 0u;
+                } else {
                     tmem_ld32(tl + kColO + 32 * q, r);
                     tmem_wait_ld();
-                    if (!(l > 0.f) || nch == 0) {           // nothing selected: O = 0 (TMEM never written)
+                }
+                if (!part) {
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) r[i] = 0u;
-                    }
-                    uint32_t pk[16];
-#pragma unroll
-                    for (int i = 0; i < 16; ++i)
-                        pk[i] = pack_bf16x2(__uint_as_float(r[2 * i]) * inv, __uint_as_float(r[2 * i + 1]) * inv);
-                    uint4* dst = reinterpret_cast<uint4*>(orow + 32 * q);
-#pragma unroll
-                    for (int i = 0; i < 4; ++i)
-                        dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
-                    if (o_f32) {
-                        float4* df = reinterpret_cast<float4*>(o_f32 + grow * D + 32 * q);
-#pragma unroll
-                        for (int i = 0; i < 8; ++i)
-                            df[i] = make_float4(__uint_as_float(r[4 * i]) * inv, __uint_as_float(r[4 * i + 1]) * inv,
-                                                __uint_as_float(r[4 * i + 2]) * inv,
-                                                __uint_as_float(r[4 * i + 3]) * inv);
+                    for (int k = 0; k < 4; ++k) {           // 4 chunks of 8 bf16
+                        const int g = 4 * q + k;
+                        uint4 v;
+                        v.x = pack_bf16x2(__uint_as_float(r[8 * k + 0]) * inv, __uint_as_float(r[8 * k + 1]) * inv);
+                        v.y = pack_bf16x2(__uint_as_float(r[8 * k + 2]) * inv, __uint_as_float(r[8 * k + 3]) * inv);
+                        v.z = pack_bf16x2(__uint_as_float(r[8 * k + 4]) * inv, __uint_as_float(r[8 * k + 5]) * inv);
+                        v.w = pack_bf16x2(__uint_as_float(r[8 * k + 6]) * inv, __uint_as_float(r[8 * k + 7]) * inv);
+                        *reinterpret_cast<uint4*>(sQ + (g >> 3) * kRegion + row * 128 + (((g & 7) ^ sw) << 4)) = v;
                     }
                 }
+                if (part || o_f32) {
+                    const float mul = part ? 1.f : inv;     // the partial stays unnormalised
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {           // 8 chunks of 4 fp32
+                        const int g = 8 * q + k;
+                        const float4 v = make_float4(__uint_as_float(r[4 * k]) * mul, __uint_as_float(r[4 * k + 1]) * mul,
+                                                     __uint_as_float(r[4 * k + 2]) * mul,
+                                                     __uint_as_float(r[4 * k + 3]) * mul);
+                        *reinterpret_cast<float4*>(sK + (g >> 3) * kRegion + row * 128 + (((g & 7) ^ sw) << 4)) = v;
+                    }
+                }
+            }
+            fence_proxy_async_smem();
+            if (!part) {
                 if (lse) lse[grow] = l > 0.f ? (m_run + log2f(l)) * kLn2 : -INFINITY;
             } else {
-                // partial of a split tile: unnormalised O, running max and denominator
-                float* po = parts.o + ((int64_t)slot * 128 + row) * D;
-#pragma unroll
-                for (int q = 0; q < D / 32; ++q) {
-                    uint32_t r[32];
-                    tmem_ld32(tl + kColO + 32 * q, r);
-                    tmem_wait_ld();
-                    if (nch == 0) {
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) r[i] = 0u;
-                    }
-                    float4* df = reinterpret_cast<float4*>(po + 32 * q);
-#pragma unroll
-                    for (int i = 0; i < 8; ++i)
-                        df[i] = make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
-                                            __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]));
-                }
                 parts.m[(int64_t)slot * 128 + row] = m_run;
                 parts.l[(int64_t)slot * 128 + row] = l;
             }
+        }
+        named_sync(1, 128);
+        if (fin && warp == 2 && lane == 0) {
+            if (!part) {
+                tma_store_3d(&tmO, sQ, 0, (int)(row0 + 128 * tile), 0);
+                if (o_f32) tma_store_3d(&tmOf, sK, 0, (int)(row0 + 128 * tile), 0);
+            } else {
+                tma_store_3d(&tmPo, sK, 0, slot * 128, 0);
+            }
+            bulk_commit();
+            bulk_wait_read();                               // shared memory stays valid until read
         }
     }
 
@@ -401,12 +412,18 @@ template <int D>
 prism_status_t launch_fwd(const Dims& d, const void* Qp, const void* Kp, const void* Vp, const uint32_t* gsel,
                           float scale, void* Op, float* lse, float* o_f32, uint32_t* dev_status, void* ws,
                           cudaStream_t s) {
-    CUtensorMap mQ, mK, mV;
+    CUtensorMap mQ, mK, mV, mO, mOf, mPo;
     const int64_t rows = (int64_t)d.heads * d.N;
     if (!make_map_bf16(&mQ, Qp, rows, D, 128) || !make_map_bf16(&mK, Kp, rows, D, 64) ||
         !make_map_bf16(&mV, Vp, rows, D, 64))
         return PRISM_ERR_CUDA;
     FwdWs w = carve_fwd(ws, d);
+    const int64_t slots = 2 * (int64_t)plan_target(device_sms());
+    // output maps: whole 128-row tiles (the fp32 O map is only built, and used, when o_f32 is given)
+    if (!make_map_bf16_rows(&mO, Op, rows, D, 128) || !make_map_f32_rows(&mPo, w.parts.o, slots * 128, D, 128) ||
+        (o_f32 && !make_map_f32_rows(&mOf, o_f32, rows, D, 128)))
+        return PRISM_ERR_CUDA;
+    if (!o_f32) mOf = mPo;                              // never used
     const int target = plan_target(device_sms());
     prism_status_t st = plan_work(w.plan, gsel, d, 2, 2, target, kSegMinChunks, s);
     if (st != PRISM_OK) return st;
@@ -414,7 +431,8 @@ prism_status_t launch_fwd(const Dims& d, const void* Qp, const void* Kp, const v
     const int smem = FwdLayout<D>::alloc((int)d.SW);
     if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return PRISM_ERR_CUDA;
-    k<<<(unsigned)w.plan.items_max, 192, smem, s>>>(mQ, mK, mV, gsel, w.plan.hdr, w.plan.items, w.parts, d.N, d.MB,
+    k<<<(unsigned)w.plan.items_max, 192, smem, s>>>(mQ, mK, mV, mO, mOf, mPo, gsel, w.plan.hdr, w.plan.items, w.parts,
+                                                    d.N, d.MB,
                                                     (int)d.SW, scale, (__nv_bfloat16*)Op, lse, o_f32, dev_status);
     st = launch_status(1);
     if (st != PRISM_OK) return st;
