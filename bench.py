@@ -170,30 +170,46 @@ def unpack_sel_dev(words: torch.Tensor, nb: int) -> torch.Tensor:
     return b[..., :nb].bool()
 
 
-def selected_flops(mod) -> dict:
-    """F_fwd = 4 d sum_h sum_i |B_i| sum_{j in S_i} |B_j| and density figures."""
+def _popcount_rows(words: torch.Tensor) -> torch.Tensor:
+    """Set bits per row of an int32 [..., SW] bitmask (int64)."""
+    w = words.to(torch.int64) & 0xFFFFFFFF
+    cnt = torch.zeros(w.shape[:-1], dtype=torch.int64, device=w.device)
+    for s in range(32):
+        cnt += ((w >> s) & 1).sum(-1)
+    return cnt
+
+
+def selected_flops(mod, rows_per_chunk=1024) -> dict:
+    """F_fwd = 4 d sum_h sum_i |B_i| sum_{j in S_i} |B_j| and density figures.
+
+    Works one head and a bounded chunk of selection rows at a time, so that it
+    fits beside the layer at every grid size."""
     nb = mod.num_blocks()
     bs = mod.blk_start[: nb + 1].to(torch.int64)
     sz = (bs[1:] - bs[:-1]).to(torch.float64)
-    sel = unpack_sel_dev(mod.sel, nb).to(torch.float64)
-    keys_per_row = sel @ sz                                   # [h, nb] selected key tokens
+    keys_per_row = torch.empty((mod.heads, nb), dtype=torch.float64, device=sz.device)
+    n_sel = torch.empty((mod.heads, nb), dtype=torch.float64, device=sz.device)
+    for hh in range(mod.heads):
+        for r0 in range(0, nb, rows_per_chunk):
+            r1 = min(nb, r0 + rows_per_chunk)
+            w = mod.sel[hh, r0:r1].to(torch.int64) & 0xFFFFFFFF
+            sh = torch.arange(32, device=w.device, dtype=torch.int64)
+            bits = ((w.unsqueeze(-1) >> sh) & 1).reshape(r1 - r0, -1)[:, :nb].to(torch.float64)
+            keys_per_row[hh, r0:r1] = bits @ sz
+            n_sel[hh, r0:r1] = bits.sum(-1)
     f_fwd = 4.0 * mod.d * float((keys_per_row * sz).sum().item())
     dense = 4.0 * mod.d * mod.heads * float(sz.sum().item()) ** 2
     vol = {int(v): int((sz == v).sum().item()) for v in (64, 128, 256)}
     # work per 128-row tile of the attention kernels: union of its granules' selections
-    g = mod.gsel.to(torch.int64) & 0xFFFFFFFF
-    pop = lambda w: sum(((w >> s) & 1) for s in range(32))
-    tile_gran = pop(g[:, 0::2, :] | g[:, 1::2, :]).sum(-1).double()            # [h, N/128]
-    q = torch.tensor([0.5, 0.99, 1.0], dtype=torch.float64, device=tile_gran.device)
-    tq = torch.quantile(tile_gran.flatten(), q).tolist()
+    q = torch.tensor([0.5, 0.99, 1.0], dtype=torch.float64, device=sz.device)
+    tile_gran = torch.cat([_popcount_rows(mod.gsel[hh, 0::2] | mod.gsel[hh, 1::2]) for hh in range(mod.heads)])
+    tq = torch.quantile(tile_gran.double(), q).tolist()
     kq = None
     if mod.gselT is not None:
-        gT = mod.gselT.to(torch.int64) & 0xFFFFFFFF
-        key_gran = pop(gT[:, 0::2, :] | gT[:, 1::2, :]).sum(-1).double()
-        kq = torch.quantile(key_gran.flatten(), q).tolist()
+        key_gran = torch.cat([_popcount_rows(mod.gselT[hh, 0::2] | mod.gselT[hh, 1::2]) for hh in range(mod.heads)])
+        kq = torch.quantile(key_gran.double(), q).tolist()
     return {"F_fwd": f_fwd, "F_dense_fwd": dense, "n_blk": nb, "density": f_fwd / dense,
-            "mean_sel_blocks": float(sel.sum(-1).mean().item()),
-            "max_sel_blocks": float(sel.sum(-1).max().item()),
+            "mean_sel_blocks": float(n_sel.mean().item()), "max_sel_blocks": float(n_sel.max().item()),
             "mean_sel_tokens": float(keys_per_row.mean().item()), "block_volumes": vol,
             "tile_key_granules_p50_p99_max": tq, "tile_query_granules_p50_p99_max": kq}
 
@@ -386,6 +402,12 @@ def bench_prism(args, cfg, rank, world, local_rank):
 
 
 def bench_e2e(args, cfg, mod, x, dev, world, attn_flops):
+    """The same metric end to end through the library's host-buffer step
+    (prism_layer_step_host): every step uploads its inputs from page-locked host
+    memory, runs the layer and downloads its outputs, one cudaMemcpyAsync per
+    tensor on two copy streams beside the compute stream.  Timed from an event
+    on the compute stream before the first step to one on the download stream
+    after the last, where every step's work ends."""
     names = ("Q", "K", "V", "hhat", "dO") if mod.with_backward else ("Q", "K", "V", "hhat")
     hin = {k: torch.empty(x[k].shape, dtype=x[k].dtype, pin_memory=True) for k in names}
     for k in names:
@@ -393,32 +415,31 @@ def bench_e2e(args, cfg, mod, x, dev, world, attn_flops):
     dx = {k: torch.empty_like(x[k]) for k in names}
     n_out = 4 if mod.with_backward else 1
     hout = [torch.empty(x["Q"].shape, dtype=x["Q"].dtype, pin_memory=True) for _ in range(n_out)]
-    out = torch.empty_like(x["Q"])
-    grads = [torch.empty_like(x["Q"]) for _ in range(n_out - 1)]
+    douts = [torch.empty_like(x["Q"]) for _ in range(n_out)]
+    mod.attach_io(dx["Q"], dx["K"], dx["V"], dx["hhat"], douts[0], dx.get("dO"), *(douts[1:] + [None] * (4 - n_out)))
+    compute, h2d, d2h = (torch.cuda.Stream(device=dev) for _ in range(3))
     steps = max(1, min(args.steps, 3))
+    hargs = [hin["Q"], hin["K"], hin["V"], hin["hhat"], hin.get("dO")] + hout + [None] * (4 - n_out)
 
     def one():
-        for k in names:
-            dx[k].copy_(hin[k], non_blocking=True)
-        run_step(mod, dx, out, grads)
-        for h, d in zip(hout, [out] + grads):
-            h.copy_(d, non_blocking=True)
+        mod.step_host(*hargs, compute, h2d, d2h)
 
     one()
     torch.cuda.synchronize()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record()
+    a.record(compute)
     for _ in range(steps):
         one()
-    b.record()
+    b.record(d2h)
     torch.cuda.synchronize()
     ms = a.elapsed_time(b) / steps
     ms = max_over_ranks([ms], dev)[0]
-    h2d = sum(hin[k].numel() * hin[k].element_size() for k in names)
-    d2h = sum(h.numel() * h.element_size() for h in hout)
+    h2d_b = sum(hin[k].numel() * hin[k].element_size() for k in names)
+    d2h_b = sum(h.numel() * h.element_size() for h in hout)
     return {"value": round(job_tflops(world, attn_flops, ms), 3), "unit": "TFLOP/s",
-            "ms_per_step": round(ms, 3), "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-            "steps": steps, "note": "selected-block FLOPs over the whole layer step incl. host copies"}
+            "ms_per_step": round(ms, 3), "h2d_bytes_per_step": int(h2d_b), "d2h_bytes_per_step": int(d2h_b),
+            "steps": steps, "api": "prism_layer_step_host (C ABI, host buffers, three streams)",
+            "note": "selected-block FLOPs over the whole layer step incl. host copies"}
 
 
 def bench_reference(args, cfg):

@@ -23,7 +23,10 @@ EXPORTS = ("prism_query_sizes", "prism_zone_indicator", "prism_assign_shapes", "
            "prism_unpermute", "prism_block_pool_score", "prism_block_select",
            "prism_sparse_attn_fwd", "prism_sparse_attn_bwd", "prism_read_status",
            "prism_status_string", "prism_version", "prism_launch_count",
-           "prism_zone_indicator_noalloc", "prism_zone_indicator_ex", "prism_assign_shapes_ex")
+           "prism_zone_indicator_noalloc", "prism_zone_indicator_ex", "prism_assign_shapes_ex",
+           "prism_layer_init", "prism_layer_arena_bytes", "prism_layer_bind", "prism_layer_forward",
+           "prism_layer_backward", "prism_layer_step_host", "prism_layer_sizeof",
+           "prism_zone_partials", "prism_zone_finalize")
 GUIDANCE = {"joint": 0, "video": 1, "audio": 2}
 NOALLOC_SCRATCH_BYTES = 2 << 20
 
@@ -39,6 +42,28 @@ class Sizes(ctypes.Structure):
                 ("max_blocks", ctypes.c_int64), ("sel_words", ctypes.c_int64),
                 ("ws_indicator", ctypes.c_size_t), ("ws_attn_fwd", ctypes.c_size_t),
                 ("ws_attn_bwd", ctypes.c_size_t), ("bytes_P_max", ctypes.c_size_t)]
+
+
+_VP = ctypes.c_void_p
+
+
+class LayerT(ctypes.Structure):
+    """Mirror of prism_layer_t (field order and types as in include/prism.h)."""
+    _fields_ = [("prob", Problem), ("top_k", ctypes.c_int32), ("top_p", ctypes.c_float),
+                ("eps", ctypes.c_float), ("tau128", ctypes.c_float), ("tau256", ctypes.c_float),
+                ("scale", ctypes.c_float), ("guidance", ctypes.c_int32), ("fixed_shape", ctypes.c_int32),
+                ("with_backward", ctypes.c_int32), ("with_io", ctypes.c_int32), ("p_blocks", ctypes.c_int64),
+                ("g", _VP), ("rho", _VP), ("abar", _VP), ("zone_stats", _VP),
+                ("ws_ind", _VP), ("ws_ind_bytes", ctypes.c_size_t),
+                ("shape_id", _VP), ("perm", _VP), ("blk_start", _VP), ("gran_blk", _VP), ("n_blk", _VP),
+                ("margin_shape", _VP), ("Qp", _VP), ("Kp", _VP), ("Vp", _VP),
+                ("Qbar", _VP), ("Kbar", _VP), ("P", _VP), ("sel", _VP), ("gsel", _VP), ("gselT", _VP),
+                ("sel_count", _VP), ("margin_sel", _VP), ("dev_status", _VP),
+                ("Op", _VP), ("Of32", _VP), ("lse", _VP), ("ws_fwd", _VP), ("ws_fwd_bytes", ctypes.c_size_t),
+                ("dOp", _VP), ("dQp", _VP), ("dKp", _VP), ("dVp", _VP),
+                ("ws_bwd", _VP), ("ws_bwd_bytes", ctypes.c_size_t),
+                ("Q", _VP), ("K", _VP), ("V", _VP), ("hhat", _VP), ("O", _VP), ("dO", _VP),
+                ("dQ", _VP), ("dK", _VP), ("dV", _VP)]
 
 
 class PrismError(RuntimeError):
@@ -78,6 +103,14 @@ _SIGS = {
     "prism_sparse_attn_fwd": [_PROB, _P, _P, _P, _P, _F, _P, _P, _P, _P, _P, _SZ, _P],
     "prism_sparse_attn_bwd": [_PROB, _P, _P, _P, _P, _P, _P, _P, _P, _P, _F, _P, _P, _P, _P, _P, _SZ, _P],
     "prism_read_status": [_P, ctypes.POINTER(ctypes.c_uint32), _P],
+    "prism_zone_partials": [_PROB, _P, _P, _P, _P, _SZ, _P],
+    "prism_zone_finalize": [_PROB, _P, _F, _I, _P, _P, _P, _P, _P, _SZ, _P],
+    "prism_layer_init": [ctypes.POINTER(LayerT), _PROB],
+    "prism_layer_arena_bytes": [ctypes.POINTER(LayerT), ctypes.POINTER(ctypes.c_size_t)],
+    "prism_layer_bind": [ctypes.POINTER(LayerT), _P, _SZ],
+    "prism_layer_forward": [ctypes.POINTER(LayerT), _P, _P, _P, _P, _P, _P],
+    "prism_layer_backward": [ctypes.POINTER(LayerT), _P, _P, _P, _P, _P],
+    "prism_layer_step_host": [ctypes.POINTER(LayerT), _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P],
 }
 
 
@@ -100,6 +133,8 @@ def lib(path: str | None = None):
         L.prism_version.restype = ctypes.c_char_p
         L.prism_launch_count.argtypes = []
         L.prism_launch_count.restype = ctypes.c_ulonglong
+        L.prism_layer_sizeof.argtypes = []
+        L.prism_layer_sizeof.restype = ctypes.c_size_t
         _lib = L
     return _lib
 
@@ -229,3 +264,46 @@ def version() -> str:
 
 def launch_count() -> int:
     return int(lib().prism_launch_count())
+
+
+# ---------------------------------------------------------------- the layer object
+def layer_init(prob) -> LayerT:
+    L = LayerT()
+    _check("prism_layer_init", lib().prism_layer_init(ctypes.byref(L), ctypes.byref(prob)))
+    return L
+
+
+def layer_arena_bytes(L: LayerT) -> int:
+    n = ctypes.c_size_t(0)
+    _check("prism_layer_arena_bytes", lib().prism_layer_arena_bytes(ctypes.byref(L), ctypes.byref(n)))
+    return n.value
+
+
+def prism_layer_forward(L: LayerT, Q, K, V, hhat, O, stream=None):
+    _check("prism_layer_forward", lib().prism_layer_forward(ctypes.byref(L), _ptr(Q), _ptr(K), _ptr(V),
+                                                            _ptr(hhat), _ptr(O), _stream(stream)))
+
+
+def prism_layer_backward(L: LayerT, dO, dQ, dK, dV, stream=None):
+    _check("prism_layer_backward", lib().prism_layer_backward(ctypes.byref(L), _ptr(dO), _ptr(dQ), _ptr(dK),
+                                                              _ptr(dV), _stream(stream)))
+
+
+def prism_layer_step_host(L: LayerT, hQ, hK, hV, hhhat, hdO, hO, hdQ, hdK, hdV, compute, h2d, d2h):
+    """One step from host (pinned CPU tensor) buffers; see include/prism.h."""
+    _check("prism_layer_step_host", lib().prism_layer_step_host(
+        ctypes.byref(L), _ptr(hQ), _ptr(hK), _ptr(hV), _ptr(hhhat), _ptr(hdO), _ptr(hO), _ptr(hdQ), _ptr(hdK),
+        _ptr(hdV), _stream(compute), _stream(h2d), _stream(d2h)))
+
+
+# ---------------------------------------------------------------- head-sharded indicator
+def prism_zone_partials(prob_local, V_local, hhat, partials, ws, stream=None):
+    _check("prism_zone_partials", lib().prism_zone_partials(ctypes.byref(prob_local), _ptr(V_local), _ptr(hhat),
+                                                            _ptr(partials), _ptr(ws), ws.numel(),
+                                                            _stream(stream)))
+
+
+def prism_zone_finalize(prob, partials, eps, guidance, g, rho, abar, zone_stats, ws, stream=None):
+    _check("prism_zone_finalize", lib().prism_zone_finalize(
+        ctypes.byref(prob), _ptr(partials), eps, GUIDANCE.get(guidance, guidance), _ptr(g), _ptr(rho), _ptr(abar),
+        _ptr(zone_stats), _ptr(ws), ws.numel(), _stream(stream)))

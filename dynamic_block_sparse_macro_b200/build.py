@@ -3,7 +3,9 @@
     python -m dynamic_block_sparse_macro_b200.build [--force] [-v]
 
 Compiles every ``csrc/*.cu`` with nvcc in parallel and links them into
-``dynamic_block_sparse_macro_b200/libprism.so``.  Rebuilds only what changed.
+``dynamic_block_sparse_macro_b200/libprism.so``, then builds the C example
+``prism_layer_driver`` (``csrc/prism_layer_driver.c``: one layer step from host
+buffers through the C ABI alone) against it.  Rebuilds only what changed.
 """
 from __future__ import annotations
 
@@ -20,6 +22,8 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 OBJ = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libprism.so")
+DRIVER_SRC = os.path.join(CSRC, "prism_layer_driver.c")
+DRIVER = os.path.join(PKG, "prism_layer_driver")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",
@@ -72,7 +76,23 @@ def build(force: bool = False, verbose: bool = False, extra: list[str] | None = 
         if r.returncode != 0:
             raise RuntimeError(f"link failed:\n{r.stderr}")
         os.replace(tmp, LIB)
+    build_driver()
     return LIB
+
+
+def build_driver() -> str:
+    """The C driver, linked to libprism.so (found next to it at run time)."""
+    if os.path.exists(DRIVER) and os.path.getmtime(DRIVER) >= max(os.path.getmtime(LIB),
+                                                                  os.path.getmtime(DRIVER_SRC), _headers_mtime()):
+        return DRIVER
+    tmp = DRIVER + ".tmp"
+    cmd = [nvcc(), *ARCH, "-O2", "-x", "c", DRIVER_SRC, "-I", INCLUDE, "-L", PKG, "-lprism",
+           "-Xlinker", "-rpath,$ORIGIN", "-o", tmp]
+    r = subprocess.run(cmd, capture_output=True, text=True)
+    if r.returncode != 0:
+        raise RuntimeError(f"driver build failed:\n{r.stderr}")
+    os.replace(tmp, DRIVER)
+    return DRIVER
 
 
 if __name__ == "__main__":

@@ -84,7 +84,8 @@ struct SelCut {
     int n;
     uint32_t vb;
     int need_eq;
-    float gap_p;     // cumulative-sum margin of the Top-p decision (inf if Top-p cannot set n)
+    float gap_p;     // cumulative-sum margin: the sum of the n selected above p (when n can
+                     // still grow) and, when Top-p sets n (n_p > n_k), p above the sum of n-1
 };
 
 // count_ge(t) = #{P >= t}, sum_ge(t) = sum{P >= t} for bit patterns t (row-wide)
@@ -94,7 +95,16 @@ __device__ __forceinline__ SelCut select_cut(int nb, int top_k, float top_p, Cou
     const int n_k = min(top_k, nb);
     const float total = sum_ge(0u);
     if (!(top_p < 1.f) || total < top_p) {       // Top-p takes the whole row
-        if (top_p < 1.f) c.gap_p = fabsf(total - top_p);
+        if (top_p < 1.f && nb > n_k && nb >= 2) {
+            // n_p = nb falls to nb - 1 once the nb - 1 largest reach p
+            uint32_t lo = 0u, hi = 0x3F800001u;      // smallest value: count{P >= lo} == nb
+            while (hi - lo > 1u) {
+                const uint32_t mid = lo + ((hi - lo) >> 1);
+                if (count_ge(mid) >= nb) lo = mid;
+                else hi = mid;
+            }
+            c.gap_p = top_p - (total - __uint_as_float(lo));
+        }
         return c;
     }
     constexpr uint32_t kHi = 0x3F800001u;        // (1.0f bits) + 1: no P reaches it
@@ -113,10 +123,9 @@ __device__ __forceinline__ SelCut select_cut(int nb, int top_k, float top_p, Cou
         gt_k = count_ge(lo + 1u);
         const float vk = __uint_as_float(lo);
         const float S_k = sum_ge(lo + 1u) + (float)(n_k - gt_k) * vk;
-        if (S_k >= top_p) {                      // n_p <= n_k
-            k_sets = true;
-            const float S_prev = n_k >= 2 ? S_k - vk : -INFINITY;
-            if (S_prev < top_p) c.gap_p = fminf(fabsf(S_k - top_p), fabsf(top_p - S_prev));   // n_p == n_k
+        if (S_k >= top_p) {                      // n_p <= n_k: Top-k sets n; a shorter Top-p
+            k_sets = true;                       // prefix changes nothing, a longer one does
+            if (n_k < nb) c.gap_p = S_k - top_p;
         }
     }
     if (!k_sets) {
@@ -138,8 +147,9 @@ __device__ __forceinline__ SelCut select_cut(int nb, int top_k, float top_p, Cou
         const int n_p = c_gt + m;
         if (n_p >= n_k) {
             const float c_at = s_gt + (float)m * vstar;
-            const float c_before = n_p >= 2 ? c_at - vstar : -INFINITY;
-            c.gap_p = fminf(fabsf(c_at - top_p), fabsf(top_p - c_before));
+            const float up = n_p < nb ? c_at - top_p : INFINITY;
+            const float down = (n_p > n_k && n_p >= 2) ? top_p - (c_at - vstar) : INFINITY;
+            c.gap_p = fminf(up, down);
             c.n = n_p;
             c.vb = lo;
             c.need_eq = m;

@@ -293,6 +293,68 @@ extern "C" prism_status_t prism_zone_indicator(const prism_problem_t* prob, cons
 }
 
 // ---------------------------------------------------------------------------
+// Head-sharded indicator: a rank holding some of the heads computes the
+// per-zone sums over its own channels (prism_zone_partials); one all-reduce
+// (sum) of the [Z][4] video sums over the ranks makes them the sums over all
+// D channels; prism_zone_finalize then forms g, rho and abar exactly as
+// prism_zone_indicator does.  The audio statistics come from hhat, which every
+// rank holds whole, so they need no reduction.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) k_zone_chunk_sum(const float* __restrict__ part, int Z, int nchunk,
+                                                        float* __restrict__ out) {
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;      // (zone, statistic)
+    if (i >= Z * 4) return;
+    const int m = i >> 2, q = i & 3;
+    float s = 0.f;
+    for (int k = 0; k < nchunk; ++k) s += part[((int64_t)m * nchunk + k) * 4 + q];
+    out[i] = s;
+}
+
+extern "C" prism_status_t prism_zone_partials(const prism_problem_t* prob_local, const void* V_local,
+                                              const void* hhat, float* partials, void* ws, size_t ws_bytes,
+                                              cudaStream_t stream) {
+    Dims d;
+    prism_status_t st = make_dims(prob_local, &d);
+    if (st != PRISM_OK) return st;
+    if (!ok_ptr(V_local) || !ok_ptr(hhat) || !ok_ptr(partials) || !ok_ptr(ws)) return PRISM_ERR_INVALID_ARG;
+    if (d.Da & 1) return PRISM_ERR_UNSUPPORTED;
+    if (ws_bytes < zone_indicator_ws_bytes(d)) return PRISM_ERR_WORKSPACE;
+    const int CH = d.dtype == PRISM_BF16 ? 64 : 32;
+    const int nchunk = (int)(d.D / CH);
+    float* part = (float*)ws;
+    dim3 gv((unsigned)nchunk, (unsigned)d.Z);
+    if (d.dtype == PRISM_BF16) {
+        k_zone_video<__nv_bfloat16><<<gv, 256, 0, stream>>>((const __nv_bfloat16*)V_local, d.H, d.W, d.D,
+                                                             nchunk, part);
+        k_zone_audio<__nv_bfloat16><<<(unsigned)d.Z, 512, 0, stream>>>((const __nv_bfloat16*)hhat, d.H, d.W,
+                                                                       d.Da, partials + d.Z * 4);
+    } else {
+        k_zone_video<float><<<gv, 256, 0, stream>>>((const float*)V_local, d.H, d.W, d.D, nchunk, part);
+        k_zone_audio<float><<<(unsigned)d.Z, 512, 0, stream>>>((const float*)hhat, d.H, d.W, d.Da,
+                                                               partials + d.Z * 4);
+    }
+    k_zone_chunk_sum<<<(unsigned)((d.Z * 4 + 255) / 256), 256, 0, stream>>>(part, (int)d.Z, nchunk, partials);
+    return launch_status(3);
+}
+
+extern "C" prism_status_t prism_zone_finalize(const prism_problem_t* prob, const float* partials, float eps,
+                                              int32_t guidance, float* g, float* rho, float* abar,
+                                              float* zone_stats, void* ws, size_t ws_bytes, cudaStream_t stream) {
+    if (guidance != PRISM_GUIDE_JOINT && guidance != PRISM_GUIDE_VIDEO && guidance != PRISM_GUIDE_AUDIO)
+        return PRISM_ERR_INVALID_ARG;
+    Dims d;
+    prism_status_t st = make_dims(prob, &d);
+    if (st != PRISM_OK) return st;
+    if (!ok_ptr(partials) || !ok_ptr(g) || !ok_ptr(rho) || !ok_ptr(abar) || !ok_opt(zone_stats) || !ok_ptr(ws))
+        return PRISM_ERR_INVALID_ARG;
+    if (!(eps > 0.f) || !isfinite(eps)) return PRISM_ERR_INVALID_ARG;
+    if (ws_bytes < (size_t)d.Z * 4 * sizeof(float)) return PRISM_ERR_WORKSPACE;
+    k_zone_finalize<<<1, 1024, 0, stream>>>(partials, partials + d.Z * 4, (int)d.Z, 1, 1.f / (float)d.D, eps, g,
+                                            rho, abar, zone_stats, (float*)ws, guidance);
+    return launch_status(1);
+}
+
+// ---------------------------------------------------------------------------
 // Allocation-free variant of prism_zone_indicator.
 //
 // Some callers cannot hand us a workspace: a host that has no device

@@ -1,12 +1,16 @@
 """One Prism video self-attention layer on the GPU, stage by stage through the C ABI.
 
 ``PrismSparseAttention`` owns the device buffers of one problem size (torch
-allocations: device memory is the only thing torch provides here) and issues
-the ABI calls in order on the current CUDA stream:
+allocations: device memory is the only thing torch provides here), describes
+them to the library as one ``prism_layer_t`` and runs the stages on the current
+CUDA stream through the library's layer calls:
 
   forward:  zone_indicator(V, hhat) -> assign_shapes -> permute(Q, K, V)
             -> block_pool_score -> block_select -> sparse_attn_fwd -> unpermute(O)
   backward: permute(dO) -> sparse_attn_bwd -> unpermute(dQ, dK, dV)
+
+The per-stage methods (``plan``, ``select``, ``attend``) issue the same stage
+calls one by one, for callers that time or inspect a stage.
 
 Inputs and outputs are raster ``[N, heads, head_dim]`` tensors (``hhat`` is
 ``[N, audio_dim]``).  No step runs on the CPU and nothing synchronises the
@@ -79,6 +83,40 @@ class PrismSparseAttention:
             self.dOp = e(heads, N, head_dim, dt=self.tdt)
             self.dQp, self.dKp, self.dVp = (e(heads, N, head_dim, dt=self.tdt) for _ in range(3))
             self.ws_bwd = e(max(16, s.ws_attn_bwd), dt=torch.uint8)
+        self.L = self._describe()
+
+    def _describe(self):
+        """The library's view of this layer: parameters and buffer addresses."""
+        L = _abi.layer_init(self.prob)
+        L.top_k, L.top_p, L.eps = self.top_k, self.top_p, self.eps
+        L.tau128, L.tau256, L.scale = self.tau128, self.tau256, self.scale
+        L.guidance, L.fixed_shape = _abi.GUIDANCE[self.guidance], self.fixed_shape
+        L.with_backward, L.with_io, L.p_blocks = int(self.with_backward), 0, self.p_blocks
+        for name in ("g", "rho", "abar", "zone_stats", "ws_ind", "shape_id", "perm", "blk_start", "gran_blk",
+                     "n_blk", "margin_shape", "Qp", "Kp", "Vp", "Qbar", "Kbar", "P", "sel", "gsel", "gselT",
+                     "sel_count", "margin_sel", "dev_status", "Op", "Of32", "lse", "ws_fwd"):
+            t = getattr(self, name)
+            setattr(L, name, t.data_ptr() if t is not None else None)
+        L.ws_ind_bytes = self.ws_ind.numel()
+        L.ws_fwd_bytes = self.ws_fwd.numel()
+        if self.with_backward:
+            for name in ("dOp", "dQp", "dKp", "dVp", "ws_bwd"):
+                setattr(L, name, getattr(self, name).data_ptr())
+            L.ws_bwd_bytes = self.ws_bwd.numel()
+        return L
+
+    def attach_io(self, Q, K, V, hhat, O, dO=None, dQ=None, dK=None, dV=None):
+        """Device raster tensors that ``step_host`` uploads into and downloads from."""
+        self._io = (Q, K, V, hhat, O, dO, dQ, dK, dV)
+        for name, t in zip(("Q", "K", "V", "hhat", "O", "dO", "dQ", "dK", "dV"), self._io):
+            setattr(self.L, name, t.data_ptr() if t is not None else None)
+        self.L.with_io = 1
+
+    def step_host(self, hQ, hK, hV, hhhat, hdO, hO, hdQ, hdK, hdV, compute, h2d, d2h):
+        """One whole step from pinned host tensors through the library's host-buffer
+        call (uploads, forward, backward, downloads on three streams).  Asynchronous:
+        the host outputs are final once ``d2h`` has passed this call."""
+        _abi.prism_layer_step_host(self.L, hQ, hK, hV, hhhat, hdO, hO, hdQ, hdK, hdV, compute, h2d, d2h)
 
     # ------------------------------------------------------------------ stages
     def plan(self, V, hhat, stream=None):
@@ -115,12 +153,9 @@ class PrismSparseAttention:
         rows beyond the selection's capacity leave every selection row empty
         and O = 0, and a timed-out wait leaves outputs incomplete.  With
         check=False nothing synchronises; call ``check_status()`` later."""
-        self.plan(V, hhat, stream)
-        self.select(Q, K, V, stream)
-        self.attend(stream)
         if out is None:
             out = torch.empty_like(Q)
-        _abi.prism_unpermute(self.prob, self.Op, self.perm, out, stream)
+        _abi.prism_layer_forward(self.L, Q, K, V, hhat, out, stream)
         if check:
             self.check_status(stream)
         return out
@@ -130,17 +165,8 @@ class PrismSparseAttention:
         as in ``forward``."""
         if not self.with_backward:
             raise RuntimeError("this layer was built for inference (with_backward=False)")
-        p = self.prob
-        _abi.prism_permute(p, dO, self.perm, self.dOp, stream)
-        _abi.prism_sparse_attn_bwd(p, self.Qp, self.Kp, self.Vp, self.Op, self.Of32, self.dOp, self.lse,
-                                   self.gsel, self.gselT, self.scale, self.dQp, self.dKp, self.dVp,
-                                   self.dev_status, self.ws_bwd, stream)
-        outs = []
-        for src, dst in ((self.dQp, dQ), (self.dKp, dK), (self.dVp, dV)):
-            if dst is None:
-                dst = torch.empty_like(dO)
-            _abi.prism_unpermute(p, src, self.perm, dst, stream)
-            outs.append(dst)
+        outs = [t if t is not None else torch.empty_like(dO) for t in (dQ, dK, dV)]
+        _abi.prism_layer_backward(self.L, dO, *outs, stream)
         if check:
             self.check_status(stream)
         return tuple(outs)

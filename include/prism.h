@@ -117,6 +117,32 @@ prism_status_t prism_zone_indicator_ex(const prism_problem_t* prob, const void* 
                                        float eps, int32_t guidance, float* g, float* rho, float* abar,
                                        float* zone_stats, void* ws, size_t ws_bytes, cudaStream_t stream);
 
+/*
+ * Stage 1 split for heads spread over several GPUs.  The indicator's video
+ * statistics are sums over all D = heads*head_dim channels of V (the pages
+ * form D from every channel; one shape per zone serves every head), so a rank
+ * holding some of the heads computes the sums over its own channels, the
+ * ranks add them with one all-reduce, and each rank finishes alone:
+ *   prism_zone_partials(prob_local, V_local, hhat, partials, ws, ...)
+ *       prob_local: the problem with heads = this rank's heads;
+ *       V_local raster [N][local heads * head_dim];  hhat whole, [N][audio_dim];
+ *       partials [2][Z][4] float32: [0] per zone the sums over the local
+ *       channels of (8 sigma2_vT, 8 sigma2_vH, 8 sigma2_vW, 512 rho_raw) times
+ *       the channel count (un-normalised sums of squared deviations);
+ *       [1] the audio statistics (A, sigma2_aT, sigma2_aH, sigma2_aW), the
+ *       same on every rank.  ws >= sizes.ws_indicator of prob_local.
+ *   all-reduce (sum) of partials[0] ([Z][4] floats, contiguous) over the ranks
+ *   prism_zone_finalize(prob, partials, eps, guidance, g, rho, abar, zone_stats, ws, ...)
+ *       prob: the whole problem (all heads); outputs as prism_zone_indicator_ex;
+ *       ws >= Z*16 bytes of scratch.
+ * The result equals prism_zone_indicator_ex up to the order of the fp32 sums.
+ */
+prism_status_t prism_zone_partials(const prism_problem_t* prob_local, const void* V_local, const void* hhat,
+                                   float* partials, void* ws, size_t ws_bytes, cudaStream_t stream);
+prism_status_t prism_zone_finalize(const prism_problem_t* prob, const float* partials, float eps,
+                                   int32_t guidance, float* g, float* rho, float* abar, float* zone_stats,
+                                   void* ws, size_t ws_bytes, cudaStream_t stream);
+
 /* Size of the library-owned scratch array behind prism_zone_indicator_noalloc. */
 #define PRISM_NOALLOC_SCRATCH_BYTES (2u << 20)
 
@@ -217,8 +243,11 @@ prism_status_t prism_block_pool_score(const prism_problem_t* prob, const void* Q
  *             of the block of qg (blk_start, gran_blk from prism_assign_shapes)
  *   gselT     [heads][N/64][sel_words] uint32 (nullable): transpose of gsel, the
  *             key-major view of the backward (inference passes NULL)
- *   margin    [heads][max_blocks] float32 (nullable): smallest gap (order or
- *             cumulative-sum) that, crossed by rounding, could change S_i
+ *   margin    [heads][max_blocks] float32 (nullable): the smallest change of the
+ *             row (L1 size) that could change S_i: the gap between the last
+ *             selected and the first unselected value; the sum of S_i above p
+ *             (while n < n_blk); when Top-p sets n (n_p > n_k), p above the sum
+ *             of the n-1 largest.  inf when nothing can change S_i.
  *   dev_status  PRISM_DEV_BAD_INDEX if n_blk exceeds 16384, the longest row the
  *             selection holds on chip (rows of up to 4096 blocks sit in registers,
  *             longer ones in shared memory); every row is then left empty.
@@ -277,6 +306,84 @@ const char* prism_version(void);
 /* Number of kernels this library has launched since it was loaded (all
  * threads, all devices); a diagnostics counter for profiling harnesses. */
 unsigned long long prism_launch_count(void);
+
+/* ==========================================================================
+ * The whole layer as one object.  The pages describe the stages; this is their
+ * call sequence, in the order above, over buffers carved from one caller-owned
+ * device arena, for hosts that want one call per direction (a C program, a
+ * binding).  The struct is transparent: after prism_layer_bind every buffer
+ * pointer is set and may be read (or, with the same sizes, set by a caller that
+ * allocates the buffers one by one instead of binding an arena).
+ * ========================================================================== */
+typedef struct {
+    /* parameters (prism_layer_init sets the defaults shown) */
+    prism_problem_t prob;
+    int32_t top_k;          /* 8                                                    */
+    float top_p;            /* 0.9                                                  */
+    float eps;              /* 1e-6: the indicator's epsilon                        */
+    float tau128, tau256;   /* 0.5, 0.25: the block-volume thresholds on rho        */
+    float scale;            /* 1/sqrt(head_dim)                                     */
+    int32_t guidance;       /* PRISM_GUIDE_JOINT                                    */
+    int32_t fixed_shape;    /* -1: adaptive shapes                                  */
+    int32_t with_backward;  /* 1; 0 = inference: no LSE, fp32 O, gselT, backward buffers */
+    int32_t with_io;        /* 0; 1 = also the raster inputs/outputs, for prism_layer_step_host */
+    int64_t p_blocks;       /* 0: P sized for max_blocks; else a caller-known bound on n_blk */
+    /* device buffers; shapes and layouts as the stage calls above describe them */
+    float *g, *rho, *abar, *zone_stats;
+    void* ws_ind;
+    size_t ws_ind_bytes;
+    uint8_t* shape_id;
+    int32_t *perm, *blk_start, *gran_blk, *n_blk;
+    float* margin_shape;
+    void *Qp, *Kp, *Vp;
+    float *Qbar, *Kbar, *P;
+    uint32_t *sel, *gsel, *gselT;
+    int32_t* sel_count;
+    float* margin_sel;
+    uint32_t* dev_status;   /* cleared by the caller before the first step          */
+    void* Op;
+    float *Of32, *lse;
+    void* ws_fwd;
+    size_t ws_fwd_bytes;
+    void *dOp, *dQp, *dKp, *dVp;
+    void* ws_bwd;
+    size_t ws_bwd_bytes;
+    /* raster Q, K, V, hhat, O, dO, dQ, dK, dV on the device (with_io only) */
+    void *Q, *K, *V, *hhat, *O, *dO, *dQ, *dK, *dV;
+} prism_layer_t;
+
+/* Fill L with the defaults above for `prob` and no buffers (host only). */
+prism_status_t prism_layer_init(prism_layer_t* L, const prism_problem_t* prob);
+/* Bytes of the arena prism_layer_bind needs for L's parameters (host only). */
+prism_status_t prism_layer_arena_bytes(const prism_layer_t* L, size_t* bytes);
+/* Carve every buffer of L from `arena` (device memory, 256-byte aligned, at
+ * least prism_layer_arena_bytes; caller-owned).  Host only: no CUDA call. */
+prism_status_t prism_layer_bind(prism_layer_t* L, void* arena, size_t bytes);
+/* Stages 1-6 and the unpermute of O on `stream`: raster device Q, K, V, hhat in,
+ * raster O out.  Asynchronous; read L->dev_status (prism_read_status) after. */
+prism_status_t prism_layer_forward(const prism_layer_t* L, const void* Q, const void* K, const void* V,
+                                   const void* hhat, void* O, cudaStream_t stream);
+/* Stage 7 for the last forward on `stream`: raster device dO in, raster dQ, dK,
+ * dV out.  PRISM_ERR_UNSUPPORTED when L has no backward buffers. */
+prism_status_t prism_layer_backward(const prism_layer_t* L, const void* dO, void* dQ, void* dK, void* dV,
+                                    cudaStream_t stream);
+/* One whole step from HOST buffers (L bound with with_io = 1): uploads Q, K,
+ * V, hhat (and dO with a backward), runs the layer, downloads O (and dQ, dK,
+ * dV), with one cudaMemcpyAsync per tensor on the two copy streams: V and
+ * hhat first, dO during the forward, O during the backward.  Three distinct
+ * streams.  Host buffers should be page-locked, or the copies do not overlap.
+ * Asynchronous: every device step of the call precedes its last download on
+ * `d2h`, so the host outputs are final once `d2h` has passed this call (e.g.
+ * cudaStreamSynchronize(d2h)).  Consecutive calls with the same streams are
+ * ordered: the next call's uploads wait for this call's compute, and its
+ * writes of O and the gradients wait for this call's downloads, which may
+ * still run while the next uploads do.  Host input buffers must stay unchanged
+ * and output buffers unread until then. */
+prism_status_t prism_layer_step_host(const prism_layer_t* L, const void* hQ, const void* hK, const void* hV,
+                                     const void* hhhat, const void* hdO, void* hO, void* hdQ, void* hdK,
+                                     void* hdV, cudaStream_t compute, cudaStream_t h2d, cudaStream_t d2h);
+/* sizeof(prism_layer_t) as compiled into the library (a check for bindings). */
+size_t prism_layer_sizeof(void);
 
 #ifdef __cplusplus
 }

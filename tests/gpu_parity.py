@@ -4,9 +4,10 @@ the GPU's upstream decisions) so that one near-tie does not cascade.
 
 Tolerances (the bar): integer/index outputs bit-exact except decisions whose
 oracle margin is below NEAR_TIE (counted and returned); attention outputs
-and gradients within relative L2 error 1e-5 (f32 storage) or 1e-2 (bf16),
-over the whole tensor and, at twice that, over every (head, block) on its own
-so that one bad tile cannot hide among hundreds of good ones."""
+and gradients within relative L2 error 1e-5 (f32 storage) or 1e-2 (bf16)
+over the whole tensor, and every (head, block) on its own (O at twice that,
+gradients at five times that against at least a tenth of the typical block
+norm) so that one bad tile cannot hide among hundreds of good ones."""
 from __future__ import annotations
 
 import numpy as np
@@ -151,6 +152,12 @@ def check_layer(cfg, x, top_k=None, top_p=None, backward=True, heads=None, grad_
     badr2 = (sel_g != e2e["sel"]).any(-1)
     assert (e2e["margin"][badr2] < NEAR_TIE).all()
     rep["select_near_ties"] = int(badr2.sum())
+    # the kernel's own margin (fp32 sums) against the oracle's on the same P
+    mg = mod.margin_sel.cpu().double().numpy()[:, :nb]
+    om = tf["margin"]
+    fin = np.isfinite(om) & (om > 1e-4)
+    assert (np.isinf(mg) == np.isinf(om)).all()
+    assert np.allclose(mg[fin], om[fin], rtol=1e-3, atol=2e-6), np.abs(mg[fin] - om[fin]).max()
     rep["density"] = float(sel_g.mean())
     # granule-level view: row qg, bit kg set iff block(kg) in S_block(qg); and its transpose
     G = unpack_sel(mod.gsel, cfg.n_tokens // 64)
@@ -182,10 +189,14 @@ def check_layer(cfg, x, top_k=None, top_p=None, backward=True, heads=None, grad_
             got = host(dev)[hs]
             rep[name + "_rel_l2"] = rel_l2(got, ref, floor)
             assert rep[name + "_rel_l2"] <= tol, rep
-            # per (head, block); a key block that no query selected has an exact zero
-            # gradient, so blocks are measured against at least 1% of the RMS block norm
-            rep[name + "_block_max_rel_l2"] = block_rel_l2(got, ref, bs, floor=1e-2)
-            assert grad_floor > 0 or rep[name + "_block_max_rel_l2"] <= 2 * tol, rep
+            # per (head, block).  Every row of dS sums to zero over its keys, so a
+            # block's gradient is a cancelling sum that can be much smaller than the
+            # terms forming it (and a key block no query selected has an exact zero
+            # gradient): blocks are measured against at least 10% of the RMS block
+            # norm, at 5x the whole-tensor bar.  A wrong tile still fails by orders
+            # of magnitude.
+            rep[name + "_block_max_rel_l2"] = block_rel_l2(got, ref, bs, floor=0.1)
+            assert grad_floor > 0 or rep[name + "_block_max_rel_l2"] <= 5 * tol, rep
         for dev, out in zip((mod.dQp, mod.dKp, mod.dVp), grads):
             assert np.array_equal(bits(out), orc.unpermute(bits(dev), perm))
     assert mod.status() == 0

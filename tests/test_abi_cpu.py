@@ -96,3 +96,47 @@ def test_bad_pointers_rejected_before_launch(L):
     assert L.prism_zone_indicator(ctypes.byref(p), fake, fake, 1e-6, fake, fake, fake, None, fake, 4, None) == 4
     assert L.prism_assign_shapes(ctypes.byref(p), fake, fake, 0.25, 0.5, fake, fake, None, fake, fake, fake,
                                  None, None) == 1      # tau256 > tau128
+
+
+# ---------------------------------------------------------------- the layer object
+def test_layer_struct_matches_the_c_compiler(L):
+    # the C driver prints sizeof and every field offset as the C compiler lays them out
+    from dynamic_block_sparse_macro_b200 import build
+    drv = build.build_driver()
+    out = subprocess.run([drv, "offsets"], capture_output=True, text=True, check=True).stdout.split("\n")
+    got = dict(line.split() for line in out if line.strip())
+    assert int(got.pop("sizeof")) == ctypes.sizeof(_abi.LayerT) == L.prism_layer_sizeof()
+    names = [f[0] for f in _abi.LayerT._fields_]
+    assert sorted(got) == sorted(names)
+    for name in names:
+        assert int(got[name]) == getattr(_abi.LayerT, name).offset, name
+
+
+def test_layer_init_defaults_and_arena_carving(L):
+    p = _abi.problem(32, 72, 128, 24, 128, 64, "bf16")
+    lay = _abi.layer_init(p)
+    assert (lay.top_k, round(lay.top_p, 6), lay.fixed_shape, lay.with_backward, lay.with_io) == (8, 0.9, -1, 1, 0)
+    assert abs(lay.scale - 128 ** -0.5) < 1e-7
+    sz = _abi.query_sizes(p)
+    train = _abi.layer_arena_bytes(lay)
+    lay.with_backward = 0
+    infer = _abi.layer_arena_bytes(lay)
+    lay.with_backward, lay.with_io = 1, 1
+    io = _abi.layer_arena_bytes(lay)
+    tok = 294912 * 24 * 128 * 2
+    assert infer < train < io
+    # the training layer holds at least Qp, Kp, Vp, Op, dOp, dQp, dKp, dVp, fp32 O, P, workspaces
+    assert train >= 8 * tok + 2 * tok + sz.bytes_P_max + sz.ws_attn_bwd + sz.ws_attn_fwd
+    assert io - train >= 8 * tok                     # Q K V O dO dQ dK dV (+ hhat)
+    # bind on a fake, aligned device address: host-only pointer arithmetic
+    base = 1 << 40
+    assert L.prism_layer_bind(ctypes.byref(lay), base, io - 1) == 4              # too small
+    assert L.prism_layer_bind(ctypes.byref(lay), base + 16, io) == 1             # misaligned
+    assert L.prism_layer_bind(ctypes.byref(lay), base, io) == 0
+    ptrs = [getattr(lay, f[0]) for f in _abi.LayerT._fields_ if f[1] is ctypes.c_void_p]
+    assert all(q is not None and base <= q < base + io and q % 256 == 0 for q in ptrs)
+    assert len(set(ptrs)) == len(ptrs)
+    assert lay.ws_bwd_bytes == sz.ws_attn_bwd and lay.ws_fwd_bytes == sz.ws_attn_fwd
+    # bad parameters are refused before anything is carved
+    lay.top_p = 0.0
+    assert L.prism_layer_arena_bytes(ctypes.byref(lay), ctypes.byref(ctypes.c_size_t())) == 1
