@@ -129,29 +129,36 @@ __device__ __forceinline__ BarsP carve_p(uint8_t* ctrl) {
 static_assert((3 * kStages + 11) * 8 + 8 <= kCtrl, "barriers overflow the control block");
 
 // Epilogue with a 32 KB staging area of its own (the ring is busy with the
-// next item): the bf16 tile (D/64 regions) in one store, the fp32 partial
-// (D/32 regions) in passes of two regions.  The barrier at the top of every
-// pass makes the staging free: the leader passes it only after its previous
-// store has finished reading shared memory.  Every thread of the group runs
-// the same barriers whatever `ok` is (passes depend on `part` only).
+// next item), shared by the two elementwise warpgroups, warpgroup wg owning
+// accumulator columns 64 wg .. 64 wg + 63: the bf16 tile (D/64 regions) in one
+// store, each warpgroup writing its own region; the fp32 partial (D/32
+// regions) in passes of two regions, pass p written by warpgroup p.  The
+// barrier at the top of every pass makes the staging free: the leader passes
+// it only after its previous store has finished reading shared memory.  Every
+// thread of both warpgroups runs the same barriers whatever `ok` is (passes
+// depend on `part` only).
 template <int D>
-__device__ void store_tile_p(uint32_t tacc, int row, bool ok, bool zero, bool part, float mul, uint8_t* stage,
-                             const CUtensorMap* map_bf16, const CUtensorMap* map_f32h, int y_bf16, int y_f32,
-                             int bar_id, int nthreads, bool leader) {
+__device__ void store_tile_p(uint32_t tacc, int row, int wg, bool ok, bool zero, bool part, float mul,
+                             uint8_t* stage, const CUtensorMap* map_bf16, const CUtensorMap* map_f32h, int y_bf16,
+                             int y_f32, int bar_id, int nthreads, bool leader) {
+    static_assert(D == 128 || D == 64, "head_dim");
     const int regions = part ? D / 32 : D / 64;            // 128-byte regions of a row
     const int per_pass = regions < 2 ? regions : 2;
     const int passes = regions / per_pass;
     const uint32_t sw = (uint32_t)(row & 7);
+    constexpr int kColsWg = D / 2;                          // accumulator columns of one warpgroup
 #pragma unroll 1
     for (int p = 0; p < passes; ++p) {
         named_sync(bar_id, nthreads);
-        if (ok) {
-            // 32 fp32 TMEM columns per load: a quarter of a bf16 region pair, one fp32 region
-            const int q0 = part ? p * per_pass : 0, q1 = part ? q0 + per_pass : D / 32;
+        // fp32 pass p covers columns 32 p * per_pass ..; bf16 covers every column in one pass
+        const int c0 = part ? 32 * per_pass * p : 0, c1 = part ? c0 + 32 * per_pass : D;
+        const int w0 = kColsWg * wg, w1 = w0 + kColsWg;     // this warpgroup's columns
+        const int q0 = (c0 > w0 ? c0 : w0) / 32, q1 = (c1 < w1 ? c1 : w1) / 32;
+        if (ok && q0 < q1) {
 #pragma unroll 1
-            for (int q = q0; q < q1; ++q) {
+            for (int q = q0; q < q1; ++q) {                   // 32 fp32 TMEM columns per load
                 uint32_t r[32];
-                if (zero) {                                           // an empty item: TMEM is not read
+                if (zero) {                                   // an empty item: TMEM is not read
 #pragma unroll
                     for (int i = 0; i < 32; ++i) r[i] = 0u;
                 } else {
@@ -161,7 +168,7 @@ __device__ void store_tile_p(uint32_t tacc, int row, bool ok, bool zero, bool pa
                 if (!part) {
 #pragma unroll
                     for (int k = 0; k < 4; ++k) {
-                        const int g = 4 * q + k;                      // 16-byte chunk of the bf16 row
+                        const int g = 4 * q + k;              // 16-byte chunk of the bf16 row
                         uint4 v;
                         v.x = pack_bf16x2(__uint_as_float(r[8 * k + 0]) * mul, __uint_as_float(r[8 * k + 1]) * mul);
                         v.y = pack_bf16x2(__uint_as_float(r[8 * k + 2]) * mul, __uint_as_float(r[8 * k + 3]) * mul);
@@ -172,7 +179,7 @@ __device__ void store_tile_p(uint32_t tacc, int row, bool ok, bool zero, bool pa
                 } else {
 #pragma unroll
                     for (int k = 0; k < 8; ++k) {
-                        const int g = 8 * (q - q0) + k;               // 16-byte chunk within this pass
+                        const int g = 8 * (q - c0 / 32) + k;  // 16-byte chunk within this pass
                         const float4 v = make_float4(__uint_as_float(r[4 * k]), __uint_as_float(r[4 * k + 1]),
                                                      __uint_as_float(r[4 * k + 2]), __uint_as_float(r[4 * k + 3]));
                         *reinterpret_cast<float4*>(stage + (g >> 3) * kTile + row * 128 + (((g & 7) ^ sw) << 4)) = v;
@@ -191,32 +198,28 @@ __device__ void store_tile_p(uint32_t tacc, int row, bool ok, bool zero, bool pa
     }
 }
 
-// Q and dO rows of one tile into TMEM as bf16 (two per 32-bit column)
+// One row of Q or dO into TMEM as bf16 (two per 32-bit column)
 template <int D>
-__device__ __forceinline__ void load_qdo(uint32_t tl, uint32_t cQ, uint32_t cdO, const __nv_bfloat16* Qg,
-                                         const __nv_bfloat16* dOg, int64_t grow) {
+__device__ __forceinline__ void load_row_tmem(uint32_t taddr, const __nv_bfloat16* src_rows, int64_t grow) {
+    const uint4* src = reinterpret_cast<const uint4*>(src_rows + grow * D);
 #pragma unroll
-    for (int which = 0; which < 2; ++which) {
-        const uint4* src = reinterpret_cast<const uint4*>((which ? dOg : Qg) + grow * D);
+    for (int q = 0; q < D / 64; ++q) {
+        uint32_t r[32];
 #pragma unroll
-        for (int q = 0; q < D / 64; ++q) {
-            uint32_t r[32];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const uint4 v = __ldg(src + 8 * q + i);
-                r[4 * i] = v.x;
-                r[4 * i + 1] = v.y;
-                r[4 * i + 2] = v.z;
-                r[4 * i + 3] = v.w;
-            }
-            tmem_st32(tl + (which ? cdO : cQ) + 32 * q, r);
+        for (int i = 0; i < 8; ++i) {
+            const uint4 v = __ldg(src + 8 * q + i);
+            r[4 * i] = v.x;
+            r[4 * i + 1] = v.y;
+            r[4 * i + 2] = v.z;
+            r[4 * i + 3] = v.w;
         }
+        tmem_st32(taddr + 32 * q, r);
     }
     tmem_wait_st();
 }
 
 template <int D>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
 k_bwd_dq_persist(const __nv_bfloat16* __restrict__ Qg, const __nv_bfloat16* __restrict__ dOg,
                  const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                  const __grid_constant__ CUtensorMap tmdQ, const __grid_constant__ CUtensorMap tmPqh,
@@ -246,11 +249,11 @@ k_bwd_dq_persist(const __nv_bfloat16* __restrict__ Qg, const __nv_bfloat16* __re
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(B.prod + b, 1);
-            mbar_init(B.elem + b, 128);
+            mbar_init(B.elem + b, 256);
             mbar_init(B.rows_full + b, 32);
-            mbar_init(B.rows_empty + b, 4);
+            mbar_init(B.rows_empty + b, 8);
         }
-        mbar_init(B.qdo_full, 128);
+        mbar_init(B.qdo_full, 256);
         mbar_init(B.fin, 1);
         mbar_init(B.drain, 1);
         *B.abort_flag = 0;
@@ -377,9 +380,9 @@ k_bwd_dq_persist(const __nv_bfloat16* __restrict__ Qg, const __nv_bfloat16* __re
                     tc_fence_after();
                     const uint32_t aK = aR + s * L::STAGE;
 #pragma unroll
-                    for (int k = 0; k < 4; ++k)
-                        mma_ts_w(tb + cdQ, tb + cS + 128 * b + 8 * k, sdesc_sw128(aK + k * 2048, kGran, 1024), idQ,
-                                 (gp > 0 || k > 0) ? 1u : 0u);
+                    for (int k = 0; k < 4; ++k)              // dS keys 16 k ..: warpgroup k / 2's columns
+                        mma_ts_w(tb + cdQ, tb + cS + 128 * b + 32 * (k >> 1) + 8 * (k & 1),
+                                 sdesc_sw128(aK + k * 2048, kGran, 1024), idQ, (gp > 0 || k > 0) ? 1u : 0u);
                     tc_commit_w(B.empty + s);
                 }
                 if (g < ng) {
@@ -399,6 +402,11 @@ k_bwd_dq_persist(const __nv_bfloat16* __restrict__ Qg, const __nv_bfloat16* __re
         }
     } else {
         // ---------------------------------------------------------------- elementwise + epilogue
+        // Two warpgroups (warps 2-5, 6-9) on every granule: warpgroup wg turns key
+        // columns 32 wg .. 32 wg + 31 of S and dP into dS and writes it, as bf16,
+        // over the first 16 of those columns, so neither touches the other's
+        // columns and no barrier joins them per granule.
+        const int wg = (warp - 2) >> 2;
         const int sub = warp & 3, row = sub * 32 + lane, half = row >> 6;
         const uint32_t tl = tb + ((uint32_t)(sub * 32) << 16);
         const float sl2 = scale * kLog2e;
@@ -406,15 +414,16 @@ k_bwd_dq_persist(const __nv_bfloat16* __restrict__ Qg, const __nv_bfloat16* __re
         bool ok = true;
         int G = 0;
         int kf = 0;                                        // non-empty items so far
-        // Q and dO of a non-empty item go into TMEM once the previous non-empty
-        // item's S/dP products are consumed; the first one before the loop
+        // Q (warpgroup 0) and dO (warpgroup 1) of a non-empty item go into TMEM
+        // once both warpgroups have consumed every S/dP product of the previous
+        // non-empty item; the first one before the loop
         auto qdo_ahead = [&](int itn) {
             if (itn >= n_items) return;
             const int4 nx = items[itn];
             if (nx.z == nx.y) return;                      // empty: never reaches the MMA warp
             if (ok) {
                 const int64_t ngrow = (int64_t)(nx.x / tiles_per_head) * N + 128 * (nx.x % tiles_per_head) + row;
-                load_qdo<D>(tl, cQ, cdO, Qg, dOg, ngrow);
+                load_row_tmem<D>(tl + (wg ? cdO : cQ), wg ? dOg : Qg, ngrow);
                 tc_fence_before();
             }
             mbar_arrive(B.qdo_full);
@@ -454,44 +463,40 @@ k_bwd_dq_persist(const __nv_bfloat16* __restrict__ Qg, const __nv_bfloat16* __re
                 const bool got = mbar_wait(B.prod + b, (uint32_t)(GG >> 1) & 1, B.abort_flag, dev_status);
                 if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
                 tc_fence_after();
-                // one 32-column half of S and dP at a time (both loads in flight before one wait)
-#pragma unroll
-                for (int hq = 0; hq < 2; ++hq) {
-                    uint32_t sv[32], pv[32];
-                    if (valid) {
-                        tmem_ld32(tl + cS + 128 * b + 32 * hq, sv);
-                        tmem_ld32(tl + cP + 128 * b + 32 * hq, pv);
-                        tmem_wait_ld();
-                    }
-                    uint32_t o[16];
-                    if (valid) {
-#pragma unroll
-                        for (int i = 0; i < 16; ++i) {
-                            float x0, x1;
-                            f2unpack(ffma2(f2pack(__uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1])), sl2x2,
-                                           nlse2),
-                                     x0, x1);
-                            const uint64_t pp = f2pack(ex2(x0), ex2(x1));
-                            const uint64_t dp =
-                                fadd2(f2pack(__uint_as_float(pv[2 * i]), __uint_as_float(pv[2 * i + 1])), ndl2);
-                            float d0, d1;
-                            f2unpack(fmul2(pp, dp), d0, d1);
-                            o[i] = pack_bf16x2(d0, d1);
-                        }
-                    } else {
-#pragma unroll
-                        for (int i = 0; i < 16; ++i) o[i] = 0u;
-                    }
-                    // dS (bf16) over S columns this half has consumed: half hq writes 16 hq .. 16 hq + 15,
-                    // inside the 32 columns the first half already read
-                    tmem_st16(tl + cS + 128 * b + 16 * hq, o);
+                const uint32_t cs = cS + 128 * b + 32 * wg, cp = cP + 128 * b + 32 * wg;
+                uint32_t sv[32], pv[32];
+                if (valid) {                                   // both loads in flight before one wait
+                    tmem_ld32(tl + cs, sv);
+                    tmem_ld32(tl + cp, pv);
+                    tmem_wait_ld();
                 }
+                uint32_t o[16];
+                if (valid) {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        float x0, x1;
+                        f2unpack(ffma2(f2pack(__uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1])), sl2x2,
+                                       nlse2),
+                                 x0, x1);
+                        const uint64_t pp = f2pack(ex2(x0), ex2(x1));
+                        const uint64_t dp =
+                            fadd2(f2pack(__uint_as_float(pv[2 * i]), __uint_as_float(pv[2 * i + 1])), ndl2);
+                        float d0, d1;
+                        f2unpack(fmul2(pp, dp), d0, d1);
+                        o[i] = pack_bf16x2(d0, d1);
+                    }
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) o[i] = 0u;
+                }
+                tmem_st16(tl + cs, o);                         // dS (bf16) over this warpgroup's S columns
                 tmem_wait_st();
                 tc_fence_before();
                 mbar_arrive(B.elem + b);
             }
             if (lane == 0) mbar_arrive(B.rows_empty + (j & 1));
-            // the next non-empty item's Q and dO: this item's S/dP products are all consumed
+            // the next non-empty item's Q and dO: this warpgroup has seen every S/dP
+            // product of this item complete, and so has the other before its own load
             qdo_ahead(it + (int)gridDim.x);
             bool fin = ok;
             if (ng > 0) {
@@ -501,8 +506,8 @@ k_bwd_dq_persist(const __nv_bfloat16* __restrict__ Qg, const __nv_bfloat16* __re
             }
             ok = fin;
             // the item's dQ (or zeros when nothing was selected: ng == 0)
-            store_tile_p<D>(tl + cdQ, row, fin, ng == 0, slot >= 0, scale, staging, &tmdQ, &tmPqh,
-                            (int)(row0 + 128 * tile), slot * 128, 1, 128, warp == 2 && lane == 0);
+            store_tile_p<D>(tl + cdQ, row, wg, fin, ng == 0, slot >= 0, scale, staging, &tmdQ, &tmPqh,
+                            (int)(row0 + 128 * tile), slot * 128, 1, 256, warp == 2 && lane == 0);
             G += ng;
         }
     }
@@ -698,7 +703,7 @@ k_bwd_dkdv_persist(const __grid_constant__ CUtensorMap tmK, const __grid_constan
                             mbar_expect_tx(full + stage, L::NR * kGran);
                             tma_load_3d(sm + L::RING + stage * L::STAGE + kind * L::NR * kGran, mg, full + stage, 0,
                                         (int)(row0 + row), 0);
-                        }
+                            }
                         last_cyc = c_;
                     }
                     if (++s_ == nst) { s_ = 0; ++c_; }
@@ -768,12 +773,11 @@ k_bwd_dkdv_persist(const __grid_constant__ CUtensorMap tmK, const __grid_constan
                     tc_fence_after();
                     const uint32_t aQ = aR + s * L::STAGE, adO = aQ + L::NR * kGran;
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) {
+                    for (int k = 0; k < 4; ++k) {            // queries 16 k ..: warpgroup k / 2's columns
                         const uint32_t acc = (gp > 0 || k > 0) ? 1u : 0u;
-                        mma_ts_w(tb + cdV, tb + cS + 128 * b + 8 * k, sdesc_sw128(adO + k * 2048, kGran, 1024), idKV,
-                                 acc);
-                        mma_ts_w(tb + cdK, tb + cP + 128 * b + 8 * k, sdesc_sw128(aQ + k * 2048, kGran, 1024), idKV,
-                                 acc);
+                        const uint32_t ck = 128 * b + 32 * (k >> 1) + 8 * (k & 1);
+                        mma_ts_w(tb + cdV, tb + cS + ck, sdesc_sw128(adO + k * 2048, kGran, 1024), idKV, acc);
+                        mma_ts_w(tb + cdK, tb + cP + ck, sdesc_sw128(aQ + k * 2048, kGran, 1024), idKV, acc);
                     }
                     tc_commit_w(B.empty + s);
                 }
@@ -795,8 +799,10 @@ k_bwd_dkdv_persist(const __grid_constant__ CUtensorMap tmK, const __grid_constan
       }
     } else {
         regs_inc<kRegsHigh>();
-        // both warpgroups on every granule, warpgroup wg on its 32 query columns
-        // (see the non-persistent kernel); every thread runs every named barrier
+        // Both warpgroups on every granule, warpgroup wg on query columns 32 wg ..
+        // 32 wg + 31 of S^T and dP^T; it writes P^T and dS^T as bf16 over the first
+        // 16 of its own columns, so no barrier joins the two per granule.  Every
+        // thread runs every named barrier of the epilogue.
         const int wg = (warp - 4) >> 2;
         const int sub = warp & 3, row = sub * 32 + lane, half = row >> 6;
         const uint32_t tl = tb + ((uint32_t)(sub * 32) << 16);
@@ -845,7 +851,6 @@ k_bwd_dkdv_persist(const __grid_constant__ CUtensorMap tmK, const __grid_constan
                     }
                     tmem_wait_ld();
                 }
-                named_sync(1, 256);
                 if (!ok) continue;
                 uint32_t op[16], od[16];
                 if (valid) {
@@ -874,8 +879,8 @@ k_bwd_dkdv_persist(const __grid_constant__ CUtensorMap tmK, const __grid_constan
 #pragma unroll
                     for (int i = 0; i < 16; ++i) { op[i] = 0u; od[i] = 0u; }
                 }
-                tmem_st16(tl + cS + 128 * b + 16 * wg, op);
-                tmem_st16(tl + cP + 128 * b + 16 * wg, od);
+                tmem_st16(tl + cS + 128 * b + 32 * wg, op);       // over this warpgroup's own S^T columns
+                tmem_st16(tl + cP + 128 * b + 32 * wg, od);
                 tmem_wait_st();
                 tc_fence_before();
                 mbar_arrive(B.elem + b);
@@ -1045,7 +1050,7 @@ prism_status_t launch_bwd(const Dims& d, const void* Qp, const void* Kp, const v
         return PRISM_ERR_CUDA;
     // persistent: one CTA per SM (all 512 TMEM columns each), items strided over the CTAs
     const int64_t gq = w.pq.items_max < device_sms() ? w.pq.items_max : device_sms();
-    kq<<<(unsigned)gq, 192, smq, s>>>((const __nv_bfloat16*)Qp, (const __nv_bfloat16*)dOp, gK, gV, tdQ, tPqh,
+    kq<<<(unsigned)gq, 320, smq, s>>>((const __nv_bfloat16*)Qp, (const __nv_bfloat16*)dOp, gK, gV, tdQ, tPqh,
                                       gsel, w.pq.hdr, w.pq.items, lse, w.delta, d.N, d.MB, (int)d.SW, nq, scale,
                                       dev_status);
     const int64_t gk = w.pkv.items_max < device_sms() ? w.pkv.items_max : device_sms();
