@@ -95,8 +95,7 @@ struct DqpLayout {
 };
 
 struct BarsP {
-    uint64_t* full0;           // [kStages]
-    uint64_t* full1;           // [kStages]
+    uint64_t* full0;           // [kStages] K and V of a granule landed (two arrivals)
     uint64_t* empty;           // [kStages]
     uint64_t* prod;            // [2]
     uint64_t* elem;            // [2]
@@ -113,7 +112,6 @@ __device__ __forceinline__ BarsP carve_p(uint8_t* ctrl) {
     uint64_t* b = reinterpret_cast<uint64_t*>(ctrl);
     BarsP r;
     r.full0 = b;
-    r.full1 = b + kStages;
     r.empty = b + 2 * kStages;
     r.prod = b + 3 * kStages;
     r.elem = b + 3 * kStages + 2;
@@ -243,8 +241,7 @@ k_bwd_dq_persist(const __nv_bfloat16* __restrict__ Qg, const __nv_bfloat16* __re
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < nst; ++s) {
-            mbar_init(B.full0 + s, 1);
-            mbar_init(B.full1 + s, 1);
+            mbar_init(B.full0 + s, 2);                 // the K and the V copy lane each arrive
             mbar_init(B.empty + s, 1);
         }
         for (int b = 0; b < 2; ++b) {
@@ -274,7 +271,7 @@ k_bwd_dq_persist(const __nv_bfloat16* __restrict__ Qg, const __nv_bfloat16* __re
         // the granules of that stage; all 32 lanes copy the selection rows
         const int kind = lane / nst, stage = lane % nst;
         const bool copier = lane < 2 * nst;
-        uint64_t* full = kind == 0 ? B.full0 : B.full1;
+        uint64_t* full = B.full0;                          // one barrier for both copies of a stage
         const CUtensorMap* mg = kind == 0 ? &tmK : &tmV;
         if (copier) tma_prefetch_desc(mg);
         bool ok = true;
@@ -352,21 +349,19 @@ k_bwd_dq_persist(const __nv_bfloat16* __restrict__ Qg, const __nv_bfloat16* __re
                     const int GG = G + g;
                     const int s = s_, b = GG & 1;
                     const uint32_t ph = (uint32_t)c_ & 1;
-                    if (!mbar_wait_w(B.full0 + s, ph, B.abort_flag, dev_status) ||
-                        !mbar_wait_w(B.full1 + s, ph, B.abort_flag, dev_status)) {
+                    if (!mbar_wait_w(B.full0 + s, ph, B.abort_flag, dev_status)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t aK = aR + s * L::STAGE, aV = aK + L::NR * kGran;
+                    const uint64_t dK = sdesc_sw128(aR + s * L::STAGE, 16, 1024);
+                    const uint64_t dV = sdesc_add(dK, L::NR * kGran);
 #pragma unroll
                     for (int k = 0; k < D / 16; ++k)
-                        mma_ts_w(tb + cS + 128 * b, tb + cQ + 8 * k, sdesc_sw128(aK + kmaj_off(k, kGran), 16, 1024),
-                                 idPS, k > 0);
+                        mma_ts_w(tb + cS + 128 * b, tb + cQ + 8 * k, sdesc_add(dK, kmaj_off(k, kGran)), idPS, k > 0);
 #pragma unroll
                     for (int k = 0; k < D / 16; ++k)
-                        mma_ts_w(tb + cP + 128 * b, tb + cdO + 8 * k, sdesc_sw128(aV + kmaj_off(k, kGran), 16, 1024),
-                                 idPS, k > 0);
+                        mma_ts_w(tb + cP + 128 * b, tb + cdO + 8 * k, sdesc_add(dV, kmaj_off(k, kGran)), idPS, k > 0);
                     tc_commit_w(B.prod + b);
                 }
                 if (g > 0) {
@@ -378,11 +373,11 @@ k_bwd_dq_persist(const __nv_bfloat16* __restrict__ Qg, const __nv_bfloat16* __re
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t aK = aR + s * L::STAGE;
+                    const uint64_t dKq = sdesc_sw128(aR + s * L::STAGE, kGran, 1024);
 #pragma unroll
                     for (int k = 0; k < 4; ++k)              // dS keys 16 k ..: warpgroup k / 2's columns
-                        mma_ts_w(tb + cdQ, tb + cS + 128 * b + 32 * (k >> 1) + 8 * (k & 1),
-                                 sdesc_sw128(aK + k * 2048, kGran, 1024), idQ, (gp > 0 || k > 0) ? 1u : 0u);
+                        mma_ts_w(tb + cdQ, tb + cS + 128 * b + 32 * (k >> 1) + 8 * (k & 1), sdesc_add(dKq, k * 2048),
+                                 idQ, (gp > 0 || k > 0) ? 1u : 0u);
                     tc_commit_w(B.empty + s);
                 }
                 if (g < ng) {
@@ -546,8 +541,7 @@ struct DkvpLayout {
 };
 
 struct BarsKV {
-    uint64_t* full0;           // [kStages] Q granule landed
-    uint64_t* full1;           // [kStages] dO granule landed
+    uint64_t* full0;           // [kStages] Q and dO of a granule landed (two arrivals)
     uint64_t* fullx;           // [kStages] row data landed
     uint64_t* empty;           // [kStages]
     uint64_t* prod;            // [2]
@@ -566,7 +560,6 @@ __device__ __forceinline__ BarsKV carve_kv(uint8_t* ctrl) {
     uint64_t* b = reinterpret_cast<uint64_t*>(ctrl);
     BarsKV r;
     r.full0 = b;
-    r.full1 = b + kStages;
     r.fullx = b + 2 * kStages;
     r.empty = b + 3 * kStages;
     r.prod = b + 4 * kStages;
@@ -608,8 +601,7 @@ k_bwd_dkdv_persist(const __grid_constant__ CUtensorMap tmK, const __grid_constan
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < nst; ++s) {
-            mbar_init(B.full0 + s, 1);
-            mbar_init(B.full1 + s, 1);
+            mbar_init(B.full0 + s, 2);                 // the Q and the dO copy lane each arrive
             mbar_init(B.fullx + s, 1);
             mbar_init(B.empty + s, 1);
         }
@@ -645,7 +637,7 @@ k_bwd_dkdv_persist(const __grid_constant__ CUtensorMap tmK, const __grid_constan
         const int kind = lane / nst, stage = lane % nst;
         const bool copier = lane < 3 * nst;
         const bool stat_lane = lane >= 30;
-        uint64_t* full = kind == 0 ? B.full0 : kind == 1 ? B.full1 : B.fullx;
+        uint64_t* full = kind < 2 ? B.full0 : B.fullx;     // Q and dO share one barrier per stage
         const CUtensorMap* mg = kind == 0 ? &tmQ : &tmdO;
         if (copier && kind < 2) tma_prefetch_desc(mg);
         bool ok = true;
@@ -728,7 +720,9 @@ k_bwd_dkdv_persist(const __grid_constant__ CUtensorMap tmK, const __grid_constan
         // ---------------------------------------------------------------- MMA (whole warp, elected issue)
         const uint32_t idPS = idesc_bf16_f32(128, 64, false, false);
         const uint32_t idKV = idesc_bf16_f32(128, D, false, true);
-        const uint32_t aK = smem_u32(sm + L::A0), aV = smem_u32(sm + L::A1), aR = smem_u32(sm + L::RING);
+        const uint32_t aR = smem_u32(sm + L::RING);
+        const uint64_t dKs = sdesc_sw128(smem_u32(sm + L::A0), 16, 1024);   // stationary K, V tiles
+        const uint64_t dVs = sdesc_sw128(smem_u32(sm + L::A1), 16, 1024);
         bool ok = true;
         int G = 0, s_ = 0, c_ = 0, kq = 0;
         for (int it = blockIdx.x; ok && it < n_items; it += gridDim.x) {
@@ -744,21 +738,21 @@ k_bwd_dkdv_persist(const __grid_constant__ CUtensorMap tmK, const __grid_constan
                     const int GG = G + g;
                     const int s = s_, b = GG & 1;
                     const uint32_t ph = (uint32_t)c_ & 1;
-                    if (!mbar_wait_w(B.full0 + s, ph, B.abort_flag, dev_status) ||
-                        !mbar_wait_w(B.full1 + s, ph, B.abort_flag, dev_status)) {
+                    if (!mbar_wait_w(B.full0 + s, ph, B.abort_flag, dev_status)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t aQ = aR + s * L::STAGE, adO = aQ + L::NR * kGran;
+                    const uint64_t dQ = sdesc_sw128(aR + s * L::STAGE, 16, 1024);
+                    const uint64_t ddO = sdesc_add(dQ, L::NR * kGran);
 #pragma unroll
                     for (int k = 0; k < D / 16; ++k)
-                        mma_ss_w(tb + cS + 128 * b, sdesc_sw128(aK + kmaj_off(k, kTile), 16, 1024),
-                                 sdesc_sw128(aQ + kmaj_off(k, kGran), 16, 1024), idPS, k > 0);
+                        mma_ss_w(tb + cS + 128 * b, sdesc_add(dKs, kmaj_off(k, kTile)), sdesc_add(dQ, kmaj_off(k, kGran)),
+                                 idPS, k > 0);
 #pragma unroll
                     for (int k = 0; k < D / 16; ++k)
-                        mma_ss_w(tb + cP + 128 * b, sdesc_sw128(aV + kmaj_off(k, kTile), 16, 1024),
-                                 sdesc_sw128(adO + kmaj_off(k, kGran), 16, 1024), idPS, k > 0);
+                        mma_ss_w(tb + cP + 128 * b, sdesc_add(dVs, kmaj_off(k, kTile)),
+                                 sdesc_add(ddO, kmaj_off(k, kGran)), idPS, k > 0);
                     tc_commit_w(B.prod + b);
                     if (g == ng - 1) tc_commit_w(B.kv_free);   // K and V no longer read by this item
                 }
@@ -771,13 +765,14 @@ k_bwd_dkdv_persist(const __grid_constant__ CUtensorMap tmK, const __grid_constan
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t aQ = aR + s * L::STAGE, adO = aQ + L::NR * kGran;
+                    const uint64_t dQn = sdesc_sw128(aR + s * L::STAGE, kGran, 1024);
+                    const uint64_t ddOn = sdesc_add(dQn, L::NR * kGran);
 #pragma unroll
                     for (int k = 0; k < 4; ++k) {            // queries 16 k ..: warpgroup k / 2's columns
                         const uint32_t acc = (gp > 0 || k > 0) ? 1u : 0u;
                         const uint32_t ck = 128 * b + 32 * (k >> 1) + 8 * (k & 1);
-                        mma_ts_w(tb + cdV, tb + cS + ck, sdesc_sw128(adO + k * 2048, kGran, 1024), idKV, acc);
-                        mma_ts_w(tb + cdK, tb + cP + ck, sdesc_sw128(aQ + k * 2048, kGran, 1024), idKV, acc);
+                        mma_ts_w(tb + cdV, tb + cS + ck, sdesc_add(ddOn, k * 2048), idKV, acc);
+                        mma_ts_w(tb + cdK, tb + cP + ck, sdesc_add(dQn, k * 2048), idKV, acc);
                     }
                     tc_commit_w(B.empty + s);
                 }

@@ -250,6 +250,11 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_byt
     return d;
 }
 
+// The descriptor of the same matrix `byte_off` bytes further on: the start
+// address field holds the address >> 4 in 14 bits, and shared-memory
+// addresses stay below 2^18, so the addition never carries out of it.
+__device__ __forceinline__ uint64_t sdesc_add(uint64_t desc, uint32_t byte_off) { return desc + (byte_off >> 4); }
+
 // Instruction descriptor of kind::f16 with bf16 A and B, fp32 accumulation.
 // a_mn / b_mn: operand stored MN-major (else K-major).
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn, bool b_mn) {
