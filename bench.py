@@ -225,20 +225,33 @@ class StepTimer:
 
 
 def run_step(mod, x, out, grads, timer=None):
+    from dynamic_block_sparse_macro_b200 import _abi
     ev = timer.ev if timer else None
     rec = (lambda i: ev[i].record()) if ev else (lambda i: None)
     rec(0)
     mod.plan(x["V"], x["hhat"])
-    mod.select(x["Q"], x["K"], x["V"])
-    rec(1)
-    mod.attend()
-    rec(2)
-    from dynamic_block_sparse_macro_b200 import _abi
-    _abi.prism_unpermute(mod.prob, mod.Op, mod.perm, out)
-    rec(3)
+    if mod.raster:                            # no blocked copies: the kernels read and write raster
+        mod.select_raster(x["Q"], x["K"])
+        rec(1)
+        mod.attend_raster(x["Q"], x["K"], x["V"], out)
+        rec(2)
+        rec(3)
+    else:
+        mod.select(x["Q"], x["K"], x["V"])
+        rec(1)
+        mod.attend()
+        rec(2)
+        _abi.prism_unpermute(mod.prob, mod.Op, mod.perm, out)
+        rec(3)
     if not mod.with_backward:                 # inference: the step ends with O
         for i in (4, 5, 6):
             rec(i)
+        return
+    if mod.raster:
+        rec(4)
+        mod.attend_backward_raster(x["Q"], x["K"], x["V"], x["dO"], *grads)
+        rec(5)
+        rec(6)
         return
     _abi.prism_permute(mod.prob, x["dO"], mod.perm, mod.dOp)
     rec(4)
@@ -290,6 +303,11 @@ def make_host_sample(mod, x):
     bs = mod.blk_start[: nb + 1].cpu().numpy().astype(np.int64)
     f = lambda t: t[:1].float().cpu().double().numpy()
     from dynamic_block_sparse_macro_b200 import _abi
+    if mod.Qp is None:                        # raster layer: gather head 0 through the permutation
+        perm = mod.perm.long()
+        g = lambda t: t[perm, :1].permute(1, 0, 2).float().cpu().double().numpy()
+        dOb = g(x["dO"]) if mod.with_backward else None
+        return {"Qb": g(x["Q"]), "Kb": g(x["K"]), "Vb": g(x["V"]), "dOb": dOb, "bs": bs, "sel": sel}
     dOb = None
     if mod.with_backward:
         _abi.prism_permute(mod.prob, x["dO"], mod.perm, mod.dOp)
@@ -312,7 +330,7 @@ def bench_prism(args, cfg, rank, world, local_rank):
     torch.cuda.reset_peak_memory_stats(dev)
     mod = PrismSparseAttention(cfg.T, cfg.H, cfg.W, cfg.heads, cfg.head_dim, cfg.audio_dim, cfg.dtype,
                                cfg.top_k, cfg.top_p if not args.dense else 1.0, device=dev,
-                               with_backward=not fwd_only)
+                               with_backward=not fwd_only, raster=bool(args.raster))
     out = torch.empty_like(x["Q"])
     grads = [] if fwd_only else [torch.empty_like(x["Q"]) for _ in range(3)]
     for _ in range(max(args.warmup, 1)):
@@ -373,7 +391,8 @@ def bench_prism(args, cfg, rank, world, local_rank):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
         "attn_ms_per_layer": round(attn_ms, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic",
-        "config": {"workload": f"prism {cfg.name} layer " + ("fwd (inference)" if fwd_only else "fwd+bwd"),
+        "config": {"workload": f"prism {cfg.name} layer " + ("fwd (inference)" if fwd_only else "fwd+bwd")
+                               + (", raster operands (no blocked copies)" if args.raster else ""),
                    "grid": [cfg.T, cfg.H, cfg.W],
                    "tokens": cfg.n_tokens, "heads": cfg.heads, "head_dim": cfg.head_dim,
                    "top_k": cfg.top_k, "top_p": 1.0 if args.dense else cfg.top_p,
@@ -501,6 +520,8 @@ def main():
     ap.add_argument("--dense", action="store_true", help="select every block (all-blocks dense run)")
     ap.add_argument("--forward-only", action="store_true",
                     help="inference: the forward stages alone, no backward buffers (value = forward TFLOP/s)")
+    ap.add_argument("--raster", action="store_true",
+                    help="the attention reads Q, K, V, dO and writes O, dQ, dK, dV in the raster layout")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)

@@ -26,7 +26,8 @@ EXPORTS = ("prism_query_sizes", "prism_zone_indicator", "prism_assign_shapes", "
            "prism_zone_indicator_noalloc", "prism_zone_indicator_ex", "prism_assign_shapes_ex",
            "prism_layer_init", "prism_layer_arena_bytes", "prism_layer_bind", "prism_layer_forward",
            "prism_layer_backward", "prism_layer_step_host", "prism_layer_sizeof",
-           "prism_zone_partials", "prism_zone_finalize")
+           "prism_zone_partials", "prism_zone_finalize", "prism_block_pool_score_raster",
+           "prism_sparse_attn_fwd_raster", "prism_sparse_attn_bwd_raster")
 GUIDANCE = {"joint": 0, "video": 1, "audio": 2}
 NOALLOC_SCRATCH_BYTES = 2 << 20
 
@@ -52,7 +53,8 @@ class LayerT(ctypes.Structure):
     _fields_ = [("prob", Problem), ("top_k", ctypes.c_int32), ("top_p", ctypes.c_float),
                 ("eps", ctypes.c_float), ("tau128", ctypes.c_float), ("tau256", ctypes.c_float),
                 ("scale", ctypes.c_float), ("guidance", ctypes.c_int32), ("fixed_shape", ctypes.c_int32),
-                ("with_backward", ctypes.c_int32), ("with_io", ctypes.c_int32), ("p_blocks", ctypes.c_int64),
+                ("with_backward", ctypes.c_int32), ("with_io", ctypes.c_int32), ("raster", ctypes.c_int32),
+                ("p_blocks", ctypes.c_int64),
                 ("g", _VP), ("rho", _VP), ("abar", _VP), ("zone_stats", _VP),
                 ("ws_ind", _VP), ("ws_ind_bytes", ctypes.c_size_t),
                 ("shape_id", _VP), ("perm", _VP), ("blk_start", _VP), ("gran_blk", _VP), ("n_blk", _VP),
@@ -104,12 +106,16 @@ _SIGS = {
     "prism_sparse_attn_bwd": [_PROB, _P, _P, _P, _P, _P, _P, _P, _P, _P, _F, _P, _P, _P, _P, _P, _SZ, _P],
     "prism_read_status": [_P, ctypes.POINTER(ctypes.c_uint32), _P],
     "prism_zone_partials": [_PROB, _P, _P, _P, _P, _SZ, _P],
+    "prism_block_pool_score_raster": [_PROB, _P, _P, _P, _P, _P, _F, _P, _P, _P, _P],
+    "prism_sparse_attn_fwd_raster": [_PROB, _P, _P, _P, _P, _P, _P, _F, _P, _P, _P, _P, _P, _SZ, _P],
+    "prism_sparse_attn_bwd_raster": [_PROB, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _F, _P, _P, _P, _P, _P, _SZ,
+                                     _P],
     "prism_zone_finalize": [_PROB, _P, _F, _I, _P, _P, _P, _P, _P, _SZ, _P],
     "prism_layer_init": [ctypes.POINTER(LayerT), _PROB],
     "prism_layer_arena_bytes": [ctypes.POINTER(LayerT), ctypes.POINTER(ctypes.c_size_t)],
     "prism_layer_bind": [ctypes.POINTER(LayerT), _P, _SZ],
     "prism_layer_forward": [ctypes.POINTER(LayerT), _P, _P, _P, _P, _P, _P],
-    "prism_layer_backward": [ctypes.POINTER(LayerT), _P, _P, _P, _P, _P],
+    "prism_layer_backward": [ctypes.POINTER(LayerT), _P, _P, _P, _P, _P, _P, _P, _P],
     "prism_layer_step_host": [ctypes.POINTER(LayerT), _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P],
 }
 
@@ -284,9 +290,9 @@ def prism_layer_forward(L: LayerT, Q, K, V, hhat, O, stream=None):
                                                             _ptr(hhat), _ptr(O), _stream(stream)))
 
 
-def prism_layer_backward(L: LayerT, dO, dQ, dK, dV, stream=None):
-    _check("prism_layer_backward", lib().prism_layer_backward(ctypes.byref(L), _ptr(dO), _ptr(dQ), _ptr(dK),
-                                                              _ptr(dV), _stream(stream)))
+def prism_layer_backward(L: LayerT, Q, K, V, dO, dQ, dK, dV, stream=None):
+    _check("prism_layer_backward", lib().prism_layer_backward(ctypes.byref(L), _ptr(Q), _ptr(K), _ptr(V), _ptr(dO),
+                                                              _ptr(dQ), _ptr(dK), _ptr(dV), _stream(stream)))
 
 
 def prism_layer_step_host(L: LayerT, hQ, hK, hV, hhhat, hdO, hO, hdQ, hdK, hdV, compute, h2d, d2h):
@@ -307,3 +313,25 @@ def prism_zone_finalize(prob, partials, eps, guidance, g, rho, abar, zone_stats,
     _check("prism_zone_finalize", lib().prism_zone_finalize(
         ctypes.byref(prob), _ptr(partials), eps, GUIDANCE.get(guidance, guidance), _ptr(g), _ptr(rho), _ptr(abar),
         _ptr(zone_stats), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+# ---------------------------------------------------------------- raster (no blocked copies)
+def prism_block_pool_score_raster(prob, Q, K, perm, blk_start, n_blk, scale, Qbar, Kbar, P, stream=None):
+    _check("prism_block_pool_score_raster", lib().prism_block_pool_score_raster(
+        ctypes.byref(prob), _ptr(Q), _ptr(K), _ptr(perm), _ptr(blk_start), _ptr(n_blk), scale, _ptr(Qbar),
+        _ptr(Kbar), _ptr(P), _stream(stream)))
+
+
+def prism_sparse_attn_fwd_raster(prob, Q, K, V, perm, shape_id, gsel, scale, O, lse, o_f32, dev_status, ws,
+                                 stream=None):
+    _check("prism_sparse_attn_fwd_raster", lib().prism_sparse_attn_fwd_raster(
+        ctypes.byref(prob), _ptr(Q), _ptr(K), _ptr(V), _ptr(perm), _ptr(shape_id), _ptr(gsel), scale, _ptr(O),
+        _ptr(lse), _ptr(o_f32), _ptr(dev_status), _ptr(ws), ws.numel() if ws is not None else 0, _stream(stream)))
+
+
+def prism_sparse_attn_bwd_raster(prob, Q, K, V, o_f32, dO, lse, perm, shape_id, gsel, gselT, scale, dQ, dK, dV,
+                                 dev_status, ws, stream=None):
+    _check("prism_sparse_attn_bwd_raster", lib().prism_sparse_attn_bwd_raster(
+        ctypes.byref(prob), _ptr(Q), _ptr(K), _ptr(V), _ptr(o_f32), _ptr(dO), _ptr(lse), _ptr(perm), _ptr(shape_id),
+        _ptr(gsel), _ptr(gselT), scale, _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(dev_status), _ptr(ws), ws.numel(),
+        _stream(stream)))

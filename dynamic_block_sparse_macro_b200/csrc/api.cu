@@ -10,11 +10,19 @@ prism_status_t attn_fwd_sm100(const Dims& d, const void* Qp, const void* Kp, con
                               float scale, void* Op, float* lse, float* o_f32, uint32_t* dev_status, void* ws,
                               cudaStream_t s);
 size_t attn_fwd_sm100_ws_bytes(const Dims& d);
+size_t attn_fwd_raster_ws_bytes(const Dims& d);
+prism_status_t attn_fwd_raster(const Dims& d, const void* Q, const void* K, const void* V, const int32_t* perm,
+                               const uint8_t* shape_id, const uint32_t* gsel, float scale, void* O, float* lse,
+                               float* o_f32, uint32_t* dev_status, void* ws, cudaStream_t s);
 prism_status_t attn_bwd_sm100(const Dims& d, const void* Qp, const void* Kp, const void* Vp, const void* Op,
                               const float* o_f32, const void* dOp, const float* lse, const uint32_t* gsel,
                               const uint32_t* gselT, float scale, void* dQp, void* dKp, void* dVp,
                               uint32_t* dev_status, void* ws, cudaStream_t s);
 size_t attn_bwd_sm100_ws_bytes(const Dims& d);
+prism_status_t attn_bwd_raster(const Dims& d, const void* Q, const void* K, const void* V, const float* o_f32,
+                               const void* dO, const float* lse, const int32_t* perm, const uint8_t* shape_id,
+                               const uint32_t* gsel, const uint32_t* gselT, float scale, void* dQ, void* dK, void* dV,
+                               uint32_t* dev_status, void* ws, cudaStream_t s);
 prism_status_t attn_fwd_simt(const Dims& d, const void* Qp, const void* Kp, const void* Vp, const uint32_t* gsel,
                              float scale, void* Op, float* lse, float* o_f32, cudaStream_t s);
 prism_status_t attn_bwd_simt(const Dims& d, const void* Qp, const void* Kp, const void* Vp, const void* Op,
@@ -25,7 +33,8 @@ prism_status_t attn_bwd_simt(const Dims& d, const void* Qp, const void* Kp, cons
 static std::atomic<unsigned long long> g_launches{0};
 void note_launches(int n) { g_launches.fetch_add((unsigned long long)n, std::memory_order_relaxed); }
 
-size_t attn_fwd_ws_bytes(const Dims& d) { return d.dtype == PRISM_BF16 ? attn_fwd_sm100_ws_bytes(d) : 0; }
+// bf16: enough for either entry point (the raster one adds the per-granule positions)
+size_t attn_fwd_ws_bytes(const Dims& d) { return d.dtype == PRISM_BF16 ? attn_fwd_raster_ws_bytes(d) : 0; }
 size_t attn_bwd_ws_bytes(const Dims& d) {
     return d.dtype == PRISM_BF16 ? attn_bwd_sm100_ws_bytes(d) : (size_t)d.heads * d.N * sizeof(float);
 }
@@ -66,6 +75,23 @@ extern "C" prism_status_t prism_sparse_attn_fwd(const prism_problem_t* prob, con
     return attn_fwd_simt(d, Qp, Kp, Vp, gsel, scale, Op, lse, o_f32, stream);
 }
 
+extern "C" prism_status_t prism_sparse_attn_fwd_raster(const prism_problem_t* prob, const void* Q, const void* K,
+                                                       const void* V, const int32_t* perm, const uint8_t* shape_id,
+                                                       const uint32_t* gsel, float scale, void* O, float* lse,
+                                                       float* o_f32, uint32_t* dev_status, void* ws, size_t ws_bytes,
+                                                       cudaStream_t stream) {
+    Dims d;
+    prism_status_t st = make_dims(prob, &d);
+    if (st != PRISM_OK) return st;
+    if (d.dtype != PRISM_BF16) return PRISM_ERR_UNSUPPORTED;
+    if (!ok_ptr(Q) || !ok_ptr(K) || !ok_ptr(V) || !ok_ptr(perm) || !ok_ptr(shape_id) || !ok_ptr(gsel) || !ok_ptr(O) ||
+        !ok_opt(lse) || !ok_opt(o_f32) || !ok_ptr(dev_status) || !ok_ptr(ws))
+        return PRISM_ERR_INVALID_ARG;
+    if (!(scale > 0.f) || !isfinite(scale)) return PRISM_ERR_INVALID_ARG;
+    if (ws_bytes < attn_fwd_raster_ws_bytes(d)) return PRISM_ERR_WORKSPACE;
+    return attn_fwd_raster(d, Q, K, V, perm, shape_id, gsel, scale, O, lse, o_f32, dev_status, ws, stream);
+}
+
 extern "C" prism_status_t prism_sparse_attn_bwd(const prism_problem_t* prob, const void* Qp, const void* Kp,
                                                 const void* Vp, const void* Op, const float* o_f32,
                                                 const void* dOp, const float* lse, const uint32_t* gsel,
@@ -85,6 +111,26 @@ extern "C" prism_status_t prism_sparse_attn_bwd(const prism_problem_t* prob, con
         return attn_bwd_sm100(d, Qp, Kp, Vp, Op, o_f32, dOp, lse, gsel, gselT, scale, dQp, dKp, dVp, dev_status, ws,
                               stream);
     return attn_bwd_simt(d, Qp, Kp, Vp, Op, o_f32, dOp, lse, gsel, gselT, scale, dQp, dKp, dVp, (float*)ws, stream);
+}
+
+extern "C" prism_status_t prism_sparse_attn_bwd_raster(const prism_problem_t* prob, const void* Q, const void* K,
+                                                       const void* V, const float* o_f32, const void* dO,
+                                                       const float* lse, const int32_t* perm, const uint8_t* shape_id,
+                                                       const uint32_t* gsel, const uint32_t* gselT, float scale,
+                                                       void* dQ, void* dK, void* dV, uint32_t* dev_status, void* ws,
+                                                       size_t ws_bytes, cudaStream_t stream) {
+    Dims d;
+    prism_status_t st = make_dims(prob, &d);
+    if (st != PRISM_OK) return st;
+    if (d.dtype != PRISM_BF16) return PRISM_ERR_UNSUPPORTED;
+    if (!ok_ptr(Q) || !ok_ptr(K) || !ok_ptr(V) || !ok_ptr(o_f32) || !ok_ptr(dO) || !ok_ptr(lse) || !ok_ptr(perm) ||
+        !ok_ptr(shape_id) || !ok_ptr(gsel) || !ok_ptr(gselT) || !ok_ptr(dQ) || !ok_ptr(dK) || !ok_ptr(dV) ||
+        !ok_ptr(dev_status) || !ok_ptr(ws))
+        return PRISM_ERR_INVALID_ARG;
+    if (!(scale > 0.f) || !isfinite(scale)) return PRISM_ERR_INVALID_ARG;
+    if (ws_bytes < attn_bwd_ws_bytes(d)) return PRISM_ERR_WORKSPACE;
+    return attn_bwd_raster(d, Q, K, V, o_f32, dO, lse, perm, shape_id, gsel, gselT, scale, dQ, dK, dV, dev_status, ws,
+                           stream);
 }
 
 extern "C" prism_status_t prism_read_status(const uint32_t* dev_status, uint32_t* host_out, cudaStream_t stream) {

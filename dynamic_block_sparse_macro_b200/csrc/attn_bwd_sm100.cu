@@ -37,7 +37,7 @@ namespace prism {
 using namespace sm100;
 
 prism_status_t bwd_delta(const Dims& d, const void* Op, const float* o_f32, const void* dOp, float* delta,
-                         const float* lse, float* nld, cudaStream_t s);
+                         const float* lse, float* nld, cudaStream_t s, const int32_t* perm);
 
 namespace {
 
@@ -77,6 +77,18 @@ __device__ __forceinline__ uint32_t kmaj_off(int k, int region) { return (k >> 2
 // The dQ columns are free for item j+1's first dQ MMA once the elementwise
 // warps have arrived on that granule's elem barrier: they do so only after the
 // epilogue of item j has read dQ.
+// Raster operands (no blocked copies): the kernels read Q, K, V, dO and write
+// dQ, dK, dV in the raster layout [N][heads][d] through the permutation, every
+// 64-row granule being one 5-D box per 64-column region (make_map_raster); the
+// fp32 partials of split tiles stay in their blocked slots.
+enum { kRK = 0, kRV = 1, kRdQ = 2, kRQ = 2, kRdO = 3, kRdK = 4, kRdV = 5 };
+template <bool RASTER, int T> using BwdRasterMaps = RasterMaps<RASTER ? T : 1>;
+struct BwdRaster {
+    const int4* gpos;          // [N/64] granule positions (gran_positions)
+    const int32_t* perm;       // [N]
+    int heads;
+};
+
 constexpr int kStagingP = 2 * kTile;       // 32 KB: two 128-byte regions of 128 rows
 
 template <int D>
@@ -135,10 +147,13 @@ static_assert((3 * kStages + 11) * 8 + 8 <= kCtrl, "barriers overflow the contro
 // it only after its previous store has finished reading shared memory.  Every
 // thread of both warpgroups runs the same barriers whatever `ok` is (passes
 // depend on `part` only).
+// With `rmaps` (raster output), the bf16 tile goes out as one box per (query
+// granule, region): granule hg's position gp[hg], head-region base hreg.
 template <int D>
 __device__ void store_tile_p(uint32_t tacc, int row, int wg, bool ok, bool zero, bool part, float mul,
                              uint8_t* stage, const CUtensorMap* map_bf16, const CUtensorMap* map_f32h, int y_bf16,
-                             int y_f32, int bar_id, int nthreads, bool leader) {
+                             int y_f32, int bar_id, int nthreads, bool leader, const CUtensorMap* rmaps = nullptr,
+                             int4 gp0 = int4{}, int4 gp1 = int4{}, int hreg = 0) {
     static_assert(D == 128 || D == 64, "head_dim");
     const int regions = part ? D / 32 : D / 64;            // 128-byte regions of a row
     const int per_pass = regions < 2 ? regions : 2;
@@ -188,8 +203,19 @@ __device__ void store_tile_p(uint32_t tacc, int row, int wg, bool ok, bool zero,
         }
         named_sync(bar_id, nthreads);
         if (ok && leader) {
-            if (part) tma_store_3d(map_f32h, stage, 0, y_f32, p * per_pass);
-            else tma_store_3d(map_bf16, stage, 0, y_bf16, 0);
+            if (part) {
+                tma_store_3d(map_f32h, stage, 0, y_f32, p * per_pass);
+            } else if (rmaps) {
+#pragma unroll
+                for (int hg = 0; hg < 2; ++hg) {
+                    const int4 gp = hg ? gp1 : gp0;
+#pragma unroll
+                    for (int r = 0; r < D / 64; ++r)
+                        tma_store_5d(rmaps + gp.w, stage + r * kTile + hg * kGran, 0, hreg + r, gp.z, gp.y, gp.x);
+                }
+            } else {
+                tma_store_3d(map_bf16, stage, 0, y_bf16, 0);
+            }
             bulk_commit();
             bulk_wait_read();
         }
@@ -216,11 +242,12 @@ __device__ __forceinline__ void load_row_tmem(uint32_t taddr, const __nv_bfloat1
     tmem_wait_st();
 }
 
-template <int D>
+template <int D, bool RASTER>
 __global__ void __launch_bounds__(320, 1)
 k_bwd_dq_persist(const __nv_bfloat16* __restrict__ Qg, const __nv_bfloat16* __restrict__ dOg,
                  const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                  const __grid_constant__ CUtensorMap tmdQ, const __grid_constant__ CUtensorMap tmPqh,
+                 const __grid_constant__ BwdRasterMaps<RASTER, 3> rmaps, BwdRaster ras,
                  const uint32_t* __restrict__ gsel, const PlanHeader* __restrict__ hdr,
                  const int4* __restrict__ items, const float* __restrict__ lse,
                  const float* __restrict__ delta, int64_t N, int64_t MB, int SW, int nst, float scale,
@@ -273,7 +300,7 @@ k_bwd_dq_persist(const __nv_bfloat16* __restrict__ Qg, const __nv_bfloat16* __re
         const bool copier = lane < 2 * nst;
         uint64_t* full = B.full0;                          // one barrier for both copies of a stage
         const CUtensorMap* mg = kind == 0 ? &tmK : &tmV;
-        if (copier) tma_prefetch_desc(mg);
+        if (copier && !RASTER) tma_prefetch_desc(mg);
         bool ok = true;
         int last_cyc = -1;                                 // ring cycle of this lane's last copy
         int st0 = 0, cyc0 = 0;                             // stage and ring cycle of the item's first granule
@@ -309,8 +336,16 @@ k_bwd_dq_persist(const __nv_bfloat16* __restrict__ Qg, const __nv_bfloat16* __re
                             break;
                         }
                         mbar_expect_tx(full + stage, L::NR * kGran);
-                        tma_load_3d(sm + stage * L::STAGE + kind * L::NR * kGran, mg, full + stage, 0,
-                                    (int)(row0 + row), 0);
+                        uint8_t* dst = sm + stage * L::STAGE + kind * L::NR * kGran;
+                        if constexpr (RASTER) {
+                            const int4 gp = ras.gpos[row >> 6];
+                            const CUtensorMap* mr = rmaps.m + (kind ? kRV : kRK) * kRasterKinds + gp.w;
+#pragma unroll
+                            for (int r = 0; r < L::NR; ++r)
+                                tma_load_5d(dst + r * kGran, mr, full + stage, 0, hh * L::NR + r, gp.z, gp.y, gp.x);
+                        } else {
+                            tma_load_3d(dst, mg, full + stage, 0, (int)(row0 + row), 0);
+                        }
                         last_cyc = c_;
                     }
                     if (++s_ == nst) { s_ = 0; ++c_; }
@@ -417,8 +452,10 @@ k_bwd_dq_persist(const __nv_bfloat16* __restrict__ Qg, const __nv_bfloat16* __re
             const int4 nx = items[itn];
             if (nx.z == nx.y) return;                      // empty: never reaches the MMA warp
             if (ok) {
-                const int64_t ngrow = (int64_t)(nx.x / tiles_per_head) * N + 128 * (nx.x % tiles_per_head) + row;
-                load_row_tmem<D>(tl + (wg ? cdO : cQ), wg ? dOg : Qg, ngrow);
+                const int nh = nx.x / tiles_per_head;
+                const int64_t nrow = 128 * (int64_t)(nx.x % tiles_per_head) + row;     // within the head
+                const int64_t src = RASTER ? (int64_t)ras.perm[nrow] * ras.heads + nh : (int64_t)nh * N + nrow;
+                load_row_tmem<D>(tl + (wg ? cdO : cQ), wg ? dOg : Qg, src);
                 tc_fence_before();
             }
             mbar_arrive(B.qdo_full);
@@ -501,8 +538,14 @@ k_bwd_dq_persist(const __nv_bfloat16* __restrict__ Qg, const __nv_bfloat16* __re
             }
             ok = fin;
             // the item's dQ (or zeros when nothing was selected: ng == 0)
-            store_tile_p<D>(tl + cdQ, row, wg, fin, ng == 0, slot >= 0, scale, staging, &tmdQ, &tmPqh,
-                            (int)(row0 + 128 * tile), slot * 128, 1, 256, warp == 2 && lane == 0);
+            if constexpr (RASTER)
+                store_tile_p<D>(tl + cdQ, row, wg, fin, ng == 0, slot >= 0, scale, staging, &tmdQ, &tmPqh,
+                                (int)(row0 + 128 * tile), slot * 128, 1, 256, warp == 2 && lane == 0,
+                                rmaps.m + kRdQ * kRasterKinds, ras.gpos[2 * tile], ras.gpos[2 * tile + 1],
+                                hh * (D / 64));
+            else
+                store_tile_p<D>(tl + cdQ, row, wg, fin, ng == 0, slot >= 0, scale, staging, &tmdQ, &tmPqh,
+                                (int)(row0 + 128 * tile), slot * 128, 1, 256, warp == 2 && lane == 0);
             G += ng;
         }
     }
@@ -576,12 +619,13 @@ __device__ __forceinline__ BarsKV carve_kv(uint8_t* ctrl) {
 }
 static_assert((4 * kStages + 12) * 8 + 8 <= kCtrl, "barriers overflow the control block");
 
-template <int D>
+template <int D, bool RASTER>
 __global__ void __launch_bounds__(384, 1)
 k_bwd_dkdv_persist(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                    const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmdO,
                    const __grid_constant__ CUtensorMap tmdK1, const __grid_constant__ CUtensorMap tmdV1,
                    const __grid_constant__ CUtensorMap tmPkv1,
+                   const __grid_constant__ BwdRasterMaps<RASTER, 6> rmaps, BwdRaster ras,
                    const uint32_t* __restrict__ gselT, const PlanHeader* __restrict__ hdr,
                    const int4* __restrict__ items, const float* __restrict__ nld,
                    int64_t N, int64_t MB, int SW, int nst, float scale, uint32_t* __restrict__ dev_status) {
@@ -639,7 +683,7 @@ k_bwd_dkdv_persist(const __grid_constant__ CUtensorMap tmK, const __grid_constan
         const bool stat_lane = lane >= 30;
         uint64_t* full = kind < 2 ? B.full0 : B.fullx;     // Q and dO share one barrier per stage
         const CUtensorMap* mg = kind == 0 ? &tmQ : &tmdO;
-        if (copier && kind < 2) tma_prefetch_desc(mg);
+        if (copier && kind < 2 && !RASTER) tma_prefetch_desc(mg);
         bool ok = true;
         int last_cyc = -1;
         int last_stat = -1;                                // index of the last stationary copy issued
@@ -667,8 +711,21 @@ k_bwd_dkdv_persist(const __grid_constant__ CUtensorMap tmK, const __grid_constan
                     if (kq >= 1) ok = mbar_wait(B.kv_free, (uint32_t)(kq - 1) & 1, B.abort_flag, dev_status);
                     if (ok) {
                         mbar_expect_tx(B.stat, L::NR * kTile);
-                        tma_load_3d(sm + (lane == 30 ? L::A0 : L::A1), lane == 30 ? &tmK : &tmV, B.stat, 0,
-                                    (int)(row0 + 128 * tile), 0);
+                        uint8_t* dst = sm + (lane == 30 ? L::A0 : L::A1);
+                        if constexpr (RASTER) {
+                            // the tile's two key granules, one box per region each
+                            const CUtensorMap* mr = rmaps.m + (lane == 30 ? kRK : kRV) * kRasterKinds;
+#pragma unroll
+                            for (int hg = 0; hg < 2; ++hg) {
+                                const int4 gp = ras.gpos[2 * tile + hg];
+#pragma unroll
+                                for (int r = 0; r < L::NR; ++r)
+                                    tma_load_5d(dst + r * kTile + hg * kGran, mr + gp.w, B.stat, 0, hh * L::NR + r,
+                                                gp.z, gp.y, gp.x);
+                            }
+                        } else {
+                            tma_load_3d(dst, lane == 30 ? &tmK : &tmV, B.stat, 0, (int)(row0 + 128 * tile), 0);
+                        }
                         last_stat = kq;
                     }
                 }
@@ -693,8 +750,17 @@ k_bwd_dkdv_persist(const __grid_constant__ CUtensorMap tmK, const __grid_constan
                             bulk_load(xs + stage * kXs, nld + ((row0 + row) >> 6) * 128, kXs, full + stage);
                         } else {
                             mbar_expect_tx(full + stage, L::NR * kGran);
-                            tma_load_3d(sm + L::RING + stage * L::STAGE + kind * L::NR * kGran, mg, full + stage, 0,
-                                        (int)(row0 + row), 0);
+                            uint8_t* dst = sm + L::RING + stage * L::STAGE + kind * L::NR * kGran;
+                            if constexpr (RASTER) {
+                                const int4 gp = ras.gpos[row >> 6];
+                                const CUtensorMap* mr = rmaps.m + (kind ? kRdO : kRQ) * kRasterKinds + gp.w;
+#pragma unroll
+                                for (int r = 0; r < L::NR; ++r)
+                                    tma_load_5d(dst + r * kGran, mr, full + stage, 0, hh * L::NR + r, gp.z, gp.y,
+                                                gp.x);
+                            } else {
+                                tma_load_3d(dst, mg, full + stage, 0, (int)(row0 + row), 0);
+                            }
                             }
                         last_cyc = c_;
                     }
@@ -938,8 +1004,18 @@ k_bwd_dkdv_persist(const __grid_constant__ CUtensorMap tmK, const __grid_constan
                     }
                     named_sync(2, 256);
                     if (ok && wg == out && (warp & 3) == 0 && lane == 0) {
-                        if (part) tma_store_3d(&tmPkv1, staging, 0, (slot * 2 + out) * 128, r);
-                        else tma_store_3d(out ? &tmdV1 : &tmdK1, staging, 0, (int)(row0 + 128 * tile), r);
+                        if (part) {
+                            tma_store_3d(&tmPkv1, staging, 0, (slot * 2 + out) * 128, r);
+                        } else if constexpr (RASTER) {
+                            const CUtensorMap* mr = rmaps.m + (out ? kRdV : kRdK) * kRasterKinds;
+#pragma unroll
+                            for (int hg = 0; hg < 2; ++hg) {
+                                const int4 gp = ras.gpos[2 * tile + hg];
+                                tma_store_5d(mr + gp.w, staging + hg * kGran, 0, hh * L::NR + r, gp.z, gp.y, gp.x);
+                            }
+                        } else {
+                            tma_store_3d(out ? &tmdV1 : &tmdK1, staging, 0, (int)(row0 + 128 * tile), r);
+                        }
                         bulk_commit();
                         bulk_wait_read();
                     }
@@ -988,6 +1064,7 @@ struct BwdWs {
     Plan pq, pkv;
     float* part_q;      // [slots][128][D]
     float* part_kv;     // [slots][2][128][D]
+    int4* gpos;         // [N/64] granule positions (raster operands only)
 };
 
 BwdWs carve_bwd(void* ws, const Dims& d, size_t* total) {
@@ -1008,29 +1085,55 @@ BwdWs carve_bwd(void* ws, const Dims& d, size_t* total) {
     p += align16(slots * 128 * d.d * 4);
     w.part_kv = reinterpret_cast<float*>(p);
     p += align16(slots * 2 * 128 * d.d * 4);
+    w.gpos = reinterpret_cast<int4*>(p);
+    p += align16(d.MB * (int64_t)sizeof(int4));
     if (total) *total = (size_t)(p - static_cast<uint8_t*>(ws));
     return w;
 }
 
-template <int D>
+// RASTER: Qp, Kp, Vp, dOp, dQp, dKp, dVp are the raster tensors; perm and
+// shape_id give every granule's box (gran_positions, into the workspace)
+template <int D, bool RASTER>
 prism_status_t launch_bwd(const Dims& d, const void* Qp, const void* Kp, const void* Vp, const void* dOp,
                           const float* lse, const uint32_t* gsel, const uint32_t* gselT, float scale, void* dQp,
-                          void* dKp, void* dVp, uint32_t* dev_status, const BwdWs& w, cudaStream_t s) {
+                          void* dKp, void* dVp, uint32_t* dev_status, const BwdWs& w, const int32_t* perm,
+                          const uint8_t* shape_id, cudaStream_t s) {
     const int64_t rows = (int64_t)d.heads * d.N;
-    CUtensorMap tK, tV, gQ, gdO, gK, gV;
-    if (!make_map_bf16_rows(&tK, Kp, rows, D, 128) || !make_map_bf16_rows(&tV, Vp, rows, D, 128) ||
-        !make_map_bf16_rows(&gQ, Qp, rows, D, 64) || !make_map_bf16_rows(&gdO, dOp, rows, D, 64) ||
-        !make_map_bf16_rows(&gK, Kp, rows, D, 64) || !make_map_bf16_rows(&gV, Vp, rows, D, 64))
-        return PRISM_ERR_CUDA;
     const int target = plan_target(device_sms());
     const int64_t slots = 2 * (int64_t)target;
-    // output maps: dQ whole rows; dK, dV and the dK/dV partials one 128-byte region a box
-    CUtensorMap tdQ, tdK1, tdV1, tPqh, tPkv1;
-    if (!make_map_bf16_rows(&tdQ, dQp, rows, D, 128) || !make_map_bf16_rows_box(&tdK1, dKp, rows, D, 128, 1) ||
-        !make_map_bf16_rows_box(&tdV1, dVp, rows, D, 128, 1) ||
-        !make_map_f32_rows_box(&tPqh, w.part_q, slots * 128, D, 128, D / 32 < 2 ? D / 32 : 2) ||
+    CUtensorMap tK, tV, gQ, gdO, gK, gV, tdQ, tdK1, tdV1, tPqh, tPkv1;
+    // fp32 partials of split tiles stay blocked (their slots) in both layouts
+    if (!make_map_f32_rows_box(&tPqh, w.part_q, slots * 128, D, 128, D / 32 < 2 ? D / 32 : 2) ||
         !make_map_f32_rows_box(&tPkv1, w.part_kv, slots * 2 * 128, D, 128, 1))
         return PRISM_ERR_CUDA;
+    BwdRasterMaps<RASTER, 3> rq;
+    BwdRasterMaps<RASTER, 6> rkv;
+    BwdRaster ras{nullptr, perm, d.heads};
+    if constexpr (RASTER) {
+        const void* bq[3] = {Kp, Vp, dQp};
+        const void* bkv[6] = {Kp, Vp, Qp, dOp, dKp, dVp};
+        for (int k = 0; k < kRasterKinds; ++k) {
+            for (int t = 0; t < 3; ++t)
+                if (!make_map_raster(&rq.m[t * kRasterKinds + k], bq[t], d.heads, D, d.T, d.H, d.W, k))
+                    return PRISM_ERR_CUDA;
+            for (int t = 0; t < 6; ++t)
+                if (!make_map_raster(&rkv.m[t * kRasterKinds + k], bkv[t], d.heads, D, d.T, d.H, d.W, k))
+                    return PRISM_ERR_CUDA;
+        }
+        if (gran_positions(perm, shape_id, d, w.gpos, s) != PRISM_OK) return PRISM_ERR_CUDA;
+        ras.gpos = w.gpos;
+        tK = tV = gQ = gdO = gK = gV = tdQ = tdK1 = tdV1 = tPqh;      // the blocked maps: never used
+    } else {
+        if (!make_map_bf16_rows(&tK, Kp, rows, D, 128) || !make_map_bf16_rows(&tV, Vp, rows, D, 128) ||
+            !make_map_bf16_rows(&gQ, Qp, rows, D, 64) || !make_map_bf16_rows(&gdO, dOp, rows, D, 64) ||
+            !make_map_bf16_rows(&gK, Kp, rows, D, 64) || !make_map_bf16_rows(&gV, Vp, rows, D, 64))
+            return PRISM_ERR_CUDA;
+        // output maps: dQ whole rows; dK, dV one 128-byte region a box
+        if (!make_map_bf16_rows(&tdQ, dQp, rows, D, 128) || !make_map_bf16_rows_box(&tdK1, dKp, rows, D, 128, 1) ||
+            !make_map_bf16_rows_box(&tdV1, dVp, rows, D, 128, 1))
+            return PRISM_ERR_CUDA;
+        rq.m[0] = rkv.m[0] = tPqh;                                      // never used
+    }
     prism_status_t st = plan_work(w.pq, gsel, d, 2, 1, target, kSegMinGranules, s);
     if (st == PRISM_OK) st = plan_work(w.pkv, gselT, d, 2, 1, target, kSegMinGranules, s);
     if (st != PRISM_OK) return st;
@@ -1038,22 +1141,23 @@ prism_status_t launch_bwd(const Dims& d, const void* Qp, const void* Kp, const v
     const int smq = DqpLayout<D>::alloc(nq, (int)d.SW);
     const int smk = DkvpLayout<D>::alloc(nk, (int)d.SW);
     if (smq > kSmemMax || smk > kSmemMax) return PRISM_ERR_UNSUPPORTED;   // selection rows too long
-    auto kq = k_bwd_dq_persist<D>;
-    auto kk = k_bwd_dkdv_persist<D>;
+    auto kq = k_bwd_dq_persist<D, RASTER>;
+    auto kk = k_bwd_dkdv_persist<D, RASTER>;
     if (cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, smq) != cudaSuccess ||
         cudaFuncSetAttribute(kk, cudaFuncAttributeMaxDynamicSharedMemorySize, smk) != cudaSuccess)
         return PRISM_ERR_CUDA;
     // persistent: one CTA per SM (all 512 TMEM columns each), items strided over the CTAs
     const int64_t gq = w.pq.items_max < device_sms() ? w.pq.items_max : device_sms();
-    kq<<<(unsigned)gq, 320, smq, s>>>((const __nv_bfloat16*)Qp, (const __nv_bfloat16*)dOp, gK, gV, tdQ, tPqh,
-                                      gsel, w.pq.hdr, w.pq.items, lse, w.delta, d.N, d.MB, (int)d.SW, nq, scale,
+    kq<<<(unsigned)gq, 320, smq, s>>>((const __nv_bfloat16*)Qp, (const __nv_bfloat16*)dOp, gK, gV, tdQ, tPqh, rq,
+                                      ras, gsel, w.pq.hdr, w.pq.items, lse, w.delta, d.N, d.MB, (int)d.SW, nq, scale,
                                       dev_status);
     const int64_t gk = w.pkv.items_max < device_sms() ? w.pkv.items_max : device_sms();
-    kk<<<(unsigned)gk, 384, smk, s>>>(tK, tV, gQ, gdO, tdK1, tdV1, tPkv1, gselT, w.pkv.hdr, w.pkv.items, w.nld, d.N,
-                                      d.MB, (int)d.SW, nk, scale, dev_status);
+    kk<<<(unsigned)gk, 384, smk, s>>>(tK, tV, gQ, gdO, tdK1, tdV1, tPkv1, rkv, ras, gselT, w.pkv.hdr, w.pkv.items,
+                                      w.nld, d.N, d.MB, (int)d.SW, nk, scale, dev_status);
     st = launch_status(2);
-    if (st == PRISM_OK) st = bwd_combine(w.pq, d, 1, w.part_q, dQp, scale, nullptr, 0.f, s);
-    if (st == PRISM_OK) st = bwd_combine(w.pkv, d, 2, w.part_kv, dKp, scale, dVp, 1.f, s);
+    const int32_t* cperm = RASTER ? perm : nullptr;
+    if (st == PRISM_OK) st = bwd_combine(w.pq, d, 1, w.part_q, dQp, scale, nullptr, 0.f, s, cperm);
+    if (st == PRISM_OK) st = bwd_combine(w.pkv, d, 2, w.part_kv, dKp, scale, dVp, 1.f, s, cperm);
     return st;
 }
 
@@ -1070,11 +1174,27 @@ prism_status_t attn_bwd_sm100(const Dims& d, const void* Qp, const void* Kp, con
                               const uint32_t* gselT, float scale, void* dQp, void* dKp, void* dVp,
                               uint32_t* dev_status, void* ws, cudaStream_t s) {
     BwdWs w = carve_bwd(ws, d, nullptr);
-    prism_status_t st = bwd_delta(d, Op, o_f32, dOp, w.delta, lse, w.nld, s);
+    prism_status_t st = bwd_delta(d, Op, o_f32, dOp, w.delta, lse, w.nld, s, nullptr);
     if (st != PRISM_OK) return st;
     if (d.d == 128)
-        return launch_bwd<128>(d, Qp, Kp, Vp, dOp, lse, gsel, gselT, scale, dQp, dKp, dVp, dev_status, w, s);
-    return launch_bwd<64>(d, Qp, Kp, Vp, dOp, lse, gsel, gselT, scale, dQp, dKp, dVp, dev_status, w, s);
+        return launch_bwd<128, false>(d, Qp, Kp, Vp, dOp, lse, gsel, gselT, scale, dQp, dKp, dVp, dev_status, w,
+                                      nullptr, nullptr, s);
+    return launch_bwd<64, false>(d, Qp, Kp, Vp, dOp, lse, gsel, gselT, scale, dQp, dKp, dVp, dev_status, w, nullptr,
+                                 nullptr, s);
+}
+
+// raster Q, K, V, dO, dQ, dK, dV ([N][heads][d]); o_f32 and lse in permutation order
+prism_status_t attn_bwd_raster(const Dims& d, const void* Q, const void* K, const void* V, const float* o_f32,
+                               const void* dO, const float* lse, const int32_t* perm, const uint8_t* shape_id,
+                               const uint32_t* gsel, const uint32_t* gselT, float scale, void* dQ, void* dK, void* dV,
+                               uint32_t* dev_status, void* ws, cudaStream_t s) {
+    BwdWs w = carve_bwd(ws, d, nullptr);
+    prism_status_t st = bwd_delta(d, nullptr, o_f32, dO, w.delta, lse, w.nld, s, perm);
+    if (st != PRISM_OK) return st;
+    if (d.d == 128)
+        return launch_bwd<128, true>(d, Q, K, V, dO, lse, gsel, gselT, scale, dQ, dK, dV, dev_status, w, perm, shape_id,
+                                     s);
+    return launch_bwd<64, true>(d, Q, K, V, dO, lse, gsel, gselT, scale, dQ, dK, dV, dev_status, w, perm, shape_id, s);
 }
 
 }  // namespace prism

@@ -105,7 +105,8 @@ __global__ void __launch_bounds__(128) k_fwd_combine(const int2* __restrict__ ti
                                                      const float* __restrict__ mpart,
                                                      const float* __restrict__ lpart,
                                                      __nv_bfloat16* __restrict__ O, float* __restrict__ o_f32,
-                                                     float* __restrict__ lse) {
+                                                     float* __restrict__ lse, const int32_t* __restrict__ perm,
+                                                     int heads) {
     const int t = blockIdx.x;
     const int2 sp = tile_split[t];
     if (sp.y <= 1) return;
@@ -125,7 +126,9 @@ __global__ void __launch_bounds__(128) k_fwd_combine(const int2* __restrict__ ti
         const float inv = L > 0.f ? 1.f / L : 0.f;
         if (threadIdx.x < D) {
             const float o = acc * inv;
-            O[(grow0 + r) * D + threadIdx.x] = __float2bfloat16_rn(o);
+            // with perm, O is raster [N][heads][D] and the row goes to its token's place
+            const int64_t orow = perm ? (int64_t)perm[(int64_t)tile_rows * tile + r] * heads + hh : grow0 + r;
+            O[orow * D + threadIdx.x] = __float2bfloat16_rn(o);
             if (o_f32) o_f32[(grow0 + r) * D + threadIdx.x] = o;
         }
         if (threadIdx.x == 0 && lse) lse[grow0 + r] = L > 0.f ? (M + log2f(L)) * 0.6931471805599453f : -INFINITY;
@@ -136,7 +139,8 @@ __global__ void __launch_bounds__(128) k_fwd_combine(const int2* __restrict__ ti
 __global__ void __launch_bounds__(256) k_bwd_combine(const int2* __restrict__ tile_split, int tiles_per_head,
                                                      int64_t N, int D, int nout, const float* __restrict__ part,
                                                      __nv_bfloat16* __restrict__ out0, float mul0,
-                                                     __nv_bfloat16* __restrict__ out1, float mul1) {
+                                                     __nv_bfloat16* __restrict__ out1, float mul1,
+                                                     const int32_t* __restrict__ perm, int heads) {
     const int t = blockIdx.x;
     const int2 sp = tile_split[t];
     if (sp.y <= 1) return;
@@ -149,7 +153,9 @@ __global__ void __launch_bounds__(256) k_bwd_combine(const int2* __restrict__ ti
         for (int e = threadIdx.x; e < per; e += blockDim.x) {
             float acc = 0.f;
             for (int s = 0; s < sp.y; ++s) acc += part[((int64_t)(sp.x + s) * nout + k) * per + e];
-            out[grow0 * D + e] = __float2bfloat16_rn(acc * mul);
+            // with perm, the outputs are raster [N][heads][D]: row r goes to its token's place
+            const int64_t orow = perm ? (int64_t)perm[128 * (int64_t)tile + e / D] * heads + hh : grow0 + e / D;
+            out[orow * D + e % D] = __float2bfloat16_rn(acc * mul);
         }
     }
 }
@@ -185,17 +191,38 @@ prism_status_t plan_work(const Plan& pl, const uint32_t* rows, const Dims& d, in
     return launch_status(2);
 }
 
+__global__ void __launch_bounds__(256) k_gran_pos(const int32_t* __restrict__ perm,
+                                                  const uint8_t* __restrict__ shape_id, int64_t MB, int H, int W,
+                                                  int4* __restrict__ gpos) {
+    const int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (g >= MB) return;
+    const int r0 = perm[64 * g];
+    const int t0 = r0 / (H * W), h0 = (r0 / W) % H, w0 = r0 % W;
+    const int zone = ((t0 >> 3) * (H >> 3) + (h0 >> 3)) * (W >> 3) + (w0 >> 3);
+    int eT, eH, eW;
+    shape_exponents(shape_id[zone], &eT, &eH, &eW);
+    gpos[g] = make_int4(t0, h0, w0, 3 * (eH - 1) + (eW - 1));
+}
+
+prism_status_t gran_positions(const int32_t* perm, const uint8_t* shape_id, const Dims& d, int4* gpos,
+                              cudaStream_t s) {
+    k_gran_pos<<<(unsigned)((d.MB + 255) / 256), 256, 0, s>>>(perm, shape_id, d.MB, d.H, d.W, gpos);
+    return launch_status(1);
+}
+
 prism_status_t fwd_combine(const Plan& pl, const Dims& d, int tile_rows, const float* opart, const float* mpart,
-                           const float* lpart, void* Op, float* o_f32, float* lse, cudaStream_t s) {
+                           const float* lpart, void* Op, float* o_f32, float* lse, const int32_t* perm, cudaStream_t s) {
     k_fwd_combine<<<(unsigned)pl.tiles, 128, 0, s>>>(pl.tile_split, (int)(d.N / tile_rows), tile_rows, d.N, d.d,
-                                                     opart, mpart, lpart, (__nv_bfloat16*)Op, o_f32, lse);
+                                                     opart, mpart, lpart, (__nv_bfloat16*)Op, o_f32, lse, perm,
+                                                     d.heads);
     return launch_status(1);
 }
 
 prism_status_t bwd_combine(const Plan& pl, const Dims& d, int nout, const float* part, void* out0, float mul0,
-                           void* out1, float mul1, cudaStream_t s) {
+                           void* out1, float mul1, cudaStream_t s, const int32_t* perm) {
     k_bwd_combine<<<(unsigned)pl.tiles, 256, 0, s>>>(pl.tile_split, (int)(d.N / 128), d.N, d.d, nout, part,
-                                                     (__nv_bfloat16*)out0, mul0, (__nv_bfloat16*)out1, mul1);
+                                                     (__nv_bfloat16*)out0, mul0, (__nv_bfloat16*)out1, mul1, perm,
+                                                     d.heads);
     return launch_status(1);
 }
 

@@ -38,9 +38,16 @@ Plan carve_plan(void* base, int64_t tiles, int target);
 prism_status_t plan_work(const Plan& pl, const uint32_t* rows, const Dims& d, int tile_gran, int unit_granules,
                          int target, int seg_min, cudaStream_t s);
 prism_status_t fwd_combine(const Plan& pl, const Dims& d, int tile_rows, const float* opart, const float* mpart,
-                           const float* lpart, void* Op, float* o_f32, float* lse, cudaStream_t s);
+                           const float* lpart, void* Op, float* o_f32, float* lse, const int32_t* perm,
+                           cudaStream_t s);
+// perm != nullptr: the outputs are raster [N][heads][d] (rows scattered through it)
 prism_status_t bwd_combine(const Plan& pl, const Dims& d, int nout, const float* part, void* out0, float mul0,
-                           void* out1, float mul1, cudaStream_t s);
+                           void* out1, float mul1, cudaStream_t s, const int32_t* perm = nullptr);
+
+// per 64-row granule g of the blocked order: (t0, h0, w0, box kind) of its first
+// token perm[64 g] (the raster maps' coordinates; see make_map_raster)
+prism_status_t gran_positions(const int32_t* perm, const uint8_t* shape_id, const Dims& d, int4* gpos,
+                              cudaStream_t s);
 
 // number of SMs of the current device (cached per device ordinal; the plan
 // target and the workspace sizes depend on it)

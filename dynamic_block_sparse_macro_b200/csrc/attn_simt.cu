@@ -155,14 +155,17 @@ template <> __device__ __forceinline__ float4 load4<__nv_bfloat16>(const __nv_bf
 template <typename T, int D>
 __global__ void k_bwd_delta(const T* __restrict__ O, const float* __restrict__ o_f32,
                             const T* __restrict__ dO, int64_t rows, float* __restrict__ delta,
-                            const float* __restrict__ lse, float* __restrict__ nld) {
+                            const float* __restrict__ lse, float* __restrict__ nld,
+                            const int32_t* __restrict__ perm = nullptr, int64_t N = 0, int heads = 0) {
     constexpr int LPR = D / 4;                                // lanes per row
     const int64_t gl = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     const int64_t r = gl / LPR;
     const int c = (int)(gl % LPR) * 4;
     float s = 0.f;
     if (r < rows) {
-        const float4 g = load4<T>(dO + r * D + c);
+        // with perm, dO is raster [N][heads][D]: blocked row r of head r / N is token perm[r % N]
+        const int64_t dr = perm ? (int64_t)perm[r % N] * heads + r / N : r;
+        const float4 g = load4<T>(dO + dr * D + c);
         const float4 o = o_f32 ? __ldg(reinterpret_cast<const float4*>(o_f32 + r * D + c)) : load4<T>(O + r * D + c);
         s = o.x * g.x + o.y * g.y + o.z * g.z + o.w * g.w;
     }
@@ -416,17 +419,20 @@ prism_status_t attn_fwd_simt(const Dims& d, const void* Qp, const void* Kp, cons
 }
 
 // Delta = rowsum(dO * O) for every blocked row (shared by both backward families)
+// (perm != nullptr: dO raster, read through the permutation; O then comes from o_f32)
 prism_status_t bwd_delta(const Dims& d, const void* Op, const float* o_f32, const void* dOp, float* delta,
-                         const float* lse, float* nld, cudaStream_t s) {
+                         const float* lse, float* nld, cudaStream_t s, const int32_t* perm) {
     const int64_t rows = (int64_t)d.heads * d.N;
     const unsigned grid = (unsigned)((rows * (d.d / 4) + 255) / 256);
+    const int64_t N = d.N;
+    const int h = d.heads;
     if (d.dtype == PRISM_F32) {
-        if (d.d == 64) k_bwd_delta<float, 64><<<grid, 256, 0, s>>>((const float*)Op, o_f32, (const float*)dOp, rows, delta, lse, nld);
-        else k_bwd_delta<float, 128><<<grid, 256, 0, s>>>((const float*)Op, o_f32, (const float*)dOp, rows, delta, lse, nld);
+        if (d.d == 64) k_bwd_delta<float, 64><<<grid, 256, 0, s>>>((const float*)Op, o_f32, (const float*)dOp, rows, delta, lse, nld, perm, N, h);
+        else k_bwd_delta<float, 128><<<grid, 256, 0, s>>>((const float*)Op, o_f32, (const float*)dOp, rows, delta, lse, nld, perm, N, h);
     } else {
         using B = __nv_bfloat16;
-        if (d.d == 64) k_bwd_delta<B, 64><<<grid, 256, 0, s>>>((const B*)Op, o_f32, (const B*)dOp, rows, delta, lse, nld);
-        else k_bwd_delta<B, 128><<<grid, 256, 0, s>>>((const B*)Op, o_f32, (const B*)dOp, rows, delta, lse, nld);
+        if (d.d == 64) k_bwd_delta<B, 64><<<grid, 256, 0, s>>>((const B*)Op, o_f32, (const B*)dOp, rows, delta, lse, nld, perm, N, h);
+        else k_bwd_delta<B, 128><<<grid, 256, 0, s>>>((const B*)Op, o_f32, (const B*)dOp, rows, delta, lse, nld, perm, N, h);
     }
     return launch_status(1);
 }

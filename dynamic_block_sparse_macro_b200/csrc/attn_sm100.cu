@@ -66,11 +66,22 @@ struct FwdParts {
     float* l;       // [slots][128] denominator
 };
 
-template <int D>
+// ------------------------------------------------------------------ raster (unpermuted) operands
+enum { kMapQ = 0, kMapK = 1, kMapV = 2, kMapO = 3, kRasterMaps = 4 };
+
+// one map, unused, in the blocked-layout kernel
+template <bool RASTER>
+using FwdRasterMaps = RasterMaps<RASTER ? kRasterMaps : 1>;
+struct RasterOps {
+    const int4* gpos;           // [N/64] per-granule raster positions (gran_positions)
+};
+
+template <int D, bool RASTER>
 __global__ void __launch_bounds__(192, 2)
 k_attn_fwd_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
                  const __grid_constant__ CUtensorMap tmOf, const __grid_constant__ CUtensorMap tmPo,
+                 const __grid_constant__ FwdRasterMaps<RASTER> rmaps, RasterOps ras,
                  const uint32_t* __restrict__ gsel,
                  const PlanHeader* __restrict__ hdr, const int4* __restrict__ items, FwdParts parts,
                  int64_t N, int64_t MB, int SW, float scale, __nv_bfloat16* __restrict__ O,
@@ -140,11 +151,19 @@ k_attn_fwd_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             uint64_t* bfull = tensor ? bar_vf : bar_kf;
             uint64_t* bempty = tensor ? bar_ve : bar_ke;
             uint8_t* buf = tensor ? sV : sK;
-            tma_prefetch_desc(mt);
+            if constexpr (!RASTER) tma_prefetch_desc(mt);
             if (tensor == 0) {
-                tma_prefetch_desc(&tmQ);
                 mbar_expect_tx(bar_q, kRegion);
-                tma_load_2d(sQ + r * kRegion, &tmQ, bar_q, 64 * r, (int)(row0 + 128 * tile));
+                if constexpr (RASTER) {
+                    for (int hg = 0; hg < 2; ++hg) {             // the tile's two query granules
+                        const int4 gp = ras.gpos[2 * tile + hg];
+                        tma_load_5d(sQ + r * kRegion + hg * kGranBytes, rmaps.m + kMapQ * kRasterKinds + gp.w, bar_q,
+                                    0, hh * L::NR + r, gp.z, gp.y, gp.x);
+                    }
+                } else {
+                    tma_prefetch_desc(&tmQ);
+                    tma_load_2d(sQ + r * kRegion, &tmQ, bar_q, 64 * r, (int)(row0 + 128 * tile));
+                }
             }
             GranuleWalk walk;
             walk.init(u0, u1, wn);
@@ -157,8 +176,15 @@ k_attn_fwd_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                 if (!walk.next(rb, mb)) rb = ra;
                 if (c > 0 && !mbar_wait(bempty, (c - 1) & 1, abort_flag, dev_status)) break;
                 mbar_expect_tx(bfull, 2 * kGranBytes);
-                tma_load_2d(buf + r * kRegion, mt, bfull, 64 * r, (int)(row0 + ra));
-                tma_load_2d(buf + r * kRegion + kGranBytes, mt, bfull, 64 * r, (int)(row0 + rb));
+                if constexpr (RASTER) {
+                    const CUtensorMap* mk = rmaps.m + (tensor ? kMapV : kMapK) * kRasterKinds;
+                    const int4 pa = ras.gpos[ra >> 6], pb = ras.gpos[rb >> 6];
+                    tma_load_5d(buf + r * kRegion, mk + pa.w, bfull, 0, hh * L::NR + r, pa.z, pa.y, pa.x);
+                    tma_load_5d(buf + r * kRegion + kGranBytes, mk + pb.w, bfull, 0, hh * L::NR + r, pb.z, pb.y, pb.x);
+                } else {
+                    tma_load_2d(buf + r * kRegion, mt, bfull, 64 * r, (int)(row0 + ra));
+                    tma_load_2d(buf + r * kRegion + kGranBytes, mt, bfull, 64 * r, (int)(row0 + rb));
+                }
                 ++issued;
             }
             if (*abort_flag && issued) {
@@ -362,15 +388,37 @@ k_attn_fwd_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             }
         }
         named_sync(1, 128);
-        if (fin && warp == 2 && lane == 0) {
-            if (!part) {
-                tma_store_3d(&tmO, sQ, 0, (int)(row0 + 128 * tile), 0);
-                if (o_f32) tma_store_3d(&tmOf, sK, 0, (int)(row0 + 128 * tile), 0);
-            } else {
-                tma_store_3d(&tmPo, sK, 0, slot * 128, 0);
+        if constexpr (RASTER) {
+            // O back to the raster layout: one box per (query granule, region), a lane each;
+            // the fp32 O (kept in permutation order) and the partials as whole-row tiles
+            if (fin && warp == 2) {
+                bool issued = false;
+                if (!part && lane < 2 * L::NR) {
+                    const int hg = lane / L::NR, r = lane % L::NR;
+                    const int4 gp = ras.gpos[2 * tile + hg];
+                    tma_store_5d(rmaps.m + kMapO * kRasterKinds + gp.w, sQ + r * kRegion + hg * kGranBytes, 0,
+                                 hh * L::NR + r, gp.z, gp.y, gp.x);
+                    issued = true;
+                } else if (lane == 31) {
+                    if (!part && o_f32) { tma_store_3d(&tmOf, sK, 0, (int)(row0 + 128 * tile), 0); issued = true; }
+                    if (part) { tma_store_3d(&tmPo, sK, 0, slot * 128, 0); issued = true; }
+                }
+                if (issued) {
+                    bulk_commit();
+                    bulk_wait_read();
+                }
             }
-            bulk_commit();
-            bulk_wait_read();                               // shared memory stays valid until read
+        } else {
+            if (fin && warp == 2 && lane == 0) {
+                if (!part) {
+                    tma_store_3d(&tmO, sQ, 0, (int)(row0 + 128 * tile), 0);
+                    if (o_f32) tma_store_3d(&tmOf, sK, 0, (int)(row0 + 128 * tile), 0);
+                } else {
+                    tma_store_3d(&tmPo, sK, 0, slot * 128, 0);
+                }
+                bulk_commit();
+                bulk_wait_read();                           // shared memory stays valid until read
+            }
         }
     }
 
@@ -408,46 +456,77 @@ FwdWs carve_fwd(void* ws, const Dims& d) {
     return w;
 }
 
-template <int D>
-prism_status_t launch_fwd(const Dims& d, const void* Qp, const void* Kp, const void* Vp, const uint32_t* gsel,
-                          float scale, void* Op, float* lse, float* o_f32, uint32_t* dev_status, void* ws,
-                          cudaStream_t s) {
+// Raster operands: the workspace also holds the per-granule positions after the
+// blocked-layout workspace.
+size_t fwd_raster_extra_bytes(const Dims& d) { return align16(d.MB * (int64_t)sizeof(int4)); }
+
+template <int D, bool RASTER>
+prism_status_t launch_fwd(const Dims& d, const void* Qp, const void* Kp, const void* Vp, const int32_t* perm,
+                          const uint8_t* shape_id, const uint32_t* gsel, float scale, void* Op, float* lse,
+                          float* o_f32, uint32_t* dev_status, void* ws, cudaStream_t s) {
     CUtensorMap mQ, mK, mV, mO, mOf, mPo;
     const int64_t rows = (int64_t)d.heads * d.N;
-    if (!make_map_bf16(&mQ, Qp, rows, D, 128) || !make_map_bf16(&mK, Kp, rows, D, 64) ||
-        !make_map_bf16(&mV, Vp, rows, D, 64))
-        return PRISM_ERR_CUDA;
     FwdWs w = carve_fwd(ws, d);
     const int64_t slots = 2 * (int64_t)plan_target(device_sms());
-    // output maps: whole 128-row tiles (the fp32 O map is only built, and used, when o_f32 is given)
-    if (!make_map_bf16_rows(&mO, Op, rows, D, 128) || !make_map_f32_rows(&mPo, w.parts.o, slots * 128, D, 128) ||
+    // fp32 outputs stay in permutation order: whole 128-row tiles (the fp32 O map only when o_f32 is given)
+    if (!make_map_f32_rows(&mPo, w.parts.o, slots * 128, D, 128) ||
         (o_f32 && !make_map_f32_rows(&mOf, o_f32, rows, D, 128)))
         return PRISM_ERR_CUDA;
     if (!o_f32) mOf = mPo;                              // never used
+    FwdRasterMaps<RASTER> rm;
+    RasterOps ras{nullptr};
+    if constexpr (RASTER) {
+        const void* bases[kRasterMaps] = {Qp, Kp, Vp, Op};
+        for (int t = 0; t < kRasterMaps; ++t)
+            for (int k = 0; k < kRasterKinds; ++k)
+                if (!make_map_raster(&rm.m[t * kRasterKinds + k], bases[t], d.heads, D, d.T, d.H, d.W, k))
+                    return PRISM_ERR_CUDA;
+        int4* gpos = reinterpret_cast<int4*>(static_cast<uint8_t*>(ws) + fwd_ws_bytes_d(d));
+        if (gran_positions(perm, shape_id, d, gpos, s) != PRISM_OK) return PRISM_ERR_CUDA;
+        ras.gpos = gpos;
+        mQ = mK = mV = mO = mPo;                        // never used
+    } else {
+        if (!make_map_bf16(&mQ, Qp, rows, D, 128) || !make_map_bf16(&mK, Kp, rows, D, 64) ||
+            !make_map_bf16(&mV, Vp, rows, D, 64) || !make_map_bf16_rows(&mO, Op, rows, D, 128))
+            return PRISM_ERR_CUDA;
+        rm.m[0] = mPo;                                  // never used
+    }
     const int target = plan_target(device_sms());
     prism_status_t st = plan_work(w.plan, gsel, d, 2, 2, target, kSegMinChunks, s);
     if (st != PRISM_OK) return st;
-    auto k = k_attn_fwd_sm100<D>;
+    auto k = k_attn_fwd_sm100<D, RASTER>;
     const int smem = FwdLayout<D>::alloc((int)d.SW);
     if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return PRISM_ERR_CUDA;
-    k<<<(unsigned)w.plan.items_max, 192, smem, s>>>(mQ, mK, mV, mO, mOf, mPo, gsel, w.plan.hdr, w.plan.items, w.parts,
-                                                    d.N, d.MB,
-                                                    (int)d.SW, scale, (__nv_bfloat16*)Op, lse, o_f32, dev_status);
+    k<<<(unsigned)w.plan.items_max, 192, smem, s>>>(mQ, mK, mV, mO, mOf, mPo, rm, ras, gsel, w.plan.hdr, w.plan.items,
+                                                    w.parts, d.N, d.MB, (int)d.SW, scale, (__nv_bfloat16*)Op, lse,
+                                                    o_f32, dev_status);
     st = launch_status(1);
     if (st != PRISM_OK) return st;
-    return fwd_combine(w.plan, d, 128, w.parts.o, w.parts.m, w.parts.l, Op, o_f32, lse, s);
+    return fwd_combine(w.plan, d, 128, w.parts.o, w.parts.m, w.parts.l, Op, o_f32, lse, RASTER ? perm : nullptr, s);
 }
 
 }  // namespace
 
 size_t attn_fwd_sm100_ws_bytes(const Dims& d) { return fwd_ws_bytes_d(d); }
+size_t attn_fwd_raster_ws_bytes(const Dims& d) { return fwd_ws_bytes_d(d) + fwd_raster_extra_bytes(d); }
 
 prism_status_t attn_fwd_sm100(const Dims& d, const void* Qp, const void* Kp, const void* Vp, const uint32_t* gsel,
                               float scale, void* Op, float* lse, float* o_f32, uint32_t* dev_status, void* ws,
                               cudaStream_t s) {
-    if (d.d == 128) return launch_fwd<128>(d, Qp, Kp, Vp, gsel, scale, Op, lse, o_f32, dev_status, ws, s);
-    return launch_fwd<64>(d, Qp, Kp, Vp, gsel, scale, Op, lse, o_f32, dev_status, ws, s);
+    if (d.d == 128)
+        return launch_fwd<128, false>(d, Qp, Kp, Vp, nullptr, nullptr, gsel, scale, Op, lse, o_f32, dev_status, ws, s);
+    return launch_fwd<64, false>(d, Qp, Kp, Vp, nullptr, nullptr, gsel, scale, Op, lse, o_f32, dev_status, ws, s);
+}
+
+// raster Q, K, V, O ([N][heads][d]); perm and shape_id from prism_assign_shapes; lse and
+// o_f32 (nullable) stay in permutation order
+prism_status_t attn_fwd_raster(const Dims& d, const void* Q, const void* K, const void* V, const int32_t* perm,
+                               const uint8_t* shape_id, const uint32_t* gsel, float scale, void* O, float* lse,
+                               float* o_f32, uint32_t* dev_status, void* ws, cudaStream_t s) {
+    if (d.d == 128)
+        return launch_fwd<128, true>(d, Q, K, V, perm, shape_id, gsel, scale, O, lse, o_f32, dev_status, ws, s);
+    return launch_fwd<64, true>(d, Q, K, V, perm, shape_id, gsel, scale, O, lse, o_f32, dev_status, ws, s);
 }
 
 }  // namespace prism

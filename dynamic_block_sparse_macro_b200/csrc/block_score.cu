@@ -17,12 +17,15 @@
 
 namespace prism {
 
+// perm == nullptr: Qp, Kp blocked [heads][N][d]; otherwise raster [N][heads][d],
+// row r of the block order read at token perm[r]
 template <typename T>
 __global__ void __launch_bounds__(256) k_block_pool(const T* __restrict__ Qp, const T* __restrict__ Kp,
                                                     const int32_t* __restrict__ blk_start,
                                                     const int32_t* __restrict__ n_blk, int64_t N,
                                                     int64_t MB, int d, float* __restrict__ Qbar,
-                                                    float* __restrict__ Kbar) {
+                                                    float* __restrict__ Kbar, const int32_t* __restrict__ perm,
+                                                    int heads) {
     constexpr int VE = 16 / sizeof(T);
     __shared__ float red[256 * VE];
     const int j = blockIdx.x, hh = blockIdx.y, which = blockIdx.z;
@@ -32,14 +35,16 @@ __global__ void __launch_bounds__(256) k_block_pool(const T* __restrict__ Qp, co
         for (int c = threadIdx.x; c < d; c += blockDim.x) out[c] = 0.f;
         return;
     }
-    const T* src = (which ? Kp : Qp) + (int64_t)hh * N * d;
+    const T* base = which ? Kp : Qp;
+    const T* src = perm ? base : base + (int64_t)hh * N * d;
     const int s = blk_start[j], e = blk_start[j + 1];
     const int lpr = d / VE, rg = threadIdx.x / lpr, v = threadIdx.x % lpr, RG = blockDim.x / lpr;
     float acc[VE];
 #pragma unroll
     for (int k = 0; k < VE; ++k) acc[k] = 0.f;
     for (int r = s + rg; r < e; r += RG) {
-        const int4 raw = __ldg(reinterpret_cast<const int4*>(src + (int64_t)r * d) + v);
+        const int64_t row = perm ? (int64_t)__ldg(perm + r) * heads + hh : (int64_t)r;
+        const int4 raw = __ldg(reinterpret_cast<const int4*>(src + row * d) + v);
         const T* x = reinterpret_cast<const T*>(&raw);
 #pragma unroll
         for (int k = 0; k < VE; ++k) acc[k] += to_f32(x[k]);
@@ -133,10 +138,9 @@ __global__ void __launch_bounds__(256) k_row_softmax(float* __restrict__ P,
 
 using namespace prism;
 
-extern "C" prism_status_t prism_block_pool_score(const prism_problem_t* prob, const void* Qp,
-                                                 const void* Kp, const int32_t* blk_start,
-                                                 const int32_t* n_blk, float scale, float* Qbar,
-                                                 float* Kbar, float* P, cudaStream_t stream) {
+static prism_status_t pool_score(const prism_problem_t* prob, const void* Qp, const void* Kp,
+                                 const int32_t* perm, const int32_t* blk_start, const int32_t* n_blk, float scale,
+                                 float* Qbar, float* Kbar, float* P, cudaStream_t stream) {
     Dims d;
     prism_status_t st = make_dims(prob, &d);
     if (st != PRISM_OK) return st;
@@ -148,13 +152,29 @@ extern "C" prism_status_t prism_block_pool_score(const prism_problem_t* prob, co
     if (d.dtype == PRISM_BF16)
         k_block_pool<__nv_bfloat16><<<gp, 256, 0, stream>>>((const __nv_bfloat16*)Qp,
                                                             (const __nv_bfloat16*)Kp, blk_start,
-                                                            n_blk, d.N, d.MB, d.d, Qbar, Kbar);
+                                                            n_blk, d.N, d.MB, d.d, Qbar, Kbar, perm, d.heads);
     else
         k_block_pool<float><<<gp, 256, 0, stream>>>((const float*)Qp, (const float*)Kp, blk_start,
-                                                    n_blk, d.N, d.MB, d.d, Qbar, Kbar);
+                                                    n_blk, d.N, d.MB, d.d, Qbar, Kbar, perm, d.heads);
     const unsigned tiles = (unsigned)((d.MB + 63) / 64);
     k_block_score<<<dim3(tiles, tiles, (unsigned)d.heads), 256, 0, stream>>>(Qbar, Kbar, n_blk, d.MB,
                                                                              d.d, scale, P);
     k_row_softmax<<<dim3((unsigned)d.MB, (unsigned)d.heads), 256, 0, stream>>>(P, n_blk);
     return launch_status(3);
+}
+
+extern "C" prism_status_t prism_block_pool_score(const prism_problem_t* prob, const void* Qp,
+                                                 const void* Kp, const int32_t* blk_start,
+                                                 const int32_t* n_blk, float scale, float* Qbar,
+                                                 float* Kbar, float* P, cudaStream_t stream) {
+    return pool_score(prob, Qp, Kp, nullptr, blk_start, n_blk, scale, Qbar, Kbar, P, stream);
+}
+
+// Stage 4 from raster Q, K ([N][heads][d]) through the permutation
+extern "C" prism_status_t prism_block_pool_score_raster(const prism_problem_t* prob, const void* Q, const void* K,
+                                                        const int32_t* perm, const int32_t* blk_start,
+                                                        const int32_t* n_blk, float scale, float* Qbar, float* Kbar,
+                                                        float* P, cudaStream_t stream) {
+    if (!ok_ptr(perm)) return PRISM_ERR_INVALID_ARG;
+    return pool_score(prob, Q, K, perm, blk_start, n_blk, scale, Qbar, Kbar, P, stream);
 }

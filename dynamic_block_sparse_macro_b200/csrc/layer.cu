@@ -33,6 +33,7 @@ size_t carve(prism_layer_t* L, uint8_t* base) {
     const size_t esz = L->prob.dtype == PRISM_BF16 ? 2 : 4;
     const int64_t pb = L->p_blocks > 0 ? L->p_blocks : MB;
     const bool bwd = L->with_backward != 0, io = L->with_io != 0;
+    const bool blocked = !L->raster;                          // raster: no blocked Q, K, V, O
     size_t off = 0;
     auto take = [&](size_t bytes) -> void* {
         void* p = base ? base + off : nullptr;
@@ -52,9 +53,9 @@ size_t carve(prism_layer_t* L, uint8_t* base) {
     L->gran_blk = (int32_t*)take(MB * 4);
     L->n_blk = (int32_t*)take(4);
     L->margin_shape = (float*)take(Z * 2 * 4);
-    L->Qp = take(tok);
-    L->Kp = take(tok);
-    L->Vp = take(tok);
+    L->Qp = blocked ? take(tok) : nullptr;
+    L->Kp = blocked ? take(tok) : nullptr;
+    L->Vp = blocked ? take(tok) : nullptr;
     L->Qbar = (float*)take(h * MB * d * 4);
     L->Kbar = (float*)take(h * MB * d * 4);
     L->P = (float*)take((size_t)h * pb * pb * 4);
@@ -64,15 +65,15 @@ size_t carve(prism_layer_t* L, uint8_t* base) {
     L->sel_count = (int32_t*)take(h * MB * 4);
     L->margin_sel = (float*)take(h * MB * 4);
     L->dev_status = (uint32_t*)take(4);
-    L->Op = take(tok);
+    L->Op = blocked ? take(tok) : nullptr;
     L->Of32 = (bwd && L->prob.dtype == PRISM_BF16) ? (float*)take((size_t)N * h * d * 4) : nullptr;
     L->lse = bwd ? (float*)take(N * h * 4) : nullptr;
     L->ws_fwd_bytes = s.ws_attn_fwd;
     L->ws_fwd = take(s.ws_attn_fwd);
-    L->dOp = bwd ? take(tok) : nullptr;
-    L->dQp = bwd ? take(tok) : nullptr;
-    L->dKp = bwd ? take(tok) : nullptr;
-    L->dVp = bwd ? take(tok) : nullptr;
+    L->dOp = (bwd && blocked) ? take(tok) : nullptr;
+    L->dQp = (bwd && blocked) ? take(tok) : nullptr;
+    L->dKp = (bwd && blocked) ? take(tok) : nullptr;
+    L->dVp = (bwd && blocked) ? take(tok) : nullptr;
     L->ws_bwd_bytes = bwd ? s.ws_attn_bwd : 0;
     L->ws_bwd = bwd ? take(s.ws_attn_bwd) : nullptr;
     const size_t hh_bytes = (size_t)N * L->prob.audio_dim * esz;
@@ -91,7 +92,7 @@ size_t carve(prism_layer_t* L, uint8_t* base) {
 bool params_ok(const prism_layer_t* L) {
     return L->top_k >= 0 && L->top_p > 0.f && isfinite(L->top_p) && L->eps > 0.f && isfinite(L->eps) &&
            L->scale > 0.f && isfinite(L->scale) && L->fixed_shape >= -1 && L->fixed_shape < 16 &&
-           L->p_blocks >= 0;
+           L->p_blocks >= 0 && (L->raster == 0 || (L->raster == 1 && L->prob.dtype == PRISM_BF16));
 }
 
 #define PRISM_TRY(x)                          \
@@ -107,6 +108,17 @@ prism_status_t run_forward(const prism_layer_t* L, const void* Q, const void* K,
                                       L->ws_ind, L->ws_ind_bytes, s));
     PRISM_TRY(prism_assign_shapes_ex(p, L->g, L->rho, L->tau128, L->tau256, L->fixed_shape, L->shape_id, L->perm,
                                      nullptr, L->blk_start, L->gran_blk, L->n_blk, L->margin_shape, s));
+    if (L->raster) {
+        // the permutation is applied inside the loads and stores: no blocked copies
+        if (qk_ready && cudaStreamWaitEvent(s, qk_ready, 0) != cudaSuccess) return PRISM_ERR_CUDA;
+        PRISM_TRY(prism_block_pool_score_raster(p, Q, K, L->perm, L->blk_start, L->n_blk, L->scale, L->Qbar, L->Kbar,
+                                                L->P, s));
+        PRISM_TRY(prism_block_select(p, L->P, L->blk_start, L->gran_blk, L->n_blk, L->top_k, L->top_p, L->sel,
+                                     L->sel_count, L->gsel, L->gselT, L->margin_sel, L->dev_status, s));
+        if (out_free && cudaStreamWaitEvent(s, out_free, 0) != cudaSuccess) return PRISM_ERR_CUDA;
+        return prism_sparse_attn_fwd_raster(p, Q, K, V, L->perm, L->shape_id, L->gsel, L->scale, O, L->lse, L->Of32,
+                                            L->dev_status, L->ws_fwd, L->ws_fwd_bytes, s);
+    }
     PRISM_TRY(prism_permute(p, V, L->perm, L->Vp, s));
     if (qk_ready && cudaStreamWaitEvent(s, qk_ready, 0) != cudaSuccess) return PRISM_ERR_CUDA;
     PRISM_TRY(prism_permute(p, Q, L->perm, L->Qp, s));
@@ -120,9 +132,19 @@ prism_status_t run_forward(const prism_layer_t* L, const void* Q, const void* K,
     return prism_unpermute(p, L->Op, L->perm, O, s);
 }
 
-prism_status_t run_backward(const prism_layer_t* L, const void* dO, void* dQ, void* dK, void* dV, cudaStream_t s,
+prism_status_t run_backward(const prism_layer_t* L, const void* Q, const void* K, const void* V, const void* dO,
+                            void* dQ, void* dK, void* dV, cudaStream_t s,
                             cudaEvent_t* done /* [3] nullable: after dQ, dK, dV */) {
     const prism_problem_t* p = &L->prob;
+    if (L->raster) {
+        PRISM_TRY(prism_sparse_attn_bwd_raster(p, Q, K, V, L->Of32, dO, L->lse, L->perm, L->shape_id, L->gsel,
+                                               L->gselT, L->scale, dQ, dK, dV, L->dev_status, L->ws_bwd,
+                                               L->ws_bwd_bytes, s));
+        if (done)
+            for (int i = 0; i < 3; ++i)
+                if (cudaEventRecord(done[i], s) != cudaSuccess) return PRISM_ERR_CUDA;
+        return PRISM_OK;
+    }
     PRISM_TRY(prism_permute(p, dO, L->perm, L->dOp, s));
     PRISM_TRY(prism_sparse_attn_bwd(p, L->Qp, L->Kp, L->Vp, L->Op, L->Of32, L->dOp, L->lse, L->gsel, L->gselT,
                                     L->scale, L->dQp, L->dKp, L->dVp, L->dev_status, L->ws_bwd, L->ws_bwd_bytes,
@@ -154,6 +176,7 @@ extern "C" prism_status_t prism_layer_init(prism_layer_t* L, const prism_problem
     L->fixed_shape = -1;
     L->with_backward = 1;
     L->with_io = 0;
+    L->raster = 0;
     L->p_blocks = 0;
     return PRISM_OK;
 }
@@ -183,11 +206,11 @@ extern "C" prism_status_t prism_layer_forward(const prism_layer_t* L, const void
     return run_forward(L, Q, K, V, hhat, O, stream, nullptr, nullptr);
 }
 
-extern "C" prism_status_t prism_layer_backward(const prism_layer_t* L, const void* dO, void* dQ, void* dK, void* dV,
-                                               cudaStream_t stream) {
+extern "C" prism_status_t prism_layer_backward(const prism_layer_t* L, const void* Q, const void* K, const void* V,
+                                               const void* dO, void* dQ, void* dK, void* dV, cudaStream_t stream) {
     if (!L || !params_ok(L)) return PRISM_ERR_INVALID_ARG;
     if (!L->with_backward) return PRISM_ERR_UNSUPPORTED;
-    return run_backward(L, dO, dQ, dK, dV, stream, nullptr);
+    return run_backward(L, Q, K, V, dO, dQ, dK, dV, stream, nullptr);
 }
 
 namespace {
@@ -251,7 +274,7 @@ extern "C" prism_status_t prism_layer_step_host(const prism_layer_t* L, const vo
     if (bwd) {
         if (cudaStreamWaitEvent(compute, ev.e[kDO], 0) != cudaSuccess) return PRISM_ERR_CUDA;
         cudaEvent_t done[3] = {ev.e[kDQ], ev.e[kDK], ev.e[kDV]};
-        PRISM_TRY(run_backward(L, L->dO, L->dQ, L->dK, L->dV, compute, done));
+        PRISM_TRY(run_backward(L, L->Q, L->K, L->V, L->dO, L->dQ, L->dK, L->dV, compute, done));
         void* hs[3] = {hdQ, hdK, hdV};
         void* ds[3] = {L->dQ, L->dK, L->dV};
         for (int i = 0; i < 3; ++i) {

@@ -26,7 +26,8 @@
 static int offsets(void) {
     printf("sizeof %zu\n", sizeof(prism_layer_t));
     FIELD(prob); FIELD(top_k); FIELD(top_p); FIELD(eps); FIELD(tau128); FIELD(tau256); FIELD(scale);
-    FIELD(guidance); FIELD(fixed_shape); FIELD(with_backward); FIELD(with_io); FIELD(p_blocks);
+    FIELD(guidance); FIELD(fixed_shape); FIELD(with_backward); FIELD(with_io); FIELD(raster);
+    FIELD(p_blocks);
     FIELD(g); FIELD(rho); FIELD(abar); FIELD(zone_stats); FIELD(ws_ind); FIELD(ws_ind_bytes);
     FIELD(shape_id); FIELD(perm); FIELD(blk_start); FIELD(gran_blk); FIELD(n_blk); FIELD(margin_shape);
     FIELD(Qp); FIELD(Kp); FIELD(Vp); FIELD(Qbar); FIELD(Kbar); FIELD(P); FIELD(sel); FIELD(gsel);

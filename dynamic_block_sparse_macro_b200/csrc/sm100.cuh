@@ -91,6 +91,22 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
         ::"r"(smem_u32(dst)), "l"(map), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
         : "memory");
 }
+// 5-D forms used for granules of the raster layout (coordinates: column in a
+// 64-column region, head-region, w, h, t)
+__device__ __forceinline__ void tma_load_5d(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1, int c2,
+                                            int c3, int c4) {
+    asm volatile(
+        "cp.async.bulk.tensor.5d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5, %6, %7}], "
+        "[%2];"
+        ::"r"(smem_u32(dst)), "l"(map), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4)
+        : "memory");
+}
+__device__ __forceinline__ void tma_store_5d(const CUtensorMap* map, const void* src, int c0, int c1, int c2, int c3,
+                                             int c4) {
+    asm volatile("cp.async.bulk.tensor.5d.global.shared::cta.bulk_group [%0, {%2, %3, %4, %5, %6}], [%1];"
+                 ::"l"(map), "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4)
+                 : "memory");
+}
 // TMA tile store from shared memory (a bulk group; coordinates must be >= 0)
 __device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* src, int x, int y, int z) {
     asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];"
@@ -487,6 +503,37 @@ inline bool make_map_bf16_rows(CUtensorMap* m, const void* base, int64_t rows, i
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
+
+// A raster [N][heads][d] bf16 tensor (N = T*H*W, raster token order) viewed
+// per 64-column region as a 5-D tensor (64 columns, heads*d/64 head-regions at
+// 128 bytes, W, H, T).  The 64 tokens of one granule of a (bT, bH, bW) block
+// are the box {64, 1, bW, bH, 64/(bH bW)} at (0, head * d/64 + region, w0, h0,
+// t0), (t0, h0, w0) the raster position of the granule's first token, and a
+// copy lands them in permutation order (t, h, w raster inside the block): the
+// rows the blocked layout holds, 128-byte swizzled like the whole-row maps.
+// The box depends on (bH, bW) only: kind = 3 (log2 bH - 1) + (log2 bW - 1).
+constexpr int kRasterKinds = 9;
+
+inline bool make_map_raster(CUtensorMap* m, const void* base, int heads, int hd, int T, int H, int W, int kind) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    const int eH = kind / 3 + 1, eW = kind % 3 + 1;
+    const uint64_t row = (uint64_t)heads * hd * 2;                 // bytes of one raster token
+    cuuint64_t dims[5] = {64, (cuuint64_t)(heads * hd / 64), (cuuint64_t)W, (cuuint64_t)H, (cuuint64_t)T};
+    cuuint64_t strides[4] = {128, (cuuint64_t)row, (cuuint64_t)(row * W), (cuuint64_t)(row * W * H)};
+    cuuint32_t box[5] = {64, 1, (cuuint32_t)(1 << eW), (cuuint32_t)(1 << eH), (cuuint32_t)(64 >> (eH + eW))};
+    cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// the raster maps of `tensors` tensors, all box kinds, passed to a kernel by
+// value (parameter space holds up to 32 KB), so no copy and no synchronisation
+template <int TENSORS>
+struct RasterMaps {
+    CUtensorMap m[TENSORS * kRasterKinds];
+};
 
 }  // namespace sm100
 }  // namespace prism

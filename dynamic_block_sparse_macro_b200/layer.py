@@ -30,7 +30,7 @@ _TORCH_DT = {"f32": torch.float32, "bf16": torch.bfloat16}
 class PrismSparseAttention:
     def __init__(self, T, H, W, heads, head_dim, audio_dim=64, dtype="bf16", top_k=8, top_p=0.9,
                  eps=1e-6, tau128=0.5, tau256=0.25, scale=None, device="cuda", p_blocks=None,
-                 with_backward=True, guidance="joint", fixed_shape=-1):
+                 with_backward=True, guidance="joint", fixed_shape=-1, raster=False):
         self.prob = _abi.problem(T, H, W, heads, head_dim, audio_dim, dtype)
         self.sizes = _abi.query_sizes(self.prob)
         self.dtype = dtype
@@ -44,6 +44,12 @@ class PrismSparseAttention:
         # with_backward=False is the inference path: no backward buffers, no key-major
         # selection, no fp32 copy of O and no LSE
         self.with_backward = bool(with_backward)
+        # raster=True: the attention reads Q, K, V, dO and writes O, dQ, dK, dV in place
+        # through the permutation (no blocked copies); bf16 only
+        self.raster = bool(raster)
+        if self.raster and dtype != "bf16":
+            raise ValueError("raster=True needs dtype='bf16'")
+        self._fwd_inputs = None
         dev = torch.device(device)
         self.device = dev
         s = self.sizes
@@ -61,7 +67,10 @@ class PrismSparseAttention:
         self.n_blk = e(1, dt=i32)
         self.margin_shape = e(Z, 2)
         # stage 3-5
-        self.Qp, self.Kp, self.Vp = (e(heads, N, head_dim, dt=self.tdt) for _ in range(3))
+        if self.raster:
+            self.Qp = self.Kp = self.Vp = None
+        else:
+            self.Qp, self.Kp, self.Vp = (e(heads, N, head_dim, dt=self.tdt) for _ in range(3))
         self.Qbar, self.Kbar = e(heads, MB, head_dim), e(heads, MB, head_dim)
         pb = MB if p_blocks is None else int(p_blocks)
         self.p_blocks = pb
@@ -74,14 +83,17 @@ class PrismSparseAttention:
         self.margin_sel = e(heads, MB)
         self.dev_status = torch.zeros(1, dtype=i32, device=dev)
         # stage 6-7
-        self.Op = e(heads, N, head_dim, dt=self.tdt)
+        self.Op = None if self.raster else e(heads, N, head_dim, dt=self.tdt)
         # unrounded O for the backward's Delta (bf16 storage only)
         self.Of32 = e(heads, N, head_dim) if (with_backward and dtype == "bf16") else None
         self.lse = e(heads, N) if with_backward else None
         self.ws_fwd = e(max(16, s.ws_attn_fwd), dt=torch.uint8)
         if with_backward:
-            self.dOp = e(heads, N, head_dim, dt=self.tdt)
-            self.dQp, self.dKp, self.dVp = (e(heads, N, head_dim, dt=self.tdt) for _ in range(3))
+            if self.raster:
+                self.dOp = self.dQp = self.dKp = self.dVp = None
+            else:
+                self.dOp = e(heads, N, head_dim, dt=self.tdt)
+                self.dQp, self.dKp, self.dVp = (e(heads, N, head_dim, dt=self.tdt) for _ in range(3))
             self.ws_bwd = e(max(16, s.ws_attn_bwd), dt=torch.uint8)
         self.L = self._describe()
 
@@ -92,6 +104,7 @@ class PrismSparseAttention:
         L.tau128, L.tau256, L.scale = self.tau128, self.tau256, self.scale
         L.guidance, L.fixed_shape = _abi.GUIDANCE[self.guidance], self.fixed_shape
         L.with_backward, L.with_io, L.p_blocks = int(self.with_backward), 0, self.p_blocks
+        L.raster = int(self.raster)
         for name in ("g", "rho", "abar", "zone_stats", "ws_ind", "shape_id", "perm", "blk_start", "gran_blk",
                      "n_blk", "margin_shape", "Qp", "Kp", "Vp", "Qbar", "Kbar", "P", "sel", "gsel", "gselT",
                      "sel_count", "margin_sel", "dev_status", "Op", "Of32", "lse", "ws_fwd"):
@@ -101,7 +114,8 @@ class PrismSparseAttention:
         L.ws_fwd_bytes = self.ws_fwd.numel()
         if self.with_backward:
             for name in ("dOp", "dQp", "dKp", "dVp", "ws_bwd"):
-                setattr(L, name, getattr(self, name).data_ptr())
+                t = getattr(self, name)
+                setattr(L, name, t.data_ptr() if t is not None else None)
             L.ws_bwd_bytes = self.ws_bwd.numel()
         return L
 
@@ -140,6 +154,26 @@ class PrismSparseAttention:
                                 self.sel, self.sel_count, self.gsel, self.gselT, self.margin_sel,
                                 self.dev_status, stream)
 
+    def select_raster(self, Q, K, stream=None):
+        """Stages 4-5 reading raster Q, K through the permutation (no blocked copies)."""
+        p = self.prob
+        _abi.prism_block_pool_score_raster(p, Q, K, self.perm, self.blk_start, self.n_blk, self.scale, self.Qbar,
+                                           self.Kbar, self.P, stream)
+        _abi.prism_block_select(p, self.P, self.blk_start, self.gran_blk, self.n_blk, self.top_k, self.top_p,
+                                self.sel, self.sel_count, self.gsel, self.gselT, self.margin_sel, self.dev_status,
+                                stream)
+
+    def attend_raster(self, Q, K, V, out, stream=None):
+        """Stage 6 from raster Q, K, V into raster O (``out``)."""
+        _abi.prism_sparse_attn_fwd_raster(self.prob, Q, K, V, self.perm, self.shape_id, self.gsel, self.scale, out,
+                                          self.lse, self.Of32, self.dev_status, self.ws_fwd, stream)
+
+    def attend_backward_raster(self, Q, K, V, dO, dQ, dK, dV, stream=None):
+        """Stage 7 from raster Q, K, V, dO into raster dQ, dK, dV."""
+        _abi.prism_sparse_attn_bwd_raster(self.prob, Q, K, V, self.Of32, dO, self.lse, self.perm, self.shape_id,
+                                          self.gsel, self.gselT, self.scale, dQ, dK, dV, self.dev_status, self.ws_bwd,
+                                          stream)
+
     def attend(self, stream=None):
         """Stage 6 on the blocked tensors."""
         _abi.prism_sparse_attn_fwd(self.prob, self.Qp, self.Kp, self.Vp, self.gsel, self.scale, self.Op,
@@ -156,6 +190,8 @@ class PrismSparseAttention:
         if out is None:
             out = torch.empty_like(Q)
         _abi.prism_layer_forward(self.L, Q, K, V, hhat, out, stream)
+        if self.raster and self.with_backward:
+            self._fwd_inputs = (Q, K, V)          # the raster backward reads them again
         if check:
             self.check_status(stream)
         return out
@@ -166,7 +202,10 @@ class PrismSparseAttention:
         if not self.with_backward:
             raise RuntimeError("this layer was built for inference (with_backward=False)")
         outs = [t if t is not None else torch.empty_like(dO) for t in (dQ, dK, dV)]
-        _abi.prism_layer_backward(self.L, dO, *outs, stream)
+        q, k, v = self._fwd_inputs if self.raster else (None, None, None)
+        if self.raster and q is None:
+            raise RuntimeError("backward before forward")
+        _abi.prism_layer_backward(self.L, q, k, v, dO, *outs, stream)
         if check:
             self.check_status(stream)
         return tuple(outs)

@@ -294,6 +294,42 @@ prism_status_t prism_sparse_attn_bwd(const prism_problem_t* prob, const void* Qp
                                      void* dVp, uint32_t* dev_status, void* ws, size_t ws_bytes,
                                      cudaStream_t stream);
 
+/*
+ * Stages 4, 6 and 7 straight from the raster layout (news page, "工作原理" step 4:
+ * the kernel runs over the permuted blocks and the original layout comes back;
+ * here the permutation is applied inside the loads and stores instead of by
+ * copies).  Q, K, V, O raster [N][heads][head_dim]; perm and shape_id from
+ * prism_assign_shapes.  The results equal, bit for bit, those of the blocked
+ * calls on prism_permute'd inputs followed by prism_unpermute of O.
+ *   prism_block_pool_score_raster: as prism_block_pool_score, rows read
+ *     through perm.
+ *   prism_sparse_attn_fwd_raster: as prism_sparse_attn_fwd; every 64-row
+ *     granule of the blocked order is one tensor-map box of the raster tensor
+ *     (its tokens are an (n_T, b_H, b_W) sub-box of the block), so Q, K and V are
+ *     loaded and O is stored in place.  lse and o_f32 (nullable) stay in
+ *     permutation order ([heads][N]).  bf16 only (PRISM_ERR_UNSUPPORTED else);
+ *     ws >= sizes.ws_attn_fwd.
+ */
+prism_status_t prism_block_pool_score_raster(const prism_problem_t* prob, const void* Q, const void* K,
+                                             const int32_t* perm, const int32_t* blk_start, const int32_t* n_blk,
+                                             float scale, float* Qbar, float* Kbar, float* P, cudaStream_t stream);
+prism_status_t prism_sparse_attn_fwd_raster(const prism_problem_t* prob, const void* Q, const void* K,
+                                            const void* V, const int32_t* perm, const uint8_t* shape_id,
+                                            const uint32_t* gsel, float scale, void* O, float* lse, float* o_f32,
+                                            uint32_t* dev_status, void* ws, size_t ws_bytes, cudaStream_t stream);
+/*
+ * Stage 7 on raster operands: as prism_sparse_attn_bwd with Q, K, V, dO, dQ,
+ * dK, dV raster [N][heads][head_dim]; o_f32 (required: the forward's unrounded
+ * O) and lse in permutation order, as prism_sparse_attn_fwd_raster leaves
+ * them.  Bit for bit the blocked call's results, unpermuted.  bf16 only;
+ * ws >= sizes.ws_attn_bwd.
+ */
+prism_status_t prism_sparse_attn_bwd_raster(const prism_problem_t* prob, const void* Q, const void* K,
+                                            const void* V, const float* o_f32, const void* dO, const float* lse,
+                                            const int32_t* perm, const uint8_t* shape_id, const uint32_t* gsel,
+                                            const uint32_t* gselT, float scale, void* dQ, void* dK, void* dV,
+                                            uint32_t* dev_status, void* ws, size_t ws_bytes, cudaStream_t stream);
+
 /* Copy a device status word to the host (synchronises `stream`). */
 prism_status_t prism_read_status(const uint32_t* dev_status, uint32_t* host_out, cudaStream_t stream);
 
@@ -327,6 +363,8 @@ typedef struct {
     int32_t fixed_shape;    /* -1: adaptive shapes                                  */
     int32_t with_backward;  /* 1; 0 = inference: no LSE, fp32 O, gselT, backward buffers */
     int32_t with_io;        /* 0; 1 = also the raster inputs/outputs, for prism_layer_step_host */
+    int32_t raster;         /* 0; 1 = the attention reads Q, K, V, dO and writes O, dQ, dK, dV
+                               in the raster layout: no blocked copies (bf16 only)          */
     int64_t p_blocks;       /* 0: P sized for max_blocks; else a caller-known bound on n_blk */
     /* device buffers; shapes and layouts as the stage calls above describe them */
     float *g, *rho, *abar, *zone_stats;
@@ -364,9 +402,11 @@ prism_status_t prism_layer_bind(prism_layer_t* L, void* arena, size_t bytes);
 prism_status_t prism_layer_forward(const prism_layer_t* L, const void* Q, const void* K, const void* V,
                                    const void* hhat, void* O, cudaStream_t stream);
 /* Stage 7 for the last forward on `stream`: raster device dO in, raster dQ, dK,
- * dV out.  PRISM_ERR_UNSUPPORTED when L has no backward buffers. */
-prism_status_t prism_layer_backward(const prism_layer_t* L, const void* dO, void* dQ, void* dK, void* dV,
-                                    cudaStream_t stream);
+ * dV out.  Q, K, V: the last forward's raster inputs, unchanged since (read
+ * only when L->raster; may be NULL otherwise).  PRISM_ERR_UNSUPPORTED when L
+ * has no backward buffers. */
+prism_status_t prism_layer_backward(const prism_layer_t* L, const void* Q, const void* K, const void* V,
+                                    const void* dO, void* dQ, void* dK, void* dV, cudaStream_t stream);
 /* One whole step from HOST buffers (L bound with with_io = 1): uploads Q, K,
  * V, hhat (and dO with a backward), runs the layer, downloads O (and dQ, dK,
  * dV), with one cudaMemcpyAsync per tensor on the two copy streams: V and
