@@ -3,9 +3,12 @@ runs them (same configuration, same calls).  What the oracle can do in full is
 checked in full (the shapes of every zone, the permutation, the block table);
 the rest on samples the oracle computes one by one: raw statistics of sampled
 zones (each zone on its own), the grid-wide normalisation from the GPU's own
-statistics, bit-exact permuted rows, P rows, selection rows, O / LSE of sampled
-query blocks, dQ of sampled query blocks and dK / dV of sampled key blocks,
-all on one sampled head and under the GPU's own upstream decisions."""
+statistics, bit-exact permuted rows, P rows, O / LSE of sampled query blocks,
+dQ of sampled query blocks and dK / dV of sampled key blocks on one sampled
+head (the samples always include the query block with the most selected blocks
+and the key block most query blocks selected: the split tiles), and every
+selection row of every head (two heads at the long grid), all under the GPU's
+own upstream decisions."""
 import numpy as np
 import pytest
 import torch
@@ -29,10 +32,11 @@ def _f64(t):
     return t.detach().float().cpu().numpy().astype(np.float64)
 
 
-@pytest.mark.parametrize("name,fixed", [("720p", -1), ("1080p", -1), ("2k", -1), ("2k", 3)])
+@pytest.mark.parametrize("name,fixed", [("720p", -1), ("1080p", -1), ("2k", -1), ("2k", 3), ("long", -1)])
 def test_full_size_sampled(name, fixed):
     # ("2k", 3): the fixed-shape baseline with 64-token blocks everywhere, 4608 blocks a row,
-    # which takes the one-CTA-per-row selection (rows of more than 4096 blocks)
+    # which takes the one-CTA-per-row selection (rows of more than 4096 blocks).
+    # "long": 1,032,192 tokens, the first grid whose element offsets pass 2^31.
     cfg = get_config(name)
     T, H, W = cfg.T, cfg.H, cfg.W
     N, Z = cfg.n_tokens, cfg.n_tokens // 512
@@ -93,14 +97,28 @@ def test_full_size_sampled(name, fixed):
     # stage 4: P rows of sampled query blocks (the oracle pools every block of the head)
     _, _, P = orc.block_pool_score(Qh, Kh, bs, heads=[0])
     Pg = mod.P_view()[hh].cpu().double().numpy()
-    qsamp = rng.choice(nb, 5, replace=False).tolist()
+    sel_g = unpack_sel(mod.sel[hh:hh + 1], nb)[0]
+    # the heaviest rows are the split tiles the combine kernels merge: always sampled
+    q_heavy = int(sel_g.sum(1).argmax())
+    k_heavy = int(sel_g.sum(0).argmax())
+    qsamp = sorted(set(rng.choice(nb, 4, replace=False).tolist()) | {q_heavy})
     np.testing.assert_allclose(Pg[qsamp], P[0][qsamp], rtol=1e-4, atol=1e-7)
 
-    # stage 5: selection rows teacher-forced on the GPU's P rows
-    sel_g = unpack_sel(mod.sel[hh:hh + 1], nb)[0]
-    tsel = orc.block_select(Pg[qsamp], cfg.top_k, cfg.top_p)
-    badr = (sel_g[qsamp] != tsel["sel"]).any(-1)
-    assert (tsel["margin"][badr] < NEAR_TIE).all()
+    # stage 5: every selection row, teacher-forced on the GPU's own P (every head; two at the
+    # long grid, whose P holds 4 GB), mismatches only where the oracle's margin is below NEAR_TIE
+    heads_sel = range(cfg.heads) if name != "long" else sorted({hh, (hh + cfg.heads // 2) % cfg.heads})
+    ties = rows = 0
+    for h in heads_sel:
+        Ph = mod.P_view()[h].cpu().double().numpy()
+        sh = unpack_sel(mod.sel[h:h + 1], nb)[0]
+        tsel = orc.block_select(Ph, cfg.top_k, cfg.top_p)
+        badr = (sh != tsel["sel"]).any(-1)
+        assert (tsel["margin"][badr] < NEAR_TIE).all(), (h, np.nonzero(badr), tsel["margin"][badr])
+        ties += int(badr.sum())
+        rows += nb
+    print(f"{name}: selection near-ties {ties} of {rows} rows ({len(heads_sel)} heads); "
+          f"heaviest query block {q_heavy} ({int(sel_g[q_heavy].sum())} blocks), "
+          f"key block {k_heavy} selected by {int(sel_g[:, k_heavy].sum())}")
 
     # stage 6: O and LSE of sampled query blocks under the GPU's selection
     tol = REL_L2[cfg.dtype]
@@ -116,18 +134,22 @@ def test_full_size_sampled(name, fixed):
 
     # stage 7: dQ of the sampled query blocks, dK / dV of sampled key blocks
     dOh = _f64(x["dO"][perm_t, hh])[None]
-    ksamp = rng.choice(nb, 3, replace=False).tolist()
+    ksamp = sorted(set(rng.choice(nb, 2, replace=False).tolist()) | {k_heavy})
     dQ_ref, _, _ = orc.sparse_attention_bwd(Qh, Kh, Vh, dOh, bs, sel_g[None], heads=[0], q_blocks=qsamp)
     # dK, dV of the sampled key blocks visit every query row that selected them: teacher-forced on
     # the forward's LSE and fp32 O (both checked on samples above) instead of re-normalising each row
     Of = _f64(mod.Of32[hh])[None] if mod.Of32 is not None else Ob[None]
     dK_ref, dV_ref = orc.sparse_attention_bwd_keys(Qh, Kh, Vh, dOh, bs, sel_g[None], lse[None], Of, heads=[0],
                                                    k_blocks=ksamp)
-    floor = 1e-4 * float(np.linalg.norm(dOh))
+    # per block, as on the small grids: a block's gradient is a cancelling sum (each row of
+    # dS sums to zero), so it is measured against at least a tenth of the sampled blocks' RMS
+    # norm, at five times the whole-tensor bar
     for dst, ref, blocks in ((mod.dQp, dQ_ref, qsamp), (mod.dKp, dK_ref, ksamp), (mod.dVp, dV_ref, ksamp)):
         got = _f64(dst[hh])
+        norms = [float(np.linalg.norm(ref[0, bs[i]:bs[i + 1]])) for i in blocks]
+        rms = float(np.sqrt(np.mean(np.square(norms))))
         for i in blocks:
             r0, r1 = bs[i], bs[i + 1]
-            assert rel_l2(got[r0:r1], ref[0, r0:r1], floor * (r1 - r0) / N) <= tol, i
+            assert rel_l2(got[r0:r1], ref[0, r0:r1], 0.1 * rms) <= 5 * tol, i
     for dst, out in zip((mod.dQp, mod.dKp, mod.dVp), grads):
         assert torch.equal(out[perm_t, hh], dst[hh])
