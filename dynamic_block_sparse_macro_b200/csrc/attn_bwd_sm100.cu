@@ -113,9 +113,10 @@ struct BarsP {
     uint64_t* elem;            // [2]
     uint64_t* qdo_full;
     uint64_t* fin;
-    uint64_t* drain;           // teardown after an abort: every issued MMA complete
+    uint64_t* drain;           // [3] teardown after an abort: every MMA an issuer issued complete
     uint64_t* rows_full;       // [2]
     uint64_t* rows_empty;      // [2]
+    uint64_t* dq_done;         // [2] dQ MMAs of the buffer's granule complete (its dS read)
     uint32_t* tmem_slot;
     volatile int* abort_flag;
 };
@@ -130,13 +131,14 @@ __device__ __forceinline__ BarsP carve_p(uint8_t* ctrl) {
     r.qdo_full = b + 3 * kStages + 4;
     r.fin = b + 3 * kStages + 5;
     r.drain = b + 3 * kStages + 6;
-    r.rows_full = b + 3 * kStages + 7;
-    r.rows_empty = b + 3 * kStages + 9;
-    r.tmem_slot = reinterpret_cast<uint32_t*>(b + 3 * kStages + 11);
+    r.rows_full = b + 3 * kStages + 9;
+    r.rows_empty = b + 3 * kStages + 11;
+    r.dq_done = b + 3 * kStages + 13;
+    r.tmem_slot = reinterpret_cast<uint32_t*>(b + 3 * kStages + 15);
     r.abort_flag = reinterpret_cast<volatile int*>(r.tmem_slot + 1);
     return r;
 }
-static_assert((3 * kStages + 11) * 8 + 8 <= kCtrl, "barriers overflow the control block");
+static_assert((3 * kStages + 15) * 8 + 8 <= kCtrl, "barriers overflow the control block");
 
 // Epilogue with a 32 KB staging area of its own (the ring is busy with the
 // next item), shared by the two elementwise warpgroups, warpgroup wg owning
@@ -243,7 +245,7 @@ __device__ __forceinline__ void load_row_tmem(uint32_t taddr, const __nv_bfloat1
 }
 
 template <int D, bool RASTER>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(384, 1)
 k_bwd_dq_persist(const __nv_bfloat16* __restrict__ Qg, const __nv_bfloat16* __restrict__ dOg,
                  const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                  const __grid_constant__ CUtensorMap tmdQ, const __grid_constant__ CUtensorMap tmPqh,
@@ -272,14 +274,15 @@ k_bwd_dq_persist(const __nv_bfloat16* __restrict__ Qg, const __nv_bfloat16* __re
             mbar_init(B.empty + s, 1);
         }
         for (int b = 0; b < 2; ++b) {
-            mbar_init(B.prod + b, 1);
+            mbar_init(B.prod + b, 2);                  // the S and the dP issuer each commit
             mbar_init(B.elem + b, 256);
             mbar_init(B.rows_full + b, 32);
             mbar_init(B.rows_empty + b, 8);
+            mbar_init(B.dq_done + b, 1);
         }
         mbar_init(B.qdo_full, 256);
         mbar_init(B.fin, 1);
-        mbar_init(B.drain, 1);
+        for (int i = 0; i < 3; ++i) mbar_init(B.drain + i, 1);
         *B.abort_flag = 0;
         fence_mbar_init();
     }
@@ -362,8 +365,17 @@ k_bwd_dq_persist(const __nv_bfloat16* __restrict__ Qg, const __nv_bfloat16* __re
             volatile int no_abort = 0;                     // let this lane's last copy land
             mbar_wait(full + stage, (uint32_t)last_cyc & 1, &no_abort, dev_status);
         }
-    } else if (warp == 1) {
-        // ---------------------------------------------------------------- MMA (whole warp, elected issue)
+    } else if (warp == 1 || warp >= 10) {
+        // ---------------------------------------------------------------- MMA issue, three warps
+        // Three accumulation chains, each issued in order by one warp on its own
+        // SM sub-partition: warp 1 S = Q K^T, warp 10 dP = dO V^T, warp 11
+        // dQ += dS K.  Per TMEM buffer b and its u-th use (granule GG, b = GG & 1,
+        // u = GG >> 1): S(GG) waits elem(b) and dq_done(b) of use u - 1 (its
+        // columns consumed and dS read), dP(GG) waits elem(b) of use u - 1,
+        // dQ(GG) waits elem(b) of use u; prod(b) completes when both S and dP
+        // have.  No barrier can run two phases ahead of its waiter: every phase
+        // needs the waiter's own earlier issue.
+        const int role = warp == 1 ? 0 : warp - 9;          // 0: S, 1: dP, 2: dQ
         const uint32_t idPS = idesc_bf16_f32(128, 64, false, false);
         const uint32_t idQ = idesc_bf16_f32(128, D, false, true);
         const uint32_t aR = smem_u32(sm);
@@ -375,60 +387,60 @@ k_bwd_dq_persist(const __nv_bfloat16* __restrict__ Qg, const __nv_bfloat16* __re
             const int4 item = items[it];
             const int ng = item.z - item.y;
             if (ng == 0) continue;
-            ok = mbar_wait_w(B.qdo_full, kq & 1, B.abort_flag, dev_status);
-            if (!ok) break;
-            tc_fence_after();
-            int prev_s = 0;
-            for (int g = 0; ok && g <= ng; ++g) {
-                if (g < ng) {
-                    const int GG = G + g;
-                    const int s = s_, b = GG & 1;
-                    const uint32_t ph = (uint32_t)c_ & 1;
-                    if (!mbar_wait_w(B.full0 + s, ph, B.abort_flag, dev_status)) {
-                        ok = false;
-                        break;
+            if (role < 2) {
+                ok = mbar_wait_w(B.qdo_full, kq & 1, B.abort_flag, dev_status);
+                if (!ok) break;
+                tc_fence_after();
+            }
+            for (int g = 0; g < ng; ++g) {
+                const int GG = G + g;
+                const int s = s_, b = GG & 1, u = GG >> 1;
+                const uint32_t ph = (uint32_t)c_ & 1;
+                if (++s_ == nst) { s_ = 0; ++c_; }
+                if (role < 2) {
+                    if (!mbar_wait_w(B.full0 + s, ph, B.abort_flag, dev_status)) { ok = false; break; }
+                    if (GG >= 2) {
+                        if (!mbar_wait_w(B.elem + b, (uint32_t)(u - 1) & 1, B.abort_flag, dev_status) ||
+                            (role == 0 && !mbar_wait_w(B.dq_done + b, (uint32_t)(u - 1) & 1, B.abort_flag, dev_status))) {
+                            ok = false;
+                            break;
+                        }
                     }
                     tc_fence_after();
                     const uint64_t dK = sdesc_sw128(aR + s * L::STAGE, 16, 1024);
-                    const uint64_t dV = sdesc_add(dK, L::NR * kGran);
+                    if (role == 0) {
 #pragma unroll
-                    for (int k = 0; k < D / 16; ++k)
-                        mma_ts_w(tb + cS + 128 * b, tb + cQ + 8 * k, sdesc_add(dK, kmaj_off(k, kGran)), idPS, k > 0);
+                        for (int k = 0; k < D / 16; ++k)
+                            mma_ts_w(tb + cS + 128 * b, tb + cQ + 8 * k, sdesc_add(dK, kmaj_off(k, kGran)), idPS, k > 0);
+                    } else {
+                        const uint64_t dV = sdesc_add(dK, L::NR * kGran);
 #pragma unroll
-                    for (int k = 0; k < D / 16; ++k)
-                        mma_ts_w(tb + cP + 128 * b, tb + cdO + 8 * k, sdesc_add(dV, kmaj_off(k, kGran)), idPS, k > 0);
-                    tc_commit_w(B.prod + b);
-                }
-                if (g > 0) {
-                    const int gp = g - 1;
-                    const int GGp = G + gp;
-                    const int s = prev_s, b = GGp & 1;
-                    if (!mbar_wait_w(B.elem + b, (uint32_t)(GGp >> 1) & 1, B.abort_flag, dev_status)) {
-                        ok = false;
-                        break;
+                        for (int k = 0; k < D / 16; ++k)
+                            mma_ts_w(tb + cP + 128 * b, tb + cdO + 8 * k, sdesc_add(dV, kmaj_off(k, kGran)), idPS,
+                                     k > 0);
                     }
+                    tc_commit_w(B.prod + b);
+                } else {
+                    if (!mbar_wait_w(B.elem + b, (uint32_t)u & 1, B.abort_flag, dev_status)) { ok = false; break; }
                     tc_fence_after();
                     const uint64_t dKq = sdesc_sw128(aR + s * L::STAGE, kGran, 1024);
 #pragma unroll
                     for (int k = 0; k < 4; ++k)              // dS keys 16 k ..: warpgroup k / 2's columns
                         mma_ts_w(tb + cdQ, tb + cS + 128 * b + 32 * (k >> 1) + 8 * (k & 1), sdesc_add(dKq, k * 2048),
-                                 idQ, (gp > 0 || k > 0) ? 1u : 0u);
+                                 idQ, (g > 0 || k > 0) ? 1u : 0u);
                     tc_commit_w(B.empty + s);
-                }
-                if (g < ng) {
-                    prev_s = s_;
-                    if (++s_ == nst) { s_ = 0; ++c_; }
+                    tc_commit_w(B.dq_done + b);
                 }
             }
             if (!ok) break;
-            tc_commit_w(B.fin);
+            if (role == 2) tc_commit_w(B.fin);
             G += ng;
             ++kq;
         }
         if (!ok) {
-            tc_commit_w(B.drain);                          // every MMA issued so far complete
+            tc_commit_w(B.drain + role);                   // every MMA this warp issued complete
             volatile int no_abort = 0;
-            mbar_wait(B.drain, 0, &no_abort, dev_status);
+            mbar_wait(B.drain + role, 0, &no_abort, dev_status);
         }
     } else {
         // ---------------------------------------------------------------- elementwise + epilogue
@@ -1148,7 +1160,7 @@ prism_status_t launch_bwd(const Dims& d, const void* Qp, const void* Kp, const v
         return PRISM_ERR_CUDA;
     // persistent: one CTA per SM (all 512 TMEM columns each), items strided over the CTAs
     const int64_t gq = w.pq.items_max < device_sms() ? w.pq.items_max : device_sms();
-    kq<<<(unsigned)gq, 320, smq, s>>>((const __nv_bfloat16*)Qp, (const __nv_bfloat16*)dOp, gK, gV, tdQ, tPqh, rq,
+    kq<<<(unsigned)gq, 384, smq, s>>>((const __nv_bfloat16*)Qp, (const __nv_bfloat16*)dOp, gK, gV, tdQ, tPqh, rq,
                                       ras, gsel, w.pq.hdr, w.pq.items, lse, w.delta, d.N, d.MB, (int)d.SW, nq, scale,
                                       dev_status);
     const int64_t gk = w.pkv.items_max < device_sms() ? w.pkv.items_max : device_sms();
