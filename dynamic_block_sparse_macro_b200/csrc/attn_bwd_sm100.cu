@@ -155,7 +155,7 @@ template <int D>
 __device__ void store_tile_p(uint32_t tacc, int row, int wg, bool ok, bool zero, bool part, float mul,
                              uint8_t* stage, const CUtensorMap* map_bf16, const CUtensorMap* map_f32h, int y_bf16,
                              int y_f32, int bar_id, int nthreads, bool leader, const CUtensorMap* rmaps = nullptr,
-                             int4 gp0 = int4{}, int4 gp1 = int4{}, int hreg = 0) {
+                             int4 gp0 = int4{}, int4 gp1 = int4{}, int hreg = 0, int store_lane = 0) {
     static_assert(D == 128 || D == 64, "head_dim");
     const int regions = part ? D / 32 : D / 64;            // 128-byte regions of a row
     const int per_pass = regions < 2 ? regions : 2;
@@ -204,17 +204,15 @@ __device__ void store_tile_p(uint32_t tacc, int row, int wg, bool ok, bool zero,
             fence_proxy_async_smem();
         }
         named_sync(bar_id, nthreads);
-        if (ok && leader) {
+        // leader: lane 0 of the storing warp, or (raster bf16 tile) the lanes
+        // store_lane = 0 .. 2 D/64 - 1, each with its own (granule, region) box
+        if (ok && leader && (store_lane == 0 || (rmaps && !part))) {
             if (part) {
                 tma_store_3d(map_f32h, stage, 0, y_f32, p * per_pass);
             } else if (rmaps) {
-#pragma unroll
-                for (int hg = 0; hg < 2; ++hg) {
-                    const int4 gp = hg ? gp1 : gp0;
-#pragma unroll
-                    for (int r = 0; r < D / 64; ++r)
-                        tma_store_5d(rmaps + gp.w, stage + r * kTile + hg * kGran, 0, hreg + r, gp.z, gp.y, gp.x);
-                }
+                const int hg = store_lane / (D / 64), r = store_lane % (D / 64);
+                const int4 gp = hg ? gp1 : gp0;
+                tma_store_5d(rmaps + gp.w, stage + r * kTile + hg * kGran, 0, hreg + r, gp.z, gp.y, gp.x);
             } else {
                 tma_store_3d(map_bf16, stage, 0, y_bf16, 0);
             }
@@ -255,6 +253,7 @@ k_bwd_dq_persist(const __nv_bfloat16* __restrict__ Qg, const __nv_bfloat16* __re
                  const float* __restrict__ delta, int64_t N, int64_t MB, int SW, int nst, float scale,
                  uint32_t* __restrict__ dev_status) {
     using L = DqpLayout<D>;
+    constexpr int kRL = RASTER ? L::NR : 1;            // copy lanes per (stream, stage)
     constexpr uint32_t cdQ = 0, cS = 128, cP = 192;   // + 128 * buffer for S / dP
     constexpr uint32_t cQ = 384, cdO = 384 + D / 2;
     const int n_items = hdr->n_items;
@@ -270,7 +269,7 @@ k_bwd_dq_persist(const __nv_bfloat16* __restrict__ Qg, const __nv_bfloat16* __re
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < nst; ++s) {
-            mbar_init(B.full0 + s, 2);                 // the K and the V copy lane each arrive
+            mbar_init(B.full0 + s, 2 * kRL);           // each K and V copy lane arrives
             mbar_init(B.empty + s, 1);
         }
         for (int b = 0; b < 2; ++b) {
@@ -299,8 +298,11 @@ k_bwd_dq_persist(const __nv_bfloat16* __restrict__ Qg, const __nv_bfloat16* __re
         // ---------------------------------------------------------------- producer
         // lane kind * nst + stage (kind 0: K, 1: V) issues its stream's copies for
         // the granules of that stage; all 32 lanes copy the selection rows
-        const int kind = lane / nst, stage = lane % nst;
-        const bool copier = lane < 2 * nst;
+        // lane (kind * nst + stage) * kRL + region: a raster granule is one box per
+        // 64-column region, each from a lane of its own (copies of one thread
+        // complete one after another)
+        const int kind = lane / (nst * kRL), stage = (lane / kRL) % nst, region = lane % kRL;
+        const bool copier = lane < 2 * nst * kRL;
         uint64_t* full = B.full0;                          // one barrier for both copies of a stage
         const CUtensorMap* mg = kind == 0 ? &tmK : &tmV;
         if (copier && !RASTER) tma_prefetch_desc(mg);
@@ -338,15 +340,14 @@ k_bwd_dq_persist(const __nv_bfloat16* __restrict__ Qg, const __nv_bfloat16* __re
                             ok = false;
                             break;
                         }
-                        mbar_expect_tx(full + stage, L::NR * kGran);
                         uint8_t* dst = sm + stage * L::STAGE + kind * L::NR * kGran;
                         if constexpr (RASTER) {
                             const int4 gp = ras.gpos[row >> 6];
-                            const CUtensorMap* mr = rmaps.m + (kind ? kRV : kRK) * kRasterKinds + gp.w;
-#pragma unroll
-                            for (int r = 0; r < L::NR; ++r)
-                                tma_load_5d(dst + r * kGran, mr, full + stage, 0, hh * L::NR + r, gp.z, gp.y, gp.x);
+                            mbar_expect_tx(full + stage, kGran);
+                            tma_load_5d(dst + region * kGran, rmaps.m + (kind ? kRV : kRK) * kRasterKinds + gp.w,
+                                        full + stage, 0, hh * L::NR + region, gp.z, gp.y, gp.x);
                         } else {
+                            mbar_expect_tx(full + stage, L::NR * kGran);
                             tma_load_3d(dst, mg, full + stage, 0, (int)(row0 + row), 0);
                         }
                         last_cyc = c_;
@@ -552,9 +553,9 @@ k_bwd_dq_persist(const __nv_bfloat16* __restrict__ Qg, const __nv_bfloat16* __re
             // the item's dQ (or zeros when nothing was selected: ng == 0)
             if constexpr (RASTER)
                 store_tile_p<D>(tl + cdQ, row, wg, fin, ng == 0, slot >= 0, scale, staging, &tmdQ, &tmPqh,
-                                (int)(row0 + 128 * tile), slot * 128, 1, 256, warp == 2 && lane == 0,
+                                (int)(row0 + 128 * tile), slot * 128, 1, 256, warp == 2 && lane < 2 * (D / 64),
                                 rmaps.m + kRdQ * kRasterKinds, ras.gpos[2 * tile], ras.gpos[2 * tile + 1],
-                                hh * (D / 64));
+                                hh * (D / 64), lane);
             else
                 store_tile_p<D>(tl + cdQ, row, wg, fin, ng == 0, slot >= 0, scale, staging, &tmdQ, &tmPqh,
                                 (int)(row0 + 128 * tile), slot * 128, 1, 256, warp == 2 && lane == 0);
@@ -642,6 +643,8 @@ k_bwd_dkdv_persist(const __grid_constant__ CUtensorMap tmK, const __grid_constan
                    const int4* __restrict__ items, const float* __restrict__ nld,
                    int64_t N, int64_t MB, int SW, int nst, float scale, uint32_t* __restrict__ dev_status) {
     using L = DkvpLayout<D>;
+    constexpr int kRL = RASTER ? L::NR : 1;            // copy lanes per (stream, stage)
+    constexpr int kStatLanes = RASTER ? 2 * 2 * L::NR : 2;   // stationary copies: (tensor, granule, region)
     constexpr uint32_t cdK = 0, cdV = 128, cS = 256, cP = 320;   // + 128 * buffer for S^T / dP^T
     const int n_items = hdr->n_items;
     if ((int)blockIdx.x >= n_items) return;
@@ -657,7 +660,7 @@ k_bwd_dkdv_persist(const __grid_constant__ CUtensorMap tmK, const __grid_constan
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < nst; ++s) {
-            mbar_init(B.full0 + s, 2);                 // the Q and the dO copy lane each arrive
+            mbar_init(B.full0 + s, 2 * kRL);           // each Q and dO copy lane arrives
             mbar_init(B.fullx + s, 1);
             mbar_init(B.empty + s, 1);
         }
@@ -667,7 +670,7 @@ k_bwd_dkdv_persist(const __grid_constant__ CUtensorMap tmK, const __grid_constan
             mbar_init(B.rows_full + b, 32);
             mbar_init(B.rows_empty + b, 8);
         }
-        mbar_init(B.stat, 2);
+        mbar_init(B.stat, kStatLanes);
         mbar_init(B.kv_free, 1);
         mbar_init(B.fin, 1);
         mbar_init(B.drain, 1);
@@ -687,12 +690,19 @@ k_bwd_dkdv_persist(const __grid_constant__ CUtensorMap tmK, const __grid_constan
       regs_dec<kRegsLow>();
       if (warp == 0) {
         // ---------------------------------------------------------------- producer
-        // lanes kind * nst + stage (kind 0: Q, 1: dO, 2: the granule's row data)
-        // stream the ring; lanes 30 (K) and 31 (V) load the stationary tiles of
-        // each non-empty item once the previous one's S^T/dP^T MMAs are done
-        const int kind = lane / nst, stage = lane % nst;
-        const bool copier = lane < 3 * nst;
-        const bool stat_lane = lane >= 30;
+        // lanes (kind * nst + stage) * kRL + region stream Q (kind 0) and dO
+        // (kind 1) of the ring, one 64-column region each in the raster layout;
+        // the next nst lanes the granules' row data (kind 2); the top kStatLanes
+        // lanes load the stationary K and V tiles of each non-empty item once the
+        // previous one's S^T/dP^T MMAs are done (copies of one thread complete
+        // one after another, so each copy has a lane)
+        const int nqd = 2 * nst * kRL;                     // Q and dO copy lanes
+        const int kind = lane < nqd ? lane / (nst * kRL) : 2;
+        const int stage = lane < nqd ? (lane / kRL) % nst : lane - nqd;
+        const int region = lane < nqd ? lane % kRL : 0;
+        const bool copier = lane < nqd + nst;
+        const int si = lane - (32 - kStatLanes);           // stationary copy index
+        const bool stat_lane = si >= 0;
         uint64_t* full = kind < 2 ? B.full0 : B.fullx;     // Q and dO share one barrier per stage
         const CUtensorMap* mg = kind == 0 ? &tmQ : &tmdO;
         if (copier && kind < 2 && !RASTER) tma_prefetch_desc(mg);
@@ -722,21 +732,18 @@ k_bwd_dkdv_persist(const __grid_constant__ CUtensorMap tmK, const __grid_constan
                 if (stat_lane && ok) {
                     if (kq >= 1) ok = mbar_wait(B.kv_free, (uint32_t)(kq - 1) & 1, B.abort_flag, dev_status);
                     if (ok) {
-                        mbar_expect_tx(B.stat, L::NR * kTile);
-                        uint8_t* dst = sm + (lane == 30 ? L::A0 : L::A1);
                         if constexpr (RASTER) {
-                            // the tile's two key granules, one box per region each
-                            const CUtensorMap* mr = rmaps.m + (lane == 30 ? kRK : kRV) * kRasterKinds;
-#pragma unroll
-                            for (int hg = 0; hg < 2; ++hg) {
-                                const int4 gp = ras.gpos[2 * tile + hg];
-#pragma unroll
-                                for (int r = 0; r < L::NR; ++r)
-                                    tma_load_5d(dst + r * kTile + hg * kGran, mr + gp.w, B.stat, 0, hh * L::NR + r,
-                                                gp.z, gp.y, gp.x);
-                            }
+                            // copy si: tensor si / (2 NR), key granule (si / NR) % 2, region si % NR
+                            const int tens = si / (2 * L::NR), hg = (si / L::NR) % 2, r = si % L::NR;
+                            const int4 gp = ras.gpos[2 * tile + hg];
+                            mbar_expect_tx(B.stat, kGran);
+                            tma_load_5d(sm + (tens ? L::A1 : L::A0) + r * kTile + hg * kGran,
+                                        rmaps.m + (tens ? kRV : kRK) * kRasterKinds + gp.w, B.stat, 0, hh * L::NR + r,
+                                        gp.z, gp.y, gp.x);
                         } else {
-                            tma_load_3d(dst, lane == 30 ? &tmK : &tmV, B.stat, 0, (int)(row0 + 128 * tile), 0);
+                            mbar_expect_tx(B.stat, L::NR * kTile);
+                            tma_load_3d(sm + (si ? L::A1 : L::A0), si ? &tmV : &tmK, B.stat, 0,
+                                        (int)(row0 + 128 * tile), 0);
                         }
                         last_stat = kq;
                     }
@@ -761,16 +768,15 @@ k_bwd_dkdv_persist(const __grid_constant__ CUtensorMap tmK, const __grid_constan
                             mbar_expect_tx(full + stage, kXs);
                             bulk_load(xs + stage * kXs, nld + ((row0 + row) >> 6) * 128, kXs, full + stage);
                         } else {
-                            mbar_expect_tx(full + stage, L::NR * kGran);
                             uint8_t* dst = sm + L::RING + stage * L::STAGE + kind * L::NR * kGran;
                             if constexpr (RASTER) {
                                 const int4 gp = ras.gpos[row >> 6];
-                                const CUtensorMap* mr = rmaps.m + (kind ? kRdO : kRQ) * kRasterKinds + gp.w;
-#pragma unroll
-                                for (int r = 0; r < L::NR; ++r)
-                                    tma_load_5d(dst + r * kGran, mr, full + stage, 0, hh * L::NR + r, gp.z, gp.y,
-                                                gp.x);
+                                mbar_expect_tx(full + stage, kGran);
+                                tma_load_5d(dst + region * kGran,
+                                            rmaps.m + (kind ? kRdO : kRQ) * kRasterKinds + gp.w, full + stage, 0,
+                                            hh * L::NR + region, gp.z, gp.y, gp.x);
                             } else {
+                                mbar_expect_tx(full + stage, L::NR * kGran);
                                 tma_load_3d(dst, mg, full + stage, 0, (int)(row0 + row), 0);
                             }
                             }
@@ -1015,16 +1021,15 @@ k_bwd_dkdv_persist(const __grid_constant__ CUtensorMap tmK, const __grid_constan
                         fence_proxy_async_smem();
                     }
                     named_sync(2, 256);
-                    if (ok && wg == out && (warp & 3) == 0 && lane == 0) {
+                    // lane 0 of the warpgroup's first warp stores; in the raster layout
+                    // lanes 0 and 1 store the region's two key granules
+                    if (ok && wg == out && (warp & 3) == 0 && (lane == 0 || (RASTER && !part && lane == 1))) {
                         if (part) {
                             tma_store_3d(&tmPkv1, staging, 0, (slot * 2 + out) * 128, r);
                         } else if constexpr (RASTER) {
-                            const CUtensorMap* mr = rmaps.m + (out ? kRdV : kRdK) * kRasterKinds;
-#pragma unroll
-                            for (int hg = 0; hg < 2; ++hg) {
-                                const int4 gp = ras.gpos[2 * tile + hg];
-                                tma_store_5d(mr + gp.w, staging + hg * kGran, 0, hh * L::NR + r, gp.z, gp.y, gp.x);
-                            }
+                            const int4 gp = ras.gpos[2 * tile + lane];
+                            tma_store_5d(rmaps.m + (out ? kRdV : kRdK) * kRasterKinds + gp.w, staging + lane * kGran, 0,
+                                         hh * L::NR + r, gp.z, gp.y, gp.x);
                         } else {
                             tma_store_3d(out ? &tmdV1 : &tmdK1, staging, 0, (int)(row0 + 128 * tile), r);
                         }
