@@ -91,6 +91,15 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
         ::"r"(smem_u32(dst)), "l"(map), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
         : "memory");
 }
+// 4-D form (the zone statistics: channels, w, h, t)
+__device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1, int c2,
+                                            int c3) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5, %6}], "
+        "[%2];"
+        ::"r"(smem_u32(dst)), "l"(map), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+        : "memory");
+}
 // 5-D forms used for granules of the raster layout (coordinates: column in a
 // 64-column region, head-region, w, h, t)
 __device__ __forceinline__ void tma_load_5d(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1, int c2,
@@ -502,6 +511,22 @@ inline bool make_map_bf16_rows(CUtensorMap* m, const void* base, int64_t rows, i
     return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// A raster [T][H][W][D] tensor (bf16 or fp32) as the 4-D tensor (D, W, H, T):
+// box {128 bytes of channels, 8, 8, 8} = one 8x8x8 macro-zone's slice of
+// 128 / esz channels, landed unswizzled as [t][h][w][channel] (64 KB)
+inline bool make_map_zone(CUtensorMap* m, const void* base, bool bf16, int T, int H, int W, int64_t D) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    const uint64_t esz = bf16 ? 2 : 4, row = (uint64_t)D * esz;
+    cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)W, (cuuint64_t)H, (cuuint64_t)T};
+    cuuint64_t strides[3] = {(cuuint64_t)row, (cuuint64_t)(row * W), (cuuint64_t)(row * W * H)};
+    cuuint32_t box[4] = {(cuuint32_t)(128 / esz), 8, 8, 8};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    return enc(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<void*>(base),
+               dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // A raster [N][heads][d] bf16 tensor (N = T*H*W, raster token order) viewed

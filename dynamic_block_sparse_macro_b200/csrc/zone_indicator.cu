@@ -13,114 +13,188 @@
 //
 // Kernels (all reductions in a fixed order, no float atomics, so the result
 // is deterministic):
-//   k_zone_video    grid (D/CH, Z): one CTA per channel chunk x zone, chunks
-//                   fastest (the CTAs resident together read whole token rows
-//                   of one zone; zones fastest measured the same); warp w
-//                   holds temporal slice t = w of the zone, each lane CPL
-//                   channels, 64 tokens kept in registers for the two-pass
-//                   (mean first, then squared deviations) variance.
+//   k_zone_video    persistent, one CTA per SM over the (zone, 128-byte channel
+//                   chunk) items, chunks fastest; each item's 8x8x8 x 128-byte
+//                   slice lands in shared memory as one 64 KB TMA copy, two
+//                   stages deep; warp w holds temporal slice t = w of the
+//                   zone, each lane CPL channels, 64 tokens kept in registers
+//                   for the two-pass (mean first, then squared deviations)
+//                   variance.
 //   k_zone_audio    grid Z: one thread per token of the zone.
 //   k_zone_finalize one CTA: per-zone sums over chunks, grid maxima, outputs.
 #include <mutex>
 
+#include "attn_plan.cuh"
 #include "common.cuh"
+#include "sm100.cuh"
 
 namespace prism {
+
+using namespace sm100;
 
 template <typename T> struct VidTraits;
 template <> struct VidTraits<__nv_bfloat16> { static constexpr int CPL = 2; };  // 4 B per lane
 template <> struct VidTraits<float> { static constexpr int CPL = 1; };          // 4 B per lane
 
-// ws layout: video partial sums [Z][nchunk][4] then audio stats [Z][4]
+constexpr int kZoneStage = 512 * 128;                       // one zone x 128 bytes of channels
+constexpr int kZoneScratch = 2 * 8 * 8 * 64 * 4 + 8 * 64 * 4 + 8 * 4 * 4;   // sH, sW, sT, red (bf16 sizes)
+constexpr int kZoneSmem = 2 * kZoneStage + kZoneScratch + 64 + 1024;       // + barriers, + alignment
+
+// bounded wait on a copy this thread issued, for the wind-down after a timeout
+__device__ __forceinline__ void zone_drain(uint64_t* bar, uint32_t parity) {
+    const uint64_t t0 = globaltimer();
+    while (!mbar_try_wait(bar, parity) && globaltimer() - t0 < kWaitLimitNs) {
+    }
+}
+
+// ws layout: video partial sums [Z][nchunk][4] then audio stats [Z][4].
+// Persistent: CTA b takes items b, b + gridDim.x, ... (item = zone * nchunk +
+// chunk, chunks fastest, so the CTAs in flight together read whole token rows
+// of a few zones); each item's zone slice comes in as one 64 KB TMA copy, two
+// stages deep, the next-but-one copy issued as soon as a stage has been read.
+// If a copy never lands (2 s), the CTA marks its remaining items' sums NaN,
+// lets its copies in flight land (bounded) and exits.
 template <typename T>
-__global__ void __launch_bounds__(256, 2) k_zone_video(const T* __restrict__ V, int H, int W, int64_t D,
-                                                    int nchunk, float* __restrict__ part) {
+__global__ void __launch_bounds__(256, 1) k_zone_video(const __grid_constant__ CUtensorMap tmV, int H, int W,
+                                                       int nchunk, int n_items, float* __restrict__ part) {
     constexpr int CPL = VidTraits<T>::CPL;
-    constexpr int CH = 32 * CPL;                    // channels per CTA
-    __shared__ float sH[8][8][CH];                  // [t][h][c] row sums over w
-    __shared__ float sW[8][8][CH];                  // [t][w][c] column sums over h
-    __shared__ float sT[8][CH];                     // [t][c] slice sums
-    __shared__ float red[8][4];
+    constexpr int CH = 32 * CPL;                    // channels per item (128 bytes)
+    extern __shared__ uint8_t zraw[];
+    uint8_t* zs = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(zraw) + 1023) & ~uintptr_t(1023));
+    float(*sH)[8][CH] = reinterpret_cast<float(*)[8][CH]>(zs + 2 * kZoneStage);              // [t][h][c]
+    float(*sW)[8][CH] = reinterpret_cast<float(*)[8][CH]>(zs + 2 * kZoneStage + 256 * CH);    // [t][w][c]
+    float(*sT)[CH] = reinterpret_cast<float(*)[CH]>(zs + 2 * kZoneStage + 512 * CH);          // [t][c]
+    float(*red)[4] = reinterpret_cast<float(*)[4]>(zs + 2 * kZoneStage + 544 * CH);
+    uint64_t* full = reinterpret_cast<uint64_t*>(zs + 2 * kZoneStage + kZoneScratch);
+    int* abort_flag = reinterpret_cast<int*>(full + 2);
+    uint32_t* wstat = reinterpret_cast<uint32_t*>(abort_flag + 1);
 
     const int lane = threadIdx.x & 31, t = threadIdx.x >> 5;
-    const int chunk = blockIdx.x, m = blockIdx.y;
     const int ZH = H / 8, ZW = W / 8;
-    const int zt = m / (ZH * ZW), zh = (m / ZW) % ZH, zw = m % ZW;
-    const int64_t c0 = (int64_t)chunk * CH + lane * CPL;
-    const int64_t row0 = ((int64_t)(zt * 8 + t) * H + zh * 8) * W + zw * 8;
-
-    // raw storage: one 32-bit word per token (a bf16 pair or one float) keeps
-    // the zone slice at 64 registers for the second (deviation) pass
-    uint32_t raw[8][8];
-#pragma unroll
-    for (int h = 0; h < 8; ++h)
-#pragma unroll
-        for (int w = 0; w < 8; ++w)
-            raw[h][w] = __ldg(reinterpret_cast<const unsigned int*>(V + (row0 + (int64_t)h * W + w) * D + c0));
-    auto val = [&](int h, int w, int k) -> float {
-        if constexpr (CPL == 2) return __uint_as_float(k == 0 ? (raw[h][w] << 16) : (raw[h][w] & 0xffff0000u));
-        else return __uint_as_float(raw[h][w]);
+    auto issue = [&](int it, int buf) {
+        const int chunk = it % nchunk, m = it / nchunk;
+        const int zt = m / (ZH * ZW), zh = (m / ZW) % ZH, zw = m % ZW;
+        mbar_expect_tx(full + buf, kZoneStage);
+        tma_load_4d(zs + buf * kZoneStage, &tmV, full + buf, chunk * CH, zw * 8, zh * 8, zt * 8);
     };
-
-#pragma unroll
-    for (int k = 0; k < CPL; ++k) {
-        float tot = 0.f;
-#pragma unroll
-        for (int h = 0; h < 8; ++h) {
-            float rs = 0.f;
-#pragma unroll
-            for (int w = 0; w < 8; ++w) rs += val(h, w, k);
-            sH[t][h][lane * CPL + k] = rs;
-            tot += rs;
-        }
-#pragma unroll
-        for (int w = 0; w < 8; ++w) {
-            float cs = 0.f;
-#pragma unroll
-            for (int h = 0; h < 8; ++h) cs += val(h, w, k);
-            sW[t][w][lane * CPL + k] = cs;
-        }
-        sT[t][lane * CPL + k] = tot;
+    if (threadIdx.x == 0) {
+        mbar_init(full, 1);
+        mbar_init(full + 1, 1);
+        *abort_flag = 0;
+        *wstat = 0;
+        fence_mbar_init();
     }
     __syncthreads();
+    if (threadIdx.x == 0)
+        for (int b = 0; b < 2; ++b)
+            if (blockIdx.x + b * gridDim.x < n_items) issue(blockIdx.x + b * gridDim.x, b);
 
-    // this thread handles profile index i = t along every axis
-    float aT = 0.f, aH = 0.f, aW = 0.f, aTok = 0.f;
-#pragma unroll
-    for (int k = 0; k < CPL; ++k) {
-        const int c = lane * CPL + k;
-        float zsum = 0.f, hsum = 0.f, wsum = 0.f;
-#pragma unroll
-        for (int tt = 0; tt < 8; ++tt) {
-            zsum += sT[tt][c];
-            hsum += sH[tt][t][c];
-            wsum += sW[tt][t][c];
-        }
-        const float mu = zsum * (1.f / 512.f);
-        const float pT = sT[t][c] * (1.f / 64.f) - mu;
-        const float pH = hsum * (1.f / 64.f) - mu;
-        const float pW = wsum * (1.f / 64.f) - mu;
-        aT += pT * pT;
-        aH += pH * pH;
-        aW += pW * pW;
-        float tv = 0.f;
+    for (int it = blockIdx.x, k = 0; it < n_items; it += gridDim.x, ++k) {
+        const int buf = k & 1;
+        const bool got = mbar_wait(full + buf, (uint32_t)(k >> 1) & 1u, abort_flag, wstat);
+        // one 32-bit word per token (a bf16 pair or one float) of this warp's slice t
+        // keeps the slice at 64 registers for the second (deviation) pass
+        const uint32_t* src = reinterpret_cast<const uint32_t*>(zs + buf * kZoneStage) + t * 2048 + lane;
+        uint32_t raw[8][8];
 #pragma unroll
         for (int h = 0; h < 8; ++h)
 #pragma unroll
-            for (int w = 0; w < 8; ++w) {
-                float dv = val(h, w, k) - mu;
-                tv += dv * dv;
+            for (int w = 0; w < 8; ++w) raw[h][w] = src[(h * 8 + w) * 32];
+        // the stage has been read by every thread, and sH, sW, sT, red are free
+        if (__syncthreads_or(!got)) {
+            if (threadIdx.x == 0) {
+                zone_drain(full + buf, (uint32_t)(k >> 1) & 1u);
+                if (it + gridDim.x < n_items) zone_drain(full + (buf ^ 1), (uint32_t)((k + 1) >> 1) & 1u);
             }
-        aTok += tv;
+            for (int r = it; r < n_items; r += gridDim.x)
+                if (threadIdx.x < 4) part[(int64_t)r * 4 + threadIdx.x] = __int_as_float(0x7fc00000);
+            return;
+        }
+        if (threadIdx.x == 0 && it + 2 * gridDim.x < n_items) issue(it + 2 * gridDim.x, buf);
+        auto val = [&](int h, int w, int c) -> float {
+            if constexpr (CPL == 2) return __uint_as_float(c == 0 ? (raw[h][w] << 16) : (raw[h][w] & 0xffff0000u));
+            else return __uint_as_float(raw[h][w]);
+        };
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) {
+            float tot = 0.f;
+#pragma unroll
+            for (int h = 0; h < 8; ++h) {
+                float rs = 0.f;
+#pragma unroll
+                for (int w = 0; w < 8; ++w) rs += val(h, w, c);
+                sH[t][h][lane * CPL + c] = rs;
+                tot += rs;
+            }
+#pragma unroll
+            for (int w = 0; w < 8; ++w) {
+                float cs = 0.f;
+#pragma unroll
+                for (int h = 0; h < 8; ++h) cs += val(h, w, c);
+                sW[t][w][lane * CPL + c] = cs;
+            }
+            sT[t][lane * CPL + c] = tot;
+        }
+        __syncthreads();
+
+        // this thread handles profile index i = t along every axis
+        float aT = 0.f, aH = 0.f, aW = 0.f, aTok = 0.f;
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) {
+            const int ch = lane * CPL + c;
+            float zsum = 0.f, hsum = 0.f, wsum = 0.f;
+#pragma unroll
+            for (int tt = 0; tt < 8; ++tt) {
+                zsum += sT[tt][ch];
+                hsum += sH[tt][t][ch];
+                wsum += sW[tt][t][ch];
+            }
+            const float mu = zsum * (1.f / 512.f);
+            const float pT = sT[t][ch] * (1.f / 64.f) - mu;
+            const float pH = hsum * (1.f / 64.f) - mu;
+            const float pW = wsum * (1.f / 64.f) - mu;
+            aT += pT * pT;
+            aH += pH * pH;
+            aW += pW * pW;
+            float tv = 0.f;
+#pragma unroll
+            for (int h = 0; h < 8; ++h)
+#pragma unroll
+                for (int w = 0; w < 8; ++w) {
+                    const float dv = val(h, w, c) - mu;
+                    tv += dv * dv;
+                }
+            aTok += tv;
+        }
+        aT = warp_sum(aT); aH = warp_sum(aH); aW = warp_sum(aW); aTok = warp_sum(aTok);
+        if (lane == 0) { red[t][0] = aT; red[t][1] = aH; red[t][2] = aW; red[t][3] = aTok; }
+        __syncthreads();
+        if (threadIdx.x < 4) {
+            float sum = 0.f;
+            for (int q = 0; q < 8; ++q) sum += red[q][threadIdx.x];
+            part[(int64_t)it * 4 + threadIdx.x] = sum;
+        }
     }
-    aT = warp_sum(aT); aH = warp_sum(aH); aW = warp_sum(aW); aTok = warp_sum(aTok);
-    if (lane == 0) { red[t][0] = aT; red[t][1] = aH; red[t][2] = aW; red[t][3] = aTok; }
-    __syncthreads();
-    if (threadIdx.x < 4) {
-        float s = 0.f;
-        for (int k = 0; k < 8; ++k) s += red[k][threadIdx.x];
-        part[((int64_t)m * nchunk + chunk) * 4 + threadIdx.x] = s;
+}
+
+// Launch of k_zone_video over V ([T][H][W][D] raster, bf16 or fp32)
+static prism_status_t launch_zone_video(const Dims& d, const void* V, int nchunk, float* part, cudaStream_t s) {
+    CUtensorMap tm;
+    if (!make_map_zone(&tm, V, d.dtype == PRISM_BF16, d.T, d.H, d.W, d.D)) return PRISM_ERR_CUDA;
+    const int n_items = (int)(d.Z * nchunk);
+    const int grid = n_items < device_sms() ? n_items : device_sms();
+    if (d.dtype == PRISM_BF16) {
+        if (cudaFuncSetAttribute(k_zone_video<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kZoneSmem) != cudaSuccess)
+            return PRISM_ERR_CUDA;
+        k_zone_video<__nv_bfloat16><<<grid, 256, kZoneSmem, s>>>(tm, d.H, d.W, nchunk, n_items, part);
+    } else {
+        if (cudaFuncSetAttribute(k_zone_video<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, kZoneSmem) !=
+            cudaSuccess)
+            return PRISM_ERR_CUDA;
+        k_zone_video<float><<<grid, 256, kZoneSmem, s>>>(tm, d.H, d.W, nchunk, n_items, part);
     }
+    return PRISM_OK;
 }
 
 template <typename T>
@@ -268,17 +342,14 @@ extern "C" prism_status_t prism_zone_indicator_ex(const prism_problem_t* prob, c
     float* part = (float*)ws;
     float* astat = part + d.Z * nchunk * 4;
     float* vsum = astat + d.Z * 4;
-    dim3 gv((unsigned)nchunk, (unsigned)d.Z);                 // Z <= 2^24 / 512 = 32768 < 65536
-    if (d.dtype == PRISM_BF16) {
-        k_zone_video<__nv_bfloat16><<<gv, 256, 0, stream>>>((const __nv_bfloat16*)V, d.H, d.W, d.D,
-                                                             nchunk, part);
+    st = launch_zone_video(d, V, nchunk, part, stream);
+    if (st != PRISM_OK) return st;
+    if (d.dtype == PRISM_BF16)
         k_zone_audio<__nv_bfloat16><<<(unsigned)d.Z, 512, 0, stream>>>((const __nv_bfloat16*)hhat,
                                                                        d.H, d.W, d.Da, astat);
-    } else {
-        k_zone_video<float><<<gv, 256, 0, stream>>>((const float*)V, d.H, d.W, d.D, nchunk, part);
+    else
         k_zone_audio<float><<<(unsigned)d.Z, 512, 0, stream>>>((const float*)hhat, d.H, d.W, d.Da,
                                                                astat);
-    }
     k_zone_finalize<<<1, 1024, 0, stream>>>(part, astat, (int)d.Z, nchunk, 1.f / (float)d.D, eps, g,
                                             rho, abar, zone_stats, vsum, guidance);
     return launch_status(3);
@@ -322,17 +393,14 @@ extern "C" prism_status_t prism_zone_partials(const prism_problem_t* prob_local,
     const int CH = d.dtype == PRISM_BF16 ? 64 : 32;
     const int nchunk = (int)(d.D / CH);
     float* part = (float*)ws;
-    dim3 gv((unsigned)nchunk, (unsigned)d.Z);
-    if (d.dtype == PRISM_BF16) {
-        k_zone_video<__nv_bfloat16><<<gv, 256, 0, stream>>>((const __nv_bfloat16*)V_local, d.H, d.W, d.D,
-                                                             nchunk, part);
+    st = launch_zone_video(d, V_local, nchunk, part, stream);
+    if (st != PRISM_OK) return st;
+    if (d.dtype == PRISM_BF16)
         k_zone_audio<__nv_bfloat16><<<(unsigned)d.Z, 512, 0, stream>>>((const __nv_bfloat16*)hhat, d.H, d.W,
                                                                        d.Da, partials + d.Z * 4);
-    } else {
-        k_zone_video<float><<<gv, 256, 0, stream>>>((const float*)V_local, d.H, d.W, d.D, nchunk, part);
+    else
         k_zone_audio<float><<<(unsigned)d.Z, 512, 0, stream>>>((const float*)hhat, d.H, d.W, d.Da,
                                                                partials + d.Z * 4);
-    }
     k_zone_chunk_sum<<<(unsigned)((d.Z * 4 + 255) / 256), 256, 0, stream>>>(part, (int)d.Z, nchunk, partials);
     return launch_status(3);
 }
