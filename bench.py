@@ -42,7 +42,7 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM bytes (read + write) of one backward call, by (config, heads), from an ncu capture of
 # the backward kernels (profiles/attn_kernels_2k_4heads.md: 4 heads scaled by 6, plus the
 # Delta kernel's algorithmic 5.5 GB)
-BWD_DRAM_BYTES = {("2k", 24): 33.5e9}
+BWD_DRAM_BYTES = {("2k", 24): 33.2e9}
 
 
 def metric_name(cfg, fwd_only):
@@ -380,7 +380,9 @@ def bench_prism(args, cfg, rank, world, local_rank):
     bwd_ach = 2.5 * fl["F_fwd"] / (stage_ms["attn_bwd"] * 1e-3) / 1e12
     dom = "attn_bwd" if stage_ms["attn_bwd"] >= stage_ms["attn_fwd"] else "attn_fwd"
     ach = bwd_ach if dom == "attn_bwd" else fwd_ach
-    traffic = BWD_DRAM_BYTES.get((cfg.name, cfg.heads)) if dom == "attn_bwd" and not args.dense else None
+    # the capture is of the blocked-operand kernels: none for the raster ones
+    traffic = (BWD_DRAM_BYTES.get((cfg.name, cfg.heads)) if dom == "attn_bwd" and not args.dense and not args.raster
+               else None)
     # the attention kernels run at 1.85-1.97 GHz (clocks below): the burst peak is the fair
     # denominator; the sustained one (measured at ~1.33 GHz under the power cap) is reported beside it
     peak = peaks["bf16_tflops"]
