@@ -18,7 +18,10 @@
 //               warp, one elected lane):
 //               S = Q K^T (M=128, N=128, fp32 in TMEM), then O += P V with
 //               P read from TMEM (aliasing S) and V MN-major from shared memory.
-//   warps 2-5   one query row per thread: S row from TMEM, masked online
+//   warps 2-9   two softmax warpgroups, one query row per thread, warpgroup g
+//               owning key granule g of every chunk (S columns 64 g ..) and O
+//               columns (D/2) g ..; the row maxima are exchanged through shared
+//               memory once a chunk.  Per row: S from TMEM, masked online
 //               softmax in the exp2 domain with lazy rescaling (the running
 //               max only moves when it grows by more than 2^8), packed fp32
 //               arithmetic, P as bf16 back into TMEM, then the epilogue.
@@ -39,7 +42,7 @@ constexpr int kRegion = 128 * 128;         // bytes of a 128-row x 64-col bf16 t
 constexpr int kGranBytes = 64 * 128;       // 64 rows x 64 cols bf16
 constexpr uint32_t kTmemCols = 256;
 constexpr uint32_t kColO = 0;              // O accumulator: D columns
-constexpr uint32_t kColS = 128;            // S (fp32, 128 columns); P (bf16) aliases its first 64
+constexpr uint32_t kColS = 128;            // S (fp32, 128 columns); P (bf16) over the first 32 of each granule's 64
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
@@ -51,7 +54,8 @@ struct FwdLayout {
     static constexpr int K = NR * kRegion;
     static constexpr int V = 2 * NR * kRegion;
     static constexpr int CTRL = 3 * NR * kRegion;
-    static constexpr int ROWS = CTRL + 256;        // two selection rows of SW words follow
+    static constexpr int XCH = CTRL + 256;         // [3][2][128] floats: row maxima (two parities), denominators
+    static constexpr int ROWS = XCH + 3 * 2 * 128 * 4;   // two selection rows of SW words follow
     // bytes to request: + slack for 1024-byte alignment; at least 80 KB so that
     // no more than two CTAs (2 x 256 of the SM's 512 TMEM columns) share an SM
     static int alloc(int SW) {
@@ -77,7 +81,7 @@ struct RasterOps {
 };
 
 template <int D, bool RASTER>
-__global__ void __launch_bounds__(192, 2)
+__global__ void __launch_bounds__(320, 2)
 k_attn_fwd_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
                  const __grid_constant__ CUtensorMap tmOf, const __grid_constant__ CUtensorMap tmPo,
@@ -125,7 +129,7 @@ k_attn_fwd_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         mbar_init(bar_vf, L::NR);
         mbar_init(bar_ve, 1);
         mbar_init(bar_s, 1);
-        mbar_init(bar_p, 128);
+        mbar_init(bar_p, 256);
         mbar_init(bar_o, 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -218,7 +222,8 @@ k_attn_fwd_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                 tc_fence_after();
 #pragma unroll
                 for (int k = 0; k < 8; ++k)
-                    mma_ts_w(tbase + kColO, tbase + kColS + 8 * k, sdesc_sw128(aV + k * 2048, kRegion, 1024), idO,
+                    mma_ts_w(tbase + kColO, tbase + kColS + 64 * (k >> 2) + 8 * (k & 3),
+                             sdesc_sw128(aV + k * 2048, kRegion, 1024), idO,
                              (c > 0 || k > 0) ? 1u : 0u);
                 tc_commit_w(bar_ve);
             }
@@ -230,10 +235,17 @@ k_attn_fwd_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         }
     } else {
         // ---------------------------------------------------- softmax + epilogue
+        // Warpgroup g (warps 2-5: 0, 6-9: 1) owns key granule g of every chunk; both keep
+        // the same running max (the row maxima are exchanged through shared memory, two
+        // buffers by chunk parity so that one barrier a chunk suffices) and each sums its
+        // own part of the denominator, added in a fixed order at the end.
+        const int g = (warp - 2) >> 2;
         const int sub = warp & 3;                          // TMEM lane quarter of this warp
         const int row = sub * 32 + lane;                   // query row within the tile
         const uint32_t tl = tbase + ((uint32_t)(sub * 32) << 16);
         const int half = row >> 6;
+        float* xmax = reinterpret_cast<float*>(sm + L::XCH);   // [parity][g][128]
+        float* xden = xmax + 2 * 2 * 128;                      // [g][128]
         const float sl2 = scale * kLog2e;
         const uint64_t sl2x2 = f2pack(sl2, sl2);
         float m_run = -INFINITY, l = 0.f;
@@ -253,30 +265,38 @@ k_attn_fwd_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                 mk = ma | (mb << 2);
             }
             mk = __shfl_sync(0xffffffffu, mk, 0);
-            const bool v0 = (mk >> half) & 1u, v1 = (mk >> (2 + half)) & 1u;   // warp-uniform
-            const bool got = mbar_wait(bar_s, c & 1, abort_flag, dev_status);
-            if (!__all_sync(0xffffffffu, got)) { ok = false; break; }   // warp-uniform exit
-            tc_fence_after();
-            // pass 1: row max over the valid columns
+            const bool vg = (mk >> (2 * g + half)) & 1u;                     // warp-uniform
+            const uint32_t tS = tl + kColS + 64 * g;                          // this granule's S
+            bool got = ok && mbar_wait(bar_s, c & 1, abort_flag, dev_status);
+            got = __all_sync(0xffffffffu, got);
+            if (got) tc_fence_after();
+            // pass 1: this granule's row max, then the other warpgroup's
             float mx = -INFINITY;
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                if (!(q < 2 ? v0 : v1)) continue;
+            if (got && vg) {
                 uint32_t r[32];
-                tmem_ld32(tl + kColS + 32 * q, r);
-                tmem_wait_ld();
 #pragma unroll
-                for (int i = 0; i < 32; i += 2) mx = fmax3(mx, __uint_as_float(r[i]), __uint_as_float(r[i + 1]));
+                for (int q = 0; q < 2; ++q) {
+                    tmem_ld32(tS + 32 * q, r);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 32; i += 2) mx = fmax3(mx, __uint_as_float(r[i]), __uint_as_float(r[i + 1]));
+                }
             }
+            xmax[((c & 1) * 2 + g) * 128 + row] = mx;
+            named_sync(2, 256);                                // every thread, also after a timeout
+            mx = fmaxf(mx, xmax[((c & 1) * 2 + (g ^ 1)) * 128 + row]);
+            ok = ok && got;
+            if (!ok) continue;                                 // winds down: barriers only
             const float mx2 = mx * sl2;
             const bool need = mx2 > m_run + kRescaleThreshold || (m_run == -INFINITY && mx2 > -INFINITY);
             const float alpha = need ? ex2(m_run - mx2) : 1.f;      // 0 when m_run = -inf
             // O holds chunks < c, all complete (S of chunk c was issued after them).
-            // TMEM access is warp-collective: the whole warp rescales if any row must.
+            // TMEM access is warp-collective: the whole warp rescales if any row must (both
+            // warpgroups see the same rows and maxima, so they agree), each its O columns.
             if (c > 0 && __any_sync(0xffffffffu, need && m_run > -INFINITY)) {
                 const uint64_t a2 = f2pack(alpha, alpha);
 #pragma unroll
-                for (int q = 0; q < D / 32; ++q) {
+                for (int q = (D / 64) * g; q < (D / 64) * (g + 1); ++q) {
                     uint32_t r[32];
                     tmem_ld32(tl + kColO + 32 * q, r);
                     tmem_wait_ld();
@@ -294,36 +314,32 @@ k_attn_fwd_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                 l *= alpha;
                 m_run = mx2;
             }
-            // pass 2: P = 2^(s * scale * log2e - m) as bf16 into the first 64 columns of S
+            // pass 2: P = 2^(s * scale * log2e - m) as bf16 over the first 32 of the granule's
+            // own 64 S columns (already read), 32 S columns per load
+            const bool v = vg && m_run > -INFINITY;
             const uint64_t negm = f2pack(-m_run, -m_run);
             uint64_t rs2 = f2pack(0.f, 0.f);
 #pragma unroll
-            for (int hq = 0; hq < 2; ++hq) {
-                const bool v = (hq == 0 ? v0 : v1) && m_run > -INFINITY;
-                uint32_t pk[32];
-                if (__any_sync(0xffffffffu, v)) {
+            for (int q = 0; q < 2; ++q) {
+                uint32_t pk[16];
+                if (v) {
+                    uint32_t r[32];
+                    tmem_ld32(tS + 32 * q, r);
+                    tmem_wait_ld();
 #pragma unroll
-                    for (int q2 = 0; q2 < 2; ++q2) {
-                        uint32_t r[32];
-                        tmem_ld32(tl + kColS + 64 * hq + 32 * q2, r);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int i = 0; i < 16; ++i) {
-                            float x0, x1;
-                            f2unpack(ffma2(f2pack(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1])), sl2x2,
-                                           negm),
-                                     x0, x1);
-                            float p0 = ex2(x0), p1 = ex2(x1);
-                            if (!v) { p0 = 0.f; p1 = 0.f; }
-                            rs2 = fadd2(rs2, f2pack(p0, p1));
-                            pk[16 * q2 + i] = pack_bf16x2(p0, p1);
-                        }
+                    for (int i = 0; i < 16; ++i) {
+                        float x0, x1;
+                        f2unpack(ffma2(f2pack(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1])), sl2x2, negm),
+                                 x0, x1);
+                        const float p0 = ex2(x0), p1 = ex2(x1);
+                        rs2 = fadd2(rs2, f2pack(p0, p1));
+                        pk[i] = pack_bf16x2(p0, p1);
                     }
                 } else {
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) pk[i] = 0u;
+                    for (int i = 0; i < 16; ++i) pk[i] = 0u;
                 }
-                tmem_st32(tl + kColS + 32 * hq, pk);
+                tmem_st16(tl + kColS + 64 * g + 16 * q, pk);
             }
             float rsa, rsb;
             f2unpack(rs2, rsa, rsb);
@@ -334,19 +350,23 @@ k_attn_fwd_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         }
         const bool fin = __all_sync(0xffffffffu, ok && mbar_wait(bar_o, 0, abort_flag, dev_status));
         if (fin) tc_fence_after();
+        // the denominator: the two warpgroups' parts, added in a fixed order
+        xden[g * 128 + row] = l;
+        named_sync(2, 256);
+        const float lt = xden[row] + xden[128 + row];
         // Epilogue.  Every MMA is complete, so Q, K and V are free: O (bf16) is
         // staged in the Q buffer and the fp32 O or a split tile's partial in the
         // K and V buffers, as 16-byte chunks in the 128-byte-swizzled image of the
-        // whole-row maps, and each goes out in one TMA store.  Every thread runs
-        // the barrier, also after a timeout.
+        // whole-row maps, each warpgroup its own columns, and each goes out in one
+        // TMA store.  Every thread runs the barrier, also after a timeout.
         const int64_t grow = row0 + 128 * tile + row;
         const bool part = slot >= 0;
-        const bool zero = part ? nch == 0 : (!(l > 0.f) || nch == 0);   // nothing selected: O = 0
-        const float inv = l > 0.f ? 1.f / l : 0.f;
+        const bool zero = part ? nch == 0 : (!(lt > 0.f) || nch == 0);   // nothing selected: O = 0
+        const float inv = lt > 0.f ? 1.f / lt : 0.f;
         const uint32_t sw = (uint32_t)(row & 7);
         if (fin) {
 #pragma unroll 1
-            for (int q = 0; q < D / 32; ++q) {
+            for (int q = (D / 64) * g; q < (D / 64) * (g + 1); ++q) {
                 uint32_t r[32];
                 if (zero) {                                 // TMEM never written
 #pragma unroll
@@ -358,36 +378,38 @@ k_attn_fwd_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                 if (!part) {
 #pragma unroll
                     for (int k = 0; k < 4; ++k) {           // 4 chunks of 8 bf16
-                        const int g = 4 * q + k;
-                        uint4 v;
-                        v.x = pack_bf16x2(__uint_as_float(r[8 * k + 0]) * inv, __uint_as_float(r[8 * k + 1]) * inv);
-                        v.y = pack_bf16x2(__uint_as_float(r[8 * k + 2]) * inv, __uint_as_float(r[8 * k + 3]) * inv);
-                        v.z = pack_bf16x2(__uint_as_float(r[8 * k + 4]) * inv, __uint_as_float(r[8 * k + 5]) * inv);
-                        v.w = pack_bf16x2(__uint_as_float(r[8 * k + 6]) * inv, __uint_as_float(r[8 * k + 7]) * inv);
-                        *reinterpret_cast<uint4*>(sQ + (g >> 3) * kRegion + row * 128 + (((g & 7) ^ sw) << 4)) = v;
+                        const int gc = 4 * q + k;
+                        uint4 v4;
+                        v4.x = pack_bf16x2(__uint_as_float(r[8 * k + 0]) * inv, __uint_as_float(r[8 * k + 1]) * inv);
+                        v4.y = pack_bf16x2(__uint_as_float(r[8 * k + 2]) * inv, __uint_as_float(r[8 * k + 3]) * inv);
+                        v4.z = pack_bf16x2(__uint_as_float(r[8 * k + 4]) * inv, __uint_as_float(r[8 * k + 5]) * inv);
+                        v4.w = pack_bf16x2(__uint_as_float(r[8 * k + 6]) * inv, __uint_as_float(r[8 * k + 7]) * inv);
+                        *reinterpret_cast<uint4*>(sQ + (gc >> 3) * kRegion + row * 128 + (((gc & 7) ^ sw) << 4)) = v4;
                     }
                 }
                 if (part || o_f32) {
                     const float mul = part ? 1.f : inv;     // the partial stays unnormalised
 #pragma unroll
                     for (int k = 0; k < 8; ++k) {           // 8 chunks of 4 fp32
-                        const int g = 8 * q + k;
-                        const float4 v = make_float4(__uint_as_float(r[4 * k]) * mul, __uint_as_float(r[4 * k + 1]) * mul,
-                                                     __uint_as_float(r[4 * k + 2]) * mul,
-                                                     __uint_as_float(r[4 * k + 3]) * mul);
-                        *reinterpret_cast<float4*>(sK + (g >> 3) * kRegion + row * 128 + (((g & 7) ^ sw) << 4)) = v;
+                        const int gc = 8 * q + k;
+                        const float4 v4 = make_float4(__uint_as_float(r[4 * k]) * mul, __uint_as_float(r[4 * k + 1]) * mul,
+                                                      __uint_as_float(r[4 * k + 2]) * mul,
+                                                      __uint_as_float(r[4 * k + 3]) * mul);
+                        *reinterpret_cast<float4*>(sK + (gc >> 3) * kRegion + row * 128 + (((gc & 7) ^ sw) << 4)) = v4;
                     }
                 }
             }
             fence_proxy_async_smem();
-            if (!part) {
-                if (lse) lse[grow] = l > 0.f ? (m_run + log2f(l)) * kLn2 : -INFINITY;
-            } else {
-                parts.m[(int64_t)slot * 128 + row] = m_run;
-                parts.l[(int64_t)slot * 128 + row] = l;
+            if (g == 0) {
+                if (!part) {
+                    if (lse) lse[grow] = lt > 0.f ? (m_run + log2f(lt)) * kLn2 : -INFINITY;
+                } else {
+                    parts.m[(int64_t)slot * 128 + row] = m_run;
+                    parts.l[(int64_t)slot * 128 + row] = lt;
+                }
             }
         }
-        named_sync(1, 128);
+        named_sync(1, 256);
         if constexpr (RASTER) {
             // O back to the raster layout: one box per (query granule, region), a lane each;
             // the fp32 O (kept in permutation order) and the partials as whole-row tiles
@@ -498,7 +520,7 @@ prism_status_t launch_fwd(const Dims& d, const void* Qp, const void* Kp, const v
     const int smem = FwdLayout<D>::alloc((int)d.SW);
     if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return PRISM_ERR_CUDA;
-    k<<<(unsigned)w.plan.items_max, 192, smem, s>>>(mQ, mK, mV, mO, mOf, mPo, rm, ras, gsel, w.plan.hdr, w.plan.items,
+    k<<<(unsigned)w.plan.items_max, 320, smem, s>>>(mQ, mK, mV, mO, mOf, mPo, rm, ras, gsel, w.plan.hdr, w.plan.items,
                                                     w.parts, d.N, d.MB, (int)d.SW, scale, (__nv_bfloat16*)Op, lse,
                                                     o_f32, dev_status);
     st = launch_status(1);
