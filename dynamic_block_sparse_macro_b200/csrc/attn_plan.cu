@@ -1,9 +1,10 @@
 // Work planning for the tensor-core attention kernels.
 //
 // A tile's work is the union of the granule-level selection rows of its
-// 64-row granules (two: forward and backward both use 128-row tiles).  That union is data dependent and very uneven (a
-// query block with flat block probabilities makes Top-p select most keys), so
-// one CTA per tile would leave a few CTAs running long after the rest.  The
+// 64-row granules (two: forward and backward both use 128-row tiles).  That
+// union is data dependent and very uneven (a query block with flat block
+// probabilities makes Top-p select most keys), so one CTA per tile would
+// leave a few CTAs running long after the rest.  The
 // plan cuts every tile into segments of at most `seg` work units, choosing
 // seg from the total so that the item count stays near a fixed target, and
 // gives each segment of a split tile a slot for its partial result; a
