@@ -25,8 +25,11 @@
 // stages, buffers and barrier phases carry across item edges, so the next
 // item's loads and first products overlap the current item's epilogue.
 // Roles: warp 0 TMA (one lane per ring stage and stream, one whole-row copy
-// per granule), warp 1 TMEM allocation + MMA issue (the whole warp, one
-// elected lane issues), the other warps one tile row per thread.
+// per granule), warp 1 TMEM allocation; MMA issue (the whole warp, one elected
+// lane issues) by warps 1, 10, 11 in dQ (S, dP, dQ) and warps 1, 2 in dK/dV
+// (S^T and dP^T; dV and dK), one accumulation chain each, so that one warp's
+// barrier waits leave the others' MMAs in the tensor pipe; the elementwise
+// warps one tile row per thread.
 // Every wait is bounded; a timeout sets PRISM_DEV_TIMEOUT.
 #include "attn_plan.cuh"
 #include "common.cuh"
@@ -605,7 +608,8 @@ struct BarsKV {
     uint64_t* stat;            // K, V tiles of a non-empty item landed (2 copies)
     uint64_t* kv_free;         // the item's last S^T/dP^T MMAs complete
     uint64_t* fin;
-    uint64_t* drain;
+    uint64_t* drain;           // [2] teardown after an abort, per MMA-issuing warp
+    uint64_t* kv_done;         // [2] dV/dK MMAs of the buffer's granule complete (its P^T, dS^T read)
     uint64_t* rows_full;       // [2] (32 arrivals)
     uint64_t* rows_empty;      // [2] (8 arrivals: one per elementwise warp)
     uint32_t* tmem_slot;
@@ -624,13 +628,14 @@ __device__ __forceinline__ BarsKV carve_kv(uint8_t* ctrl) {
     r.kv_free = b + 4 * kStages + 5;
     r.fin = b + 4 * kStages + 6;
     r.drain = b + 4 * kStages + 7;
-    r.rows_full = b + 4 * kStages + 8;
-    r.rows_empty = b + 4 * kStages + 10;
-    r.tmem_slot = reinterpret_cast<uint32_t*>(b + 4 * kStages + 12);
+    r.rows_full = b + 4 * kStages + 9;
+    r.rows_empty = b + 4 * kStages + 11;
+    r.kv_done = b + 4 * kStages + 13;
+    r.tmem_slot = reinterpret_cast<uint32_t*>(b + 4 * kStages + 15);
     r.abort_flag = reinterpret_cast<volatile int*>(r.tmem_slot + 1);
     return r;
 }
-static_assert((4 * kStages + 12) * 8 + 8 <= kCtrl, "barriers overflow the control block");
+static_assert((4 * kStages + 15) * 8 + 8 <= kCtrl, "barriers overflow the control block");
 
 template <int D, bool RASTER>
 __global__ void __launch_bounds__(384, 1)
@@ -669,11 +674,12 @@ k_bwd_dkdv_persist(const __grid_constant__ CUtensorMap tmK, const __grid_constan
             mbar_init(B.elem + b, 256);
             mbar_init(B.rows_full + b, 32);
             mbar_init(B.rows_empty + b, 8);
+            mbar_init(B.kv_done + b, 1);
+            mbar_init(B.drain + b, 1);
         }
         mbar_init(B.stat, kStatLanes);
         mbar_init(B.kv_free, 1);
         mbar_init(B.fin, 1);
-        mbar_init(B.drain, 1);
         *B.abort_flag = 0;
         fence_mbar_init();
     }
@@ -800,8 +806,17 @@ k_bwd_dkdv_persist(const __grid_constant__ CUtensorMap tmK, const __grid_constan
             volatile int no_abort = 0;                     // bounded: the other lane's copy may be missing
             mbar_wait(B.stat, (uint32_t)last_stat & 1, &no_abort, dev_status);
         }
-      } else if (warp == 1) {
-        // ---------------------------------------------------------------- MMA (whole warp, elected issue)
+      } else if (warp == 1 || warp == 2) {
+        // ---------------------------------------------------------------- MMA, two warps
+        // Two accumulation chains, each issued in order by one warp (whole warp,
+        // elected issue): warp 1 S^T = K Q^T and dP^T = V dO^T, warp 2 dV += P^T dO
+        // and dK += dS^T Q, so that one warp's waits leave the other's MMAs in the
+        // tensor pipe.  Per TMEM buffer b and its u-th use (granule GG, b = GG & 1,
+        // u = GG >> 1): S^T/dP^T(GG) wait kv_done(b) of use u - 1 (the previous
+        // granule's P^T and dS^T in those columns read), dV/dK(GG) wait elem(b) of
+        // use u.  No barrier can run two phases ahead of its waiter: every phase
+        // needs the waiter's own earlier issue.
+        const int role = warp - 1;                         // 0: S^T, dP^T; 1: dV, dK
         const uint32_t idPS = idesc_bf16_f32(128, 64, false, false);
         const uint32_t idKV = idesc_bf16_f32(128, D, false, true);
         const uint32_t aR = smem_u32(sm + L::RING);
@@ -813,16 +828,19 @@ k_bwd_dkdv_persist(const __grid_constant__ CUtensorMap tmK, const __grid_constan
             const int4 item = items[it];
             const int ng = item.z - item.y;
             if (ng == 0) continue;
-            ok = mbar_wait_w(B.stat, kq & 1, B.abort_flag, dev_status);
-            if (!ok) break;
-            tc_fence_after();
-            int prev_s = 0;
-            for (int g = 0; ok && g <= ng; ++g) {
-                if (g < ng) {
-                    const int GG = G + g;
-                    const int s = s_, b = GG & 1;
-                    const uint32_t ph = (uint32_t)c_ & 1;
-                    if (!mbar_wait_w(B.full0 + s, ph, B.abort_flag, dev_status)) {
+            if (role == 0) {
+                ok = mbar_wait_w(B.stat, kq & 1, B.abort_flag, dev_status);
+                if (!ok) break;
+                tc_fence_after();
+            }
+            for (int g = 0; g < ng; ++g) {
+                const int GG = G + g;
+                const int s = s_, b = GG & 1, u = GG >> 1;
+                const uint32_t ph = (uint32_t)c_ & 1;
+                if (++s_ == nst) { s_ = 0; ++c_; }
+                if (role == 0) {
+                    if (!mbar_wait_w(B.full0 + s, ph, B.abort_flag, dev_status) ||
+                        (GG >= 2 && !mbar_wait_w(B.kv_done + b, (uint32_t)(u - 1) & 1, B.abort_flag, dev_status))) {
                         ok = false;
                         break;
                     }
@@ -839,12 +857,8 @@ k_bwd_dkdv_persist(const __grid_constant__ CUtensorMap tmK, const __grid_constan
                                  sdesc_add(ddO, kmaj_off(k, kGran)), idPS, k > 0);
                     tc_commit_w(B.prod + b);
                     if (g == ng - 1) tc_commit_w(B.kv_free);   // K and V no longer read by this item
-                }
-                if (g > 0) {
-                    const int gp = g - 1;
-                    const int GGp = G + gp;
-                    const int s = prev_s, b = GGp & 1;
-                    if (!mbar_wait_w(B.elem + b, (uint32_t)(GGp >> 1) & 1, B.abort_flag, dev_status)) {
+                } else {
+                    if (!mbar_wait_w(B.elem + b, (uint32_t)u & 1, B.abort_flag, dev_status)) {
                         ok = false;
                         break;
                     }
@@ -853,27 +867,24 @@ k_bwd_dkdv_persist(const __grid_constant__ CUtensorMap tmK, const __grid_constan
                     const uint64_t ddOn = sdesc_add(dQn, L::NR * kGran);
 #pragma unroll
                     for (int k = 0; k < 4; ++k) {            // queries 16 k ..: warpgroup k / 2's columns
-                        const uint32_t acc = (gp > 0 || k > 0) ? 1u : 0u;
+                        const uint32_t acc = (g > 0 || k > 0) ? 1u : 0u;
                         const uint32_t ck = 128 * b + 32 * (k >> 1) + 8 * (k & 1);
                         mma_ts_w(tb + cdV, tb + cS + ck, sdesc_add(ddOn, k * 2048), idKV, acc);
                         mma_ts_w(tb + cdK, tb + cP + ck, sdesc_add(dQn, k * 2048), idKV, acc);
                     }
                     tc_commit_w(B.empty + s);
-                }
-                if (g < ng) {
-                    prev_s = s_;
-                    if (++s_ == nst) { s_ = 0; ++c_; }
+                    tc_commit_w(B.kv_done + b);
                 }
             }
             if (!ok) break;
-            tc_commit_w(B.fin);
+            if (role == 1) tc_commit_w(B.fin);
             G += ng;
             ++kq;
         }
         if (!ok) {
-            tc_commit_w(B.drain);
+            tc_commit_w(B.drain + role);                   // every MMA this warp issued complete
             volatile int no_abort = 0;
-            mbar_wait(B.drain, 0, &no_abort, dev_status);
+            mbar_wait(B.drain + role, 0, &no_abort, dev_status);
         }
       }
     } else {
