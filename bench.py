@@ -42,7 +42,7 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM bytes (read + write) of one backward call, by (config, heads), from an ncu capture of
 # the backward kernels (profiles/attn_kernels_2k_4heads.md: 4 heads scaled by 6, plus the
 # Delta kernel's algorithmic 5.5 GB)
-BWD_DRAM_BYTES = {}
+BWD_DRAM_BYTES = {("2k", 24): 33.2e9}
 
 
 def metric_name(cfg, fwd_only):
