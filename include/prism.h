@@ -97,6 +97,11 @@ prism_status_t prism_query_sizes(const prism_problem_t* prob, prism_sizes_t* siz
  *   A(m)/max A, A = zone mean of a;  zone_stats [Z][8] (nullable) =
  *   (sigma2_vT, sigma2_vH, sigma2_vW, rho_raw, A, sigma2_aT, sigma2_aH, sigma2_aW).
  * ws: >= sizes.ws_indicator bytes of scratch.
+ * V is read through a TMA tensor map, one 8x8x8-zone box of 128 bytes of
+ * channels per copy (V 16-byte aligned, like every pointer argument);
+ * PRISM_ERR_CUDA if the map cannot be encoded.  A copy that never lands (a
+ * failing device; the wait gives up after 2 s) leaves NaN statistics for the
+ * zones that CTA had left, rather than stale ones.
  */
 prism_status_t prism_zone_indicator(const prism_problem_t* prob, const void* V, const void* hhat,
                                     float eps, float* g, float* rho, float* abar,
