@@ -25,7 +25,7 @@ EXPORTS = ("prism_query_sizes", "prism_zone_indicator", "prism_assign_shapes", "
            "prism_status_string", "prism_version", "prism_launch_count",
            "prism_zone_indicator_noalloc", "prism_zone_indicator_ex", "prism_assign_shapes_ex",
            "prism_layer_init", "prism_layer_arena_bytes", "prism_layer_bind", "prism_layer_forward",
-           "prism_layer_backward", "prism_layer_step_host", "prism_layer_sizeof",
+           "prism_layer_backward", "prism_layer_step_host", "prism_layer_release", "prism_layer_sizeof",
            "prism_zone_partials", "prism_zone_finalize", "prism_block_pool_score_raster",
            "prism_sparse_attn_fwd_raster", "prism_sparse_attn_bwd_raster")
 GUIDANCE = {"joint": 0, "video": 1, "audio": 2}
@@ -65,7 +65,7 @@ class LayerT(ctypes.Structure):
                 ("dOp", _VP), ("dQp", _VP), ("dKp", _VP), ("dVp", _VP),
                 ("ws_bwd", _VP), ("ws_bwd_bytes", ctypes.c_size_t),
                 ("Q", _VP), ("K", _VP), ("V", _VP), ("hhat", _VP), ("O", _VP), ("dO", _VP),
-                ("dQ", _VP), ("dK", _VP), ("dV", _VP)]
+                ("dQ", _VP), ("dK", _VP), ("dV", _VP), ("io_events", _VP)]
 
 
 class PrismError(RuntimeError):
@@ -117,6 +117,7 @@ _SIGS = {
     "prism_layer_forward": [ctypes.POINTER(LayerT), _P, _P, _P, _P, _P, _P],
     "prism_layer_backward": [ctypes.POINTER(LayerT), _P, _P, _P, _P, _P, _P, _P, _P],
     "prism_layer_step_host": [ctypes.POINTER(LayerT), _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P],
+    "prism_layer_release": [ctypes.POINTER(LayerT)],
 }
 
 
@@ -300,6 +301,11 @@ def prism_layer_step_host(L: LayerT, hQ, hK, hV, hhhat, hdO, hO, hdQ, hdK, hdV, 
     _check("prism_layer_step_host", lib().prism_layer_step_host(
         ctypes.byref(L), _ptr(hQ), _ptr(hK), _ptr(hV), _ptr(hhhat), _ptr(hdO), _ptr(hO), _ptr(hdQ), _ptr(hdK),
         _ptr(hdV), _stream(compute), _stream(h2d), _stream(d2h)))
+
+
+def prism_layer_release(L: LayerT):
+    """Destroy the CUDA events a host-buffer step created in L (see include/prism.h)."""
+    _check("prism_layer_release", lib().prism_layer_release(ctypes.byref(L)))
 
 
 # ---------------------------------------------------------------- head-sharded indicator

@@ -11,8 +11,10 @@
 // prism_layer_step_host adds the host copies, one cudaMemcpyAsync per tensor,
 // on two copy streams: V and hhat first (the indicator needs only them), then
 // Q and K, then dO, whose upload overlaps the forward; O downloads while the
-// backward runs.  Across calls, one step's gradient downloads overlap the next
-// step's uploads (opposite PCIe directions).
+// backward runs.  Across calls, the next step's uploads wait only for this
+// step's last read of the raster inputs (two events kept in L->io_events), so in
+// the blocked layout they overlap this step's attention and its downloads
+// (opposite PCIe directions).
 #include <math.h>
 #include <string.h>
 
@@ -101,8 +103,13 @@ bool params_ok(const prism_layer_t* L) {
         if (st_ != PRISM_OK) return st_;      \
     } while (0)
 
+// inputs_read (nullable): recorded once the raster Q, K, V and hhat have been read
+// for the last time in the forward (blocked layout: after the permutes; the
+// raster-layout attention reads them until the end of the backward, so then it
+// is not recorded here)
 prism_status_t run_forward(const prism_layer_t* L, const void* Q, const void* K, const void* V, const void* hhat,
-                           void* O, cudaStream_t s, cudaEvent_t qk_ready, cudaEvent_t out_free) {
+                           void* O, cudaStream_t s, cudaEvent_t qk_ready, cudaEvent_t out_free,
+                           cudaEvent_t inputs_read = nullptr) {
     const prism_problem_t* p = &L->prob;
     PRISM_TRY(prism_zone_indicator_ex(p, V, hhat, L->eps, L->guidance, L->g, L->rho, L->abar, L->zone_stats,
                                       L->ws_ind, L->ws_ind_bytes, s));
@@ -123,6 +130,7 @@ prism_status_t run_forward(const prism_layer_t* L, const void* Q, const void* K,
     if (qk_ready && cudaStreamWaitEvent(s, qk_ready, 0) != cudaSuccess) return PRISM_ERR_CUDA;
     PRISM_TRY(prism_permute(p, Q, L->perm, L->Qp, s));
     PRISM_TRY(prism_permute(p, K, L->perm, L->Kp, s));
+    if (inputs_read && cudaEventRecord(inputs_read, s) != cudaSuccess) return PRISM_ERR_CUDA;
     PRISM_TRY(prism_block_pool_score(p, L->Qp, L->Kp, L->blk_start, L->n_blk, L->scale, L->Qbar, L->Kbar, L->P, s));
     PRISM_TRY(prism_block_select(p, L->P, L->blk_start, L->gran_blk, L->n_blk, L->top_k, L->top_p, L->sel,
                                  L->sel_count, L->gsel, L->gselT, L->margin_sel, L->dev_status, s));
@@ -132,9 +140,11 @@ prism_status_t run_forward(const prism_layer_t* L, const void* Q, const void* K,
     return prism_unpermute(p, L->Op, L->perm, O, s);
 }
 
+// do_read (nullable): recorded once the raster dO has been read for the last time
+// (blocked layout: after its permute; raster layout: not recorded here)
 prism_status_t run_backward(const prism_layer_t* L, const void* Q, const void* K, const void* V, const void* dO,
                             void* dQ, void* dK, void* dV, cudaStream_t s,
-                            cudaEvent_t* done /* [3] nullable: after dQ, dK, dV */) {
+                            cudaEvent_t* done /* [3] nullable: after dQ, dK, dV */, cudaEvent_t do_read = nullptr) {
     const prism_problem_t* p = &L->prob;
     if (L->raster) {
         PRISM_TRY(prism_sparse_attn_bwd_raster(p, Q, K, V, L->Of32, dO, L->lse, L->perm, L->shape_id, L->gsel,
@@ -146,6 +156,7 @@ prism_status_t run_backward(const prism_layer_t* L, const void* Q, const void* K
         return PRISM_OK;
     }
     PRISM_TRY(prism_permute(p, dO, L->perm, L->dOp, s));
+    if (do_read && cudaEventRecord(do_read, s) != cudaSuccess) return PRISM_ERR_CUDA;
     PRISM_TRY(prism_sparse_attn_bwd(p, L->Qp, L->Kp, L->Vp, L->Op, L->Of32, L->dOp, L->lse, L->gsel, L->gselT,
                                     L->scale, L->dQp, L->dKp, L->dVp, L->dev_status, L->ws_bwd, L->ws_bwd_bytes,
                                     s));
@@ -233,7 +244,26 @@ prism_status_t copy(void* dst, const void* src, size_t bytes, cudaMemcpyKind kin
 }
 }  // namespace
 
-extern "C" prism_status_t prism_layer_step_host(const prism_layer_t* L, const void* hQ, const void* hK,
+namespace {
+// The events that carry "the raster inputs have been read" from one host-buffer
+// step to the next; created by the first step, kept in L->io_events.
+struct IoEvents {
+    cudaEvent_t inputs_read = nullptr;   // Q, K, V, hhat
+    cudaEvent_t do_read = nullptr;       // dO
+};
+}  // namespace
+
+extern "C" prism_status_t prism_layer_release(prism_layer_t* L) {
+    if (!L) return PRISM_ERR_INVALID_ARG;
+    IoEvents* io = static_cast<IoEvents*>(L->io_events);
+    if (!io) return PRISM_OK;
+    const bool ok = cudaEventDestroy(io->inputs_read) == cudaSuccess && cudaEventDestroy(io->do_read) == cudaSuccess;
+    delete io;
+    L->io_events = nullptr;
+    return ok ? PRISM_OK : PRISM_ERR_CUDA;
+}
+
+extern "C" prism_status_t prism_layer_step_host(prism_layer_t* L, const void* hQ, const void* hK,
                                                 const void* hV, const void* hhhat, const void* hdO, void* hO,
                                                 void* hdQ, void* hdK, void* hdV, cudaStream_t compute,
                                                 cudaStream_t h2d, cudaStream_t d2h) {
@@ -246,15 +276,28 @@ extern "C" prism_status_t prism_layer_step_host(const prism_layer_t* L, const vo
     const size_t esz = L->prob.dtype == PRISM_BF16 ? 2 : 4;
     const size_t tok = (size_t)s.n_tokens * L->prob.heads * L->prob.head_dim * esz;
     const size_t hhb = (size_t)s.n_tokens * L->prob.audio_dim * esz;
-    enum { kPrevCompute, kPrevD2H, kVH, kQK, kDO, kO, kDQ, kDK, kDV, kCount };
+    if (!L->io_events) {
+        IoEvents* fresh = new IoEvents;
+        if (cudaEventCreateWithFlags(&fresh->inputs_read, cudaEventDisableTiming) != cudaSuccess ||
+            cudaEventCreateWithFlags(&fresh->do_read, cudaEventDisableTiming) != cudaSuccess) {
+            if (fresh->inputs_read) cudaEventDestroy(fresh->inputs_read);
+            delete fresh;
+            return PRISM_ERR_CUDA;
+        }
+        L->io_events = fresh;
+    }
+    IoEvents* io = static_cast<IoEvents*>(L->io_events);
+    enum { kPrevD2H, kVH, kQK, kDO, kO, kDQ, kDK, kDV, kCount };
     Events ev;
     if (!ev.make(kCount)) return PRISM_ERR_CUDA;
     const cudaMemcpyKind H2D = cudaMemcpyHostToDevice, D2H = cudaMemcpyDeviceToHost;
-    // the previous step's compute still reads the raster inputs, and its downloads
-    // still read the raster outputs: uploads wait for the first, writes of O, dQ,
-    // dK, dV for the second
-    if (cudaEventRecord(ev.e[kPrevCompute], compute) != cudaSuccess ||
-        cudaEventRecord(ev.e[kPrevD2H], d2h) != cudaSuccess || cudaStreamWaitEvent(h2d, ev.e[kPrevCompute], 0) != cudaSuccess)
+    // The previous step may still read the raster inputs, and its downloads still
+    // read the raster outputs.  Uploads of Q, K, V, hhat wait for its last read of
+    // them, the upload of dO for its last read of dO (events the previous call
+    // recorded; a never-recorded event counts as complete), and writes of O, dQ,
+    // dK, dV wait for its downloads.
+    if (cudaEventRecord(ev.e[kPrevD2H], d2h) != cudaSuccess ||
+        cudaStreamWaitEvent(h2d, io->inputs_read, 0) != cudaSuccess)
         return PRISM_ERR_CUDA;
     PRISM_TRY(copy(L->V, hV, tok, H2D, h2d));
     PRISM_TRY(copy(L->hhat, hhhat, hhb, H2D, h2d));
@@ -263,18 +306,22 @@ extern "C" prism_status_t prism_layer_step_host(const prism_layer_t* L, const vo
     PRISM_TRY(copy(L->K, hK, tok, H2D, h2d));
     if (cudaEventRecord(ev.e[kQK], h2d) != cudaSuccess) return PRISM_ERR_CUDA;
     if (bwd) {
+        if (cudaStreamWaitEvent(h2d, io->do_read, 0) != cudaSuccess) return PRISM_ERR_CUDA;
         PRISM_TRY(copy(L->dO, hdO, tok, H2D, h2d));
         if (cudaEventRecord(ev.e[kDO], h2d) != cudaSuccess) return PRISM_ERR_CUDA;
     }
     if (cudaStreamWaitEvent(compute, ev.e[kVH], 0) != cudaSuccess) return PRISM_ERR_CUDA;
-    PRISM_TRY(run_forward(L, L->Q, L->K, L->V, L->hhat, L->O, compute, ev.e[kQK], ev.e[kPrevD2H]));
+    const bool early = !L->raster;             // blocked layout: inputs read by the permutes only
+    PRISM_TRY(run_forward(L, L->Q, L->K, L->V, L->hhat, L->O, compute, ev.e[kQK], ev.e[kPrevD2H],
+                          early ? io->inputs_read : nullptr));
     if (cudaEventRecord(ev.e[kO], compute) != cudaSuccess || cudaStreamWaitEvent(d2h, ev.e[kO], 0) != cudaSuccess)
         return PRISM_ERR_CUDA;
     PRISM_TRY(copy(hO, L->O, tok, D2H, d2h));
     if (bwd) {
         if (cudaStreamWaitEvent(compute, ev.e[kDO], 0) != cudaSuccess) return PRISM_ERR_CUDA;
         cudaEvent_t done[3] = {ev.e[kDQ], ev.e[kDK], ev.e[kDV]};
-        PRISM_TRY(run_backward(L, L->Q, L->K, L->V, L->dO, L->dQ, L->dK, L->dV, compute, done));
+        PRISM_TRY(run_backward(L, L->Q, L->K, L->V, L->dO, L->dQ, L->dK, L->dV, compute, done,
+                               early ? io->do_read : nullptr));
         void* hs[3] = {hdQ, hdK, hdV};
         void* ds[3] = {L->dQ, L->dK, L->dV};
         for (int i = 0; i < 3; ++i) {
@@ -282,6 +329,10 @@ extern "C" prism_status_t prism_layer_step_host(const prism_layer_t* L, const vo
             PRISM_TRY(copy(hs[i], ds[i], tok, D2H, d2h));
         }
     }
+    // raster layout: the inputs are read until the step's compute ends
+    if (!early && (cudaEventRecord(io->inputs_read, compute) != cudaSuccess ||
+                   cudaEventRecord(io->do_read, compute) != cudaSuccess))
+        return PRISM_ERR_CUDA;
     // no join here: all of the step's device work precedes its last download, so
     // the d2h stream marks completion, and the next step's uploads can overlap
     // this step's downloads

@@ -34,7 +34,7 @@ static int offsets(void) {
     FIELD(gselT); FIELD(sel_count); FIELD(margin_sel); FIELD(dev_status); FIELD(Op); FIELD(Of32);
     FIELD(lse); FIELD(ws_fwd); FIELD(ws_fwd_bytes); FIELD(dOp); FIELD(dQp); FIELD(dKp); FIELD(dVp);
     FIELD(ws_bwd); FIELD(ws_bwd_bytes); FIELD(Q); FIELD(K); FIELD(V); FIELD(hhat); FIELD(O); FIELD(dO);
-    FIELD(dQ); FIELD(dK); FIELD(dV);
+    FIELD(dQ); FIELD(dK); FIELD(dV); FIELD(io_events);
     return 0;
 }
 
@@ -134,6 +134,7 @@ static int run(const char* dir) {
     cudaStreamDestroy(compute);
     cudaStreamDestroy(h2d);
     cudaStreamDestroy(d2h);
+    PK(prism_layer_release(&L));
     cudaFree(arena);
     return st == 0 ? 0 : 2;
 }

@@ -132,6 +132,17 @@ class PrismSparseAttention:
         the host outputs are final once ``d2h`` has passed this call."""
         _abi.prism_layer_step_host(self.L, hQ, hK, hV, hhhat, hdO, hO, hdQ, hdK, hdV, compute, h2d, d2h)
 
+    def release(self):
+        """Destroy the CUDA events the host-buffer step created (once its last call has completed)."""
+        if getattr(self, "L", None) is not None and self.L.io_events:
+            _abi.prism_layer_release(self.L)
+
+    def __del__(self):
+        try:
+            self.release()
+        except Exception:       # interpreter shutdown: the library may be gone already
+            pass
+
     # ------------------------------------------------------------------ stages
     def plan(self, V, hhat, stream=None):
         """Stages 1-2: zone indicator, shapes, permutation, block table."""

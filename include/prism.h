@@ -393,6 +393,11 @@ typedef struct {
     size_t ws_bwd_bytes;
     /* raster Q, K, V, hhat, O, dO, dQ, dK, dV on the device (with_io only) */
     void *Q, *K, *V, *hhat, *O, *dO, *dQ, *dK, *dV;
+    /* library-owned state of prism_layer_step_host (two CUDA events that carry
+       "this step has read its raster inputs" to the next call): NULL after
+       prism_layer_init, created by the first host-buffer step, destroyed by
+       prism_layer_release.  Callers do not touch it. */
+    void* io_events;
 } prism_layer_t;
 
 /* Fill L with the defaults above for `prob` and no buffers (host only). */
@@ -420,13 +425,21 @@ prism_status_t prism_layer_backward(const prism_layer_t* L, const void* Q, const
  * Asynchronous: every device step of the call precedes its last download on
  * `d2h`, so the host outputs are final once `d2h` has passed this call (e.g.
  * cudaStreamSynchronize(d2h)).  Consecutive calls with the same streams are
- * ordered: the next call's uploads wait for this call's compute, and its
- * writes of O and the gradients wait for this call's downloads, which may
- * still run while the next uploads do.  Host input buffers must stay unchanged
- * and output buffers unread until then. */
-prism_status_t prism_layer_step_host(const prism_layer_t* L, const void* hQ, const void* hK, const void* hV,
+ * ordered.  The next call's uploads wait only until this call has read the
+ * raster inputs.  In the blocked layout that is the permutes at the start of
+ * the forward (Q, K, V, hhat) and of the backward (dO), so the next uploads
+ * overlap this call's attention and downloads; with L->raster it is the end of
+ * the backward.  The next call's writes of O and the gradients wait for this
+ * call's downloads.  Host input buffers must stay unchanged and output buffers
+ * unread until then.  The first call creates L->io_events (two CUDA events);
+ * prism_layer_release destroys them. */
+prism_status_t prism_layer_step_host(prism_layer_t* L, const void* hQ, const void* hK, const void* hV,
                                      const void* hhhat, const void* hdO, void* hO, void* hdQ, void* hdK,
                                      void* hdV, cudaStream_t compute, cudaStream_t h2d, cudaStream_t d2h);
+/* Destroy the CUDA events a host-buffer step created in L (L->io_events),
+ * after every call that used them has completed; a no-op when there are none.
+ * The device buffers stay the caller's. */
+prism_status_t prism_layer_release(prism_layer_t* L);
 /* sizeof(prism_layer_t) as compiled into the library (a check for bindings). */
 size_t prism_layer_sizeof(void);
 

@@ -133,8 +133,10 @@ def test_layer_init_defaults_and_arena_carving(L):
     assert L.prism_layer_bind(ctypes.byref(lay), base, io - 1) == 4              # too small
     assert L.prism_layer_bind(ctypes.byref(lay), base + 16, io) == 1             # misaligned
     assert L.prism_layer_bind(ctypes.byref(lay), base, io) == 0
-    ptrs = [getattr(lay, f[0]) for f in _abi.LayerT._fields_ if f[1] is ctypes.c_void_p]
+    ptrs = [getattr(lay, f[0]) for f in _abi.LayerT._fields_ if f[1] is ctypes.c_void_p and f[0] != "io_events"]
     assert all(q is not None and base <= q < base + io and q % 256 == 0 for q in ptrs)
+    assert lay.io_events is None                      # the host-buffer step's events: none until one runs
+    assert L.prism_layer_release(ctypes.byref(lay)) == 0     # nothing to release: a no-op
     assert len(set(ptrs)) == len(ptrs)
     assert lay.ws_bwd_bytes == sz.ws_attn_bwd and lay.ws_fwd_bytes == sz.ws_attn_fwd
     # bad parameters are refused before anything is carved

@@ -90,3 +90,43 @@ def test_host_step_twice_on_three_streams():
             assert torch.equal(a, b), (step, k)
     compute.synchronize()
     assert mod.status() == 0
+
+
+@pytest.mark.parametrize("raster", [False, True])
+def test_host_steps_back_to_back_with_different_inputs(raster):
+    """Two host-buffer steps issued back to back, with different inputs and no
+    synchronisation between them.  The second step's uploads may start as soon as
+    the first has read its raster inputs (in the blocked layout, after its
+    permutes), so an upload that overwrote an input still being read would change
+    the first step's outputs.  Each step must give the device-buffer layer's bits
+    for its own inputs."""
+    cfg_a = get_config("720p", T=16, H=32, W=32, heads=3)
+    cfg_b = get_config("720p", T=16, H=32, W=32, heads=3, seed=cfg_a.seed + 7)
+    xs = [inputs.make_inputs(c, "cuda") for c in (cfg_a, cfg_b)]
+    mod = PrismSparseAttention(cfg_a.T, cfg_a.H, cfg_a.W, cfg_a.heads, cfg_a.head_dim, cfg_a.audio_dim, cfg_a.dtype,
+                               cfg_a.top_k, cfg_a.top_p, raster=raster)
+    refs = []
+    for x in xs:
+        O = mod.forward(x["Q"], x["K"], x["V"], x["hhat"])
+        grads = mod.backward(x["dO"])
+        torch.cuda.synchronize()
+        refs.append([t.cpu() for t in (O,) + tuple(grads)])
+    assert not all(torch.equal(a, b) for a, b in zip(*refs))      # the two steps differ
+    names = ("Q", "K", "V", "hhat", "dO")
+    dev = {k: torch.empty_like(xs[0][k]) for k in names}
+    outs = [torch.empty_like(xs[0]["Q"]) for _ in range(4)]
+    mod.attach_io(dev["Q"], dev["K"], dev["V"], dev["hhat"], outs[0], dev["dO"], *outs[1:])
+    hins = [{k: x[k].cpu().pin_memory() for k in names} for x in xs]
+    houts = [[torch.empty(xs[0]["Q"].shape, dtype=xs[0]["Q"].dtype).pin_memory() for _ in range(4)] for _ in xs]
+    compute, h2d, d2h = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    for rep in range(2):
+        for hin, hout in zip(hins, houts):
+            mod.step_host(hin["Q"], hin["K"], hin["V"], hin["hhat"], hin["dO"], *hout, compute, h2d, d2h)
+        d2h.synchronize()
+        for step, (hout, ref) in enumerate(zip(houts, refs)):
+            for k, a, b in zip(("O", "dQ", "dK", "dV"), hout, ref):
+                assert torch.equal(a, b), (rep, step, k)
+    compute.synchronize()
+    assert mod.status() == 0
+    mod.release()
+    assert not mod.L.io_events
