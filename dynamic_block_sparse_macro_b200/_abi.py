@@ -27,7 +27,8 @@ EXPORTS = ("prism_query_sizes", "prism_zone_indicator", "prism_assign_shapes", "
            "prism_layer_init", "prism_layer_arena_bytes", "prism_layer_bind", "prism_layer_forward",
            "prism_layer_backward", "prism_layer_step_host", "prism_layer_release", "prism_layer_sizeof",
            "prism_zone_partials", "prism_zone_finalize", "prism_block_pool_score_raster",
-           "prism_sparse_attn_fwd_raster", "prism_sparse_attn_bwd_raster")
+           "prism_sparse_attn_fwd_raster", "prism_sparse_attn_bwd_raster", "prism_attn_bwd_ds_bytes",
+           "prism_sparse_attn_bwd_ds", "prism_sparse_attn_bwd_raster_ds")
 GUIDANCE = {"joint": 0, "video": 1, "audio": 2}
 NOALLOC_SCRATCH_BYTES = 2 << 20
 
@@ -110,6 +111,11 @@ _SIGS = {
     "prism_sparse_attn_fwd_raster": [_PROB, _P, _P, _P, _P, _P, _P, _F, _P, _P, _P, _P, _P, _SZ, _P],
     "prism_sparse_attn_bwd_raster": [_PROB, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _F, _P, _P, _P, _P, _P, _SZ,
                                      _P],
+    "prism_attn_bwd_ds_bytes": [_PROB, ctypes.c_int64, ctypes.POINTER(ctypes.c_size_t)],
+    "prism_sparse_attn_bwd_ds": [_PROB, _P, _P, _P, _P, _P, _P, _P, _P, _P, _F, _P, _P, _P, _P, _P, _SZ, _P, _SZ,
+                                 _P],
+    "prism_sparse_attn_bwd_raster_ds": [_PROB, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _F, _P, _P, _P, _P, _P, _SZ,
+                                        _P, _SZ, _P],
     "prism_zone_finalize": [_PROB, _P, _F, _I, _P, _P, _P, _P, _P, _SZ, _P],
     "prism_layer_init": [ctypes.POINTER(LayerT), _PROB],
     "prism_layer_arena_bytes": [ctypes.POINTER(LayerT), ctypes.POINTER(ctypes.c_size_t)],
@@ -258,6 +264,21 @@ def prism_sparse_attn_bwd(prob, Qp, Kp, Vp, Op, o_f32, dOp, lse, gsel, gselT, sc
         ws.numel() * ws.element_size(), _stream(stream)))
 
 
+def prism_attn_bwd_ds_bytes(prob, pieces: int) -> int:
+    out = ctypes.c_size_t(0)
+    _check("prism_attn_bwd_ds_bytes", lib().prism_attn_bwd_ds_bytes(ctypes.byref(prob), int(pieces),
+                                                                    ctypes.byref(out)))
+    return out.value
+
+
+def prism_sparse_attn_bwd_ds(prob, Qp, Kp, Vp, Op, o_f32, dOp, lse, gsel, gselT, scale, dQp, dKp, dVp,
+                             dev_status, ws, ds, stream=None):
+    _check("prism_sparse_attn_bwd_ds", lib().prism_sparse_attn_bwd_ds(
+        ctypes.byref(prob), _ptr(Qp), _ptr(Kp), _ptr(Vp), _ptr(Op), _ptr(o_f32), _ptr(dOp), _ptr(lse),
+        _ptr(gsel), _ptr(gselT), scale, _ptr(dQp), _ptr(dKp), _ptr(dVp), _ptr(dev_status), _ptr(ws),
+        ws.numel() * ws.element_size(), _ptr(ds), ds.numel() * ds.element_size(), _stream(stream)))
+
+
 def prism_read_status(dev_status, stream=None) -> int:
     out = ctypes.c_uint32(0)
     _check("prism_read_status", lib().prism_read_status(_ptr(dev_status), ctypes.byref(out),
@@ -341,3 +362,11 @@ def prism_sparse_attn_bwd_raster(prob, Q, K, V, o_f32, dO, lse, perm, shape_id, 
         ctypes.byref(prob), _ptr(Q), _ptr(K), _ptr(V), _ptr(o_f32), _ptr(dO), _ptr(lse), _ptr(perm), _ptr(shape_id),
         _ptr(gsel), _ptr(gselT), scale, _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(dev_status), _ptr(ws), ws.numel(),
         _stream(stream)))
+
+
+def prism_sparse_attn_bwd_raster_ds(prob, Q, K, V, o_f32, dO, lse, perm, shape_id, gsel, gselT, scale, dQ, dK,
+                                    dV, dev_status, ws, ds, stream=None):
+    _check("prism_sparse_attn_bwd_raster_ds", lib().prism_sparse_attn_bwd_raster_ds(
+        ctypes.byref(prob), _ptr(Q), _ptr(K), _ptr(V), _ptr(o_f32), _ptr(dO), _ptr(lse), _ptr(perm), _ptr(shape_id),
+        _ptr(gsel), _ptr(gselT), scale, _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(dev_status), _ptr(ws),
+        ws.numel() * ws.element_size(), _ptr(ds), ds.numel() * ds.element_size(), _stream(stream)))

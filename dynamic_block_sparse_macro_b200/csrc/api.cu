@@ -3,6 +3,7 @@
 #include <atomic>
 
 #include "common.cuh"
+#include "ds_handoff.cuh"
 
 namespace prism {
 size_t zone_indicator_ws_bytes(const Dims& d);
@@ -17,12 +18,13 @@ prism_status_t attn_fwd_raster(const Dims& d, const void* Q, const void* K, cons
 prism_status_t attn_bwd_sm100(const Dims& d, const void* Qp, const void* Kp, const void* Vp, const void* Op,
                               const float* o_f32, const void* dOp, const float* lse, const uint32_t* gsel,
                               const uint32_t* gselT, float scale, void* dQp, void* dKp, void* dVp,
-                              uint32_t* dev_status, void* ws, cudaStream_t s);
+                              uint32_t* dev_status, void* ws, cudaStream_t s, void* ds, size_t ds_bytes);
 size_t attn_bwd_sm100_ws_bytes(const Dims& d);
+size_t attn_bwd_ds_bytes(const Dims& d, int64_t pieces);
 prism_status_t attn_bwd_raster(const Dims& d, const void* Q, const void* K, const void* V, const float* o_f32,
                                const void* dO, const float* lse, const int32_t* perm, const uint8_t* shape_id,
                                const uint32_t* gsel, const uint32_t* gselT, float scale, void* dQ, void* dK, void* dV,
-                               uint32_t* dev_status, void* ws, cudaStream_t s);
+                               uint32_t* dev_status, void* ws, cudaStream_t s, void* ds, size_t ds_bytes);
 prism_status_t attn_fwd_simt(const Dims& d, const void* Qp, const void* Kp, const void* Vp, const uint32_t* gsel,
                              float scale, void* Op, float* lse, float* o_f32, cudaStream_t s);
 prism_status_t attn_bwd_simt(const Dims& d, const void* Qp, const void* Kp, const void* Vp, const void* Op,
@@ -92,25 +94,57 @@ extern "C" prism_status_t prism_sparse_attn_fwd_raster(const prism_problem_t* pr
     return attn_fwd_raster(d, Q, K, V, perm, shape_id, gsel, scale, O, lse, o_f32, dev_status, ws, stream);
 }
 
+namespace {
+// argument checks shared by the backward entry points; ds == nullptr: no handoff
+prism_status_t bwd_blocked(const prism_problem_t* prob, const void* Qp, const void* Kp, const void* Vp,
+                           const void* Op, const float* o_f32, const void* dOp, const float* lse,
+                           const uint32_t* gsel, const uint32_t* gselT, float scale, void* dQp, void* dKp, void* dVp,
+                           uint32_t* dev_status, void* ws, size_t ws_bytes, void* ds, size_t ds_bytes,
+                           cudaStream_t stream) {
+    Dims d;
+    prism_status_t st = make_dims(prob, &d);
+    if (st != PRISM_OK) return st;
+    if (!ok_ptr(Qp) || !ok_ptr(Kp) || !ok_ptr(Vp) || !ok_ptr(Op) || !ok_opt(o_f32) || !ok_ptr(dOp) ||
+        !ok_ptr(lse) || !ok_ptr(gsel) || !ok_ptr(gselT) || !ok_ptr(dQp) || !ok_ptr(dKp) || !ok_ptr(dVp) ||
+        !ok_ptr(dev_status) || !ok_ptr(ws) || !ok_opt(ds))
+        return PRISM_ERR_INVALID_ARG;
+    if (!(scale > 0.f) || !isfinite(scale)) return PRISM_ERR_INVALID_ARG;
+    if (ws_bytes < attn_bwd_ws_bytes(d)) return PRISM_ERR_WORKSPACE;
+    if (d.dtype == PRISM_BF16)
+        return attn_bwd_sm100(d, Qp, Kp, Vp, Op, o_f32, dOp, lse, gsel, gselT, scale, dQp, dKp, dVp, dev_status, ws,
+                              stream, ds, ds_bytes);
+    if (ds) return PRISM_ERR_UNSUPPORTED;
+    return attn_bwd_simt(d, Qp, Kp, Vp, Op, o_f32, dOp, lse, gsel, gselT, scale, dQp, dKp, dVp, (float*)ws, stream);
+}
+
+prism_status_t bwd_raster(const prism_problem_t* prob, const void* Q, const void* K, const void* V,
+                          const float* o_f32, const void* dO, const float* lse, const int32_t* perm,
+                          const uint8_t* shape_id, const uint32_t* gsel, const uint32_t* gselT, float scale, void* dQ,
+                          void* dK, void* dV, uint32_t* dev_status, void* ws, size_t ws_bytes, void* ds,
+                          size_t ds_bytes, cudaStream_t stream) {
+    Dims d;
+    prism_status_t st = make_dims(prob, &d);
+    if (st != PRISM_OK) return st;
+    if (d.dtype != PRISM_BF16) return PRISM_ERR_UNSUPPORTED;
+    if (!ok_ptr(Q) || !ok_ptr(K) || !ok_ptr(V) || !ok_ptr(o_f32) || !ok_ptr(dO) || !ok_ptr(lse) || !ok_ptr(perm) ||
+        !ok_ptr(shape_id) || !ok_ptr(gsel) || !ok_ptr(gselT) || !ok_ptr(dQ) || !ok_ptr(dK) || !ok_ptr(dV) ||
+        !ok_ptr(dev_status) || !ok_ptr(ws) || !ok_opt(ds))
+        return PRISM_ERR_INVALID_ARG;
+    if (!(scale > 0.f) || !isfinite(scale)) return PRISM_ERR_INVALID_ARG;
+    if (ws_bytes < attn_bwd_ws_bytes(d)) return PRISM_ERR_WORKSPACE;
+    return attn_bwd_raster(d, Q, K, V, o_f32, dO, lse, perm, shape_id, gsel, gselT, scale, dQ, dK, dV, dev_status, ws,
+                           stream, ds, ds_bytes);
+}
+}  // namespace
+
 extern "C" prism_status_t prism_sparse_attn_bwd(const prism_problem_t* prob, const void* Qp, const void* Kp,
                                                 const void* Vp, const void* Op, const float* o_f32,
                                                 const void* dOp, const float* lse, const uint32_t* gsel,
                                                 const uint32_t* gselT, float scale, void* dQp, void* dKp,
                                                 void* dVp, uint32_t* dev_status, void* ws, size_t ws_bytes,
                                                 cudaStream_t stream) {
-    Dims d;
-    prism_status_t st = make_dims(prob, &d);
-    if (st != PRISM_OK) return st;
-    if (!ok_ptr(Qp) || !ok_ptr(Kp) || !ok_ptr(Vp) || !ok_ptr(Op) || !ok_opt(o_f32) || !ok_ptr(dOp) ||
-        !ok_ptr(lse) || !ok_ptr(gsel) || !ok_ptr(gselT) || !ok_ptr(dQp) || !ok_ptr(dKp) || !ok_ptr(dVp) ||
-        !ok_ptr(dev_status) || !ok_ptr(ws))
-        return PRISM_ERR_INVALID_ARG;
-    if (!(scale > 0.f) || !isfinite(scale)) return PRISM_ERR_INVALID_ARG;
-    if (ws_bytes < attn_bwd_ws_bytes(d)) return PRISM_ERR_WORKSPACE;
-    if (d.dtype == PRISM_BF16)
-        return attn_bwd_sm100(d, Qp, Kp, Vp, Op, o_f32, dOp, lse, gsel, gselT, scale, dQp, dKp, dVp, dev_status, ws,
-                              stream);
-    return attn_bwd_simt(d, Qp, Kp, Vp, Op, o_f32, dOp, lse, gsel, gselT, scale, dQp, dKp, dVp, (float*)ws, stream);
+    return bwd_blocked(prob, Qp, Kp, Vp, Op, o_f32, dOp, lse, gsel, gselT, scale, dQp, dKp, dVp, dev_status, ws,
+                       ws_bytes, nullptr, 0, stream);
 }
 
 extern "C" prism_status_t prism_sparse_attn_bwd_raster(const prism_problem_t* prob, const void* Q, const void* K,
@@ -119,18 +153,40 @@ extern "C" prism_status_t prism_sparse_attn_bwd_raster(const prism_problem_t* pr
                                                        const uint32_t* gsel, const uint32_t* gselT, float scale,
                                                        void* dQ, void* dK, void* dV, uint32_t* dev_status, void* ws,
                                                        size_t ws_bytes, cudaStream_t stream) {
+    return bwd_raster(prob, Q, K, V, o_f32, dO, lse, perm, shape_id, gsel, gselT, scale, dQ, dK, dV, dev_status, ws,
+                      ws_bytes, nullptr, 0, stream);
+}
+
+extern "C" prism_status_t prism_attn_bwd_ds_bytes(const prism_problem_t* prob, int64_t pieces, size_t* bytes) {
     Dims d;
     prism_status_t st = make_dims(prob, &d);
     if (st != PRISM_OK) return st;
-    if (d.dtype != PRISM_BF16) return PRISM_ERR_UNSUPPORTED;
-    if (!ok_ptr(Q) || !ok_ptr(K) || !ok_ptr(V) || !ok_ptr(o_f32) || !ok_ptr(dO) || !ok_ptr(lse) || !ok_ptr(perm) ||
-        !ok_ptr(shape_id) || !ok_ptr(gsel) || !ok_ptr(gselT) || !ok_ptr(dQ) || !ok_ptr(dK) || !ok_ptr(dV) ||
-        !ok_ptr(dev_status) || !ok_ptr(ws))
-        return PRISM_ERR_INVALID_ARG;
-    if (!(scale > 0.f) || !isfinite(scale)) return PRISM_ERR_INVALID_ARG;
-    if (ws_bytes < attn_bwd_ws_bytes(d)) return PRISM_ERR_WORKSPACE;
-    return attn_bwd_raster(d, Q, K, V, o_f32, dO, lse, perm, shape_id, gsel, gselT, scale, dQ, dK, dV, dev_status, ws,
-                           stream);
+    if (!bytes || pieces < 1 || pieces > ds::kMaxPieces) return PRISM_ERR_INVALID_ARG;
+    *bytes = attn_bwd_ds_bytes(d, pieces);
+    return PRISM_OK;
+}
+
+extern "C" prism_status_t prism_sparse_attn_bwd_ds(const prism_problem_t* prob, const void* Qp, const void* Kp,
+                                                   const void* Vp, const void* Op, const float* o_f32,
+                                                   const void* dOp, const float* lse, const uint32_t* gsel,
+                                                   const uint32_t* gselT, float scale, void* dQp, void* dKp,
+                                                   void* dVp, uint32_t* dev_status, void* ws, size_t ws_bytes,
+                                                   void* ds, size_t ds_bytes, cudaStream_t stream) {
+    if (!ok_ptr(ds)) return PRISM_ERR_INVALID_ARG;
+    return bwd_blocked(prob, Qp, Kp, Vp, Op, o_f32, dOp, lse, gsel, gselT, scale, dQp, dKp, dVp, dev_status, ws,
+                       ws_bytes, ds, ds_bytes, stream);
+}
+
+extern "C" prism_status_t prism_sparse_attn_bwd_raster_ds(const prism_problem_t* prob, const void* Q, const void* K,
+                                                          const void* V, const float* o_f32, const void* dO,
+                                                          const float* lse, const int32_t* perm,
+                                                          const uint8_t* shape_id, const uint32_t* gsel,
+                                                          const uint32_t* gselT, float scale, void* dQ, void* dK,
+                                                          void* dV, uint32_t* dev_status, void* ws, size_t ws_bytes,
+                                                          void* ds, size_t ds_bytes, cudaStream_t stream) {
+    if (!ok_ptr(ds)) return PRISM_ERR_INVALID_ARG;
+    return bwd_raster(prob, Q, K, V, o_f32, dO, lse, perm, shape_id, gsel, gselT, scale, dQ, dK, dV, dev_status, ws,
+                      ws_bytes, ds, ds_bytes, stream);
 }
 
 extern "C" prism_status_t prism_read_status(const uint32_t* dev_status, uint32_t* host_out, cudaStream_t stream) {

@@ -19,6 +19,9 @@
 //                       transposed granule-level selection); per 64-query granule
 //                       S^T = K Q^T and dP^T = V dO^T, then P^T and dS^T as bf16
 //                       in TMEM, dV += P^T dO and dK += dS^T Q.
+// With a dS handoff buffer (ds_handoff.cuh) the key-stationary kernel also
+// stores its dS^T blocks, and k_bwd_dq_ds replaces the query-stationary kernel
+// with one GEMM per key granule, dQ += dS K, so that S and dP are formed once.
 // Both double-buffer the granule products in TMEM so that the tensor core
 // works on granule g+1 while the elementwise warps work on granule g, and
 // stream granules through a TMA ring as deep as shared memory allows; ring
@@ -33,6 +36,7 @@
 // Every wait is bounded; a timeout sets PRISM_DEV_TIMEOUT.
 #include "attn_plan.cuh"
 #include "common.cuh"
+#include "ds_handoff.cuh"
 #include "sm100.cuh"
 
 namespace prism {
@@ -90,6 +94,17 @@ struct BwdRaster {
     const int4* gpos;          // [N/64] granule positions (gran_positions)
     const int32_t* perm;       // [N]
     int heads;
+};
+
+// Device side of the dS handoff (ds_handoff.cuh): `on` is written by k_ds_bases
+// before any kernel that reads it, 1 when every piece and entry fits
+struct DsDev {
+    int* on;
+    int64_t* base_q;           // [tiles] exclusive prefix of the query tiles' units
+    int64_t* base_kv;          // [tiles] exclusive prefix of the key tiles' units
+    int32_t* pre;              // [tiles][SW] word prefixes of the key tiles' unions
+    int4* entries;             // [cap_q] look-up entries of the query-stationary walk
+    __nv_bfloat16* pieces;     // [1 + cap_units][128][64] dS^T; piece 0 stays zero
 };
 
 constexpr int kStagingP = 2 * kTile;       // 32 KB: two 128-byte regions of 128 rows
@@ -245,7 +260,8 @@ __device__ __forceinline__ void load_row_tmem(uint32_t taddr, const __nv_bfloat1
     tmem_wait_st();
 }
 
-template <int D, bool RASTER>
+// DS: launched beside k_bwd_dq_ds, which does the work when *ds_on is set
+template <int D, bool RASTER, bool DS = false>
 __global__ void __launch_bounds__(384, 1)
 k_bwd_dq_persist(const __nv_bfloat16* __restrict__ Qg, const __nv_bfloat16* __restrict__ dOg,
                  const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
@@ -254,7 +270,10 @@ k_bwd_dq_persist(const __nv_bfloat16* __restrict__ Qg, const __nv_bfloat16* __re
                  const uint32_t* __restrict__ gsel, const PlanHeader* __restrict__ hdr,
                  const int4* __restrict__ items, const float* __restrict__ lse,
                  const float* __restrict__ delta, int64_t N, int64_t MB, int SW, int nst, float scale,
-                 uint32_t* __restrict__ dev_status) {
+                 uint32_t* __restrict__ dev_status, const int* __restrict__ ds_on) {
+    if constexpr (DS) {
+        if (*ds_on) return;                           // uniform: dQ comes from the stored dS
+    }
     using L = DqpLayout<D>;
     constexpr int kRL = RASTER ? L::NR : 1;            // copy lanes per (stream, stage)
     constexpr uint32_t cdQ = 0, cS = 128, cP = 192;   // + 128 * buffer for S / dP
@@ -637,7 +656,9 @@ __device__ __forceinline__ BarsKV carve_kv(uint8_t* ctrl) {
 }
 static_assert((4 * kStages + 15) * 8 + 8 <= kCtrl, "barriers overflow the control block");
 
-template <int D, bool RASTER>
+// DS: the elementwise warps also store the dS^T blocks (pieces, ds_handoff.cuh)
+// when *ds.on is set
+template <int D, bool RASTER, bool DS = false>
 __global__ void __launch_bounds__(384, 1)
 k_bwd_dkdv_persist(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                    const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmdO,
@@ -646,7 +667,8 @@ k_bwd_dkdv_persist(const __grid_constant__ CUtensorMap tmK, const __grid_constan
                    const __grid_constant__ BwdRasterMaps<RASTER, 6> rmaps, BwdRaster ras,
                    const uint32_t* __restrict__ gselT, const PlanHeader* __restrict__ hdr,
                    const int4* __restrict__ items, const float* __restrict__ nld,
-                   int64_t N, int64_t MB, int SW, int nst, float scale, uint32_t* __restrict__ dev_status) {
+                   int64_t N, int64_t MB, int SW, int nst, float scale, uint32_t* __restrict__ dev_status,
+                   DsDev ds) {
     using L = DkvpLayout<D>;
     constexpr int kRL = RASTER ? L::NR : 1;            // copy lanes per (stream, stage)
     constexpr int kStatLanes = RASTER ? 2 * 2 * L::NR : 2;   // stationary copies: (tensor, granule, region)
@@ -901,11 +923,20 @@ k_bwd_dkdv_persist(const __grid_constant__ CUtensorMap tmK, const __grid_constan
         bool ok = true;
         int G = 0, kf = 0;
         int st_ = 0, cy_ = 0;                              // ring stage and cycle of granule G
+        bool ds_live = false;
+        if constexpr (DS) ds_live = *ds.on != 0;
         for (int it = blockIdx.x, j = 0; it < n_items; it += gridDim.x, ++j) {
             const int4 item = items[it];
             const int hh = item.x / tiles_per_head, tile = item.x % tiles_per_head;
             const int g_begin = item.y, ng = item.z - item.y, slot = item.w;
             const int64_t row0 = (int64_t)hh * N;
+            // this thread's 64 bytes (key `row`, queries 32 wg ..) of the item's first piece
+            uint8_t* ds_row = nullptr;
+            if constexpr (DS) {
+                if (ds_live && ng > 0)
+                    ds_row = reinterpret_cast<uint8_t*>(ds.pieces) +
+                             ds::piece_row_offset(ds.base_kv[item.x], g_begin, row) + 64 * wg;
+            }
             const uint32_t* u0 = rows_base + (j & 1) * 2 * SW;
             GranuleWalk walk;
             if (lane == 0) {
@@ -968,6 +999,16 @@ k_bwd_dkdv_persist(const __grid_constant__ CUtensorMap tmK, const __grid_constan
                 } else {
 #pragma unroll
                     for (int i = 0; i < 16; ++i) { op[i] = 0u; od[i] = 0u; }
+                }
+                if constexpr (DS) {
+                    // the piece's unread halves (a key granule this query granule did
+                    // not select) are never stored: the look-up sends those to piece 0
+                    if (ds_row && valid) {
+                        uint4* dst = reinterpret_cast<uint4*>(ds_row + (int64_t)g * ds::kPieceBytes);
+#pragma unroll
+                        for (int k = 0; k < 4; ++k)
+                            __stcs(dst + k, make_uint4(od[4 * k], od[4 * k + 1], od[4 * k + 2], od[4 * k + 3]));
+                    }
                 }
                 tmem_st16(tl + cS + 128 * b + 32 * wg, op);       // over this warpgroup's own S^T columns
                 tmem_st16(tl + cP + 128 * b + 32 * wg, od);
@@ -1058,6 +1099,354 @@ k_bwd_dkdv_persist(const __grid_constant__ CUtensorMap tmK, const __grid_constan
     if (warp == 1) tmem_dealloc(tb, kTmemCols);
 }
 
+// ============================================================================ dS handoff
+// Set-up kernels of the handoff (index arithmetic in ds_handoff.cuh), run after
+// the two work plans and before the backward kernels:
+//   k_ds_bases    one CTA: base_q, base_kv (exclusive prefix sums of the plans'
+//                 per-tile units) and the gate `on`
+//   k_ds_prefix   one warp per key tile: word prefixes of its gselT union
+//   k_ds_entries  one warp per query tile: an entry per key granule of its walk
+__global__ void __launch_bounds__(1024) k_ds_bases(const int32_t* __restrict__ units_q,
+                                                   const int32_t* __restrict__ units_kv, int64_t tiles,
+                                                   const PlanHeader* __restrict__ hq,
+                                                   const PlanHeader* __restrict__ hkv, int64_t cap_units,
+                                                   int64_t cap_q, DsDev ds) {
+    __shared__ long long wsum[2][32];
+    __shared__ long long carry[2];
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5, nw = blockDim.x >> 5;
+    if (tid == 0) {
+        carry[0] = carry[1] = 0;
+        *ds.on = ((long long)hkv->total_units <= cap_units && (long long)hq->total_units <= cap_q) ? 1 : 0;
+    }
+    __syncthreads();
+    for (int64_t base = 0; base < tiles; base += blockDim.x) {
+        const int64_t t = base + tid;
+        const long long v0 = t < tiles ? units_q[t] : 0, v1 = t < tiles ? units_kv[t] : 0;
+        long long a = v0, b = v1;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const long long x = __shfl_up_sync(0xffffffffu, a, o), y = __shfl_up_sync(0xffffffffu, b, o);
+            if (lane >= o) { a += x; b += y; }
+        }
+        if (lane == 31) { wsum[0][wid] = a; wsum[1][wid] = b; }
+        __syncthreads();
+        if (wid == 0) {
+            long long x = lane < nw ? wsum[0][lane] : 0, y = lane < nw ? wsum[1][lane] : 0;
+            const long long x0 = x, y0 = y;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const long long p = __shfl_up_sync(0xffffffffu, x, o), q = __shfl_up_sync(0xffffffffu, y, o);
+                if (lane >= o) { x += p; y += q; }
+            }
+            if (lane < nw) { wsum[0][lane] = x - x0; wsum[1][lane] = y - y0; }
+        }
+        __syncthreads();
+        if (t < tiles) {
+            ds.base_q[t] = carry[0] + wsum[0][wid] + a - v0;
+            ds.base_kv[t] = carry[1] + wsum[1][wid] + b - v1;
+        }
+        __syncthreads();
+        if (tid == blockDim.x - 1) {
+            carry[0] += wsum[0][wid] + a;
+            carry[1] += wsum[1][wid] + b;
+        }
+        __syncthreads();
+    }
+}
+
+__global__ void __launch_bounds__(256) k_ds_prefix(const uint32_t* __restrict__ gselT, int64_t MB, int64_t SW,
+                                                   int64_t tph, int heads, DsDev ds) {
+    if (!*ds.on) return;
+    const int lane = threadIdx.x & 31;
+    const int64_t t = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    if (t >= tph * heads) return;                          // whole warps
+    const int64_t r = (t / tph) * MB + 2 * (t % tph);       // the key tile's first gselT row
+    int carry = 0;
+    for (int64_t w0 = 0; w0 < SW; w0 += 32) {
+        const int64_t w = w0 + lane;
+        const int x = w < SW ? ds::popc32(ds::union_word(gselT, r, SW, w)) : 0;
+        int inc = x;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, inc, o);
+            if (lane >= o) inc += y;
+        }
+        if (w < SW) ds.pre[t * SW + w] = carry + inc - x;
+        carry += __shfl_sync(0xffffffffu, inc, 31);
+    }
+}
+
+__global__ void __launch_bounds__(256) k_ds_entries(const uint32_t* __restrict__ gsel,
+                                                    const uint32_t* __restrict__ gselT, int64_t MB, int64_t SW,
+                                                    int64_t tph, int heads, DsDev ds) {
+    if (!*ds.on) return;
+    const int lane = threadIdx.x & 31;
+    const int64_t t = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    if (t >= tph * heads) return;
+    const int hh = (int)(t / tph);
+    const int64_t tq = t % tph, r = (int64_t)hh * MB + 2 * tq;
+    int64_t j = ds.base_q[t];                               // entry of the walk's next granule
+    for (int64_t w0 = 0; w0 < SW; w0 += 32) {
+        const int64_t w = w0 + lane;
+        uint32_t bits = w < SW ? ds::union_word(gsel, r, SW, w) : 0u;
+        const int x = ds::popc32(bits);
+        int inc = x;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, inc, o);
+            if (lane >= o) inc += y;
+        }
+        int64_t e = j + inc - x;
+        while (bits) {
+            const int b = __ffs(bits) - 1;
+            bits &= bits - 1;
+            int32_t o4[4];
+            ds::make_entry(gsel, gselT, ds.pre, ds.base_kv, hh, MB, SW, tph, tq, (int)(32 * w + b), o4);
+            ds.entries[e++] = make_int4(o4[0], o4[1], o4[2], o4[3]);
+        }
+        j += __shfl_sync(0xffffffffu, inc, 31);
+    }
+}
+
+// ============================================================================ dQ from stored dS (persistent)
+// With the handoff the query-stationary pass is one GEMM per key granule,
+// dQ += dS K: dS as two 64 x 64 blocks of stored dS^T (the MN-major A operand,
+// queries contiguous), K a whole-row granule (the MN-major B operand).  One CTA
+// per SM over the same plan items as k_bwd_dq_persist; the accumulator is
+// double-buffered in TMEM so that the next item's MMAs run during this item's
+// epilogue.
+//   warp 0      copies: a lane per (stage, K region) and per (stage, query
+//               granule half); each lane reads the entries of its own stage's
+//               granules, so no selection rows are needed
+//   warp 1      TMEM allocation and MMA issue (4 MMAs of K = 16 a granule)
+//   warps 2-9   epilogue (store_tile_p), warpgroup wg on accumulator columns
+//               D/2 wg .. D/2 wg + D/2 - 1
+// Per non-empty item k (buffer b = k & 1): fin(b) completes when the item's
+// MMAs have; acc_free(b) when the epilogue has read the buffer (256
+// arrivals).  The MMA warp waits acc_free(b) of item k - 2 before the first
+// MMA of item k, and the epilogue waits fin(b) of item k only after its own
+// arrival for item k - 2, so neither barrier runs two phases ahead of its waiter.
+template <int D>
+struct DqdLayout {
+    static constexpr int NR = D / 64;
+    static constexpr int STAGE = NR * kGran + 2 * kGran;   // K granule, then dS^T of the two query granules
+    __host__ __device__ static int staging(int nst) { return nst * STAGE; }
+    __host__ __device__ static int ctrl(int nst) { return staging(nst) + kStagingP; }
+    static int alloc(int nst) { return ctrl(nst) + kCtrl + 1024; }
+    static int stages(int lanes_per_stage) {
+        int n = kStages;
+        while (n > 2 && (alloc(n) > kSmemMax || n * lanes_per_stage > 32)) --n;
+        return n;
+    }
+};
+
+struct BarsD {
+    uint64_t* full;            // [kStages] K and both dS^T blocks of a granule landed
+    uint64_t* empty;           // [kStages]
+    uint64_t* fin;             // [2]
+    uint64_t* acc_free;        // [2]
+    uint64_t* drain;
+    uint32_t* tmem_slot;
+    volatile int* abort_flag;
+};
+
+__device__ __forceinline__ BarsD carve_d(uint8_t* ctrl) {
+    uint64_t* b = reinterpret_cast<uint64_t*>(ctrl);
+    BarsD r;
+    r.full = b;
+    r.empty = b + kStages;
+    r.fin = b + 2 * kStages;
+    r.acc_free = b + 2 * kStages + 2;
+    r.drain = b + 2 * kStages + 4;
+    r.tmem_slot = reinterpret_cast<uint32_t*>(b + 2 * kStages + 5);
+    r.abort_flag = reinterpret_cast<volatile int*>(r.tmem_slot + 1);
+    return r;
+}
+static_assert((2 * kStages + 5) * 8 + 8 <= kCtrl, "barriers overflow the control block");
+
+template <int D, bool RASTER>
+__global__ void __launch_bounds__(320, 1)
+k_bwd_dq_ds(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmS,
+            const __grid_constant__ CUtensorMap tmdQ, const __grid_constant__ CUtensorMap tmPqh,
+            const __grid_constant__ BwdRasterMaps<RASTER, 3> rmaps, BwdRaster ras, DsDev ds,
+            const PlanHeader* __restrict__ hdr, const int4* __restrict__ items, int64_t N, int nst, float scale,
+            uint32_t* __restrict__ dev_status) {
+    using L = DqdLayout<D>;
+    constexpr int kRL = RASTER ? L::NR : 1;                // K copy lanes per stage
+    constexpr uint32_t kCols = 2 * D;                      // two accumulators
+    if (!*ds.on) return;                                   // uniform: k_bwd_dq_persist does the work
+    const int n_items = hdr->n_items;
+    if ((int)blockIdx.x >= n_items) return;
+    const int tiles_per_head = (int)(N / 128);
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    BarsD B = carve_d(sm + L::ctrl(nst));
+    uint8_t* staging = sm + L::staging(nst);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < nst; ++s) {
+            mbar_init(B.full + s, kRL + 2);                // every K and dS^T copy lane arrives
+            mbar_init(B.empty + s, 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(B.fin + b, 1);
+            mbar_init(B.acc_free + b, 256);
+        }
+        mbar_init(B.drain, 1);
+        *B.abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(B.tmem_slot, kCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tb = *B.tmem_slot;
+
+    if (warp == 0) {
+        // ---------------------------------------------------------------- producer
+        // lanes stage * kRL + region copy K; lanes nst * kRL + 2 * stage + h copy
+        // the dS^T block of query granule h
+        const int nk = nst * kRL;
+        const bool is_k = lane < nk;
+        const int stage = is_k ? lane / kRL : (lane - nk) >> 1;
+        const int part = is_k ? lane % kRL : (lane - nk) & 1;  // K region or query granule
+        const bool copier = lane < nk + 2 * nst;
+        if (copier) {
+            if (!is_k) tma_prefetch_desc(&tmS);
+            else if (!RASTER) tma_prefetch_desc(&tmK);
+        }
+        bool ok = true;
+        int last_cyc = -1;
+        int st0 = 0, cyc0 = 0;
+        for (int it = blockIdx.x; it < n_items; it += gridDim.x) {
+            const int4 item = items[it];
+            const int hh = item.x / tiles_per_head;
+            const int ng = item.z - item.y;
+            const int64_t row0 = (int64_t)hh * N;
+            int s_ = st0, c_ = cyc0;
+            if (copier && ok && ng > 0) {
+                const int4* ent = ds.entries + ds.base_q[item.x] + item.y;
+                for (int g = 0; g < ng; ++g) {
+                    if (s_ == stage) {
+                        const int4 e = ent[g];             // read before the wait
+                        if (c_ >= 1 && !mbar_wait(B.empty + stage, (uint32_t)(c_ - 1) & 1, B.abort_flag, dev_status)) {
+                            ok = false;
+                            break;
+                        }
+                        uint8_t* dst = sm + stage * L::STAGE;
+                        if (is_k) {
+                            if constexpr (RASTER) {
+                                const int4 gp = ras.gpos[e.x >> 6];
+                                mbar_expect_tx(B.full + stage, kGran);
+                                tma_load_5d(dst + part * kGran, rmaps.m + kRK * kRasterKinds + gp.w, B.full + stage, 0,
+                                            hh * L::NR + part, gp.z, gp.y, gp.x);
+                            } else {
+                                mbar_expect_tx(B.full + stage, L::NR * kGran);
+                                tma_load_3d(dst, &tmK, B.full + stage, 0, (int)(row0 + e.x), 0);
+                            }
+                        } else {
+                            mbar_expect_tx(B.full + stage, kGran);
+                            tma_load_2d(dst + (L::NR + part) * kGran, &tmS, B.full + stage, 0, part ? e.z : e.y);
+                        }
+                        last_cyc = c_;
+                    }
+                    if (++s_ == nst) { s_ = 0; ++c_; }
+                }
+            }
+            __syncwarp();
+            if (*B.abort_flag) ok = false;
+            const int tot = st0 + ng;                      // every lane advances the ring position
+            cyc0 += tot / nst;
+            st0 = tot % nst;
+        }
+        if (!ok && copier && last_cyc >= 0) {
+            volatile int no_abort = 0;                     // let this lane's last copy land
+            mbar_wait(B.full + stage, (uint32_t)last_cyc & 1, &no_abort, dev_status);
+        }
+    } else if (warp == 1) {
+        // ---------------------------------------------------------------- MMA issue
+        const uint32_t idQ = idesc_bf16_f32(128, D, true, true);
+        const uint32_t aR = smem_u32(sm);
+        bool ok = true;
+        int s_ = 0, c_ = 0, kq = 0;
+        for (int it = blockIdx.x; ok && it < n_items; it += gridDim.x) {
+            const int4 item = items[it];
+            const int ng = item.z - item.y;
+            if (ng == 0) continue;
+            const int b = kq & 1;
+            if (kq >= 2) {
+                if (!mbar_wait_w(B.acc_free + b, (uint32_t)((kq >> 1) - 1) & 1, B.abort_flag, dev_status)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+            }
+            for (int g = 0; g < ng; ++g) {
+                const int s = s_;
+                const uint32_t ph = (uint32_t)c_ & 1;
+                if (++s_ == nst) { s_ = 0; ++c_; }
+                if (!mbar_wait_w(B.full + s, ph, B.abort_flag, dev_status)) { ok = false; break; }
+                tc_fence_after();
+                const uint64_t dK = sdesc_sw128(aR + s * L::STAGE, kGran, 1024);
+                const uint64_t dS = sdesc_sw128(aR + s * L::STAGE + L::NR * kGran, kGran, 1024);
+#pragma unroll
+                for (int k = 0; k < 4; ++k)                // keys 16 k .. 16 k + 15
+                    mma_ss_w(tb + D * b, sdesc_add(dS, k * 2048), sdesc_add(dK, k * 2048), idQ,
+                             (g > 0 || k > 0) ? 1u : 0u);
+                tc_commit_w(B.empty + s);
+            }
+            if (!ok) break;
+            tc_commit_w(B.fin + b);
+            ++kq;
+        }
+        if (!ok) {
+            tc_commit_w(B.drain);                          // every MMA this warp issued complete
+            volatile int no_abort = 0;
+            mbar_wait(B.drain, 0, &no_abort, dev_status);
+        }
+    } else {
+        // ---------------------------------------------------------------- epilogue
+        const int wg = (warp - 2) >> 2;
+        const int sub = warp & 3, row = sub * 32 + lane;
+        const uint32_t tl = tb + ((uint32_t)(sub * 32) << 16);
+        bool ok = true;
+        int kq = 0;
+        for (int it = blockIdx.x; it < n_items; it += gridDim.x) {
+            const int4 item = items[it];
+            const int hh = item.x / tiles_per_head, tile = item.x % tiles_per_head;
+            const int ng = item.z - item.y, slot = item.w;
+            const int64_t row0 = (int64_t)hh * N;
+            const int b = kq & 1;
+            if (ng > 0) {
+                ok = __all_sync(0xffffffffu, ok && mbar_wait(B.fin + b, (uint32_t)(kq >> 1) & 1, B.abort_flag, dev_status));
+                if (ok) tc_fence_after();
+            }
+            // the item's dQ (or zeros when nothing was selected: ng == 0)
+            if constexpr (RASTER)
+                store_tile_p<D>(tl + D * b, row, wg, ok, ng == 0, slot >= 0, scale, staging, &tmdQ, &tmPqh,
+                                (int)(row0 + 128 * tile), slot * 128, 1, 256, warp == 2 && lane < 2 * (D / 64),
+                                rmaps.m + kRdQ * kRasterKinds, ras.gpos[2 * tile], ras.gpos[2 * tile + 1],
+                                hh * (D / 64), lane);
+            else
+                store_tile_p<D>(tl + D * b, row, wg, ok, ng == 0, slot >= 0, scale, staging, &tmdQ, &tmPqh,
+                                (int)(row0 + 128 * tile), slot * 128, 1, 256, warp == 2 && lane == 0);
+            if (ng > 0) {
+                tc_fence_before();
+                mbar_arrive(B.acc_free + b);
+                ++kq;
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tb, kCols);
+}
+
 // ------------------------------------------------------------------ host side
 // whole-row view of a [rows][d] fp32 tensor (d/32 regions of 32 columns) whose
 // box covers `box_regions` regions: the persistent dQ epilogue stores an fp32
@@ -1119,13 +1508,55 @@ BwdWs carve_bwd(void* ws, const Dims& d, size_t* total) {
     return w;
 }
 
+// Host view of a dS handoff buffer: [gate 256 B][base_q][base_kv][pre][entries]
+// [pieces], the pieces 256-byte aligned: cap_units pieces after the zero piece,
+// and cap_q = 2 cap_units entries.  Every selected (query granule, key granule)
+// pair lies in exactly one unit of each walk, and a unit holds one or two
+// pairs, so the query walk never has more than twice the key walk's units:
+// whenever the pieces fit, so do the entries.
+struct DsHost {
+    DsDev dev;
+    int64_t cap_units = 0, cap_q = 0;
+};
+
+size_t ds_fixed_bytes(const Dims& d) {
+    const int64_t tiles = (int64_t)d.heads * (d.N / 128);
+    return 256 + 2 * align16(tiles * 8) + align16(tiles * d.SW * 4) + 256;
+}
+
+constexpr int64_t kDsUnitBytes = ds::kPieceBytes + 2 * ds::kEntryBytes;
+
+bool carve_ds(void* buf, size_t bytes, const Dims& d, DsHost* h) {
+    const size_t fixed = ds_fixed_bytes(d);
+    if (!buf || bytes < fixed + (size_t)(ds::kPieceBytes + kDsUnitBytes)) return false;
+    int64_t cap = (int64_t)((bytes - fixed - (size_t)ds::kPieceBytes) / (size_t)kDsUnitBytes);
+    if (cap > ds::kMaxPieces) cap = ds::kMaxPieces;
+    const int64_t tiles = (int64_t)d.heads * (d.N / 128);
+    uint8_t* p = static_cast<uint8_t*>(buf);
+    h->dev.on = reinterpret_cast<int*>(p);
+    p += 256;
+    h->dev.base_q = reinterpret_cast<int64_t*>(p);
+    p += align16(tiles * 8);
+    h->dev.base_kv = reinterpret_cast<int64_t*>(p);
+    p += align16(tiles * 8);
+    h->dev.pre = reinterpret_cast<int32_t*>(p);
+    p += align16(tiles * d.SW * 4);
+    h->dev.entries = reinterpret_cast<int4*>(p);
+    p += 2 * cap * ds::kEntryBytes;
+    p = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 255) & ~uintptr_t(255));
+    h->dev.pieces = reinterpret_cast<__nv_bfloat16*>(p);
+    h->cap_units = cap;
+    h->cap_q = 2 * cap;
+    return true;
+}
+
 // RASTER: Qp, Kp, Vp, dOp, dQp, dKp, dVp are the raster tensors; perm and
 // shape_id give every granule's box (gran_positions, into the workspace)
 template <int D, bool RASTER>
 prism_status_t launch_bwd(const Dims& d, const void* Qp, const void* Kp, const void* Vp, const void* dOp,
                           const float* lse, const uint32_t* gsel, const uint32_t* gselT, float scale, void* dQp,
                           void* dKp, void* dVp, uint32_t* dev_status, const BwdWs& w, const int32_t* perm,
-                          const uint8_t* shape_id, cudaStream_t s) {
+                          const uint8_t* shape_id, cudaStream_t s, const DsHost* ds = nullptr) {
     const int64_t rows = (int64_t)d.heads * d.N;
     const int target = plan_target(device_sms());
     const int64_t slots = 2 * (int64_t)target;
@@ -1169,20 +1600,53 @@ prism_status_t launch_bwd(const Dims& d, const void* Qp, const void* Kp, const v
     const int smq = DqpLayout<D>::alloc(nq, (int)d.SW);
     const int smk = DkvpLayout<D>::alloc(nk, (int)d.SW);
     if (smq > kSmemMax || smk > kSmemMax) return PRISM_ERR_UNSUPPORTED;   // selection rows too long
-    auto kq = k_bwd_dq_persist<D, RASTER>;
-    auto kk = k_bwd_dkdv_persist<D, RASTER>;
-    if (cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, smq) != cudaSuccess ||
-        cudaFuncSetAttribute(kk, cudaFuncAttributeMaxDynamicSharedMemorySize, smk) != cudaSuccess)
-        return PRISM_ERR_CUDA;
-    // persistent: one CTA per SM (all 512 TMEM columns each), items strided over the CTAs
     const int64_t gq = w.pq.items_max < device_sms() ? w.pq.items_max : device_sms();
-    kq<<<(unsigned)gq, 384, smq, s>>>((const __nv_bfloat16*)Qp, (const __nv_bfloat16*)dOp, gK, gV, tdQ, tPqh, rq,
-                                      ras, gsel, w.pq.hdr, w.pq.items, lse, w.delta, d.N, d.MB, (int)d.SW, nq, scale,
-                                      dev_status);
     const int64_t gk = w.pkv.items_max < device_sms() ? w.pkv.items_max : device_sms();
-    kk<<<(unsigned)gk, 384, smk, s>>>(tK, tV, gQ, gdO, tdK1, tdV1, tPkv1, rkv, ras, gselT, w.pkv.hdr, w.pkv.items,
-                                      w.nld, d.N, d.MB, (int)d.SW, nk, scale, dev_status);
-    st = launch_status(2);
+    if (!ds) {
+        auto kq = k_bwd_dq_persist<D, RASTER, false>;
+        auto kk = k_bwd_dkdv_persist<D, RASTER, false>;
+        if (cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, smq) != cudaSuccess ||
+            cudaFuncSetAttribute(kk, cudaFuncAttributeMaxDynamicSharedMemorySize, smk) != cudaSuccess)
+            return PRISM_ERR_CUDA;
+        // persistent: one CTA per SM (all 512 TMEM columns each), items strided over the CTAs
+        kq<<<(unsigned)gq, 384, smq, s>>>((const __nv_bfloat16*)Qp, (const __nv_bfloat16*)dOp, gK, gV, tdQ, tPqh,
+                                          rq, ras, gsel, w.pq.hdr, w.pq.items, lse, w.delta, d.N, d.MB, (int)d.SW, nq,
+                                          scale, dev_status, nullptr);
+        kk<<<(unsigned)gk, 384, smk, s>>>(tK, tV, gQ, gdO, tdK1, tdV1, tPkv1, rkv, ras, gselT, w.pkv.hdr,
+                                          w.pkv.items, w.nld, d.N, d.MB, (int)d.SW, nk, scale, dev_status, DsDev{});
+        st = launch_status(2);
+    } else {
+        // dS handoff: the gate and the look-up tables, then dK/dV (storing dS^T),
+        // then dQ from the stored dS, or, when the selection does not fit, the
+        // recomputing dQ kernel (each of the two exits at once when it is not chosen)
+        const int64_t tiles = (int64_t)d.heads * (d.N / 128), tph = d.N / 128;
+        const unsigned gw = (unsigned)((tiles * 32 + 255) / 256);
+        CUtensorMap tS;
+        if (!make_map_bf16(&tS, ds->dev.pieces, (1 + ds->cap_units) * ds::kPieceRows, 64, 64)) return PRISM_ERR_CUDA;
+        constexpr int kRLd = RASTER ? D / 64 : 1;
+        const int nd = DqdLayout<D>::stages(kRLd + 2);
+        const int smd = DqdLayout<D>::alloc(nd);
+        auto kq = k_bwd_dq_persist<D, RASTER, true>;
+        auto kk = k_bwd_dkdv_persist<D, RASTER, true>;
+        auto kd = k_bwd_dq_ds<D, RASTER>;
+        if (smd > kSmemMax || cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, smq) != cudaSuccess ||
+            cudaFuncSetAttribute(kk, cudaFuncAttributeMaxDynamicSharedMemorySize, smk) != cudaSuccess ||
+            cudaFuncSetAttribute(kd, cudaFuncAttributeMaxDynamicSharedMemorySize, smd) != cudaSuccess)
+            return PRISM_ERR_CUDA;
+        if (cudaMemsetAsync(ds->dev.pieces, 0, (size_t)ds::kPieceBytes, s) != cudaSuccess) return PRISM_ERR_CUDA;
+        k_ds_bases<<<1, 1024, 0, s>>>(w.pq.tile_units, w.pkv.tile_units, tiles, w.pq.hdr, w.pkv.hdr, ds->cap_units,
+                                      ds->cap_q, ds->dev);
+        k_ds_prefix<<<gw, 256, 0, s>>>(gselT, d.MB, d.SW, tph, d.heads, ds->dev);
+        k_ds_entries<<<gw, 256, 0, s>>>(gsel, gselT, d.MB, d.SW, tph, d.heads, ds->dev);
+        kk<<<(unsigned)gk, 384, smk, s>>>(tK, tV, gQ, gdO, tdK1, tdV1, tPkv1, rkv, ras, gselT, w.pkv.hdr,
+                                          w.pkv.items, w.nld, d.N, d.MB, (int)d.SW, nk, scale, dev_status, ds->dev);
+        kq<<<(unsigned)gq, 384, smq, s>>>((const __nv_bfloat16*)Qp, (const __nv_bfloat16*)dOp, gK, gV, tdQ, tPqh,
+                                          rq, ras, gsel, w.pq.hdr, w.pq.items, lse, w.delta, d.N, d.MB, (int)d.SW, nq,
+                                          scale, dev_status, ds->dev.on);
+        kd<<<(unsigned)gq, 320, smd, s>>>(gK, tS, tdQ, tPqh, rq, ras, ds->dev, w.pq.hdr, w.pq.items, d.N, nd, scale,
+                                          dev_status);
+        st = launch_status(6);
+    }
     const int32_t* cperm = RASTER ? perm : nullptr;
     if (st == PRISM_OK) st = bwd_combine(w.pq, d, 1, w.part_q, dQp, scale, nullptr, 0.f, s, cperm);
     if (st == PRISM_OK) st = bwd_combine(w.pkv, d, 2, w.part_kv, dKp, scale, dVp, 1.f, s, cperm);
@@ -1197,32 +1661,45 @@ size_t attn_bwd_sm100_ws_bytes(const Dims& d) {
     return total;
 }
 
+size_t attn_bwd_ds_bytes(const Dims& d, int64_t pieces) {
+    return ds_fixed_bytes(d) + (size_t)ds::kPieceBytes + (size_t)pieces * (size_t)kDsUnitBytes;
+}
+
+// ds/ds_bytes: a dS handoff buffer (ds_handoff.cuh), or nullptr: S and dP are
+// recomputed by the query-stationary kernel
 prism_status_t attn_bwd_sm100(const Dims& d, const void* Qp, const void* Kp, const void* Vp, const void* Op,
                               const float* o_f32, const void* dOp, const float* lse, const uint32_t* gsel,
                               const uint32_t* gselT, float scale, void* dQp, void* dKp, void* dVp,
-                              uint32_t* dev_status, void* ws, cudaStream_t s) {
+                              uint32_t* dev_status, void* ws, cudaStream_t s, void* ds, size_t ds_bytes) {
     BwdWs w = carve_bwd(ws, d, nullptr);
+    DsHost dh;
+    const DsHost* dsp = carve_ds(ds, ds_bytes, d, &dh) ? &dh : nullptr;
+    if (ds && !dsp) return PRISM_ERR_WORKSPACE;
     prism_status_t st = bwd_delta(d, Op, o_f32, dOp, w.delta, lse, w.nld, s, nullptr);
     if (st != PRISM_OK) return st;
     if (d.d == 128)
         return launch_bwd<128, false>(d, Qp, Kp, Vp, dOp, lse, gsel, gselT, scale, dQp, dKp, dVp, dev_status, w,
-                                      nullptr, nullptr, s);
+                                      nullptr, nullptr, s, dsp);
     return launch_bwd<64, false>(d, Qp, Kp, Vp, dOp, lse, gsel, gselT, scale, dQp, dKp, dVp, dev_status, w, nullptr,
-                                 nullptr, s);
+                                 nullptr, s, dsp);
 }
 
 // raster Q, K, V, dO, dQ, dK, dV ([N][heads][d]); o_f32 and lse in permutation order
 prism_status_t attn_bwd_raster(const Dims& d, const void* Q, const void* K, const void* V, const float* o_f32,
                                const void* dO, const float* lse, const int32_t* perm, const uint8_t* shape_id,
                                const uint32_t* gsel, const uint32_t* gselT, float scale, void* dQ, void* dK, void* dV,
-                               uint32_t* dev_status, void* ws, cudaStream_t s) {
+                               uint32_t* dev_status, void* ws, cudaStream_t s, void* ds, size_t ds_bytes) {
     BwdWs w = carve_bwd(ws, d, nullptr);
+    DsHost dh;
+    const DsHost* dsp = carve_ds(ds, ds_bytes, d, &dh) ? &dh : nullptr;
+    if (ds && !dsp) return PRISM_ERR_WORKSPACE;
     prism_status_t st = bwd_delta(d, nullptr, o_f32, dO, w.delta, lse, w.nld, s, perm);
     if (st != PRISM_OK) return st;
     if (d.d == 128)
         return launch_bwd<128, true>(d, Q, K, V, dO, lse, gsel, gselT, scale, dQ, dK, dV, dev_status, w, perm, shape_id,
-                                     s);
-    return launch_bwd<64, true>(d, Q, K, V, dO, lse, gsel, gselT, scale, dQ, dK, dV, dev_status, w, perm, shape_id, s);
+                                     s, dsp);
+    return launch_bwd<64, true>(d, Q, K, V, dO, lse, gsel, gselT, scale, dQ, dK, dV, dev_status, w, perm, shape_id, s,
+                                dsp);
 }
 
 }  // namespace prism

@@ -335,6 +335,43 @@ prism_status_t prism_sparse_attn_bwd_raster(const prism_problem_t* prob, const v
                                             const uint32_t* gselT, float scale, void* dQ, void* dK, void* dV,
                                             uint32_t* dev_status, void* ws, size_t ws_bytes, cudaStream_t stream);
 
+/*
+ * Stage 7 with a dS handoff (same gradients as the FAQ formulas above; a
+ * different split of the work).  The key-stationary kernel forms dS^T for
+ * every selected (128-key tile, 64-query granule) pair anyway.  Given a
+ * caller-owned buffer `ds` of ds_bytes, it also stores those blocks there as
+ * bf16, and dQ = scale*dS K is then one GEMM per selected key granule, in
+ * place of recomputing S = Q K^T and dP = dO V^T for dQ.
+ *   Pieces: one 16 KB block (128 keys x 64 queries) per unit of the
+ *   key-stationary walk, i.e. per (key tile, query granule that selected one of
+ *   its two key granules).
+ *   Whether the selection's pieces fit is decided on the device, with no host
+ *   synchronisation.  When they do not fit, the call recomputes S and dP, as
+ *   prism_sparse_attn_bwd does.
+ *   dQ may differ from the recomputing call's in the last bf16 bit: S^T and S
+ *   are accumulated in different orders.  dK and dV are the same.
+ *   ds: 16-byte aligned, not aliased with any other argument.  ds_bytes: at
+ *   least prism_attn_bwd_ds_bytes(prob, 1), else PRISM_ERR_WORKSPACE.
+ *   prism_attn_bwd_ds_bytes: the bytes for a buffer that holds `pieces`
+ *   pieces, 1 <= pieces < 2^24 (PRISM_ERR_INVALID_ARG else).  A selection
+ *   needs at most the number of its selected (query granule, key granule)
+ *   pairs.
+ *   bf16 only: PRISM_ERR_UNSUPPORTED for f32.
+ */
+prism_status_t prism_attn_bwd_ds_bytes(const prism_problem_t* prob, int64_t pieces, size_t* bytes);
+prism_status_t prism_sparse_attn_bwd_ds(const prism_problem_t* prob, const void* Qp, const void* Kp,
+                                        const void* Vp, const void* Op, const float* o_f32,
+                                        const void* dOp, const float* lse, const uint32_t* gsel,
+                                        const uint32_t* gselT, float scale, void* dQp, void* dKp,
+                                        void* dVp, uint32_t* dev_status, void* ws, size_t ws_bytes,
+                                        void* ds, size_t ds_bytes, cudaStream_t stream);
+prism_status_t prism_sparse_attn_bwd_raster_ds(const prism_problem_t* prob, const void* Q, const void* K,
+                                               const void* V, const float* o_f32, const void* dO,
+                                               const float* lse, const int32_t* perm, const uint8_t* shape_id,
+                                               const uint32_t* gsel, const uint32_t* gselT, float scale,
+                                               void* dQ, void* dK, void* dV, uint32_t* dev_status, void* ws,
+                                               size_t ws_bytes, void* ds, size_t ds_bytes, cudaStream_t stream);
+
 /* Copy a device status word to the host (synchronises `stream`). */
 prism_status_t prism_read_status(const uint32_t* dev_status, uint32_t* host_out, cudaStream_t stream);
 
