@@ -7,7 +7,9 @@ S and dP recomputed. The checks:
   - dQ meets the oracle at the bf16 bar, whole-tensor and per (head, block);
   - a buffer too small for the selection leaves the gate off, and the call then
     gives the recomputing call's dQ bit for bit.
-Opt-in with PRISM_TEST_DS=1.
+The grid of several split tiles is opt-in (PRISM_TEST_DS=1) until it has run on
+a B200; the 2K layer's split tiles gave dQ, dK and dV bit-identical to the
+recomputing call.
 """
 import os
 
@@ -18,14 +20,14 @@ import torch
 from dynamic_block_sparse_macro_b200 import _abi, inputs
 from dynamic_block_sparse_macro_b200.configs import get_config
 
-pytestmark = [pytest.mark.gpu,
-              pytest.mark.skipif(os.environ.get("PRISM_TEST_DS") != "1",
-                                 reason="dS handoff kernels: set PRISM_TEST_DS=1")]
+pytestmark = pytest.mark.gpu
 
 CASES = {
     "tiny_grid": dict(T=8, H=16, W=16, heads=2),
     "aniso_split_tiles": dict(T=16, H=32, W=32, heads=3),
 }
+_OPT_IN = pytest.mark.skipif(os.environ.get("PRISM_TEST_DS") != "1", reason="set PRISM_TEST_DS=1")
+NAMES = [pytest.param("tiny_grid"), pytest.param("aniso_split_tiles", marks=_OPT_IN)]
 
 
 def _run(name, d):
@@ -47,7 +49,7 @@ def _pairs(mod, cfg):
 
 
 @pytest.mark.parametrize("d", [128, 64])
-@pytest.mark.parametrize("name", list(CASES))
+@pytest.mark.parametrize("name", NAMES)
 def test_blocked_handoff(name, d):
     import oracle as orc
     from gpu_parity import REL_L2, bits, block_rel_l2, host, rel_l2, unpack_sel
@@ -74,7 +76,7 @@ def test_blocked_handoff(name, d):
     assert rel_l2(got, host(mod.dQp)) <= 2e-3
 
 
-@pytest.mark.parametrize("name", list(CASES))
+@pytest.mark.parametrize("name", NAMES)
 def test_blocked_handoff_too_small_falls_back(name):
     from gpu_parity import bits
     cfg, x, mod, _ = _run(name, 128)
@@ -89,7 +91,7 @@ def test_blocked_handoff_too_small_falls_back(name):
         assert np.array_equal(bits(a), bits(b))
 
 
-@pytest.mark.parametrize("name", list(CASES))
+@pytest.mark.parametrize("name", NAMES)
 def test_raster_handoff(name):
     from gpu_parity import bits, host, rel_l2
     cfg, x, mod, grads = _run(name, 128)
