@@ -20,10 +20,11 @@ import pytest
 
 
 class Bar:
-    """An mbarrier: `count` arrivals complete a phase; `done` phases completed."""
+    """An mbarrier: `count` arrivals complete a phase; `done` phases completed.
+    `name` is the barrier's name in the kernel (a family shares one)."""
 
-    def __init__(self, count=1):
-        self.count, self.left, self.done = count, count, 0
+    def __init__(self, count=1, name=""):
+        self.count, self.left, self.done, self.name = count, count, 0, name
 
     def arrive(self):
         self.left -= 1
@@ -40,11 +41,13 @@ class Deadlock(AssertionError):
 class Sim:
     """Random interleaving of agents (generators) and asynchronous work."""
 
-    def __init__(self, seed):
+    def __init__(self, seed, drop=None):
         self.rng = random.Random(seed)
         self.agents = {}            # name -> [generator, pending action]
         self.fifo = {}              # issuing warp -> queued MMA / commit entries
         self.copies = []            # in-flight TMA copies: (fn, barrier)
+        self.drop = drop            # (agent, barrier name): those waits pass at once
+        self.sites = set()          # (agent, barrier name) of every wait met
 
     def add(self, name, gen):
         self.agents[name] = [gen, None]
@@ -70,6 +73,9 @@ class Sim:
             return act[1]()
         if act[0] == "wait":
             _, bar, n = act
+            self.sites.add((name, bar.name))
+            if (name, bar.name) == self.drop:
+                return True
             # a parity wait for phase n is only sound while the barrier has
             # completed n or n + 1 phases
             assert n <= bar.done <= n + 1, (name, n, bar.done)
@@ -120,18 +126,19 @@ def make_items(rng, n_items):
 
 
 # ---------------------------------------------------------------------------- dK/dV
-def dkdv_model(seed, items, nst):
+def dkdv_model(seed, items, nst, drop=None):
     """k_bwd_dkdv_persist: producer (ring lanes and stationary-tile lanes of one
     warp, reconverging once an item), warp 1 S^T/dP^T, warp 2 dV/dK, and the
     elementwise warpgroups with the epilogue."""
-    sim = Sim(seed)
+    sim = Sim(seed, drop)
     W = Sim.wait
-    full0 = [Bar() for _ in range(nst)]
-    fullx = [Bar() for _ in range(nst)]
-    empty = [Bar() for _ in range(nst)]
-    prod, elem, kv_done = [Bar(), Bar()], [Bar(), Bar()], [Bar(), Bar()]
-    rows_full, rows_empty = [Bar(), Bar()], [Bar(), Bar()]
-    stat, kv_free, fin = Bar(), Bar(), Bar()
+    full0 = [Bar(name="full0") for _ in range(nst)]
+    fullx = [Bar(name="fullx") for _ in range(nst)]
+    empty = [Bar(name="empty") for _ in range(nst)]
+    prod, elem = [Bar(name="prod") for _ in range(2)], [Bar(name="elem") for _ in range(2)]
+    kv_done = [Bar(name="kv_done") for _ in range(2)]
+    rows_full, rows_empty = [Bar(name="rows_full") for _ in range(2)], [Bar(name="rows_empty") for _ in range(2)]
+    stat, kv_free, fin = Bar(name="stat"), Bar(name="kv_free"), Bar(name="fin")
     st = dict(ring=[None] * nst, xs=[None] * nst, tmem=[None, None], kvtile=None, acc="free",
               rows=[None, None], sdp_done=set(), dvdk_done=set(), item_sync={})
     # granule numbering over the CTA's items, and each item's first granule
@@ -265,6 +272,7 @@ def dkdv_model(seed, items, nst):
         sim.add(name, gen)
     sim.run()
     assert len(st["dvdk_done"]) == sum(items)
+    return sim
 
 
 @pytest.mark.parametrize("nst", [2, 3, 4, 5])
@@ -276,18 +284,18 @@ def test_dkdv_protocol_random_schedules(nst):
 
 
 # ---------------------------------------------------------------------------- dQ
-def dq_model(seed, items, nst):
+def dq_model(seed, items, nst, drop=None):
     """k_bwd_dq_persist: producer (selection rows, K and V ring), warp 1 S, warp 10
     dP, warp 11 dQ, and the elementwise warpgroups, which write the next non-empty
     item's Q and dO into TMEM and run the epilogue."""
-    sim = Sim(seed)
+    sim = Sim(seed, drop)
     W = Sim.wait
-    full0 = [Bar() for _ in range(nst)]
-    empty = [Bar() for _ in range(nst)]
-    prod = [Bar(2), Bar(2)]                  # the S and the dP issuer each commit
-    elem, dq_done = [Bar(), Bar()], [Bar(), Bar()]
-    rows_full, rows_empty = [Bar(), Bar()], [Bar(), Bar()]
-    qdo_full, fin = Bar(), Bar()
+    full0 = [Bar(name="full0") for _ in range(nst)]
+    empty = [Bar(name="empty") for _ in range(nst)]
+    prod = [Bar(2, "prod") for _ in range(2)]   # the S and the dP issuer each commit
+    elem, dq_done = [Bar(name="elem") for _ in range(2)], [Bar(name="dq_done") for _ in range(2)]
+    rows_full, rows_empty = [Bar(name="rows_full") for _ in range(2)], [Bar(name="rows_empty") for _ in range(2)]
+    qdo_full, fin = Bar(name="qdo_full"), Bar(name="fin")
     st = dict(ring=[None] * nst, S=[None, None], P=[None, None], qdo=None, acc="free", rows=[None, None],
               s_done=set(), p_done=set(), q_done=set())
     first, G = [], 0
@@ -414,6 +422,7 @@ def dq_model(seed, items, nst):
         sim.add(name, gen)
     sim.run()
     assert len(st["q_done"]) == sum(items)
+    return sim
 
 
 @pytest.mark.parametrize("nst", [2, 3, 4, 5])
@@ -424,18 +433,106 @@ def test_dq_protocol_random_schedules(nst):
         dq_model(2000 * nst + trial, items, nst)
 
 
+# ---------------------------------------------------------------------------- dQ from stored dS
+def dq_ds_model(seed, items, nst, drop=None):
+    """k_bwd_dq_ds: the copy lanes (K and both dS^T blocks of a granule into one
+    ring stage), the MMA warp (dQ += dS K into accumulator b = k & 1 of non-empty
+    item k) and the epilogue warps, which read accumulator b and free it."""
+    sim = Sim(seed, drop)
+    W = Sim.wait
+    full = [Bar(name="full") for _ in range(nst)]
+    empty = [Bar(name="empty") for _ in range(nst)]
+    fin = [Bar(name="fin") for _ in range(2)]
+    acc_free = [Bar(name="acc_free") for _ in range(2)]
+    st = dict(ring=[None] * nst, acc=["free", "free"], done=set(), stored=[])
+    first, G = [], 0
+    for ng in items:
+        first.append(G)
+        G += ng
+    nonempty = [j for j, ng in enumerate(items) if ng > 0]
+    kq_of = {j: k for k, j in enumerate(nonempty)}
+
+    def producer():
+        for j, ng in enumerate(items):
+            for g in range(ng):
+                Gg = first[j] + g
+                s, cyc = Gg % nst, Gg // nst
+                if cyc >= 1:
+                    yield W(empty[s], cyc - 1)
+
+                def land(Gg=Gg, s=s):
+                    assert Gg < nst or (Gg - nst) in st["done"], ("ring stage reused early", Gg)
+                    st["ring"][s] = Gg
+                yield ("copy", land, full[s])
+
+    def mma_warp():
+        for j in nonempty:
+            kq, ng = kq_of[j], items[j]
+            b = kq & 1
+            if kq >= 2:
+                yield W(acc_free[b], (kq >> 1) - 1)
+            for g in range(ng):
+                Gg = first[j] + g
+                s = Gg % nst
+                yield W(full[s], Gg // nst)
+
+                def mma(Gg=Gg, s=s, b=b, j=j, g=g):
+                    assert st["ring"][s] == Gg, ("MMA before its operands", Gg)
+                    if g == 0:
+                        assert st["acc"][b] == "free", ("dQ over an unread accumulator", j)
+                        st["acc"][b] = (j, 1)
+                    else:
+                        assert st["acc"][b] == (j, g)
+                        st["acc"][b] = (j, g + 1)
+                    st["done"].add(Gg)
+                yield ("mma", mma)
+                yield ("commit", empty[s])
+            yield ("commit", fin[b])
+
+    def epilogue():
+        for j, ng in enumerate(items):
+            if ng == 0:
+                yield ("do", lambda j=j: st["stored"].append(j))      # zeros, no TMEM
+                continue
+            kq = kq_of[j]
+            b = kq & 1
+            yield W(fin[b], kq >> 1)
+
+            def store(j=j, ng=ng, b=b):
+                assert st["acc"][b] == (j, ng), ("epilogue", j, st["acc"][b])
+                st["acc"][b] = "free"
+                st["stored"].append(j)
+                acc_free[b].arrive()
+            yield ("do", store)
+
+    for name, gen in (("producer", producer()), ("mma", mma_warp()), ("epi", epilogue())):
+        sim.add(name, gen)
+    sim.run()
+    assert st["stored"] == list(range(len(items))) and len(st["done"]) == sum(items)
+    return sim
+
+
+@pytest.mark.parametrize("nst", [2, 3, 6, 8])
+def test_dq_ds_protocol_random_schedules(nst):
+    rng = random.Random(300 + nst)
+    for trial in range(200):
+        items = make_items(rng, rng.randint(1, 9))
+        dq_ds_model(3000 * nst + trial, items, nst)
+
+
 # ---------------------------------------------------------------------------- forward
-def fwd_model(seed, nch, p_quarter=lambda g: 2 * g):
+def fwd_model(seed, nch, p_quarter=lambda g: 2 * g, drop=None):
     """k_attn_fwd_sm100, one CTA (one item): producer (Q once; K and V of each chunk
     in one buffer each), warp 1 (S = Q K^T into the one S buffer, then O += P V),
     and the two softmax warpgroups as two agents. The S buffer is tracked in four
     32-column quarters; warpgroup g reads quarters 2g and 2g+1 (its key granule)
     twice, with the row-maximum exchange between the reads, and writes its P into
     quarter p_quarter(g)."""
-    sim = Sim(seed)
+    sim = Sim(seed, drop)
     W = Sim.wait
-    bar_q, bar_kf, bar_ke, bar_vf, bar_ve = Bar(), Bar(), Bar(), Bar(), Bar()
-    bar_s, bar_p, bar_o = Bar(), Bar(2), Bar()
+    bar_q, bar_kf, bar_ke = Bar(name="bar_q"), Bar(name="bar_kf"), Bar(name="bar_ke")
+    bar_vf, bar_ve = Bar(name="bar_vf"), Bar(name="bar_ve")
+    bar_s, bar_p, bar_o = Bar(name="bar_s"), Bar(2, "bar_p"), Bar(name="bar_o")
     st = dict(K=None, V=None, S=[None] * 4, O=[], xmax=[[None, None], [None, None]], xbar={}, pv_done=set())
 
     def producer_k():
@@ -461,13 +558,13 @@ def fwd_model(seed, nch, p_quarter=lambda g: 2 * g):
     st["s_done"] = set()
 
     def mma_warp():
-        yield ("copy", lambda: None, bar_q)
+        yield ("copy", lambda: st.update(Q=True), bar_q)
         yield W(bar_q, 0)
         for c in range(nch):
             yield W(bar_kf, c)
 
             def s_mma(c=c):
-                assert st["K"] == c
+                assert st.get("Q") and st["K"] == c
                 # the previous chunk's P has been read by PV(c - 1), issued earlier by this warp
                 assert all(q is None or q[0] == "read" for q in st["S"]), ("S over unread P", c, st["S"])
                 st["S"] = [("S", c)] * 4
@@ -520,6 +617,7 @@ def fwd_model(seed, nch, p_quarter=lambda g: 2 * g):
                       ("wg1", softmax(1))):
         sim.add(name, gen)
     sim.run()
+    return sim
 
 
 def test_fwd_protocol_random_schedules():
@@ -533,3 +631,49 @@ def test_fwd_model_catches_p_over_the_other_granules_columns():
     with pytest.raises(AssertionError):
         for trial in range(400):
             fwd_model(trial, 1 + trial % 9, p_quarter=lambda g: g)
+
+
+# ---------------------------------------------------------------------------- every wait is needed
+def _catches(run):
+    """True when some random schedule breaks a check (a hazard, an unsound parity
+    wait or a deadlock)."""
+    try:
+        run()
+    except AssertionError:
+        return True
+    return False
+
+
+def _items_runs(model, base, nst):
+    rng = random.Random(base)
+    cases = [(base + t, make_items(rng, rng.randint(2, 9))) for t in range(300)]
+    return lambda drop: [model(seed, items, nst, drop) for seed, items in cases]
+
+
+MODELS = {
+    "dkdv": lambda: _items_runs(dkdv_model, 7000, 3),
+    "dq": lambda: _items_runs(dq_model, 8000, 3),
+    "dq_ds": lambda: _items_runs(dq_ds_model, 9000, 3),
+    "fwd": lambda: (lambda drop: [fwd_model(t, 1 + t % 9, drop=drop) for t in range(400)]),
+}
+
+
+# Waits that another wait of the same role already implies.  In k_bwd_dq_persist
+# the S issuer waits elem(b) and then dq_done(b) of the buffer's previous use;
+# the dQ MMA that dq_done(b) tracks was itself issued only after that elem(b)
+# phase, so the first wait adds nothing to the second.
+REDUNDANT = {"dq": [("w1", "elem")]}
+
+
+@pytest.mark.parametrize("model", list(MODELS))
+def test_dropping_any_wait_is_caught(model):
+    """Each (role, barrier) wait of the model, dropped on its own, lets some
+    schedule break a check, except the waits listed as implied by another: the
+    model's checks see what each wait guards."""
+    runs = MODELS[model]()
+    sites = set()
+    for sim in runs(None):
+        sites |= sim.sites
+    assert sites
+    missed = [site for site in sorted(sites) if not _catches(lambda site=site: runs(site))]
+    assert missed == REDUNDANT.get(model, []), missed
