@@ -4,6 +4,7 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config 2k] [--dense]
     python bench.py --impl reference      # the fp64 CPU oracle on a bounded sample
     python bench.py --forward-only        # inference: the forward stages, no backward state
+    python bench.py --bwd-ds              # backward with the dS handoff (no e2e figure)
 
 One step = one pass of the whole hot path over the configured synthetic layer:
 zone indicator -> shapes/permutation -> permute Q,K,V -> pooled block
@@ -224,7 +225,9 @@ class StepTimer:
         return {n: self.ev[i].elapsed_time(self.ev[i + 1]) for i, n in enumerate(self.NAMES)}
 
 
-def run_step(mod, x, out, grads, timer=None):
+def run_step(mod, x, out, grads, timer=None, ds=None):
+    """One layer step; ds: a dS handoff buffer for the backward (None: S and dP
+    are recomputed for dQ)."""
     from dynamic_block_sparse_macro_b200 import _abi
     ev = timer.ev if timer else None
     rec = (lambda i: ev[i].record()) if ev else (lambda i: None)
@@ -249,15 +252,25 @@ def run_step(mod, x, out, grads, timer=None):
         return
     if mod.raster:
         rec(4)
-        mod.attend_backward_raster(x["Q"], x["K"], x["V"], x["dO"], *grads)
+        if ds is None:
+            mod.attend_backward_raster(x["Q"], x["K"], x["V"], x["dO"], *grads)
+        else:
+            _abi.prism_sparse_attn_bwd_raster_ds(mod.prob, x["Q"], x["K"], x["V"], mod.Of32, x["dO"], mod.lse,
+                                                 mod.perm, mod.shape_id, mod.gsel, mod.gselT, mod.scale, *grads,
+                                                 mod.dev_status, mod.ws_bwd, ds)
         rec(5)
         rec(6)
         return
     _abi.prism_permute(mod.prob, x["dO"], mod.perm, mod.dOp)
     rec(4)
-    _abi.prism_sparse_attn_bwd(mod.prob, mod.Qp, mod.Kp, mod.Vp, mod.Op, mod.Of32, mod.dOp, mod.lse,
-                               mod.gsel, mod.gselT, mod.scale, mod.dQp, mod.dKp, mod.dVp, mod.dev_status,
-                               mod.ws_bwd)
+    if ds is None:
+        _abi.prism_sparse_attn_bwd(mod.prob, mod.Qp, mod.Kp, mod.Vp, mod.Op, mod.Of32, mod.dOp, mod.lse,
+                                   mod.gsel, mod.gselT, mod.scale, mod.dQp, mod.dKp, mod.dVp, mod.dev_status,
+                                   mod.ws_bwd)
+    else:
+        _abi.prism_sparse_attn_bwd_ds(mod.prob, mod.Qp, mod.Kp, mod.Vp, mod.Op, mod.Of32, mod.dOp, mod.lse,
+                                      mod.gsel, mod.gselT, mod.scale, mod.dQp, mod.dKp, mod.dVp, mod.dev_status,
+                                      mod.ws_bwd, ds)
     rec(5)
     for src, dst in zip((mod.dQp, mod.dKp, mod.dVp), grads):
         _abi.prism_unpermute(mod.prob, src, mod.perm, dst)
@@ -333,8 +346,15 @@ def bench_prism(args, cfg, rank, world, local_rank):
                                with_backward=not fwd_only, raster=bool(args.raster))
     out = torch.empty_like(x["Q"])
     grads = [] if fwd_only else [torch.empty_like(x["Q"]) for _ in range(3)]
-    for _ in range(max(args.warmup, 1)):
+    ds = None
+    if args.bwd_ds and not fwd_only:
+        # dS handoff: a buffer for every selected (query granule, key granule) pair of
+        # this selection (the inputs are fixed, so the selection is the same each step)
         run_step(mod, x, out, grads)
+        pairs = int(sum(_popcount_rows(mod.gsel[hh]).sum().item() for hh in range(mod.heads)))
+        ds = torch.empty(_abi.prism_attn_bwd_ds_bytes(mod.prob, max(1, pairs)), dtype=torch.uint8, device=dev)
+    for _ in range(max(args.warmup, 1)):
+        run_step(mod, x, out, grads, ds=ds)
     torch.cuda.synchronize()
     fl = selected_flops(mod)
 
@@ -350,7 +370,7 @@ def bench_prism(args, cfg, rank, world, local_rank):
     clocks.mark()
     start.record()
     for t in timers:
-        run_step(mod, x, out, grads, t)
+        run_step(mod, x, out, grads, t, ds=ds)
     stop.record()
     torch.cuda.synchronize()
     launches = _abi.launch_count() - n0
@@ -367,11 +387,13 @@ def bench_prism(args, cfg, rank, world, local_rank):
     tflops = job_tflops(world, attn_flops, attn_ms)
     memory = mod.memory_report()
     memory["inputs_outputs"] = int(sum(t.numel() * t.element_size() for t in list(x.values()) + [out] + grads))
+    if ds is not None:
+        memory["ds_handoff"] = int(ds.numel())
     memory["peak_allocated"] = int(torch.cuda.max_memory_allocated(dev))
 
     # end to end through the public API from pinned host buffers
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and ds is None:        # the host-buffer step runs the layer's own backward
         e2e = bench_e2e(args, cfg, mod, x, dev, world, attn_flops)
 
     peaks = load_peaks()
@@ -381,8 +403,8 @@ def bench_prism(args, cfg, rank, world, local_rank):
     dom = "attn_bwd" if stage_ms["attn_bwd"] >= stage_ms["attn_fwd"] else "attn_fwd"
     ach = bwd_ach if dom == "attn_bwd" else fwd_ach
     # the capture is of the blocked-operand kernels: none for the raster ones
-    traffic = (BWD_DRAM_BYTES.get((cfg.name, cfg.heads)) if dom == "attn_bwd" and not args.dense and not args.raster
-               else None)
+    traffic = (BWD_DRAM_BYTES.get((cfg.name, cfg.heads))
+               if dom == "attn_bwd" and not args.dense and not args.raster and ds is None else None)
     # the attention kernels run at 1.85-1.97 GHz (clocks below): the burst peak is the fair
     # denominator; the sustained one (measured at ~1.33 GHz under the power cap) is reported beside it
     peak = peaks["bf16_tflops"]
@@ -399,11 +421,13 @@ def bench_prism(args, cfg, rank, world, local_rank):
                    "tokens": cfg.n_tokens, "heads": cfg.heads, "head_dim": cfg.head_dim,
                    "top_k": cfg.top_k, "top_p": 1.0 if args.dense else cfg.top_p,
                    "all_blocks_dense": bool(args.dense), "global_batch": world,
+                   "backward": "dS handoff" if ds is not None else "recompute S, dP for dQ",
                    "parallelism": f"replicas{world}" if world > 1 else "single",
                    "l2": "inputs larger than L2 (126 MB): no flush"},
         "stage_ms": {k: round(v, 4) for k, v in stage_ms.items()},
         "selection": {k: (round(v, 6) if isinstance(v, float) else v) for k, v in fl.items()},
-        "roofline": {"kernel": "prism_sparse_attn_bwd" if dom == "attn_bwd" else "prism_sparse_attn_fwd",
+        "roofline": {"kernel": ("prism_sparse_attn_bwd" + ("_ds" if ds is not None else "")) if dom == "attn_bwd"
+                     else "prism_sparse_attn_fwd",
                      "bound": "tensor", "achieved": round(ach, 3), "peak": peak, "unit": "TFLOP/s",
                      "frac": round(ach / peak, 4), "traffic": traffic,
                      "peak_source": f"{peaks['source']} bf16_tflops (burst)",
@@ -526,6 +550,8 @@ def main():
                     help="inference: the forward stages alone, no backward buffers (value = forward TFLOP/s)")
     ap.add_argument("--raster", action="store_true",
                     help="the attention reads Q, K, V, dO and writes O, dQ, dK, dV in the raster layout")
+    ap.add_argument("--bwd-ds", action="store_true",
+                    help="backward through prism_sparse_attn_bwd_ds (dS handoff) instead of recomputing S, dP")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
