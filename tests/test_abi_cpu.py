@@ -98,6 +98,35 @@ def test_bad_pointers_rejected_before_launch(L):
                                  None, None) == 1      # tau256 > tau128
 
 
+def test_ds_handoff_sizes_and_checks(L):
+    """The dS handoff buffer: a fixed part (gate, the plans' unit prefixes, the key
+    tiles' word prefixes, alignment) plus, per piece, 16 KB of dS^T and two 16-byte
+    look-up entries; bad buffers are refused before any launch."""
+    p = _abi.problem(32, 72, 128, 24, 128, 64, "bf16")
+    s = _abi.query_sizes(p)
+    tiles = 24 * s.n_tokens // 128
+    a16 = lambda b: (b + 15) // 16 * 16
+    fixed = 256 + 2 * a16(8 * tiles) + a16(4 * tiles * s.sel_words) + 256
+    for pieces in (1, 1000, 2_215_883):
+        assert _abi.prism_attn_bwd_ds_bytes(p, pieces) == fixed + 16384 + pieces * (16384 + 32)
+    out = ctypes.c_size_t(0)
+    for bad in (0, -1, 1 << 24):
+        assert L.prism_attn_bwd_ds_bytes(ctypes.byref(p), bad, ctypes.byref(out)) == 1
+    fake, ws = 1 << 40, s.ws_attn_bwd
+    args = [fake] * 9 + [1.0 / 128 ** 0.5] + [fake] * 5
+    need = _abi.prism_attn_bwd_ds_bytes(p, 1)
+    bwd = L.prism_sparse_attn_bwd_ds
+    assert bwd(ctypes.byref(p), *args, ws, None, need, None) == 1            # no buffer
+    assert bwd(ctypes.byref(p), *args, ws, fake + 8, need, None) == 1        # misaligned
+    assert bwd(ctypes.byref(p), *args, ws, fake, need - 1, None) == 4        # too small for one piece
+    assert bwd(ctypes.byref(p), *args, ws - 1, fake, need, None) == 4        # workspace too small
+    pf = _abi.problem(32, 72, 128, 24, 128, 64, "f32")
+    assert bwd(ctypes.byref(pf), *args, _abi.query_sizes(pf).ws_attn_bwd, fake, need, None) == 3
+    rargs = [fake] * 10 + [1.0 / 128 ** 0.5] + [fake] * 5
+    assert L.prism_sparse_attn_bwd_raster_ds(ctypes.byref(p), *rargs, ws, fake, need - 1, None) == 4
+    assert L.prism_sparse_attn_bwd_raster_ds(ctypes.byref(p), *rargs, ws, None, need, None) == 1
+
+
 # ---------------------------------------------------------------- the layer object
 def test_layer_struct_matches_the_c_compiler(L):
     # the C driver prints sizeof and every field offset as the C compiler lays them out
