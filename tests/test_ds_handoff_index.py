@@ -99,6 +99,7 @@ CASES = [
     (1, 72, 0.15, ((0, 35),), ((0, 0), (0, 71))),
     (2, 64, 0.9, (), ()),
     (1, 96, 0.02, ((0, 10), (0, 11)), ()),
+    (1, 512, 0.03, ((0, 100),), ((0, 511),)),      # 16 words a row: ranks across many word prefixes
 ]
 
 
